@@ -1,0 +1,297 @@
+"""CPU fp64 oracle of the 4-bit weight-quantised linear layer (W4A16 and W4A8).
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU
+legs of ``bench.py`` may import this module. The library never does: it has no
+CPU path, and it shares no code, table or helper with this file.
+
+What it computes, and where that comes from:
+
+* "MARLIN: Mixed-Precision Auto-Regressive Parallel Inference on Large Language
+  Models", Abstract: a linear layer whose weights are quantised to 4 bits per
+  element and whose activations stay in fp16. The layer is
+  ``Y[M,N] = A[M,K] . W[K,N]``.
+* "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+  proposed method (fine-grained group quantisation): one scale per group of
+  ``g`` consecutive rows of ``W`` and output column. The zero point is fixed at
+  8, so ``W[k,n] = (q[k,n] - 8) * s[k // g, n]``.
+* "A Speed Odyssey for Deployable Quantization of LLMs", Abstract (FastGEMM,
+  W4A8): int8 activations times the same 4-bit weights, with a per-token scale
+  (Atom, dynamic activation quantisation) and a per-channel weight scale:
+  ``Y[m,n] = sa[m] * sw[n] * sum_k A[m,k] * (q[k,n] - 8)``.
+
+The pages do not fix the packing of the codes; the reading used here is the
+plainest one for "8 codes per int32" of a K x N weight: ``Q`` is ``[K/8, N]``
+and code ``k = 8*i + j`` of column ``n`` sits in bits ``4j .. 4j+3`` of
+``Q[i, n]``.
+
+The layer reaches the exact product up to rounding, so the oracle is that
+definition written out in float64: unpack, dequantise exactly in fp64, then one
+fp64 matrix product (a library primitive). The W4A8 integer accumulator is
+computed exactly as well (see ``w4a8_acc``).
+
+The prepacked weight format (``prepack_w4a16`` / ``prepack_w4a8``) is this
+library's own design: the "Efficient Arbitrary Precision Acceleration for Large
+Language Models on GPU Tensor Cores" page names a matrix preprocessing step
+that reorders the weights for the kernel, but gives no layout. The functions
+below restate the documented layout plainly, so that the CUDA prepack can be
+compared with it byte for byte.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "unpack_codes", "dequant", "w4a16", "w4a16_absdot", "w4a16_entry",
+    "tolerance", "w4a8_acc", "w4a8", "w4a8_absdot",
+    "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
+    "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
+]
+
+ZERO_POINT = 8          # w = (q - 8) * s  (fixed symmetric zero point)
+REL_TOL = 2.0 ** -10    # |y - y_ref| <= 2^-10 |y_ref| + 1e-3 sum_k |a_k w_k|
+ABS_DOT_TOL = 1e-3
+
+
+# --------------------------------------------------------------------------
+# the layer
+# --------------------------------------------------------------------------
+def unpack_codes(Q: np.ndarray) -> np.ndarray:
+    """Codes ``q[K, N]`` from the packed ``Q[K/8, N]``: ``q[8i+j, n] = (Q[i,n] >> 4j) & 15``."""
+    Qu = np.asarray(Q).view(np.uint32)
+    K8, N = Qu.shape
+    q = np.empty((K8, 8, N), dtype=np.uint8)
+    for j in range(8):
+        q[:, j, :] = (Qu >> np.uint32(4 * j)) & np.uint32(0xF)
+    return q.reshape(K8 * 8, N)
+
+
+def dequant(q: np.ndarray, s: np.ndarray, g: int) -> np.ndarray:
+    """``W[k,n] = (q[k,n] - 8) * s[k // g, n]`` in float64 (exact: an int times an fp16)."""
+    K, N = q.shape
+    if K % g:
+        raise ValueError("g must divide K")
+    group = np.arange(K) // g
+    return (q.astype(np.float64) - ZERO_POINT) * np.asarray(s, dtype=np.float64)[group, :]
+
+
+def _w_columns(Q, s, g, n0, n1):
+    return dequant(unpack_codes(np.asarray(Q)[:, n0:n1]), np.asarray(s)[:, n0:n1], g)
+
+
+def w4a16(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, chunk: int = 4096) -> np.ndarray:
+    """``Y = A . W`` in float64, with ``W`` dequantised in float64; chunked along N to bound memory."""
+    A64 = np.asarray(A, dtype=np.float64)
+    N = np.asarray(Q).shape[1]
+    Y = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        Y[:, n0:n1] = A64 @ _w_columns(Q, s, g, n0, n1)
+    return Y
+
+
+def w4a16_absdot(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, chunk: int = 4096) -> np.ndarray:
+    """``sum_k |A[m,k] * W[k,n]|`` in float64: the scale of the tolerance's second term."""
+    A64 = np.abs(np.asarray(A, dtype=np.float64))
+    N = np.asarray(Q).shape[1]
+    out = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        out[:, n0:n1] = A64 @ np.abs(_w_columns(Q, s, g, n0, n1))
+    return out
+
+
+def w4a16_entry(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, m: int, n: int):
+    """One output ``(y[m,n], sum_k |a w|)`` computed on its own, for sampled checks of large layers."""
+    w = _w_columns(Q, s, g, n, n + 1)[:, 0]
+    a = np.asarray(A[m], dtype=np.float64)
+    return float(a @ w), float(np.abs(a) @ np.abs(w))
+
+
+def tolerance(y_ref: np.ndarray, absdot: np.ndarray) -> np.ndarray:
+    """Allowed error: ``2^-10 |y_ref| + 1e-3 sum_k |a_k w_k|``."""
+    return REL_TOL * np.abs(y_ref) + ABS_DOT_TOL * absdot
+
+
+def w4a8_acc(A: np.ndarray, Q: np.ndarray, chunk: int = 4096) -> np.ndarray:
+    """Exact integer accumulator ``sum_k A[m,k] * (q[k,n] - 8)`` as int64.
+
+    The product runs in float64 through BLAS: every operand is an integer of
+    magnitude <= 127 or <= 8 and every partial sum stays far below 2^53, so
+    each float64 operation is exact and the order of summation cannot change
+    the result.
+    """
+    A64 = np.asarray(A, dtype=np.float64)
+    K = A64.shape[1]
+    if 127 * 8 * K >= 2 ** 53:
+        raise ValueError("K too large for an exact float64 accumulation")
+    N = np.asarray(Q).shape[1]
+    acc = np.empty((A64.shape[0], N), dtype=np.int64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        wq = unpack_codes(np.asarray(Q)[:, n0:n1]).astype(np.float64) - ZERO_POINT
+        acc[:, n0:n1] = (A64 @ wq).astype(np.int64)
+    return acc
+
+
+def w4a8(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray):
+    """``(acc, Y)``: the exact int64 accumulator and ``Y = acc * sa[m] * sw[n]`` in float64."""
+    acc = w4a8_acc(A, Q)
+    Y = acc.astype(np.float64) * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+    return acc, Y
+
+
+def w4a8_absdot(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray, chunk: int = 4096) -> np.ndarray:
+    """``sa[m] * sw[n] * sum_k |A[m,k] * (q[k,n] - 8)|`` in float64."""
+    A64 = np.abs(np.asarray(A, dtype=np.float64))
+    N = np.asarray(Q).shape[1]
+    out = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        wq = np.abs(unpack_codes(np.asarray(Q)[:, n0:n1]).astype(np.float64) - ZERO_POINT)
+        out[:, n0:n1] = A64 @ wq
+    return out * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+
+
+# --------------------------------------------------------------------------
+# the prepacked weight format (this library's layout, restated plainly)
+# --------------------------------------------------------------------------
+TILE_N = 128      # output columns per tile
+TILE_K = 128      # rows of W per k-block
+# nibble position of code j (j = 0..7 within a word) in a prepacked word
+NIBBLE_POS_W4A16 = (0, 4, 1, 5, 2, 6, 3, 7)
+NIBBLE_POS_W4A8 = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
+def _check_kn(K, N):
+    if K <= 0 or K % TILE_K:
+        raise ValueError("K must be a positive multiple of 128")
+    if N <= 0 or N % 8:
+        raise ValueError("N must be a positive multiple of 8")
+
+
+def _group_slots(K: int, g: int) -> int:
+    """Scale rows stored per blob: ``128/g`` for g in {32, 64, 128}; 1 for g a multiple of 128 below K; 0 for g == K."""
+    if g == K:
+        return 0
+    if g in (32, 64, 128):
+        return TILE_K // g
+    if g % TILE_K == 0 and K % g == 0:
+        return 1
+    raise ValueError("unsupported group size")
+
+
+def prepacked_bytes_w4a16(K: int, N: int, g: int) -> int:
+    _check_kn(K, N)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    slots = _group_slots(K, g)
+    blob = TILE_N * TILE_K // 2 + 2 * TILE_N * slots
+    tail = 0 if slots else ((2 * nt * TILE_N + 15) // 16) * 16
+    return nt * kt * blob + tail
+
+
+def prepacked_bytes_w4a8(K: int, N: int) -> int:
+    _check_kn(K, N)
+    return -(-N // TILE_N) * (K // TILE_K) * (TILE_N * TILE_K // 2)
+
+
+def _blob_words(q: np.ndarray, nibble_pos) -> np.ndarray:
+    """Code words of every blob: ``[NT, KT, h=2, v=2, r=128, i=4]`` uint32.
+
+    Word ``(nt, kt, h, v, r, i)`` holds the 8 codes of column ``nt*128 + r``,
+    rows ``kt*128 + 64h + 32v + 8i + j`` for ``j = 0..7``; code ``j`` sits at
+    nibble ``nibble_pos[j]``. Columns past N hold code 8 (a zero weight).
+    """
+    K, N = q.shape
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    qp = np.full((K, nt * TILE_N), ZERO_POINT, dtype=np.uint32)
+    qp[:, :N] = q
+    # [kt, h, v, i, j, nt, r]
+    qv = qp.reshape(kt, 2, 2, 4, 8, nt, TILE_N)
+    words = np.zeros((kt, 2, 2, 4, nt, TILE_N), dtype=np.uint32)
+    for j in range(8):
+        words |= qv[:, :, :, :, j, :, :] << np.uint32(4 * nibble_pos[j])
+    # -> [nt, kt, h, v, r, i]
+    return np.ascontiguousarray(words.transpose(4, 0, 1, 2, 5, 3))
+
+
+def prepack_w4a16(Q: np.ndarray, s: np.ndarray, g: int) -> np.ndarray:
+    """The W4A16 prepacked buffer as bytes (uint8), following the library's documented layout.
+
+    Blob ``(nt, kt)`` starts at byte ``(nt*KT + kt) * blob_bytes``: 8192 bytes
+    of code words (``_blob_words`` order) followed by ``slots`` rows of 128
+    fp16 scales, row ``u`` holding ``s[(kt*128 + u*g) // g, nt*128 + r]`` for
+    ``g <= 128`` and ``s[(kt*128) // g, ...]`` for larger ``g``. For ``g == K``
+    the blobs hold codes only and one fp16 scale per (padded) column follows
+    all blobs. Scales of padded columns are 0.
+    """
+    q = unpack_codes(Q)
+    K, N = q.shape
+    slots = _group_slots(K, g)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    words = _blob_words(q, NIBBLE_POS_W4A16).reshape(nt, kt, -1)
+    s = np.asarray(s, dtype=np.float16)
+    sp = np.zeros((s.shape[0], nt * TILE_N), dtype=np.float16)
+    sp[:, :N] = s
+    parts = []
+    if slots:
+        krow = np.arange(kt)[:, None] * TILE_K + np.arange(slots)[None, :] * g   # first row of each slot
+        grp = krow // g                                                          # [kt, slots]
+        sc = sp[grp]                                                             # [kt, slots, nt*128]
+        sc = sc.reshape(kt, slots, nt, TILE_N).transpose(2, 0, 1, 3).reshape(nt, kt, -1)
+        blob = np.concatenate([words.view(np.uint8), sc.view(np.uint8)], axis=2)
+        parts.append(blob.reshape(-1))
+    else:
+        parts.append(words.view(np.uint8).reshape(-1))
+        tail = np.zeros(prepacked_bytes_w4a16(K, N, g) - words.nbytes, dtype=np.uint8)
+        tail[: 2 * nt * TILE_N] = sp[0].view(np.uint8)
+        parts.append(tail)
+    out = np.concatenate(parts)
+    assert out.nbytes == prepacked_bytes_w4a16(K, N, g)
+    return out
+
+
+def prepack_w4a8(Q: np.ndarray) -> np.ndarray:
+    """The W4A8 prepacked buffer as bytes: the code blobs only, with the W4A8 nibble order."""
+    q = unpack_codes(Q)
+    out = _blob_words(q, NIBBLE_POS_W4A8).view(np.uint8).reshape(-1)
+    assert out.nbytes == prepacked_bytes_w4a8(*q.shape)
+    return out
+
+
+def _codes_from_words(words: np.ndarray, nibble_pos, K: int, N: int) -> np.ndarray:
+    nt, kt = words.shape[:2]
+    w = words.reshape(nt, kt, 2, 2, TILE_N, 4)
+    q = np.zeros((kt, 2, 2, 4, 8, nt, TILE_N), dtype=np.uint8)
+    wt = w.transpose(1, 2, 3, 5, 0, 4)  # [kt, h, v, i, nt, r]
+    for j in range(8):
+        q[:, :, :, :, j, :, :] = (wt >> np.uint32(4 * nibble_pos[j])) & np.uint32(0xF)
+    return q.reshape(K, nt * TILE_N)[:, :N]
+
+
+def unprepack_w4a16(Wp: np.ndarray, K: int, N: int, g: int):
+    """Inverse of ``prepack_w4a16``: ``(q[K,N] uint8, s[K/g, N] fp16)``."""
+    slots = _group_slots(K, g)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    code_bytes = TILE_N * TILE_K // 2
+    Wp = np.asarray(Wp, dtype=np.uint8)
+    if slots:
+        blob = Wp.reshape(nt, kt, code_bytes + 2 * TILE_N * slots)
+        words = np.ascontiguousarray(blob[:, :, :code_bytes]).view(np.uint32)
+        sc = np.ascontiguousarray(blob[:, :, code_bytes:]).view(np.float16).reshape(nt, kt, slots, TILE_N)
+        sc = sc.transpose(1, 2, 0, 3).reshape(kt * slots, nt * TILE_N)  # rows in k order
+        krow = (np.arange(kt)[:, None] * TILE_K + np.arange(slots)[None, :] * g).reshape(-1)
+        s = np.zeros((K // g, nt * TILE_N), dtype=np.float16)
+        s[krow // g] = sc
+        s = s[:, :N]
+    else:
+        words = np.ascontiguousarray(Wp[: nt * kt * code_bytes]).view(np.uint32).reshape(nt, kt, -1)
+        s = np.ascontiguousarray(Wp[nt * kt * code_bytes: nt * kt * code_bytes + 2 * nt * TILE_N]).view(np.float16)
+        s = s[None, :N].copy()
+    return _codes_from_words(words, NIBBLE_POS_W4A16, K, N), s
+
+
+def unprepack_w4a8(Wp: np.ndarray, K: int, N: int) -> np.ndarray:
+    """Inverse of ``prepack_w4a8``: codes ``q[K,N]`` uint8."""
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    words = np.ascontiguousarray(np.asarray(Wp, dtype=np.uint8)).view(np.uint32).reshape(nt, kt, -1)
+    return _codes_from_words(words, NIBBLE_POS_W4A8, K, N)

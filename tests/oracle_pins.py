@@ -1,0 +1,233 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Each ``pin_*`` takes the oracle module (so that a test can hand it a copy with
+a planted mistake) and raises ``AssertionError`` when the oracle disagrees
+with the fact it is pinned to:
+
+* hand-worked examples (``tests/golden``), exact in binary;
+* exact rational brute force (``fractions.Fraction``) on tiny layers, using the
+  raw codes from the generator rather than the oracle's unpacking;
+* closed forms of special cases: identity activations reproduce the
+  dequantised weights, all-8 codes give zero, all-0 codes give
+  ``-8 * sum_k a_k s_k``;
+* invariants: power-of-two scale homogeneity, row permutation, linearity;
+* W4A8: the integer accumulator against Python integer loops.
+"""
+from __future__ import annotations
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line
+
+
+def golden_words():
+    out = []
+    for line in _rows("unpack_words.txt"):
+        w, codes = line.split(":")
+        out.append((int(w, 16), [int(c) for c in codes.split()]))
+    return out
+
+
+def golden_hand():
+    out = []
+    for line in _rows("hand_examples.txt"):
+        kind, words, scales, g, acts, sasw, expect = [p.strip() for p in line.split("|")]
+        words = [int(w, 16) for w in words.split()]
+        out.append({
+            "kind": kind,
+            "Q": np.array(words, dtype=np.uint32).view(np.int32).reshape(-1, 1),
+            "s": None if scales == "-" else np.array([float(x) for x in scales.split()], dtype=np.float16).reshape(-1, 1),
+            "g": None if g == "-" else int(g),
+            "A": np.array([float(x) for x in acts.split()]).reshape(1, -1),
+            "sasw": None if sasw == "-" else [float(x) for x in sasw.split()],
+            "expect": [float(x) for x in expect.split()],
+        })
+    return out
+
+
+# ---------------------------------------------------------------- unpacking
+def pin_unpack_golden(o):
+    for word, codes in golden_words():
+        Q = np.array([[word]], dtype=np.uint32).view(np.int32)
+        got = o.unpack_codes(Q)[:, 0].tolist()
+        assert got == codes, (hex(word), got, codes)
+
+
+def pin_unpack_matches_generator(o):
+    d = synth.w4a16_inputs(64, 24, 32, 1, seed=3)
+    assert np.array_equal(o.unpack_codes(d["Q"]), d["q"])
+
+
+# ---------------------------------------------------------------- W4A16
+def pin_hand_examples(o):
+    for ex in golden_hand():
+        if ex["kind"] == "w4a16":
+            A = ex["A"].astype(np.float16)
+            y = o.w4a16(A, ex["Q"], ex["s"], ex["g"])
+            assert y.shape == (1, 1)
+            assert y[0, 0] == ex["expect"][0], (y, ex)
+        else:
+            A = ex["A"].astype(np.int8)
+            sa = np.array([ex["sasw"][0]], np.float32)
+            sw = np.array([ex["sasw"][1]], np.float32)
+            acc, y = o.w4a8(A, sa, ex["Q"], sw)
+            assert int(acc[0, 0]) == int(ex["expect"][1]), (acc, ex)
+            assert y[0, 0] == ex["expect"][0], (y, ex)
+
+
+def _exact_w4a16(A, q, s, g):
+    M, K = A.shape
+    N = q.shape[1]
+    y = [[Fraction(0)] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                acc += Fraction(float(A[m, k])) * (int(q[k, n]) - 8) * Fraction(float(s[k // g, n]))
+            y[m][n] = acc
+    return y
+
+
+def pin_bruteforce_w4a16(o):
+    # M, K, N all different so that a transposed operand cannot pass
+    for (M, K, N, g, seed) in [(3, 64, 5, 16, 1), (2, 48, 7, 48, 2), (4, 32, 3, 8, 3), (1, 128, 9, 32, 4)]:
+        d = synth.w4a16_inputs(K, N, g, M, seed=seed)
+        y = o.w4a16(d["A"], d["Q"], d["s"], g)
+        assert y.shape == (M, N)
+        ex = _exact_w4a16(d["A"], d["q"], d["s"], g)
+        for m in range(M):
+            for n in range(N):
+                absdot = sum(abs(float(d["A"][m, k]) * (int(d["q"][k, n]) - 8) * float(d["s"][k // g, n]))
+                             for k in range(K))
+                err = abs(Fraction(float(y[m, n])) - ex[m][n])
+                assert err <= Fraction(K * 2.0 ** -52 * absdot + 1e-300), (M, K, N, g, m, n, float(err))
+
+
+def pin_absdot(o):
+    d = synth.w4a16_inputs(64, 6, 16, 2, seed=5)
+    got = o.w4a16_absdot(d["A"], d["Q"], d["s"], 16)
+    for m in range(2):
+        for n in range(6):
+            ref = math.fsum(abs(float(d["A"][m, k]) * (int(d["q"][k, n]) - 8) * float(d["s"][k // 16, n]))
+                            for k in range(64))
+            assert abs(got[m, n] - ref) <= 1e-12 * ref
+    y1, a1 = o.w4a16_entry(d["A"], d["Q"], d["s"], 16, 1, 4)
+    assert abs(a1 - got[1, 4]) <= 1e-12 * got[1, 4]
+    assert abs(y1 - o.w4a16(d["A"], d["Q"], d["s"], 16)[1, 4]) <= 1e-12 * a1
+
+
+def pin_identity_activation(o):
+    # A = I reproduces W exactly; W[k,n] = (q-8)*s written out per element
+    for (K, N, g) in [(64, 5, 16), (32, 3, 32), (128, 2, 64)]:
+        d = synth.w4a16_inputs(K, N, g, 1, seed=7)
+        A = np.eye(K, dtype=np.float16)
+        y = o.w4a16(A, d["Q"], d["s"], g)
+        for k in range(K):
+            for n in range(N):
+                assert y[k, n] == (int(d["q"][k, n]) - 8) * float(d["s"][k // g, n]), (K, N, g, k, n)
+
+
+def pin_all_eight(o):
+    K, N, g = 64, 6, 16
+    d = synth.w4a16_inputs(K, N, g, 3, seed=8)
+    Q = synth.pack_q(np.full((K, N), 8, np.uint8))
+    y = o.w4a16(d["A"], Q, d["s"], g)
+    assert np.all(y == 0.0)
+
+
+def pin_all_zero_codes(o):
+    K, N, g = 64, 6, 16
+    d = synth.w4a16_inputs(K, N, g, 3, seed=9)
+    Q = synth.pack_q(np.zeros((K, N), np.uint8))
+    y = o.w4a16(d["A"], Q, d["s"], g)
+    for m in range(3):
+        for n in range(N):
+            ref = -8.0 * math.fsum(float(d["A"][m, k]) * float(d["s"][k // g, n]) for k in range(K))
+            scale = 8.0 * math.fsum(abs(float(d["A"][m, k]) * float(d["s"][k // g, n])) for k in range(K))
+            assert abs(y[m, n] - ref) <= K * 2.0 ** -52 * scale
+
+
+def pin_scale_homogeneity(o):
+    d = synth.w4a16_inputs(128, 10, 32, 4, seed=10)
+    y1 = o.w4a16(d["A"], d["Q"], d["s"], 32)
+    y2 = o.w4a16(d["A"], d["Q"], (d["s"].astype(np.float32) * 2).astype(np.float16), 32)
+    assert np.array_equal(y2, 2 * y1)
+
+
+def pin_row_permutation(o):
+    d = synth.w4a16_inputs(128, 10, 32, 6, seed=11)
+    perm = np.array([3, 0, 5, 1, 4, 2])
+    y = o.w4a16(d["A"], d["Q"], d["s"], 32)
+    yp = o.w4a16(d["A"][perm], d["Q"], d["s"], 32)
+    ad = o.w4a16_absdot(d["A"], d["Q"], d["s"], 32)
+    assert np.all(np.abs(yp - y[perm]) <= 128 * 2.0 ** -52 * ad[perm])
+
+
+def pin_linearity(o):
+    d = synth.w4a16_inputs(128, 10, 32, 4, seed=12)
+    e = synth.w4a16_inputs(128, 10, 32, 4, seed=13)
+    A1, A2 = d["A"].astype(np.float64), e["A"].astype(np.float64)
+    y12 = o.w4a16(A1 + A2, d["Q"], d["s"], 32)
+    y1 = o.w4a16(A1, d["Q"], d["s"], 32)
+    y2 = o.w4a16(A2, d["Q"], d["s"], 32)
+    ad = o.w4a16_absdot(np.abs(A1) + np.abs(A2), d["Q"], d["s"], 32)
+    assert np.all(np.abs(y12 - (y1 + y2)) <= 4 * 128 * 2.0 ** -52 * ad)
+
+
+def pin_tolerance_formula(o):
+    y = np.array([1.0, -2.0, 0.0])
+    ad = np.array([2.0, 0.5, 3.0])
+    t = o.tolerance(y, ad)
+    assert np.allclose(t, [2.0 ** -10 + 2e-3, 2.0 ** -9 + 5e-4, 3e-3], rtol=1e-15, atol=0)
+
+
+# ---------------------------------------------------------------- W4A8
+def pin_bruteforce_w4a8(o):
+    for (M, K, N, seed) in [(3, 64, 5, 1), (2, 40, 7, 2), (5, 16, 3, 3)]:
+        d = synth.w4a8_inputs(K, N, M, seed=seed)
+        acc, y = o.w4a8(d["A"], d["sa"], d["Q"], d["sw"])
+        assert acc.shape == (M, N) and acc.dtype == np.int64
+        for m in range(M):
+            for n in range(N):
+                ref = sum(int(d["A"][m, k]) * (int(d["q"][k, n]) - 8) for k in range(K))
+                assert int(acc[m, n]) == ref, (m, n)
+                yex = Fraction(ref) * Fraction(float(d["sa"][m])) * Fraction(float(d["sw"][n]))
+                assert abs(Fraction(float(y[m, n])) - yex) <= abs(yex) * Fraction(2.0 ** -51)
+        ad = o.w4a8_absdot(d["A"], d["sa"], d["Q"], d["sw"])
+        for m in range(M):
+            for n in range(N):
+                ref = sum(abs(int(d["A"][m, k]) * (int(d["q"][k, n]) - 8)) for k in range(K))
+                exp = ref * float(d["sa"][m]) * float(d["sw"][n])
+                assert abs(ad[m, n] - exp) <= 1e-12 * max(exp, 1e-30)
+
+
+def pin_w4a8_extremes(o):
+    # the largest accumulator magnitude: a = -127 everywhere, all codes 0 -> 8*127*K
+    K, N = 1024, 3
+    A = np.full((1, K), -127, np.int8)
+    Q = synth.pack_q(np.zeros((K, N), np.uint8))
+    acc = o.w4a8_acc(A, Q)
+    assert np.all(acc == 8 * 127 * K)
+    Q = synth.pack_q(np.full((K, N), 15, np.uint8))
+    assert np.all(o.w4a8_acc(A, Q) == -7 * 127 * K)
+
+
+ALL_PINS = [
+    pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
+    pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
+    pin_row_permutation, pin_linearity, pin_tolerance_formula, pin_bruteforce_w4a8, pin_w4a8_extremes,
+]

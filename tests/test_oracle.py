@@ -1,0 +1,154 @@
+"""CPU tests of the oracle: its pins, its prepack-layout restatement, and that the pins catch planted mistakes."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from oracle import wq_oracle as O
+
+from oracle_pins import ALL_PINS
+
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
+def test_pin(pin):
+    pin(O)
+
+
+# ------------------------------------------------------------ planted mistakes
+def _mut_zero_point(mp):
+    mp.setattr(O, "ZERO_POINT", 7)
+
+
+def _mut_group_mod(mp):
+    def dequant(q, s, g):
+        K = q.shape[0]
+        G = np.asarray(s).shape[0]
+        return (q.astype(np.float64) - 8) * np.asarray(s, np.float64)[np.arange(K) % G, :]
+    mp.setattr(O, "dequant", dequant)
+
+
+def _mut_group_off_by_one(mp):
+    def dequant(q, s, g):
+        K = q.shape[0]
+        G = np.asarray(s).shape[0]
+        return (q.astype(np.float64) - 8) * np.asarray(s, np.float64)[(np.arange(K) // g + 1) % G, :]
+    mp.setattr(O, "dequant", dequant)
+
+
+def _mut_scale_dropped(mp):
+    mp.setattr(O, "dequant", lambda q, s, g: q.astype(np.float64) - 8)
+
+
+def _mut_nibbles_reversed(mp):
+    def unpack_codes(Q):
+        Qu = np.asarray(Q).view(np.uint32)
+        K8, N = Qu.shape
+        q = np.empty((K8, 8, N), np.uint8)
+        for j in range(8):
+            q[:, j, :] = (Qu >> np.uint32(4 * (7 - j))) & np.uint32(15)
+        return q.reshape(K8 * 8, N)
+    mp.setattr(O, "unpack_codes", unpack_codes)
+
+
+def _mut_k_reversed(mp):
+    orig = O._w_columns
+    mp.setattr(O, "_w_columns", lambda Q, s, g, n0, n1: orig(Q, s, g, n0, n1)[::-1])
+
+
+def _mut_sign_flipped(mp):
+    mp.setattr(O, "dequant", lambda q, s, g: (8 - q.astype(np.float64)) *
+               np.asarray(s, np.float64)[np.arange(q.shape[0]) // g, :])
+
+
+def _mut_w4a8_no_zero_point(mp):
+    def w4a8_acc(A, Q, chunk=4096):
+        return (np.asarray(A, np.float64) @ O.unpack_codes(Q).astype(np.float64)).astype(np.int64)
+    mp.setattr(O, "w4a8_acc", w4a8_acc)
+
+
+def _mut_w4a8_sw_dropped(mp):
+    def w4a8(A, sa, Q, sw):
+        acc = O.w4a8_acc(A, Q)
+        return acc, acc.astype(np.float64) * np.asarray(sa, np.float64)[:, None]
+    mp.setattr(O, "w4a8", w4a8)
+
+
+def _mut_absdot_signed(mp):
+    def absdot(A, Q, s, g, chunk=4096):
+        return np.abs(np.asarray(A, np.float64)) @ O.dequant(O.unpack_codes(Q), s, g)
+    mp.setattr(O, "w4a16_absdot", absdot)
+
+
+def _mut_tolerance_rel_dropped(mp):
+    mp.setattr(O, "tolerance", lambda y, ad: 1e-3 * ad)
+
+
+MUTATIONS = [_mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
+             _mut_k_reversed, _mut_sign_flipped, _mut_w4a8_no_zero_point, _mut_w4a8_sw_dropped,
+             _mut_absdot_signed, _mut_tolerance_rel_dropped]
+
+
+@pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__[5:])
+def test_pins_catch_planted_mistake(mutate, monkeypatch):
+    mutate(monkeypatch)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(O)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin.__name__)
+    assert caught, "no pin caught the planted mistake"
+
+
+# ------------------------------------------------------------ prepack layout (the library's own format)
+SHAPES = [(128, 128, 128), (256, 200, 64), (384, 136, 32), (512, 8, 256), (256, 264, 256), (1024, 392, 128)]
+
+
+@pytest.mark.parametrize("K,N,g", SHAPES)
+def test_prepack_roundtrip(K, N, g):
+    d = synth.w4a16_inputs(K, N, g, 1, seed=K + N + g)
+    Wp = O.prepack_w4a16(d["Q"], d["s"], g)
+    assert Wp.nbytes == O.prepacked_bytes_w4a16(K, N, g)
+    q, s = O.unprepack_w4a16(Wp, K, N, g)
+    assert np.array_equal(q, d["q"])
+    assert np.array_equal(s.view(np.uint16), d["s"].view(np.uint16))
+
+
+@pytest.mark.parametrize("K,N", [(128, 128), (256, 200), (640, 24)])
+def test_prepack_w4a8_roundtrip(K, N):
+    d = synth.w4a8_inputs(K, N, 1, seed=K + N)
+    Wp = O.prepack_w4a8(d["Q"])
+    assert Wp.nbytes == O.prepacked_bytes_w4a8(K, N)
+    assert np.array_equal(O.unprepack_w4a8(Wp, K, N), d["q"])
+
+
+def test_prepack_blob_locality():
+    # a code of column n and row k lands inside blob (n // 128, k // 128), and nowhere else
+    K, N, g = 384, 296, 128
+    nt, kt = 3, 3
+    blob = O.prepacked_bytes_w4a16(K, N, g) // (nt * kt)
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        k, n = int(rng.integers(K)), int(rng.integers(N))
+        q = np.full((K, N), 8, np.uint8)
+        q[k, n] = 3
+        s = np.zeros((K // g, N), np.float16)
+        Wp = O.prepack_w4a16(synth.pack_q(q), s, g)
+        base = O.prepack_w4a16(synth.pack_q(np.full((K, N), 8, np.uint8)), s, g)
+        diff = np.nonzero(Wp != base)[0]
+        assert diff.size == 1
+        assert diff[0] // blob == (n // 128) * kt + (k // 128)
+
+
+def test_prepack_padding_is_zero_weight():
+    K, N, g = 256, 72, 64
+    d = synth.w4a16_inputs(K, N, g, 1, seed=1)
+    Wp = O.prepack_w4a16(d["Q"], d["s"], g)
+    full = O.unprepack_w4a16(Wp, K, 128, g)
+    assert np.all(full[0][:, N:] == 8)
+    assert np.all(full[1][:, N:] == 0)
+
+
+def test_package_reexports():
+    assert oracle.w4a16 is O.w4a16
