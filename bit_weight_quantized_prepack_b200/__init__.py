@@ -1,0 +1,212 @@
+"""Python binding of ``libwq.so``, the C ABI declared in ``include/wq.h``.
+
+Argument marshalling only: every computation runs in the library's CUDA kernels. The
+functions keep the C names; shapes are read from the tensors where the tensors carry them.
+torch provides device memory and streams. The binding raises ``ImportError`` when the
+library is not built and ``WqError`` when a call returns an error status: there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "WqError", "lib", "LIB_PATH", "status_string", "wq_version",
+    "wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepack", "wq_prepack_w4a8",
+    "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a8",
+    "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan",
+    "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
+    "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
+    "WQ_ERR_UNSUPPORTED_DEVICE", "WQ_ERR_CUDA", "WQ_ERR_TIMEOUT", "WQ_ERR_NO_MEMORY", "WQ_ERR_CAPTURING",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
+
+(WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_UNSUPPORTED_SHAPE, WQ_ERR_MISALIGNED, WQ_ERR_UNSUPPORTED_DEVICE,
+ WQ_ERR_CUDA, WQ_ERR_TIMEOUT, WQ_ERR_NO_MEMORY, WQ_ERR_CAPTURING) = range(9)
+
+
+class WqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)}")
+        self.status = status
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("grid", ctypes.c_int), ("tile_m", ctypes.c_int), ("m_tiles", ctypes.c_int),
+                ("n_tiles", ctypes.c_int), ("k_blocks", ctypes.c_int), ("stages", ctypes.c_int),
+                ("smem_bytes", ctypes.c_int), ("threads", ctypes.c_int), ("units", ctypes.c_longlong)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m bit_weight_quantized_prepack_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, Z, V = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, None
+    sigs = {
+        "wq_status_string": (ctypes.c_char_p, [I]),
+        "wq_version": (I, []),
+        "wq_prepacked_bytes": (Z, [I, I, I]),
+        "wq_prepacked_bytes_w4a8": (Z, [I, I]),
+        "wq_prepack": (I, [P, P, I, I, I, P, P]),
+        "wq_prepack_w4a8": (I, [P, I, I, P, P]),
+        "wq_unpack": (I, [P, I, I, I, P, P, P]),
+        "wq_unpack_w4a8": (I, [P, I, I, P, P]),
+        "wq_gemm_w4a16": (I, [P, P, P, I, I, I, I, P]),
+        "wq_gemm_w4a8": (I, [P, P, P, P, P, P, I, I, I, P]),
+        "wq_workspace_bytes": (Z, [I, I, I, I]),
+        "wq_workspace_reserve": (I, [Z, P]),
+        "wq_get_device_status": (I, [P]),
+        "wq_plan": (I, [I, I, I, I, I, ctypes.POINTER(_Plan)]),
+        "wq_debug_set_wait_timeout_ns": (I, [ctypes.c_ulonglong]),
+        "wq_debug_skip_publish": (I, [I]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    del V
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.wq_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != WQ_OK:
+        raise WqError(rc, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev_tensor(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def wq_version() -> int:
+    return lib.wq_version()
+
+
+def wq_prepacked_bytes(K: int, N: int, g: int) -> int:
+    return lib.wq_prepacked_bytes(K, N, g)
+
+
+def wq_prepacked_bytes_w4a8(K: int, N: int) -> int:
+    return lib.wq_prepacked_bytes_w4a8(K, N)
+
+
+def wq_prepack(Q: torch.Tensor, s: torch.Tensor, g: int, Wp: torch.Tensor | None = None, stream=None):
+    """Q int32 [K/8, N], s fp16 [K/g, N] -> Wp uint8 [wq_prepacked_bytes(K, N, g)]."""
+    _dev_tensor(Q, torch.int32, "Q")
+    _dev_tensor(s, torch.float16, "s")
+    K, N = Q.shape[0] * 8, Q.shape[1]
+    nbytes = wq_prepacked_bytes(K, N, g)
+    if nbytes == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack")
+    if Wp is None:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack(_ptr(Q), _ptr(s), K, N, g, _ptr(Wp), _stream(stream)), "wq_prepack")
+    return Wp
+
+
+def wq_prepack_w4a8(Q: torch.Tensor, Wp: torch.Tensor | None = None, stream=None):
+    _dev_tensor(Q, torch.int32, "Q")
+    K, N = Q.shape[0] * 8, Q.shape[1]
+    nbytes = wq_prepacked_bytes_w4a8(K, N)
+    if nbytes == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack_w4a8")
+    if Wp is None:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack_w4a8(_ptr(Q), K, N, _ptr(Wp), _stream(stream)), "wq_prepack_w4a8")
+    return Wp
+
+
+def wq_unpack(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
+    """Inverse of wq_prepack: (Q int32 [K/8, N], s fp16 [K/g, N])."""
+    Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
+    s = torch.empty((K // g, N), dtype=torch.float16, device=Wp.device)
+    _check(lib.wq_unpack(_ptr(Wp), K, N, g, _ptr(Q), _ptr(s), _stream(stream)), "wq_unpack")
+    return Q, s
+
+
+def wq_unpack_w4a8(Wp: torch.Tensor, K: int, N: int, stream=None):
+    Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
+    _check(lib.wq_unpack_w4a8(_ptr(Wp), K, N, _ptr(Q), _stream(stream)), "wq_unpack_w4a8")
+    return Q
+
+
+def wq_gemm_w4a16(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor | None = None, stream=None):
+    """Y fp16 [M, N] = A fp16 [M, K] . dequant(Wp)."""
+    _dev_tensor(A, torch.float16, "A")
+    M, K = A.shape
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _dev_tensor(Y, torch.float16, "Y")
+    _check(lib.wq_gemm_w4a16(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)), "wq_gemm_w4a16")
+    return Y
+
+
+def wq_gemm_w4a8(A: torch.Tensor, sa: torch.Tensor, Wp: torch.Tensor, sw: torch.Tensor, N: int,
+                 Y: torch.Tensor | None = None, acc_out: torch.Tensor | None = None, stream=None):
+    """Y fp16 [M, N] = (A int8 [M, K] . (q - 8)) * sa[m] * sw[n]; acc_out (optional) gets the int32 sums."""
+    _dev_tensor(A, torch.int8, "A")
+    _dev_tensor(sa, torch.float32, "sa")
+    _dev_tensor(sw, torch.float32, "sw")
+    M, K = A.shape
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    if acc_out is not None:
+        _dev_tensor(acc_out, torch.int32, "acc_out")
+    _check(lib.wq_gemm_w4a8(_ptr(A), _ptr(sa), _ptr(Wp), _ptr(sw), _ptr(Y), _ptr(acc_out), M, N, K,
+                            _stream(stream)), "wq_gemm_w4a8")
+    return Y
+
+
+def wq_workspace_bytes(kind: int, M: int, N: int, K: int) -> int:
+    return lib.wq_workspace_bytes(kind, M, N, K)
+
+
+def wq_workspace_reserve(nbytes: int, stream=None) -> None:
+    _check(lib.wq_workspace_reserve(nbytes, _stream(stream)), "wq_workspace_reserve")
+
+
+def wq_get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status: WQ_OK or WQ_ERR_TIMEOUT."""
+    return lib.wq_get_device_status(_stream(stream))
+
+
+def wq_plan(kind: int, M: int, N: int, K: int, g: int) -> dict:
+    p = _Plan()
+    _check(lib.wq_plan(kind, M, N, K, g, ctypes.byref(p)), "wq_plan")
+    return {f: getattr(p, f) for f, _ in _Plan._fields_}
+
+
+def wq_debug_set_wait_timeout_ns(ns: int) -> None:
+    _check(lib.wq_debug_set_wait_timeout_ns(ns), "wq_debug_set_wait_timeout_ns")
+
+
+def wq_debug_skip_publish(cta: int) -> None:
+    _check(lib.wq_debug_skip_publish(cta), "wq_debug_skip_publish")

@@ -1,0 +1,434 @@
+// C ABI of the library (declared in include/wq.h): argument checks, launch plans, the
+// per-(device, stream) stream-K workspace, tensor maps for the activation loads, and the
+// device status word that reports expired waits.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "wq.h"
+#include "wq_internal.h"
+
+namespace {
+
+using namespace wq;
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+std::mutex g_mu;
+unsigned long long g_timeout_ns = kDefaultTimeoutNs;
+int g_skip_publish = -1;
+
+struct DeviceState {
+    bool init = false;
+    bool supported = false;
+    int num_sms = 0;
+    int smem_optin = 0;
+    int* status = nullptr;  // device status word
+};
+std::map<int, DeviceState> g_devices;
+
+struct Workspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+std::map<std::pair<int, uintptr_t>, Workspace> g_workspaces;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Initialise (once) and return the state of the current device; nullptr on CUDA failure.
+DeviceState* device_state(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    *dev_out = dev;
+    DeviceState& d = g_devices[dev];
+    if (d.init) return &d;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return nullptr;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return nullptr;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+    if (cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return nullptr;
+    d.supported = (major == 10 && minor == 0);
+    if (d.supported) {
+        if (cudaMalloc(&d.status, sizeof(int)) != cudaSuccess) return nullptr;
+        if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return nullptr;
+        if (configure_gemm_kernels(d.smem_optin - 2048) != cudaSuccess) return nullptr;
+    }
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return nullptr;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.init = true;
+    return &d;
+}
+
+// Status of the current device for a compute call: WQ_OK with *out set, or an error.
+int require_device(int* dev, DeviceState** out, cudaStream_t stream, bool need_init_outside_capture) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return WQ_ERR_CUDA;
+    {
+        int d = 0;
+        if (cudaGetDevice(&d) != cudaSuccess) return WQ_ERR_CUDA;
+        auto it = g_devices.find(d);
+        if ((it == g_devices.end() || !it->second.init) && cs != cudaStreamCaptureStatusNone &&
+            need_init_outside_capture)
+            return WQ_ERR_CAPTURING;
+    }
+    DeviceState* st = device_state(dev);
+    if (!st) return WQ_ERR_CUDA;
+    if (!st->supported) return WQ_ERR_UNSUPPORTED_DEVICE;
+    *out = st;
+    return WQ_OK;
+}
+
+// Workspace of (dev, stream) with at least `bytes`; grows it (not while capturing).
+int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
+    Workspace& w = g_workspaces[{dev, reinterpret_cast<uintptr_t>(stream)}];
+    if (w.bytes >= bytes && w.ptr) {
+        *ptr = w.ptr;
+        return WQ_OK;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return WQ_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return WQ_ERR_CAPTURING;
+    size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+    if (w.ptr) {
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return WQ_ERR_CUDA;
+        cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
+    }
+    if (cudaMalloc(&w.ptr, want) != cudaSuccess) {
+        cudaGetLastError();
+        w.ptr = nullptr;
+        return WQ_ERR_NO_MEMORY;
+    }
+    if (cudaMemsetAsync(w.ptr, 0, want, stream) != cudaSuccess) return WQ_ERR_CUDA;
+    w.bytes = want;
+    *ptr = w.ptr;
+    return WQ_OK;
+}
+
+// Layout of a workspace: flags [grid] int32 at offset 0, partial tiles from offset 4096 on.
+size_t workspace_bytes_for(const Plan& pl) {
+    return 4096 + static_cast<size_t>(pl.grid) * pl.tile_m * kTileN * 4;
+}
+
+int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* pl) {
+    int mode;
+    int slots = 0;
+    if (kind == 0) {
+        slots = scale_slots(K, g);
+        if (slots < 0) return WQ_ERR_INVALID_ARG;
+        mode = slots > 0 ? kModeGroup : kModeChannel;
+    } else {
+        mode = kModeW4A8;
+    }
+    if (make_plan(mode, M, N, K, slots, d.num_sms, d.smem_optin, pl) != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
+    return WQ_OK;
+}
+
+int encode_activation_map(CUtensorMap* map, const void* A, int M, int K, int tile_m, bool int8) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * (int8 ? 1u : 2u)};
+    const cuuint32_t box[2] = {int8 ? 128u : 64u, static_cast<cuuint32_t>(tile_m)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                          const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? WQ_OK : WQ_ERR_CUDA;
+}
+
+int check_shape(int K, int N) {
+    if (K <= 0 || N <= 0) return WQ_ERR_INVALID_ARG;
+    if (!shape_ok(K, N)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    return WQ_OK;
+}
+
+int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y,
+             int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream) {
+    int rc = check_shape(K, N);
+    if (rc) return rc;
+    if (M < 0) return WQ_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (kind == 0 && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (kind == 1 && K > 131072) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (!Wp) return WQ_ERR_INVALID_ARG;
+    if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
+    if (M == 0) return WQ_OK;
+    if (!A || !Y || (kind == 1 && (!sa || !sw))) return WQ_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(Y, 16) || (acc_out && !aligned(acc_out, 16))) return WQ_ERR_MISALIGNED;
+    if (kind == 1 && (!aligned(sa, 4) || !aligned(sw, 4))) return WQ_ERR_MISALIGNED;
+
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, stream, true);
+    if (rc) return rc;
+    Plan pl;
+    rc = plan_for(kind, M, N, K, g, *d, &pl);
+    if (rc) return rc;
+    void* ws = nullptr;
+    rc = get_workspace(dev, stream, workspace_bytes_for(pl), &ws);
+    if (rc) return rc;
+    CUtensorMap map;
+    rc = encode_activation_map(&map, A, M, K, pl.tile_m, kind == 1);
+    if (rc) return rc;
+
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.wp = static_cast<const uint8_t*>(Wp);
+    a.s_chan = (pl.mode == kModeChannel)
+                   ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
+                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * kCodeBytes)
+                   : nullptr;
+    a.sa = sa;
+    a.sw = sw;
+    a.y = Y;
+    a.acc_out = acc_out;
+    a.ws_flags = static_cast<int*>(ws);
+    a.ws_partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 4096);
+    a.status = d->status;
+    a.M = M;
+    a.N = N;
+    a.m_tiles = pl.m_tiles;
+    a.n_tiles = pl.n_tiles;
+    a.k_blocks = pl.k_blocks;
+    a.tile_m = pl.tile_m;
+    a.stages = pl.stages;
+    a.stage_bytes = pl.stage_bytes;
+    a.act_bytes = pl.act_bytes;
+    a.blob_bytes = pl.blob_bytes;
+    a.group_rows = (kind == 0 && g < kTileK) ? g : kTileK;
+    a.units = pl.units;
+    a.grid = pl.grid;
+    a.timeout_ns = g_timeout_ns;
+    a.skip_publish = g_skip_publish;
+    if (launch_gemm(pl.mode, map, a, pl, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int prepack_common_checks(const void* Q, int K, int N, const void* Wp, cudaStream_t stream) {
+    int rc = check_shape(K, N);
+    if (rc) return rc;
+    if (!Q || !Wp) return WQ_ERR_INVALID_ARG;
+    if (!aligned(Q, 16) || !aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
+    (void)stream;
+    return WQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wq_status_string(int status) {
+    switch (status) {
+        case WQ_OK: return "WQ_OK";
+        case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG: null pointer, negative size or unsupported group size";
+        case WQ_ERR_UNSUPPORTED_SHAPE:
+            return "WQ_ERR_UNSUPPORTED_SHAPE: K must be a multiple of 128, N a multiple of 8, M at most 2^24";
+        case WQ_ERR_MISALIGNED: return "WQ_ERR_MISALIGNED: a pointer breaks the alignment rule";
+        case WQ_ERR_UNSUPPORTED_DEVICE: return "WQ_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (sm_100a)";
+        case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or kernel launch failed";
+        case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: a device-side wait expired";
+        case WQ_ERR_NO_MEMORY: return "WQ_ERR_NO_MEMORY: workspace allocation failed";
+        case WQ_ERR_CAPTURING: return "WQ_ERR_CAPTURING: reserve the workspace before capturing the stream";
+        default: return "WQ_ERR_UNKNOWN";
+    }
+}
+
+int wq_version(void) { return kVersion; }
+
+size_t wq_prepacked_bytes(int K, int N, int g) {
+    if (!shape_ok(K, N)) return 0;
+    const int slots = scale_slots(K, g);
+    if (slots < 0) return 0;
+    const size_t nblob = static_cast<size_t>(n_tiles(N)) * (K / kTileK);
+    if (slots == 0) return nblob * kCodeBytes + channel_tail_bytes(N);
+    return nblob * blob_bytes_w4a16(slots);
+}
+
+size_t wq_prepacked_bytes_w4a8(int K, int N) {
+    if (!shape_ok(K, N)) return 0;
+    return static_cast<size_t>(n_tiles(N)) * (K / kTileK) * kCodeBytes;
+}
+
+int wq_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (!s) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_prepack(Q, s, K, N, g, Wp, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_prepack_w4a8(Q, K, N, Wp, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_unpack(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q_out, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (!s_out) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s_out, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_unpack(Wp, K, N, g, Q_out, s_out, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q_out, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q_out, K, N, Wp, st);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_unpack_w4a8(Wp, K, N, Q_out, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g, void* stream) {
+    return run_gemm(0, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
+}
+
+int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
+                 int M, int N, int K, void* stream) {
+    return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
+}
+
+size_t wq_workspace_bytes(int kind, int M, int N, int K) {
+    if (!shape_ok(K, N) || M <= 0 || (kind != 0 && kind != 1)) return 0;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = device_state(&dev);
+    if (!d || !d->supported) return 0;
+    Plan pl;
+    if (plan_for(kind, M, N, K, kind == 0 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
+    return workspace_bytes_for(pl);
+}
+
+int wq_workspace_reserve(size_t bytes, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    int rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    void* p = nullptr;
+    return get_workspace(dev, st, bytes, &p);
+}
+
+int wq_get_device_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    int rc = require_device(&dev, &d, st, false);
+    if (rc) return rc;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return WQ_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WQ_ERR_CUDA;
+    if (h == WQ_OK) return WQ_OK;
+    // a wait expired: clear the status word and every workspace's flags of this device
+    if (cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess) return WQ_ERR_CUDA;
+    for (auto& kv : g_workspaces)
+        if (kv.first.first == dev && kv.second.ptr)
+            if (cudaMemset(kv.second.ptr, 0, 4096) != cudaSuccess) return WQ_ERR_CUDA;
+    return h;
+}
+
+int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
+    if (!plan) return WQ_ERR_INVALID_ARG;
+    int rc = check_shape(K, N);
+    if (rc) return rc;
+    if (M <= 0) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1) return WQ_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = device_state(&dev);
+    if (!d) return WQ_ERR_CUDA;
+    if (!d->supported) return WQ_ERR_UNSUPPORTED_DEVICE;
+    Plan pl;
+    rc = plan_for(kind, M, N, K, kind == 0 ? g : K, *d, &pl);
+    if (rc) return rc;
+    plan->grid = pl.grid;
+    plan->tile_m = pl.tile_m;
+    plan->m_tiles = pl.m_tiles;
+    plan->n_tiles = pl.n_tiles;
+    plan->k_blocks = pl.k_blocks;
+    plan->stages = pl.stages;
+    plan->smem_bytes = pl.smem_bytes;
+    plan->threads = kThreads;
+    plan->units = pl.units;
+    return WQ_OK;
+}
+
+int wq_debug_set_wait_timeout_ns(unsigned long long ns) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_timeout_ns = ns ? ns : kDefaultTimeoutNs;
+    return WQ_OK;
+}
+
+int wq_debug_skip_publish(int cta) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    g_skip_publish = cta;
+    return WQ_OK;
+}
+
+}  // extern "C"

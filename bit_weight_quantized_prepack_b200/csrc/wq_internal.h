@@ -1,0 +1,55 @@
+// Declarations shared by the library's translation units (not part of the public ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "wq_layout.h"
+
+namespace wq {
+
+// Arguments of the GEMM kernel (all three modes). Pointers are device pointers.
+struct GemmArgs {
+    const uint8_t* wp;         // prepacked blobs
+    const uint16_t* s_chan;    // W4A16, g == K: fp16 column scales (n_tiles*128 entries)
+    const float* sa;           // W4A8: per-token scales [M]
+    const float* sw;           // W4A8: per-column scales [N]
+    uint16_t* y;               // fp16 output [M, N]
+    int32_t* acc_out;          // W4A8: optional int32 accumulators [M, N]
+    float* ws_partial;         // stream-K partial tiles: [grid][tile_m][128] (fp32 or int32 bits)
+    int* ws_flags;             // stream-K publish flags: [grid]
+    int* status;               // device status word (0 = ok)
+    int M, N;
+    int m_tiles, n_tiles, k_blocks;
+    int tile_m;                // MMA N extent (multiple of 16, <= 256)
+    int stages;
+    int stage_bytes;           // bytes of one pipeline stage (activation tile + blob), 1024-aligned
+    int act_bytes;             // bytes of the activation tile of one stage
+    int blob_bytes;            // bytes of one weight blob
+    int group_rows;            // W4A16 grouped: rows per scale slot, min(g, 128)
+    long long units;           // tiles * k_blocks
+    int grid;
+    unsigned long long timeout_ns;
+    int skip_publish;          // test hook: CTA that skips publishing its partial (-1: none)
+};
+
+struct Plan {
+    int mode;
+    int tile_m, m_tiles, n_tiles, k_blocks;
+    long long units;
+    int grid, stages, stage_bytes, act_bytes, blob_bytes, smem_bytes;
+};
+
+int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan);
+
+cudaError_t configure_gemm_kernels(int max_dynamic_smem);
+
+cudaError_t launch_gemm(int mode, const CUtensorMap& tmap, const GemmArgs& args, const Plan& plan,
+                        cudaStream_t stream);
+
+int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, cudaStream_t st);
+int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t st);
+int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st);
+int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st);
+
+}  // namespace wq

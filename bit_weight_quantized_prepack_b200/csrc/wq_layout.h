@@ -1,0 +1,62 @@
+// Tile geometry and prepacked-weight layout of the library (host and device).
+//
+// Prepacked W4A16 buffer (the layout pass named by "Efficient Arbitrary Precision
+// Acceleration for Large Language Models on GPU Tensor Cores", Abstract: matrix
+// preprocessing that reorders data for the kernel; the layout itself is this library's):
+//   n-tiles of 128 columns (NT = ceil(N/128)), k-blocks of 128 rows (KT = K/128).
+//   Blob (nt, kt) starts at byte (nt*KT + kt) * blob_bytes, so the k-blocks of one column
+//   tile are contiguous. A blob is
+//     8192 bytes of code words: word ((h*2 + v)*128 + r)*4 + i  (h, v in {0,1}, r < 128,
+//       i < 4) holds the 8 codes of column nt*128 + r, rows kt*128 + 64h + 32v + 8i + j
+//       (j = 0..7), code j at nibble position kNibblePos[j];
+//     then `slots` rows of 128 fp16 scales (slot u covers rows kt*128 + u*min(g,128) ..).
+//   For g == K the blobs hold codes only and one row of fp16 column scales (padded to
+//   NT*128 entries, then to 16 bytes) follows the last blob.
+//   Columns past N hold code 8 and scale 0: zero weights.
+// Prepacked W4A8 buffer: the same blobs, codes only, with the W4A8 nibble order.
+//
+// Nibble orders. Within a word the W4A16 order puts codes (2p, 2p+1) at nibble positions
+// (p, p+4) for p = 0..3, so that masking 0x000F000F (p = 0) or 0x00F000F0 (p = 1) of the
+// word, or of the word shifted right by 8 (p = 2, 3), leaves one code in each 16-bit half:
+// the two halves become the fp16 pair (k, k+1). The W4A8 order puts codes 0..3 at the low
+// nibbles of bytes 0..3 and codes 4..7 at the high nibbles, so that two masks yield four
+// int8 lanes in k order each.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+namespace wq {
+
+constexpr int kTileN = 128;                   // weight columns per tile = tcgen05 M extent
+constexpr int kTileK = 128;                   // weight rows per k-block = one pipeline stage
+constexpr int kCodeBytes = kTileN * kTileK / 2;  // 8192 bytes of 4-bit codes per blob
+constexpr int kNumDqWarps = 8;                // dequant + epilogue warps (2 per TMEM lane quarter)
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = (kNumDqWarps + 2) * 32;
+constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
+constexpr int kMaxStages = 24;
+constexpr int kASlots = 4;                    // dequantised weight tiles in tensor memory
+constexpr int kTmemCols = 512;
+constexpr int kTmemAOffset = 256;             // accumulator in columns [0, 256), A slots above
+
+enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2 };
+
+// Scale rows per blob for W4A16; 0 means per-column scales (g == K); -1 unsupported.
+inline int scale_slots(int K, int g) {
+    if (g <= 0 || K <= 0 || K % g) return -1;
+    if (g == K) return 0;
+    if (g == 32 || g == 64 || g == 128) return kTileK / g;
+    if (g % kTileK == 0) return 1;
+    return -1;
+}
+
+inline bool shape_ok(int K, int N) { return K > 0 && K % kTileK == 0 && N > 0 && N % 8 == 0; }
+
+inline int n_tiles(int N) { return (N + kTileN - 1) / kTileN; }
+
+inline size_t blob_bytes_w4a16(int slots) { return kCodeBytes + 2u * kTileN * static_cast<size_t>(slots); }
+
+inline size_t channel_tail_bytes(int N) { return ((2u * n_tiles(N) * kTileN) + 15u) / 16u * 16u; }
+
+}  // namespace wq

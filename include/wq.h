@@ -1,0 +1,157 @@
+/*
+ * wq.h -- C ABI of the 4-bit weight-quantised linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes Y[M,N] = A[M,K] . W[K,N], with W[k,n] = (q[k,n] - 8) * s[k/g, n]:
+ *   - "MARLIN: Mixed-Precision Auto-Regressive Parallel Inference on Large Language Models",
+ *     Abstract: a linear layer with weights quantised to 4 bits per element and fp16
+ *     activations, kept memory-bound over batch sizes 1..128 by asynchronous memory access,
+ *     task scheduling, pipelining and bespoke quantisation support;
+ *   - "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving", method:
+ *     fine-grained group quantisation (one scale per group of g rows and column) and
+ *     per-token dynamic activation scales;
+ *   - "A Speed Odyssey for Deployable Quantization of LLMs", Abstract: the W4A8 kernel
+ *     (int8 activations x 4-bit weights), exposed here as wq_gemm_w4a8;
+ *   - "Efficient Arbitrary Precision Acceleration for Large Language Models on GPU Tensor
+ *     Cores", Abstract: a matrix preprocessing step that reorders the weights into the
+ *     layout the kernel reads, exposed here as wq_prepack / wq_prepack_w4a8.
+ *
+ * Conventions shared by every entry point
+ *   - Matrices are dense and row-major. fp16 values are passed as their IEEE binary16 bit
+ *     patterns (uint16_t).
+ *   - Q holds the 4-bit codes packed 8 per int32 along K: Q is [K/8, N] and code
+ *     q[8i+j, n] sits in bits 4j..4j+3 of Q[i, n] (lowest nibble first).
+ *   - Every tensor pointer is a DEVICE pointer on the current CUDA device, owned by the
+ *     caller; the library never frees or retains it beyond the call's stream work.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     Calls are stream-ordered and asynchronous: they enqueue work and return without
+ *     waiting for the device.
+ *   - Shapes: K a positive multiple of 128, N a positive multiple of 8, 0 <= M <= 2^24.
+ *     M == 0 returns WQ_OK and launches nothing. Group size g: 32, 64, 128, any multiple
+ *     of 128 that divides K, or g == K (one scale per column).
+ *   - Alignment: A, Q, s, Wp, Y, acc_out: 16 bytes; sa, sw: 4 bytes.
+ *   - All preconditions are checked on the host before any launch; a failed check
+ *     returns an error status and launches nothing. Launch failures return WQ_ERR_CUDA.
+ *     Device-side waits are time-bounded; a wait that expires records WQ_ERR_TIMEOUT in a
+ *     per-device status word that wq_get_device_status reports. No call traps or aborts.
+ *   - Entry points are thread-safe. Calls in flight at the same time on DIFFERENT streams
+ *     use different library workspaces and do not interfere.
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WQ_API __attribute__((visibility("default")))
+#else
+#define WQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad group size */
+    WQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K not a multiple of 128, N not a multiple of 8, M too large */
+    WQ_ERR_MISALIGNED = 3,         /* a pointer breaks the alignment rule above */
+    WQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+    WQ_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+    WQ_ERR_TIMEOUT = 6,            /* a device-side bounded wait expired (see wq_get_device_status) */
+    WQ_ERR_NO_MEMORY = 7,          /* the library could not allocate its workspace */
+    WQ_ERR_CAPTURING = 8           /* the workspace must grow while the stream is being captured */
+} wq_status_t;
+
+/* Human-readable name of a status code. Never NULL. */
+WQ_API const char* wq_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+WQ_API int wq_version(void);
+
+/* ---------------------------------------------------------------- prepack (the layout pass)
+ * Size in bytes of the prepacked W4A16 buffer for a K x N weight with group size g, or 0
+ * when (K, N, g) is not supported. Layout: blobs of 128 columns x 128 rows, each 8192
+ * bytes of reordered codes followed by that blob's fp16 group scales; for g == K a single
+ * row of fp16 column scales follows all blobs instead. */
+WQ_API size_t wq_prepacked_bytes(int K, int N, int g);
+
+/* Size in bytes of the prepacked W4A8 buffer (codes only), or 0 when unsupported. */
+WQ_API size_t wq_prepacked_bytes_w4a8(int K, int N);
+
+/* Reorder codes Q [K/8, N] int32 and fp16 scales s [K/g, N] into Wp (caller-allocated,
+ * wq_prepacked_bytes(K,N,g) bytes). Columns padded up to a multiple of 128 get code 8 and
+ * scale 0, i.e. zero weights. Runs once per weight; Wp is read-only afterwards. */
+WQ_API int wq_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, void* stream);
+
+/* Reorder codes Q [K/8, N] into the W4A8 layout Wp (wq_prepacked_bytes_w4a8 bytes). */
+WQ_API int wq_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, void* stream);
+
+/* Inverse of wq_prepack: recovers Q [K/8, N] and s [K/g, N] bit for bit (test aid). */
+WQ_API int wq_unpack(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, void* stream);
+
+/* Inverse of wq_prepack_w4a8 (test aid). */
+WQ_API int wq_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q_out, void* stream);
+
+/* ---------------------------------------------------------------- the layer
+ * W4A16: Y[M,N] (fp16) = A[M,K] (fp16) . W, W from the prepacked Wp of the same (K, N, g).
+ * Products accumulate in fp32; Y is rounded to nearest-even fp16. For g < K the weight
+ * (q-8)*s is rounded once to fp16 before the product; for g == K the column scale is
+ * applied to the fp32 sum instead. Uses the workspace of (current device, stream).
+ * Results are deterministic: the same call gives the same bits every time. */
+WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
+                  int M, int N, int K, int g, void* stream);
+
+/* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
+ * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
+ * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
+ * Requires K <= 131072 so that no int32 partial sum can overflow. */
+WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw,
+                 uint16_t* Y, int32_t* acc_out, int M, int N, int K, void* stream);
+
+/* ---------------------------------------------------------------- workspace and status
+ * Bytes of library workspace one call of the given kind and shape needs
+ * (kind 0 = W4A16, 1 = W4A8). */
+WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
+
+/* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it
+ * before capturing the stream into a CUDA graph: a call that has to grow the workspace
+ * while the stream is capturing returns WQ_ERR_CAPTURING. Synchronises `stream` when it
+ * grows the buffer. */
+WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
+
+/* Synchronise `stream`, then return and clear the current device's status word:
+ * WQ_OK, or WQ_ERR_TIMEOUT when a device-side wait expired since the last call (the
+ * outputs of that call are then undefined). On error it also clears the device's
+ * workspace flags so that later calls start clean. */
+WQ_API int wq_get_device_status(void* stream);
+
+/* ---------------------------------------------------------------- introspection and test hooks
+ * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8. */
+typedef struct {
+    int grid;         /* persistent CTAs launched (<= number of SMs) */
+    int tile_m;       /* activation rows per tile (the MMA's N extent) */
+    int m_tiles;      /* tiles along M */
+    int n_tiles;      /* tiles of 128 columns along N */
+    int k_blocks;     /* blocks of 128 rows along K */
+    int stages;       /* shared-memory pipeline depth */
+    int smem_bytes;   /* dynamic shared memory per CTA */
+    int threads;      /* threads per CTA */
+    long long units;  /* (tile, k-block) work units split across the CTAs */
+} wq_plan_t;
+WQ_API int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan);
+
+/* Test hooks. wq_debug_set_wait_timeout_ns sets the limit of every device-side wait
+ * (default 2e9 ns; 0 restores the default). wq_debug_skip_publish(c) makes CTA c skip
+ * publishing its partial sum to the tile that owns it (c = -1 disables), so that the
+ * owner's bounded wait expires: the call then reports WQ_ERR_TIMEOUT through
+ * wq_get_device_status instead of hanging. Both apply to later calls on every device. */
+WQ_API int wq_debug_set_wait_timeout_ns(unsigned long long ns);
+WQ_API int wq_debug_skip_publish(int cta);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */
