@@ -1,0 +1,438 @@
+"""Benchmark of the W4A16 linear layer: effective HBM GB/s and TFLOP/s against the roofline.
+
+One step = the Llama-7B-shaped W4A16 layer set ((K, N) = (4096, 12288) fused QKV,
+(4096, 4096) out-proj, (4096, 22016) gate+up, (11008, 4096) down; g = 128) at every batch
+size M in {1, 2, 4, 8, 16, 32, 64, 128}: 32 calls of the layer. Inputs are seeded synthetic
+data with the distributions of the layer configuration (fp16 N(0,1) activations, uniform
+4-bit codes, fp16 scales 0.002 + 0.01|N(0,1)|). Prepacking happens once, outside timing.
+
+Four prepacked copies of the layer set (404 MB of weights) rotate across the M values, so a
+copy is re-read only after three other copies (303 MB) went through the 126 MB L2: every
+weight byte of a call comes from HBM. The step is captured once in a CUDA graph and replayed.
+
+Printed: one JSON line (rank 0). ``value`` = algorithmic bytes of all ranks' steps / the
+slowest rank's device time (GB/s); algorithmic bytes of one call = K*N/2 (codes) +
+2*(K/g)*N (scales) + 2*M*K (A) + 2*M*N (Y). ``--gpus N`` runs N independent replicas (the
+layer does not shard across GPUs here), one process per GPU under torchrun.
+``--impl reference`` times the CPU fp64 oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+LAYERS = [(4096, 12288), (4096, 4096), (4096, 22016), (11008, 4096)]
+M_SWEEP = [1, 2, 4, 8, 16, 32, 64, 128]
+G = 128
+COPIES = 4
+METRIC = "W4A16 GEMM TFLOP/s and effective HBM GB/s vs roofline fraction at M=1..128"
+WORKLOAD = "llama7b_w4a16_layer_set_M1-128_g128"
+
+# Fallback denominators (an earlier measurement on this machine) when MEASURED_PEAKS.json is absent.
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+# DRAM traffic per launch of the GEMM kernel over this step's 32 launches, from the ncu capture
+# summarised in profiles/wq_gemm_w4a16_llama7b_step.md, valid for the kernel sources whose
+# hash is recorded with it. Null when the kernel changed since.
+TRAFFIC = {"kernel_sha": None, "bytes_per_launch": None}
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_weight_quantized_prepack_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def algo_bytes(M, K, N, g=G):
+    return K * N // 2 + 2 * (K // g) * N + 2 * M * K + 2 * M * N
+
+
+def algo_flops(M, K, N):
+    return 2 * M * N * K
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def step_totals():
+    b = sum(algo_bytes(M, K, N) for M in M_SWEEP for (K, N) in LAYERS)
+    f = sum(algo_flops(M, K, N) for M in M_SWEEP for (K, N) in LAYERS)
+    return b, f
+
+
+def roofline_time(M, K, N, hbm_gbs, tflops):
+    return max(algo_bytes(M, K, N) / (hbm_gbs * 1e9), algo_flops(M, K, N) / (tflops * 1e12))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+        self.t_start = self.t_stop = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, "t_" + which, datetime.datetime.now())
+
+    def stop(self):
+        time.sleep(0.15)
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t_start and self.t_stop and self.t_start <= r[0] <= self.t_stop]
+        used = inside if inside else rows
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        sm = [float(r[1][2]) for r in used if r[1][2].replace(".", "").isdigit()]
+        smax = [float(r[1][3]) for r in used if r[1][3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in used for i, v in enumerate(r[1][6:10]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------------ our implementation
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_weight_quantized_prepack_b200 as wq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    hbm_gbs, tflops, tflops_sus, peak_src = peaks()
+
+    # inputs: one seeded draw per layer; A holds 128 rows, smaller M use the first rows
+    layers = []
+    for li, (K, N) in enumerate(LAYERS):
+        d = synth.w4a16_inputs(K, N, G, max(M_SWEEP), seed=li)
+        Q = torch.from_numpy(d["Q"]).to(dev)
+        s = torch.from_numpy(d["s"]).to(dev)
+        Wp0 = wq.wq_prepack(Q, s, G)
+        copies = [Wp0] + [Wp0.clone() for _ in range(COPIES - 1)]
+        A = torch.from_numpy(d["A"]).to(dev)
+        layers.append({"K": K, "N": N, "Wp": copies, "A": {M: A[:M].contiguous() for M in M_SWEEP},
+                       "Y": {M: torch.empty((M, N), dtype=torch.float16, device=dev) for M in M_SWEEP},
+                       "A_host": {M: A[:M].cpu().pin_memory() for M in M_SWEEP},
+                       "Y_host": {M: torch.empty((M, N), dtype=torch.float16).pin_memory() for M in M_SWEEP}})
+        del Q, s
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+    ws = max(wq.wq_workspace_bytes(0, M, L["N"], L["K"]) for M in M_SWEEP for L in layers)
+    wq.wq_workspace_reserve(ws, stream=stream)
+
+    def step_calls(st):
+        for mi, M in enumerate(M_SWEEP):
+            c = mi % COPIES
+            for L in layers:
+                wq.wq_gemm_w4a16(L["A"][M], L["Wp"][c], L["N"], G, Y=L["Y"][M], stream=st)
+
+    launches_per_step = len(M_SWEEP) * len(LAYERS)
+    with torch.cuda.stream(stream):
+        step_calls(stream)  # eager once (also checks the status path)
+    stream.synchronize()
+    if wq.wq_get_device_status(stream) != wq.WQ_OK:
+        raise RuntimeError("device status not OK after the first step")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            step_calls(stream)
+    stream.synchronize()
+
+    for _ in range(args.warmup):
+        with torch.cuda.stream(stream):
+            graph.replay()
+    stream.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "") or "")
+    sampler = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local_rank)))
+    sampler.start()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("start")
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("stop")
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    t_local = ev0.elapsed_time(ev1) / 1e3
+    t = t_local
+    if world > 1:
+        tt = torch.tensor([t_local], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    if wq.wq_get_device_status(stream) != wq.WQ_OK:
+        raise RuntimeError("device status not OK after the timed region")
+
+    bytes_step, flops_step = step_totals()
+    value = world * bytes_step * args.steps / t / 1e9
+    ms_per_step = t / args.steps * 1e3
+
+    # ---------------------------------------------------------- end to end through the public API
+    # every call: pinned host A -> device, the layer, device Y -> pinned host, all inside the timed region
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    h2d = sum(2 * M * L["K"] for M in M_SWEEP for L in layers)
+    d2h = sum(2 * M * L["N"] for M in M_SWEEP for L in layers)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            for mi, M in enumerate(M_SWEEP):
+                c = mi % COPIES
+                for L in layers:
+                    L["A"][M].copy_(L["A_host"][M], non_blocking=True)
+                    wq.wq_gemm_w4a16(L["A"][M], L["Wp"][c], L["N"], G, Y=L["Y"][M], stream=stream)
+                    L["Y_host"][M].copy_(L["Y"][M], non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    te = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([te], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        te = float(tt.item())
+    e2e_value = world * bytes_step * e2e_steps / te / 1e9
+
+    # ---------------------------------------------------------- per-M breakdown (rank 0, outside timing)
+    per_m = {}
+    if rank == 0 and not args.no_breakdown:
+        for mi, M in enumerate(M_SWEEP):
+            g2 = torch.cuda.CUDAGraph()
+            reps = 8
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(g2, stream=stream):
+                    for r in range(reps):
+                        for L in layers:
+                            wq.wq_gemm_w4a16(L["A"][M], L["Wp"][r % COPIES], L["N"], G, Y=L["Y"][M], stream=stream)
+                g2.replay()
+                stream.synchronize()
+                a0 = torch.cuda.Event(enable_timing=True)
+                a1 = torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                for _ in range(10):
+                    g2.replay()
+                a1.record(stream)
+            stream.synchronize()
+            tm = a0.elapsed_time(a1) / 1e3 / (10 * reps)
+            b = sum(algo_bytes(M, L["K"], L["N"]) for L in layers)
+            f = sum(algo_flops(M, L["K"], L["N"]) for L in layers)
+            troof = sum(roofline_time(M, L["K"], L["N"], hbm_gbs, tflops) for L in layers)
+            per_m[str(M)] = {"us": round(tm * 1e6, 2), "gbs": round(b / tm / 1e9, 1),
+                             "tflops": round(f / tm / 1e12, 2), "roofline_frac": round(troof / tm, 3)}
+            del g2
+
+    troof_step = sum(roofline_time(M, K, N, hbm_gbs, tflops) for M in M_SWEEP for (K, N) in LAYERS)
+    achieved = bytes_step / (t_local / args.steps) / 1e9  # per-launch average over the step's launches
+    sha = kernel_sha()
+    traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["kernel_sha"] == sha else None
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers_KN": LAYERS, "M": M_SWEEP, "g": G,
+                   "l2": f"inputs larger than L2: {COPIES} rotated prepacked copies of the layer set "
+                         f"({COPIES * sum(K * N // 2 + 2 * (K // G) * N for K, N in LAYERS) / 1e6:.0f} MB)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "tflops": round(world * flops_step * args.steps / t / 1e12, 2),
+        "roofline_time_frac": round(troof_step / (t_local / args.steps), 3),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": round(achieved / hbm_gbs, 3), "traffic": traffic,
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                     "note": "achieved = algorithmic bytes of the step's 32 launches / step device time"},
+        "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "per_m": per_m,
+        "kernel_sha": sha,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_sample)
+    del graph
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ the oracle as the CPU baseline
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def _oracle_pairs():
+    return [(M, K, N, li) for M in M_SWEEP for li, (K, N) in enumerate(LAYERS)]
+
+
+def cpu_baseline(n_pairs: int):
+    """The oracle as it stands, on the host cores, over the first n (M, layer) pairs of the step."""
+    import oracle
+    pairs = _oracle_pairs()[:n_pairs]
+    inputs = {li: synth.w4a16_inputs(K, N, G, max(M_SWEEP), seed=li) for li, (K, N) in enumerate(LAYERS)}
+    t0 = time.perf_counter()
+    b = 0
+    for (M, K, N, li) in pairs:
+        d = inputs[li]
+        oracle.w4a16(d["A"][:M], d["Q"], d["s"], G)
+        b += algo_bytes(M, K, N)
+    dt = time.perf_counter() - t0
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{len(pairs)} of the step's 32 (M, layer) calls, fp64 dequantise + numpy BLAS matmul, "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle timed on this host, same metric and workload, rank 0 only.
+
+    One step = the oracle on one (M, layer) call of the step, cycling through the 32 calls,
+    restricted to a block of output columns sized so that the whole run stays near
+    ``--reference-budget`` seconds whatever --steps is. The bytes counted are the algorithmic
+    bytes of the columns computed.
+    """
+    if rank != 0:
+        return
+    import oracle
+    pairs = _oracle_pairs()
+    inputs = {li: synth.w4a16_inputs(K, N, G, max(M_SWEEP), seed=li) for li, (K, N) in enumerate(LAYERS)}
+    # calibration (untimed): seconds per output column of each layer at M = 128
+    per_col = {}
+    for li, (K, N) in enumerate(LAYERS):
+        d = inputs[li]
+        c = min(N, 1024)
+        t0 = time.perf_counter()
+        oracle.w4a16(d["A"], d["Q"][:, :c], d["s"][:, :c], G)
+        per_col[li] = (time.perf_counter() - t0) / c
+    per_step = args.reference_budget / max(1, args.steps + args.warmup)
+
+    def one(i):
+        M, K, N, li = pairs[i % len(pairs)]
+        d = inputs[li]
+        cols = int(min(N, max(8, per_step / per_col[li]))) // 8 * 8
+        n0 = (i * 4096) % (N - cols + 1)
+        oracle.w4a16(d["A"][:M], d["Q"][:, n0:n0 + cols], d["s"][:, n0:n0 + cols], G)
+        return algo_bytes(M, K, cols), cols
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    b = 0
+    ncols = 0
+    for i in range(args.steps):
+        bi, ci = one(args.warmup + i)
+        b += bi
+        ncols += ci
+    dt = time.perf_counter() - t0
+    v = b / dt / 1e9
+    sample = (f"{args.steps} steps, each the fp64 oracle on one (M, layer) call of the 32, "
+              f"{ncols / args.steps:.0f} output columns on average, {dt:.1f} s")
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "layers_KN": LAYERS, "M": M_SWEEP, "g": G,
+                      "step": "one (M, layer) call of the layer set on a block of output columns"},
+           "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-sample", type=int, default=32, help="(M, layer) calls the oracle baseline times")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true", help="skip the per-M breakdown (short profiler runs)")
+    ap.add_argument("--reference-budget", type=float, default=90.0, help="seconds the reference arm aims for")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("for --gpus N > 1 launch with torchrun --nproc-per-node N")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -144,16 +144,28 @@ int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* p
     return WQ_OK;
 }
 
-int encode_activation_map(CUtensorMap* map, const void* A, int M, int K, int tile_m, bool int8) {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * (int8 ? 1u : 2u)};
-    const cuuint32_t box[2] = {int8 ? 128u : 64u, static_cast<cuuint32_t>(tile_m)};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                          const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? WQ_OK : WQ_ERR_CUDA;
+// Activation maps for chunks of 1..chunk k-blocks. A [M, K] is seen as 3-D with the k-block
+// split into swizzle-wide pieces: dims {64 fp16 or 128 int8, M, K/piece}, strides {K*elem (rows),
+// piece bytes}; a box of {piece, tile_m, c*pieces_per_kblock} lands in shared memory as
+// [piece index][row][128 bytes], the K-major 128-byte-swizzled layout the MMA reads.
+int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_m, int chunk, bool int8) {
+    const int piece = int8 ? 128 : 64;                 // elements per 128-byte row
+    const int per_kblock = kTileK / piece;             // 1 (int8) or 2 (fp16)
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(piece), static_cast<cuuint64_t>(M),
+                                static_cast<cuuint64_t>(K / piece)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * (int8 ? 1u : 2u), 128u};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    std::memset(maps, 0, sizeof(*maps));
+    for (int c = 1; c <= chunk; ++c) {
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(piece), static_cast<cuuint32_t>(tile_m),
+                                   static_cast<cuuint32_t>(c * per_kblock)};
+        CUresult r = g_encode(&maps->m[c - 1], int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                              const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
 }
 
 int check_shape(int K, int N) {
@@ -188,8 +200,8 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     void* ws = nullptr;
     rc = get_workspace(dev, stream, workspace_bytes_for(pl), &ws);
     if (rc) return rc;
-    CUtensorMap map;
-    rc = encode_activation_map(&map, A, M, K, pl.tile_m, kind == 1);
+    ActMaps maps;
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1);
     if (rc) return rc;
 
     GemmArgs a;
@@ -212,16 +224,21 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.n_tiles = pl.n_tiles;
     a.k_blocks = pl.k_blocks;
     a.tile_m = pl.tile_m;
-    a.stages = pl.stages;
-    a.stage_bytes = pl.stage_bytes;
-    a.act_bytes = pl.act_bytes;
+    a.issuers = pl.issuers;
+    a.slots = pl.slots;
+    a.chunk = pl.chunk;
+    a.act_slot = pl.act_slot;
     a.blob_bytes = pl.blob_bytes;
     a.group_rows = (kind == 0 && g < kTileK) ? g : kTileK;
+    a.small = pl.small ? 1 : 0;
+    // large tiles round (q - 8) * s to fp16 in the dequant; small tiles apply a group scale of
+    // g >= 128 to each k-block's fp32 partial instead (g = 32, 64 stay in the dequant)
+    a.scale_in_dequant = (pl.mode == kModeGroup && (!pl.small || g < kTileK)) ? 1 : 0;
     a.units = pl.units;
     a.grid = pl.grid;
     a.timeout_ns = g_timeout_ns;
     a.skip_publish = g_skip_publish;
-    if (launch_gemm(pl.mode, map, a, pl, stream) != cudaSuccess) {
+    if (launch_gemm(pl.mode, maps, a, pl, stream) != cudaSuccess) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -412,9 +429,9 @@ int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
     plan->m_tiles = pl.m_tiles;
     plan->n_tiles = pl.n_tiles;
     plan->k_blocks = pl.k_blocks;
-    plan->stages = pl.stages;
+    plan->stages = pl.slots;
     plan->smem_bytes = pl.smem_bytes;
-    plan->threads = kThreads;
+    plan->threads = pl.threads;
     plan->units = pl.units;
     return WQ_OK;
 }

@@ -11,19 +11,33 @@
 //     its N operand (tile_m rows, 16..256), so even M = 1 uses a legal tcgen05 shape.
 //   * One persistent CTA per SM walks a contiguous range of (tile, k-block) units (stream-K).
 //     A tile split between CTAs is finished by the CTA holding its last k-block, which adds
-//     the other CTAs' fp32 partials in a fixed order: results are deterministic.
-//   * Warp roles per CTA (320 threads):
-//       warp 8      TMA producer: one bulk copy per weight blob (codes + scales, contiguous in
-//                   HBM by construction of the prepack) and 2-D tensor copies of the
-//                   activation tile (128-byte swizzle), into a ring of `stages` buffers;
+//     the other CTAs' partial sums in a fixed order: results are deterministic.
+//   * Warp roles per CTA:
+//       warp 12     weight producer: one bulk copy moves up to 4 consecutive blobs (codes +
+//                   scales of 4 k-blocks, contiguous in HBM by construction of the prepack);
+//       warp 13     activation producer: one 3-D tensor copy moves the same k-blocks of the
+//                   activation tile (128-byte swizzle, the MMA's K-major B layout);
 //       warps 0..7  dequantisation: each thread owns one weight column of the tile (one
-//                   tensor-memory lane) and half of the k-block; it turns 8 packed words into
+//                   tensor-memory lane) and half of each k-block; it turns 8 packed words into
 //                   64 fp16 (or int8) values in registers and stores them into tensor memory,
 //                   where they are the MMA's A operand: the dequantised weights never touch
-//                   shared memory. The same warps run the epilogue;
-//       warp 9      MMA issuer: tcgen05.mma with A from tensor memory, B (activations) from
-//                   shared memory, accumulator in tensor memory; commits release the buffers.
-//     Dequantisation of k-block i+1 overlaps the MMA of k-block i (4 tensor-memory slots).
+//                   shared memory;
+//       warps 8..11 MMA issuers, one accumulator each.
+//     Two ways to split the MMAs, by tile height:
+//       small tiles (tile_m <= 32, the memory-bound decode regime; 576 threads): issuer q owns
+//                   every fourth k-block and writes each k-block's product into a fresh
+//                   partial; warps 14..17 add the partials in k order in fp32 registers,
+//                   applying the group scale there (acc += s * P), and run the epilogue
+//                   while the other warps stream the next tile. The dequant then emits exact
+//                   (q - 8) and skips the per-weight scale multiply (for g >= 128);
+//       large tiles (448 threads): issuer q owns a quarter (or half, or all) of every
+//                   k-block's K range and accumulates the whole segment in tensor memory; the
+//                   dequant applies the scale and its warps run the epilogue.
+//     Measured on B200: a thread issuing tcgen05.mma back to back gets one instruction per
+//     ~75-85 cycles whatever the shape, and one issuing bulk copies gets one copy per ~270 ns;
+//     several issuing warps and copies of 16-33 KB take both costs off the critical path.
+//     Integer ALU and packed-fp16 instructions each run at 16 lanes per cycle per SM
+//     sub-partition, so the dequant instruction count sets the small-M ceiling.
 //   * Every wait is bounded by a global-timer limit; an expired wait records WQ_ERR_TIMEOUT
 //     and the CTA winds down (drains its copies and MMAs, frees tensor memory) instead of
 //     hanging.
@@ -38,16 +52,19 @@
 namespace wq {
 
 struct Barriers {
-    uint64_t full[kMaxStages];    // stage loaded (TMA transaction bytes)
-    uint64_t empty[kMaxStages];   // stage consumed (8 dequant warps + 1 MMA commit)
-    uint64_t afull[kASlots];      // dequantised weights in tensor memory (8 warps)
-    uint64_t aempty[kASlots];     // MMA finished reading a tensor-memory slot (commit)
-    uint64_t dfull;               // accumulator of a segment complete (commit)
-    uint64_t drain;               // all MMAs of the CTA complete (commit)
+    uint64_t full[kMaxSlots];      // chunk landed: both producers' bytes (count 2 + transactions)
+    uint64_t empty_w[kMaxSlots];   // weight slot read by the 8 dequant warps
+    uint64_t empty_a[kMaxSlots];   // activation slot read by the MMAs of every issuer (commits)
+    uint64_t afull[kASlots][2];    // dequantised half-k-block in tensor memory (4 warps each)
+    uint64_t aempty[kASlots];      // every issuer's MMAs done with a tensor-memory slot
+    uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
+    uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
+    uint64_t pfull[kMaxIssuers];   // small tiles: an issuer's per-k-block partial is ready (commit)
+    uint64_t pempty[kMaxIssuers];  // small tiles: the accumulate warps have read it (4 warps)
 };
 
 struct Ctl {
-    volatile int* abort_flag;     // shared: set by the first wait that gives up
+    volatile int* abort_flag;      // shared: set by the first wait that gives up
     int* status;
     unsigned long long timeout_ns;
 };
@@ -58,15 +75,18 @@ __device__ __forceinline__ void raise_error(const Ctl& c, int code) {
 }
 
 // Bounded wait on an mbarrier phase. Returns false when the CTA aborts or the limit expires.
+// The global timer is read only every 32 unsuccessful polls.
 __device__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c, bool honour_abort = true) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (true) {
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (honour_abort && *c.abort_flag) return false;
-        if (global_timer_ns() - t0 > c.timeout_ns) {
-            raise_error(c, WQ_ERR_TIMEOUT);
-            return false;
+        if ((i & 31) == 0) {
+            if (honour_abort && *c.abort_flag) return false;
+            if (global_timer_ns() - t0 > c.timeout_ns) {
+                raise_error(c, WQ_ERR_TIMEOUT);
+                return false;
+            }
         }
     }
 }
@@ -82,7 +102,7 @@ __device__ bool wait_flag(const int* flag, const Ctl& c) {
             raise_error(c, WQ_ERR_TIMEOUT);
             return false;
         }
-        __nanosleep(100);
+        __nanosleep(64);
     }
 }
 
@@ -91,10 +111,11 @@ __device__ __forceinline__ long long unit_start(int c, long long units, int grid
     return static_cast<long long>(c) * units / grid;
 }
 
-// Walks a CTA's unit range [beg, end) backwards, one segment (a run of k-blocks of one tile)
-// at a time. Going backwards makes the CTA holding a tile's last k-block, which finishes the
-// tile, the one that reaches that tile last, while the CTAs it waits for have lower indices
-// and reach their part of the tile first.
+// Walks a CTA's unit range [beg, end) one segment (a run of k-blocks of one tile) at a time,
+// last segment first. Going backwards makes the CTA holding a tile's last k-block, which
+// finishes the tile, reach that tile last, while the CTAs it waits for have lower indices
+// and reach their part of the tile first. Inside a segment the k-blocks go forward, so the
+// blobs of a chunk are contiguous in HBM and in the shared-memory ring.
 struct SegCursor {
     long long it, beg;
     int k_blocks;
@@ -114,6 +135,15 @@ struct SegCursor {
         return true;
     }
 };
+
+// Length of the chunk that starts at k-block kb of a segment ending at kb_hi, at ring slot pos:
+// at most `chunk` k-blocks, never past the segment, never wrapping the ring.
+__device__ __forceinline__ int chunk_len(int chunk, int kb, int kb_hi, int pos, int slots) {
+    int c = kb_hi - kb + 1;
+    if (c > chunk) c = chunk;
+    if (c > slots - pos) c = slots - pos;
+    return c;
+}
 
 // ------------------------------------------------------------------ dequantisation
 // fp16 constants from the binary16 format: 0x6400 = 1024 (exponent field 25, so the 10
@@ -156,6 +186,25 @@ __device__ __forceinline__ void dequant_word_i8(uint32_t x, uint32_t* out) {
 }
 
 // ------------------------------------------------------------------ epilogue
+// Sum of the issuers' accumulators for 8 columns (fixed order), as raw 32-bit values.
+template <int MODE>
+__device__ __forceinline__ void load_acc8(uint32_t taddr, int issuers, int tile_m, uint32_t (&v)[8]) {
+    tmem_ld_x8(taddr, v);
+    for (int q = 1; q < issuers; ++q) {
+        uint32_t w[8];
+        tmem_ld_x8(taddr + static_cast<uint32_t>(q * tile_m), w);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (MODE == kModeW4A8)
+                v[j] = static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(w[j]));
+            else
+                v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
+        }
+    }
+    tmem_ld_wait();
+}
+
 template <int MODE>
 __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ctl& ctl, const SegCursor& seg,
                          int seg_index, int half, int quarter, int lane) {
@@ -176,8 +225,7 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
         for (int c = 0; c < cols; c += 8) {
             uint32_t v[8];
             if (ok) {
-                tmem_ld_x8(tmem + lane_base + static_cast<uint32_t>(c_begin + c), v);
-                tmem_ld_wait();
+                load_acc8<MODE>(tmem + lane_base + static_cast<uint32_t>(c_begin + c), p.issuers, p.tile_m, v);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) part[static_cast<size_t>(c_begin + c + j) * kTileN + row] = v[j];
             }
@@ -210,8 +258,7 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
     for (int c = 0; c < cols; c += 8) {
         uint32_t v[8];
         if (!ok) continue;
-        tmem_ld_x8(tmem + lane_base + static_cast<uint32_t>(c_begin + c), v);
-        tmem_ld_wait();
+        load_acc8<MODE>(tmem + lane_base + static_cast<uint32_t>(c_begin + c), p.issuers, p.tile_m, v);
         for (int cc = c_first; cc >= c_last; --cc) {
             const uint32_t* part =
                 reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(cc) * p.tile_m * kTileN;
@@ -254,174 +301,426 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
 }
 
 // ------------------------------------------------------------------ roles
-template <int MODE>
-__device__ void dequant_role(const GemmArgs& p, uint8_t* smem, Barriers& b, uint32_t tmem, const Ctl& ctl,
+template <int MODE, bool kSmall>
+__device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem, const Ctl& ctl,
                              long long beg, long long end) {
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    uint32_t iter = 0;
-    int seg_index = 0;
+    const int u0 = (64 * half) / p.group_rows, u1 = (64 * half + 32) / p.group_rows;
+    uint32_t fbits = 0, iter = 0;
+    int pos = 0, seg_index = 0;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
-        for (int kb = seg.kb_hi; kb >= seg.kb_lo; --kb, ++iter) {
-            const uint32_t s = iter % p.stages, ph = (iter / p.stages) & 1;
-            const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
-            bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[s], ph, ctl));
-            uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
-            uint16_t sc0 = 0, sc1 = 0;
-            if (ok) {
-                const uint8_t* blob = smem + static_cast<size_t>(s) * p.stage_bytes + p.act_bytes;
-                const uint4* words = reinterpret_cast<const uint4*>(blob);
-                w0 = words[(half * 2 + 0) * kTileN + row];
-                w1 = words[(half * 2 + 1) * kTileN + row];
-                if (MODE == kModeGroup) {
-                    const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
-                    sc0 = sc[((64 * half) / p.group_rows) * kTileN + row];
-                    sc1 = sc[((64 * half + 32) / p.group_rows) * kTileN + row];
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl));
+            fbits ^= 1u << pos;
+            for (int t = 0; t < c; ++t, ++iter) {
+                const int s = pos + t;
+                const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
+                uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
+                uint16_t sc0 = 0, sc1 = 0;
+                if (ok) {
+                    const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
+                    const uint4* words = reinterpret_cast<const uint4*>(blob);
+                    w0 = words[(half * 2 + 0) * kTileN + row];
+                    w1 = words[(half * 2 + 1) * kTileN + row];
+                    if (MODE == kModeGroup && p.scale_in_dequant) {
+                        const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+                        sc0 = sc[u0 * kTileN + row];
+                        sc1 = sc[u1 * kTileN + row];
+                    }
                 }
-            }
-            __syncwarp();
-            if (ok && lane == 0) mbar_arrive(&b.empty[s]);
-            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[a], aph ^ 1, ctl));
-            if (ok) {
-                const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                const uint32_t taddr = tmem + lane_base + kTmemAOffset + a * kSlotCols + half * (kSlotCols / 2);
-                if (MODE == kModeW4A8) {
-                    uint32_t out[16];
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[a], aph ^ 1, ctl));
+                if (ok) {
+                    const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    const uint32_t taddr = tmem + lane_base + kTmemAOffset + a * kSlotCols + half * (kSlotCols / 2);
+                    if (MODE == kModeW4A8) {
+                        uint32_t out[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) dequant_word_i8(wv[i], out + 2 * i);
-                    tmem_st_x16(taddr, out);
-                } else {
-                    uint32_t out[32];
-                    const __half2 s0 = __half2half2(__ushort_as_half(sc0));
-                    const __half2 s1 = __half2half2(__ushort_as_half(sc1));
+                        for (int i = 0; i < 8; ++i) dequant_word_i8(wv[i], out + 2 * i);
+                        tmem_st_x16(taddr, out);
+                    } else {
+                        uint32_t out[32];
+                        const __half2 s0 = __half2half2(__ushort_as_half(sc0));
+                        const __half2 s1 = __half2half2(__ushort_as_half(sc1));
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dequant_word_f16(wv[i], i < 4 ? s0 : s1, MODE == kModeGroup, out + 4 * i);
-                    tmem_st_x32(taddr, out);
+                        if (MODE == kModeGroup && p.scale_in_dequant) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) dequant_word_f16(wv[i], i < 4 ? s0 : s1, true, out + 4 * i);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) dequant_word_f16(wv[i], s0, false, out + 4 * i);
+                        }
+                        tmem_st_x32(taddr, out);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
                 }
-                tmem_st_wait();
-                tc_fence_before();
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&b.afull[a][half]);
             }
-            __syncwarp();
-            if (ok && lane == 0) mbar_arrive(&b.afull[a]);
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
         }
-        epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, half, quarter, lane);
+        if (!kSmall) epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, half, quarter, lane);
         ++seg_index;
     }
 }
 
-template <int MODE>
-__device__ void producer_role(const CUtensorMap* tmap, const GemmArgs& p, uint8_t* smem, Barriers& b,
+// Weight producer (kWeightWarp, one thread) or activation producer (kActWarp, one thread).
+template <int MODE, bool kWeights>
+__device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* aring, uint8_t* wring, Barriers& b,
                               const Ctl& ctl, long long beg, long long end) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
-    uint32_t iter = 0, issued = 0;
+    uint32_t ebits = 0, ubits = 0, armed = 0, lastp = 0;
+    int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
         const uint8_t* wtile = p.wp + static_cast<size_t>(nt) * p.k_blocks * p.blob_bytes;
-        const int y0 = mt * p.tile_m;
-        for (int kb = seg.kb_hi; kb >= seg.kb_lo; --kb, ++iter) {
-            const uint32_t s = iter % p.stages, ph = (iter / p.stages) & 1;
-            if (ok) ok = wait_bar(&b.empty[s], ph ^ 1, ctl);
-            if (!ok) continue;
-            uint8_t* st = smem + static_cast<size_t>(s) * p.stage_bytes;
-            mbar_arrive_expect_tx(&b.full[s], static_cast<uint32_t>(p.act_bytes + p.blob_bytes));
-            if (MODE == kModeW4A8) {
-                tma_load_2d(st, tmap, kb * kTileK, y0, &b.full[s]);
-            } else {
-                tma_load_2d(st, tmap, kb * kTileK, y0, &b.full[s]);
-                tma_load_2d(st + p.tile_m * 128, tmap, kb * kTileK + 64, y0, &b.full[s]);
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            for (int t = 0; t < c; ++t) {
+                const int s = pos + t;
+                if (ok) ok = wait_bar(kWeights ? &b.empty_w[s] : &b.empty_a[s], ((ebits >> s) & 1u) ^ 1u, ctl);
+                ebits ^= 1u << s;
             }
-            bulk_g2s(st + p.act_bytes, wtile + static_cast<size_t>(kb) * p.blob_bytes,
-                     static_cast<uint32_t>(p.blob_bytes), &b.full[s], policy);
-            issued = iter + 1;
+            if (ok) {
+                // the phase this chunk completes on full[pos] has the parity of its use count
+                lastp = (lastp & ~(1u << pos)) | (((ubits >> pos) & 1u) << pos);
+                ubits ^= 1u << pos;
+                armed |= 1u << pos;
+                if (kWeights) {
+                    mbar_arrive_expect_tx(&b.full[pos], static_cast<uint32_t>(c * p.blob_bytes));
+                    bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes,
+                             wtile + static_cast<size_t>(kb) * p.blob_bytes, static_cast<uint32_t>(c * p.blob_bytes),
+                             &b.full[pos], policy);
+                } else {
+                    mbar_arrive_expect_tx(&b.full[pos], static_cast<uint32_t>(c * p.act_slot));
+                    tma_load_3d(aring + static_cast<size_t>(pos) * p.act_slot, &maps->m[c - 1], 0, mt * p.tile_m,
+                                (MODE == kModeW4A8) ? kb : 2 * kb, &b.full[pos]);
+                }
+            }
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
         }
     }
     // wind-down: every copy this CTA started must land before the CTA exits
-    const uint32_t n_stages = static_cast<uint32_t>(p.stages);
-    for (uint32_t s = 0; s < n_stages && s < issued; ++s) {
-        const uint32_t last = issued - 1 - ((issued - 1 - s) % n_stages);
-        wait_bar(&b.full[s], (last / n_stages) & 1, ctl, false);
-    }
+    for (int s = 0; s < p.slots; ++s)
+        if ((armed >> s) & 1u) wait_bar(&b.full[s], (lastp >> s) & 1u, ctl, false);
 }
 
 template <int MODE>
-__device__ void mma_role(const GemmArgs& p, uint8_t* smem, Barriers& b, uint32_t tmem, const Ctl& ctl,
-                         long long beg, long long end) {
+__device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
+                            const Ctl& ctl, long long beg, long long end) {
     constexpr int kSteps = (MODE == kModeW4A8) ? 4 : 8;          // MMA K: 32 int8 or 16 fp16
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
     const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, p.tile_m) : idesc_f16_f32(kTileN, p.tile_m);
-    const uint32_t smem_base = smem_addr(smem);
-    uint32_t iter = 0;
+    const int steps = kSteps / p.issuers;
+    const int k0 = q * steps;                                     // first k-step of this issuer
+    const int hw = (p.issuers == 1) ? -1 : (k0 * (kSteps == 8 ? 16 : 32)) / 64;  // A half it needs (-1: both)
+    const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * p.tile_m);
+    const uint32_t a_base = smem_addr(aring);
+    uint32_t fbits = 0, iter = 0;
+    int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
-        for (int kb = seg.kb_hi; kb >= seg.kb_lo; --kb, ++iter) {
-            const uint32_t s = iter % p.stages, ph = (iter / p.stages) & 1;
-            const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
-            if (ok) ok = wait_bar(&b.full[s], ph, ctl);
-            if (ok) ok = wait_bar(&b.afull[a], aph, ctl);
-            if (!ok) continue;
-            tc_fence_after();
-            const uint32_t act = smem_base + s * static_cast<uint32_t>(p.stage_bytes);
-            const uint32_t a_tmem = tmem + kTmemAOffset + a * kSlotCols;
-#pragma unroll
-            for (int kk = 0; kk < kSteps; ++kk) {
-                const uint32_t boff = (MODE == kModeW4A8)
-                                          ? static_cast<uint32_t>(kk * 32)
-                                          : static_cast<uint32_t>((kk >> 2) * p.tile_m * 128 + (kk & 3) * 32);
-                const uint64_t bdesc = smem_desc_sw128(act + boff);
-                const uint32_t accumulate = (kb != seg.kb_hi || kk != 0) ? 1u : 0u;
-                if (MODE == kModeW4A8)
-                    mma_i8_ts(tmem, a_tmem + kk * 8, bdesc, idesc, accumulate);
-                else
-                    mma_f16_ts(tmem, a_tmem + kk * 8, bdesc, idesc, accumulate);
+        bool first = true;
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            if (ok) ok = wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl);
+            fbits ^= 1u << pos;
+            for (int t = 0; t < c; ++t, ++iter) {
+                const int s = pos + t;
+                const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
+                if (ok) {
+                    if (hw >= 0) {
+                        ok = wait_bar(&b.afull[a][hw], aph, ctl);
+                    } else {
+                        ok = wait_bar(&b.afull[a][0], aph, ctl);
+                        if (ok) ok = wait_bar(&b.afull[a][1], aph, ctl);
+                    }
+                }
+                if (!ok) continue;
+                tc_fence_after();
+                const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+                const uint32_t a_tmem = tmem + kTmemAOffset + a * kSlotCols;
+                for (int kk = k0; kk < k0 + steps; ++kk) {
+                    const uint32_t boff = (MODE == kModeW4A8)
+                                              ? static_cast<uint32_t>(kk * 32)
+                                              : static_cast<uint32_t>((kk >> 2) * p.tile_m * 128 + (kk & 3) * 32);
+                    const uint64_t bdesc = smem_desc_sw128(act + boff);
+                    const uint32_t accumulate = first ? 0u : 1u;
+                    first = false;
+                    if (MODE == kModeW4A8)
+                        mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, accumulate);
+                    else
+                        mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, accumulate);
+                }
+                tc_commit(&b.aempty[a]);
+                tc_commit(&b.empty_a[s]);
             }
-            tc_commit(&b.empty[s]);
-            tc_commit(&b.aempty[a]);
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
         }
         if (ok) tc_commit(&b.dfull);
     }
-    tc_commit(&b.drain);
-    wait_bar(&b.drain, 0, ctl, false);
+    tc_commit(&b.drain[q]);
+    wait_bar(&b.drain[q], 0, ctl, false);
+}
+
+// ------------------------------------------------------------------ small tiles
+// Issuer q of a small tile: every k-block whose walk index is q mod 4 is its own; it waits for
+// the k-block's activations (full), its dequantised weights (both halves of A slot q) and for
+// the accumulate warps to have read its previous partial, then writes the k-block's product
+// into its partial buffer with a fresh accumulation.
+template <int MODE, int TM>
+__device__ void issuer_role_small(int q, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
+                                  const Ctl& ctl, long long beg, long long end) {
+    constexpr int kSteps = (MODE == kModeW4A8) ? 4 : 8;
+    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
+    const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, TM) : idesc_f16_f32(kTileN, TM);
+    const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * TM);
+    const uint32_t a_tmem = tmem + kTmemAOffset + static_cast<uint32_t>(q * kSlotCols);
+    const uint32_t a_base = smem_addr(aring);
+    uint32_t fbits = 0, iter = 0, j = 0;
+    int pos = 0;
+    bool ok = true;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            bool waited = false;
+            for (int t = 0; t < c; ++t, ++iter) {
+                if (static_cast<int>(iter & 3u) != q) continue;
+                const int s = pos + t;
+                const uint32_t jp = j & 1u;
+                ++j;
+                if (ok && !waited) {
+                    ok = wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl);
+                    waited = true;
+                }
+                if (ok) ok = wait_bar(&b.afull[q][0], jp, ctl);
+                if (ok) ok = wait_bar(&b.afull[q][1], jp, ctl);
+                if (ok) ok = wait_bar(&b.pempty[q], jp ^ 1u, ctl);
+                if (!ok) continue;
+                tc_fence_after();
+                const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+#pragma unroll
+                for (int kk = 0; kk < kSteps; ++kk) {
+                    const uint32_t boff = (MODE == kModeW4A8) ? static_cast<uint32_t>(kk * 32)
+                                                              : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
+                    const uint64_t bdesc = smem_desc_sw128(act + boff);
+                    if (MODE == kModeW4A8)
+                        mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                    else
+                        mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                }
+                tc_commit(&b.aempty[q]);
+                tc_commit(&b.empty_a[s]);
+                tc_commit(&b.pfull[q]);
+            }
+            fbits ^= 1u << pos;
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+    }
+    tc_commit(&b.drain[q]);
+    wait_bar(&b.drain[q], 0, ctl, false);
+}
+
+// Epilogue of a small tile from the accumulate warps' registers: thread (quarter, lane) holds
+// the TM sums of output column n = tile*128 + quarter*32 + lane for rows 0..TM-1.
+template <int MODE, int TM>
+__device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&acc)[TM], bool ok,
+                               int quarter, int lane) {
+    const int row = quarter * 32 + lane;
+    const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
+    const int n = nt * kTileN + row;
+    const int m_base = mt * TM;
+    const bool leader = static_cast<int>(threadIdx.x) == kAccWarp0 * 32;
+    if (!seg.owner) {
+        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(blockIdx.x) * TM * kTileN;
+        if (ok) {
+#pragma unroll
+            for (int c = 0; c < TM; ++c) part[static_cast<size_t>(c) * kTileN + row] = acc[c];
+        }
+        __threadfence();
+        named_barrier_sync(2, 128);
+        if (leader && ok && !*ctl.abort_flag && static_cast<int>(blockIdx.x) != p.skip_publish)
+            st_release_gpu(&p.ws_flags[blockIdx.x], 1);
+        return;
+    }
+    const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+    const int c_first = static_cast<int>(blockIdx.x) - 1;
+    int c_last = c_first + 1;
+    if (!seg.whole) {
+        for (int c = c_first; c >= 0; --c) {
+            c_last = c;
+            if (ok) ok = wait_flag(&p.ws_flags[c], ctl);
+            if (unit_start(c, p.units, p.grid) <= tbase) break;
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            for (int cc = c_first; cc >= c_last; --cc) {
+                const uint32_t* part =
+                    reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(cc) * TM * kTileN;
+#pragma unroll
+                for (int c = 0; c < TM; ++c) {
+                    const uint32_t v = __ldcg(part + static_cast<size_t>(c) * kTileN + row);
+                    if (MODE == kModeW4A8)
+                        acc[c] = static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(v));
+                    else
+                        acc[c] = __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(v));
+                }
+            }
+        }
+    }
+    if (ok && n < p.N) {
+        float s_col = 1.0f, sw_col = 0.0f;
+        if (MODE == kModeChannel) s_col = __half2float(__ushort_as_half(p.s_chan[n]));
+        if (MODE == kModeW4A8) sw_col = p.sw[n];
+#pragma unroll
+        for (int c = 0; c < TM; ++c) {
+            const int m = m_base + c;
+            if (m < p.M) {
+                const size_t o = static_cast<size_t>(m) * p.N + n;
+                float y;
+                if (MODE == kModeW4A8) {
+                    const int32_t a = static_cast<int32_t>(acc[c]) >> 4;
+                    if (p.acc_out) p.acc_out[o] = a;
+                    const float t = static_cast<float>(a) * p.sa[m];
+                    y = t * sw_col;
+                } else if (MODE == kModeChannel) {
+                    y = __uint_as_float(acc[c]) * s_col;
+                } else {
+                    y = __uint_as_float(acc[c]);
+                }
+                p.y[o] = __half_as_ushort(__float2half_rn(y));
+            }
+        }
+    }
+    if (!seg.whole) {
+        named_barrier_sync(2, 128);
+        if (leader)
+            for (int cc = c_first; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
+    }
+}
+
+// Accumulate warp (one per tensor-memory lane quarter, quarter = warp % 4) of a small tile: adds every k-block's
+// partial, in k order, into fp32 (or int32) registers, applying the k-block's group scale
+// when the dequant did not, then runs the segment's epilogue.
+template <int MODE, int TM>
+__device__ void accum_role(int quarter, const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
+                           const Ctl& ctl, long long beg, long long end) {
+    const int lane = threadIdx.x & 31;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool scale_here = (MODE == kModeGroup) && !p.scale_in_dequant;
+    uint32_t fbits = 0, iter = 0;
+    int pos = 0;
+    bool ok = true;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        uint32_t acc[TM];
+#pragma unroll
+        for (int c = 0; c < TM; ++c) acc[c] = 0;  // +0.0f and int 0 share the bit pattern
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl));
+            fbits ^= 1u << pos;
+            for (int t = 0; t < c; ++t, ++iter) {
+                const int s = pos + t;
+                const uint32_t q = iter & 3u, ph = (iter >> 2) & 1u;
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
+                uint32_t v[TM];
+                float sc = 1.0f;
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int c0 = 0; c0 < TM; c0 += 16)
+                        tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v + c0);
+                    tmem_ld_wait();
+                    if (scale_here)
+                        sc = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(
+                            wring + static_cast<size_t>(s) * p.blob_bytes + kCodeBytes)[row]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (ok && lane == 0) {
+                    mbar_arrive(&b.pempty[q]);
+                    mbar_arrive(&b.empty_w[s]);
+                }
+                if (ok) {
+#pragma unroll
+                    for (int c2 = 0; c2 < TM; ++c2) {
+                        if (MODE == kModeW4A8)
+                            acc[c2] = static_cast<uint32_t>(static_cast<int32_t>(acc[c2]) + static_cast<int32_t>(v[c2]));
+                        else
+                            acc[c2] = __float_as_uint(fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c2])));
+                    }
+                }
+            }
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+        epilogue_small<MODE, TM>(p, ctl, seg, acc, ok, quarter, lane);
+    }
+}
+
+// ------------------------------------------------------------------ kernels
+__device__ __forceinline__ uint8_t* align_ring(uint8_t* smem_dyn) {
+    const uint32_t raw = smem_addr(smem_dyn);
+    return smem_dyn + ((1024u - (raw & 1023u)) & 1023u);  // swizzle atoms need 1024-byte alignment
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
-    wq_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const GemmArgs p) {
+__global__ void __launch_bounds__(kThreadsLarge, 1)
+    wq_gemm_large(const __grid_constant__ ActMaps maps, const GemmArgs p) {
     extern __shared__ uint8_t smem_dyn[];
     __shared__ Barriers bars;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
-    const uint32_t raw = smem_addr(smem_dyn);
-    uint8_t* smem = smem_dyn + ((1024u - (raw & 1023u)) & 1023u);  // swizzle atoms need 1024-byte alignment
+    uint8_t* aring = align_ring(smem_dyn);
+    uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s) {
-            mbar_init(&bars.full[s], 1);
-            mbar_init(&bars.empty[s], kNumDqWarps + 1);
+        for (int s = 0; s < p.slots; ++s) {
+            mbar_init(&bars.full[s], 2);
+            mbar_init(&bars.empty_w[s], kNumDqWarps);
+            mbar_init(&bars.empty_a[s], p.issuers);
         }
         for (int a = 0; a < kASlots; ++a) {
-            mbar_init(&bars.afull[a], kNumDqWarps);
-            mbar_init(&bars.aempty[a], 1);
+            mbar_init(&bars.afull[a][0], 4);
+            mbar_init(&bars.afull[a][1], 4);
+            mbar_init(&bars.aempty[a], p.issuers);
         }
-        mbar_init(&bars.dfull, 1);
-        mbar_init(&bars.drain, 1);
+        mbar_init(&bars.dfull, p.issuers);
+        for (int q = 0; q < kMaxIssuers; ++q) mbar_init(&bars.drain[q], 1);
         abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kMmaWarp) {
+    if (warp == kIssuerWarp0) {
         tmem_alloc(&tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == kTmaWarp && lane == 0) prefetch_tensor_map(&tmap_a);
+    if (warp == kActWarp && lane == 0)
+        for (int c = 0; c < p.chunk; ++c) prefetch_tensor_map(&maps.m[c]);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -432,16 +731,88 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
 
     if (warp < kNumDqWarps) {
-        dequant_role<MODE>(p, smem, bars, tmem, ctl, beg, end);
-    } else if (warp == kTmaWarp) {
-        if (lane == 0) producer_role<MODE>(&tmap_a, p, smem, bars, ctl, beg, end);
+        dequant_role<MODE, false>(p, wring, bars, tmem, ctl, beg, end);
+    } else if (warp < kIssuerWarp0 + kMaxIssuers) {
+        const int q = warp - kIssuerWarp0;
+        if (q < p.issuers && lane == 0) issuer_role<MODE>(q, p, aring, bars, tmem, ctl, beg, end);
+    } else if (warp == kWeightWarp) {
+        if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
-        if (lane == 0) mma_role<MODE>(p, smem, bars, tmem, ctl, beg, end);
+        if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kIssuerWarp0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int MODE, int TM>
+__global__ void __launch_bounds__(kThreadsSmall, 1)
+    wq_gemm_small(const __grid_constant__ ActMaps maps, const GemmArgs p) {
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ Barriers bars;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+
+    uint8_t* aring = align_ring(smem_dyn);
+    uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.slots; ++s) {
+            mbar_init(&bars.full[s], 2);
+            mbar_init(&bars.empty_w[s], kNumDqWarps + 4);  // dequant warps + accumulate warps (scales)
+            mbar_init(&bars.empty_a[s], 1);                // the owning issuer
+        }
+        for (int a = 0; a < kASlots; ++a) {
+            mbar_init(&bars.afull[a][0], 4);
+            mbar_init(&bars.afull[a][1], 4);
+            mbar_init(&bars.aempty[a], 1);
+        }
+        for (int q = 0; q < kMaxIssuers; ++q) {
+            mbar_init(&bars.drain[q], 1);
+            mbar_init(&bars.pfull[q], 1);
+            mbar_init(&bars.pempty[q], 4);
+        }
+        mbar_init(&bars.dfull, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kIssuerWarp0) {
+        tmem_alloc(&tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == kActWarp && lane == 0)
+        for (int c = 0; c < p.chunk; ++c) prefetch_tensor_map(&maps.m[c]);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
+    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
+    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+
+    if (warp < kNumDqWarps) {
+        dequant_role<MODE, true>(p, wring, bars, tmem, ctl, beg, end);
+    } else if (warp < kIssuerWarp0 + kMaxIssuers) {
+        if (lane == 0) issuer_role_small<MODE, TM>(warp - kIssuerWarp0, p, aring, bars, tmem, ctl, beg, end);
+    } else if (warp == kWeightWarp) {
+        if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
+    } else if (warp == kActWarp) {
+        if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
+    } else {
+        // a warp may only touch tensor-memory lanes 32*(warp % 4) .. +31
+        accum_role<MODE, TM>(warp & 3, p, wring, bars, tmem, ctl, beg, end);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kIssuerWarp0) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -461,37 +832,50 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->tile_m = tm;
     pl->m_tiles = (M + tm - 1) / tm;
     if (pl->m_tiles < 1) pl->m_tiles = 1;
-    pl->act_bytes = (mode == kModeW4A8) ? tm * 128 : tm * 256;
+    pl->small = tm <= kSmallTileMax;
+    pl->threads = pl->small ? kThreadsSmall : kThreadsLarge;
+    pl->issuers = pl->small ? kMaxIssuers : (tm <= 64 ? 4 : (tm <= 128 ? 2 : 1));
+    pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;
     pl->blob_bytes = (mode == kModeGroup) ? static_cast<int>(blob_bytes_w4a16(slots)) : kCodeBytes;
-    pl->stage_bytes = (pl->act_bytes + pl->blob_bytes + 1023) / 1024 * 1024;
     const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */;
-    int stages = budget / pl->stage_bytes;
-    if (stages > kMaxStages) stages = kMaxStages;
-    if (stages < 2) return -1;
-    pl->stages = stages;
-    pl->smem_bytes = stages * pl->stage_bytes + 1024;
+    int s = budget / (pl->act_slot + pl->blob_bytes);
+    if (s > kMaxSlots) s = kMaxSlots;
+    if (s < 2) return -1;
+    pl->slots = s;
+    int c = s / 2;
+    if (c > kMaxChunk) c = kMaxChunk;
+    if (c < 1) c = 1;
+    pl->chunk = c;
+    pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024;
     pl->units = static_cast<long long>(pl->n_tiles) * pl->m_tiles * pl->k_blocks;
     pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
     return 0;
 }
 
+template <typename Kernel>
+static cudaError_t allow_smem(Kernel k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
-    cudaError_t e = cudaFuncSetAttribute(wq_gemm_kernel<kModeGroup>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         max_dynamic_smem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(wq_gemm_kernel<kModeChannel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_dynamic_smem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(wq_gemm_kernel<kModeW4A8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_dynamic_smem);
+    cudaError_t e = allow_smem(wq_gemm_large<kModeGroup>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeChannel>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeW4A8>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroup, 16>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroup, 32>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeChannel, 16>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeChannel, 32>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 16>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 32>, max_dynamic_smem);
     return e;
 }
 
-template <int MODE>
-static cudaError_t launch_mode(const CUtensorMap& tmap, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
+template <typename Kernel>
+static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& args, const Plan& plan,
+                                 cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(static_cast<unsigned>(plan.threads));
     cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem_bytes);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -499,15 +883,21 @@ static cudaError_t launch_mode(const CUtensorMap& tmap, const GemmArgs& args, co
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, wq_gemm_kernel<MODE>, tmap, args);
+    return cudaLaunchKernelEx(&cfg, k, maps, args);
 }
 
-cudaError_t launch_gemm(int mode, const CUtensorMap& tmap, const GemmArgs& args, const Plan& plan,
-                        cudaStream_t stream) {
+template <int MODE>
+static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
+    if (!plan.small) return launch_kernel(wq_gemm_large<MODE>, maps, args, plan, st);
+    if (plan.tile_m == 16) return launch_kernel(wq_gemm_small<MODE, 16>, maps, args, plan, st);
+    return launch_kernel(wq_gemm_small<MODE, 32>, maps, args, plan, st);
+}
+
+cudaError_t launch_gemm(int mode, const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t stream) {
     switch (mode) {
-        case kModeGroup: return launch_mode<kModeGroup>(tmap, args, plan, stream);
-        case kModeChannel: return launch_mode<kModeChannel>(tmap, args, plan, stream);
-        default: return launch_mode<kModeW4A8>(tmap, args, plan, stream);
+        case kModeGroup: return launch_mode<kModeGroup>(maps, args, plan, stream);
+        case kModeChannel: return launch_mode<kModeChannel>(maps, args, plan, stream);
+        default: return launch_mode<kModeW4A8>(maps, args, plan, stream);
     }
 }
 

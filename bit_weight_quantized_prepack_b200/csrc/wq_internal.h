@@ -22,29 +22,38 @@ struct GemmArgs {
     int M, N;
     int m_tiles, n_tiles, k_blocks;
     int tile_m;                // MMA N extent (multiple of 16, <= 256)
-    int stages;
-    int stage_bytes;           // bytes of one pipeline stage (activation tile + blob), 1024-aligned
-    int act_bytes;             // bytes of the activation tile of one stage
-    int blob_bytes;            // bytes of one weight blob
+    int issuers;               // MMA-issuing warps (1, 2 or 4); issuers * tile_m <= 256
+    int slots;                 // shared-memory ring slots
+    int chunk;                 // most k-blocks per copy
+    int act_slot;              // bytes of one activation slot (one k-block of tile_m rows)
+    int blob_bytes;            // bytes of one weight blob = one weight slot
     int group_rows;            // W4A16 grouped: rows per scale slot, min(g, 128)
+    int small;                 // 1: per-k-block partials summed by the accumulate warps (tile_m <= 32)
+    int scale_in_dequant;      // 1: the dequant multiplies by the group scale (fp16 weights)
     long long units;           // tiles * k_blocks
     int grid;
     unsigned long long timeout_ns;
     int skip_publish;          // test hook: CTA that skips publishing its partial (-1: none)
 };
 
+// Activation tensor maps, one per chunk length 1..kMaxChunk (the box spans that many k-blocks).
+struct ActMaps {
+    CUtensorMap m[kMaxChunk];
+};
+
 struct Plan {
     int mode;
     int tile_m, m_tiles, n_tiles, k_blocks;
     long long units;
-    int grid, stages, stage_bytes, act_bytes, blob_bytes, smem_bytes;
+    int grid, issuers, slots, chunk, act_slot, blob_bytes, smem_bytes, threads;
+    bool small;
 };
 
 int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan);
 
 cudaError_t configure_gemm_kernels(int max_dynamic_smem);
 
-cudaError_t launch_gemm(int mode, const CUtensorMap& tmap, const GemmArgs& args, const Plan& plan,
+cudaError_t launch_gemm(int mode, const ActMaps& maps, const GemmArgs& args, const Plan& plan,
                         cudaStream_t stream);
 
 int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, cudaStream_t st);

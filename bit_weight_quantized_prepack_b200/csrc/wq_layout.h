@@ -30,15 +30,21 @@ namespace wq {
 constexpr int kTileN = 128;                   // weight columns per tile = tcgen05 M extent
 constexpr int kTileK = 128;                   // weight rows per k-block = one pipeline stage
 constexpr int kCodeBytes = kTileN * kTileK / 2;  // 8192 bytes of 4-bit codes per blob
-constexpr int kNumDqWarps = 8;                // dequant + epilogue warps (2 per TMEM lane quarter)
-constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = (kNumDqWarps + 2) * 32;
+constexpr int kNumDqWarps = 8;                // dequant warps (2 per TMEM lane quarter)
+constexpr int kMaxIssuers = 4;                // MMA-issuing warps, one accumulator each
+constexpr int kIssuerWarp0 = kNumDqWarps;     // warps 8..11
+constexpr int kWeightWarp = kIssuerWarp0 + kMaxIssuers;  // warp 12: weight-blob copies
+constexpr int kActWarp = kWeightWarp + 1;     // warp 13: activation-tile copies
+constexpr int kAccWarp0 = kActWarp + 1;       // warps 14..17: accumulate + epilogue (small tiles)
+constexpr int kThreadsLarge = (kActWarp + 1) * 32;   // 448: epilogue runs in the dequant warps
+constexpr int kThreadsSmall = (kAccWarp0 + 4) * 32;  // 576
+constexpr int kSmallTileMax = 32;             // tiles of at most this many rows use per-k-block partials
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
-constexpr int kMaxStages = 24;
+constexpr int kMaxSlots = 32;                 // shared-memory ring slots (one k-block each)
+constexpr int kMaxChunk = 4;                  // k-blocks moved by one copy
 constexpr int kASlots = 4;                    // dequantised weight tiles in tensor memory
 constexpr int kTmemCols = 512;
-constexpr int kTmemAOffset = 256;             // accumulator in columns [0, 256), A slots above
+constexpr int kTmemAOffset = 256;             // accumulators in columns [0, 256), A slots above
 
 enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2 };
 

@@ -59,6 +59,25 @@ def test_identity_activation_reproduces_weights_bitwise(K, g):
         f"{int((Y.astype(np.float32) != exp.astype(np.float32)).sum())} weights differ"
 
 
+@pytest.mark.parametrize("K,g,M", [(1024, 128, 16), (1024, 1024, 16), (2048, 256, 32), (512, 64, 16), (1024, 32, 9)])
+def test_unit_rows_reproduce_weights_bitwise(K, g, M):
+    # small batches (one tile of <= 32 rows): row i of A is the unit vector e_{k_i}, so
+    # Y[i, n] = fp16_rn((q[k_i, n] - 8) * s[k_i // g, n]) bit for bit, whichever of the two
+    # scale placements the kernel uses (a single exact product, one rounding)
+    wq = _wq()
+    N = 264
+    d = synth.w4a16_inputs(K, N, g, 1, seed=K + g + M)
+    ks = np.random.default_rng(M).choice(K, size=M, replace=False)
+    A = np.zeros((M, K), np.float16)
+    A[np.arange(M), ks] = 1
+    Wp = wq.wq_prepack(to_dev(d["Q"]), to_dev(d["s"]), g)
+    Y = wq.wq_gemm_w4a16(to_dev(A), Wp, N, g).cpu().numpy()
+    exact = (d["q"][ks].astype(np.float64) - 8) * d["s"][ks // g].astype(np.float64)
+    exp = exact.astype(np.float16)  # one round-to-nearest-even of the exact product
+    assert np.array_equal(Y.astype(np.float32), exp.astype(np.float32)), \
+        f"{int((Y.astype(np.float32) != exp.astype(np.float32)).sum())} weights differ"
+
+
 @pytest.mark.parametrize("g", [128, 1024])
 def test_all_eight_codes_give_zero(g):
     wq = _wq()
