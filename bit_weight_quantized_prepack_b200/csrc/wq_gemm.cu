@@ -52,11 +52,12 @@
 namespace wq {
 
 struct Barriers {
-    uint64_t full[kMaxSlots];      // chunk landed: both producers' bytes (count 2 + transactions)
+    uint64_t full[kChunkBars];     // chunk landed: both producers' bytes (count 2 + transactions),
+                                   // indexed by chunk sequence number mod kChunkBars
     uint64_t empty_w[kMaxSlots];   // weight slot read by the 8 dequant warps
     uint64_t empty_a[kMaxSlots];   // activation slot read by the MMAs of every issuer (commits)
-    uint64_t afull[kASlots][2];    // dequantised half-k-block in tensor memory (4 warps each)
-    uint64_t aempty[kASlots];      // every issuer's MMAs done with a tensor-memory slot
+    uint64_t afull[kASlotsS][2];   // dequantised k-block (half) in tensor memory (4 warps each)
+    uint64_t aempty[kASlotsS];     // MMAs done with a tensor-memory slot
     uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
     uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
     uint64_t pfull[kMaxIssuers];   // small tiles: an issuer's per-k-block partial is ready (commit)
@@ -144,6 +145,14 @@ __device__ __forceinline__ int chunk_len(int chunk, int kb, int kb_hi, int pos, 
     if (c > slots - pos) c = slots - pos;
     return c;
 }
+
+// The full barrier of chunk number ch (counted along the CTA's walk) is full[ch % kChunkBars]
+// and the chunk completes that barrier's phase ch / kChunkBars. With more barriers than ring
+// slots, a barrier is re-armed only after the ring has moved past every slot of the chunk that
+// last used it, so a role that still holds one of that chunk's k-blocks can never see the
+// barrier two phases ahead (a slot-indexed barrier could, when chunk boundaries shift).
+__device__ __forceinline__ uint32_t chunk_bar(uint32_t ch) { return ch % kChunkBars; }
+__device__ __forceinline__ uint32_t chunk_parity(uint32_t ch) { return (ch / kChunkBars) & 1u; }
 
 // ------------------------------------------------------------------ dequantisation
 // fp16 constants from the binary16 format: 0x6400 = 1024 (exponent field 25, so the 10
@@ -301,7 +310,7 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
 }
 
 // ------------------------------------------------------------------ roles
-template <int MODE, bool kSmall>
+template <int MODE>
 __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem, const Ctl& ctl,
                              long long beg, long long end) {
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
@@ -310,14 +319,14 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int u0 = (64 * half) / p.group_rows, u1 = (64 * half + 32) / p.group_rows;
-    uint32_t fbits = 0, iter = 0;
+    uint32_t ch = 0, iter = 0;
     int pos = 0, seg_index = 0;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl));
-            fbits ^= 1u << pos;
+            bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[chunk_bar(ch)], chunk_parity(ch), ctl));
+            ++ch;
             for (int t = 0; t < c; ++t, ++iter) {
                 const int s = pos + t;
                 const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
@@ -349,7 +358,6 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
                         uint32_t out[32];
                         const __half2 s0 = __half2half2(__ushort_as_half(sc0));
                         const __half2 s1 = __half2half2(__ushort_as_half(sc1));
-#pragma unroll
                         if (MODE == kModeGroup && p.scale_in_dequant) {
 #pragma unroll
                             for (int i = 0; i < 8; ++i) dequant_word_f16(wv[i], i < 4 ? s0 : s1, true, out + 4 * i);
@@ -369,7 +377,7 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
             pos += c;
             if (pos == p.slots) pos = 0;
         }
-        if (!kSmall) epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, half, quarter, lane);
+        epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, half, quarter, lane);
         ++seg_index;
     }
 }
@@ -379,7 +387,7 @@ template <int MODE, bool kWeights>
 __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* aring, uint8_t* wring, Barriers& b,
                               const Ctl& ctl, long long beg, long long end) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
-    uint32_t ebits = 0, ubits = 0, armed = 0, lastp = 0;
+    uint32_t ebits = 0, ch = 0, armed = 0;
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
@@ -394,29 +402,28 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                 ebits ^= 1u << s;
             }
             if (ok) {
-                // the phase this chunk completes on full[pos] has the parity of its use count
-                lastp = (lastp & ~(1u << pos)) | (((ubits >> pos) & 1u) << pos);
-                ubits ^= 1u << pos;
-                armed |= 1u << pos;
                 if (kWeights) {
-                    mbar_arrive_expect_tx(&b.full[pos], static_cast<uint32_t>(c * p.blob_bytes));
+                    mbar_arrive_expect_tx(&b.full[chunk_bar(ch)], static_cast<uint32_t>(c * p.blob_bytes));
                     bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes,
                              wtile + static_cast<size_t>(kb) * p.blob_bytes, static_cast<uint32_t>(c * p.blob_bytes),
-                             &b.full[pos], policy);
+                             &b.full[chunk_bar(ch)], policy);
                 } else {
-                    mbar_arrive_expect_tx(&b.full[pos], static_cast<uint32_t>(c * p.act_slot));
+                    mbar_arrive_expect_tx(&b.full[chunk_bar(ch)], static_cast<uint32_t>(c * p.act_slot));
                     tma_load_3d(aring + static_cast<size_t>(pos) * p.act_slot, &maps->m[c - 1], 0, mt * p.tile_m,
-                                (MODE == kModeW4A8) ? kb : 2 * kb, &b.full[pos]);
+                                (MODE == kModeW4A8) ? kb : 2 * kb, &b.full[chunk_bar(ch)]);
                 }
+                armed = ch + 1;
             }
+            ++ch;
             kb += c;
             pos += c;
             if (pos == p.slots) pos = 0;
         }
     }
-    // wind-down: every copy this CTA started must land before the CTA exits
-    for (int s = 0; s < p.slots; ++s)
-        if ((armed >> s) & 1u) wait_bar(&b.full[s], (lastp >> s) & 1u, ctl, false);
+    // wind-down: every copy this CTA started must land before the CTA exits (after an expired
+    // wait, one more bounded wait is the most this spends)
+    for (uint32_t k = armed > kChunkBars ? armed - kChunkBars : 0; k < armed; ++k)
+        if (!wait_bar(&b.full[chunk_bar(k)], chunk_parity(k), ctl, false)) break;
 }
 
 template <int MODE>
@@ -430,7 +437,7 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
     const int hw = (p.issuers == 1) ? -1 : (k0 * (kSteps == 8 ? 16 : 32)) / 64;  // A half it needs (-1: both)
     const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * p.tile_m);
     const uint32_t a_base = smem_addr(aring);
-    uint32_t fbits = 0, iter = 0;
+    uint32_t ch = 0, iter = 0;
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
@@ -438,8 +445,8 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
         bool first = true;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            if (ok) ok = wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl);
-            fbits ^= 1u << pos;
+            if (ok) ok = wait_bar(&b.full[chunk_bar(ch)], chunk_parity(ch), ctl);
+            ++ch;
             for (int t = 0; t < c; ++t, ++iter) {
                 const int s = pos + t;
                 const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
@@ -481,10 +488,96 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
 }
 
 // ------------------------------------------------------------------ small tiles
+// Roles of the small-tile design split the walk's k-blocks round-robin: a role with period R
+// and residue r handles the k-blocks whose walk index is r mod R. All roles still follow every
+// chunk (to keep the full barriers' phases) but wait only for chunks holding one of theirs.
+__device__ __forceinline__ bool chunk_has(uint32_t iter0, int c, uint32_t period, uint32_t residue) {
+    return ((residue + period - iter0 % period) % period) < static_cast<uint32_t>(c);
+}
+
+// Dequant warp of a small tile: lane quarter = warp % 4, residue = warp / 4 (period 3). It turns
+// all 16 packed words of its row of a k-block into 128 fp16 (or int8) values and stores them
+// into tensor-memory slot (walk index mod 6), where they are the MMA's A operand.
+template <int MODE>
+__device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
+                                   const Ctl& ctl, long long beg, long long end) {
+    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;
+    const uint32_t residue = static_cast<uint32_t>(warp >> 2);
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool scaled = (MODE == kModeGroup) && p.scale_in_dequant;
+    uint32_t ch = 0, iter = 0;
+    int pos = 0;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
+            ++ch;
+            if (chunk_has(iter, c, 3, residue)) {
+                bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
+                for (int t = 0; t < c; ++t) {
+                    const uint32_t i = iter + t;
+                    if (i % 3 != residue) continue;
+                    const int s = pos + t;
+                    const uint32_t a = i % kASlotsS, aph = (i / kASlotsS) & 1;
+                    uint4 w[4];
+                    uint16_t sc[4] = {0, 0, 0, 0};
+                    if (ok) {
+                        const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
+                        const uint4* words = reinterpret_cast<const uint4*>(blob);
+#pragma unroll
+                        for (int hv = 0; hv < 4; ++hv) w[hv] = words[hv * kTileN + row];
+                        if (scaled) {
+                            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+#pragma unroll
+                            for (int hv = 0; hv < 4; ++hv) sc[hv] = scs[((32 * hv) / p.group_rows) * kTileN + row];
+                        }
+                    }
+                    __syncwarp();
+                    if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);
+                    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[a], aph ^ 1, ctl));
+                    if (ok) {
+                        const uint32_t taddr = tmem + lane_base + kTmemAOffsetS + a * kSlotCols;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t wv[8] = {w[2 * h].x,     w[2 * h].y,     w[2 * h].z,     w[2 * h].w,
+                                                    w[2 * h + 1].x, w[2 * h + 1].y, w[2 * h + 1].z, w[2 * h + 1].w};
+                            if (MODE == kModeW4A8) {
+                                uint32_t out[16];
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) dequant_word_i8(wv[k], out + 2 * k);
+                                tmem_st_x16(taddr + h * 16, out);
+                            } else {
+                                uint32_t out[32];
+                                const __half2 s0 = __half2half2(__ushort_as_half(sc[2 * h]));
+                                const __half2 s1 = __half2half2(__ushort_as_half(sc[2 * h + 1]));
+#pragma unroll
+                                for (int k = 0; k < 8; ++k) dequant_word_f16(wv[k], k < 4 ? s0 : s1, scaled, out + 4 * k);
+                                tmem_st_x32(taddr + h * 32, out);
+                            }
+                        }
+                        tmem_st_wait();
+                        tc_fence_before();
+                    }
+                    __syncwarp();
+                    if (ok && lane == 0) mbar_arrive(&b.afull[a][0]);
+                }
+            }
+            iter += c;
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+    }
+}
+
 // Issuer q of a small tile: every k-block whose walk index is q mod 4 is its own; it waits for
-// the k-block's activations (full), its dequantised weights (both halves of A slot q) and for
-// the accumulate warps to have read its previous partial, then writes the k-block's product
-// into its partial buffer with a fresh accumulation.
+// the k-block's activations (full), its dequantised weights (A slot) and for the accumulate
+// warps to have read its previous partial, then writes the k-block's product into its partial
+// buffer with a fresh accumulation.
 template <int MODE, int TM>
 __device__ void issuer_role_small(int q, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
                                   const Ctl& ctl, long long beg, long long end) {
@@ -492,46 +585,48 @@ __device__ void issuer_role_small(int q, const GemmArgs& p, const uint8_t* aring
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
     const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, TM) : idesc_f16_f32(kTileN, TM);
     const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * TM);
-    const uint32_t a_tmem = tmem + kTmemAOffset + static_cast<uint32_t>(q * kSlotCols);
     const uint32_t a_base = smem_addr(aring);
-    uint32_t fbits = 0, iter = 0, j = 0;
+    uint32_t ch = 0, iter = 0, j = 0;
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            bool waited = false;
-            for (int t = 0; t < c; ++t, ++iter) {
-                if (static_cast<int>(iter & 3u) != q) continue;
-                const int s = pos + t;
-                const uint32_t jp = j & 1u;
-                ++j;
-                if (ok && !waited) {
-                    ok = wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl);
-                    waited = true;
-                }
-                if (ok) ok = wait_bar(&b.afull[q][0], jp, ctl);
-                if (ok) ok = wait_bar(&b.afull[q][1], jp, ctl);
-                if (ok) ok = wait_bar(&b.pempty[q], jp ^ 1u, ctl);
-                if (!ok) continue;
-                tc_fence_after();
-                const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
+            ++ch;
+            if (chunk_has(iter, c, 4, static_cast<uint32_t>(q))) {
+                if (ok) ok = wait_bar(&b.full[fb], fpar, ctl);
+                for (int t = 0; t < c; ++t) {
+                    const uint32_t i = iter + t;
+                    if (static_cast<int>(i & 3u) != q) continue;
+                    const int s = pos + t;
+                    const uint32_t a = i % kASlotsS, aph = (i / kASlotsS) & 1;
+                    const uint32_t jp = j & 1u;
+                    ++j;
+                    if (ok) ok = wait_bar(&b.afull[a][0], aph, ctl);
+                    if (ok) ok = wait_bar(&b.pempty[q], jp ^ 1u, ctl);
+                    if (!ok) continue;
+                    tc_fence_after();
+                    const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+                    const uint32_t a_tmem = tmem + kTmemAOffsetS + a * kSlotCols;
 #pragma unroll
-                for (int kk = 0; kk < kSteps; ++kk) {
-                    const uint32_t boff = (MODE == kModeW4A8) ? static_cast<uint32_t>(kk * 32)
-                                                              : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
-                    const uint64_t bdesc = smem_desc_sw128(act + boff);
-                    if (MODE == kModeW4A8)
-                        mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
-                    else
-                        mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                    for (int kk = 0; kk < kSteps; ++kk) {
+                        const uint32_t boff = (MODE == kModeW4A8)
+                                                  ? static_cast<uint32_t>(kk * 32)
+                                                  : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
+                        const uint64_t bdesc = smem_desc_sw128(act + boff);
+                        if (MODE == kModeW4A8)
+                            mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                        else
+                            mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                    }
+                    tc_commit(&b.aempty[a]);
+                    tc_commit(&b.empty_a[s]);
+                    tc_commit(&b.pfull[q]);
                 }
-                tc_commit(&b.aempty[q]);
-                tc_commit(&b.empty_a[s]);
-                tc_commit(&b.pfull[q]);
             }
-            fbits ^= 1u << pos;
+            iter += c;
             kb += c;
             pos += c;
             if (pos == p.slots) pos = 0;
@@ -550,7 +645,7 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
     const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
     const int n = nt * kTileN + row;
     const int m_base = mt * TM;
-    const bool leader = static_cast<int>(threadIdx.x) == kAccWarp0 * 32;
+    const bool leader = static_cast<int>(threadIdx.x) == kAccWarp0S * 32;
     if (!seg.owner) {
         uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(blockIdx.x) * TM * kTileN;
         if (ok) {
@@ -619,18 +714,23 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
     }
 }
 
-// Accumulate warp (one per tensor-memory lane quarter, quarter = warp % 4) of a small tile: adds every k-block's
-// partial, in k order, into fp32 (or int32) registers, applying the k-block's group scale
-// when the dequant did not, then runs the segment's epilogue.
+// Accumulate warp of a small tile: lane quarter = warp % 4, parity = which k-blocks (walk index
+// mod 2) it adds. Each k-block's partial is added in k order into fp32 (or int32) registers,
+// with the k-block's group scale applied when the dequant did not. At the end of a segment the
+// odd-parity warp hands its sums to the even-parity warp of its quarter through shared memory
+// (double-buffered by segment), which adds them (even + odd, a fixed order) and runs the
+// epilogue.
 template <int MODE, int TM>
-__device__ void accum_role(int quarter, const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
-                           const Ctl& ctl, long long beg, long long end) {
-    const int lane = threadIdx.x & 31;
+__device__ void accum_role_small(const GemmArgs& p, const uint8_t* wring, uint32_t* cbuf, Barriers& b, uint32_t tmem,
+                                 const Ctl& ctl, long long beg, long long end) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;  // a warp may only touch tensor-memory lanes 32*(warp % 4) .. +31
+    const uint32_t parity = static_cast<uint32_t>((warp - kAccWarp0S) >> 2);
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool scale_here = (MODE == kModeGroup) && !p.scale_in_dequant;
-    uint32_t fbits = 0, iter = 0;
-    int pos = 0;
+    uint32_t ch = 0, iter = 0;
+    int pos = 0, seg_index = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
@@ -639,45 +739,71 @@ __device__ void accum_role(int quarter, const GemmArgs& p, const uint8_t* wring,
         for (int c = 0; c < TM; ++c) acc[c] = 0;  // +0.0f and int 0 share the bit pattern
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[pos], (fbits >> pos) & 1u, ctl));
-            fbits ^= 1u << pos;
-            for (int t = 0; t < c; ++t, ++iter) {
-                const int s = pos + t;
-                const uint32_t q = iter & 3u, ph = (iter >> 2) & 1u;
-                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
-                uint32_t v[TM];
-                float sc = 1.0f;
-                if (ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int c0 = 0; c0 < TM; c0 += 16)
-                        tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v + c0);
-                    tmem_ld_wait();
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
+            ++ch;
+            if (chunk_has(iter, c, 2, parity)) {
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
+                for (int t = 0; t < c; ++t) {
+                    const uint32_t i = iter + t;
+                    if ((i & 1u) != parity) continue;
+                    const int s = pos + t;
+                    const uint32_t q = i & 3u, ph = (i >> 2) & 1u;
+                    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
+                    if (!ok) continue;
+                    float sc = 1.0f;
                     if (scale_here)
                         sc = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(
                             wring + static_cast<size_t>(s) * p.blob_bytes + kCodeBytes)[row]));
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (ok && lane == 0) {
-                    mbar_arrive(&b.pempty[q]);
-                    mbar_arrive(&b.empty_w[s]);
-                }
-                if (ok) {
+                    tc_fence_after();
 #pragma unroll
-                    for (int c2 = 0; c2 < TM; ++c2) {
-                        if (MODE == kModeW4A8)
-                            acc[c2] = static_cast<uint32_t>(static_cast<int32_t>(acc[c2]) + static_cast<int32_t>(v[c2]));
-                        else
-                            acc[c2] = __float_as_uint(fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c2])));
+                    for (int c0 = 0; c0 < TM; c0 += 16) {  // 16 columns at a time keeps registers low
+                        uint32_t v[16];
+                        tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v);
+                        tmem_ld_wait();
+                        if (c0 + 16 >= TM) {  // every column read: hand the partial buffer back
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                mbar_arrive(&b.pempty[q]);
+                                mbar_arrive(&b.empty_w[s]);
+                            }
+                        }
+#pragma unroll
+                        for (int c2 = 0; c2 < 16; ++c2) {
+                            if (MODE == kModeW4A8)
+                                acc[c0 + c2] = static_cast<uint32_t>(static_cast<int32_t>(acc[c0 + c2]) +
+                                                                     static_cast<int32_t>(v[c2]));
+                            else
+                                acc[c0 + c2] = __float_as_uint(
+                                    fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c0 + c2])));
+                        }
                     }
                 }
             }
+            iter += c;
             kb += c;
             pos += c;
             if (pos == p.slots) pos = 0;
         }
-        epilogue_small<MODE, TM>(p, ctl, seg, acc, ok, quarter, lane);
+        // combine the two parities of this quarter, then the even warp runs the epilogue
+        uint32_t* buf = cbuf + (static_cast<size_t>(seg_index & 1) * 4 + quarter) * (32 * TM);
+        if (parity == 1) {
+#pragma unroll
+            for (int c = 0; c < TM; ++c) buf[c * 32 + lane] = acc[c];
+            named_barrier_sync(3 + quarter, 64);
+        } else {
+            named_barrier_sync(3 + quarter, 64);
+#pragma unroll
+            for (int c = 0; c < TM; ++c) {
+                const uint32_t o = buf[c * 32 + lane];
+                if (MODE == kModeW4A8)
+                    acc[c] = static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(o));
+                else
+                    acc[c] = __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(o));
+            }
+            epilogue_small<MODE, TM>(p, ctl, seg, acc, ok && !*ctl.abort_flag, quarter, lane);
+        }
+        ++seg_index;
     }
 }
 
@@ -700,8 +826,8 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        for (int k = 0; k < kChunkBars; ++k) mbar_init(&bars.full[k], 2);
         for (int s = 0; s < p.slots; ++s) {
-            mbar_init(&bars.full[s], 2);
             mbar_init(&bars.empty_w[s], kNumDqWarps);
             mbar_init(&bars.empty_a[s], p.issuers);
         }
@@ -731,7 +857,7 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
 
     if (warp < kNumDqWarps) {
-        dequant_role<MODE, false>(p, wring, bars, tmem, ctl, beg, end);
+        dequant_role<MODE>(p, wring, bars, tmem, ctl, beg, end);
     } else if (warp < kIssuerWarp0 + kMaxIssuers) {
         const int q = warp - kIssuerWarp0;
         if (q < p.issuers && lane == 0) issuer_role<MODE>(q, p, aring, bars, tmem, ctl, beg, end);
@@ -760,17 +886,17 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
 
     uint8_t* aring = align_ring(smem_dyn);
     uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
+    uint32_t* cbuf = reinterpret_cast<uint32_t*>(wring + static_cast<size_t>(p.slots) * p.blob_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        for (int k = 0; k < kChunkBars; ++k) mbar_init(&bars.full[k], 2);
         for (int s = 0; s < p.slots; ++s) {
-            mbar_init(&bars.full[s], 2);
-            mbar_init(&bars.empty_w[s], kNumDqWarps + 4);  // dequant warps + accumulate warps (scales)
-            mbar_init(&bars.empty_a[s], 1);                // the owning issuer
+            mbar_init(&bars.empty_w[s], 8);  // the k-block's 4 dequant warps + 4 accumulate warps
+            mbar_init(&bars.empty_a[s], 1);  // the owning issuer
         }
-        for (int a = 0; a < kASlots; ++a) {
+        for (int a = 0; a < kASlotsS; ++a) {
             mbar_init(&bars.afull[a][0], 4);
-            mbar_init(&bars.afull[a][1], 4);
             mbar_init(&bars.aempty[a], 1);
         }
         for (int q = 0; q < kMaxIssuers; ++q) {
@@ -778,15 +904,14 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
             mbar_init(&bars.pfull[q], 1);
             mbar_init(&bars.pempty[q], 4);
         }
-        mbar_init(&bars.dfull, 1);
         abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kIssuerWarp0) {
+    if (warp == kIssuerWarp0S) {
         tmem_alloc(&tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == kActWarp && lane == 0)
+    if (warp == kActWarpS && lane == 0)
         for (int c = 0; c < p.chunk; ++c) prefetch_tensor_map(&maps.m[c]);
     tc_fence_before();
     __syncthreads();
@@ -797,22 +922,21 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
 
-    if (warp < kNumDqWarps) {
-        dequant_role<MODE, true>(p, wring, bars, tmem, ctl, beg, end);
-    } else if (warp < kIssuerWarp0 + kMaxIssuers) {
-        if (lane == 0) issuer_role_small<MODE, TM>(warp - kIssuerWarp0, p, aring, bars, tmem, ctl, beg, end);
-    } else if (warp == kWeightWarp) {
+    if (warp < kDqWarpsS) {
+        dequant_role_small<MODE>(p, wring, bars, tmem, ctl, beg, end);
+    } else if (warp < kIssuerWarp0S + kMaxIssuers) {
+        if (lane == 0) issuer_role_small<MODE, TM>(warp - kIssuerWarp0S, p, aring, bars, tmem, ctl, beg, end);
+    } else if (warp == kWeightWarpS) {
         if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
-    } else if (warp == kActWarp) {
+    } else if (warp == kActWarpS) {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
-        // a warp may only touch tensor-memory lanes 32*(warp % 4) .. +31
-        accum_role<MODE, TM>(warp & 3, p, wring, bars, tmem, ctl, beg, end);
+        accum_role_small<MODE, TM>(p, wring, cbuf, bars, tmem, ctl, beg, end);
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kIssuerWarp0) {
+    if (warp == kIssuerWarp0S) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -837,7 +961,8 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->issuers = pl->small ? kMaxIssuers : (tm <= 64 ? 4 : (tm <= 128 ? 2 : 1));
     pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;
     pl->blob_bytes = (mode == kModeGroup) ? static_cast<int>(blob_bytes_w4a16(slots)) : kCodeBytes;
-    const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */;
+    const int cbuf_bytes = pl->small ? 2 * 4 * 32 * tm * 4 : 0;  // accumulate warps' hand-over buffers
+    const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */ - cbuf_bytes;
     int s = budget / (pl->act_slot + pl->blob_bytes);
     if (s > kMaxSlots) s = kMaxSlots;
     if (s < 2) return -1;
@@ -846,7 +971,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     if (c > kMaxChunk) c = kMaxChunk;
     if (c < 1) c = 1;
     pl->chunk = c;
-    pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024;
+    pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + cbuf_bytes;
     pl->units = static_cast<long long>(pl->n_tiles) * pl->m_tiles * pl->k_blocks;
     pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
     return 0;

@@ -35,13 +35,21 @@ constexpr int kMaxIssuers = 4;                // MMA-issuing warps, one accumula
 constexpr int kIssuerWarp0 = kNumDqWarps;     // warps 8..11
 constexpr int kWeightWarp = kIssuerWarp0 + kMaxIssuers;  // warp 12: weight-blob copies
 constexpr int kActWarp = kWeightWarp + 1;     // warp 13: activation-tile copies
-constexpr int kAccWarp0 = kActWarp + 1;       // warps 14..17: accumulate + epilogue (small tiles)
 constexpr int kThreadsLarge = (kActWarp + 1) * 32;   // 448: epilogue runs in the dequant warps
-constexpr int kThreadsSmall = (kAccWarp0 + 4) * 32;  // 576
+// small tiles (tile_m <= 32): more warps, each on its own k-blocks
+constexpr int kDqWarpsS = 12;                 // 3 per TMEM lane quarter, round-robin over k-blocks
+constexpr int kIssuerWarp0S = kDqWarpsS;      // warps 12..15
+constexpr int kWeightWarpS = kIssuerWarp0S + kMaxIssuers;  // warp 16
+constexpr int kActWarpS = kWeightWarpS + 1;   // warp 17
+constexpr int kAccWarp0S = kActWarpS + 1;     // warps 18..25: 2 per lane quarter (k-block parity)
+constexpr int kThreadsSmall = (kAccWarp0S + 8) * 32;  // 832
+constexpr int kASlotsS = 6;                   // dequantised k-blocks in tensor memory (small tiles)
 constexpr int kSmallTileMax = 32;             // tiles of at most this many rows use per-k-block partials
+constexpr int kTmemAOffsetS = 128;            // small tiles: partials in columns [0, 128), 6 A slots above
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
 constexpr int kMaxSlots = 32;                 // shared-memory ring slots (one k-block each)
 constexpr int kMaxChunk = 4;                  // k-blocks moved by one copy
+constexpr int kChunkBars = kMaxSlots + 1;     // chunk barriers: more than ring slots
 constexpr int kASlots = 4;                    // dequantised weight tiles in tensor memory
 constexpr int kTmemCols = 512;
 constexpr int kTmemAOffset = 256;             // accumulators in columns [0, 256), A slots above
