@@ -76,18 +76,18 @@ __device__ __forceinline__ void raise_error(const Ctl& c, int code) {
 }
 
 // Bounded wait on an mbarrier phase. Returns false when the CTA aborts or the limit expires.
-// The global timer is read only every 32 unsuccessful polls.
+// Each poll lets the thread sleep in hardware until the phase completes (up to 20 us), so
+// waiting warps do not take issue slots or ALU cycles from the dequantising warps.
 __device__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c, bool honour_abort = true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    constexpr uint32_t kSuspendNs = 20000;
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 31) == 0) {
-            if (honour_abort && *c.abort_flag) return false;
-            if (global_timer_ns() - t0 > c.timeout_ns) {
-                raise_error(c, WQ_ERR_TIMEOUT);
-                return false;
-            }
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (honour_abort && *c.abort_flag) return false;
+        if (global_timer_ns() - t0 > c.timeout_ns) {
+            raise_error(c, WQ_ERR_TIMEOUT);
+            return false;
         }
     }
 }
@@ -495,9 +495,15 @@ __device__ __forceinline__ bool chunk_has(uint32_t iter0, int c, uint32_t period
     return ((residue + period - iter0 % period) % period) < static_cast<uint32_t>(c);
 }
 
-// Dequant warp of a small tile: lane quarter = warp % 4, residue = warp / 4 (period 3). It turns
+// Dequant warp of a small tile: lane quarter = warp % 4, residue = warp / 4 (period 2). It turns
 // all 16 packed words of its row of a k-block into 128 fp16 (or int8) values and stores them
-// into tensor-memory slot (walk index mod 6), where they are the MMA's A operand.
+// into tensor-memory slot (walk index mod 4), where they are the MMA's A operand.
+//
+// Every mbarrier is waited on with a parity bit, so a waiter must never run two phases ahead
+// of the barrier. The periods are chosen so that each barrier has fixed participants that see
+// all of its phases in order: A slot a (walk index = a mod 4) is always written by residue
+// group a % 2 and always read by issuer a, and partial buffer q is always read by the
+// accumulate warps of parity q % 2.
 template <int MODE>
 __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
                                    const Ctl& ctl, long long beg, long long end) {
@@ -516,11 +522,11 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
             const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
             ++ch;
-            if (chunk_has(iter, c, 3, residue)) {
+            if (chunk_has(iter, c, 2, residue)) {
                 bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
                 for (int t = 0; t < c; ++t) {
                     const uint32_t i = iter + t;
-                    if (i % 3 != residue) continue;
+                    if ((i & 1u) != residue) continue;
                     const int s = pos + t;
                     const uint32_t a = i % kASlotsS, aph = (i / kASlotsS) & 1;
                     uint4 w[4];
@@ -721,7 +727,7 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
 // (double-buffered by segment), which adds them (even + odd, a fixed order) and runs the
 // epilogue.
 template <int MODE, int TM>
-__device__ void accum_role_small(const GemmArgs& p, const uint8_t* wring, uint32_t* cbuf, Barriers& b, uint32_t tmem,
+__device__ void accum_role_small(const GemmArgs& p, uint32_t* cbuf, Barriers& b, uint32_t tmem,
                                  const Ctl& ctl, long long beg, long long end) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3;  // a warp may only touch tensor-memory lanes 32*(warp % 4) .. +31
@@ -729,61 +735,49 @@ __device__ void accum_role_small(const GemmArgs& p, const uint8_t* wring, uint32
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const bool scale_here = (MODE == kModeGroup) && !p.scale_in_dequant;
-    uint32_t ch = 0, iter = 0;
-    int pos = 0, seg_index = 0;
+    uint32_t iter = 0;
+    int seg_index = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         uint32_t acc[TM];
 #pragma unroll
         for (int c = 0; c < TM; ++c) acc[c] = 0;  // +0.0f and int 0 share the bit pattern
-        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
-            if (chunk_has(iter, c, 2, parity)) {
-                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
-                for (int t = 0; t < c; ++t) {
-                    const uint32_t i = iter + t;
-                    if ((i & 1u) != parity) continue;
-                    const int s = pos + t;
-                    const uint32_t q = i & 3u, ph = (i >> 2) & 1u;
-                    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
-                    if (!ok) continue;
-                    float sc = 1.0f;
-                    if (scale_here)
-                        sc = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(
-                            wring + static_cast<size_t>(s) * p.blob_bytes + kCodeBytes)[row]));
-                    tc_fence_after();
+        // the group scale of this column for k-block kb of the tile: read from the prepacked
+        // blob in global memory (it is L2-resident: the blob was just streamed), so these warps
+        // never hold a shared-memory ring slot
+        const int nt = seg.tile / p.m_tiles;
+        const uint8_t* tile_blobs = p.wp + static_cast<size_t>(nt) * p.k_blocks * p.blob_bytes + kCodeBytes + 2 * row;
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi; ++kb, ++iter) {
+            if ((iter & 1u) != parity) continue;
+            const uint32_t q = iter & 3u, ph = (iter >> 2) & 1u;
+            uint16_t sraw = 0;
+            if (scale_here)  // issued before the wait, consumed after it
+                sraw = __ldg(reinterpret_cast<const uint16_t*>(tile_blobs + static_cast<size_t>(kb) * p.blob_bytes));
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
+            if (!ok) continue;
+            const float sc = scale_here ? __half2float(__ushort_as_half(sraw)) : 1.0f;
+            tc_fence_after();
 #pragma unroll
-                    for (int c0 = 0; c0 < TM; c0 += 16) {  // 16 columns at a time keeps registers low
-                        uint32_t v[16];
-                        tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v);
-                        tmem_ld_wait();
-                        if (c0 + 16 >= TM) {  // every column read: hand the partial buffer back
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                mbar_arrive(&b.pempty[q]);
-                                mbar_arrive(&b.empty_w[s]);
-                            }
-                        }
+            for (int c0 = 0; c0 < TM; c0 += 16) {  // 16 columns at a time keeps registers low
+                uint32_t v[16];
+                tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v);
+                tmem_ld_wait();
+                if (c0 + 16 >= TM) {  // every column read: hand the partial buffer back
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&b.pempty[q]);
+                }
 #pragma unroll
-                        for (int c2 = 0; c2 < 16; ++c2) {
-                            if (MODE == kModeW4A8)
-                                acc[c0 + c2] = static_cast<uint32_t>(static_cast<int32_t>(acc[c0 + c2]) +
-                                                                     static_cast<int32_t>(v[c2]));
-                            else
-                                acc[c0 + c2] = __float_as_uint(
-                                    fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c0 + c2])));
-                        }
-                    }
+                for (int c2 = 0; c2 < 16; ++c2) {
+                    if (MODE == kModeW4A8)
+                        acc[c0 + c2] =
+                            static_cast<uint32_t>(static_cast<int32_t>(acc[c0 + c2]) + static_cast<int32_t>(v[c2]));
+                    else
+                        acc[c0 + c2] =
+                            __float_as_uint(fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c0 + c2])));
                 }
             }
-            iter += c;
-            kb += c;
-            pos += c;
-            if (pos == p.slots) pos = 0;
         }
         // combine the two parities of this quarter, then the even warp runs the epilogue
         uint32_t* buf = cbuf + (static_cast<size_t>(seg_index & 1) * 4 + quarter) * (32 * TM);
@@ -876,6 +870,13 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     }
 }
 
+// The small-tile protocol relies on A slot a being written by one residue group and read by one
+// issuer (period 2 dequant, period 4 issue, 4 slots) and on the A slots fitting in tensor memory
+// beside the 4 partial buffers.
+static_assert(kDqWarpsS == 8 && kASlotsS == kMaxIssuers && kMaxIssuers == 4, "small-tile periods");
+static_assert(kMaxIssuers * kSmallTileMax <= kTmemAOffsetS && kTmemAOffsetS + kASlotsS * 64 <= kTmemCols,
+              "small-tile tensor-memory columns");
+
 template <int MODE, int TM>
 __global__ void __launch_bounds__(kThreadsSmall, 1)
     wq_gemm_small(const __grid_constant__ ActMaps maps, const GemmArgs p) {
@@ -892,7 +893,7 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     if (threadIdx.x == 0) {
         for (int k = 0; k < kChunkBars; ++k) mbar_init(&bars.full[k], 2);
         for (int s = 0; s < p.slots; ++s) {
-            mbar_init(&bars.empty_w[s], 8);  // the k-block's 4 dequant warps + 4 accumulate warps
+            mbar_init(&bars.empty_w[s], 4);  // the k-block's 4 dequant warps (one per lane quarter)
             mbar_init(&bars.empty_a[s], 1);  // the owning issuer
         }
         for (int a = 0; a < kASlotsS; ++a) {
@@ -931,7 +932,7 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     } else if (warp == kActWarpS) {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
-        accum_role_small<MODE, TM>(p, wring, cbuf, bars, tmem, ctl, beg, end);
+        accum_role_small<MODE, TM>(p, cbuf, bars, tmem, ctl, beg, end);
     }
 
     tc_fence_before();

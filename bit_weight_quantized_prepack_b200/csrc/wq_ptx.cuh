@@ -49,6 +49,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
+// Like mbar_try_wait, but the thread may sleep in hardware for up to `suspend_ns` nanoseconds
+// while the phase is incomplete (it wakes as soon as the phase completes); a waiting warp
+// then issues no instructions instead of re-polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return done != 0;
+}
+
 // ------------------------------------------------------------------ TMA (bulk async copies)
 // 1-D bulk copy global -> shared, completion counted in bytes on `bar`. Both addresses
 // 16-byte aligned, size a multiple of 16.

@@ -3,19 +3,26 @@
 Every warp role of every CTA is a generator of barrier operations that follows the kernel's
 walk over its (tile, k-block) units: segments last-first, k-blocks forward, chunks of up to
 `chunk` k-blocks that never wrap the shared-memory ring, chunk barriers indexed by chunk
-number modulo 33, ring slots, tensor-memory A slots (6), partial buffers (4 issuers), the
-two accumulate parities, the named barriers of the epilogue and the stream-K publish flags.
+number modulo 33, ring slots, tensor-memory A slots (4), partial buffers (4 issuers), the
+two accumulate parities (which read only the partial buffers, never the ring), the named barriers of the epilogue and the stream-K publish flags.
 mbarriers follow the PTX phase/parity rules: a wait on parity p passes once the phase with
 that parity has completed, i.e. while the current phase's parity differs from p.
 
-`simulate` runs all roles of all CTAs until nothing can move and returns the roles still
-blocked: an empty list means the protocol cannot deadlock for that launch plan.
+Every wait also carries the number of completed phases its role means to wait for. A parity
+wait cannot tell phase n from phase n - 2 (or n + 2), so a wait that passes while the barrier
+has completed any other number of phases is a protocol error (an "alias") even when nothing
+deadlocks: the role would read a slot before it was written, or after it was overwritten.
+
+`simulate` runs all roles of all CTAs until nothing can move and returns the aliased waits and
+the roles still blocked: an empty list means the protocol is sound for that launch plan and
+that interleaving.
 """
 from collections import defaultdict
 
 NCB = 33          # chunk barriers
-NA = 6            # tensor-memory A slots
+NA = 4            # tensor-memory A slots (slot i % 4: writer residue i % 2, reader issuer i % 4)
 NQ = 4            # MMA issuers
+DQ_PERIOD = 2     # dequant warps per lane quarter; each takes the walk indices of one residue
 
 
 class Bar:
@@ -30,8 +37,9 @@ class Bar:
             self.phase += 1
             self.pending = self.count
 
-    def ready(self, parity):
-        return parity != (self.phase & 1)
+    def ready(self, need):
+        # the role waits on parity (need - 1) & 1, the parity of the phase whose completion it wants
+        return ((need - 1) & 1) != (self.phase & 1)
 
 
 def unit_start(c, units, grid):
@@ -63,7 +71,9 @@ def chunks(beg, end, kbs, chunk, slots):
         yield seg, None, None, it, ch
 
 
-def _roles(cta, units, grid, kbs, chunk, slots, B):
+def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
+    """Operations: ("wait", bar, need, walk index), ("arrive", bar), ("nbar", name, count),
+    ("flag_set", cta), ("flag_wait", cta)."""
     beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
 
     def has(it0, c, period, residue):
@@ -71,40 +81,38 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
 
     def dq(residue):
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
-            if pos is None or not has(it0, c, 3, residue):
+            if pos is None or not has(it0, c, DQ_PERIOD, residue):
                 continue
-            yield ("wait", B["full"][ch % NCB], (ch // NCB) & 1)
+            yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
             for t in range(c):
                 i = it0 + t
-                if i % 3 == residue:
+                if i % DQ_PERIOD == residue:
                     yield ("arrive", B["empty_w"][pos + t])
-                    yield ("wait", B["aempty"][i % NA], ((i // NA) & 1) ^ 1)
+                    yield ("wait", B["aempty"][i % NA], i // NA, i)
                     yield ("arrive", B["afull"][i % NA])
 
     def issuer(q):
-        j = 0
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None or not has(it0, c, NQ, q):
                 continue
-            yield ("wait", B["full"][ch % NCB], (ch // NCB) & 1)
+            yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
             for t in range(c):
                 i = it0 + t
                 if i % NQ == q:
-                    yield ("wait", B["afull"][i % NA], (i // NA) & 1)
-                    yield ("wait", B["pempty"][q], (j & 1) ^ 1)
-                    j += 1
+                    yield ("wait", B["afull"][i % NA], i // NA + 1, i)
+                    yield ("wait", B["pempty"][q], i // NQ, i)
                     yield ("arrive", B["aempty"][i % NA])
                     yield ("arrive", B["empty_a"][pos + t])
                     yield ("arrive", B["pfull"][q])
 
     def producer(which):
-        ebits = [0] * slots
+        uses = [0] * slots
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
                 continue
             for t in range(c):
-                yield ("wait", B[which][pos + t], ebits[pos + t] ^ 1)
-                ebits[pos + t] ^= 1
+                yield ("wait", B[which][pos + t], uses[pos + t], it0 + t)
+                uses[pos + t] += 1
             yield ("arrive", B["full"][ch % NCB])
 
     def acc(quarter, parity):
@@ -126,18 +134,20 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
                             cc -= 1
                         yield ("nbar", "epi", 4)
                 continue
-            if not has(it0, c, 2, parity):
-                continue
-            yield ("wait", B["full"][ch % NCB], (ch // NCB) & 1)
+            if acc_in_ring:  # an earlier protocol: the accumulate warps read scales from the ring
+                if not has(it0, c, 2, parity):
+                    continue
+                yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
             for t in range(c):
                 i = it0 + t
                 if i % 2 == parity:
-                    yield ("wait", B["pfull"][i % NQ], (i // NQ) & 1)
+                    yield ("wait", B["pfull"][i % NQ], i // NQ + 1, i)
                     yield ("arrive", B["pempty"][i % NQ])
-                    yield ("arrive", B["empty_w"][pos + t])
+                    if acc_in_ring:
+                        yield ("arrive", B["empty_w"][pos + t])
 
     roles = {}
-    for w in range(12):          # 3 dequant warps per lane quarter; the quarters move together
+    for w in range(4 * DQ_PERIOD):
         roles[f"dq{w}"] = dq(w >> 2)
     for q in range(NQ):
         roles[f"iss{q}"] = issuer(q)
@@ -148,51 +158,72 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
     return roles
 
 
-def simulate(units, grid, kbs, chunk, slots):
+def simulate(units, grid, kbs, chunk, slots, acc_in_ring=False, rng=None, ctas_only=None):
+    """Runs the roles of the CTAs (all, or `ctas_only`) to a standstill. With `rng` the roles
+    move in a random order and a random number of operations at a time (any object with
+    `shuffle(list)` and `randint(a, b)` can bias the interleaving). Returns a list of problems:
+    ("alias", cta, role, barrier, phases needed, phases completed) for each wait that passed on
+    the wrong phase, and (cta, role, pending operation) for each role left blocked."""
     flags = {}
+    if ctas_only is not None:  # CTAs outside the subset count as having published
+        flags = {c: 1 for c in range(grid) if c not in ctas_only}
     ctas = []
-    for cta in range(grid):
+    for cta in (range(grid) if ctas_only is None else ctas_only):
         B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
-             "empty_w": [Bar(8, f"empty_w{s}") for s in range(slots)],
+             "empty_w": [Bar(8 if acc_in_ring else 4, f"empty_w{s}") for s in range(slots)],
              "empty_a": [Bar(1, f"empty_a{s}") for s in range(slots)],
              "afull": [Bar(4, f"afull{a}") for a in range(NA)],
              "aempty": [Bar(1, f"aempty{a}") for a in range(NA)],
              "pfull": [Bar(1, f"pfull{q}") for q in range(NQ)],
              "pempty": [Bar(4, f"pempty{q}") for q in range(NQ)]}
-        roles = _roles(cta, units, grid, kbs, chunk, slots, B)
+        roles = _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
                      "nbar": defaultdict(list)})
+    problems = []
     moved = True
     while moved:
         moved = False
-        for st in ctas:
-            for name, gen in st["roles"].items():
-                while name not in st["done"]:
-                    op = st["cur"][name]
-                    if op is None:
-                        try:
-                            op = st["cur"][name] = next(gen)
-                        except StopIteration:
-                            st["done"].add(name)
-                            break
-                    kind = op[0]
-                    if kind == "wait" and not op[1].ready(op[2]):
-                        break
-                    if kind == "flag_wait" and not flags.get(op[1]):
-                        break
-                    if kind == "arrive":
-                        op[1].arrive()
-                    elif kind == "flag_set":
-                        flags[op[1]] = 1
-                    elif kind == "nbar":
-                        waiting = st["nbar"][op[1]]
-                        if name not in waiting:
-                            waiting.append(name)
-                        if len(waiting) < op[2]:
-                            break
-                        for other in waiting:
-                            st["cur"][other] = None
-                        st["nbar"][op[1]] = []
-                    st["cur"][name] = None
+        order = [(st, name) for st in ctas for name in st["roles"]]
+        if rng is not None:
+            rng.shuffle(order)
+        for st, name in order:
+            gen = st["roles"][name]
+            steps = 0
+            while name not in st["done"]:
+                if rng is not None and steps >= rng.randint(1, 4):
                     moved = True
-    return [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+                    break
+                steps += 1
+                op = st["cur"][name]
+                if op is None:
+                    try:
+                        op = st["cur"][name] = next(gen)
+                    except StopIteration:
+                        st["done"].add(name)
+                        break
+                kind = op[0]
+                if kind == "wait":
+                    if not op[1].ready(op[2]):
+                        break
+                    if op[1].phase != op[2]:
+                        problems.append(("alias", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "flag_wait":
+                    if not flags.get(op[1]):
+                        break
+                elif kind == "arrive":
+                    op[1].arrive()
+                elif kind == "flag_set":
+                    flags[op[1]] = 1
+                elif kind == "nbar":
+                    waiting = st["nbar"][op[1]]
+                    if name not in waiting:
+                        waiting.append(name)
+                    if len(waiting) < op[2]:
+                        break
+                    for other in waiting:
+                        st["cur"][other] = None
+                    st["nbar"][op[1]] = []
+                st["cur"][name] = None
+                moved = True
+    stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+    return problems + stuck

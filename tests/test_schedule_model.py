@@ -26,9 +26,9 @@ def test_no_deadlock(K, N, slots):
 
 
 def test_model_catches_slot_indexed_barrier_hazard():
-    # the earlier protocol indexed chunk barriers by ring slot; the same model with that
-    # indexing deadlocks on the 8192 x 10240 layer with a 17-slot ring (seen on the GPU as an
-    # expired wait on 4 tiles)
+    # an earlier protocol (accumulate warps reading scales from the ring) with chunk barriers
+    # indexed by ring slot deadlocks on the 8192 x 10240 layer with a 17-slot ring; the GPU
+    # showed it as an expired wait on 4 tiles. Chunk-number indexing removes it.
     import schedule_model as sm
     orig = sm.chunks
 
@@ -45,6 +45,62 @@ def test_model_catches_slot_indexed_barrier_hazard():
     sm.chunks = slot_indexed
     try:
         units, grid, kbs = _plan(8192, 10240)
-        assert simulate(units, grid, kbs, 4, 17)
+        assert simulate(units, grid, kbs, 4, 17, acc_in_ring=True)
     finally:
         sm.chunks = orig
+    assert not simulate(units, grid, kbs, 4, 17, acc_in_ring=True)
+
+
+class _Biased:
+    """An interleaving that always moves the roles `first` picks before the others (random
+    order within each group), each as far as it can: the extreme schedules that let one kind
+    of warp run ahead of the rest."""
+
+    def __init__(self, first, seed):
+        import random
+        self.r, self.first = random.Random(seed), first
+
+    def shuffle(self, order):
+        keyed = sorted((0 if self.first(x[1]) else 1, self.r.random(), k) for k, x in enumerate(order))
+        order[:] = [order[k[2]] for k in keyed]
+
+    def randint(self, a, b):
+        return 1 << 30
+
+
+_KINDS = ["dq", "iss", "prod", "acc"]
+_BIASES = {f"{k}-first": (lambda k: lambda n: n.startswith(k))(k) for k in _KINDS}
+_BIASES.update({f"{k}-last": (lambda k: lambda n: not n.startswith(k))(k) for k in _KINDS})
+_BIASES["one-dq-warp-first"] = lambda n: n == "dq0"
+_BIASES["one-dq-warp-last"] = lambda n: n != "dq1"
+
+
+@pytest.mark.parametrize("K,N", [(8192, 57344), (4096, 22016), (8192, 10240), (1024, 136)])
+@pytest.mark.parametrize("slots", [9, 16, 17])
+def test_no_alias_or_deadlock_under_skewed_schedules(K, N, slots):
+    import random
+    units, grid, kbs = _plan(K, N)
+    for cta in sorted({0, grid // 2, grid - 1}):
+        for name, first in _BIASES.items():
+            problems = simulate(units, grid, kbs, min(4, slots // 2), slots, rng=_Biased(first, cta), ctas_only=[cta])
+            assert not problems, (name, cta, problems[:3])
+        for seed in range(3):
+            problems = simulate(units, grid, kbs, min(4, slots // 2), slots, rng=random.Random(seed), ctas_only=[cta])
+            assert not problems, ("random", seed, cta, problems[:3])
+
+
+def test_model_catches_period_mismatch():
+    # an earlier protocol had 3 dequant warps per lane quarter and 6 A slots against 4 issuers:
+    # an issuer could wait on A slot (i mod 6) two phases early and pass on the parity of an
+    # older phase. Enough skew (accumulate warps always first) makes it happen on the
+    # 8192 x 57344 layer with a 9-slot ring; the GPU showed it as expired waits.
+    import schedule_model as sm
+    units, grid, kbs = _plan(8192, 57344)
+    saved = sm.NA, sm.DQ_PERIOD
+    sm.NA, sm.DQ_PERIOD = 6, 3
+    try:
+        problems = simulate(units, grid, kbs, 4, 9, rng=_Biased(_BIASES["acc-first"], 0), ctas_only=[0])
+    finally:
+        sm.NA, sm.DQ_PERIOD = saved
+    assert any(p[0] == "alias" and p[3].startswith("afull") for p in problems)
+    assert not simulate(units, grid, kbs, 4, 9, rng=_Biased(_BIASES["acc-first"], 0), ctas_only=[0])
