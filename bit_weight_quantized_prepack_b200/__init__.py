@@ -16,17 +16,18 @@ import torch
 __all__ = [
     "WqError", "lib", "LIB_PATH", "status_string", "wq_version",
     "wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepack", "wq_prepack_w4a8",
-    "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a8",
+    "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a16_noalloc", "wq_gemm_w4a8",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
     "WQ_ERR_UNSUPPORTED_DEVICE", "WQ_ERR_CUDA", "WQ_ERR_TIMEOUT", "WQ_ERR_NO_MEMORY", "WQ_ERR_CAPTURING",
+    "WQ_ERR_SCRATCH_LIMIT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
 
 (WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_UNSUPPORTED_SHAPE, WQ_ERR_MISALIGNED, WQ_ERR_UNSUPPORTED_DEVICE,
- WQ_ERR_CUDA, WQ_ERR_TIMEOUT, WQ_ERR_NO_MEMORY, WQ_ERR_CAPTURING) = range(9)
+ WQ_ERR_CUDA, WQ_ERR_TIMEOUT, WQ_ERR_NO_MEMORY, WQ_ERR_CAPTURING, WQ_ERR_SCRATCH_LIMIT) = range(10)
 
 
 class WqError(RuntimeError):
@@ -56,6 +57,7 @@ def _load():
         "wq_unpack": (I, [P, I, I, I, P, P, P]),
         "wq_unpack_w4a8": (I, [P, I, I, P, P]),
         "wq_gemm_w4a16": (I, [P, P, P, I, I, I, I, P]),
+        "wq_gemm_w4a16_noalloc": (I, [P, P, P, I, I, I, I, P]),
         "wq_gemm_w4a8": (I, [P, P, P, P, P, P, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
@@ -166,6 +168,18 @@ def wq_gemm_w4a16(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Te
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _dev_tensor(Y, torch.float16, "Y")
     _check(lib.wq_gemm_w4a16(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)), "wq_gemm_w4a16")
+    return Y
+
+
+def wq_gemm_w4a16_noalloc(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor, stream=None):
+    """wq_gemm_w4a16 for callers that must not allocate: the library's stream-K scratch is a
+    fixed 8 MiB device array (M <= 64 on a 148-SM B200) and Y must be given. Calls whose
+    kernels overlap on the GPU race on that array."""
+    _dev_tensor(A, torch.float16, "A")
+    _dev_tensor(Y, torch.float16, "Y")
+    M, K = A.shape
+    _check(lib.wq_gemm_w4a16_noalloc(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)),
+           "wq_gemm_w4a16_noalloc")
     return Y
 
 

@@ -256,6 +256,79 @@ int prepack_common_checks(const void* Q, int K, int N, const void* Wp, cudaStrea
 
 }  // namespace
 
+// ---------------------------------------------------------------- fixed-scratch W4A16 call
+// Some callers cannot call cudaMalloc at the point where they run the layer: an engine that
+// hands all free device memory to its own pool (KV cache, activations) at start-up and must
+// not see outside allocations fail or fragment it; a plugin whose host framework owns every
+// allocation; a latency-critical loop that must not risk the implicit synchronisation of an
+// allocation. wq_gemm_w4a16 grows a per-(device, stream) workspace with cudaMalloc on first
+// use; wq_gemm_w4a16_noalloc runs the same kernels with their stream-K scratch (publish flags
+// and partial tiles) in the fixed array below instead, which the CUDA module loader sets
+// aside on every device that loads this library, for the life of the process.
+//
+// Layout: flags int32 [grid] at offset 0 (must be zero at launch; cleared by every call),
+// partial tiles from offset 4096, the kernels' status word in the last 256 bytes.
+constexpr size_t kNoAllocScratchBytes = WQ_NOALLOC_SCRATCH_BYTES;
+constexpr size_t kNoAllocStatusOffset = kNoAllocScratchBytes - 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocDevice {
+    bool ready = false;
+    int num_sms = 0;
+    int smem_optin = 0;
+    unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocDevice g_noalloc[kNoAllocMaxDevices];
+
+// One-time set-up of the current device for the fixed-scratch call: no allocation, only
+// attribute queries, kernel attributes, the symbol's device address and two blocking clears.
+int noalloc_device(int* dev_out, NoAllocDevice** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return WQ_ERR_UNSUPPORTED_DEVICE;
+    NoAllocDevice& d = g_noalloc[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return WQ_ERR_CUDA;
+        if (major != 10 || minor != 0) return WQ_ERR_UNSUPPORTED_DEVICE;
+        if (configure_gemm_kernels(d.smem_optin - 2048) != cudaSuccess) return WQ_ERR_CUDA;
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return WQ_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        // host code must not use g_noalloc_scratch itself: on the host it names a stand-in
+        // object, not device memory. The device address is per device, taken with it current.
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return WQ_ERR_CUDA;
+        }
+        unsigned char* base = static_cast<unsigned char*>(p);
+        if (cudaMemset(base, 0, 4096) != cudaSuccess) return WQ_ERR_CUDA;
+        if (cudaMemset(base + kNoAllocStatusOffset, 0, 256) != cudaSuccess) return WQ_ERR_CUDA;
+        d.scratch = base;
+        d.ready = true;
+    }
+    *dev_out = dev;
+    *out = &d;
+    return WQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* wq_status_string(int status) {
@@ -270,6 +343,9 @@ const char* wq_status_string(int status) {
         case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: a device-side wait expired";
         case WQ_ERR_NO_MEMORY: return "WQ_ERR_NO_MEMORY: workspace allocation failed";
         case WQ_ERR_CAPTURING: return "WQ_ERR_CAPTURING: reserve the workspace before capturing the stream";
+        case WQ_ERR_SCRATCH_LIMIT:
+            return "WQ_ERR_SCRATCH_LIMIT: the call needs more stream-K scratch than the fixed array of "
+                   "wq_gemm_w4a16_noalloc holds (use wq_gemm_w4a16)";
         default: return "WQ_ERR_UNKNOWN";
     }
 }
@@ -445,6 +521,79 @@ int wq_debug_set_wait_timeout_ns(unsigned long long ns) {
 int wq_debug_skip_publish(int cta) {
     std::lock_guard<std::mutex> lock(g_mu);
     g_skip_publish = cta;
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g,
+                          void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = check_shape(K, N);
+    if (rc) return rc;
+    if (M < 0) return WQ_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (!Wp) return WQ_ERR_INVALID_ARG;
+    if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
+    if (M == 0) return WQ_OK;
+    if (!A || !Y) return WQ_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(Y, 16)) return WQ_ERR_MISALIGNED;
+
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    NoAllocDevice* d = nullptr;
+    rc = noalloc_device(&dev, &d);
+    if (rc) return rc;
+    DeviceState ds;
+    ds.init = ds.supported = true;
+    ds.num_sms = d->num_sms;
+    ds.smem_optin = d->smem_optin;
+    Plan pl;
+    rc = plan_for(0, M, N, K, g, ds, &pl);
+    if (rc) return rc;
+    if (workspace_bytes_for(pl) > kNoAllocStatusOffset) return WQ_ERR_SCRATCH_LIMIT;
+    ActMaps maps;
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false);
+    if (rc) return rc;
+    // the scratch keeps whatever the last call left; the publish flags must start at zero
+    if (cudaMemsetAsync(d->scratch, 0, static_cast<size_t>(pl.grid) * sizeof(int), st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+
+    // the same launch arguments as wq_gemm_w4a16, with the scratch in place of the workspace
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.wp = static_cast<const uint8_t*>(Wp);
+    a.s_chan = (pl.mode == kModeChannel)
+                   ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
+                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * kCodeBytes)
+                   : nullptr;
+    a.y = Y;
+    a.ws_flags = reinterpret_cast<int*>(d->scratch);
+    a.ws_partial = reinterpret_cast<float*>(d->scratch + 4096);
+    a.status = reinterpret_cast<int*>(d->scratch + kNoAllocStatusOffset);
+    a.M = M;
+    a.N = N;
+    a.m_tiles = pl.m_tiles;
+    a.n_tiles = pl.n_tiles;
+    a.k_blocks = pl.k_blocks;
+    a.tile_m = pl.tile_m;
+    a.issuers = pl.issuers;
+    a.slots = pl.slots;
+    a.chunk = pl.chunk;
+    a.act_slot = pl.act_slot;
+    a.blob_bytes = pl.blob_bytes;
+    a.group_rows = g < kTileK ? g : kTileK;
+    a.small = pl.small ? 1 : 0;
+    a.scale_in_dequant = (pl.mode == kModeGroup && (!pl.small || g < kTileK)) ? 1 : 0;
+    a.units = pl.units;
+    a.grid = pl.grid;
+    a.timeout_ns = g_timeout_ns;
+    a.skip_publish = -1;
+    if (launch_gemm(pl.mode, maps, a, pl, st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
     return WQ_OK;
 }
 

@@ -61,7 +61,8 @@ typedef enum {
     WQ_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
     WQ_ERR_TIMEOUT = 6,            /* a device-side bounded wait expired (see wq_get_device_status) */
     WQ_ERR_NO_MEMORY = 7,          /* the library could not allocate its workspace */
-    WQ_ERR_CAPTURING = 8           /* the workspace must grow while the stream is being captured */
+    WQ_ERR_CAPTURING = 8,          /* the workspace must grow while the stream is being captured */
+    WQ_ERR_SCRATCH_LIMIT = 9       /* wq_gemm_w4a16_noalloc: the plan needs more than its fixed scratch */
 } wq_status_t;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -109,6 +110,31 @@ WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
  * Requires K <= 131072 so that no int32 partial sum can overflow. */
 WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw,
                  uint16_t* Y, int32_t* acc_out, int M, int N, int K, void* stream);
+
+/* W4A16 without any allocation. No counterpart in the paper: it exists for callers that
+ * cannot allocate device memory when they run the layer (an engine that gave all free
+ * memory to its own pool at start-up, a plugin whose host framework owns every
+ * allocation, a latency-critical loop that must not risk an allocation's implicit
+ * synchronisation). Same arguments, result bits and status codes as wq_gemm_w4a16, but
+ * the stream-K scratch (publish flags, partial tiles) lives in one fixed array of
+ * WQ_NOALLOC_SCRATCH_BYTES (8 MiB) that every device loading the library holds until
+ * the process exits; this call never calls cudaMalloc or cudaFree.
+ * - Limit: a plan whose scratch (4 KiB + grid * tile rows * 128 * 4 bytes) does not fit
+ *   returns WQ_ERR_SCRATCH_LIMIT and launches nothing. On a 148-SM B200 every M <= 64
+ *   fits; larger M (tiles of 128 or 256 rows) does not.
+ * - Set-up: the first call on a device (with that device current) configures the
+ *   kernels, looks up the array's device address and clears it with blocking memsets;
+ *   make that first call before any stream capture.
+ * - Every call clears the publish flags on `stream` before its kernel, so a call does not
+ *   depend on what an earlier one left in the array.
+ * - All calls on one device share the array: two calls whose kernels overlap on the GPU
+ *   (different streams without ordering between them) race and give wrong results.
+ *   Order them on one stream or with events.
+ * - A device-side wait that expires stops the kernel as in wq_gemm_w4a16, but is recorded
+ *   in the array, not in the word wq_get_device_status reads: it is not reported. */
+#define WQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
+                  int M, int N, int K, int g, void* stream);
 
 /* ---------------------------------------------------------------- workspace and status
  * Bytes of library workspace one call of the given kind and shape needs
