@@ -15,6 +15,8 @@ slowest rank's device time (GB/s); algorithmic bytes of one call = K*N/2 (codes)
 2*(K/g)*N (scales) + 2*M*K (A) + 2*M*N (Y). ``--gpus N`` runs N independent replicas (the
 layer does not shard across GPUs here), one process per GPU under torchrun.
 ``--impl reference`` times the CPU fp64 oracle on a bounded sample of the same workload.
+``--case K,N,g,M`` replaces the layer set by one layer (profiling runs): a step is then one
+call on each of enough rotated prepacked copies to exceed L2 three times over.
 """
 from __future__ import annotations
 
@@ -420,7 +422,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-M breakdown (short profiler runs)")
     ap.add_argument("--reference-budget", type=float, default=90.0, help="seconds the reference arm aims for")
+    ap.add_argument("--case", default=None, help="K,N,g,M: one layer instead of the layer set (profiling)")
     args = ap.parse_args(argv)
+    if args.case:
+        global LAYERS, M_SWEEP, G, COPIES, WORKLOAD
+        K, N, g, M = (int(v) for v in args.case.split(","))
+        LAYERS, G = [(K, N)], g
+        COPIES = int(min(64, max(2, -(-3 * 126e6 // (K * N // 2 + 2 * (K // g) * N)))))
+        M_SWEEP = [M] * COPIES
+        WORKLOAD = f"single_layer_K{K}_N{N}_g{g}_M{M}_x{COPIES}_copies"
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank = int(os.environ.get("RANK", "0"))
