@@ -388,6 +388,7 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                               const Ctl& ctl, long long beg, long long end) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
     uint32_t ebits = 0, ch = 0, armed = 0;
+    uint32_t first_pass_chunks = 0xffffffffu;  // chunks before the ring first wraps
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
@@ -398,7 +399,8 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
             for (int t = 0; t < c; ++t) {
                 const int s = pos + t;
-                if (ok) ok = wait_bar(kWeights ? &b.empty_w[s] : &b.empty_a[s], ((ebits >> s) & 1u) ^ 1u, ctl);
+                if (ok && ch >= first_pass_chunks)  // a slot's first use needs no wait
+                    ok = wait_bar(kWeights ? &b.empty_w[s] : &b.empty_a[s], ((ebits >> s) & 1u) ^ 1u, ctl);
                 ebits ^= 1u << s;
             }
             if (ok) {
@@ -417,7 +419,10 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
             ++ch;
             kb += c;
             pos += c;
-            if (pos == p.slots) pos = 0;
+            if (pos == p.slots) {
+                pos = 0;
+                if (first_pass_chunks == 0xffffffffu) first_pass_chunks = ch;
+            }
         }
     }
     // wind-down: every copy this CTA started must land before the CTA exits (after an expired
@@ -642,49 +647,74 @@ __device__ void issuer_role_small(int q, const GemmArgs& p, const uint8_t* aring
     wait_bar(&b.drain[q], 0, ctl, false);
 }
 
-// Epilogue of a small tile from the accumulate warps' registers: thread (quarter, lane) holds
-// the TM sums of output column n = tile*128 + quarter*32 + lane for rows 0..TM-1.
+// Epilogue of a small tile, shared by the two accumulate parities: the warp of parity h in lane
+// quarter q holds, in lane l, the sums of output column n = tile*128 + 32q + l for the tile rows
+// h*TM/2 .. h*TM/2 + TM/2 - 1. Only rows below M are stored, published or fetched.
+//
+// A CTA that does not own the tile writes its partial rows to its workspace slot and (after
+// all 8 accumulate warps have written) releases its flag. The owner finds the contributing
+// CTAs directly (those before it whose unit range reaches into the tile), lets each lane poll
+// one contributor's flag, then adds the contributors' partials in descending CTA order with
+// several contributors' loads in flight at a time.
 template <int MODE, int TM>
-__device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&acc)[TM], bool ok,
-                               int quarter, int lane) {
+__device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM / 2], bool ok,
+                               int quarter, int lane, int half) {
+    constexpr int H = TM / 2;
+    constexpr int kBatch = (H <= 8) ? 4 : 1;  // contributors whose loads are in flight together
     const int row = quarter * 32 + lane;
     const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
     const int n = nt * kTileN + row;
-    const int m_base = mt * TM;
+    const int r0 = half * H;  // first tile row of this half
+    int live = p.M - mt * TM - r0;
+    live = live < 0 ? 0 : (live > H ? H : live);
     const bool leader = static_cast<int>(threadIdx.x) == kAccWarp0S * 32;
+    const int me = static_cast<int>(blockIdx.x);
     if (!seg.owner) {
-        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(blockIdx.x) * TM * kTileN;
+        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(me) * TM * kTileN;
         if (ok) {
 #pragma unroll
-            for (int c = 0; c < TM; ++c) part[static_cast<size_t>(c) * kTileN + row] = acc[c];
+            for (int c = 0; c < H; ++c)
+                if (c < live) part[static_cast<size_t>(r0 + c) * kTileN + row] = v[c];
         }
         __threadfence();
-        named_barrier_sync(2, 128);
-        if (leader && ok && !*ctl.abort_flag && static_cast<int>(blockIdx.x) != p.skip_publish)
-            st_release_gpu(&p.ws_flags[blockIdx.x], 1);
+        named_barrier_sync(2, 256);
+        if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
         return;
     }
-    const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
-    const int c_first = static_cast<int>(blockIdx.x) - 1;
-    int c_last = c_first + 1;
+    int c_last = me;  // contributors are CTAs c_last .. me - 1
     if (!seg.whole) {
-        for (int c = c_first; c >= 0; --c) {
-            c_last = c;
-            if (ok) ok = wait_flag(&p.ws_flags[c], ctl);
-            if (unit_start(c, p.units, p.grid) <= tbase) break;
+        // the CTA holding the tile's first unit: the smallest c with unit_start(c + 1) > tbase
+        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        const int ncontrib = me - c_last;
+        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
+            bool good = true;
+            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
+            ok = __all_sync(0xffffffffu, good) && ok;
         }
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok) {
-            for (int cc = c_first; cc >= c_last; --cc) {
-                const uint32_t* part =
-                    reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(cc) * TM * kTileN;
+        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
+        if (ok && live > 0) {
+            for (int j = 0; j < ncontrib; j += kBatch) {
+                uint32_t w[kBatch][H];
 #pragma unroll
-                for (int c = 0; c < TM; ++c) {
-                    const uint32_t v = __ldcg(part + static_cast<size_t>(c) * kTileN + row);
-                    if (MODE == kModeW4A8)
-                        acc[c] = static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(v));
-                    else
-                        acc[c] = __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(v));
+                for (int b = 0; b < kBatch; ++b) {
+                    const uint32_t* part =
+                        reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
+#pragma unroll
+                    for (int c = 0; c < H; ++c)
+                        w[b][c] = (j + b < ncontrib && c < live) ? __ldcg(part + static_cast<size_t>(r0 + c) * kTileN + row) : 0u;
+                }
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    if (j + b < ncontrib) {
+#pragma unroll
+                        for (int c = 0; c < H; ++c) {
+                            if (MODE == kModeW4A8)
+                                v[c] = static_cast<uint32_t>(static_cast<int32_t>(v[c]) + static_cast<int32_t>(w[b][c]));
+                            else
+                                v[c] = __float_as_uint(__uint_as_float(v[c]) + __uint_as_float(w[b][c]));
+                        }
+                    }
                 }
             }
         }
@@ -694,38 +724,38 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
         if (MODE == kModeChannel) s_col = __half2float(__ushort_as_half(p.s_chan[n]));
         if (MODE == kModeW4A8) sw_col = p.sw[n];
 #pragma unroll
-        for (int c = 0; c < TM; ++c) {
-            const int m = m_base + c;
-            if (m < p.M) {
+        for (int c = 0; c < H; ++c) {
+            if (c < live) {
+                const int m = mt * TM + r0 + c;
                 const size_t o = static_cast<size_t>(m) * p.N + n;
                 float y;
                 if (MODE == kModeW4A8) {
-                    const int32_t a = static_cast<int32_t>(acc[c]) >> 4;
+                    const int32_t a = static_cast<int32_t>(v[c]) >> 4;
                     if (p.acc_out) p.acc_out[o] = a;
                     const float t = static_cast<float>(a) * p.sa[m];
                     y = t * sw_col;
                 } else if (MODE == kModeChannel) {
-                    y = __uint_as_float(acc[c]) * s_col;
+                    y = __uint_as_float(v[c]) * s_col;
                 } else {
-                    y = __uint_as_float(acc[c]);
+                    y = __uint_as_float(v[c]);
                 }
                 p.y[o] = __half_as_ushort(__float2half_rn(y));
             }
         }
     }
     if (!seg.whole) {
-        named_barrier_sync(2, 128);
+        named_barrier_sync(2, 256);  // every accumulate warp has read the partials
         if (leader)
-            for (int cc = c_first; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
+            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
     }
 }
 
 // Accumulate warp of a small tile: lane quarter = warp % 4, parity = which k-blocks (walk index
 // mod 2) it adds. Each k-block's partial is added in k order into fp32 (or int32) registers,
 // with the k-block's group scale applied when the dequant did not. At the end of a segment the
-// odd-parity warp hands its sums to the even-parity warp of its quarter through shared memory
-// (double-buffered by segment), which adds them (even + odd, a fixed order) and runs the
-// epilogue.
+// two parity warps of a quarter swap halves of their sums through shared memory (double-
+// buffered by segment): each then holds the complete sums of half of the tile rows (even +
+// odd, a fixed order) and runs the epilogue for them.
 template <int MODE, int TM>
 __device__ void accum_role_small(const GemmArgs& p, uint32_t* cbuf, Barriers& b, uint32_t tmem,
                                  const Ctl& ctl, long long beg, long long end) {
@@ -779,24 +809,39 @@ __device__ void accum_role_small(const GemmArgs& p, uint32_t* cbuf, Barriers& b,
                 }
             }
         }
-        // combine the two parities of this quarter, then the even warp runs the epilogue
+        // the two parities of this quarter exchange halves: parity h keeps tile rows h*TM/2 ..
+        // and adds the other parity's sums for them (even + odd, a fixed order)
+        constexpr int H = TM / 2;
         uint32_t* buf = cbuf + (static_cast<size_t>(seg_index & 1) * 4 + quarter) * (32 * TM);
-        if (parity == 1) {
+        const int mt = seg.tile % p.m_tiles;
+        const int live = p.M - mt * TM;  // tile rows below M
+        uint32_t v[H];
+        if (parity == 0) {
 #pragma unroll
-            for (int c = 0; c < TM; ++c) buf[c * 32 + lane] = acc[c];
-            named_barrier_sync(3 + quarter, 64);
-        } else {
+            for (int c = 0; c < H; ++c)
+                if (H + c < live) buf[(H + c) * 32 + lane] = acc[H + c];
             named_barrier_sync(3 + quarter, 64);
 #pragma unroll
-            for (int c = 0; c < TM; ++c) {
-                const uint32_t o = buf[c * 32 + lane];
-                if (MODE == kModeW4A8)
-                    acc[c] = static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(o));
-                else
-                    acc[c] = __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(o));
+            for (int c = 0; c < H; ++c) {
+                const uint32_t o = (c < live) ? buf[c * 32 + lane] : 0u;
+                v[c] = (MODE == kModeW4A8)
+                           ? static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(o))
+                           : __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(o));
             }
-            epilogue_small<MODE, TM>(p, ctl, seg, acc, ok && !*ctl.abort_flag, quarter, lane);
+        } else {
+#pragma unroll
+            for (int c = 0; c < H; ++c)
+                if (c < live) buf[c * 32 + lane] = acc[c];
+            named_barrier_sync(3 + quarter, 64);
+#pragma unroll
+            for (int c = 0; c < H; ++c) {
+                const uint32_t e = (H + c < live) ? buf[(H + c) * 32 + lane] : 0u;
+                v[c] = (MODE == kModeW4A8)
+                           ? static_cast<uint32_t>(static_cast<int32_t>(e) + static_cast<int32_t>(acc[H + c]))
+                           : __float_as_uint(__uint_as_float(e) + __uint_as_float(acc[H + c]));
+            }
         }
+        epilogue_small<MODE, TM>(p, ctl, seg, v, ok && !*ctl.abort_flag, quarter, lane, static_cast<int>(parity));
         ++seg_index;
     }
 }
@@ -805,6 +850,23 @@ __device__ void accum_role_small(const GemmArgs& p, uint32_t* cbuf, Barriers& b,
 __device__ __forceinline__ uint8_t* align_ring(uint8_t* smem_dyn) {
     const uint32_t raw = smem_addr(smem_dyn);
     return smem_dyn + ((1024u - (raw & 1023u)) & 1023u);  // swizzle atoms need 1024-byte alignment
+}
+
+// Number of weight blobs each CTA asks L2 to prefetch at kernel entry: HBM starts streaming
+// the first k-blocks while the CTA initialises barriers and tensor memory.
+constexpr int kPrefetchBlobs = 8;
+
+__device__ void prefetch_first_blobs(const GemmArgs& p, long long beg, long long end) {
+    SegCursor seg(beg, end, p.k_blocks);
+    int left = kPrefetchBlobs;
+    while (left > 0 && seg.next()) {
+        const int nt = seg.tile / p.m_tiles;
+        int n = seg.kb_hi - seg.kb_lo + 1;
+        if (n > left) n = left;
+        prefetch_l2_bulk(p.wp + (static_cast<size_t>(nt) * p.k_blocks + seg.kb_lo) * p.blob_bytes,
+                         static_cast<uint32_t>(n * p.blob_bytes));
+        left -= n;
+    }
 }
 
 template <int MODE>
@@ -819,20 +881,25 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
-        for (int k = 0; k < kChunkBars; ++k) mbar_init(&bars.full[k], 2);
-        for (int s = 0; s < p.slots; ++s) {
+    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
+    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+    if (warp == kWeightWarp && lane == 0) prefetch_first_blobs(p, beg, end);
+    if (warp == 0) {  // the lanes of warp 0 initialise the barriers side by side
+        for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
+        for (int s = lane; s < p.slots; s += 32) {
             mbar_init(&bars.empty_w[s], kNumDqWarps);
             mbar_init(&bars.empty_a[s], p.issuers);
         }
-        for (int a = 0; a < kASlots; ++a) {
-            mbar_init(&bars.afull[a][0], 4);
-            mbar_init(&bars.afull[a][1], 4);
-            mbar_init(&bars.aempty[a], p.issuers);
+        if (lane < kASlots) {
+            mbar_init(&bars.afull[lane][0], 4);
+            mbar_init(&bars.afull[lane][1], 4);
+            mbar_init(&bars.aempty[lane], p.issuers);
         }
-        mbar_init(&bars.dfull, p.issuers);
-        for (int q = 0; q < kMaxIssuers; ++q) mbar_init(&bars.drain[q], 1);
-        abort_flag = 0;
+        if (lane == 0) {
+            mbar_init(&bars.dfull, p.issuers);
+            abort_flag = 0;
+        }
+        if (lane < kMaxIssuers) mbar_init(&bars.drain[lane], 1);
         fence_barrier_init();
     }
     if (warp == kIssuerWarp0) {
@@ -847,8 +914,6 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     const uint32_t tmem = tmem_slot;
 
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
-    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
-    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
 
     if (warp < kNumDqWarps) {
         dequant_role<MODE>(p, wring, bars, tmem, ctl, beg, end);
@@ -890,22 +955,25 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     uint32_t* cbuf = reinterpret_cast<uint32_t*>(wring + static_cast<size_t>(p.slots) * p.blob_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    if (threadIdx.x == 0) {
-        for (int k = 0; k < kChunkBars; ++k) mbar_init(&bars.full[k], 2);
-        for (int s = 0; s < p.slots; ++s) {
+    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
+    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+    if (warp == kWeightWarpS && lane == 0) prefetch_first_blobs(p, beg, end);
+    if (warp == 0) {  // the lanes of warp 0 initialise the barriers side by side
+        for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
+        for (int s = lane; s < p.slots; s += 32) {
             mbar_init(&bars.empty_w[s], 4);  // the k-block's 4 dequant warps (one per lane quarter)
             mbar_init(&bars.empty_a[s], 1);  // the owning issuer
         }
-        for (int a = 0; a < kASlotsS; ++a) {
-            mbar_init(&bars.afull[a][0], 4);
-            mbar_init(&bars.aempty[a], 1);
+        if (lane < kASlotsS) {
+            mbar_init(&bars.afull[lane][0], 4);
+            mbar_init(&bars.aempty[lane], 1);
         }
-        for (int q = 0; q < kMaxIssuers; ++q) {
-            mbar_init(&bars.drain[q], 1);
-            mbar_init(&bars.pfull[q], 1);
-            mbar_init(&bars.pempty[q], 4);
+        if (lane < kMaxIssuers) {
+            mbar_init(&bars.drain[lane], 1);
+            mbar_init(&bars.pfull[lane], 1);
+            mbar_init(&bars.pempty[lane], 4);
         }
-        abort_flag = 0;
+        if (lane == 0) abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == kIssuerWarp0S) {
@@ -920,8 +988,6 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     const uint32_t tmem = tmem_slot;
 
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
-    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
-    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
 
     if (warp < kDqWarpsS) {
         dequant_role_small<MODE>(p, wring, bars, tmem, ctl, beg, end);

@@ -46,6 +46,12 @@ def unit_start(c, units, grid):
     return c * units // grid
 
 
+def first_contributor(tbase, units, grid):
+    """The CTA holding unit `tbase` (a tile's first unit): the smallest c with
+    unit_start(c + 1) > tbase, in closed form."""
+    return ((tbase + 1) * grid + units - 1) // units - 1
+
+
 def segments(beg, end, kbs):
     it = end - 1
     while it >= beg:
@@ -118,21 +124,17 @@ def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
     def acc(quarter, parity):
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
+                # the two parities of a quarter swap halves, then all 8 warps run the epilogue
                 yield ("nbar", f"comb{quarter}", 2)
-                if parity == 0:
-                    tile, kb_lo, kb_hi, owner, whole = seg
-                    if not owner:
-                        yield ("nbar", "epi", 4)
-                        if quarter == 0:
-                            yield ("flag_set", cta)
-                    elif not whole:
-                        cc = cta - 1
-                        while cc >= 0:
-                            yield ("flag_wait", cc)
-                            if unit_start(cc, units, grid) <= tile * kbs:
-                                break
-                            cc -= 1
-                        yield ("nbar", "epi", 4)
+                tile, kb_lo, kb_hi, owner, whole = seg
+                if not owner:
+                    yield ("nbar", "epi", 8)
+                    if quarter == 0 and parity == 0:
+                        yield ("flag_set", cta)
+                elif not whole:
+                    for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                        yield ("flag_wait", cc)
+                    yield ("nbar", "epi", 8)
                 continue
             if acc_in_ring:  # an earlier protocol: the accumulate warps read scales from the ring
                 if not has(it0, c, 2, parity):

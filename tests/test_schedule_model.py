@@ -42,13 +42,14 @@ def test_model_catches_slot_indexed_barrier_hazard():
             # the phase parity is the slot's use count
             yield seg, pos, c, it0, pos + sm.NCB * uses[pos]
             uses[pos] += 1
+    import random
     sm.chunks = slot_indexed
     try:
         units, grid, kbs = _plan(8192, 10240)
-        assert simulate(units, grid, kbs, 4, 17, acc_in_ring=True)
+        assert simulate(units, grid, kbs, 4, 17, acc_in_ring=True, rng=random.Random(0))
     finally:
         sm.chunks = orig
-    assert not simulate(units, grid, kbs, 4, 17, acc_in_ring=True)
+    assert not simulate(units, grid, kbs, 4, 17, acc_in_ring=True, rng=random.Random(0))
 
 
 class _Biased:
@@ -92,15 +93,39 @@ def test_no_alias_or_deadlock_under_skewed_schedules(K, N, slots):
 def test_model_catches_period_mismatch():
     # an earlier protocol had 3 dequant warps per lane quarter and 6 A slots against 4 issuers:
     # an issuer could wait on A slot (i mod 6) two phases early and pass on the parity of an
-    # older phase. Enough skew (accumulate warps always first) makes it happen on the
-    # 8192 x 57344 layer with a 9-slot ring; the GPU showed it as expired waits.
+    # older phase. Skewed interleavings make it happen on the 8192 x 57344 layer with a 9-slot
+    # ring; the GPU showed it as expired waits. The current periods never alias.
     import schedule_model as sm
     units, grid, kbs = _plan(8192, 57344)
+
+    def aliases():
+        found = []
+        for name, first in _BIASES.items():
+            for cta in (0, 1, 5):
+                found += [p for p in simulate(units, grid, kbs, 4, 9, rng=_Biased(first, cta), ctas_only=[cta])
+                          if p[0] == "alias"]
+        return found
     saved = sm.NA, sm.DQ_PERIOD
     sm.NA, sm.DQ_PERIOD = 6, 3
     try:
-        problems = simulate(units, grid, kbs, 4, 9, rng=_Biased(_BIASES["acc-first"], 0), ctas_only=[0])
+        old = aliases()
     finally:
         sm.NA, sm.DQ_PERIOD = saved
-    assert any(p[0] == "alias" and p[3].startswith("afull") for p in problems)
-    assert not simulate(units, grid, kbs, 4, 9, rng=_Biased(_BIASES["acc-first"], 0), ctas_only=[0])
+    assert any(p[3].startswith("afull") for p in old)
+    assert not aliases()
+
+
+def test_first_contributor_closed_form():
+    # the owner finds the CTA holding its tile's first unit in closed form; it must be the CTA
+    # whose range [unit_start(c), unit_start(c + 1)) contains that unit
+    import random
+    from schedule_model import first_contributor, unit_start
+    r = random.Random(3)
+    cases = [(units, grid) for units in (1, 7, 148, 149, 1024, 5504, 28672, 200000) for grid in (1, 3, 148)]
+    cases += [(r.randint(1, 10 ** 6), r.randint(1, 148)) for _ in range(200)]
+    for units, grid in cases:
+        grid = min(grid, units)
+        for t in {0, units - 1, units // 2, r.randrange(units)}:
+            c = first_contributor(t, units, grid)
+            assert 0 <= c < grid
+            assert unit_start(c, units, grid) <= t < unit_start(c + 1, units, grid), (units, grid, t, c)
