@@ -60,8 +60,6 @@ struct Barriers {
     uint64_t aempty[kASlotsS];     // MMAs done with a tensor-memory slot
     uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
     uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
-    uint64_t pfull[kMaxIssuers];   // small tiles: an issuer's per-k-block partial is ready (commit)
-    uint64_t pempty[kMaxIssuers];  // small tiles: the accumulate warps have read it (4 warps)
 };
 
 struct Ctl {
@@ -492,360 +490,6 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
     wait_bar(&b.drain[q], 0, ctl, false);
 }
 
-// ------------------------------------------------------------------ small tiles
-// Roles of the small-tile design split the walk's k-blocks round-robin: a role with period R
-// and residue r handles the k-blocks whose walk index is r mod R. All roles still follow every
-// chunk (to keep the full barriers' phases) but wait only for chunks holding one of theirs.
-__device__ __forceinline__ bool chunk_has(uint32_t iter0, int c, uint32_t period, uint32_t residue) {
-    return ((residue + period - iter0 % period) % period) < static_cast<uint32_t>(c);
-}
-
-// Dequant warp of a small tile: lane quarter = warp % 4, residue = warp / 4 (period 2). It turns
-// all 16 packed words of its row of a k-block into 128 fp16 (or int8) values and stores them
-// into tensor-memory slot (walk index mod 4), where they are the MMA's A operand.
-//
-// Every mbarrier is waited on with a parity bit, so a waiter must never run two phases ahead
-// of the barrier. The periods are chosen so that each barrier has fixed participants that see
-// all of its phases in order: A slot a (walk index = a mod 4) is always written by residue
-// group a % 2 and always read by issuer a, and partial buffer q is always read by the
-// accumulate warps of parity q % 2.
-template <int MODE>
-__device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
-                                   const Ctl& ctl, long long beg, long long end) {
-    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3;
-    const uint32_t residue = static_cast<uint32_t>(warp >> 2);
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool scaled = (MODE == kModeGroup) && p.scale_in_dequant;
-    uint32_t ch = 0, iter = 0;
-    int pos = 0;
-    SegCursor seg(beg, end, p.k_blocks);
-    while (seg.next()) {
-        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
-            if (chunk_has(iter, c, 2, residue)) {
-                bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
-                for (int t = 0; t < c; ++t) {
-                    const uint32_t i = iter + t;
-                    if ((i & 1u) != residue) continue;
-                    const int s = pos + t;
-                    const uint32_t a = i % kASlotsS, aph = (i / kASlotsS) & 1;
-                    uint4 w[4];
-                    uint16_t sc[4] = {0, 0, 0, 0};
-                    if (ok) {
-                        const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
-                        const uint4* words = reinterpret_cast<const uint4*>(blob);
-#pragma unroll
-                        for (int hv = 0; hv < 4; ++hv) w[hv] = words[hv * kTileN + row];
-                        if (scaled) {
-                            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
-#pragma unroll
-                            for (int hv = 0; hv < 4; ++hv) sc[hv] = scs[((32 * hv) / p.group_rows) * kTileN + row];
-                        }
-                    }
-                    __syncwarp();
-                    if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);
-                    if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[a], aph ^ 1, ctl));
-                    if (ok) {
-                        const uint32_t taddr = tmem + lane_base + kTmemAOffsetS + a * kSlotCols;
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t wv[8] = {w[2 * h].x,     w[2 * h].y,     w[2 * h].z,     w[2 * h].w,
-                                                    w[2 * h + 1].x, w[2 * h + 1].y, w[2 * h + 1].z, w[2 * h + 1].w};
-                            if (MODE == kModeW4A8) {
-                                uint32_t out[16];
-#pragma unroll
-                                for (int k = 0; k < 8; ++k) dequant_word_i8(wv[k], out + 2 * k);
-                                tmem_st_x16(taddr + h * 16, out);
-                            } else {
-                                uint32_t out[32];
-                                const __half2 s0 = __half2half2(__ushort_as_half(sc[2 * h]));
-                                const __half2 s1 = __half2half2(__ushort_as_half(sc[2 * h + 1]));
-#pragma unroll
-                                for (int k = 0; k < 8; ++k) dequant_word_f16(wv[k], k < 4 ? s0 : s1, scaled, out + 4 * k);
-                                tmem_st_x32(taddr + h * 32, out);
-                            }
-                        }
-                        tmem_st_wait();
-                        tc_fence_before();
-                    }
-                    __syncwarp();
-                    if (ok && lane == 0) mbar_arrive(&b.afull[a][0]);
-                }
-            }
-            iter += c;
-            kb += c;
-            pos += c;
-            if (pos == p.slots) pos = 0;
-        }
-    }
-}
-
-// Issuer q of a small tile: every k-block whose walk index is q mod 4 is its own; it waits for
-// the k-block's activations (full), its dequantised weights (A slot) and for the accumulate
-// warps to have read its previous partial, then writes the k-block's product into its partial
-// buffer with a fresh accumulation.
-template <int MODE, int TM>
-__device__ void issuer_role_small(int q, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
-                                  const Ctl& ctl, long long beg, long long end) {
-    constexpr int kSteps = (MODE == kModeW4A8) ? 4 : 8;
-    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
-    const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, TM) : idesc_f16_f32(kTileN, TM);
-    const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * TM);
-    const uint32_t a_base = smem_addr(aring);
-    uint32_t ch = 0, iter = 0, j = 0;
-    int pos = 0;
-    bool ok = true;
-    SegCursor seg(beg, end, p.k_blocks);
-    while (seg.next()) {
-        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
-            if (chunk_has(iter, c, 4, static_cast<uint32_t>(q))) {
-                if (ok) ok = wait_bar(&b.full[fb], fpar, ctl);
-                for (int t = 0; t < c; ++t) {
-                    const uint32_t i = iter + t;
-                    if (static_cast<int>(i & 3u) != q) continue;
-                    const int s = pos + t;
-                    const uint32_t a = i % kASlotsS, aph = (i / kASlotsS) & 1;
-                    const uint32_t jp = j & 1u;
-                    ++j;
-                    if (ok) ok = wait_bar(&b.afull[a][0], aph, ctl);
-                    if (ok) ok = wait_bar(&b.pempty[q], jp ^ 1u, ctl);
-                    if (!ok) continue;
-                    tc_fence_after();
-                    const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
-                    const uint32_t a_tmem = tmem + kTmemAOffsetS + a * kSlotCols;
-#pragma unroll
-                    for (int kk = 0; kk < kSteps; ++kk) {
-                        const uint32_t boff = (MODE == kModeW4A8)
-                                                  ? static_cast<uint32_t>(kk * 32)
-                                                  : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
-                        const uint64_t bdesc = smem_desc_sw128(act + boff);
-                        if (MODE == kModeW4A8)
-                            mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
-                        else
-                            mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
-                    }
-                    tc_commit(&b.aempty[a]);
-                    tc_commit(&b.empty_a[s]);
-                    tc_commit(&b.pfull[q]);
-                }
-            }
-            iter += c;
-            kb += c;
-            pos += c;
-            if (pos == p.slots) pos = 0;
-        }
-    }
-    tc_commit(&b.drain[q]);
-    wait_bar(&b.drain[q], 0, ctl, false);
-}
-
-// Epilogue of a small tile, shared by the two accumulate parities: the warp of parity h in lane
-// quarter q holds, in lane l, the sums of output column n = tile*128 + 32q + l for the tile rows
-// h*TM/2 .. h*TM/2 + TM/2 - 1. Only rows below M are stored, published or fetched.
-//
-// A CTA that does not own the tile writes its partial rows to its workspace slot and (after
-// all 8 accumulate warps have written) releases its flag. The owner finds the contributing
-// CTAs directly (those before it whose unit range reaches into the tile), lets each lane poll
-// one contributor's flag, then adds the contributors' partials in descending CTA order with
-// several contributors' loads in flight at a time.
-template <int MODE, int TM>
-__device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM / 2], bool ok,
-                               int quarter, int lane, int half) {
-    constexpr int H = TM / 2;
-    constexpr int kBatch = (H <= 8) ? 4 : 1;  // contributors whose loads are in flight together
-    const int row = quarter * 32 + lane;
-    const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
-    const int n = nt * kTileN + row;
-    const int r0 = half * H;  // first tile row of this half
-    int live = p.M - mt * TM - r0;
-    live = live < 0 ? 0 : (live > H ? H : live);
-    const bool leader = static_cast<int>(threadIdx.x) == kAccWarp0S * 32;
-    const int me = static_cast<int>(blockIdx.x);
-    if (!seg.owner) {
-        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(me) * TM * kTileN;
-        if (ok) {
-#pragma unroll
-            for (int c = 0; c < H; ++c)
-                if (c < live) part[static_cast<size_t>(r0 + c) * kTileN + row] = v[c];
-        }
-        __threadfence();
-        named_barrier_sync(2, 256);
-        if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
-        return;
-    }
-    int c_last = me;  // contributors are CTAs c_last .. me - 1
-    if (!seg.whole) {
-        // the CTA holding the tile's first unit: the smallest c with unit_start(c + 1) > tbase
-        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
-        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
-        const int ncontrib = me - c_last;
-        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
-            bool good = true;
-            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
-            ok = __all_sync(0xffffffffu, good) && ok;
-        }
-        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
-        if (ok && live > 0) {
-            for (int j = 0; j < ncontrib; j += kBatch) {
-                uint32_t w[kBatch][H];
-#pragma unroll
-                for (int b = 0; b < kBatch; ++b) {
-                    const uint32_t* part =
-                        reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
-#pragma unroll
-                    for (int c = 0; c < H; ++c)
-                        w[b][c] = (j + b < ncontrib && c < live) ? __ldcg(part + static_cast<size_t>(r0 + c) * kTileN + row) : 0u;
-                }
-#pragma unroll
-                for (int b = 0; b < kBatch; ++b) {
-                    if (j + b < ncontrib) {
-#pragma unroll
-                        for (int c = 0; c < H; ++c) {
-                            if (MODE == kModeW4A8)
-                                v[c] = static_cast<uint32_t>(static_cast<int32_t>(v[c]) + static_cast<int32_t>(w[b][c]));
-                            else
-                                v[c] = __float_as_uint(__uint_as_float(v[c]) + __uint_as_float(w[b][c]));
-                        }
-                    }
-                }
-            }
-        }
-    }
-    if (ok && n < p.N) {
-        float s_col = 1.0f, sw_col = 0.0f;
-        if (MODE == kModeChannel) s_col = __half2float(__ushort_as_half(p.s_chan[n]));
-        if (MODE == kModeW4A8) sw_col = p.sw[n];
-#pragma unroll
-        for (int c = 0; c < H; ++c) {
-            if (c < live) {
-                const int m = mt * TM + r0 + c;
-                const size_t o = static_cast<size_t>(m) * p.N + n;
-                float y;
-                if (MODE == kModeW4A8) {
-                    const int32_t a = static_cast<int32_t>(v[c]) >> 4;
-                    if (p.acc_out) p.acc_out[o] = a;
-                    const float t = static_cast<float>(a) * p.sa[m];
-                    y = t * sw_col;
-                } else if (MODE == kModeChannel) {
-                    y = __uint_as_float(v[c]) * s_col;
-                } else {
-                    y = __uint_as_float(v[c]);
-                }
-                p.y[o] = __half_as_ushort(__float2half_rn(y));
-            }
-        }
-    }
-    if (!seg.whole) {
-        named_barrier_sync(2, 256);  // every accumulate warp has read the partials
-        if (leader)
-            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
-    }
-}
-
-// Accumulate warp of a small tile: lane quarter = warp % 4, parity = which k-blocks (walk index
-// mod 2) it adds. Each k-block's partial is added in k order into fp32 (or int32) registers,
-// with the k-block's group scale applied when the dequant did not. At the end of a segment the
-// two parity warps of a quarter swap halves of their sums through shared memory (double-
-// buffered by segment): each then holds the complete sums of half of the tile rows (even +
-// odd, a fixed order) and runs the epilogue for them.
-template <int MODE, int TM>
-__device__ void accum_role_small(const GemmArgs& p, uint32_t* cbuf, Barriers& b, uint32_t tmem,
-                                 const Ctl& ctl, long long beg, long long end) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3;  // a warp may only touch tensor-memory lanes 32*(warp % 4) .. +31
-    const uint32_t parity = static_cast<uint32_t>((warp - kAccWarp0S) >> 2);
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool scale_here = (MODE == kModeGroup) && !p.scale_in_dequant;
-    uint32_t iter = 0;
-    int seg_index = 0;
-    bool ok = true;
-    SegCursor seg(beg, end, p.k_blocks);
-    while (seg.next()) {
-        uint32_t acc[TM];
-#pragma unroll
-        for (int c = 0; c < TM; ++c) acc[c] = 0;  // +0.0f and int 0 share the bit pattern
-        // the group scale of this column for k-block kb of the tile: read from the prepacked
-        // blob in global memory (it is L2-resident: the blob was just streamed), so these warps
-        // never hold a shared-memory ring slot
-        const int nt = seg.tile / p.m_tiles;
-        const uint8_t* tile_blobs = p.wp + static_cast<size_t>(nt) * p.k_blocks * p.blob_bytes + kCodeBytes + 2 * row;
-        for (int kb = seg.kb_lo; kb <= seg.kb_hi; ++kb, ++iter) {
-            if ((iter & 1u) != parity) continue;
-            const uint32_t q = iter & 3u, ph = (iter >> 2) & 1u;
-            uint16_t sraw = 0;
-            if (scale_here)  // issued before the wait, consumed after it
-                sraw = __ldg(reinterpret_cast<const uint16_t*>(tile_blobs + static_cast<size_t>(kb) * p.blob_bytes));
-            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.pfull[q], ph, ctl));
-            if (!ok) continue;
-            const float sc = scale_here ? __half2float(__ushort_as_half(sraw)) : 1.0f;
-            tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < TM; c0 += 16) {  // 16 columns at a time keeps registers low
-                uint32_t v[16];
-                tmem_ld_x16(tmem + lane_base + q * TM + static_cast<uint32_t>(c0), v);
-                tmem_ld_wait();
-                if (c0 + 16 >= TM) {  // every column read: hand the partial buffer back
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&b.pempty[q]);
-                }
-#pragma unroll
-                for (int c2 = 0; c2 < 16; ++c2) {
-                    if (MODE == kModeW4A8)
-                        acc[c0 + c2] =
-                            static_cast<uint32_t>(static_cast<int32_t>(acc[c0 + c2]) + static_cast<int32_t>(v[c2]));
-                    else
-                        acc[c0 + c2] =
-                            __float_as_uint(fmaf(sc, __uint_as_float(v[c2]), __uint_as_float(acc[c0 + c2])));
-                }
-            }
-        }
-        // the two parities of this quarter exchange halves: parity h keeps tile rows h*TM/2 ..
-        // and adds the other parity's sums for them (even + odd, a fixed order)
-        constexpr int H = TM / 2;
-        uint32_t* buf = cbuf + (static_cast<size_t>(seg_index & 1) * 4 + quarter) * (32 * TM);
-        const int mt = seg.tile % p.m_tiles;
-        const int live = p.M - mt * TM;  // tile rows below M
-        uint32_t v[H];
-        if (parity == 0) {
-#pragma unroll
-            for (int c = 0; c < H; ++c)
-                if (H + c < live) buf[(H + c) * 32 + lane] = acc[H + c];
-            named_barrier_sync(3 + quarter, 64);
-#pragma unroll
-            for (int c = 0; c < H; ++c) {
-                const uint32_t o = (c < live) ? buf[c * 32 + lane] : 0u;
-                v[c] = (MODE == kModeW4A8)
-                           ? static_cast<uint32_t>(static_cast<int32_t>(acc[c]) + static_cast<int32_t>(o))
-                           : __float_as_uint(__uint_as_float(acc[c]) + __uint_as_float(o));
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < H; ++c)
-                if (c < live) buf[c * 32 + lane] = acc[c];
-            named_barrier_sync(3 + quarter, 64);
-#pragma unroll
-            for (int c = 0; c < H; ++c) {
-                const uint32_t e = (H + c < live) ? buf[(H + c) * 32 + lane] : 0u;
-                v[c] = (MODE == kModeW4A8)
-                           ? static_cast<uint32_t>(static_cast<int32_t>(e) + static_cast<int32_t>(acc[H + c]))
-                           : __float_as_uint(__uint_as_float(e) + __uint_as_float(acc[H + c]));
-            }
-        }
-        epilogue_small<MODE, TM>(p, ctl, seg, v, ok && !*ctl.abort_flag, quarter, lane, static_cast<int>(parity));
-        ++seg_index;
-    }
-}
-
 // ------------------------------------------------------------------ kernels
 __device__ __forceinline__ uint8_t* align_ring(uint8_t* smem_dyn) {
     const uint32_t raw = smem_addr(smem_dyn);
@@ -935,12 +579,375 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     }
 }
 
-// The small-tile protocol relies on A slot a being written by one residue group and read by one
-// issuer (period 2 dequant, period 4 issue, 4 slots) and on the A slots fitting in tensor memory
-// beside the 4 partial buffers.
-static_assert(kDqWarpsS == 8 && kASlotsS == kMaxIssuers && kMaxIssuers == 4, "small-tile periods");
+// ------------------------------------------------------------------ small tiles
+// Small tiles (at most 32 rows of A) split the walk's k-blocks round-robin over 4 residues: walk
+// index i belongs to residue r = i mod 4. Residue r owns one dequantised A slot and one partial
+// buffer in tensor memory, one MMA issuer and one dequant warp per lane quarter; so every
+// mbarrier has fixed participants that see all of its phases in order (a parity wait can never
+// pass on a phase two ahead or behind).
+//
+// Per k-block i of residue r (the u-th of that residue, u = i / 4):
+//   dequant warps (4 quarters): wait for the chunk's copies (full), read the 16 code words of
+//     their column and release the ring slot (empty_w); wait until the MMAs of their previous
+//     k-block are done (aempty[r], phase u - 1): that frees A slot r and completes partial
+//     buffer r, which they add into fp32 (int32) registers with that k-block's group scale;
+//     then dequantise k-block i into A slot r and signal afull[r].
+//   issuer r: wait for the activations (full) and afull[r] (phase u), issue the 8 MMAs
+//     (K = 16 each) of the k-block into partial buffer r, commit aempty[r] and the ring slot's
+//     activation half (empty_a).
+// Reading partial r before signalling afull[r] is what keeps the next MMA from overwriting it.
+// At a segment's end each dequant warp waits for its last MMA and adds that partial too; the
+// 4 residue warps of a quarter then sum their registers through tensor memory (fixed order
+// r = 0..3) and each finishes a quarter of the tile rows in the epilogue.
+__device__ __forceinline__ bool chunk_has(uint32_t iter0, int c, uint32_t period, uint32_t residue) {
+    return ((residue + period - iter0 % period) % period) < static_cast<uint32_t>(c);
+}
+
+// Rows of the tile below M (tiles past the last full one are partly padding).
+__device__ __forceinline__ int live_rows(const GemmArgs& p, int tile, int TM) {
+    const int live = p.M - (tile % p.m_tiles) * TM;
+    return live < TM ? live : TM;
+}
+
+// Adds partial buffer r (this warp's lane quarter) into acc, the first `live` columns only.
+template <int MODE, int TM>
+__device__ __forceinline__ void add_partial(uint32_t (&acc)[TM], uint32_t paddr, float sc, int live) {
+#pragma unroll
+    for (int c0 = 0; c0 < TM; c0 += 8) {
+        if (c0 < live) {  // warp-uniform
+            uint32_t v[8];
+            tmem_ld_x8(paddr + static_cast<uint32_t>(c0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (MODE == kModeW4A8)
+                    acc[c0 + c] = static_cast<uint32_t>(static_cast<int32_t>(acc[c0 + c]) + static_cast<int32_t>(v[c]));
+                else
+                    acc[c0 + c] = __float_as_uint(fmaf(sc, __uint_as_float(v[c]), __uint_as_float(acc[c0 + c])));
+            }
+        }
+    }
+}
+
+// Epilogue of a small tile for one residue warp: lane l of the warp in lane quarter q holds in
+// v the complete sums of output column n = tile*128 + 32q + l for the tile rows r*TM/4 ..
+// r*TM/4 + TM/4 - 1. Only rows below M are stored, published or fetched.
+//
+// A CTA that does not own the tile writes its partial rows to its workspace slot and (after
+// all 16 dequant warps have written) releases its flag. The owner finds the contributing CTAs
+// directly (those before it whose unit range reaches into the tile), lets each lane poll one
+// contributor's flag, then adds the contributors' partials in descending CTA order with
+// several contributors' loads in flight at a time.
+template <int MODE, int TM>
+__device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM / 4], bool ok,
+                               int quarter, int lane, int r) {
+    constexpr int H = TM / 4;
+    constexpr int kBatch = (H <= 4) ? 4 : 2;  // contributors whose loads are in flight together
+    const int row = quarter * 32 + lane;
+    const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
+    const int n = nt * kTileN + row;
+    const int r0 = r * H;  // first tile row of this warp
+    int live = live_rows(p, seg.tile, TM) - r0;
+    live = live < 0 ? 0 : (live > H ? H : live);
+    const bool leader = threadIdx.x == 0;
+    const int me = static_cast<int>(blockIdx.x);
+    if (!seg.owner) {
+        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(me) * TM * kTileN;
+        if (ok) {
+#pragma unroll
+            for (int c = 0; c < H; ++c)
+                if (c < live) part[static_cast<size_t>(r0 + c) * kTileN + row] = v[c];
+        }
+        __threadfence();
+        named_barrier_sync(2, kDqWarpsS * 32);
+        if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
+        return;
+    }
+    int c_last = me;  // contributors are CTAs c_last .. me - 1
+    if (!seg.whole) {
+        // the CTA holding the tile's first unit: the smallest c with unit_start(c + 1) > tbase
+        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        const int ncontrib = me - c_last;
+        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
+            bool good = true;
+            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
+            ok = __all_sync(0xffffffffu, good) && ok;
+        }
+        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
+        if (ok && live > 0) {
+            for (int j = 0; j < ncontrib; j += kBatch) {
+                uint32_t w[kBatch][H];
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const uint32_t* part = reinterpret_cast<const uint32_t*>(p.ws_partial) +
+                                           static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
+#pragma unroll
+                    for (int c = 0; c < H; ++c)
+                        w[b][c] = (j + b < ncontrib && c < live)
+                                      ? __ldcg(part + static_cast<size_t>(r0 + c) * kTileN + row)
+                                      : 0u;
+                }
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    if (j + b < ncontrib) {
+#pragma unroll
+                        for (int c = 0; c < H; ++c) {
+                            if (MODE == kModeW4A8)
+                                v[c] = static_cast<uint32_t>(static_cast<int32_t>(v[c]) + static_cast<int32_t>(w[b][c]));
+                            else
+                                v[c] = __float_as_uint(__uint_as_float(v[c]) + __uint_as_float(w[b][c]));
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (ok && n < p.N) {
+        float s_col = 1.0f, sw_col = 0.0f;
+        if (MODE == kModeChannel) s_col = __half2float(__ushort_as_half(p.s_chan[n]));
+        if (MODE == kModeW4A8) sw_col = p.sw[n];
+#pragma unroll
+        for (int c = 0; c < H; ++c) {
+            if (c < live) {
+                const int m = mt * TM + r0 + c;
+                const size_t o = static_cast<size_t>(m) * p.N + n;
+                float y;
+                if (MODE == kModeW4A8) {
+                    const int32_t a = static_cast<int32_t>(v[c]) >> 4;
+                    if (p.acc_out) p.acc_out[o] = a;
+                    const float t = static_cast<float>(a) * p.sa[m];
+                    y = t * sw_col;
+                } else if (MODE == kModeChannel) {
+                    y = __uint_as_float(v[c]) * s_col;
+                } else {
+                    y = __uint_as_float(v[c]);
+                }
+                p.y[o] = __half_as_ushort(__float2half_rn(y));
+            }
+        }
+    }
+    if (!seg.whole) {
+        named_barrier_sync(2, kDqWarpsS * 32);  // every dequant warp has read the partials
+        if (leader)
+            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
+    }
+}
+
+// Dequant (and accumulate) warp of a small tile: lane quarter = warp % 4, residue r = warp / 4.
+// kScaled: the group scale multiplies the fp16 weight (g < 128); otherwise group scales
+// (g >= 128) multiply each k-block's fp32 partial as it is added.
+template <int MODE, int TM, bool kScaled>
+__device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barriers& b, uint32_t tmem,
+                                   const Ctl& ctl, long long beg, long long end) {
+    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
+    constexpr int H = TM / 4;
+    constexpr bool kScaleAtAdd = (MODE == kModeGroup) && !kScaled;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3;
+    const uint32_t r = static_cast<uint32_t>(warp >> 2);
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t slot_addr = tmem + lane_base + kTmemAOffsetS + r * kSlotCols;  // A slot r, this quarter
+    const uint32_t part_addr = tmem + lane_base + r * TM;                        // partial buffer r
+    uint32_t ch = 0, iter = 0, uses = 0;  // uses: k-blocks of residue r handed to the MMA so far
+    int pos = 0;
+    bool ok = true;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        const int live = live_rows(p, seg.tile, TM);
+        uint32_t acc[TM];
+#pragma unroll
+        for (int c = 0; c < TM; ++c) acc[c] = 0;  // +0.0f and int 0 share the bit pattern
+        bool pending = false;                      // a k-block of this segment whose partial is not added yet
+        float sc_pending = 1.0f;
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
+            ++ch;
+            if (chunk_has(iter, c, 4, r)) {
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
+                const int t = static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block in the chunk
+                const int s = pos + t;
+                // TM = 32 keeps 32 accumulators live: it reads the code words one half at a time
+                // (and so holds the ring slot until the second half is read)
+                constexpr bool kSplitLoad = TM > 16;
+                const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
+                const uint4* words = reinterpret_cast<const uint4*>(blob);
+                const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+                uint4 w[4];
+                uint16_t sc[4] = {0, 0, 0, 0};
+                uint16_t sc_add = 0;
+                if (ok) {
+#pragma unroll
+                    for (int hv = 0; hv < (kSplitLoad ? 2 : 4); ++hv) w[hv] = words[hv * kTileN + row];
+                    if (kScaled) {
+#pragma unroll
+                        for (int hv = 0; hv < 4; ++hv) sc[hv] = scs[((32 * hv) / p.group_rows) * kTileN + row];
+                    }
+                    if (kScaleAtAdd) sc_add = scs[row];
+                }
+                if (!kSplitLoad) {
+                    __syncwarp();
+                    if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);
+                }
+                // MMAs of this residue's previous k-block done: A slot r is free, partial r complete
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[r], (uses & 1u) ^ 1u, ctl));
+                if (ok) {
+                    tc_fence_after();
+                    if (pending) add_partial<MODE, TM>(acc, part_addr, sc_pending, live);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (kSplitLoad && h == 1) {
+                            w[0] = words[2 * kTileN + row];
+                            w[1] = words[3 * kTileN + row];
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&b.empty_w[s]);
+                        }
+                        const int i0 = kSplitLoad ? 0 : 2 * h;
+                        const uint32_t wv[8] = {w[i0].x,     w[i0].y,     w[i0].z,     w[i0].w,
+                                                w[i0 + 1].x, w[i0 + 1].y, w[i0 + 1].z, w[i0 + 1].w};
+                        if (MODE == kModeW4A8) {
+                            uint32_t out[16];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) dequant_word_i8(wv[k], out + 2 * k);
+                            tmem_st_x16(slot_addr + h * 16, out);
+                        } else {
+                            const __half2 s0 = __half2half2(__ushort_as_half(sc[2 * h]));
+                            const __half2 s1 = __half2half2(__ushort_as_half(sc[2 * h + 1]));
+#pragma unroll
+                            for (int q2 = 0; q2 < 2; ++q2) {  // 16 registers per store keeps the live set small
+                                uint32_t out[16];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    dequant_word_f16(wv[4 * q2 + k], q2 == 0 ? s0 : s1, kScaled, out + 4 * k);
+                                tmem_st_x16(slot_addr + h * 32 + q2 * 16, out);
+                            }
+                        }
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                } else if (kSplitLoad) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&b.empty_w[s]);  // a failed wait still releases the slot
+                }
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&b.afull[r][0]);
+                ++uses;
+                pending = true;
+                sc_pending = kScaleAtAdd ? __half2float(__ushort_as_half(sc_add)) : 1.0f;
+            }
+            iter += c;
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+        // the segment's last k-block of this residue: wait for its MMAs and add its partial
+        if (pending) {
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[r], (uses & 1u) ^ 1u, ctl));
+            if (ok) {
+                tc_fence_after();
+                add_partial<MODE, TM>(acc, part_addr, sc_pending, live);
+            }
+        }
+        // the 4 residue warps of this quarter sum their registers (r = 0..3 in order) through
+        // the partial buffers, each finishing TM/4 rows: buffer r holds no MMA result now,
+        // and none is issued into it before this warp signals its next afull
+        ok = ok && !*ctl.abort_flag;
+        if constexpr (TM == 16)
+            tmem_st_x16(part_addr, acc);
+        else
+            tmem_st_x32(part_addr, acc);
+        tmem_st_wait();
+        tc_fence_before();
+        named_barrier_sync(3 + quarter, 4 * 32);
+        tc_fence_after();
+        uint32_t v[H];
+#pragma unroll
+        for (int c = 0; c < H; ++c) v[c] = 0;
+        if (static_cast<int>(r) * H < live) {
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                uint32_t x[H];
+                if constexpr (H == 4)
+                    tmem_ld_x4(tmem + lane_base + rr * TM + r * H, x);
+                else
+                    tmem_ld_x8(tmem + lane_base + rr * TM + r * H, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < H; ++c)
+                    v[c] = (MODE == kModeW4A8)
+                               ? static_cast<uint32_t>(static_cast<int32_t>(v[c]) + static_cast<int32_t>(x[c]))
+                               : __float_as_uint(__uint_as_float(v[c]) + __uint_as_float(x[c]));
+            }
+        }
+        tc_fence_before();
+        named_barrier_sync(3 + quarter, 4 * 32);  // all reads done before any MMA refills a buffer
+        epilogue_small<MODE, TM>(p, ctl, seg, v, ok, quarter, lane, static_cast<int>(r));
+    }
+}
+
+// Issuer r of a small tile: every k-block whose walk index is r mod 4 is its own; it waits for
+// the k-block's activations (full) and its dequantised weights (A slot r), then writes the
+// k-block's product into partial buffer r with a fresh accumulation.
+template <int MODE, int TM>
+__device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
+                                  const Ctl& ctl, long long beg, long long end) {
+    constexpr int kSteps = (MODE == kModeW4A8) ? 4 : 8;
+    constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
+    const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, TM) : idesc_f16_f32(kTileN, TM);
+    const uint32_t d_tmem = tmem + static_cast<uint32_t>(r * TM);
+    const uint32_t a_tmem = tmem + kTmemAOffsetS + static_cast<uint32_t>(r * kSlotCols);
+    const uint32_t a_base = smem_addr(aring);
+    uint32_t ch = 0, iter = 0, uses = 0;
+    int pos = 0;
+    bool ok = true;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
+            ++ch;
+            if (chunk_has(iter, c, 4, static_cast<uint32_t>(r))) {
+                const int t = static_cast<int>((static_cast<uint32_t>(r) + 4 - iter % 4) % 4);
+                const int s = pos + t;
+                if (ok) ok = wait_bar(&b.full[fb], fpar, ctl);
+                if (ok) ok = wait_bar(&b.afull[r][0], uses & 1u, ctl);
+                ++uses;
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+#pragma unroll
+                    for (int kk = 0; kk < kSteps; ++kk) {
+                        const uint32_t boff = (MODE == kModeW4A8)
+                                                  ? static_cast<uint32_t>(kk * 32)
+                                                  : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
+                        const uint64_t bdesc = smem_desc_sw128(act + boff);
+                        if (MODE == kModeW4A8)
+                            mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                        else
+                            mma_f16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
+                    }
+                    tc_commit(&b.aempty[r]);
+                    tc_commit(&b.empty_a[s]);
+                }
+            }
+            iter += c;
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+    }
+    tc_commit(&b.drain[r]);
+    wait_bar(&b.drain[r], 0, ctl, false);
+}
+
+// The small-tile protocol relies on one period (4) for dequant residues, A slots, issuers and
+// partial buffers, and on the A slots fitting in tensor memory beside the partial buffers.
+static_assert(kDqWarpsS == 16 && kASlotsS == kMaxIssuers && kMaxIssuers == 4, "small-tile periods");
 static_assert(kMaxIssuers * kSmallTileMax <= kTmemAOffsetS && kTmemAOffsetS + kASlotsS * 64 <= kTmemCols,
               "small-tile tensor-memory columns");
+static_assert(kChunkBars > kMaxSlots && kMaxChunk <= 4, "one k-block per residue per chunk");
 
 template <int MODE, int TM>
 __global__ void __launch_bounds__(kThreadsSmall, 1)
@@ -952,7 +959,6 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
 
     uint8_t* aring = align_ring(smem_dyn);
     uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
-    uint32_t* cbuf = reinterpret_cast<uint32_t*>(wring + static_cast<size_t>(p.slots) * p.blob_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
@@ -962,16 +968,12 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
         for (int s = lane; s < p.slots; s += 32) {
             mbar_init(&bars.empty_w[s], 4);  // the k-block's 4 dequant warps (one per lane quarter)
-            mbar_init(&bars.empty_a[s], 1);  // the owning issuer
+            mbar_init(&bars.empty_a[s], 1);  // the k-block's issuer
         }
         if (lane < kASlotsS) {
             mbar_init(&bars.afull[lane][0], 4);
             mbar_init(&bars.aempty[lane], 1);
-        }
-        if (lane < kMaxIssuers) {
             mbar_init(&bars.drain[lane], 1);
-            mbar_init(&bars.pfull[lane], 1);
-            mbar_init(&bars.pempty[lane], 4);
         }
         if (lane == 0) abort_flag = 0;
         fence_barrier_init();
@@ -990,15 +992,20 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
 
     if (warp < kDqWarpsS) {
-        dequant_role_small<MODE>(p, wring, bars, tmem, ctl, beg, end);
+        if constexpr (MODE == kModeGroup) {
+            if (p.scale_in_dequant)
+                dequant_role_small<MODE, TM, true>(p, wring, bars, tmem, ctl, beg, end);
+            else
+                dequant_role_small<MODE, TM, false>(p, wring, bars, tmem, ctl, beg, end);
+        } else {
+            dequant_role_small<MODE, TM, false>(p, wring, bars, tmem, ctl, beg, end);
+        }
     } else if (warp < kIssuerWarp0S + kMaxIssuers) {
         if (lane == 0) issuer_role_small<MODE, TM>(warp - kIssuerWarp0S, p, aring, bars, tmem, ctl, beg, end);
     } else if (warp == kWeightWarpS) {
         if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else if (warp == kActWarpS) {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
-    } else {
-        accum_role_small<MODE, TM>(p, cbuf, bars, tmem, ctl, beg, end);
     }
 
     tc_fence_before();
@@ -1028,8 +1035,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->issuers = pl->small ? kMaxIssuers : (tm <= 64 ? 4 : (tm <= 128 ? 2 : 1));
     pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;
     pl->blob_bytes = (mode == kModeGroup) ? static_cast<int>(blob_bytes_w4a16(slots)) : kCodeBytes;
-    const int cbuf_bytes = pl->small ? 2 * 4 * 32 * tm * 4 : 0;  // accumulate warps' hand-over buffers
-    const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */ - cbuf_bytes;
+    const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */;
     int s = budget / (pl->act_slot + pl->blob_bytes);
     if (s > kMaxSlots) s = kMaxSlots;
     if (s < 2) return -1;
@@ -1038,7 +1044,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     if (c > kMaxChunk) c = kMaxChunk;
     if (c < 1) c = 1;
     pl->chunk = c;
-    pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + cbuf_bytes;
+    pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024;
     pl->units = static_cast<long long>(pl->n_tiles) * pl->m_tiles * pl->k_blocks;
     pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
     return 0;

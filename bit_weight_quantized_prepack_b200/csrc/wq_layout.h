@@ -37,15 +37,14 @@ constexpr int kWeightWarp = kIssuerWarp0 + kMaxIssuers;  // warp 12: weight-blob
 constexpr int kActWarp = kWeightWarp + 1;     // warp 13: activation-tile copies
 constexpr int kThreadsLarge = (kActWarp + 1) * 32;   // 448: epilogue runs in the dequant warps
 // small tiles (tile_m <= 32): more warps, each on its own k-blocks
-constexpr int kDqWarpsS = 8;                  // 2 per TMEM lane quarter (k-block parity)
-constexpr int kIssuerWarp0S = kDqWarpsS;      // warps 8..11
-constexpr int kWeightWarpS = kIssuerWarp0S + kMaxIssuers;  // warp 12
-constexpr int kActWarpS = kWeightWarpS + 1;   // warp 13
-constexpr int kAccWarp0S = kActWarpS + 1;     // warps 14..21: 2 per lane quarter (k-block parity)
-constexpr int kThreadsSmall = (kAccWarp0S + 8) * 32;  // 704
+constexpr int kDqWarpsS = 16;                 // 4 per TMEM lane quarter, one per k-block residue (mod 4)
+constexpr int kIssuerWarp0S = kDqWarpsS;      // warps 16..19: one MMA issuer per residue
+constexpr int kWeightWarpS = kIssuerWarp0S + kMaxIssuers;  // warp 20
+constexpr int kActWarpS = kWeightWarpS + 1;   // warp 21
+constexpr int kThreadsSmall = (kActWarpS + 1) * 32;  // 704
 constexpr int kASlotsS = 4;                   // dequantised k-blocks in tensor memory (small tiles)
 constexpr int kSmallTileMax = 32;             // tiles of at most this many rows use per-k-block partials
-constexpr int kTmemAOffsetS = 128;            // small tiles: partials in columns [0, 128), 6 A slots above
+constexpr int kTmemAOffsetS = 128;            // small tiles: partials in columns [0, 128), 4 A slots above
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
 constexpr int kMaxSlots = 32;                 // shared-memory ring slots (one k-block each)
 constexpr int kMaxChunk = 4;                  // k-blocks moved by one copy

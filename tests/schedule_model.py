@@ -3,8 +3,11 @@
 Every warp role of every CTA is a generator of barrier operations that follows the kernel's
 walk over its (tile, k-block) units: segments last-first, k-blocks forward, chunks of up to
 `chunk` k-blocks that never wrap the shared-memory ring, chunk barriers indexed by chunk
-number modulo 33, ring slots, tensor-memory A slots (4), partial buffers (4 issuers), the
-two accumulate parities (which read only the partial buffers, never the ring), the named barriers of the epilogue and the stream-K publish flags.
+number modulo 33, ring slots. Walk index i belongs to residue i mod 4: a dequant warp per
+lane quarter, tensor-memory A slot i mod 4 and MMA issuer i mod 4. The dequant warps also
+add the MMA partials (the commit that frees an A slot also completes its partial), so at a
+segment's end each waits for its last MMA; then the named barriers of the 4-way combine and of
+the epilogue, and the stream-K publish flags.
 mbarriers follow the PTX phase/parity rules: a wait on parity p passes once the phase with
 that parity has completed, i.e. while the current phase's parity differs from p.
 
@@ -15,14 +18,16 @@ deadlocks: the role would read a slot before it was written, or after it was ove
 
 `simulate` runs all roles of all CTAs until nothing can move and returns the aliased waits and
 the roles still blocked: an empty list means the protocol is sound for that launch plan and
-that interleaving.
+that interleaving. The module constants NA (A slots), DQ_PERIOD (dequant residues) and NQ
+(issuers) are all 4 in the kernel; tests change them to check that the model catches a
+mismatch.
 """
 from collections import defaultdict
 
 NCB = 33          # chunk barriers
-NA = 4            # tensor-memory A slots (slot i % 4: writer residue i % 2, reader issuer i % 4)
-NQ = 4            # MMA issuers
-DQ_PERIOD = 2     # dequant warps per lane quarter; each takes the walk indices of one residue
+NA = 4            # tensor-memory A slots: k-block i uses slot i % NA
+NQ = 4            # MMA issuers: issuer i % NQ
+DQ_PERIOD = 4     # dequant warps per lane quarter: warp (quarter, i % DQ_PERIOD)
 
 
 class Bar:
@@ -77,7 +82,7 @@ def chunks(beg, end, kbs, chunk, slots):
         yield seg, None, None, it, ch
 
 
-def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
+def _roles(cta, units, grid, kbs, chunk, slots, B):
     """Operations: ("wait", bar, need, walk index), ("arrive", bar), ("nbar", name, count),
     ("flag_set", cta), ("flag_wait", cta)."""
     beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
@@ -85,9 +90,26 @@ def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
     def has(it0, c, period, residue):
         return ((residue + period - it0 % period) % period) < c
 
-    def dq(residue):
+    def dq(quarter, residue):
+        last = None  # walk index of this residue's last k-block in the current segment
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
-            if pos is None or not has(it0, c, DQ_PERIOD, residue):
+            if pos is None:
+                if last is not None:  # the segment's last k-block of this residue: its MMAs
+                    yield ("wait", B["aempty"][last % NA], last // NA + 1, last)
+                yield ("nbar", f"comb{quarter}", DQ_PERIOD)
+                yield ("nbar", f"comb{quarter}", DQ_PERIOD)
+                tile, kb_lo, kb_hi, owner, whole = seg
+                if not owner:
+                    yield ("nbar", "epi", 4 * DQ_PERIOD)
+                    if quarter == 0 and residue == 0:
+                        yield ("flag_set", cta)
+                elif not whole:
+                    for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                        yield ("flag_wait", cc)
+                    yield ("nbar", "epi", 4 * DQ_PERIOD)
+                last = None
+                continue
+            if not has(it0, c, DQ_PERIOD, residue):
                 continue
             yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
             for t in range(c):
@@ -96,6 +118,7 @@ def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
                     yield ("arrive", B["empty_w"][pos + t])
                     yield ("wait", B["aempty"][i % NA], i // NA, i)
                     yield ("arrive", B["afull"][i % NA])
+                    last = i
 
     def issuer(q):
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
@@ -106,10 +129,8 @@ def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
                 i = it0 + t
                 if i % NQ == q:
                     yield ("wait", B["afull"][i % NA], i // NA + 1, i)
-                    yield ("wait", B["pempty"][q], i // NQ, i)
                     yield ("arrive", B["aempty"][i % NA])
                     yield ("arrive", B["empty_a"][pos + t])
-                    yield ("arrive", B["pfull"][q])
 
     def producer(which):
         uses = [0] * slots
@@ -121,46 +142,17 @@ def _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring):
                 uses[pos + t] += 1
             yield ("arrive", B["full"][ch % NCB])
 
-    def acc(quarter, parity):
-        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
-            if pos is None:
-                # the two parities of a quarter swap halves, then all 8 warps run the epilogue
-                yield ("nbar", f"comb{quarter}", 2)
-                tile, kb_lo, kb_hi, owner, whole = seg
-                if not owner:
-                    yield ("nbar", "epi", 8)
-                    if quarter == 0 and parity == 0:
-                        yield ("flag_set", cta)
-                elif not whole:
-                    for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
-                        yield ("flag_wait", cc)
-                    yield ("nbar", "epi", 8)
-                continue
-            if acc_in_ring:  # an earlier protocol: the accumulate warps read scales from the ring
-                if not has(it0, c, 2, parity):
-                    continue
-                yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
-            for t in range(c):
-                i = it0 + t
-                if i % 2 == parity:
-                    yield ("wait", B["pfull"][i % NQ], i // NQ + 1, i)
-                    yield ("arrive", B["pempty"][i % NQ])
-                    if acc_in_ring:
-                        yield ("arrive", B["empty_w"][pos + t])
-
     roles = {}
     for w in range(4 * DQ_PERIOD):
-        roles[f"dq{w}"] = dq(w >> 2)
+        roles[f"dq{w}"] = dq(w & 3, w >> 2)
     for q in range(NQ):
         roles[f"iss{q}"] = issuer(q)
     roles["prod_w"] = producer("empty_w")
     roles["prod_a"] = producer("empty_a")
-    for w in range(8):
-        roles[f"acc{w}"] = acc(w & 3, w >> 2)
     return roles
 
 
-def simulate(units, grid, kbs, chunk, slots, acc_in_ring=False, rng=None, ctas_only=None):
+def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
     """Runs the roles of the CTAs (all, or `ctas_only`) to a standstill. With `rng` the roles
     move in a random order and a random number of operations at a time (any object with
     `shuffle(list)` and `randint(a, b)` can bias the interleaving). Returns a list of problems:
@@ -172,13 +164,11 @@ def simulate(units, grid, kbs, chunk, slots, acc_in_ring=False, rng=None, ctas_o
     ctas = []
     for cta in (range(grid) if ctas_only is None else ctas_only):
         B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
-             "empty_w": [Bar(8 if acc_in_ring else 4, f"empty_w{s}") for s in range(slots)],
+             "empty_w": [Bar(4, f"empty_w{s}") for s in range(slots)],
              "empty_a": [Bar(1, f"empty_a{s}") for s in range(slots)],
              "afull": [Bar(4, f"afull{a}") for a in range(NA)],
-             "aempty": [Bar(1, f"aempty{a}") for a in range(NA)],
-             "pfull": [Bar(1, f"pfull{q}") for q in range(NQ)],
-             "pempty": [Bar(4, f"pempty{q}") for q in range(NQ)]}
-        roles = _roles(cta, units, grid, kbs, chunk, slots, B, acc_in_ring)
+             "aempty": [Bar(1, f"aempty{a}") for a in range(NA)]}
+        roles = _roles(cta, units, grid, kbs, chunk, slots, B)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
                      "nbar": defaultdict(list)})
     problems = []

@@ -26,9 +26,9 @@ def test_no_deadlock(K, N, slots):
 
 
 def test_model_catches_slot_indexed_barrier_hazard():
-    # an earlier protocol (accumulate warps reading scales from the ring) with chunk barriers
-    # indexed by ring slot deadlocks on the 8192 x 10240 layer with a 17-slot ring; the GPU
-    # showed it as an expired wait on 4 tiles. Chunk-number indexing removes it.
+    # chunk barriers indexed by ring slot (instead of chunk number) let a barrier advance two
+    # phases while a role still waits for the older one; the GPU showed it as expired waits on
+    # the 8192 x 10240 layer with a 17-slot ring. Chunk-number indexing removes it.
     import schedule_model as sm
     orig = sm.chunks
 
@@ -46,10 +46,10 @@ def test_model_catches_slot_indexed_barrier_hazard():
     sm.chunks = slot_indexed
     try:
         units, grid, kbs = _plan(8192, 10240)
-        assert simulate(units, grid, kbs, 4, 17, acc_in_ring=True, rng=random.Random(0))
+        assert simulate(units, grid, kbs, 4, 17, rng=random.Random(0))
     finally:
         sm.chunks = orig
-    assert not simulate(units, grid, kbs, 4, 17, acc_in_ring=True, rng=random.Random(0))
+    assert not simulate(units, grid, kbs, 4, 17, rng=random.Random(0))
 
 
 class _Biased:
@@ -91,10 +91,10 @@ def test_no_alias_or_deadlock_under_skewed_schedules(K, N, slots):
 
 
 def test_model_catches_period_mismatch():
-    # an earlier protocol had 3 dequant warps per lane quarter and 6 A slots against 4 issuers:
-    # an issuer could wait on A slot (i mod 6) two phases early and pass on the parity of an
-    # older phase. Skewed interleavings make it happen on the 8192 x 57344 layer with a 9-slot
-    # ring; the GPU showed it as expired waits. The current periods never alias.
+    # every barrier needs fixed participants: A slots indexed with a period (6) other than
+    # that of the dequant residues and issuers (4) let a role wait on a slot two phases early
+    # and pass on the parity of an older phase. An earlier version of the kernel had such a
+    # mismatch; the GPU showed it as expired waits on the 8192 x 57344 layer.
     import schedule_model as sm
     units, grid, kbs = _plan(8192, 57344)
 
@@ -105,13 +105,13 @@ def test_model_catches_period_mismatch():
                 found += [p for p in simulate(units, grid, kbs, 4, 9, rng=_Biased(first, cta), ctas_only=[cta])
                           if p[0] == "alias"]
         return found
-    saved = sm.NA, sm.DQ_PERIOD
-    sm.NA, sm.DQ_PERIOD = 6, 3
+    saved = sm.NA
+    sm.NA = 6
     try:
         old = aliases()
     finally:
-        sm.NA, sm.DQ_PERIOD = saved
-    assert any(p[3].startswith("afull") for p in old)
+        sm.NA = saved
+    assert any(p[3].startswith(("afull", "aempty")) for p in old)
     assert not aliases()
 
 
