@@ -12,27 +12,29 @@
 //   * One persistent CTA per SM walks a contiguous range of (tile, k-block) units (stream-K).
 //     A tile split between CTAs is finished by the CTA holding its last k-block, which adds
 //     the other CTAs' partial sums in a fixed order: results are deterministic.
-//   * Warp roles per CTA:
-//       warp 12     weight producer: one bulk copy moves up to 4 consecutive blobs (codes +
+//   * Warp roles per CTA (704 threads in both designs):
+//       warp 20     weight producer: one bulk copy moves up to 4 consecutive blobs (codes +
 //                   scales of 4 k-blocks, contiguous in HBM by construction of the prepack);
-//       warp 13     activation producer: one 3-D tensor copy moves the same k-blocks of the
+//       warp 21     activation producer: one 3-D tensor copy moves the same k-blocks of the
 //                   activation tile (128-byte swizzle, the MMA's K-major B layout);
-//       warps 0..7  dequantisation: each thread owns one weight column of the tile (one
-//                   tensor-memory lane) and half of each k-block; it turns 8 packed words into
-//                   64 fp16 (or int8) values in registers and stores them into tensor memory,
-//                   where they are the MMA's A operand: the dequantised weights never touch
-//                   shared memory;
-//       warps 8..11 MMA issuers, one accumulator each.
-//     Two ways to split the MMAs, by tile height:
-//       small tiles (tile_m <= 32, the memory-bound decode regime; 576 threads): issuer q owns
+//       warps 0..15 dequantisation: each thread owns one weight column of the tile (one
+//                   tensor-memory lane); it turns packed words into fp16 (or int8) values in
+//                   registers and stores them into tensor memory, where they are the MMA's A
+//                   operand: the dequantised weights never touch shared memory. The walk's
+//                   k-blocks are dealt round-robin to groups of these warps, so that several
+//                   k-blocks per lane quarter are in flight at once;
+//       warps 16..19 MMA issuers (one elected thread each).
+//     Two ways to split the work, by tile height:
+//       small tiles (tile_m <= 32, the memory-bound decode regime): 4 residues; issuer r owns
 //                   every fourth k-block and writes each k-block's product into a fresh
-//                   partial; warps 14..17 add the partials in k order in fp32 registers,
-//                   applying the group scale there (acc += s * P), and run the epilogue
-//                   while the other warps stream the next tile. The dequant then emits exact
-//                   (q - 8) and skips the per-weight scale multiply (for g >= 128);
-//       large tiles (448 threads): issuer q owns a quarter (or half, or all) of every
-//                   k-block's K range and accumulates the whole segment in tensor memory; the
-//                   dequant applies the scale and its warps run the epilogue.
+//                   partial in tensor memory, which the dequant warps of residue r add in fp32
+//                   registers (applying the group scale there, acc += s * P, for g >= 128, so
+//                   the dequant emits exact q - 8) before they reuse their A slot; the four
+//                   residues combine at each segment's end and run the epilogue;
+//       large tiles: 2 residues of 8 dequant warps (4 lane quarters x 2 halves of a
+//                   k-block); issuer q owns a quarter (or half, or all) of every k-block's K
+//                   range and accumulates the whole segment in tensor memory; the dequant
+//                   applies the scale and the dequant warps run the epilogue.
 //     Measured on B200: a thread issuing tcgen05.mma back to back gets one instruction per
 //     ~75-85 cycles whatever the shape, and one issuing bulk copies gets one copy per ~270 ns;
 //     several issuing warps and copies of 16-33 KB take both costs off the critical path.
@@ -195,7 +197,7 @@ __device__ __forceinline__ void dequant_word_i8(uint32_t x, uint32_t* out) {
 // ------------------------------------------------------------------ epilogue
 // Sum of the issuers' accumulators for 8 columns (fixed order), as raw 32-bit values.
 template <int MODE>
-__device__ __forceinline__ void load_acc8(uint32_t taddr, int issuers, int tile_m, uint32_t (&v)[8]) {
+__device__ __forceinline__ void load_acc8(uint32_t taddr, int issuers, int tile_m, uint32_t* v) {
     tmem_ld_x8(taddr, v);
     for (int q = 1; q < issuers; ++q) {
         uint32_t w[8];
@@ -214,13 +216,17 @@ __device__ __forceinline__ void load_acc8(uint32_t taddr, int issuers, int tile_
 
 template <int MODE>
 __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ctl& ctl, const SegCursor& seg,
-                         int seg_index, int half, int quarter, int lane) {
+                         int seg_index, int part, int quarter, int lane) {
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
     const int n = nt * kTileN + row;
-    const int cols = p.tile_m >> 1;
-    const int c_begin = half * cols;
+    // the 4 dequant warps of a lane quarter split the tile rows in runs of a multiple of 8
+    // (tile_m is a multiple of 16, so every run is too; the last may be short or empty)
+    const int cols_per = ((p.tile_m / 4 + 7) / 8) * 8;
+    const int c_begin = part * cols_per;
+    int cols = p.tile_m - c_begin;
+    cols = cols < 0 ? 0 : (cols > cols_per ? cols_per : cols);
     const int m_base = mt * p.tile_m + c_begin;
 
     bool ok = __all_sync(0xffffffffu, wait_bar(&b.dfull, seg_index & 1, ctl));
@@ -238,23 +244,28 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
             }
         }
         __threadfence();
-        named_barrier_sync(1, kNumDqWarps * 32);
+        tc_fence_before();
+        named_barrier_sync(1, kNumDqWarps * 32);  // also: every warp has read the accumulators
         if (threadIdx.x == 0 && ok && !*ctl.abort_flag && static_cast<int>(blockIdx.x) != p.skip_publish)
             st_release_gpu(&p.ws_flags[blockIdx.x], 1);
         return;
     }
 
-    // owner: wait for the CTAs that hold the tile's lower k-blocks, nearest first
-    const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
-    const int c_first = static_cast<int>(blockIdx.x) - 1;
-    int c_last = c_first + 1;  // lowest contributing CTA index; c_first + 1 means none
+    // owner: the contributing CTAs are those before it whose unit range reaches into the tile
+    // (closed form: the CTA holding the tile's first unit is the smallest c with
+    // unit_start(c + 1) > tbase); each lane polls one contributor's flag
+    const int me = static_cast<int>(blockIdx.x);
+    int c_last = me;  // contributors are CTAs c_last .. me - 1
     if (!seg.whole) {
-        for (int c = c_first; c >= 0; --c) {
-            c_last = c;
-            if (ok) ok = wait_flag(&p.ws_flags[c], ctl);
-            if (unit_start(c, p.units, p.grid) <= tbase) break;
+        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        const int ncontrib = me - c_last;
+        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
+            bool good = true;
+            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
+            ok = __all_sync(0xffffffffu, good) && ok;
         }
-        ok = __all_sync(0xffffffffu, ok);
+        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
     }
 
     float s_col = 1.0f;
@@ -262,27 +273,32 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
     float sw_col = 0.0f;
     if (MODE == kModeW4A8) sw_col = n < p.N ? p.sw[n] : 0.0f;
 
-    for (int c = 0; c < cols; c += 8) {
-        uint32_t v[8];
-        if (!ok) continue;
+    // 16 columns at a time: the 16 loads of a contributor's partial are in flight together
+    for (int c = 0; c < cols && ok; c += 16) {
+        uint32_t v[16];
+        const bool two = c + 8 < cols;
         load_acc8<MODE>(tmem + lane_base + static_cast<uint32_t>(c_begin + c), p.issuers, p.tile_m, v);
-        for (int cc = c_first; cc >= c_last; --cc) {
+        if (two) load_acc8<MODE>(tmem + lane_base + static_cast<uint32_t>(c_begin + c + 8), p.issuers, p.tile_m, v + 8);
+        for (int cc = me - 1; cc >= c_last; --cc) {
             const uint32_t* part =
                 reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(cc) * p.tile_m * kTileN;
+            uint32_t w[16];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t q = __ldcg(part + static_cast<size_t>(c_begin + c + j) * kTileN + row);
+            for (int j = 0; j < 16; ++j)
+                w[j] = (j < 8 || two) ? __ldcg(part + static_cast<size_t>(c_begin + c + j) * kTileN + row) : 0u;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
                 if (MODE == kModeW4A8)
-                    v[j] = static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(q));
+                    v[j] = static_cast<uint32_t>(static_cast<int32_t>(v[j]) + static_cast<int32_t>(w[j]));
                 else
-                    v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(q));
+                    v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(w[j]));
             }
         }
         if (n < p.N) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const int m = m_base + c + j;
-                if (m < p.M) {
+                if ((j < 8 || two) && m < p.M) {
                     const size_t o = static_cast<size_t>(m) * p.N + n;
                     float y;
                     if (MODE == kModeW4A8) {
@@ -300,11 +316,12 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
             }
         }
     }
-    if (!seg.whole) {
-        named_barrier_sync(1, kNumDqWarps * 32);
-        if (threadIdx.x == 0)
-            for (int cc = c_first; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
-    }
+    // every dequant warp has read the accumulators (and the partials): only then may one of
+    // them hand the next segment's first k-block to the MMA, which overwrites the accumulators
+    tc_fence_before();
+    named_barrier_sync(1, kNumDqWarps * 32);
+    if (!seg.whole && threadIdx.x == 0)
+        for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
 }
 
 // ------------------------------------------------------------------ roles
@@ -313,7 +330,8 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
                              long long beg, long long end) {
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3, half = warp >> 2;
+    const int quarter = warp & 3, half = (warp >> 2) & 1;
+    const uint32_t residue = static_cast<uint32_t>(warp >> 3);  // this group's k-blocks: walk index mod 2
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int u0 = (64 * half) / p.group_rows, u1 = (64 * half + 32) / p.group_rows;
@@ -323,9 +341,12 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            bool ok = __all_sync(0xffffffffu, wait_bar(&b.full[chunk_bar(ch)], chunk_parity(ch), ctl));
+            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
             ++ch;
+            const bool mine = ((residue + kDqResidues - iter % kDqResidues) % kDqResidues) < static_cast<uint32_t>(c);
+            bool ok = !mine || __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
             for (int t = 0; t < c; ++t, ++iter) {
+                if (iter % kDqResidues != residue) continue;
                 const int s = pos + t;
                 const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
                 uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
@@ -375,7 +396,7 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
             pos += c;
             if (pos == p.slots) pos = 0;
         }
-        epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, half, quarter, lane);
+        epilogue<MODE>(p, b, tmem, ctl, seg, seg_index, static_cast<int>(residue) * 2 + half, quarter, lane);
         ++seg_index;
     }
 }
@@ -531,7 +552,7 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
     if (warp == 0) {  // the lanes of warp 0 initialise the barriers side by side
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
         for (int s = lane; s < p.slots; s += 32) {
-            mbar_init(&bars.empty_w[s], kNumDqWarps);
+            mbar_init(&bars.empty_w[s], kNumDqWarps / kDqResidues);  // the k-block's dequant group
             mbar_init(&bars.empty_a[s], p.issuers);
         }
         if (lane < kASlots) {

@@ -30,12 +30,13 @@ namespace wq {
 constexpr int kTileN = 128;                   // weight columns per tile = tcgen05 M extent
 constexpr int kTileK = 128;                   // weight rows per k-block = one pipeline stage
 constexpr int kCodeBytes = kTileN * kTileK / 2;  // 8192 bytes of 4-bit codes per blob
-constexpr int kNumDqWarps = 8;                // dequant warps (2 per TMEM lane quarter)
+constexpr int kDqResidues = 2;                // large tiles: k-blocks alternate between 2 dequant groups
+constexpr int kNumDqWarps = 8 * kDqResidues;  // per group: 4 lane quarters x 2 halves of a k-block
 constexpr int kMaxIssuers = 4;                // MMA-issuing warps, one accumulator each
-constexpr int kIssuerWarp0 = kNumDqWarps;     // warps 8..11
-constexpr int kWeightWarp = kIssuerWarp0 + kMaxIssuers;  // warp 12: weight-blob copies
-constexpr int kActWarp = kWeightWarp + 1;     // warp 13: activation-tile copies
-constexpr int kThreadsLarge = (kActWarp + 1) * 32;   // 448: epilogue runs in the dequant warps
+constexpr int kIssuerWarp0 = kNumDqWarps;     // warps 16..19
+constexpr int kWeightWarp = kIssuerWarp0 + kMaxIssuers;  // warp 20: weight-blob copies
+constexpr int kActWarp = kWeightWarp + 1;     // warp 21: activation-tile copies
+constexpr int kThreadsLarge = (kActWarp + 1) * 32;   // 704: epilogue runs in the dequant warps
 // small tiles (tile_m <= 32): more warps, each on its own k-blocks
 constexpr int kDqWarpsS = 16;                 // 4 per TMEM lane quarter, one per k-block residue (mod 4)
 constexpr int kIssuerWarp0S = kDqWarpsS;      // warps 16..19: one MMA issuer per residue
