@@ -410,6 +410,11 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
     uint32_t first_pass_chunks = 0xffffffffu;  // chunks before the ring first wraps
     int pos = 0;
     bool ok = true;
+    // A preceding kernel of the stream may still be writing the activations or the prepacked
+    // weights: nothing is copied before it has completed. Everything else in the CTA that
+    // reads or writes memory shared with it (the partials, flags and Y) comes after these
+    // copies.
+    griddep_wait();
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
@@ -518,8 +523,10 @@ __device__ __forceinline__ uint8_t* align_ring(uint8_t* smem_dyn) {
 }
 
 // Number of weight blobs each CTA asks L2 to prefetch at kernel entry: HBM starts streaming
-// the first k-blocks while the CTA initialises barriers and tensor memory.
-constexpr int kPrefetchBlobs = 8;
+// the first k-blocks while the CTA initialises barriers and tensor memory, and, when the
+// kernel was launched early behind another one of the stream, while that one finishes.
+// (A prefetch only fills L2, the point of coherence: it cannot observe stale data.)
+constexpr int kPrefetchBlobs = 24;
 
 __device__ void prefetch_first_blobs(const GemmArgs& p, long long beg, long long end) {
     SegCursor seg(beg, end, p.k_blocks);
@@ -548,6 +555,7 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
 
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+    if (threadIdx.x == 0) griddep_launch_dependents();
     if (warp == kWeightWarp && lane == 0) prefetch_first_blobs(p, beg, end);
     if (warp == 0) {  // the lanes of warp 0 initialise the barriers side by side
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
@@ -984,6 +992,7 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
 
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+    if (threadIdx.x == 0) griddep_launch_dependents();
     if (warp == kWeightWarpS && lane == 0) prefetch_first_blobs(p, beg, end);
     if (warp == 0) {  // the lanes of warp 0 initialise the barriers side by side
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
@@ -1097,11 +1106,13 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
     cfg.blockDim = dim3(static_cast<unsigned>(plan.threads));
     cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem_bytes);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the stream-K waits always end
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start before the
+    attr[1].val.programmaticStreamSerializationAllowed = 1;           // previous kernel ends
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k, maps, args);
 }
 

@@ -84,6 +84,14 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
+// Programmatic dependent launch. launch_dependents lets the next kernel of the stream start
+// (its CTAs still need free SMs); wait blocks until every grid this one depends on has
+// completed and its memory writes are visible. Without a dependency both return at once.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Prefetch `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2, no completion.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
