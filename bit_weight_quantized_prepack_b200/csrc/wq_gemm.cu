@@ -76,9 +76,10 @@ __device__ __forceinline__ void raise_error(const Ctl& c, int code) {
 }
 
 // Bounded wait on an mbarrier phase. Returns false when the CTA aborts or the limit expires.
-// Each poll lets the thread sleep in hardware until the phase completes (up to 20 us), so
-// waiting warps do not take issue slots or ALU cycles from the dequantising warps.
-__device__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c, bool honour_abort = true) {
+// The common case (phase already complete) is one inline non-blocking test; otherwise each
+// poll lets the thread sleep in hardware until the phase completes (up to 20 us), so waiting
+// warps do not take issue slots or ALU cycles from the dequantising warps.
+__device__ __forceinline__ bool wait_bar_slow(uint64_t* bar, uint32_t parity, const Ctl& c, bool honour_abort) {
     constexpr uint32_t kSuspendNs = 20000;
     if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
     const uint64_t t0 = global_timer_ns();
@@ -90,6 +91,11 @@ __device__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c, bool hono
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Ctl& c, bool honour_abort = true) {
+    if (mbar_test_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, c, honour_abort);
 }
 
 // Bounded wait for a stream-K publish flag written by another CTA.
@@ -153,6 +159,17 @@ __device__ __forceinline__ int chunk_len(int chunk, int kb, int kb_hi, int pos, 
 // barrier two phases ahead (a slot-indexed barrier could, when chunk boundaries shift).
 __device__ __forceinline__ uint32_t chunk_bar(uint32_t ch) { return ch % kChunkBars; }
 __device__ __forceinline__ uint32_t chunk_parity(uint32_t ch) { return (ch / kChunkBars) & 1u; }
+
+// The same two numbers kept incrementally along the walk (no division per chunk).
+struct ChunkBar {
+    uint32_t bar = 0, parity = 0;
+    __device__ __forceinline__ void next() {
+        if (++bar == static_cast<uint32_t>(kChunkBars)) {
+            bar = 0;
+            parity ^= 1u;
+        }
+    }
+};
 
 // ------------------------------------------------------------------ dequantisation
 // fp16 constants from the binary16 format: 0x6400 = 1024 (exponent field 25, so the 10
@@ -335,14 +352,15 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int u0 = (64 * half) / p.group_rows, u1 = (64 * half + 32) / p.group_rows;
-    uint32_t ch = 0, iter = 0;
+    ChunkBar cb;
+    uint32_t iter = 0;
     int pos = 0, seg_index = 0;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
+            const uint32_t fb = cb.bar, fpar = cb.parity;
+            cb.next();
             const bool mine = ((residue + kDqResidues - iter % kDqResidues) % kDqResidues) < static_cast<uint32_t>(c);
             bool ok = !mine || __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
             for (int t = 0; t < c; ++t, ++iter) {
@@ -407,6 +425,7 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                               const Ctl& ctl, long long beg, long long end) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
     uint32_t ebits = 0, ch = 0, armed = 0;
+    ChunkBar cb;
     uint32_t first_pass_chunks = 0xffffffffu;  // chunks before the ring first wraps
     int pos = 0;
     bool ok = true;
@@ -428,19 +447,21 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                 ebits ^= 1u << s;
             }
             if (ok) {
+                uint64_t* fbar = &b.full[cb.bar];
                 if (kWeights) {
-                    mbar_arrive_expect_tx(&b.full[chunk_bar(ch)], static_cast<uint32_t>(c * p.blob_bytes));
+                    mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(c * p.blob_bytes));
                     bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes,
                              wtile + static_cast<size_t>(kb) * p.blob_bytes, static_cast<uint32_t>(c * p.blob_bytes),
-                             &b.full[chunk_bar(ch)], policy);
+                             fbar, policy);
                 } else {
-                    mbar_arrive_expect_tx(&b.full[chunk_bar(ch)], static_cast<uint32_t>(c * p.act_slot));
+                    mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(c * p.act_slot));
                     tma_load_3d(aring + static_cast<size_t>(pos) * p.act_slot, &maps->m[c - 1], 0, mt * p.tile_m,
-                                (MODE == kModeW4A8) ? kb : 2 * kb, &b.full[chunk_bar(ch)]);
+                                (MODE == kModeW4A8) ? kb : 2 * kb, fbar);
                 }
                 armed = ch + 1;
             }
             ++ch;
+            cb.next();
             kb += c;
             pos += c;
             if (pos == p.slots) {
@@ -466,7 +487,8 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
     const int hw = (p.issuers == 1) ? -1 : (k0 * (kSteps == 8 ? 16 : 32)) / 64;  // A half it needs (-1: both)
     const uint32_t d_tmem = tmem + static_cast<uint32_t>(q * p.tile_m);
     const uint32_t a_base = smem_addr(aring);
-    uint32_t ch = 0, iter = 0;
+    ChunkBar cb;
+    uint32_t iter = 0;
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
@@ -474,8 +496,8 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
         bool first = true;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            if (ok) ok = wait_bar(&b.full[chunk_bar(ch)], chunk_parity(ch), ctl);
-            ++ch;
+            if (ok) ok = wait_bar(&b.full[cb.bar], cb.parity, ctl);
+            cb.next();
             for (int t = 0; t < c; ++t, ++iter) {
                 const int s = pos + t;
                 const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
@@ -779,7 +801,8 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t slot_addr = tmem + lane_base + kTmemAOffsetS + r * kSlotCols;  // A slot r, this quarter
     const uint32_t part_addr = tmem + lane_base + r * TM;                        // partial buffer r
-    uint32_t ch = 0, iter = 0, uses = 0;  // uses: k-blocks of residue r handed to the MMA so far
+    ChunkBar cb;
+    uint32_t iter = 0, uses = 0;  // uses: k-blocks of residue r handed to the MMA so far
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
@@ -792,8 +815,8 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
         float sc_pending = 1.0f;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
+            const uint32_t fb = cb.bar, fpar = cb.parity;
+            cb.next();
             if (chunk_has(iter, c, 4, r)) {
                 if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
                 const int t = static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block in the chunk
@@ -928,15 +951,16 @@ __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring
     const uint32_t d_tmem = tmem + static_cast<uint32_t>(r * TM);
     const uint32_t a_tmem = tmem + kTmemAOffsetS + static_cast<uint32_t>(r * kSlotCols);
     const uint32_t a_base = smem_addr(aring);
-    uint32_t ch = 0, iter = 0, uses = 0;
+    ChunkBar cb;
+    uint32_t iter = 0, uses = 0;
     int pos = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
-            const uint32_t fb = chunk_bar(ch), fpar = chunk_parity(ch);
-            ++ch;
+            const uint32_t fb = cb.bar, fpar = cb.parity;
+            cb.next();
             if (chunk_has(iter, c, 4, static_cast<uint32_t>(r))) {
                 const int t = static_cast<int>((static_cast<uint32_t>(r) + 4 - iter % 4) % 4);
                 const int s = pos + t;
