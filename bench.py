@@ -145,6 +145,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(inside)}
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (the slowest rank's time); x itself when not distributed."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, bytes_per_step: float, steps: int, seconds: float) -> float:
+    """Whole-job GB/s: every rank runs the same step (replicas), timed by the slowest rank."""
+    return world * bytes_per_step * steps / seconds / 1e9
+
+
 # ------------------------------------------------------------------ our implementation
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -223,16 +240,12 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop()
     t_local = ev0.elapsed_time(ev1) / 1e3
-    t = t_local
-    if world > 1:
-        tt = torch.tensor([t_local], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
+    t = max_over_ranks(t_local, dev)
     if wq.wq_get_device_status(stream) != wq.WQ_OK:
         raise RuntimeError("device status not OK after the timed region")
 
     bytes_step, flops_step = step_totals()
-    value = world * bytes_step * args.steps / t / 1e9
+    value = job_throughput(world, bytes_step, args.steps, t)
     ms_per_step = t / args.steps * 1e3
 
     # ---------------------------------------------------------- end to end through the public API
@@ -256,12 +269,8 @@ def run_ours(args, rank, world, local_rank):
                     L["Y_host"][M].copy_(L["Y"][M], non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize()
-    te = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        tt = torch.tensor([te], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        te = float(tt.item())
-    e2e_value = world * bytes_step * e2e_steps / te / 1e9
+    te = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+    e2e_value = job_throughput(world, bytes_step, e2e_steps, te)
 
     # ---------------------------------------------------------- per-M breakdown (rank 0, outside timing)
     per_m = {}
