@@ -28,7 +28,7 @@ struct GemmArgs {
     int act_slot;              // bytes of one activation slot (one k-block of tile_m rows)
     int blob_bytes;            // bytes of one weight blob = one weight slot
     int group_rows;            // W4A16 grouped: rows per scale slot, min(g, 128)
-    int small;                 // 1: per-k-block partials summed by the accumulate warps (tile_m <= 32)
+    int small;                 // 1: per-k-block partials summed by the dequant warps (tile_m <= 32)
     int scale_in_dequant;      // 1: the dequant multiplies by the group scale (fp16 weights)
     long long units;           // tiles * k_blocks
     int grid;

@@ -29,7 +29,7 @@ SMALL = [
     (128, 128, 128, 1), (256, 256, 64, 3), (384, 136, 32, 16), (1024, 264, 128, 17), (1024, 1024, 128, 33),
     (512, 392, 256, 100), (640, 520, 640, 129), (1024, 512, 1024, 256), (2048, 256, 128, 300),
     (1280, 1000, 128, 64), (4096, 128, 4096, 5), (256, 8, 128, 2), (768, 2056, 32, 48), (512, 640, 512, 513),
-    (2048, 2048, 64, 1), (3072, 1536, 128, 8),
+    (2048, 2048, 64, 1), (3072, 1536, 128, 8), (512, 264, 128, 32), (1024, 136, 1024, 32), (1024, 392, 128, 65),
 ]
 
 

@@ -28,7 +28,7 @@ def _run(d, with_acc=True):
 
 
 SMALL = [(128, 128, 1), (256, 136, 3), (1024, 264, 17), (2048, 1000, 129), (512, 512, 256), (1280, 392, 300),
-         (384, 8, 2), (4096, 256, 64)]
+         (384, 8, 2), (4096, 256, 64), (512, 264, 16), (1024, 392, 32)]
 
 
 @pytest.mark.parametrize("K,N,M", SMALL)
