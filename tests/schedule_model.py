@@ -219,3 +219,161 @@ def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
                 moved = True
     stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
     return problems + stuck
+
+
+# ---------------------------------------------------------------------------- large tiles
+def _roles_large(cta, units, grid, kbs, chunk, slots, issuers, B, state, owner_barrier=True):
+    """The large-tile kernel: 16 dequant warps in 2 residues (walk index mod 2) x 2 halves of
+    a k-block x 4 lane quarters; A slot i mod 4; `issuers` MMA issuers splitting every
+    k-block's K range, each accumulating the whole segment into its own accumulator; the
+    segment-done barrier; the epilogue in the dequant warps. Besides barrier operations the
+    roles report ("acc_read_done", segment) once a dequant warp has read the segment's
+    accumulators and ("acc_overwrite", segment) when an issuer starts a segment's fresh
+    accumulation: an overwrite before all 16 reads of the previous segment is a race."""
+    beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
+
+    def has(it0, c, residue):
+        return ((residue + 2 - it0 % 2) % 2) < c
+
+    def dq(quarter, half, residue):
+        seg_index = 0
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                yield ("wait", B["dfull"], seg_index + 1, seg_index)
+                tile, kb_lo, kb_hi, owner, whole = seg
+                if not owner:
+                    yield ("acc_read_done", seg_index)
+                    yield ("nbar", "epi", 16)
+                    if quarter == 0 and half == 0 and residue == 0:
+                        yield ("flag_set", cta)
+                else:
+                    if not whole:
+                        for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                            yield ("flag_wait", cc)
+                    yield ("acc_read_done", seg_index)
+                    if owner_barrier or not whole:
+                        yield ("nbar", "epi", 16)
+                seg_index += 1
+                continue
+            if not has(it0, c, residue):
+                continue
+            yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
+            for t in range(c):
+                i = it0 + t
+                if i % 2 == residue:
+                    yield ("arrive", B["empty_w"][pos + t])
+                    yield ("wait", B["aempty"][i % 4], i // 4, i)
+                    yield ("arrive", B["afull"][i % 4][half])
+
+    def issuer(q):
+        halves = [0, 1] if issuers == 1 else [(q * (8 // issuers) * 16) // 64]
+        seg_index = 0
+        first = True
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                yield ("arrive", B["dfull"])
+                seg_index += 1
+                first = True
+                continue
+            yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
+            for t in range(c):
+                i = it0 + t
+                for h in halves:
+                    yield ("wait", B["afull"][i % 4][h], i // 4 + 1, i)
+                if first:
+                    yield ("acc_overwrite", seg_index)
+                    first = False
+                yield ("arrive", B["aempty"][i % 4])
+                yield ("arrive", B["empty_a"][pos + t])
+
+    def producer(which):
+        uses = [0] * slots
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                continue
+            for t in range(c):
+                yield ("wait", B[which][pos + t], uses[pos + t], it0 + t)
+                uses[pos + t] += 1
+            yield ("arrive", B["full"][ch % NCB])
+
+    roles = {}
+    for w in range(16):
+        roles[f"dq{w}"] = dq(w & 3, (w >> 2) & 1, w >> 3)
+    for q in range(issuers):
+        roles[f"iss{q}"] = issuer(q)
+    roles["prod_w"] = producer("empty_w")
+    roles["prod_a"] = producer("empty_a")
+    return roles
+
+
+def simulate_large(units, grid, kbs, chunk, slots, issuers, rng=None, ctas_only=None, owner_barrier=True):
+    """Like simulate, for the large-tile kernel; problems also include ("race", cta, segment)
+    for an accumulator overwrite before the previous segment's reads were done."""
+    flags = {}
+    if ctas_only is not None:
+        flags = {c: 1 for c in range(grid) if c not in ctas_only}
+    ctas = []
+    for cta in (range(grid) if ctas_only is None else ctas_only):
+        B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
+             "empty_w": [Bar(8, f"empty_w{s}") for s in range(slots)],
+             "empty_a": [Bar(issuers, f"empty_a{s}") for s in range(slots)],
+             "afull": [[Bar(4, f"afull{a}.{h}") for h in range(2)] for a in range(4)],
+             "aempty": [Bar(issuers, f"aempty{a}") for a in range(4)],
+             "dfull": Bar(issuers, "dfull")}
+        state = {"reads": defaultdict(int)}
+        roles = _roles_large(cta, units, grid, kbs, chunk, slots, issuers, B, state, owner_barrier)
+        ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
+                     "nbar": defaultdict(list), "state": state})
+    problems = []
+    moved = True
+    while moved:
+        moved = False
+        order = [(st, name) for st in ctas for name in st["roles"]]
+        if rng is not None:
+            rng.shuffle(order)
+        for st, name in order:
+            gen = st["roles"][name]
+            steps = 0
+            while name not in st["done"]:
+                if rng is not None and steps >= rng.randint(1, 4):
+                    moved = True
+                    break
+                steps += 1
+                op = st["cur"][name]
+                if op is None:
+                    try:
+                        op = st["cur"][name] = next(gen)
+                    except StopIteration:
+                        st["done"].add(name)
+                        break
+                kind = op[0]
+                if kind == "wait":
+                    if not op[1].ready(op[2]):
+                        break
+                    if op[1].phase != op[2]:
+                        problems.append(("alias", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "flag_wait":
+                    if not flags.get(op[1]):
+                        break
+                elif kind == "arrive":
+                    op[1].arrive()
+                elif kind == "flag_set":
+                    flags[op[1]] = 1
+                elif kind == "acc_read_done":
+                    st["state"]["reads"][op[1]] += 1
+                elif kind == "acc_overwrite":
+                    if op[1] > 0 and st["state"]["reads"][op[1] - 1] < 16:
+                        problems.append(("race", st["cta"], op[1]))
+                elif kind == "nbar":
+                    waiting = st["nbar"][op[1]]
+                    if name not in waiting:
+                        waiting.append(name)
+                    if len(waiting) < op[2]:
+                        break
+                    for other in waiting:
+                        st["cur"][other] = None
+                    st["nbar"][op[1]] = []
+                st["cur"][name] = None
+                moved = True
+    stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+    return problems + stuck

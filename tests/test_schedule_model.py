@@ -129,3 +129,40 @@ def test_first_contributor_closed_form():
             c = first_contributor(t, units, grid)
             assert 0 <= c < grid
             assert unit_start(c, units, grid) <= t < unit_start(c + 1, units, grid), (units, grid, t, c)
+
+
+def _plan_large(K, N):
+    kbs = K // 128
+    units = -(-N // 128) * kbs
+    return units, min(148, units), kbs
+
+
+@pytest.mark.parametrize("K,N", [(4096, 22016), (8192, 8192), (1024, 1024), (4096, 2048)])
+@pytest.mark.parametrize("slots,issuers", [(5, 2), (9, 4), (3, 1), (11, 4)])
+def test_large_tiles_no_alias_deadlock_or_race(K, N, slots, issuers):
+    import random
+    from schedule_model import simulate_large
+    units, grid, kbs = _plan_large(K, N)
+    for cta in sorted({0, grid // 2, grid - 1}):
+        for name, first in _BIASES.items():
+            problems = simulate_large(units, grid, kbs, min(4, slots // 2), slots, issuers,
+                                      rng=_Biased(first, cta), ctas_only=[cta])
+            assert not problems, (name, cta, problems[:3])
+        problems = simulate_large(units, grid, kbs, min(4, slots // 2), slots, issuers,
+                                  rng=random.Random(cta), ctas_only=[cta])
+        assert not problems, ("random", cta, problems[:3])
+
+
+def test_large_model_catches_missing_epilogue_barrier():
+    # the dequant warps of one residue may reach the next segment (and let the MMA start a
+    # fresh accumulation) while the other residue still reads the accumulators, unless every
+    # segment's epilogue ends with a barrier over all dequant warps. An earlier version had
+    # no such barrier after a whole-tile owner epilogue; the GPU showed it as wrong results.
+    from schedule_model import simulate_large
+    units, grid, kbs = _plan_large(4096, 22016)  # 37 units per CTA: whole-tile owner segments
+    races = []
+    for cta in range(20):
+        for name, first in _BIASES.items():
+            races += [p for p in simulate_large(units, grid, kbs, 2, 5, 2, rng=_Biased(first, cta), ctas_only=[cta],
+                                                owner_barrier=False) if p[0] == "race"]
+    assert races
