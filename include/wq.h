@@ -100,7 +100,12 @@ WQ_API int wq_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q_out, void* st
  * Products accumulate in fp32; Y is rounded to nearest-even fp16. For g < K the weight
  * (q-8)*s is rounded once to fp16 before the product; for g == K the column scale is
  * applied to the fp32 sum instead. Uses the workspace of (current device, stream).
- * Results are deterministic: the same call gives the same bits every time. */
+ * Results are deterministic: the same call gives the same bits every time.
+ * The GEMM kernels use programmatic dependent launch: a GEMM may be scheduled while the
+ * previous kernel of the stream is still running, but it reads and writes no caller memory
+ * (A, Wp, Y, acc_out, sa, sw) until that kernel has completed; and it lets the next kernel
+ * of the stream start early only if that kernel was itself launched with programmatic
+ * stream serialisation (a plain launch still waits for the GEMM to complete). */
 WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
                   int M, int N, int K, int g, void* stream);
 
