@@ -102,8 +102,9 @@ WQ_API int wq_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q_out, void* st
  * applied to the fp32 sum instead. Uses the workspace of (current device, stream).
  * Results are deterministic: the same call gives the same bits every time.
  * The GEMM kernels use programmatic dependent launch: a GEMM may be scheduled while the
- * previous kernel of the stream is still running, but it reads and writes no caller memory
- * (A, Wp, Y, acc_out, sa, sw) until that kernel has completed; and it lets the next kernel
+ * previous kernel of the stream is still running, but it uses no caller memory (A, Wp, Y,
+ * acc_out, sa, sw) until that kernel has completed (before then it only asks L2 to prefetch
+ * part of Wp, which reads nothing into the kernel); and it lets the next kernel
  * of the stream start early only if that kernel was itself launched with programmatic
  * stream serialisation (a plain launch still waits for the GEMM to complete). */
 WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
