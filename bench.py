@@ -163,6 +163,76 @@ def job_throughput(world: int, bytes_per_step: float, steps: int, seconds: float
     return world * bytes_per_step * steps / seconds / 1e9
 
 
+# ------------------------------------------------------------------ breakdowns outside the timed region
+COMPUTE_SWEEP = {"K": 8192, "N": 8192, "g": 128, "M": [256, 512, 1024, 4096]}
+W4A8_LAYERS = [(4096, 11008), (11008, 4096)]
+W4A8_M = [1, 16, 128, 1024]
+
+
+def _graph_time(torch, stream, fn, reps):
+    """Seconds per call of fn(r) for r in 0..reps-1, captured once in a CUDA graph and replayed."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(reps):
+                fn(r)
+        g.replay()
+        stream.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(5):
+            g.replay()
+        a1.record(stream)
+    stream.synchronize()
+    t = a0.elapsed_time(a1) / 1e3 / (5 * reps)
+    del g
+    return t
+
+
+def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
+    """The compute-bound W4A16 sweep (K = N = 8192) and the W4A8 layers, each timed alone."""
+    out = {"compute_sweep": {}, "w4a8": {}}
+    cs = COMPUTE_SWEEP
+    K, N, g = cs["K"], cs["N"], cs["g"]
+    d = synth.w4a16_inputs(K, N, g, max(cs["M"]), seed=11)
+    Wp = wq.wq_prepack(torch.from_numpy(d["Q"]).to(dev), torch.from_numpy(d["s"]).to(dev), g)
+    A = torch.from_numpy(d["A"]).to(dev)
+    for M in cs["M"]:
+        Am = A[:M].contiguous()
+        Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wq.wq_workspace_reserve(wq.wq_workspace_bytes(0, M, N, K), stream=stream)
+        t = _graph_time(torch, stream, lambda r: wq.wq_gemm_w4a16(Am, Wp, N, g, Y=Y, stream=stream), 4)
+        f = 2 * M * N * K
+        out["compute_sweep"][str(M)] = {"us": round(t * 1e6, 2), "tflops": round(f / t / 1e12, 1),
+                                        "tensor_frac": round(f / t / 1e12 / tflops, 3)}
+    del Wp, A
+    int8_peak = 2 * tflops  # int8 dense peak: the measured bf16 peak times the nominal 2x ratio
+    for K, N in W4A8_LAYERS:
+        d = synth.w4a8_inputs(K, N, max(W4A8_M), seed=12)
+        Q = torch.from_numpy(d["Q"]).to(dev)
+        copies = max(2, -(-3 * 126_000_000 // (K * N // 2)))
+        Wps = [wq.wq_prepack_w4a8(Q) for _ in range(copies)]
+        sw = torch.from_numpy(d["sw"]).to(dev)
+        A = torch.from_numpy(d["A"]).to(dev)
+        sa = torch.from_numpy(d["sa"]).to(dev)
+        for M in W4A8_M:
+            Am, sam = A[:M].contiguous(), sa[:M].contiguous()
+            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            wq.wq_workspace_reserve(wq.wq_workspace_bytes(1, M, N, K), stream=stream)
+            t = _graph_time(torch, stream,
+                            lambda r: wq.wq_gemm_w4a8(Am, sam, Wps[r % copies], sw, N, Y=Y, stream=stream), 2 * copies)
+            b = K * N // 2 + 4 * N + M * K + 4 * M + 2 * M * N
+            ops = 2 * M * N * K
+            troof = max(b / (hbm_gbs * 1e9), ops / (int8_peak * 1e12))
+            out["w4a8"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
+                                           "tops": round(ops / t / 1e12, 1), "roofline_frac": round(troof / t, 3)}
+        del Wps
+    out["peaks"] = {"tensor_tflops": tflops, "int8_tops": int8_peak,
+                    "note": "int8 peak = measured bf16 peak x the nominal 2x ratio"}
+    return out
+
+
 # ------------------------------------------------------------------ our implementation
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -338,6 +408,10 @@ def run_ours(args, rank, world, local_rank):
                              "tflops": round(f / tm / 1e12, 2), "roofline_frac": round(troof / tm, 3)}
             del g2
 
+    extras = {}
+    if rank == 0 and not args.no_breakdown and not args.case:
+        extras = extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops)
+
     troof_step = sum(roofline_time(M, K, N, hbm_gbs, tflops) for M in M_SWEEP for (K, N) in LAYERS)
     achieved = bytes_step / (t_local / args.steps) / 1e9  # per-launch average over the step's launches
     sha = kernel_sha()
@@ -364,6 +438,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "per_m": per_m,
+        **extras,
         "kernel_sha": sha,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
