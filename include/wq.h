@@ -150,7 +150,9 @@ WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it
  * before capturing the stream into a CUDA graph: a call that has to grow the workspace
  * while the stream is capturing returns WQ_ERR_CAPTURING. Synchronises `stream` when it
- * grows the buffer. */
+ * grows the buffer. A workspace (one int32 flag and one tile_m x 128 fp32 partial per CTA,
+ * at least 1 MiB) is kept for the life of the process; each stream used gets its own, so
+ * calls on different streams may overlap. */
 WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
 
 /* Synchronise `stream`, then return and clear the current device's status word:
