@@ -1130,13 +1130,17 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
     cfg.blockDim = dim3(static_cast<unsigned>(plan.threads));
     cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem_bytes);
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: the stream-K waits always end
-    attr[0].val.cooperative = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // may start before the
-    attr[1].val.programmaticStreamSerializationAllowed = 1;           // previous kernel ends
+    // Programmatic dependent launch: a CTA may start on an SM that the previous kernel of the
+    // stream has already left, set itself up and prefetch its first weights into L2 there.
+    // No cooperative attribute: a cooperative grid is placed all at once, only after the
+    // previous kernel has left every SM. The stream-K waits do not need it. A grid has at most
+    // one CTA per SM and a CTA waits only for CTAs of lower index, so with CTAs dispatched in
+    // index order every CTA waited for is resident, and the waits are bounded regardless.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k, maps, args);
 }
 
