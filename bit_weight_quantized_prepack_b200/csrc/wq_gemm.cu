@@ -632,21 +632,23 @@ __global__ void __launch_bounds__(kThreadsLarge, 1)
 
 // ------------------------------------------------------------------ small tiles
 // Small tiles (at most 32 rows of A) split the walk's k-blocks round-robin over 4 residues: walk
-// index i belongs to residue r = i mod 4. Residue r owns one dequantised A slot and one partial
-// buffer in tensor memory, one MMA issuer and one dequant warp per lane quarter; so every
-// mbarrier has fixed participants that see all of its phases in order (a parity wait can never
-// pass on a phase two ahead or behind).
+// index i belongs to residue r = i mod 4. Residue r owns one dequantised A slot and two partial
+// buffers (2r, 2r + 1) in tensor memory, one MMA issuer and one dequant warp per lane quarter;
+// so every mbarrier has fixed participants that see all of its phases in order (a parity wait
+// can never pass on a phase two ahead or behind).
 //
 // Per k-block i of residue r (the u-th of that residue, u = i / 4):
 //   dequant warps (4 quarters): wait for the chunk's copies (full), read the 16 code words of
 //     their column and release the ring slot (empty_w); wait until the MMAs of their previous
 //     k-block are done (aempty[r], phase u - 1): that frees A slot r and completes partial
-//     buffer r, which they add into fp32 (int32) registers with that k-block's group scale;
-//     then dequantise k-block i into A slot r and signal afull[r].
+//     buffer 2r + (u - 1) % 2; dequantise k-block i into A slot r and signal afull[r]; then,
+//     while the MMAs of k-block i run into the other buffer, add partial u - 1 into fp32
+//     (int32) registers with that k-block's group scale.
 //   issuer r: wait for the activations (full) and afull[r] (phase u), issue the 8 MMAs
-//     (K = 16 each) of the k-block into partial buffer r, commit aempty[r] and the ring slot's
-//     activation half (empty_a).
-// Reading partial r before signalling afull[r] is what keeps the next MMA from overwriting it.
+//     (K = 16 each) of the k-block into partial buffer 2r + u % 2, commit aempty[r] and the
+//     ring slot's activation half (empty_a).
+// The next MMA into buffer 2r + (u - 1) % 2 is that of k-block u + 1, which waits for afull[r]
+// phase u + 1: the dequant warps signal it only after they have read partial u - 1.
 // At a segment's end each dequant warp waits for its last MMA and adds that partial too; the
 // 4 residue warps of a quarter then sum their registers through tensor memory (fixed order
 // r = 0..3) and each finishes a quarter of the tile rows in the epilogue.
@@ -660,7 +662,7 @@ __device__ __forceinline__ int live_rows(const GemmArgs& p, int tile, int TM) {
     return live < TM ? live : TM;
 }
 
-// Adds partial buffer r (this warp's lane quarter) into acc, the first `live` columns only.
+// Adds the partial buffer at paddr (this warp's lane quarter) into acc, the first `live` columns only.
 template <int MODE, int TM>
 __device__ __forceinline__ void add_partial(uint32_t (&acc)[TM], uint32_t paddr, float sc, int live) {
 #pragma unroll
@@ -800,7 +802,7 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t slot_addr = tmem + lane_base + kTmemAOffsetS + r * kSlotCols;  // A slot r, this quarter
-    const uint32_t part_addr = tmem + lane_base + r * TM;                        // partial buffer r
+    const uint32_t part_base = tmem + lane_base + 2 * r * TM;  // partial buffers 2r, 2r + 1 (by use parity)
     ChunkBar cb;
     uint32_t iter = 0, uses = 0;  // uses: k-blocks of residue r handed to the MMA so far
     int pos = 0;
@@ -843,11 +845,10 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
                     __syncwarp();
                     if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);
                 }
-                // MMAs of this residue's previous k-block done: A slot r is free, partial r complete
+                // MMAs of this residue's previous k-block done: A slot r is free, its partial complete
                 if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[r], (uses & 1u) ^ 1u, ctl));
                 if (ok) {
                     tc_fence_after();
-                    if (pending) add_partial<MODE, TM>(acc, part_addr, sc_pending, live);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (kSplitLoad && h == 1) {
@@ -885,6 +886,9 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
                 }
                 __syncwarp();
                 if (ok && lane == 0) mbar_arrive(&b.afull[r][0]);
+                // the previous k-block's partial, in the other buffer, while the MMAs of this
+                // one run; the next MMA into that buffer waits for this warp's next afull
+                if (ok && pending) add_partial<MODE, TM>(acc, part_base + ((uses - 1) & 1u) * TM, sc_pending, live);
                 ++uses;
                 pending = true;
                 sc_pending = kScaleAtAdd ? __half2float(__ushort_as_half(sc_add)) : 1.0f;
@@ -899,17 +903,17 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
             if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.aempty[r], (uses & 1u) ^ 1u, ctl));
             if (ok) {
                 tc_fence_after();
-                add_partial<MODE, TM>(acc, part_addr, sc_pending, live);
+                add_partial<MODE, TM>(acc, part_base + ((uses - 1) & 1u) * TM, sc_pending, live);
             }
         }
         // the 4 residue warps of this quarter sum their registers (r = 0..3 in order) through
-        // the partial buffers, each finishing TM/4 rows: buffer r holds no MMA result now,
-        // and none is issued into it before this warp signals its next afull
+        // partial buffers 0, 2, 4, 6, each finishing TM/4 rows: buffer 2r holds no MMA result
+        // now, and none is issued into it before this warp signals its next afull
         ok = ok && !*ctl.abort_flag;
         if constexpr (TM == 16)
-            tmem_st_x16(part_addr, acc);
+            tmem_st_x16(part_base, acc);
         else
-            tmem_st_x32(part_addr, acc);
+            tmem_st_x32(part_base, acc);
         tmem_st_wait();
         tc_fence_before();
         named_barrier_sync(3 + quarter, 4 * 32);
@@ -922,9 +926,9 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
             for (int rr = 0; rr < 4; ++rr) {
                 uint32_t x[H];
                 if constexpr (H == 4)
-                    tmem_ld_x4(tmem + lane_base + rr * TM + r * H, x);
+                    tmem_ld_x4(tmem + lane_base + 2 * rr * TM + r * H, x);
                 else
-                    tmem_ld_x8(tmem + lane_base + rr * TM + r * H, x);
+                    tmem_ld_x8(tmem + lane_base + 2 * rr * TM + r * H, x);
                 tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < H; ++c)
@@ -941,14 +945,13 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
 
 // Issuer r of a small tile: every k-block whose walk index is r mod 4 is its own; it waits for
 // the k-block's activations (full) and its dequantised weights (A slot r), then writes the
-// k-block's product into partial buffer r with a fresh accumulation.
+// k-block's product into partial buffer 2r + (its use count mod 2) with a fresh accumulation.
 template <int MODE, int TM>
 __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring, Barriers& b, uint32_t tmem,
                                   const Ctl& ctl, long long beg, long long end) {
     constexpr int kSteps = (MODE == kModeW4A8) ? 4 : 8;
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;
     const uint32_t idesc = (MODE == kModeW4A8) ? idesc_s8_s32(kTileN, TM) : idesc_f16_f32(kTileN, TM);
-    const uint32_t d_tmem = tmem + static_cast<uint32_t>(r * TM);
     const uint32_t a_tmem = tmem + kTmemAOffsetS + static_cast<uint32_t>(r * kSlotCols);
     const uint32_t a_base = smem_addr(aring);
     ChunkBar cb;
@@ -966,6 +969,7 @@ __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring
                 const int s = pos + t;
                 if (ok) ok = wait_bar(&b.full[fb], fpar, ctl);
                 if (ok) ok = wait_bar(&b.afull[r][0], uses & 1u, ctl);
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>((2 * r + static_cast<int>(uses & 1u)) * TM);
                 ++uses;
                 if (ok) {
                     tc_fence_after();
@@ -998,7 +1002,7 @@ __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring
 // The small-tile protocol relies on one period (4) for dequant residues, A slots, issuers and
 // partial buffers, and on the A slots fitting in tensor memory beside the partial buffers.
 static_assert(kDqWarpsS == 16 && kASlotsS == kMaxIssuers && kMaxIssuers == 4, "small-tile periods");
-static_assert(kMaxIssuers * kSmallTileMax <= kTmemAOffsetS && kTmemAOffsetS + kASlotsS * 64 <= kTmemCols,
+static_assert(2 * kMaxIssuers * kSmallTileMax <= kTmemAOffsetS && kTmemAOffsetS + kASlotsS * 64 <= kTmemCols,
               "small-tile tensor-memory columns");
 static_assert(kChunkBars > kMaxSlots && kMaxChunk <= 4, "one k-block per residue per chunk");
 

@@ -45,7 +45,7 @@ constexpr int kActWarpS = kWeightWarpS + 1;   // warp 21
 constexpr int kThreadsSmall = (kActWarpS + 1) * 32;  // 704
 constexpr int kASlotsS = 4;                   // dequantised k-blocks in tensor memory (small tiles)
 constexpr int kSmallTileMax = 32;             // tiles of at most this many rows use per-k-block partials
-constexpr int kTmemAOffsetS = 128;            // small tiles: partials in columns [0, 128), 4 A slots above
+constexpr int kTmemAOffsetS = 256;            // small tiles: 2 partials per residue in [0, 256), 4 A slots above
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
 constexpr int kMaxSlots = 32;                 // shared-memory ring slots (one k-block each)
 constexpr int kMaxChunk = 4;                  // k-blocks moved by one copy

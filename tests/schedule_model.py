@@ -8,6 +8,12 @@ lane quarter, tensor-memory A slot i mod 4 and MMA issuer i mod 4. The dequant w
 add the MMA partials (the commit that frees an A slot also completes its partial), so at a
 segment's end each waits for its last MMA; then the named barriers of the 4-way combine and of
 the epilogue, and the stream-K publish flags.
+
+A residue's k-blocks alternate between two partial buffers (its u-th k-block writes buffer
+u % 2). A dequant warp reads the partial of its previous k-block after it has handed the next
+one to the MMA (afull); the model records each read and reports a "race" when an MMA starts
+writing a buffer whose previous partial (two k-blocks of the residue back) has not been read
+by all four lane quarters.
 mbarriers follow the PTX phase/parity rules: a wait on parity p passes once the phase with
 that parity has completed, i.e. while the current phase's parity differs from p.
 
@@ -28,6 +34,7 @@ NCB = 33          # chunk barriers
 NA = 4            # tensor-memory A slots: k-block i uses slot i % NA
 NQ = 4            # MMA issuers: issuer i % NQ
 DQ_PERIOD = 4     # dequant warps per lane quarter: warp (quarter, i % DQ_PERIOD)
+READ_DELAY = 1    # a dequant warp reads a partial after handing this many later k-blocks to the MMA
 
 
 class Bar:
@@ -92,10 +99,14 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
 
     def dq(quarter, residue):
         last = None  # walk index of this residue's last k-block in the current segment
+        unread = []  # this segment's k-blocks of the residue whose partial is not read yet
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
                 if last is not None:  # the segment's last k-block of this residue: its MMAs
                     yield ("wait", B["aempty"][last % NA], last // NA + 1, last)
+                for j in unread:
+                    yield ("part_read", j)
+                unread = []
                 yield ("nbar", f"comb{quarter}", DQ_PERIOD)
                 yield ("nbar", f"comb{quarter}", DQ_PERIOD)
                 tile, kb_lo, kb_hi, owner, whole = seg
@@ -118,6 +129,9 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
                     yield ("arrive", B["empty_w"][pos + t])
                     yield ("wait", B["aempty"][i % NA], i // NA, i)
                     yield ("arrive", B["afull"][i % NA])
+                    unread.append(i)
+                    while len(unread) > READ_DELAY:
+                        yield ("part_read", unread.pop(0))
                     last = i
 
     def issuer(q):
@@ -129,6 +143,7 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
                 i = it0 + t
                 if i % NQ == q:
                     yield ("wait", B["afull"][i % NA], i // NA + 1, i)
+                    yield ("part_write", i)
                     yield ("arrive", B["aempty"][i % NA])
                     yield ("arrive", B["empty_a"][pos + t])
 
@@ -157,7 +172,8 @@ def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
     move in a random order and a random number of operations at a time (any object with
     `shuffle(list)` and `randint(a, b)` can bias the interleaving). Returns a list of problems:
     ("alias", cta, role, barrier, phases needed, phases completed) for each wait that passed on
-    the wrong phase, and (cta, role, pending operation) for each role left blocked."""
+    the wrong phase, ("race", cta, walk index) for each partial overwritten before all four
+    lane quarters read it, and (cta, role, pending operation) for each role left blocked."""
     flags = {}
     if ctas_only is not None:  # CTAs outside the subset count as having published
         flags = {c: 1 for c in range(grid) if c not in ctas_only}
@@ -170,7 +186,7 @@ def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
              "aempty": [Bar(1, f"aempty{a}") for a in range(NA)]}
         roles = _roles(cta, units, grid, kbs, chunk, slots, B)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
-                     "nbar": defaultdict(list)})
+                     "nbar": defaultdict(list), "reads": defaultdict(int)})
     problems = []
     moved = True
     while moved:
@@ -206,6 +222,12 @@ def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
                     op[1].arrive()
                 elif kind == "flag_set":
                     flags[op[1]] = 1
+                elif kind == "part_read":
+                    st["reads"][op[1]] += 1
+                elif kind == "part_write":
+                    # the buffer's previous partial: two k-blocks of the residue back
+                    if op[1] >= 2 * NQ and st["reads"][op[1] - 2 * NQ] < 4:
+                        problems.append(("race", st["cta"], op[1] - 2 * NQ))
                 elif kind == "nbar":
                     waiting = st["nbar"][op[1]]
                     if name not in waiting:

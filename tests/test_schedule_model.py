@@ -166,3 +166,24 @@ def test_large_model_catches_missing_epilogue_barrier():
             races += [p for p in simulate_large(units, grid, kbs, 2, 5, 2, rng=_Biased(first, cta), ctas_only=[cta],
                                                 owner_barrier=False) if p[0] == "race"]
     assert races
+
+
+def test_model_catches_partial_read_too_late():
+    # a residue's k-blocks alternate between two partial buffers, so a dequant warp must read a
+    # partial before it hands the k-block two uses later to the MMA: with the read delayed by
+    # one more k-block, the MMA may overwrite a partial that was never read
+    import random
+    import schedule_model as sm
+    units, grid, kbs = _plan(4096, 22016)
+    saved = sm.READ_DELAY
+    sm.READ_DELAY = 2
+    try:
+        races = []
+        for seed in range(4):
+            races += [p for p in simulate(units, grid, kbs, 4, 16, rng=random.Random(seed), ctas_only=[3])
+                      if p[0] == "race"]
+    finally:
+        sm.READ_DELAY = saved
+    assert races
+    for seed in range(4):
+        assert not simulate(units, grid, kbs, 4, 16, rng=random.Random(seed), ctas_only=[3])
