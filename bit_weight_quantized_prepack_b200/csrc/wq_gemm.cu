@@ -513,11 +513,12 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
                 tc_fence_after();
                 const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
                 const uint32_t a_tmem = tmem + kTmemAOffset + a * kSlotCols;
+                const uint64_t bdesc0 = smem_desc_sw128(act);
                 for (int kk = k0; kk < k0 + steps; ++kk) {
                     const uint32_t boff = (MODE == kModeW4A8)
                                               ? static_cast<uint32_t>(kk * 32)
                                               : static_cast<uint32_t>((kk >> 2) * p.tile_m * 128 + (kk & 3) * 32);
-                    const uint64_t bdesc = smem_desc_sw128(act + boff);
+                    const uint64_t bdesc = smem_desc_advance(bdesc0, boff);
                     const uint32_t accumulate = first ? 0u : 1u;
                     first = false;
                     if (MODE == kModeW4A8)
@@ -974,12 +975,13 @@ __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring
                 if (ok) {
                     tc_fence_after();
                     const uint32_t act = a_base + static_cast<uint32_t>(s * p.act_slot);
+                    const uint64_t bdesc0 = smem_desc_sw128(act);
 #pragma unroll
                     for (int kk = 0; kk < kSteps; ++kk) {
                         const uint32_t boff = (MODE == kModeW4A8)
                                                   ? static_cast<uint32_t>(kk * 32)
                                                   : static_cast<uint32_t>((kk >> 2) * TM * 128 + (kk & 3) * 32);
-                        const uint64_t bdesc = smem_desc_sw128(act + boff);
+                        const uint64_t bdesc = smem_desc_advance(bdesc0, boff);
                         if (MODE == kModeW4A8)
                             mma_i8_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc, kk != 0);
                         else

@@ -225,6 +225,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_byte_addr) {
     return d;
 }
 
+// The descriptor of the operand `bytes` further on (a multiple of 16): the start address field
+// (bits 0-13) holds address >> 4, and shared-memory addresses stay below 2^18, so adding to the
+// low word never carries out of the field. One add per MMA instead of rebuilding the descriptor.
+__device__ __forceinline__ uint64_t smem_desc_advance(uint64_t desc, uint32_t bytes) {
+    const uint32_t lo = static_cast<uint32_t>(desc) + (bytes >> 4);
+    return (desc & 0xFFFFFFFF00000000ull) | lo;
+}
+
 // Instruction descriptor of a dense tcgen05.mma with both operands K-major.
 //  c_format (bits 4-5): 1 = F32, 2 = S32;  a/b format (bits 7-9, 10-12): F16 = 0, S8 = 1;
 //  N >> 3 at bits 17-22; M >> 4 at bits 24-28.
