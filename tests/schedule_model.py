@@ -14,6 +14,13 @@ u % 2). A dequant warp reads the partial of its previous k-block after it has ha
 one to the MMA (afull); the model records each read and reports a "race" when an MMA starts
 writing a buffer whose previous partial (two k-blocks of the residue back) has not been read
 by all four lane quarters.
+
+With TWO_A_SLOTS (and NA = 2 * DQ_PERIOD = 2 * NQ) the model describes a candidate design in
+which every residue alternates between two A slots as well: the dequant warps of k-block u
+wait only for the MMAs of k-block u - 2 (which frees the slot and completes the partial
+buffer that k-block u will write), read that partial, dequantise into the slot and signal it,
+so that they work on k-block u while the MMAs of k-block u - 1 run. At a segment's end they
+wait for, and read, the partials of the last two k-blocks.
 mbarriers follow the PTX phase/parity rules: a wait on parity p passes once the phase with
 that parity has completed, i.e. while the current phase's parity differs from p.
 
@@ -35,6 +42,7 @@ NA = 4            # tensor-memory A slots: k-block i uses slot i % NA
 NQ = 4            # MMA issuers: issuer i % NQ
 DQ_PERIOD = 4     # dequant warps per lane quarter: warp (quarter, i % DQ_PERIOD)
 READ_DELAY = 1    # a dequant warp reads a partial after handing this many later k-blocks to the MMA
+TWO_A_SLOTS = False  # a design with two A slots per residue (NA = 2 * DQ_PERIOD); see below
 
 
 class Bar:
@@ -102,10 +110,15 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
         unread = []  # this segment's k-blocks of the residue whose partial is not read yet
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
-                if last is not None:  # the segment's last k-block of this residue: its MMAs
-                    yield ("wait", B["aempty"][last % NA], last // NA + 1, last)
-                for j in unread:
-                    yield ("part_read", j)
+                if TWO_A_SLOTS:  # the MMAs of the residue's last two k-blocks, then their partials
+                    for j in unread:
+                        yield ("wait", B["aempty"][j % NA], j // NA + 1, j)
+                        yield ("part_read", j)
+                else:
+                    if last is not None:  # the segment's last k-block of this residue: its MMAs
+                        yield ("wait", B["aempty"][last % NA], last // NA + 1, last)
+                    for j in unread:
+                        yield ("part_read", j)
                 unread = []
                 yield ("nbar", f"comb{quarter}", DQ_PERIOD)
                 yield ("nbar", f"comb{quarter}", DQ_PERIOD)
@@ -128,9 +141,11 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
                 if i % DQ_PERIOD == residue:
                     yield ("arrive", B["empty_w"][pos + t])
                     yield ("wait", B["aempty"][i % NA], i // NA, i)
+                    if TWO_A_SLOTS and unread and unread[0] == i - NA:
+                        yield ("part_read", unread.pop(0))  # completed by the MMAs just waited for
                     yield ("arrive", B["afull"][i % NA])
                     unread.append(i)
-                    while len(unread) > READ_DELAY:
+                    while not TWO_A_SLOTS and len(unread) > READ_DELAY:
                         yield ("part_read", unread.pop(0))
                     last = i
 

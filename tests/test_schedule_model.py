@@ -187,3 +187,67 @@ def test_model_catches_partial_read_too_late():
     assert races
     for seed in range(4):
         assert not simulate(units, grid, kbs, 4, 16, rng=random.Random(seed), ctas_only=[3])
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 22016), (8192, 57344), (1024, 136)])
+def test_candidate_two_a_slots_per_residue(K, N):
+    # the candidate next design: 3 residues, each alternating between two A slots and two
+    # partial buffers (6 A slots, 3 issuers, chunks of at most 3 k-blocks): no alias, no stuck
+    # role, no partial overwritten before it is read, under skewed and random interleavings
+    import random
+    import schedule_model as sm
+    units, grid, kbs = _plan(K, N)
+    saved = (sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS)
+    sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS = 6, 3, 3, True
+    try:
+        for cta in sorted({0, grid // 2, grid - 1}):
+            for name, first in _BIASES.items():
+                problems = simulate(units, grid, kbs, 3, 17, rng=_Biased(first, cta), ctas_only=[cta])
+                assert not problems, (name, cta, problems[:3])
+            for seed in range(3):
+                problems = simulate(units, grid, kbs, 3, 17, rng=random.Random(seed), ctas_only=[cta])
+                assert not problems, ("random", seed, cta, problems[:3])
+    finally:
+        sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS = saved
+
+
+def test_candidate_two_a_slots_needs_the_partial_read_before_the_signal():
+    # in the candidate design the partial of k-block u - 2 must be read before k-block u is
+    # handed to the MMA; reading it one k-block later lets the MMA of u overwrite it
+    import random
+    import schedule_model as sm
+    units, grid, kbs = _plan(4096, 22016)
+    saved = (sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS)
+    sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS = 6, 3, 3, True
+    orig = sm._roles
+
+    def late(*args, **kw):
+        roles = orig(*args, **kw)
+        for name, gen in list(roles.items()):
+            if name.startswith("dq"):
+                roles[name] = _delay_reads(gen)
+        return roles
+    sm._roles = late
+    try:
+        races = []
+        for seed in range(4):
+            races += [p for p in simulate(units, grid, kbs, 3, 17, rng=random.Random(seed), ctas_only=[3])
+                      if p[0] == "race"]
+    finally:
+        sm._roles = orig
+        sm.NA, sm.NQ, sm.DQ_PERIOD, sm.TWO_A_SLOTS = saved
+    assert races
+
+
+def _delay_reads(gen):
+    """Moves every partial read after the dequant warp's next A-slot signal."""
+    held = []
+    for op in gen:
+        if op[0] == "part_read":
+            held.append(op)
+            continue
+        yield op
+        if op[0] == "arrive" and op[1].name.startswith("afull") and held:
+            yield from held
+            held = []
+    yield from held
