@@ -53,3 +53,20 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = types.SimpleNamespace(steps=3, warmup=3, reference_budget=1.0)
     assert bench.run_reference(args, rank=1, world=2) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(capsys):
+    # the reference arm times the CPU oracle and prints the same metric as the GPU arm, with
+    # impl "reference", no host<->device bytes and a cpu_baseline describing the run
+    import json
+    import bench
+    args = types.SimpleNamespace(steps=1, warmup=3, reference_budget=2.0)
+    bench.run_reference(args, rank=0, world=1)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "GB/s" and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["e2e"]["value"] == line["value"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
