@@ -27,10 +27,11 @@
 //     Two ways to split the work, by tile height:
 //       small tiles (tile_m <= 32, the memory-bound decode regime): 4 residues; issuer r owns
 //                   every fourth k-block and writes each k-block's product into a fresh
-//                   partial in tensor memory, which the dequant warps of residue r add in fp32
-//                   registers (applying the group scale there, acc += s * P, for g >= 128, so
-//                   the dequant emits exact q - 8) before they reuse their A slot; the four
-//                   residues combine at each segment's end and run the epilogue;
+//                   partial in tensor memory (two buffers per residue, used in turn), which
+//                   the dequant warps of residue r add in fp32 registers (applying the group
+//                   scale there, acc += s * P, for g >= 128, so the dequant emits exact q - 8)
+//                   while the MMAs of the next k-block run; the four residues combine at
+//                   each segment's end and run the epilogue;
 //       large tiles: 2 residues of 8 dequant warps (4 lane quarters x 2 halves of a
 //                   k-block); issuer q owns a quarter (or half, or all) of every k-block's K
 //                   range and accumulates the whole segment in tensor memory; the dequant
@@ -38,8 +39,8 @@
 //     Measured on B200: a thread issuing tcgen05.mma back to back gets one instruction per
 //     ~75-85 cycles whatever the shape, and one issuing bulk copies gets one copy per ~270 ns;
 //     several issuing warps and copies of 16-33 KB take both costs off the critical path.
-//     Integer ALU and packed-fp16 instructions each run at 16 lanes per cycle per SM
-//     sub-partition, so the dequant instruction count sets the small-M ceiling.
+//     At small M each residue's k-block is a chain (dequant into the A slot, MMA issue,
+//     completion, next dequant) whose length, with four chains per SM, sets the ceiling.
 //   * Every wait is bounded by a global-timer limit; an expired wait records WQ_ERR_TIMEOUT
 //     and the CTA winds down (drains its copies and MMAs, frees tensor memory) instead of
 //     hanging.
