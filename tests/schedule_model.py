@@ -21,6 +21,10 @@ wait only for the MMAs of k-block u - 2 (which frees the slot and completes the 
 buffer that k-block u will write), read that partial, dequantise into the slot and signal it,
 so that they work on k-block u while the MMAs of k-block u - 1 run. At a segment's end they
 wait for, and read, the partials of the last two k-blocks.
+
+With ISSUERS_PER_RESIDUE = 2 (another candidate) two issuers serve each residue, each issuing
+half of every k-block's MMAs into a partial of its own; both wait for the same A-slot signal
+and both commit to the slot's barrier and to the ring slot (counts 2).
 mbarriers follow the PTX phase/parity rules: a wait on parity p passes once the phase with
 that parity has completed, i.e. while the current phase's parity differs from p.
 
@@ -43,6 +47,7 @@ NQ = 4            # MMA issuers: issuer i % NQ
 DQ_PERIOD = 4     # dequant warps per lane quarter: warp (quarter, i % DQ_PERIOD)
 READ_DELAY = 1    # a dequant warp reads a partial after handing this many later k-blocks to the MMA
 TWO_A_SLOTS = False  # a design with two A slots per residue (NA = 2 * DQ_PERIOD); see below
+ISSUERS_PER_RESIDUE = 1  # 2: a design in which two issuers split each k-block's MMAs (K halves)
 
 
 class Bar:
@@ -176,7 +181,8 @@ def _roles(cta, units, grid, kbs, chunk, slots, B):
     for w in range(4 * DQ_PERIOD):
         roles[f"dq{w}"] = dq(w & 3, w >> 2)
     for q in range(NQ):
-        roles[f"iss{q}"] = issuer(q)
+        for h in range(ISSUERS_PER_RESIDUE):
+            roles[f"iss{q}" + (f".{h}" if ISSUERS_PER_RESIDUE > 1 else "")] = issuer(q)
     roles["prod_w"] = producer("empty_w")
     roles["prod_a"] = producer("empty_a")
     return roles
@@ -196,9 +202,9 @@ def simulate(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
     for cta in (range(grid) if ctas_only is None else ctas_only):
         B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
              "empty_w": [Bar(4, f"empty_w{s}") for s in range(slots)],
-             "empty_a": [Bar(1, f"empty_a{s}") for s in range(slots)],
+             "empty_a": [Bar(ISSUERS_PER_RESIDUE, f"empty_a{s}") for s in range(slots)],
              "afull": [Bar(4, f"afull{a}") for a in range(NA)],
-             "aempty": [Bar(1, f"aempty{a}") for a in range(NA)]}
+             "aempty": [Bar(ISSUERS_PER_RESIDUE, f"aempty{a}") for a in range(NA)]}
         roles = _roles(cta, units, grid, kbs, chunk, slots, B)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
                      "nbar": defaultdict(list), "reads": defaultdict(int)})

@@ -251,3 +251,24 @@ def _delay_reads(gen):
             yield from held
             held = []
     yield from held
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 22016), (8192, 57344), (1024, 136)])
+def test_candidate_two_issuers_per_residue(K, N):
+    # another candidate: 4 residues, each k-block's 8 MMAs split between two issuers with
+    # partials of their own; the A-slot and ring-slot barriers then count two commits
+    import random
+    import schedule_model as sm
+    units, grid, kbs = _plan(K, N)
+    saved = sm.ISSUERS_PER_RESIDUE
+    sm.ISSUERS_PER_RESIDUE = 2
+    try:
+        for cta in sorted({0, grid // 2, grid - 1}):
+            for name, first in _BIASES.items():
+                problems = simulate(units, grid, kbs, 4, 17, rng=_Biased(first, cta), ctas_only=[cta])
+                assert not problems, (name, cta, problems[:3])
+            for seed in range(3):
+                problems = simulate(units, grid, kbs, 4, 17, rng=random.Random(seed), ctas_only=[cta])
+                assert not problems, ("random", seed, cta, problems[:3])
+    finally:
+        sm.ISSUERS_PER_RESIDUE = saved
