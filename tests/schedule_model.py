@@ -48,6 +48,7 @@ DQ_PERIOD = 4     # dequant warps per lane quarter: warp (quarter, i % DQ_PERIOD
 READ_DELAY = 1    # a dequant warp reads a partial after handing this many later k-blocks to the MMA
 TWO_A_SLOTS = False  # a design with two A slots per residue (NA = 2 * DQ_PERIOD); see below
 ISSUERS_PER_RESIDUE = 1  # 2: a design in which two issuers split each k-block's MMAs (K halves)
+PAIR_MULTICAST_COMMIT = True  # CTA-pair model: the leader's commits reach both CTAs' barriers
 
 
 class Bar:
@@ -419,4 +420,171 @@ def simulate_large(units, grid, kbs, chunk, slots, issuers, rng=None, ctas_only=
                 st["cur"][name] = None
                 moved = True
     stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+    return problems + stuck
+
+
+# ---------------------------------------------------------------------------- large tiles, CTA pairs
+def _roles_large_pair(pair, units, grid, kbs, chunk, slots, issuers, B, state):
+    """The planned 2-SM form of the large-tile kernel: a pair of CTAs (k = 0 leader, 1 follower)
+    walks the same (tile pair, k-block) units. Each CTA dequantises its own 128 weight columns
+    into its own A slots and loads half of the activation rows. The leader's issuers issue the
+    paired MMAs: they wait on the leader's barriers, which count arrivals from both CTAs (the
+    follower's dequant warps arrive remotely, its activation copy signals the leader's barrier),
+    and their commits are multicast to the same barrier in both CTAs. Both CTAs' accumulators are
+    written by every MMA, so a segment's fresh accumulation must wait for all 32 dequant warps
+    of the pair to have read the previous segment's accumulators."""
+    beg, end = unit_start(pair, units, grid), unit_start(pair + 1, units, grid)
+    L = B[0]  # the leader's barriers
+
+    def has(it0, c, residue):
+        return ((residue + 2 - it0 % 2) % 2) < c
+
+    def dq(k, quarter, half, residue):
+        seg_index = 0
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                yield ("wait", B[k]["dfull"], seg_index + 1, seg_index)
+                tile, kb_lo, kb_hi, owner, whole = seg
+                if not owner:
+                    yield ("acc_read_done", seg_index)
+                    yield ("nbar", f"epi{k}", 16)
+                    if quarter == 0 and half == 0 and residue == 0:
+                        yield ("flag_set", (pair, k))
+                else:
+                    if not whole:
+                        for cc in range(pair - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                            yield ("flag_wait", (cc, k))
+                    yield ("acc_read_done", seg_index)
+                    yield ("nbar", f"epi{k}", 16)
+                seg_index += 1
+                continue
+            if not has(it0, c, residue):
+                continue
+            yield ("wait", B[k]["full_w"][ch % NCB], ch // NCB + 1, it0)
+            for t in range(c):
+                i = it0 + t
+                if i % 2 == residue:
+                    yield ("arrive", B[k]["empty_w"][pos + t])
+                    yield ("wait", B[k]["aempty"][i % 4], i // 4, i)
+                    yield ("arrive", L["afull"][i % 4][half])  # remote for the follower
+
+    def issuer(q):
+        halves = [0, 1] if issuers == 1 else [(q * (8 // issuers) * 16) // 64]
+        seg_index = 0
+        first = True
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                for kk in ((0, 1) if PAIR_MULTICAST_COMMIT else (0,)):  # multicast commit
+                    yield ("arrive", B[kk]["dfull"])
+                seg_index += 1
+                first = True
+                continue
+            yield ("wait", L["full_a"][ch % NCB], ch // NCB + 1, it0)
+            for t in range(c):
+                i = it0 + t
+                for h in halves:
+                    yield ("wait", L["afull"][i % 4][h], i // 4 + 1, i)
+                if first:
+                    yield ("acc_overwrite", seg_index)
+                    first = False
+                for kk in ((0, 1) if PAIR_MULTICAST_COMMIT else (0,)):
+                    yield ("arrive", B[kk]["aempty"][i % 4])
+                    yield ("arrive", B[kk]["empty_a"][pos + t])
+
+    def producer(k, which):
+        uses = [0] * slots
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                continue
+            empty = "empty_w" if which == "w" else "empty_a"
+            for t in range(c):
+                yield ("wait", B[k][empty][pos + t], uses[pos + t], it0 + t)
+                uses[pos + t] += 1
+            yield ("arrive", B[k]["full_w"][ch % NCB] if which == "w" else L["full_a"][ch % NCB])
+
+    roles = {}
+    for k in (0, 1):
+        for w in range(16):
+            roles[f"dq{k}.{w}"] = dq(k, w & 3, (w >> 2) & 1, w >> 3)
+        roles[f"prod_w{k}"] = producer(k, "w")
+        roles[f"prod_a{k}"] = producer(k, "a")
+    for q in range(issuers):
+        roles[f"iss{q}"] = issuer(q)
+    return roles
+
+
+def simulate_large_pair(units, grid, kbs, chunk, slots, issuers, rng=None, pairs_only=None):
+    """Like simulate_large, for CTA pairs (`grid` pairs over `units` (tile pair, k-block) units)."""
+    flags = {}
+    if pairs_only is not None:
+        flags = {(c, k): 1 for c in range(grid) if c not in pairs_only for k in (0, 1)}
+    pairs = []
+    for pair in (range(grid) if pairs_only is None else pairs_only):
+        B = []
+        for k in (0, 1):
+            b = {"full_w": [Bar(1, f"full_w{k}.{x}") for x in range(NCB)],
+                 "empty_w": [Bar(8, f"empty_w{k}.{s}") for s in range(slots)],
+                 "empty_a": [Bar(issuers, f"empty_a{k}.{s}") for s in range(slots)],
+                 "aempty": [Bar(issuers, f"aempty{k}.{a}") for a in range(4)],
+                 "dfull": Bar(issuers, f"dfull{k}")}
+            if k == 0:
+                b["full_a"] = [Bar(2, f"full_a.{x}") for x in range(NCB)]
+                b["afull"] = [[Bar(8, f"afull{a}.{h}") for h in range(2)] for a in range(4)]
+            B.append(b)
+        state = {"reads": defaultdict(int)}
+        roles = _roles_large_pair(pair, units, grid, kbs, chunk, slots, issuers, B, state)
+        pairs.append({"cta": pair, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
+                      "nbar": defaultdict(list), "state": state})
+    problems = []
+    moved = True
+    while moved:
+        moved = False
+        order = [(st, name) for st in pairs for name in st["roles"]]
+        if rng is not None:
+            rng.shuffle(order)
+        for st, name in order:
+            gen = st["roles"][name]
+            steps = 0
+            while name not in st["done"]:
+                if rng is not None and steps >= rng.randint(1, 4):
+                    moved = True
+                    break
+                steps += 1
+                op = st["cur"][name]
+                if op is None:
+                    try:
+                        op = st["cur"][name] = next(gen)
+                    except StopIteration:
+                        st["done"].add(name)
+                        break
+                kind = op[0]
+                if kind == "wait":
+                    if not op[1].ready(op[2]):
+                        break
+                    if op[1].phase != op[2]:
+                        problems.append(("alias", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "flag_wait":
+                    if not flags.get(op[1]):
+                        break
+                elif kind == "arrive":
+                    op[1].arrive()
+                elif kind == "flag_set":
+                    flags[op[1]] = 1
+                elif kind == "acc_read_done":
+                    st["state"]["reads"][op[1]] += 1
+                elif kind == "acc_overwrite":
+                    if op[1] > 0 and st["state"]["reads"][op[1] - 1] < 32:
+                        problems.append(("race", st["cta"], op[1]))
+                elif kind == "nbar":
+                    waiting = st["nbar"][op[1]]
+                    if name not in waiting:
+                        waiting.append(name)
+                    if len(waiting) < op[2]:
+                        break
+                    for other in waiting:
+                        st["cur"][other] = None
+                    st["nbar"][op[1]] = []
+                st["cur"][name] = None
+                moved = True
+    stuck = [(st["cta"], name, st["cur"][name]) for st in pairs for name in st["roles"] if name not in st["done"]]
     return problems + stuck

@@ -272,3 +272,39 @@ def test_candidate_two_issuers_per_residue(K, N):
                 assert not problems, ("random", seed, cta, problems[:3])
     finally:
         sm.ISSUERS_PER_RESIDUE = saved
+
+
+def _plan_pairs(K, N):
+    kbs = K // 128
+    units = -(-N // 256) * kbs  # (256-column tile pair, k-block) units
+    return units, min(74, units), kbs
+
+
+@pytest.mark.parametrize("K,N", [(8192, 8192), (4096, 22016), (1024, 1024), (4096, 2048)])
+@pytest.mark.parametrize("slots,issuers", [(3, 1), (5, 2), (9, 4)])
+def test_planned_cta_pair_large_tiles(K, N, slots, issuers):
+    # the planned 2-SM form of the large-tile kernel: the leader's barriers count both CTAs'
+    # arrivals and its commits are multicast to both; no alias, stuck role or accumulator race
+    import random
+    from schedule_model import simulate_large_pair
+    units, grid, kbs = _plan_pairs(K, N)
+    for pair in sorted({0, grid // 2, grid - 1}):
+        for name, first in _BIASES.items():
+            problems = simulate_large_pair(units, grid, kbs, min(4, slots // 2), slots, issuers,
+                                           rng=_Biased(first, pair), pairs_only=[pair])
+            assert not problems, (name, pair, problems[:3])
+        problems = simulate_large_pair(units, grid, kbs, min(4, slots // 2), slots, issuers,
+                                       rng=random.Random(pair), pairs_only=[pair])
+        assert not problems, ("random", pair, problems[:3])
+
+
+def test_cta_pair_model_catches_a_commit_that_reaches_one_cta():
+    # without the multicast, the follower's dequant warps never see their A slots freed
+    import schedule_model as sm
+    units, grid, kbs = _plan_pairs(4096, 22016)
+    sm.PAIR_MULTICAST_COMMIT = False
+    try:
+        problems = sm.simulate_large_pair(units, grid, kbs, 2, 5, 2, pairs_only=[3])
+    finally:
+        sm.PAIR_MULTICAST_COMMIT = True
+    assert any(isinstance(p[1], str) and p[1].startswith("dq1.") for p in problems)
