@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import sys
 
 import torch
 
@@ -17,7 +18,7 @@ __all__ = [
     "WqError", "lib", "LIB_PATH", "status_string", "wq_version",
     "wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepack", "wq_prepack_w4a8",
     "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a16_noalloc", "wq_gemm_w4a8",
-    "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan",
+    "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
     "WQ_ERR_UNSUPPORTED_DEVICE", "WQ_ERR_CUDA", "WQ_ERR_TIMEOUT", "WQ_ERR_NO_MEMORY", "WQ_ERR_CAPTURING",
@@ -63,6 +64,7 @@ def _load():
         "wq_workspace_reserve": (I, [Z, P]),
         "wq_get_device_status": (I, [P]),
         "wq_plan": (I, [I, I, I, I, I, ctypes.POINTER(_Plan)]),
+        "wq_plan_for": (I, [I, I, I, I, I, I, I, ctypes.POINTER(_Plan)]),
         "wq_debug_set_wait_timeout_ns": (I, [ctypes.c_ulonglong]),
         "wq_debug_skip_publish": (I, [I]),
     }
@@ -74,7 +76,14 @@ def _load():
     return L
 
 
-lib = _load()
+try:
+    lib = _load()
+except (ImportError, OSError, AttributeError) as _err:  # missing, unloadable or older than the header
+    # `python -m bit_weight_quantized_prepack_b200.build` imports this package before it runs the
+    # build (sys.argv[0] is "-m" while Python locates the module): let that command proceed.
+    if sys.argv[:1] != ["-m"]:
+        raise ImportError(f"libwq.so is missing or older than include/wq.h ({_err})") from _err
+    lib = None
 
 
 def status_string(status: int) -> str:
@@ -215,6 +224,13 @@ def wq_get_device_status(stream=None) -> int:
 def wq_plan(kind: int, M: int, N: int, K: int, g: int) -> dict:
     p = _Plan()
     _check(lib.wq_plan(kind, M, N, K, g, ctypes.byref(p)), "wq_plan")
+    return {f: getattr(p, f) for f, _ in _Plan._fields_}
+
+
+def wq_plan_for(kind: int, M: int, N: int, K: int, g: int, num_sms: int, smem_optin: int) -> dict:
+    """The plan on a device with num_sms SMs and smem_optin bytes of opt-in shared memory (no GPU needed)."""
+    p = _Plan()
+    _check(lib.wq_plan_for(kind, M, N, K, g, num_sms, smem_optin, ctypes.byref(p)), "wq_plan_for")
     return {f: getattr(p, f) for f, _ in _Plan._fields_}
 
 

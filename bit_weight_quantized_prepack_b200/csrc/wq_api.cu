@@ -486,19 +486,22 @@ int wq_get_device_status(void* stream) {
     return h;
 }
 
-int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
+namespace {
+// The plan of a call on a device with `num_sms` SMs and `smem_optin` bytes of opt-in shared
+// memory per block; host arithmetic only.
+int fill_plan(int kind, int M, int N, int K, int g, int num_sms, int smem_optin, wq_plan_t* plan) {
     if (!plan) return WQ_ERR_INVALID_ARG;
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M <= 0) return WQ_ERR_INVALID_ARG;
+    if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (kind != 0 && kind != 1) return WQ_ERR_INVALID_ARG;
-    std::lock_guard<std::mutex> lock(g_mu);
-    int dev = 0;
-    DeviceState* d = device_state(&dev);
-    if (!d) return WQ_ERR_CUDA;
-    if (!d->supported) return WQ_ERR_UNSUPPORTED_DEVICE;
+    if (num_sms <= 0 || smem_optin <= 0) return WQ_ERR_INVALID_ARG;
+    DeviceState d;
+    d.num_sms = num_sms;
+    d.smem_optin = smem_optin;
     Plan pl;
-    rc = plan_for(kind, M, N, K, kind == 0 ? g : K, *d, &pl);
+    rc = plan_for(kind, M, N, K, kind == 0 ? g : K, d, &pl);
     if (rc) return rc;
     plan->grid = pl.grid;
     plan->tile_m = pl.tile_m;
@@ -510,6 +513,30 @@ int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
     plan->threads = pl.threads;
     plan->units = pl.units;
     return WQ_OK;
+}
+}  // namespace
+
+int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
+    if (!plan) return WQ_ERR_INVALID_ARG;
+    int rc = check_shape(K, N);
+    if (rc) return rc;
+    if (M <= 0) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1) return WQ_ERR_INVALID_ARG;
+    int num_sms = 0, smem_optin = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        int dev = 0;
+        DeviceState* d = device_state(&dev);
+        if (!d) return WQ_ERR_CUDA;
+        if (!d->supported) return WQ_ERR_UNSUPPORTED_DEVICE;
+        num_sms = d->num_sms;
+        smem_optin = d->smem_optin;
+    }
+    return fill_plan(kind, M, N, K, g, num_sms, smem_optin, plan);
+}
+
+int wq_plan_for(int kind, int M, int N, int K, int g, int num_sms, int smem_optin, wq_plan_t* plan) {
+    return fill_plan(kind, M, N, K, g, num_sms, smem_optin, plan);
 }
 
 int wq_debug_set_wait_timeout_ns(unsigned long long ns) {

@@ -176,6 +176,12 @@ typedef struct {
 } wq_plan_t;
 WQ_API int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan);
 
+/* The same plan for a device with `num_sms` SMs and `smem_optin` bytes of opt-in dynamic
+ * shared memory per block, without touching any device (host arithmetic only; usable on a
+ * machine without a GPU). Arguments are checked as for wq_plan; num_sms and smem_optin must
+ * be positive; WQ_ERR_UNSUPPORTED_SHAPE when no pipeline of two stages fits. */
+WQ_API int wq_plan_for(int kind, int M, int N, int K, int g, int num_sms, int smem_optin, wq_plan_t* plan);
+
 /* Test hooks. wq_debug_set_wait_timeout_ns sets the limit of every device-side wait
  * (default 2e9 ns; 0 restores the default). wq_debug_skip_publish(c) makes CTA c skip
  * publishing its partial sum to the tile that owns it (c = -1 disables), so that the

@@ -1,0 +1,71 @@
+"""CPU tests of the launch planner through wq_plan_for (host arithmetic, no GPU): for a B200's
+148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
+cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
+work."""
+import itertools
+
+import pytest
+
+SMS, SMEM = 148, 232448
+
+
+@pytest.fixture(scope="module")
+def wq():
+    return pytest.importorskip("bit_weight_quantized_prepack_b200")
+
+
+MS = [1, 2, 5, 15, 16, 17, 31, 32, 33, 48, 63, 64, 65, 100, 127, 128, 129, 200, 255, 256, 257, 511, 1024, 4096]
+SHAPES = [(128, 8), (1024, 136), (4096, 4096), (4096, 22016), (11008, 4096), (8192, 57344), (131072, 8)]
+
+
+@pytest.mark.parametrize("K,N", SHAPES)
+@pytest.mark.parametrize("kind,g", [(0, 32), (0, 64), (0, 128), (0, 256), (0, None), (1, None)])
+def test_plan_invariants(wq, K, N, kind, g):
+    if g is None:
+        g = K
+    if kind == 0 and K % g:
+        pytest.skip("group size must divide K")
+    for M in MS:
+        p = wq.wq_plan_for(kind, M, N, K, g, SMS, SMEM)
+        tm = p["tile_m"]
+        assert tm % 16 == 0 and 16 <= tm <= 256, (M, p)
+        assert p["m_tiles"] == -(-M // tm), (M, p)                     # the tiles cover M ...
+        assert (p["m_tiles"] - 1) * tm < M, (M, p)                      # ... with no empty tile
+        assert p["n_tiles"] == -(-N // 128) and p["k_blocks"] == K // 128
+        assert p["units"] == p["n_tiles"] * p["m_tiles"] * p["k_blocks"]
+        assert p["grid"] == min(SMS, p["units"])                        # every CTA has a unit
+        assert 2 <= p["stages"] <= 32
+        act = tm * (256 if kind == 0 else 128)
+        blob = 8192 + (256 * (128 // min(g, 128)) if kind == 0 and g < K else 0)
+        assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024     # ring + alignment slack
+        assert p["smem_bytes"] + 2048 <= SMEM                           # room for the static barriers
+        assert p["threads"] == 704
+
+
+def test_plan_uses_the_largest_ring_that_fits(wq):
+    for M, kind in itertools.product([1, 16, 32, 64, 256], [0, 1]):
+        p = wq.wq_plan_for(kind, M, 4096, 4096, 128 if kind == 0 else 4096, SMS, SMEM)
+        act = p["tile_m"] * (256 if kind == 0 else 128)
+        blob = 8192 + (256 if kind == 0 else 0)
+        more = (p["stages"] + 1) * (act + blob) + 1024
+        assert p["stages"] == 32 or more + 2048 > SMEM, p
+
+
+def test_plan_scales_with_the_device(wq):
+    small = wq.wq_plan_for(0, 1, 4096, 4096, 128, 20, SMEM)
+    assert small["grid"] == 20
+    tight = wq.wq_plan_for(0, 64, 4096, 4096, 128, SMS, 100 * 1024)
+    assert tight["stages"] >= 2 and tight["smem_bytes"] + 2048 <= 100 * 1024
+    with pytest.raises(wq.WqError):  # 256-row tiles need two 72 KB stages
+        wq.wq_plan_for(0, 256, 4096, 4096, 128, SMS, 100 * 1024)
+
+
+def test_plan_rejects_bad_arguments(wq):
+    bad = [(2, 1, 4096, 4096, 128, SMS, SMEM), (0, 0, 4096, 4096, 128, SMS, SMEM),
+           (0, 1, 4096, 4000, 128, SMS, SMEM), (0, 1, 4096, 4096, 100, SMS, SMEM),
+           (0, 1, 4096, 4096, 128, 0, SMEM), (0, 1, 4096, 4096, 128, SMS, 0)]
+    for args in bad:
+        with pytest.raises(wq.WqError):
+            wq.wq_plan_for(*args)
+    with pytest.raises(wq.WqError):
+        wq.wq_plan_for(0, 1, 4096, 4096, 128, SMS, 16 * 1024)  # not even two stages fit
