@@ -107,14 +107,50 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _dev_tensor(t, dtype, name):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
+def _tensor(t, dtype, name, shape=None, min_numel=None):
+    """Type, dtype, contiguity and size of one argument; raises before anything reaches the library.
+
+    ``shape`` is the exact shape the call implies; ``min_numel`` the least number of elements
+    (for the flat prepacked buffer). A wrongly sized buffer would otherwise become an
+    out-of-bounds copy or store on the device."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, the call needs at least {min_numel}")
     return t
+
+
+def _on_one_cuda_device(**tensors):
+    """Every given tensor on the same CUDA device (checked after the sizes)."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other arguments on {dev}")
+
+
+def _matrix(t, name):
+    if not isinstance(t, torch.Tensor) or t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor")
+    return t.shape
+
+
+def _prepacked_size(K, N, g, name):
+    n = wq_prepacked_bytes(K, N, g) if g is not None else wq_prepacked_bytes_w4a8(K, N)
+    if n == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE if K % 128 == 0 or g is None else WQ_ERR_INVALID_ARG, name)
+    return n
 
 
 def wq_version() -> int:
@@ -131,12 +167,16 @@ def wq_prepacked_bytes_w4a8(K: int, N: int) -> int:
 
 def wq_prepack(Q: torch.Tensor, s: torch.Tensor, g: int, Wp: torch.Tensor | None = None, stream=None):
     """Q int32 [K/8, N], s fp16 [K/g, N] -> Wp uint8 [wq_prepacked_bytes(K, N, g)]."""
-    _dev_tensor(Q, torch.int32, "Q")
-    _dev_tensor(s, torch.float16, "s")
-    K, N = Q.shape[0] * 8, Q.shape[1]
-    nbytes = wq_prepacked_bytes(K, N, g)
-    if nbytes == 0:
-        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack")
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    if g <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_prepack")
+    _tensor(s, torch.float16, "s", shape=(K // g, N))
+    nbytes = _prepacked_size(K, N, g, "wq_prepack")
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Q=Q, s=s, Wp=Wp)
     if Wp is None:
         Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
     _check(lib.wq_prepack(_ptr(Q), _ptr(s), K, N, g, _ptr(Wp), _stream(stream)), "wq_prepack")
@@ -144,11 +184,13 @@ def wq_prepack(Q: torch.Tensor, s: torch.Tensor, g: int, Wp: torch.Tensor | None
 
 
 def wq_prepack_w4a8(Q: torch.Tensor, Wp: torch.Tensor | None = None, stream=None):
-    _dev_tensor(Q, torch.int32, "Q")
-    K, N = Q.shape[0] * 8, Q.shape[1]
-    nbytes = wq_prepacked_bytes_w4a8(K, N)
-    if nbytes == 0:
-        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack_w4a8")
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    nbytes = _prepacked_size(K, N, None, "wq_prepack_w4a8")
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Q=Q, Wp=Wp)
     if Wp is None:
         Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
     _check(lib.wq_prepack_w4a8(_ptr(Q), K, N, _ptr(Wp), _stream(stream)), "wq_prepack_w4a8")
@@ -157,6 +199,10 @@ def wq_prepack_w4a8(Q: torch.Tensor, Wp: torch.Tensor | None = None, stream=None
 
 def wq_unpack(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
     """Inverse of wq_prepack: (Q int32 [K/8, N], s fp16 [K/g, N])."""
+    if g <= 0 or K <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_unpack")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_prepacked_size(K, N, g, "wq_unpack"))
+    _on_one_cuda_device(Wp=Wp)
     Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
     s = torch.empty((K // g, N), dtype=torch.float16, device=Wp.device)
     _check(lib.wq_unpack(_ptr(Wp), K, N, g, _ptr(Q), _ptr(s), _stream(stream)), "wq_unpack")
@@ -164,18 +210,30 @@ def wq_unpack(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
 
 
 def wq_unpack_w4a8(Wp: torch.Tensor, K: int, N: int, stream=None):
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_prepacked_size(K, N, None, "wq_unpack_w4a8"))
+    _on_one_cuda_device(Wp=Wp)
     Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
     _check(lib.wq_unpack_w4a8(_ptr(Wp), K, N, _ptr(Q), _stream(stream)), "wq_unpack_w4a8")
     return Q
 
 
+def _gemm_w4a16_args(A, Wp, N, g, Y, where):
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    if g <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, where)
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_prepacked_size(K, N, g, where))
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    _on_one_cuda_device(A=A, Wp=Wp, Y=Y)
+    return M, K
+
+
 def wq_gemm_w4a16(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor | None = None, stream=None):
     """Y fp16 [M, N] = A fp16 [M, K] . dequant(Wp)."""
-    _dev_tensor(A, torch.float16, "A")
-    M, K = A.shape
+    M, K = _gemm_w4a16_args(A, Wp, N, g, Y, "wq_gemm_w4a16")
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
-    _dev_tensor(Y, torch.float16, "Y")
     _check(lib.wq_gemm_w4a16(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)), "wq_gemm_w4a16")
     return Y
 
@@ -184,9 +242,9 @@ def wq_gemm_w4a16_noalloc(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: 
     """wq_gemm_w4a16 for callers that must not allocate: the library's stream-K scratch is a
     fixed 8 MiB device array (M <= 64 on a 148-SM B200) and Y must be given. Calls whose
     kernels overlap on the GPU race on that array."""
-    _dev_tensor(A, torch.float16, "A")
-    _dev_tensor(Y, torch.float16, "Y")
-    M, K = A.shape
+    if Y is None:
+        raise ValueError("wq_gemm_w4a16_noalloc: Y must be given (the call allocates nothing)")
+    M, K = _gemm_w4a16_args(A, Wp, N, g, Y, "wq_gemm_w4a16_noalloc")
     _check(lib.wq_gemm_w4a16_noalloc(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)),
            "wq_gemm_w4a16_noalloc")
     return Y
@@ -195,14 +253,18 @@ def wq_gemm_w4a16_noalloc(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: 
 def wq_gemm_w4a8(A: torch.Tensor, sa: torch.Tensor, Wp: torch.Tensor, sw: torch.Tensor, N: int,
                  Y: torch.Tensor | None = None, acc_out: torch.Tensor | None = None, stream=None):
     """Y fp16 [M, N] = (A int8 [M, K] . (q - 8)) * sa[m] * sw[n]; acc_out (optional) gets the int32 sums."""
-    _dev_tensor(A, torch.int8, "A")
-    _dev_tensor(sa, torch.float32, "sa")
-    _dev_tensor(sw, torch.float32, "sw")
-    M, K = A.shape
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.int8, "A")
+    _tensor(sa, torch.float32, "sa", shape=(M,))
+    _tensor(sw, torch.float32, "sw", shape=(N,))
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_prepacked_size(K, N, None, "wq_gemm_w4a8"))
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    if acc_out is not None:
+        _tensor(acc_out, torch.int32, "acc_out", shape=(M, N))
+    _on_one_cuda_device(A=A, sa=sa, sw=sw, Wp=Wp, Y=Y, acc_out=acc_out)
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
-    if acc_out is not None:
-        _dev_tensor(acc_out, torch.int32, "acc_out")
     _check(lib.wq_gemm_w4a8(_ptr(A), _ptr(sa), _ptr(Wp), _ptr(sw), _ptr(Y), _ptr(acc_out), M, N, K,
                             _stream(stream)), "wq_gemm_w4a8")
     return Y

@@ -19,6 +19,9 @@ using namespace wq;
 
 constexpr int kVersion = 10000;  // 1.0.0
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+// W4A8 accumulates a * 16(q - 8) in int32; |a * 16(q - 8)| <= 128 * 128 = 16384 (a = -128,
+// q = 0), and K * 16384 < 2^31 holds for every multiple of 128 up to 130944.
+constexpr int kMaxKW4A8 = 130944;
 
 std::mutex g_mu;
 unsigned long long g_timeout_ns = kDefaultTimeoutNs;
@@ -181,7 +184,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     if (M < 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (kind == 0 && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
-    if (kind == 1 && K > 131072) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (kind == 1 && K > kMaxKW4A8) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (!Wp) return WQ_ERR_INVALID_ARG;
     if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
     if (M == 0) return WQ_OK;
@@ -477,13 +480,26 @@ int wq_get_device_status(void* stream) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return WQ_ERR_CUDA;
     int h = 0;
     if (cudaMemcpy(&h, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WQ_ERR_CUDA;
-    if (h == WQ_OK) return WQ_OK;
-    // a wait expired: clear the status word and every workspace's flags of this device
-    if (cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess) return WQ_ERR_CUDA;
-    for (auto& kv : g_workspaces)
-        if (kv.first.first == dev && kv.second.ptr)
-            if (cudaMemset(kv.second.ptr, 0, 4096) != cudaSuccess) return WQ_ERR_CUDA;
-    return h;
+    // the fixed-scratch call keeps its own status word in its array (read and cleared here
+    // without any allocation)
+    int h_fixed = 0;
+    NoAllocDevice* na = (dev >= 0 && dev < kNoAllocMaxDevices && g_noalloc[dev].ready) ? &g_noalloc[dev] : nullptr;
+    if (na && cudaMemcpy(&h_fixed, na->scratch + kNoAllocStatusOffset, sizeof(int), cudaMemcpyDeviceToHost) !=
+                  cudaSuccess)
+        return WQ_ERR_CUDA;
+    if (h == WQ_OK && h_fixed == WQ_OK) return WQ_OK;
+    // a wait expired: clear the status words and every workspace's flags of this device
+    if (h != WQ_OK) {
+        if (cudaMemset(d->status, 0, sizeof(int)) != cudaSuccess) return WQ_ERR_CUDA;
+        for (auto& kv : g_workspaces)
+            if (kv.first.first == dev && kv.second.ptr)
+                if (cudaMemset(kv.second.ptr, 0, 4096) != cudaSuccess) return WQ_ERR_CUDA;
+    }
+    if (h_fixed != WQ_OK) {
+        if (cudaMemset(na->scratch + kNoAllocStatusOffset, 0, sizeof(int)) != cudaSuccess) return WQ_ERR_CUDA;
+        if (cudaMemset(na->scratch, 0, 4096) != cudaSuccess) return WQ_ERR_CUDA;
+    }
+    return h != WQ_OK ? h : h_fixed;
 }
 
 namespace {
@@ -616,7 +632,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     a.units = pl.units;
     a.grid = pl.grid;
     a.timeout_ns = g_timeout_ns;
-    a.skip_publish = -1;
+    a.skip_publish = g_skip_publish;
     if (launch_gemm(pl.mode, maps, a, pl, st) != cudaSuccess) {
         cudaGetLastError();
         return WQ_ERR_CUDA;

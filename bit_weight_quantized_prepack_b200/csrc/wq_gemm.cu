@@ -338,8 +338,11 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
     // them hand the next segment's first k-block to the MMA, which overwrites the accumulators
     tc_fence_before();
     named_barrier_sync(1, kNumDqWarps * 32);
-    if (!seg.whole && threadIdx.x == 0)
-        for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
+    // ready for the next call, but only when every wait of the CTA succeeded: after an expired
+    // wait a contributor may still publish late, and the flags stay set until the host clears
+    // them (wq_get_device_status)
+    if (!seg.whole && threadIdx.x == 0 && !*ctl.abort_flag)
+        for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;
 }
 
 // ------------------------------------------------------------------ roles
@@ -784,8 +787,8 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
     }
     if (!seg.whole) {
         named_barrier_sync(2, kDqWarpsS * 32);  // every dequant warp has read the partials
-        if (leader)
-            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;  // ready for the next call
+        if (leader && !*ctl.abort_flag)  // as in the large-tile epilogue: not after an expired wait
+            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;
     }
 }
 

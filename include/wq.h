@@ -113,7 +113,9 @@ WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
 /* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
  * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
  * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
- * Requires K <= 131072 so that no int32 partial sum can overflow. */
+ * A may hold any int8 value, -128 included. Requires K <= 130944 (the largest multiple of
+ * 128 with K * 16384 < 2^31): the kernel sums a * 16(q - 8), whose magnitude reaches
+ * 128 * 128 = 16384, in int32, so no partial sum can overflow. */
 WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw,
                  uint16_t* Y, int32_t* acc_out, int M, int N, int K, void* stream);
 
@@ -121,7 +123,7 @@ WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const 
  * cannot allocate device memory when they run the layer (an engine that gave all free
  * memory to its own pool at start-up, a plugin whose host framework owns every
  * allocation, a latency-critical loop that must not risk an allocation's implicit
- * synchronisation). Same arguments, result bits and status codes as wq_gemm_w4a16, but
+ * synchronisation). Same arguments and result bits as wq_gemm_w4a16, but
  * the stream-K scratch (publish flags, partial tiles) lives in one fixed array of
  * WQ_NOALLOC_SCRATCH_BYTES (8 MiB) that every device loading the library holds until
  * the process exits; this call never calls cudaMalloc or cudaFree.
@@ -136,8 +138,9 @@ WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const 
  * - All calls on one device share the array: two calls whose kernels overlap on the GPU
  *   (different streams without ordering between them) race and give wrong results.
  *   Order them on one stream or with events.
- * - A device-side wait that expires stops the kernel as in wq_gemm_w4a16, but is recorded
- *   in the array, not in the word wq_get_device_status reads: it is not reported. */
+ * - A device-side wait that expires stops the kernel as in wq_gemm_w4a16; it is recorded in
+ *   the array's own status word, which wq_get_device_status reads and clears as well
+ *   (without allocating). */
 #define WQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
                   int M, int N, int K, int g, void* stream);
@@ -155,10 +158,12 @@ WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
  * calls on different streams may overlap. */
 WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
 
-/* Synchronise `stream`, then return and clear the current device's status word:
- * WQ_OK, or WQ_ERR_TIMEOUT when a device-side wait expired since the last call (the
- * outputs of that call are then undefined). On error it also clears the device's
- * workspace flags so that later calls start clean. */
+/* Synchronise `stream`, then return and clear the current device's status words (that of
+ * the workspace calls and that of wq_gemm_w4a16_noalloc): WQ_OK, or WQ_ERR_TIMEOUT when a
+ * device-side wait expired since the last call. The outputs of the call whose wait expired
+ * are undefined, and so are those of every later call on the same stream (or, for
+ * wq_gemm_w4a16_noalloc, on the same device) until this function has returned: an expired
+ * wait leaves stream-K flags set, and only this function clears them. */
 WQ_API int wq_get_device_status(void* stream);
 
 /* ---------------------------------------------------------------- introspection and test hooks
@@ -186,7 +191,8 @@ WQ_API int wq_plan_for(int kind, int M, int N, int K, int g, int num_sms, int sm
  * (default 2e9 ns; 0 restores the default). wq_debug_skip_publish(c) makes CTA c skip
  * publishing its partial sum to the tile that owns it (c = -1 disables), so that the
  * owner's bounded wait expires: the call then reports WQ_ERR_TIMEOUT through
- * wq_get_device_status instead of hanging. Both apply to later calls on every device. */
+ * wq_get_device_status instead of hanging. Both apply to later calls on every device, of
+ * wq_gemm_w4a16, wq_gemm_w4a8 and wq_gemm_w4a16_noalloc alike. */
 WQ_API int wq_debug_set_wait_timeout_ns(unsigned long long ns);
 WQ_API int wq_debug_skip_publish(int cta);
 

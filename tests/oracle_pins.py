@@ -11,7 +11,10 @@ with the fact it is pinned to:
   dequantised weights, all-8 codes give zero, all-0 codes give
   ``-8 * sum_k a_k s_k``;
 * invariants: power-of-two scale homogeneity, row permutation, linearity;
-* W4A8: the integer accumulator against Python integer loops.
+* W4A8: the integer accumulator against Python integer loops;
+* the prepacked layout: single codes and scales placed by hand-worked byte
+  offsets (``tests/golden/blob_layout.txt``), independent of the oracle's own
+  inverse of its layout.
 """
 from __future__ import annotations
 
@@ -226,8 +229,58 @@ def pin_w4a8_extremes(o):
     assert np.all(o.w4a8_acc(A, Q) == -7 * 127 * K)
 
 
+# ---------------------------------------------------------------- prepacked layout
+def golden_layout():
+    out = []
+    for line in _rows("blob_layout.txt"):
+        parts = [p.strip() for p in line.split("|")]
+        kind, what = parts[0].split()
+        dims = parts[1].split()
+        K, N = int(dims[0]), int(dims[1])
+        g = None if dims[2] == "-" else int(dims[2])
+        a, b = (int(x) for x in parts[2].split())
+        offs = [int(x) for x in parts[3].split()]
+        half = parts[4] if len(parts) > 4 else None
+        out.append((kind, what, K, N, g, a, b, offs, half))
+    return out
+
+
+# a scale bit pattern whose two bytes are both non-zero and different
+_SCALE_BITS = 0x4A3C
+
+
+def pin_blob_layout_golden(o):
+    # one code (value 3 among 8s) or one scale (among zeros) at a time: exactly the bytes the
+    # hand-worked table names change, to exactly the values it implies
+    for kind, what, K, N, g, a, b, offs, half in golden_layout():
+        if what == "code":
+            q = np.full((K, N), 8, np.uint8)
+            base_q = q.copy()
+            q[a, b] = 3
+            if kind == "w4a16":
+                s = np.zeros((K // g, N), np.float16)
+                Wp, base = o.prepack_w4a16(synth.pack_q(q), s, g), o.prepack_w4a16(synth.pack_q(base_q), s, g)
+            else:
+                Wp, base = o.prepack_w4a8(synth.pack_q(q)), o.prepack_w4a8(synth.pack_q(base_q))
+            diff = np.nonzero(Wp != base)[0].tolist()
+            assert diff == offs, (kind, K, N, g, a, b, diff, offs)
+            want = 0x83 if half == "lo" else 0x38
+            assert int(Wp[offs[0]]) == want, (kind, a, b, hex(int(Wp[offs[0]])))
+        else:
+            q = np.full((K, N), 8, np.uint8)
+            s = np.zeros((K // g, N), np.float16)
+            base = o.prepack_w4a16(synth.pack_q(q), s, g)
+            s[a, b] = np.array([_SCALE_BITS], np.uint16).view(np.float16)[0]
+            Wp = o.prepack_w4a16(synth.pack_q(q), s, g)
+            diff = np.nonzero(Wp != base)[0].tolist()
+            assert diff == sorted(x for off in offs for x in (off, off + 1)), (K, N, g, a, b, diff, offs)
+            for off in offs:
+                assert int(Wp[off]) | (int(Wp[off + 1]) << 8) == _SCALE_BITS
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
     pin_row_permutation, pin_linearity, pin_tolerance_formula, pin_bruteforce_w4a8, pin_w4a8_extremes,
+    pin_blob_layout_golden,
 ]

@@ -74,6 +74,10 @@ def test_host_side_argument_checks(wq):
     assert L.wq_gemm_w4a16(good, good, good, -1, 128, 128, 128, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_gemm_w4a16(good, good, good, (1 << 24) + 1, 128, 128, 128, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
     assert L.wq_gemm_w4a8(good, good, good, good, good, None, 1, 128, 262144, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
+    # W4A8 sums a * 16(q - 8) in int32, up to 16384 per term (a = -128): K = 131072 would wrap
+    assert L.wq_gemm_w4a8(good, good, good, good, good, None, 1, 128, 131072, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
+    assert L.wq_gemm_w4a8(good, good, good, good, good, None, 0, 128, 130944, None) == wq.WQ_OK
+    assert 130944 * 16384 < 2 ** 31 <= 131072 * 16384
     # group size
     assert L.wq_gemm_w4a16(good, good, good, 1, 128, 256, 48, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_prepack(good, good, 256, 128, 96, good, None) == wq.WQ_ERR_INVALID_ARG

@@ -6,7 +6,7 @@ import oracle
 import synth
 from oracle import wq_oracle as O
 
-from oracle_pins import ALL_PINS
+from oracle_pins import ALL_PINS, pin_blob_layout_golden
 
 
 
@@ -148,6 +148,55 @@ def test_prepack_padding_is_zero_weight():
     full = O.unprepack_w4a16(Wp, K, 128, g)
     assert np.all(full[0][:, N:] == 8)
     assert np.all(full[1][:, N:] == 0)
+
+
+# Layout mistakes made in both directions at once (prepack and its inverse): the round trip and
+# the blob-locality test cannot see them; only the hand-worked byte offsets can.
+def _mut_layout_h_v_swapped(mp):
+    def blob_words(q, nibble_pos):
+        w = _ORIG_BLOB_WORDS(q, nibble_pos)           # [nt, kt, h, v, r, i]
+        return np.ascontiguousarray(w.transpose(0, 1, 3, 2, 4, 5))
+
+    def codes_from_words(words, nibble_pos, K, N):
+        nt, kt = words.shape[:2]
+        w = words.reshape(nt, kt, 2, 2, O.TILE_N, 4).transpose(0, 1, 3, 2, 4, 5)
+        return _ORIG_CODES_FROM_WORDS(np.ascontiguousarray(w).reshape(nt, kt, -1), nibble_pos, K, N)
+    mp.setattr(O, "_blob_words", blob_words)
+    mp.setattr(O, "_codes_from_words", codes_from_words)
+
+
+def _mut_layout_i_reversed(mp):
+    def blob_words(q, nibble_pos):
+        return np.ascontiguousarray(_ORIG_BLOB_WORDS(q, nibble_pos)[..., ::-1])
+
+    def codes_from_words(words, nibble_pos, K, N):
+        nt, kt = words.shape[:2]
+        w = words.reshape(nt, kt, 2, 2, O.TILE_N, 4)[..., ::-1]
+        return _ORIG_CODES_FROM_WORDS(np.ascontiguousarray(w).reshape(nt, kt, -1), nibble_pos, K, N)
+    mp.setattr(O, "_blob_words", blob_words)
+    mp.setattr(O, "_codes_from_words", codes_from_words)
+
+
+def _mut_layout_nibble_table(mp):
+    mp.setattr(O, "NIBBLE_POS_W4A16", (0, 1, 2, 3, 4, 5, 6, 7))
+
+
+_ORIG_BLOB_WORDS = O._blob_words
+_ORIG_CODES_FROM_WORDS = O._codes_from_words
+LAYOUT_MUTATIONS = [_mut_layout_h_v_swapped, _mut_layout_i_reversed, _mut_layout_nibble_table]
+
+
+@pytest.mark.parametrize("mutate", LAYOUT_MUTATIONS, ids=lambda f: f.__name__[5:])
+def test_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeypatch):
+    mutate(monkeypatch)
+    # the self-consistency checks still pass with the mistake in place ...
+    for K, N, g in SHAPES[:3]:
+        test_prepack_roundtrip(K, N, g)
+    test_prepack_w4a8_roundtrip(256, 200)
+    test_prepack_blob_locality()
+    # ... and the hand-worked byte offsets catch it
+    with pytest.raises(AssertionError):
+        pin_blob_layout_golden(O)
 
 
 def test_package_reexports():

@@ -8,11 +8,13 @@ allocation. For them the library keeps the stream-K scratch of the W4A16 kernels
 
 The test calls the entry point through the C ABI (ctypes, raw device pointers) twice in a
 row with different activations, so that the second call runs on the scratch the first one
-left behind, and compares each output with the regular entry point's on the same inputs:
-within the parity tolerance of the other tests and, since both run the same deterministic
-kernels, bit for bit. It also checks that the second call leaves the device's free memory
-unchanged and that a call needing more scratch than the array holds is refused without a
-launch. The file is named to be collected last.
+left behind. Each output is compared with the fp64 oracle within the parity tolerance of the
+other tests and, since both entry points run the same deterministic kernels, bit for bit with
+the regular entry point on the same inputs. The cases cover 16-row tiles, 32-row tiles, a
+large tile and per-column scales (g = K). The test also checks that the second call leaves
+the device's free memory unchanged, that a call needing more scratch than the array holds is
+refused without a launch, and that an expired device-side wait of the fixed-scratch call is
+reported by wq_get_device_status. The file is named to be collected last.
 """
 import ctypes
 
@@ -21,7 +23,8 @@ import pytest
 
 torch = pytest.importorskip("torch")
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
 def _c_abi(wq, A, Wp, Y, N, g):
@@ -31,11 +34,17 @@ def _c_abi(wq, A, Wp, Y, N, g):
                                         ctypes.c_void_p(Y.data_ptr()), M, N, K, g, stream)
 
 
-@pytest.mark.parametrize("K,N,g,M", [(4096, 1032, 128, 5), (2048, 2056, 64, 40)])
-def test_noalloc_matches_the_allocating_call_twice_in_a_row(K, N, g, M):
+# (K, N, g, M): 16-row tile; 32-row tile; a 48-row large tile; per-column scales on 16- and 32-row tiles
+CASES = [(4096, 1032, 128, 5), (1024, 1032, 128, 28), (2048, 2056, 64, 40), (2048, 520, 2048, 3),
+         (1024, 264, 1024, 24)]
+
+
+@pytest.mark.parametrize("K,N,g,M", CASES)
+def test_noalloc_matches_the_oracle_twice_in_a_row(K, N, g, M):
     import bit_weight_quantized_prepack_b200 as wq
     import oracle
     import synth
+    from wq_check import compare
     d = synth.w4a16_inputs(K, N, g, M, seed=11)
     Q = torch.from_numpy(d["Q"]).cuda()
     s = torch.from_numpy(d["s"]).cuda()
@@ -53,14 +62,13 @@ def test_noalloc_matches_the_allocating_call_twice_in_a_row(K, N, g, M):
         torch.cuda.synchronize()
         if call == 1:  # the first call on a device may load the library's device code
             assert torch.cuda.mem_get_info()[0] == free_before, "the call changed free device memory"
-        Y_ref = wq.wq_gemm_w4a16(A, Wp, N, g)
-        torch.cuda.synchronize()
+        assert wq.wq_get_device_status() == wq.WQ_OK
         y = Y.float().cpu().numpy().astype(np.float64)
-        y_ref = Y_ref.float().cpu().numpy().astype(np.float64)
-        assert np.all(np.isfinite(y)), f"call {call}: non-finite output"
-        bound = oracle.tolerance(y_ref, oracle.w4a16_absdot(A_np, d["Q"], d["s"], g))
-        assert np.all(np.abs(y - y_ref) <= bound), f"call {call}: outside tolerance"
-        assert torch.equal(Y.view(torch.int16), Y_ref.view(torch.int16)), f"call {call}: bits differ"
+        y_ref = oracle.w4a16(A_np, d["Q"], d["s"], g)
+        compare(y, y_ref, oracle.w4a16_absdot(A_np, d["Q"], d["s"], g), f"call {call}")
+        Y_alloc = wq.wq_gemm_w4a16(A, Wp, N, g)
+        torch.cuda.synchronize()
+        assert torch.equal(Y.view(torch.int16), Y_alloc.view(torch.int16)), f"call {call}: bits differ"
 
 
 def test_noalloc_refuses_a_plan_beyond_its_scratch():
@@ -74,3 +82,35 @@ def test_noalloc_refuses_a_plan_beyond_its_scratch():
     assert rc == wq.WQ_ERR_SCRATCH_LIMIT, wq.status_string(rc)
     torch.cuda.synchronize()
     assert bool((Y == 7.0).all()), "a refused call must launch nothing"
+
+
+def test_noalloc_expired_wait_is_reported_and_cleared():
+    # CTA 0 skips publishing its partial, so the owner of tile 0 waits on a flag that nothing
+    # sets; with a 20 ms limit the wait expires. wq_get_device_status reports it from the fixed
+    # array's own status word, clears it, and the next call is correct.
+    import bit_weight_quantized_prepack_b200 as wq
+    import oracle
+    import synth
+    from wq_check import compare
+    K, N, g, M = 4096, 4096, 128, 1
+    plan = wq.wq_plan(0, M, N, K, g)
+    assert plan["units"] > plan["grid"] > 1 and plan["units"] % plan["grid"] != 0
+    d = synth.w4a16_inputs(K, N, g, M, seed=3)
+    A = torch.from_numpy(d["A"]).cuda()
+    Wp = wq.wq_prepack(torch.from_numpy(d["Q"]).cuda(), torch.from_numpy(d["s"]).cuda(), g)
+    Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    assert wq.wq_get_device_status() == wq.WQ_OK
+    wq.wq_debug_set_wait_timeout_ns(20_000_000)
+    wq.wq_debug_skip_publish(0)
+    try:
+        assert _c_abi(wq, A, Wp, Y, N, g) == wq.WQ_OK
+        assert wq.wq_get_device_status() == wq.WQ_ERR_TIMEOUT
+    finally:
+        wq.wq_debug_skip_publish(-1)
+        wq.wq_debug_set_wait_timeout_ns(0)
+    assert wq.wq_get_device_status() == wq.WQ_OK
+    assert _c_abi(wq, A, Wp, Y, N, g) == wq.WQ_OK
+    assert wq.wq_get_device_status() == wq.WQ_OK
+    y = Y.float().cpu().numpy().astype(np.float64)
+    compare(y, oracle.w4a16(d["A"], d["Q"], d["s"], g), oracle.w4a16_absdot(d["A"], d["Q"], d["s"], g),
+            "after an expired wait")
