@@ -42,7 +42,7 @@ import numpy as np
 
 __all__ = [
     "unpack_codes", "dequant", "w4a16", "w4a16_absdot", "w4a16_entry",
-    "tolerance", "w4a8_acc", "w4a8", "w4a8_absdot",
+    "tolerance", "w4a8_acc", "w4a8", "w4a8_absdot", "quantize_act",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
 ]
@@ -150,6 +150,38 @@ def w4a8_absdot(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray, ch
         wq = np.abs(unpack_codes(np.asarray(Q)[:, n0:n1]).astype(np.float64) - ZERO_POINT)
         out[:, n0:n1] = A64 @ wq
     return out * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+
+
+# --------------------------------------------------------------------------
+# dynamic per-token activation quantisation (the step before W4A8)
+# --------------------------------------------------------------------------
+def quantize_act(A: np.ndarray):
+    """``(q, sa)``: int8 codes ``q[M,K]`` and fp32 per-token scales ``sa[M]`` of fp16 activations.
+
+    "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving", method: the
+    activations' quantisation parameters are computed from the activation matrix itself at
+    inference time, one scale per token (row). The pages fix neither the rounding nor the
+    range; the reading used here is the plainest symmetric one, written in fp32 so that the
+    integer codes are decided in one stated precision:
+
+    * ``amax[m] = max_k |A[m,k]|`` (exact: fp16 values);
+    * ``inv = fp32(127 / amax)``, ``q = rint(fp32(A[m,k] * inv))`` with ties to even, clamped
+      to ``[-127, 127]`` (-128 is never produced);
+    * ``sa[m] = fp32(amax / 127)``, so ``A[m,k] ~ q[m,k] * sa[m]``;
+    * a row of zeros gives ``q = 0`` and ``sa = 0``.
+    """
+    A32 = np.asarray(A, dtype=np.float16).astype(np.float32)
+    amax = np.max(np.abs(A32), axis=1)
+    q = np.zeros(A32.shape, dtype=np.int8)
+    sa = np.zeros(A32.shape[0], dtype=np.float32)
+    for m in range(A32.shape[0]):
+        if amax[m] == 0:
+            continue
+        inv = np.float32(127.0) / amax[m]                     # fp32 division, round to nearest
+        t = A32[m] * inv                                      # fp32 products, round to nearest
+        q[m] = np.clip(np.rint(t), -127, 127).astype(np.int8)  # ties to even
+        sa[m] = amax[m] / np.float32(127.0)
+    return q, sa
 
 
 # --------------------------------------------------------------------------

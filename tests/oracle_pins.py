@@ -12,6 +12,8 @@ with the fact it is pinned to:
   ``-8 * sum_k a_k s_k``;
 * invariants: power-of-two scale homogeneity, row permutation, linearity;
 * W4A8: the integer accumulator against Python integer loops;
+* per-token activation quantisation: hand-worked rows (``tests/golden/act_quant.txt``)
+  and exact rational bounds;
 * the prepacked layout: single codes and scales placed by hand-worked byte
   offsets (``tests/golden/blob_layout.txt``), independent of the oracle's own
   inverse of its layout.
@@ -278,9 +280,52 @@ def pin_blob_layout_golden(o):
                 assert int(Wp[off]) | (int(Wp[off + 1]) << 8) == _SCALE_BITS
 
 
+# ---------------------------------------------------------------- per-token activation quantisation
+def golden_act_quant():
+    out = []
+    for line in _rows("act_quant.txt"):
+        acts, codes, sa = [x.strip() for x in line.split("|")]
+        out.append((np.array([float(x) for x in acts.split()], np.float16),
+                    [int(x) for x in codes.split()], None if sa == "-" else float(sa)))
+    return out
+
+
+def pin_act_quant_golden(o):
+    rows = golden_act_quant()
+    q, sa = o.quantize_act(np.stack([r[0] for r in rows]))
+    assert q.dtype == np.int8 and sa.dtype == np.float32
+    for i, (a, codes, s) in enumerate(rows):
+        assert q[i].tolist() == codes, (i, q[i].tolist(), codes)
+        if s is not None:
+            assert float(sa[i]) == s, (i, float(sa[i]), s)
+
+
+def pin_act_quant_bounds(o):
+    # against exact rational arithmetic: each code is within 1/2 (plus the two fp32 roundings)
+    # of a * 127 / max|a|, never beyond +-127, equal to +-127 at the row's largest magnitude,
+    # of the activation's sign; and sa is max|a| / 127 to fp32 precision
+    rng = np.random.default_rng(4)
+    A = (rng.standard_normal((6, 96)) * np.array([[1e-3], [1.0], [30.0], [1e3], [0.5], [7.0]])).astype(np.float16)
+    A[4, :] = 0
+    A[4, 17] = -0.25
+    q, sa = o.quantize_act(A)
+    for m in range(A.shape[0]):
+        amax = max(abs(Fraction(float(x))) for x in A[m])
+        assert abs(Fraction(float(sa[m])) - amax / 127) <= amax / 127 * Fraction(2.0 ** -24)
+        for k in range(A.shape[1]):
+            a = Fraction(float(A[m, k]))
+            exact = a * 127 / amax
+            assert abs(int(q[m, k])) <= 127
+            assert abs(Fraction(int(q[m, k])) - exact) <= Fraction(1, 2) + 256 * Fraction(2.0 ** -24), (m, k)
+            if abs(a) == amax:
+                assert abs(int(q[m, k])) == 127
+            if q[m, k] != 0:
+                assert (q[m, k] > 0) == (a > 0)
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
     pin_row_permutation, pin_linearity, pin_tolerance_formula, pin_bruteforce_w4a8, pin_w4a8_extremes,
-    pin_blob_layout_golden,
+    pin_blob_layout_golden, pin_act_quant_golden, pin_act_quant_bounds,
 ]
