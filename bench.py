@@ -49,11 +49,10 @@ WORKLOAD = "llama7b_w4a16_layer_set_M1-128_g128"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# DRAM traffic per launch of the GEMM kernels over one step's 32 launches (dram__bytes_read.sum
-# + dram__bytes_write.sum, averaged), from the ncu capture summarised in
-# profiles/wq_gemm_w4a16_llama7b_step_launches.md; valid for the kernel sources whose hash is
-# recorded with it, reported as null once they change.
-TRAFFIC = {"kernel_sha": "2f7971dec97ad603", "bytes_per_launch": 26527376}
+# DRAM traffic per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum
+# from one ncu capture of a few of its launches in this workload), valid for the kernel sources
+# whose hash is recorded with it and reported as null once they change.
+TRAFFIC = {"kernel_sha": None, "bytes_per_launch": None, "algo_bytes_per_launch": None}
 
 
 def kernel_sha() -> str:
@@ -87,8 +86,36 @@ def step_totals():
     return b, f
 
 
-def roofline_time(M, K, N, hbm_gbs, tflops):
-    return max(algo_bytes(M, K, N) / (hbm_gbs * 1e9), algo_flops(M, K, N) / (tflops * 1e12))
+def roofline_time(M, K, N, hbm_gbs, tflops, g=None):
+    return max(algo_bytes(M, K, N, G if g is None else g) / (hbm_gbs * 1e9), algo_flops(M, K, N) / (tflops * 1e12))
+
+
+def fp16_bound_time(M, K, N, hbm_gbs):
+    """Time to move a dense fp16 weight, A and Y at the copy bandwidth: what the same layer with
+    fp16 weights cannot beat. (time of this bound) / (measured time) is the speedup over it."""
+    return (2 * K * N + 2 * M * K + 2 * M * N) / (hbm_gbs * 1e9)
+
+
+def launch_times(torch, stream, fns, reps):
+    """Per-launch device times (s) of isolated launches: fns are single calls, made round robin
+    (so consecutive launches read different weight copies), each between two CUDA events on the
+    launching stream. An isolated launch does not overlap its neighbours, unlike the step's
+    back-to-back launches (which set up while the previous kernel finishes)."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for fn in fns:
+            fn()
+        for i in range(reps):
+            evs[i][0].record(stream)
+            fns[i % len(fns)]()
+            evs[i][1].record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b) / 1e3 for a, b in evs]
+
+
+def pct_us(ts):
+    """(p10, median, p90) of times in seconds, as microseconds."""
+    return [round(float(np.percentile(ts, q)) * 1e6, 2) for q in (10, 50, 90)]
 
 
 # ------------------------------------------------------------------ clocks
@@ -143,7 +170,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in used for i, v in enumerate(r[1][6:10]) if v.lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(inside)}
+                "reasons": reasons, "samples": len(used), "samples_in_window": len(inside)}
 
 
 # ------------------------------------------------------------------ multi-rank helpers
@@ -190,6 +217,42 @@ def _graph_time(torch, stream, fn, reps):
     return t
 
 
+LAYERS_70B = [(8192, 10240), (8192, 8192), (8192, 57344), (28672, 8192)]
+M_70B = [1, 16, 64, 128]
+
+
+def rows_70b(torch, wq, dev, stream, hbm_gbs, tflops):
+    """The 70B-shaped W4A16 layers at M in {1, 16, 64, 128}, each with g = 128 and with one scale
+    per column (g = K): per-launch p10 / median / p90 over rotated weight copies (more than 3x
+    L2 per rotation), effective GB/s, roofline fraction and the speedup over the dense fp16
+    weight-read bound, all from the median."""
+    out = {}
+    for K, N in LAYERS_70B:
+        for g in (128, K):
+            d = synth.w4a16_inputs(K, N, g, max(M_70B), seed=21)
+            Q, s = torch.from_numpy(d["Q"]).to(dev), torch.from_numpy(d["s"]).to(dev)
+            wbytes = K * N // 2 + 2 * (K // g) * N
+            copies = int(min(12, max(2, -(-3 * 126_000_000 // wbytes))))
+            Wps = [wq.wq_prepack(Q, s, g) for _ in range(copies)]
+            A = torch.from_numpy(d["A"]).to(dev)
+            for M in M_70B:
+                Am = A[:M].contiguous()
+                Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                wq.wq_workspace_reserve(wq.wq_workspace_bytes(0, M, N, K), stream=stream)
+                fns = [(lambda W: lambda: wq.wq_gemm_w4a16(Am, W, N, g, Y=Y, stream=stream))(W) for W in Wps]
+                ts = launch_times(torch, stream, fns, max(12, 2 * copies))
+                p10, med, p90 = pct_us(ts)
+                t = med / 1e6
+                out[f"{K}x{N}_g{'K' if g == K else g}_M{M}"] = {
+                    "us_p10_med_p90": [p10, med, p90],
+                    "gbs": round(algo_bytes(M, K, N, g) / t / 1e9, 1),
+                    "tflops": round(algo_flops(M, K, N) / t / 1e12, 2),
+                    "roofline_frac": round(roofline_time(M, K, N, hbm_gbs, tflops, g) / t, 3),
+                    "speedup_vs_fp16_bound": round(fp16_bound_time(M, K, N, hbm_gbs) / t, 2)}
+            del Wps, Q, s, A
+    return out
+
+
 def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
     """The compute-bound W4A16 sweep (K = N = 8192) and the W4A8 layers, each timed alone."""
     out = {"compute_sweep": {}, "w4a8": {}}
@@ -228,8 +291,31 @@ def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
             out["w4a8"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
                                            "tops": round(ops / t / 1e12, 1), "roofline_frac": round(troof / t, 3)}
         del Wps
+    # the W4A8 layer on fp16 activations (per-token quantisation + the int8 layer, one call) and the
+    # quantisation kernel alone (HBM-bound: 2MK bytes read, MK + 4M written)
+    out["w4a8_fp16act"] = {}
+    for K, N in W4A8_LAYERS:
+        d = synth.w4a8_inputs(K, N, 1, seed=13)
+        Q = torch.from_numpy(d["Q"]).to(dev)
+        copies = max(2, -(-3 * 126_000_000 // (K * N // 2)))
+        Wps = [wq.wq_prepack_w4a8(Q) for _ in range(copies)]
+        sw = torch.from_numpy(d["sw"]).to(dev)
+        for M in W4A8_M:
+            A16 = torch.randn((M, K), generator=torch.Generator().manual_seed(M), dtype=torch.float32).half().to(dev)
+            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            Aq = torch.empty((M, K), dtype=torch.int8, device=dev)
+            sa = torch.empty((M,), dtype=torch.float32, device=dev)
+            wq.wq_workspace_reserve(wq.wq_workspace_bytes(2, M, N, K), stream=stream)
+            t = _graph_time(torch, stream,
+                            lambda r: wq.wq_gemm_w4a8_fp16act(A16, Wps[r % copies], sw, N, Y=Y, stream=stream), 2 * copies)
+            tq = _graph_time(torch, stream, lambda r: wq.wq_quantize_act(A16, Aq, sa, stream=stream), 8)
+            bq = 3 * M * K + 4 * M
+            out["w4a8_fp16act"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "quantize_us": round(tq * 1e6, 2),
+                                                   "quantize_gbs": round(bq / tq / 1e9, 1)}
+        del Wps
     out["peaks"] = {"tensor_tflops": tflops, "int8_tops": int8_peak,
                     "note": "int8 peak = measured bf16 peak x the nominal 2x ratio"}
+    out["layers_70b"] = rows_70b(torch, wq, dev, stream, hbm_gbs, tflops)
     return out
 
 
@@ -305,10 +391,23 @@ def run_ours(args, rank, world, local_rank):
             graph.replay()
         ev1.record(stream)
     torch.cuda.synchronize()
+    # a timed region shorter than the sampling period may hold no clock sample: the same step is
+    # then replayed, untimed, until half a second has passed, and the samples of that whole window
+    # are reported (the window is named in the record)
+    window = "timed region"
+    t_reg = (datetime.datetime.now() - sampler.t_start).total_seconds()
+    if t_reg < 0.5:
+        window = "timed region and untimed replays of the same step right after it (0.5 s in all)"
+        with torch.cuda.stream(stream):
+            while (datetime.datetime.now() - sampler.t_start).total_seconds() < 0.5:
+                for _ in range(20):
+                    graph.replay()
+                stream.synchronize()
     sampler.mark("stop")
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
+    clocks["window"] = window
     t_local = ev0.elapsed_time(ev1) / 1e3
     t = max_over_ranks(t_local, dev)
     if wq.wq_get_device_status(stream) != wq.WQ_OK:
@@ -382,6 +481,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---------------------------------------------------------- per-M breakdown (rank 0, outside timing)
     per_m = {}
+    c1_row = {}  # the single 4096 x 4096 layer at M = 1, g = 128, timed alone
     if rank == 0 and not args.no_breakdown:
         for mi, M in enumerate(M_SWEEP):
             g2 = torch.cuda.CUDAGraph()
@@ -404,16 +504,54 @@ def run_ours(args, rank, world, local_rank):
             b = sum(algo_bytes(M, L["K"], L["N"]) for L in layers)
             f = sum(algo_flops(M, L["K"], L["N"]) for L in layers)
             troof = sum(roofline_time(M, L["K"], L["N"], hbm_gbs, tflops) for L in layers)
+            t16 = sum(fp16_bound_time(M, L["K"], L["N"], hbm_gbs) for L in layers)
             per_m[str(M)] = {"us": round(tm * 1e6, 2), "gbs": round(b / tm / 1e9, 1),
-                             "tflops": round(f / tm / 1e12, 2), "roofline_frac": round(troof / tm, 3)}
+                             "tflops": round(f / tm / 1e12, 2), "roofline_frac": round(troof / tm, 3),
+                             "speedup_vs_fp16_bound": round(t16 / tm, 2), "launch_us_p10_med_p90": {}}
             del g2
+            # per-launch distribution: each layer alone, one launch per graph replay
+            for L in layers:
+                fns = [(lambda W: lambda: wq.wq_gemm_w4a16(L["A"][M], W, L["N"], G, Y=L["Y"][M], stream=stream))(W)
+                       for W in L["Wp"]]
+                ts = launch_times(torch, stream, fns, 4 * COPIES)
+                per_m[str(M)]["launch_us_p10_med_p90"][f"{L['K']}x{L['N']}"] = pct_us(ts)
+                if (L["K"], L["N"]) == (4096, 4096) and M == 1:
+                    t = float(np.median(ts))
+                    c1_row.update({"us_p10_med_p90": pct_us(ts), "gbs": round(algo_bytes(1, 4096, 4096) / t / 1e9, 1),
+                                   "roofline_frac": round(roofline_time(1, 4096, 4096, hbm_gbs, tflops) / t, 3),
+                                   "speedup_vs_fp16_bound": round(fp16_bound_time(1, 4096, 4096, hbm_gbs) / t, 2)})
+
+    # ---------------------------------------------------------- the dominant kernel's roofline
+    # The calls at M <= 16 run the 16-row small-tile kernel, the largest share of the step's device
+    # time. They are captured in their own graph, in the step's order and weight copies, and timed
+    # like the step (events on the launching stream around whole replays).
+    dom_ms = [M for M in M_SWEEP if M <= 16]
+    dom_calls = [(mi, M, L) for mi, M in enumerate(M_SWEEP) if M in dom_ms for L in layers]
+    gd = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gd, stream=stream):
+            for mi, M, L in dom_calls:
+                wq.wq_gemm_w4a16(L["A"][M], L["Wp"][mi % COPIES], L["N"], G, Y=L["Y"][M], stream=stream)
+        for _ in range(3):
+            gd.replay()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        dom_reps = max(5, min(args.steps, 200))
+        for _ in range(dom_reps):
+            gd.replay()
+        d1.record(stream)
+    stream.synchronize()
+    t_dom = d0.elapsed_time(d1) / 1e3 / dom_reps / len(dom_calls)  # average launch duration
+    b_dom = sum(algo_bytes(M, L["K"], L["N"]) for mi, M, L in dom_calls) / len(dom_calls)
+    del gd
 
     extras = {}
     if rank == 0 and not args.no_breakdown and not args.case:
         extras = extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops)
 
     troof_step = sum(roofline_time(M, K, N, hbm_gbs, tflops) for M in M_SWEEP for (K, N) in LAYERS)
-    achieved = bytes_step / (t_local / args.steps) / 1e9  # per-launch average over the step's launches
+    achieved = b_dom / t_dom / 1e9
     sha = kernel_sha()
     # the recorded figure belongs to the default workload (the layer set) and these kernel sources
     traffic = TRAFFIC["bytes_per_launch"] if TRAFFIC["kernel_sha"] == sha and not args.case else None
@@ -428,10 +566,21 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single"},
         "tflops": round(world * flops_step * args.steps / t / 1e12, 2),
         "roofline_time_frac": round(troof_step / (t_local / args.steps), 3),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
+        "step_roofline": {"time_frac": round(troof_step / (t_local / args.steps), 3),
+                          "note": "the step's headline fraction: the sum over its 32 calls of max(algorithmic "
+                                  "bytes / measured copy bandwidth, flops / measured bf16 peak), over the step's "
+                                  "device time (M = 64 and 128 are past the ridge, so a pure bandwidth fraction "
+                                  "of the whole step would understate them)"},
+        "roofline": {"bound": "hbm", "kernel": "wq_gemm_small<fp16 groups, 16-row tiles> (the step's M <= 16 calls)",
+                     "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(achieved / hbm_gbs, 3), "traffic": traffic,
-                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
-                     "note": f"achieved = algorithmic bytes of the step's {launches_per_step} launches / step device time"},
+                     "traffic_algo_bytes": round(b_dom),
+                     "launch_us": round(t_dom * 1e6, 2),
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth), of measured",
+                     "note": f"achieved = average algorithmic bytes per launch of the {len(dom_calls)} M <= 16 calls "
+                             f"(weights + scales + A + Y) / their average launch duration, CUDA events over "
+                             f"{dom_reps} replays of a graph holding just those calls in the step's order"},
+        "c1_4096x4096_M1": c1_row,
         "e2e": {"value": round(e2e_value, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "copies": "per step one pinned host-to-device copy of all inputs and one "
                                               "device-to-host copy of all results, on their own streams, "
@@ -460,6 +609,25 @@ def _cores():
         return os.cpu_count()
 
 
+def _host_info():
+    """CPU model and the BLAS threads numpy uses (what the oracle's matrix product runs on)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    threads = None
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads") or 0) for i in threadpool_info() if i.get("user_api") == "blas") or None
+    except Exception:
+        pass
+    return {"cpu_model": model, "blas_threads": threads}
+
+
 def _oracle_pairs():
     return [(M, K, N, li) for M in M_SWEEP for li, (K, N) in enumerate(LAYERS)]
 
@@ -478,7 +646,7 @@ def cpu_baseline(n_pairs: int):
     dt = time.perf_counter() - t0
     return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
             "sample": f"{len(pairs)} of the step's 32 (M, layer) calls, fp64 dequantise + numpy BLAS matmul, "
-                      f"{dt:.1f} s"}
+                      f"{dt:.1f} s", **_host_info()}
 
 
 def run_reference(args, rank, world):
@@ -531,7 +699,7 @@ def run_reference(args, rank, world):
            "config": {"workload": WORKLOAD, "layers_KN": LAYERS, "M": M_SWEEP, "g": G,
                       "step": "one (M, layer) call of the layer set on a block of output columns"},
            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": _cores(), "kind": "oracle",
-                            "sample": sample},
+                            "sample": sample, **_host_info()},
            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

@@ -18,6 +18,7 @@ __all__ = [
     "WqError", "lib", "LIB_PATH", "status_string", "wq_version",
     "wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepack", "wq_prepack_w4a8",
     "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a16_noalloc", "wq_gemm_w4a8",
+    "wq_quantize_act", "wq_gemm_w4a8_fp16act",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
@@ -60,6 +61,8 @@ def _load():
         "wq_gemm_w4a16": (I, [P, P, P, I, I, I, I, P]),
         "wq_gemm_w4a16_noalloc": (I, [P, P, P, I, I, I, I, P]),
         "wq_gemm_w4a8": (I, [P, P, P, P, P, P, I, I, I, P]),
+        "wq_quantize_act": (I, [P, I, I, P, P, P]),
+        "wq_gemm_w4a8_fp16act": (I, [P, P, P, P, P, P, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
         "wq_get_device_status": (I, [P]),
@@ -267,6 +270,45 @@ def wq_gemm_w4a8(A: torch.Tensor, sa: torch.Tensor, Wp: torch.Tensor, sw: torch.
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _check(lib.wq_gemm_w4a8(_ptr(A), _ptr(sa), _ptr(Wp), _ptr(sw), _ptr(Y), _ptr(acc_out), M, N, K,
                             _stream(stream)), "wq_gemm_w4a8")
+    return Y
+
+
+def wq_quantize_act(A: torch.Tensor, A_q: torch.Tensor | None = None, sa: torch.Tensor | None = None, stream=None):
+    """fp16 A [M, K] -> (int8 codes [M, K], fp32 per-token scales [M]): symmetric, 127 levels."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    if A_q is not None:
+        _tensor(A_q, torch.int8, "A_q", shape=(M, K))
+    if sa is not None:
+        _tensor(sa, torch.float32, "sa", shape=(M,))
+    _on_one_cuda_device(A=A, A_q=A_q, sa=sa)
+    if A_q is None:
+        A_q = torch.empty((M, K), dtype=torch.int8, device=A.device)
+    if sa is None:
+        sa = torch.empty((M,), dtype=torch.float32, device=A.device)
+    _check(lib.wq_quantize_act(_ptr(A), M, K, _ptr(A_q), _ptr(sa), _stream(stream)), "wq_quantize_act")
+    return A_q, sa
+
+
+def wq_gemm_w4a8_fp16act(A: torch.Tensor, Wp: torch.Tensor, sw: torch.Tensor, N: int,
+                         Y: torch.Tensor | None = None, acc_out: torch.Tensor | None = None,
+                         sa_out: torch.Tensor | None = None, stream=None):
+    """W4A8 on fp16 activations: per-token quantisation of A [M, K] then the W4A8 layer, one call."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    _tensor(sw, torch.float32, "sw", shape=(N,))
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_prepacked_size(K, N, None, "wq_gemm_w4a8_fp16act"))
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    if acc_out is not None:
+        _tensor(acc_out, torch.int32, "acc_out", shape=(M, N))
+    if sa_out is not None:
+        _tensor(sa_out, torch.float32, "sa_out", shape=(M,))
+    _on_one_cuda_device(A=A, sw=sw, Wp=Wp, Y=Y, acc_out=acc_out, sa_out=sa_out)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.wq_gemm_w4a8_fp16act(_ptr(A), _ptr(Wp), _ptr(sw), _ptr(Y), _ptr(acc_out), _ptr(sa_out), M, N, K,
+                                    _stream(stream)), "wq_gemm_w4a8_fp16act")
     return Y
 
 

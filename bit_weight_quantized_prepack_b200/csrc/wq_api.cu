@@ -177,8 +177,18 @@ int check_shape(int K, int N) {
     return WQ_OK;
 }
 
+// Bytes of the activation buffers the W4A8 call with fp16 activations keeps in the workspace
+// after the stream-K part: int8 codes [M, K] and fp32 scales [M], each 256-byte aligned.
+size_t act_quant_bytes(int M, int K) {
+    return ((static_cast<size_t>(M) * K + 255) / 256) * 256 + ((static_cast<size_t>(M) * 4 + 255) / 256) * 256;
+}
+
+// The W4A16 (kind 0) or W4A8 (kind 1) layer. A_fp16 (W4A8 only, may be null): fp16
+// activations that are first quantised per token into the workspace (the codes replace A, the
+// scales go to sa_out when given, else to the workspace).
 int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y,
-             int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream) {
+             int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream, const uint16_t* A_fp16 = nullptr,
+             float* sa_out = nullptr) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M < 0) return WQ_ERR_INVALID_ARG;
@@ -188,9 +198,15 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     if (!Wp) return WQ_ERR_INVALID_ARG;
     if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
     if (M == 0) return WQ_OK;
-    if (!A || !Y || (kind == 1 && (!sa || !sw))) return WQ_ERR_INVALID_ARG;
-    if (!aligned(A, 16) || !aligned(Y, 16) || (acc_out && !aligned(acc_out, 16))) return WQ_ERR_MISALIGNED;
-    if (kind == 1 && (!aligned(sa, 4) || !aligned(sw, 4))) return WQ_ERR_MISALIGNED;
+    if (A_fp16) {
+        if (!Y || !sw) return WQ_ERR_INVALID_ARG;
+        if (!aligned(A_fp16, 16) || (sa_out && !aligned(sa_out, 4))) return WQ_ERR_MISALIGNED;
+    } else {
+        if (!A || !Y || (kind == 1 && (!sa || !sw))) return WQ_ERR_INVALID_ARG;
+        if (!aligned(A, 16) || (kind == 1 && !aligned(sa, 4))) return WQ_ERR_MISALIGNED;
+    }
+    if (!aligned(Y, 16) || (acc_out && !aligned(acc_out, 16))) return WQ_ERR_MISALIGNED;
+    if (kind == 1 && !aligned(sw, 4)) return WQ_ERR_MISALIGNED;
 
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
@@ -201,8 +217,21 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     rc = plan_for(kind, M, N, K, g, *d, &pl);
     if (rc) return rc;
     void* ws = nullptr;
-    rc = get_workspace(dev, stream, workspace_bytes_for(pl), &ws);
+    const size_t gemm_ws = (workspace_bytes_for(pl) + 255) / 256 * 256;
+    rc = get_workspace(dev, stream, gemm_ws + (A_fp16 ? act_quant_bytes(M, K) : 0), &ws);
     if (rc) return rc;
+    if (A_fp16) {
+        int8_t* Aq = reinterpret_cast<int8_t*>(static_cast<uint8_t*>(ws) + gemm_ws);
+        float* sq = sa_out ? sa_out
+                           : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + gemm_ws +
+                                                      (static_cast<size_t>(M) * K + 255) / 256 * 256);
+        if (launch_quantize_act(A_fp16, M, K, Aq, sq, stream) != 0) {
+            cudaGetLastError();
+            return WQ_ERR_CUDA;
+        }
+        A = Aq;
+        sa = sq;
+    }
     ActMaps maps;
     rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1);
     if (rc) return rc;
@@ -448,14 +477,41 @@ int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* 
     return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
 }
 
+int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, void* stream) {
+    if (K <= 0 || M < 0) return WQ_ERR_INVALID_ARG;
+    if (K % 8 || M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return WQ_OK;
+    if (!A || !A_q || !sa) return WQ_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(A_q, 16) || !aligned(sa, 4)) return WQ_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    int rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_quantize_act(A, M, K, A_q, sa, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
+                         float* sa_out, int M, int N, int K, void* stream) {
+    if (M > 0 && !A) return WQ_ERR_INVALID_ARG;
+    return run_gemm(1, nullptr, nullptr, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream), A,
+                    sa_out);
+}
+
 size_t wq_workspace_bytes(int kind, int M, int N, int K) {
-    if (!shape_ok(K, N) || M <= 0 || (kind != 0 && kind != 1)) return 0;
+    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 2) return 0;
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
     DeviceState* d = device_state(&dev);
     if (!d || !d->supported) return 0;
     Plan pl;
-    if (plan_for(kind, M, N, K, kind == 0 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
+    if (plan_for(kind == 0 ? 0 : 1, M, N, K, kind == 0 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
+    if (kind == 2) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_quant_bytes(M, K);
     return workspace_bytes_for(pl);
 }
 

@@ -60,5 +60,6 @@ int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, voi
 int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t st);
 int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st);
 int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st);
+int launch_quantize_act(const uint16_t* A, int M, int K, int8_t* Aq, float* sa, cudaStream_t st);
 
 }  // namespace wq

@@ -119,6 +119,25 @@ WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
 WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw,
                  uint16_t* Y, int32_t* acc_out, int M, int N, int K, void* stream);
 
+/* Per-token activation quantisation, the step before the W4A8 layer ("Atom: Low-bit
+ * Quantization for Efficient and Accurate LLM Serving", method: quantisation parameters of
+ * the activations computed from them at inference time, one scale per token). For each row m
+ * of the fp16 activations A [M, K]: amax = max_k |A[m,k]|, inv = 127 / amax and
+ * sa[m] = amax / 127 (fp32 divisions, round to nearest), A_q[m,k] = round-half-even(A[m,k]
+ * * inv) (fp32 product, round to nearest) clamped to [-127, 127]; a row of zeros gives codes 0
+ * and sa[m] = 0. A must be finite. A_q int8 [M, K] and sa fp32 [M] are caller-owned device
+ * memory. K a positive multiple of 8, 0 <= M <= 2^24; A and A_q 16-byte aligned, sa 4-byte. */
+WQ_API int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, void* stream);
+
+/* The W4A8 layer on fp16 activations: wq_quantize_act into the stream's workspace, then
+ * wq_gemm_w4a8 on the codes and scales, in one call (two launches on `stream`; the layer's
+ * kernel starts streaming weights while the quantisation finishes, and reads the codes only
+ * after it). Y, acc_out and the constraints are those of wq_gemm_w4a8; sa_out (fp32 [M],
+ * nullable) receives the per-token scales. The workspace must hold
+ * wq_workspace_bytes(2, M, N, K) bytes (it grows on first use, or by wq_workspace_reserve). */
+WQ_API int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uint16_t* Y,
+                 int32_t* acc_out, float* sa_out, int M, int N, int K, void* stream);
+
 /* W4A16 without any allocation. No counterpart in the paper: it exists for callers that
  * cannot allocate device memory when they run the layer (an engine that gave all free
  * memory to its own pool at start-up, a plugin whose host framework owns every
@@ -147,7 +166,7 @@ WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
 
 /* ---------------------------------------------------------------- workspace and status
  * Bytes of library workspace one call of the given kind and shape needs
- * (kind 0 = W4A16, 1 = W4A8). */
+ * (kind 0 = W4A16, 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act). */
 WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it
@@ -163,7 +182,7 @@ WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
  * device-side wait expired since the last call. The outputs of the call whose wait expired
  * are undefined, and so are those of every later call on the same stream (or, for
  * wq_gemm_w4a16_noalloc, on the same device) until this function has returned: an expired
- * wait leaves stream-K flags set, and only this function clears them. */
+ * wait can leave stream-K flags set, and only this function clears them. */
 WQ_API int wq_get_device_status(void* stream);
 
 /* ---------------------------------------------------------------- introspection and test hooks

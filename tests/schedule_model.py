@@ -588,3 +588,212 @@ def simulate_large_pair(units, grid, kbs, chunk, slots, issuers, rng=None, pairs
                 moved = True
     stuck = [(st["cta"], name, st["cur"][name]) for st in pairs for name in st["roles"] if name not in st["done"]]
     return problems + stuck
+
+
+# ---------------------------------------------------------------------------- small tiles, A-slot ring
+# A small-tile protocol that was built, passed every GPU parity test and was measured slower
+# than the kernel as built (kept here with its tests as the record of the hazards it needed
+# to avoid): walk index j belongs to residue j % 4 (dequant warp
+# per lane quarter, issuer j % 4, partial buffers 2r, 2r + 1 by the residue's use count); the
+# dequantised k-block goes to A slot j % na. Chunks are fixed by walk position: {0}, {1},
+# {2, 3}, then runs of four; ring slot j % slots with slots a multiple of 4; chunk barrier
+# chunk % NCB. A split tile is finished by the CTA holding its last k-block, which waits for
+# the publish flags of the CTAs holding its other k-blocks (stream-K).
+#
+# na = 4: a slot's previous user is the residue's own previous k-block,
+# so the wait that frees the slot also completes that k-block's partial (RING_PARTIAL_WAIT =
+# "slot"). na = 6 or 8: the partial is
+# signalled on the barrier of its partial buffer, pfull[r][u % 2] ("pfull"); with a single
+# barrier per residue the issuer could complete the residue's next k-block (which the dequant
+# warps signal before reading the previous partial) before the warps wait: two phases ahead.
+# With na not a multiple of 4 a slot's consecutive uses belong to different issuers, so an
+# issuer can reach a slot's use u + 1 before use u was signalled; the slot's full barrier is
+# therefore a pair, afull[a][use % 2], so that a waiter is never two phases behind either.
+RING_READ_DELAY = 1  # the kernel reads a residue's partial after signalling 1 later k-block; 2 is a planted mistake
+RING_PARTIAL_WAIT = "slot"  # "slot" (na = 4) or "pfull" (na = 6, 8); "slot" with na = 6 is a planted mistake
+RING_ONE_PARTIAL_BARRIER = False  # planted mistake: one partial barrier per residue, not one per buffer
+RING_ONE_SLOT_BARRIER = False  # planted mistake: one afull barrier per A slot, not one per use parity
+
+
+def ring_chunk(j):
+    return j if j < 2 else (2 if j < 4 else j // 4 + 2)
+
+
+def ring_chunk_len(c):
+    return 1 if c < 2 else (2 if c == 2 else 4)
+
+
+def _segment_bounds(beg, end, kbs):
+    """(segment, walk index where it ends) for the CTA's walk, last segment first."""
+    out, se = [], 0
+    for seg in segments(beg, end, kbs):
+        se += seg[2] - seg[1] + 1
+        out.append((seg, se))
+    return out
+
+
+def _roles_ring(cta, units, grid, kbs, slots, na, B):
+    beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
+    L = end - beg
+    segs = _segment_bounds(beg, end, kbs)
+
+    def _afull(j):
+        return B["afull"][j % na][0 if RING_ONE_SLOT_BARRIER else (j // na) % 2]
+
+    def dq(quarter, r):
+        j, u = r, 0
+        for seg, se in segs:
+            unread = []  # (walk index, use count) of this segment's k-blocks whose partial is unread
+
+            def read(pj, pu, covered):
+                # covered: with 4 slots the wait that freed this k-block's slot for the residue's next
+                # k-block already saw these MMAs complete; the kernel reads without waiting again,
+                # and the model only checks that the phase is indeed complete
+                if RING_PARTIAL_WAIT == "slot" and covered:
+                    yield ("check", B["aempty"][pj % na], pj // na + 1, pj)
+                elif RING_PARTIAL_WAIT == "slot":
+                    yield ("wait", B["aempty"][pj % na], pj // na + 1, pj)
+                elif RING_ONE_PARTIAL_BARRIER:
+                    yield ("wait", B["pfull"][r][0], pu + 1, pj)
+                else:
+                    yield ("wait", B["pfull"][r][pu % 2], pu // 2 + 1, pj)
+                yield ("part_read", pj)
+
+            while j < se and j < L:
+                c = ring_chunk(j)
+                yield ("wait", B["full"][c % NCB], c // NCB + 1, j)
+                yield ("arrive", B["empty_w"][j % slots])
+                yield ("wait", B["aempty"][j % na], j // na, j)
+                yield ("arrive", _afull(j))
+                unread.append((j, u))
+                while len(unread) > RING_READ_DELAY:
+                    yield from read(*unread.pop(0), covered=True)
+                u += 1
+                j += 4
+            for pj, pu in unread:
+                yield from read(pj, pu, covered=False)
+            yield ("nbar", f"comb{quarter}", 4)
+            yield ("nbar", f"comb{quarter}", 4)
+            tile, kb_lo, kb_hi, owner, whole = seg
+            if not owner:
+                yield ("nbar", "epi", 16)
+                if quarter == 0 and r == 0:
+                    yield ("flag_set", cta)
+            elif not whole:
+                for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                    yield ("flag_wait", cc)
+                yield ("nbar", "epi", 16)
+
+    def issuer(q):
+        for u, j in enumerate(range(q, L, 4)):
+            c = ring_chunk(j)
+            yield ("wait", B["full"][c % NCB], c // NCB + 1, j)
+            if RING_ONE_SLOT_BARRIER:
+                yield ("wait", _afull(j), j // na + 1, j)
+            else:
+                yield ("wait", _afull(j), (j // na) // 2 + 1, j)
+            yield ("part_write", j)
+            yield ("arrive", B["aempty"][j % na])
+            yield ("arrive", B["empty_a"][j % slots])
+            if RING_PARTIAL_WAIT == "pfull":
+                yield ("arrive", B["pfull"][q][0 if RING_ONE_PARTIAL_BARRIER else u % 2])
+
+    def producer(which):
+        uses = [0] * slots
+        j, c = 0, 0
+        while j < L:
+            n = min(ring_chunk_len(c), L - j)
+            for t in range(n):
+                s = (j + t) % slots
+                yield ("wait", B[which][s], uses[s], j + t)
+                uses[s] += 1
+            yield ("arrive", B["full"][c % NCB])
+            j += n
+            c += 1
+
+    roles = {}
+    for w in range(16):
+        roles[f"dq{w}"] = dq(w & 3, w >> 2)
+    for q in range(4):
+        roles[f"iss{q}"] = issuer(q)
+    roles["prod_w"] = producer("empty_w")
+    roles["prod_a"] = producer("empty_a")
+    return roles
+
+
+def simulate_ring(units, grid, kbs, slots, na, rng=None, ctas_only=None):
+    """Like simulate, for the small-tile kernel with the A-slot ring: ("alias", ...) for a wait
+    that passed on the wrong phase, ("race", cta, walk index) for a partial overwritten before
+    all four lane quarters read it, ("unsynchronised", ...) for a partial read whose MMAs were
+    not known to be complete, and the roles left blocked."""
+    assert slots % 4 == 0 and slots >= 4
+    flags = {}
+    if ctas_only is not None:  # CTAs outside the subset count as having published
+        flags = {c: 1 for c in range(grid) if c not in ctas_only}
+    ctas = []
+    for cta in (range(grid) if ctas_only is None else ctas_only):
+        B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
+             "empty_w": [Bar(4, f"empty_w{s}") for s in range(slots)],
+             "empty_a": [Bar(1, f"empty_a{s}") for s in range(slots)],
+             "afull": [[Bar(4, f"afull{a}.{b}") for b in range(2)] for a in range(na)],
+             "aempty": [Bar(1, f"aempty{a}") for a in range(na)],
+             "pfull": [[Bar(1, f"pfull{r}.{b}") for b in range(2)] for r in range(4)]}
+        roles = _roles_ring(cta, units, grid, kbs, slots, na, B)
+        ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
+                     "nbar": defaultdict(list), "reads": defaultdict(int)})
+    problems = []
+    moved = True
+    while moved:
+        moved = False
+        order = [(st, name) for st in ctas for name in st["roles"]]
+        if rng is not None:
+            rng.shuffle(order)
+        for st, name in order:
+            gen = st["roles"][name]
+            steps = 0
+            while name not in st["done"]:
+                if rng is not None and steps >= rng.randint(1, 4):
+                    moved = True
+                    break
+                steps += 1
+                op = st["cur"][name]
+                if op is None:
+                    try:
+                        op = st["cur"][name] = next(gen)
+                    except StopIteration:
+                        st["done"].add(name)
+                        break
+                kind = op[0]
+                if kind == "wait":
+                    if not op[1].ready(op[2]):
+                        break
+                    if op[1].phase != op[2]:
+                        problems.append(("alias", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "flag_wait":
+                    if not flags.get(op[1]):
+                        break
+                elif kind == "arrive":
+                    op[1].arrive()
+                elif kind == "flag_set":
+                    flags[op[1]] = 1
+                elif kind == "check":
+                    if op[1].phase < op[2]:
+                        problems.append(("unsynchronised", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "part_read":
+                    st["reads"][op[1]] += 1
+                elif kind == "part_write":
+                    if op[1] >= 8 and st["reads"][op[1] - 8] < 4:
+                        problems.append(("race", st["cta"], op[1] - 8))
+                elif kind == "nbar":
+                    waiting = st["nbar"][op[1]]
+                    if name not in waiting:
+                        waiting.append(name)
+                    if len(waiting) < op[2]:
+                        break
+                    for other in waiting:
+                        st["cur"][other] = None
+                    st["nbar"][op[1]] = []
+                st["cur"][name] = None
+                moved = True
+    stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+    return problems + stuck

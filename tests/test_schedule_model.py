@@ -1,6 +1,15 @@
-"""CPU test: the small-tile kernel's barrier protocol cannot deadlock for the launch plans it
-uses (every layer shape of the configurations, every ring size the planner can pick, short
-and ragged stream-K ranges). The model lives in schedule_model.py."""
+"""CPU test: the GEMM kernels' barrier protocols cannot deadlock, alias a phase or race on a
+partial for the launch plans they use (every layer shape of the configurations, every ring
+size the planner can pick, short and ragged stream-K ranges). The model lives in
+schedule_model.py.
+
+``simulate`` models the small-tile kernel as built (one A slot per residue) and the candidates
+measured against it; ``simulate_large`` the large-tile kernel. ``simulate_ring`` (the
+``test_ring_*`` tests) models a small-tile protocol that was built, run through every GPU
+parity test and measured slower on B200: dequantised k-blocks in a ring of 4, 6 or 8 A slots
+indexed by walk position, chunks fixed by walk position. Its tests keep the hazards that model
+found before that kernel ran (a slot's consecutive uses by different issuers, a partial barrier
+that the residue's next k-block completes first)."""
 import pytest
 
 from schedule_model import simulate
@@ -308,3 +317,73 @@ def test_cta_pair_model_catches_a_commit_that_reaches_one_cta():
     finally:
         sm.PAIR_MULTICAST_COMMIT = True
     assert any(isinstance(p[1], str) and p[1].startswith("dq1.") for p in problems)
+
+
+# ------------------------------------------------------------------ the measured A-slot ring
+from schedule_model import simulate_ring  # noqa: E402
+
+RING_SHAPES = [(4096, 4096), (4096, 12288), (4096, 22016), (11008, 4096), (8192, 57344), (28672, 8192),
+               (128, 128), (384, 1000), (1024, 136), (256, 8)]
+
+
+def _ring_config(monkeypatch, na):
+    import schedule_model as sm
+    monkeypatch.setattr(sm, "RING_PARTIAL_WAIT", "slot" if na == 4 else "pfull")
+
+
+@pytest.mark.parametrize("K,N", RING_SHAPES)
+@pytest.mark.parametrize("slots,na", [(16, 4), (12, 4), (20, 4), (4, 4), (8, 6), (16, 6), (16, 8)])
+def test_ring_no_deadlock_alias_or_race(K, N, slots, na, monkeypatch):
+    # na = 4: one slot per residue (slots: multiples of 4, 16 at 16-row fp16 tiles, 12 at
+    # 32-row, 20 for int8); 6 and 8 slots: the ring proper
+    _ring_config(monkeypatch, na)
+    units, grid, kbs = _plan(K, N)
+    if K * N > 8192 * 10240 and (slots, na) not in ((16, 4), (12, 4)):
+        pytest.skip("large shapes: the plans the planner picks for them")
+    problems = simulate_ring(units, grid, kbs, slots, na)
+    assert not problems, problems[:5]
+
+
+_RING_BIASES = dict(_BIASES)
+_RING_BIASES["one-issuer-first"] = lambda n: n == "iss3"
+_RING_BIASES["one-issuer-last"] = lambda n: n != "iss0"
+
+
+@pytest.mark.parametrize("K,N", [(8192, 57344), (4096, 22016), (4096, 4096), (1024, 136)])
+@pytest.mark.parametrize("slots,na", [(16, 4), (12, 4), (8, 6), (16, 8)])
+def test_ring_under_skewed_schedules(K, N, slots, na, monkeypatch):
+    import random
+    _ring_config(monkeypatch, na)
+    units, grid, kbs = _plan(K, N)
+    for cta in sorted({0, grid // 2, grid - 1}):
+        for name, first in _RING_BIASES.items():
+            problems = simulate_ring(units, grid, kbs, slots, na, rng=_Biased(first, cta), ctas_only=[cta])
+            assert not problems, (name, cta, problems[:3])
+        for seed in range(2):
+            problems = simulate_ring(units, grid, kbs, slots, na, rng=random.Random(seed), ctas_only=[cta])
+            assert not problems, ("random", seed, cta, problems[:3])
+
+
+def _ring_problems_everywhere(slots=16, na=6):
+    import random
+    units, grid, kbs = _plan(8192, 57344)
+    out = []
+    for cta in (0, 1, grid // 2):
+        for name, first in _RING_BIASES.items():
+            out += simulate_ring(units, grid, kbs, slots, na, rng=_Biased(first, cta), ctas_only=[cta])
+        out += simulate_ring(units, grid, kbs, slots, na, rng=random.Random(cta), ctas_only=[cta])
+    return out
+
+
+@pytest.mark.parametrize("na,flag,value", [
+    (6, "RING_ONE_SLOT_BARRIER", True),       # one afull per A slot: an issuer passes on an older phase
+    (6, "RING_ONE_PARTIAL_BARRIER", True),    # one pfull per residue: the next k-block completes it first
+    (6, "RING_PARTIAL_WAIT", "slot"),         # 6 slots: the slot's barrier belongs to another residue's k-block
+    (6, "RING_READ_DELAY", 2),                # a partial read after the next k-block was signalled
+    (4, "RING_READ_DELAY", 2),
+])
+def test_ring_model_catches_planted_mistake(na, flag, value, monkeypatch):
+    import schedule_model as sm
+    _ring_config(monkeypatch, na)
+    monkeypatch.setattr(sm, flag, value)
+    assert _ring_problems_everywhere(na=na), f"{flag} = {value} went unnoticed at {na} slots"
