@@ -155,21 +155,25 @@ def w4a8_absdot(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray, ch
 # --------------------------------------------------------------------------
 # dynamic per-token activation quantisation (the step before W4A8)
 # --------------------------------------------------------------------------
-def quantize_act(A: np.ndarray):
-    """``(q, sa)``: int8 codes ``q[M,K]`` and fp32 per-token scales ``sa[M]`` of fp16 activations.
+def quantize_act(A: np.ndarray, bits: int = 8):
+    """``(q, sa)``: integer codes ``q[M,K]`` (int8) and fp32 per-token scales ``sa[M]`` of fp16 activations.
 
     "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving", method: the
     activations' quantisation parameters are computed from the activation matrix itself at
-    inference time, one scale per token (row). The pages fix neither the rounding nor the
-    range; the reading used here is the plainest symmetric one, written in fp32 so that the
-    integer codes are decided in one stated precision:
+    inference time, one scale per token (row); the activations are 8-bit for W4A8 and 4-bit
+    for W4A4. The pages fix neither the rounding nor the range; the reading used here is the
+    plainest symmetric one with ``L = 2^(bits-1) - 1`` levels each side (127 for 8 bits, 7 for
+    4), written in fp32 so that the integer codes are decided in one stated precision:
 
     * ``amax[m] = max_k |A[m,k]|`` (exact: fp16 values);
-    * ``inv = fp32(127 / amax)``, ``q = rint(fp32(A[m,k] * inv))`` with ties to even, clamped
-      to ``[-127, 127]`` (-128 is never produced);
-    * ``sa[m] = fp32(amax / 127)``, so ``A[m,k] ~ q[m,k] * sa[m]``;
+    * ``inv = fp32(L / amax)``, ``q = rint(fp32(A[m,k] * inv))`` with ties to even, clamped
+      to ``[-L, L]`` (-L - 1 is never produced);
+    * ``sa[m] = fp32(amax / L)``, so ``A[m,k] ~ q[m,k] * sa[m]``;
     * a row of zeros gives ``q = 0`` and ``sa = 0``.
     """
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    L = np.float32(2 ** (bits - 1) - 1)
     A32 = np.asarray(A, dtype=np.float16).astype(np.float32)
     amax = np.max(np.abs(A32), axis=1)
     q = np.zeros(A32.shape, dtype=np.int8)
@@ -177,10 +181,10 @@ def quantize_act(A: np.ndarray):
     for m in range(A32.shape[0]):
         if amax[m] == 0:
             continue
-        inv = np.float32(127.0) / amax[m]                     # fp32 division, round to nearest
-        t = A32[m] * inv                                      # fp32 products, round to nearest
-        q[m] = np.clip(np.rint(t), -127, 127).astype(np.int8)  # ties to even
-        sa[m] = amax[m] / np.float32(127.0)
+        inv = L / amax[m]                                  # fp32 division, round to nearest
+        t = A32[m] * inv                                   # fp32 products, round to nearest
+        q[m] = np.clip(np.rint(t), -L, L).astype(np.int8)  # ties to even
+        sa[m] = amax[m] / L
     return q, sa
 
 

@@ -281,23 +281,32 @@ def pin_blob_layout_golden(o):
 
 
 # ---------------------------------------------------------------- per-token activation quantisation
-def golden_act_quant():
+def golden_act_quant(bits=8):
     out = []
     for line in _rows("act_quant.txt"):
-        acts, codes, sa = [x.strip() for x in line.split("|")]
+        parts = [x.strip() for x in line.split("|")]
+        row_bits = 8
+        if parts[0].startswith("bits="):
+            row_bits = int(parts[0][5:])
+            parts = parts[1:]
+        if row_bits != bits:
+            continue
+        acts, codes, sa = parts
         out.append((np.array([float(x) for x in acts.split()], np.float16),
                     [int(x) for x in codes.split()], None if sa == "-" else float(sa)))
     return out
 
 
 def pin_act_quant_golden(o):
-    rows = golden_act_quant()
-    q, sa = o.quantize_act(np.stack([r[0] for r in rows]))
-    assert q.dtype == np.int8 and sa.dtype == np.float32
-    for i, (a, codes, s) in enumerate(rows):
-        assert q[i].tolist() == codes, (i, q[i].tolist(), codes)
-        if s is not None:
-            assert float(sa[i]) == s, (i, float(sa[i]), s)
+    for bits in (8, 4):
+        rows = golden_act_quant(bits)
+        assert rows
+        q, sa = o.quantize_act(np.stack([r[0] for r in rows]), bits=bits)
+        assert q.dtype == np.int8 and sa.dtype == np.float32
+        for i, (a, codes, s) in enumerate(rows):
+            assert q[i].tolist() == codes, (bits, i, q[i].tolist(), codes)
+            if s is not None:
+                assert float(sa[i]) == s, (bits, i, float(sa[i]), s)
 
 
 def pin_act_quant_bounds(o):
@@ -308,19 +317,20 @@ def pin_act_quant_bounds(o):
     A = (rng.standard_normal((6, 96)) * np.array([[1e-3], [1.0], [30.0], [1e3], [0.5], [7.0]])).astype(np.float16)
     A[4, :] = 0
     A[4, 17] = -0.25
-    q, sa = o.quantize_act(A)
-    for m in range(A.shape[0]):
-        amax = max(abs(Fraction(float(x))) for x in A[m])
-        assert abs(Fraction(float(sa[m])) - amax / 127) <= amax / 127 * Fraction(2.0 ** -24)
-        for k in range(A.shape[1]):
-            a = Fraction(float(A[m, k]))
-            exact = a * 127 / amax
-            assert abs(int(q[m, k])) <= 127
-            assert abs(Fraction(int(q[m, k])) - exact) <= Fraction(1, 2) + 256 * Fraction(2.0 ** -24), (m, k)
-            if abs(a) == amax:
-                assert abs(int(q[m, k])) == 127
-            if q[m, k] != 0:
-                assert (q[m, k] > 0) == (a > 0)
+    for bits, L in ((8, 127), (4, 7)):
+        q, sa = o.quantize_act(A, bits=bits)
+        for m in range(A.shape[0]):
+            amax = max(abs(Fraction(float(x))) for x in A[m])
+            assert abs(Fraction(float(sa[m])) - amax / L) <= amax / L * Fraction(2.0 ** -24)
+            for k in range(A.shape[1]):
+                a = Fraction(float(A[m, k]))
+                exact = a * L / amax
+                assert abs(int(q[m, k])) <= L
+                assert abs(Fraction(int(q[m, k])) - exact) <= Fraction(1, 2) + 2 * L * Fraction(2.0 ** -24), (bits, m, k)
+                if abs(a) == amax:
+                    assert abs(int(q[m, k])) == L
+                if q[m, k] != 0:
+                    assert (q[m, k] > 0) == (a > 0)
 
 
 ALL_PINS = [

@@ -87,23 +87,24 @@ def _mut_tolerance_rel_dropped(mp):
 def _mut_act_round_half_up(mp):
     orig = O.quantize_act
 
-    def quantize_act(A):
+    def quantize_act(A, bits=8):
         A32 = np.asarray(A, np.float16).astype(np.float32)
         amax = np.max(np.abs(A32), axis=1)
         q = np.zeros(A32.shape, np.int8)
         sa = np.zeros(A32.shape[0], np.float32)
+        L = np.float32(2 ** (bits - 1) - 1)
         for m in range(A32.shape[0]):
             if amax[m]:
-                t = A32[m] * (np.float32(127.0) / amax[m])
-                q[m] = np.clip(np.floor(t + np.float32(0.5)), -127, 127).astype(np.int8)
-                sa[m] = amax[m] / np.float32(127.0)
+                t = A32[m] * (L / amax[m])
+                q[m] = np.clip(np.floor(t + np.float32(0.5)), -L, L).astype(np.int8)
+                sa[m] = amax[m] / L
         return q, sa
     del orig
     mp.setattr(O, "quantize_act", quantize_act)
 
 
 def _mut_act_range_128(mp):
-    def quantize_act(A):
+    def quantize_act(A, bits=8):
         A32 = np.asarray(A, np.float16).astype(np.float32)
         amax = np.max(np.abs(A32), axis=1)
         q = np.zeros(A32.shape, np.int8)
@@ -117,7 +118,7 @@ def _mut_act_range_128(mp):
 
 
 def _mut_act_scale_per_tensor(mp):
-    def quantize_act(A):
+    def quantize_act(A, bits=8):
         A32 = np.asarray(A, np.float16).astype(np.float32)
         amax = np.float32(np.max(np.abs(A32)))
         if amax == 0:
@@ -127,7 +128,25 @@ def _mut_act_scale_per_tensor(mp):
     mp.setattr(O, "quantize_act", quantize_act)
 
 
-MUTATIONS = [_mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
+def _mut_act_4bit_8_levels(mp):
+    orig = O.quantize_act
+
+    def quantize_act(A, bits=8):
+        if bits == 8:
+            return orig(A, 8)
+        A32 = np.asarray(A, np.float16).astype(np.float32)
+        amax = np.max(np.abs(A32), axis=1)
+        q = np.zeros(A32.shape, np.int8)
+        sa = np.zeros(A32.shape[0], np.float32)
+        for m in range(A32.shape[0]):
+            if amax[m]:
+                q[m] = np.clip(np.rint(A32[m] * (np.float32(8.0) / amax[m])), -8, 7).astype(np.int8)
+                sa[m] = amax[m] / np.float32(8.0)
+        return q, sa
+    mp.setattr(O, "quantize_act", quantize_act)
+
+
+MUTATIONS = [_mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
              _mut_k_reversed, _mut_sign_flipped, _mut_w4a8_no_zero_point, _mut_w4a8_sw_dropped,
              _mut_absdot_signed, _mut_tolerance_rel_dropped]
 
