@@ -43,6 +43,7 @@ import numpy as np
 __all__ = [
     "unpack_codes", "dequant", "w4a16", "w4a16_absdot", "w4a16_entry",
     "tolerance", "w4a8_acc", "w4a8", "w4a8_absdot", "quantize_act",
+    "dequant_zp", "w4a16_zp", "w4a16_zp_absdot", "prepack_w4a16_zp", "prepacked_bytes_w4a16_zp", "unprepack_w4a16_zp",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
 ]
@@ -150,6 +151,50 @@ def w4a8_absdot(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray, ch
         wq = np.abs(unpack_codes(np.asarray(Q)[:, n0:n1]).astype(np.float64) - ZERO_POINT)
         out[:, n0:n1] = A64 @ wq
     return out * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+
+
+# --------------------------------------------------------------------------
+# asymmetric groups: a zero point per group and column
+# --------------------------------------------------------------------------
+def dequant_zp(q: np.ndarray, s: np.ndarray, z: np.ndarray, g: int) -> np.ndarray:
+    """``W[k,n] = (q[k,n] - z[k // g, n]) * s[k // g, n]`` in float64 (exact).
+
+    "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving", method
+    (fine-grained group quantisation), read with an asymmetric zero point per group and
+    column (the GPTQ-style format the pages leave open): a 4-bit code ``q`` and a 4-bit zero
+    ``z`` (0..15) per group, so that a group's weights need not be centred on code 8.
+    ``z = 8`` everywhere is the symmetric layer of ``dequant``.
+    """
+    K, N = q.shape
+    if K % g:
+        raise ValueError("g must divide K")
+    group = np.arange(K) // g
+    zz = np.asarray(z, dtype=np.float64)[group, :]
+    return (q.astype(np.float64) - zz) * np.asarray(s, dtype=np.float64)[group, :]
+
+
+def w4a16_zp(A: np.ndarray, Q: np.ndarray, s: np.ndarray, z: np.ndarray, g: int, chunk: int = 4096) -> np.ndarray:
+    """``Y = A . W`` with ``W = dequant_zp(...)``, in float64, chunked along N."""
+    A64 = np.asarray(A, dtype=np.float64)
+    N = np.asarray(Q).shape[1]
+    Y = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        Y[:, n0:n1] = A64 @ dequant_zp(unpack_codes(np.asarray(Q)[:, n0:n1]), np.asarray(s)[:, n0:n1],
+                                       np.asarray(z)[:, n0:n1], g)
+    return Y
+
+
+def w4a16_zp_absdot(A: np.ndarray, Q: np.ndarray, s: np.ndarray, z: np.ndarray, g: int, chunk: int = 4096) -> np.ndarray:
+    """``sum_k |A[m,k] * W[k,n]|`` for the asymmetric weights."""
+    A64 = np.abs(np.asarray(A, dtype=np.float64))
+    N = np.asarray(Q).shape[1]
+    out = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        out[:, n0:n1] = A64 @ np.abs(dequant_zp(unpack_codes(np.asarray(Q)[:, n0:n1]), np.asarray(s)[:, n0:n1],
+                                                np.asarray(z)[:, n0:n1], g))
+    return out
 
 
 # --------------------------------------------------------------------------
@@ -331,3 +376,53 @@ def unprepack_w4a8(Wp: np.ndarray, K: int, N: int) -> np.ndarray:
     nt, kt = -(-N // TILE_N), K // TILE_K
     words = np.ascontiguousarray(np.asarray(Wp, dtype=np.uint8)).view(np.uint32).reshape(nt, kt, -1)
     return _codes_from_words(words, NIBBLE_POS_W4A8, K, N)
+
+
+# --------------------------------------------------------------------------
+# the asymmetric prepacked format: the W4A16 blob followed by the blob's zero points
+# --------------------------------------------------------------------------
+def prepacked_bytes_w4a16_zp(K: int, N: int, g: int) -> int:
+    """Blobs of ``8192 + 256 * slots + 128 * slots`` bytes (codes, fp16 scales, uint8 zeros);
+    ``g`` below ``K`` (one scale and one zero per group and column)."""
+    _check_kn(K, N)
+    slots = _group_slots(K, g)
+    if slots == 0:
+        raise ValueError("zero points need g < K")
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    return nt * kt * (TILE_N * TILE_K // 2 + 3 * TILE_N * slots)
+
+
+def prepack_w4a16_zp(Q: np.ndarray, s: np.ndarray, z: np.ndarray, g: int) -> np.ndarray:
+    """Blob ``(nt, kt)`` = the W4A16 blob of ``prepack_w4a16`` (codes, then ``slots`` rows of 128
+    fp16 scales) followed by ``slots`` rows of 128 uint8 zero points, row ``u`` holding
+    ``z[(kt*128 + u*g) // g, nt*128 + r]`` for ``g <= 128`` and ``z[(kt*128) // g, ...]`` for
+    larger ``g``. Padded columns get zero point 8 and scale 0."""
+    K = np.asarray(Q).shape[0] * 8
+    N = np.asarray(Q).shape[1]
+    slots = _group_slots(K, g)
+    if slots == 0:
+        raise ValueError("zero points need g < K")
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    base = prepack_w4a16(Q, s, g).reshape(nt, kt, -1)
+    zp = np.full((np.asarray(z).shape[0], nt * TILE_N), ZERO_POINT, dtype=np.uint8)
+    zp[:, :N] = np.asarray(z, dtype=np.uint8)
+    krow = np.arange(kt)[:, None] * TILE_K + np.arange(slots)[None, :] * g
+    zz = zp[krow // g]                                                   # [kt, slots, nt*128]
+    zz = zz.reshape(kt, slots, nt, TILE_N).transpose(2, 0, 1, 3).reshape(nt, kt, -1)
+    out = np.concatenate([base, zz], axis=2).reshape(-1)
+    assert out.nbytes == prepacked_bytes_w4a16_zp(K, N, g)
+    return out
+
+
+def unprepack_w4a16_zp(Wp: np.ndarray, K: int, N: int, g: int):
+    """Inverse of ``prepack_w4a16_zp``: ``(q[K,N], s[K/g,N] fp16, z[K/g,N] uint8)``."""
+    slots = _group_slots(K, g)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    base_bytes = TILE_N * TILE_K // 2 + 2 * TILE_N * slots
+    blob = np.asarray(Wp, dtype=np.uint8).reshape(nt, kt, base_bytes + TILE_N * slots)
+    q, s = unprepack_w4a16(np.ascontiguousarray(blob[:, :, :base_bytes]).reshape(-1), K, N, g)
+    zz = blob[:, :, base_bytes:].reshape(nt, kt, slots, TILE_N).transpose(1, 2, 0, 3).reshape(kt * slots, nt * TILE_N)
+    krow = (np.arange(kt)[:, None] * TILE_K + np.arange(slots)[None, :] * g).reshape(-1)
+    z = np.zeros((K // g, nt * TILE_N), dtype=np.uint8)
+    z[krow // g] = zz
+    return q, s, z[:, :N]

@@ -14,6 +14,8 @@ with the fact it is pinned to:
 * W4A8: the integer accumulator against Python integer loops;
 * per-token activation quantisation: hand-worked rows (``tests/golden/act_quant.txt``)
   and exact rational bounds;
+* asymmetric groups (zero points): hand-worked layers (``tests/golden/zp_examples.txt``),
+  exact rational brute force, and zero point 8 reproducing the symmetric layer;
 * the prepacked layout: single codes and scales placed by hand-worked byte
   offsets (``tests/golden/blob_layout.txt``), independent of the oracle's own
   inverse of its layout.
@@ -255,6 +257,17 @@ def pin_blob_layout_golden(o):
     # one code (value 3 among 8s) or one scale (among zeros) at a time: exactly the bytes the
     # hand-worked table names change, to exactly the values it implies
     for kind, what, K, N, g, a, b, offs, half in golden_layout():
+        if what == "zero":
+            q = np.full((K, N), 8, np.uint8)
+            s = np.zeros((K // g, N), np.float16)
+            z = np.full((K // g, N), 8, np.uint8)
+            base = o.prepack_w4a16_zp(synth.pack_q(q), s, z, g)
+            z[a, b] = 3
+            Wp = o.prepack_w4a16_zp(synth.pack_q(q), s, z, g)
+            diff = np.nonzero(Wp != base)[0].tolist()
+            assert diff == offs, (K, N, g, a, b, diff, offs)
+            assert all(int(Wp[x]) == 3 for x in offs)
+            continue
         if what == "code":
             q = np.full((K, N), 8, np.uint8)
             base_q = q.copy()
@@ -262,6 +275,10 @@ def pin_blob_layout_golden(o):
             if kind == "w4a16":
                 s = np.zeros((K // g, N), np.float16)
                 Wp, base = o.prepack_w4a16(synth.pack_q(q), s, g), o.prepack_w4a16(synth.pack_q(base_q), s, g)
+            elif kind == "w4a16zp":
+                s = np.zeros((K // g, N), np.float16)
+                z = np.full((K // g, N), 8, np.uint8)
+                Wp, base = o.prepack_w4a16_zp(synth.pack_q(q), s, z, g), o.prepack_w4a16_zp(synth.pack_q(base_q), s, z, g)
             else:
                 Wp, base = o.prepack_w4a8(synth.pack_q(q)), o.prepack_w4a8(synth.pack_q(base_q))
             diff = np.nonzero(Wp != base)[0].tolist()
@@ -333,9 +350,56 @@ def pin_act_quant_bounds(o):
                     assert (q[m, k] > 0) == (a > 0)
 
 
+# ---------------------------------------------------------------- asymmetric groups (zero points)
+def golden_zp():
+    out = []
+    for line in _rows("zp_examples.txt"):
+        words, scales, zeros, g, acts, expect = [p.strip() for p in line.split("|")]
+        out.append({"Q": np.array([int(w, 16) for w in words.split()], np.uint32).view(np.int32).reshape(-1, 1),
+                    "s": np.array([float(x) for x in scales.split()], np.float16).reshape(-1, 1),
+                    "z": np.array([int(x) for x in zeros.split()], np.uint8).reshape(-1, 1),
+                    "g": int(g), "A": np.array([float(x) for x in acts.split()], np.float16).reshape(1, -1),
+                    "y": float(expect)})
+    return out
+
+
+def pin_zp_golden(o):
+    for ex in golden_zp():
+        y = o.w4a16_zp(ex["A"], ex["Q"], ex["s"], ex["z"], ex["g"])
+        assert y.shape == (1, 1) and y[0, 0] == ex["y"], (y, ex["y"])
+
+
+def pin_zp_bruteforce(o):
+    # exact rationals from the raw codes and zeros of the generator, M, K, N all different
+    for (M, K, N, g, seed) in [(3, 64, 5, 16, 1), (2, 48, 7, 48, 2), (1, 128, 9, 32, 4)]:
+        d = synth.w4a16_inputs(K, N, g, M, seed=seed)
+        z = np.random.default_rng(seed + 100).integers(0, 16, (K // g, N)).astype(np.uint8)
+        y = o.w4a16_zp(d["A"], d["Q"], d["s"], z, g)
+        ad = o.w4a16_zp_absdot(d["A"], d["Q"], d["s"], z, g)
+        assert y.shape == (M, N)
+        for m in range(M):
+            for n in range(N):
+                exact = Fraction(0)
+                absdot = Fraction(0)
+                for k in range(K):
+                    t = Fraction(float(d["A"][m, k])) * (int(d["q"][k, n]) - int(z[k // g, n])) * Fraction(float(d["s"][k // g, n]))
+                    exact += t
+                    absdot += abs(t)
+                assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(K * 2.0 ** -52) * absdot + Fraction(1e-300)
+                assert abs(Fraction(float(ad[m, n])) - absdot) <= Fraction(K * 2.0 ** -52) * absdot + Fraction(1e-300)
+
+
+def pin_zp_eight_is_symmetric(o):
+    # zero point 8 everywhere is the symmetric layer, bit for bit
+    d = synth.w4a16_inputs(256, 40, 64, 3, seed=14)
+    z = np.full((4, 40), 8, np.uint8)
+    assert np.array_equal(o.w4a16_zp(d["A"], d["Q"], d["s"], z, 64), o.w4a16(d["A"], d["Q"], d["s"], 64))
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
     pin_row_permutation, pin_linearity, pin_tolerance_formula, pin_bruteforce_w4a8, pin_w4a8_extremes,
-    pin_blob_layout_golden, pin_act_quant_golden, pin_act_quant_bounds,
+    pin_blob_layout_golden, pin_act_quant_golden, pin_act_quant_bounds, pin_zp_golden, pin_zp_bruteforce,
+    pin_zp_eight_is_symmetric,
 ]

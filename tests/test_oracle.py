@@ -146,7 +146,18 @@ def _mut_act_4bit_8_levels(mp):
     mp.setattr(O, "quantize_act", quantize_act)
 
 
-MUTATIONS = [_mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
+def _mut_zp_ignored(mp):
+    mp.setattr(O, "dequant_zp", lambda q, s, z, g: O.dequant(q, s, g))
+
+
+def _mut_zp_sign(mp):
+    def dequant_zp(q, s, z, g):
+        grp = np.arange(q.shape[0]) // g
+        return (q.astype(np.float64) + np.asarray(z, np.float64)[grp, :] - 16) * np.asarray(s, np.float64)[grp, :]
+    mp.setattr(O, "dequant_zp", dequant_zp)
+
+
+MUTATIONS = [_mut_zp_ignored, _mut_zp_sign, _mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
              _mut_k_reversed, _mut_sign_flipped, _mut_w4a8_no_zero_point, _mut_w4a8_sw_dropped,
              _mut_absdot_signed, _mut_tolerance_rel_dropped]
 
@@ -174,6 +185,17 @@ def test_prepack_roundtrip(K, N, g):
     assert Wp.nbytes == O.prepacked_bytes_w4a16(K, N, g)
     q, s = O.unprepack_w4a16(Wp, K, N, g)
     assert np.array_equal(q, d["q"])
+    assert np.array_equal(s.view(np.uint16), d["s"].view(np.uint16))
+
+
+@pytest.mark.parametrize("K,N,g", [(256, 128, 128), (256, 200, 64), (384, 136, 32), (512, 8, 256)])
+def test_prepack_zp_roundtrip(K, N, g):
+    d = synth.w4a16_inputs(K, N, g, 1, seed=K + N + g)
+    z = np.random.default_rng(K).integers(0, 16, (K // g, N)).astype(np.uint8)
+    Wp = O.prepack_w4a16_zp(d["Q"], d["s"], z, g)
+    assert Wp.nbytes == O.prepacked_bytes_w4a16_zp(K, N, g)
+    q, s, zz = O.unprepack_w4a16_zp(Wp, K, N, g)
+    assert np.array_equal(q, d["q"]) and np.array_equal(zz, z)
     assert np.array_equal(s.view(np.uint16), d["s"].view(np.uint16))
 
 
