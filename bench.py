@@ -291,8 +291,9 @@ def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
             out["w4a8"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "gbs": round(b / t / 1e9, 1),
                                            "tops": round(ops / t / 1e12, 1), "roofline_frac": round(troof / t, 3)}
         del Wps
-    # the W4A8 layer on fp16 activations (per-token quantisation + the int8 layer, one call) and the
-    # quantisation kernel alone (HBM-bound: 2MK bytes read, MK + 4M written)
+    # the layer on fp16 activations (per-token quantisation to 8 bits, W4A8, or to 4 bits, W4A4, then
+    # the int8 layer, one call) and the 8-bit quantisation kernel alone (HBM-bound: 2MK bytes read,
+    # MK + 4M written)
     out["w4a8_fp16act"] = {}
     for K, N in W4A8_LAYERS:
         d = synth.w4a8_inputs(K, N, 1, seed=13)
@@ -310,7 +311,10 @@ def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
                             lambda r: wq.wq_gemm_w4a8_fp16act(A16, Wps[r % copies], sw, N, Y=Y, stream=stream), 2 * copies)
             tq = _graph_time(torch, stream, lambda r: wq.wq_quantize_act(A16, Aq, sa, stream=stream), 8)
             bq = 3 * M * K + 4 * M
-            out["w4a8_fp16act"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "quantize_us": round(tq * 1e6, 2),
+            t4 = _graph_time(torch, stream, lambda r: wq.wq_gemm_w4a8_fp16act(A16, Wps[r % copies], sw, N, Y=Y,
+                                                                                stream=stream, act_bits=4), 2 * copies)
+            out["w4a8_fp16act"][f"{K}x{N}_M{M}"] = {"us": round(t * 1e6, 2), "w4a4_us": round(t4 * 1e6, 2),
+                                                   "quantize_us": round(tq * 1e6, 2),
                                                    "quantize_gbs": round(bq / tq / 1e9, 1)}
         del Wps
     out["peaks"] = {"tensor_tflops": tflops, "int8_tops": int8_peak,

@@ -19,6 +19,7 @@ __all__ = [
     "wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepack", "wq_prepack_w4a8",
     "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a16_noalloc", "wq_gemm_w4a8",
     "wq_quantize_act", "wq_gemm_w4a8_fp16act",
+    "wq_prepacked_bytes_zp", "wq_prepack_zp", "wq_unpack_zp", "wq_gemm_w4a16_zp",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
@@ -61,8 +62,12 @@ def _load():
         "wq_gemm_w4a16": (I, [P, P, P, I, I, I, I, P]),
         "wq_gemm_w4a16_noalloc": (I, [P, P, P, I, I, I, I, P]),
         "wq_gemm_w4a8": (I, [P, P, P, P, P, P, I, I, I, P]),
-        "wq_quantize_act": (I, [P, I, I, P, P, P]),
-        "wq_gemm_w4a8_fp16act": (I, [P, P, P, P, P, P, I, I, I, P]),
+        "wq_quantize_act": (I, [P, I, I, I, P, P, P]),
+        "wq_prepacked_bytes_zp": (Z, [I, I, I]),
+        "wq_prepack_zp": (I, [P, P, P, I, I, I, P, P]),
+        "wq_unpack_zp": (I, [P, I, I, I, P, P, P, P]),
+        "wq_gemm_w4a16_zp": (I, [P, P, P, I, I, I, I, P]),
+        "wq_gemm_w4a8_fp16act": (I, [P, P, P, P, P, P, I, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
         "wq_get_device_status": (I, [P]),
@@ -273,8 +278,71 @@ def wq_gemm_w4a8(A: torch.Tensor, sa: torch.Tensor, Wp: torch.Tensor, sw: torch.
     return Y
 
 
-def wq_quantize_act(A: torch.Tensor, A_q: torch.Tensor | None = None, sa: torch.Tensor | None = None, stream=None):
-    """fp16 A [M, K] -> (int8 codes [M, K], fp32 per-token scales [M]): symmetric, 127 levels."""
+def wq_prepacked_bytes_zp(K: int, N: int, g: int) -> int:
+    return lib.wq_prepacked_bytes_zp(K, N, g)
+
+
+def wq_prepack_zp(Q: torch.Tensor, s: torch.Tensor, z: torch.Tensor, g: int, Wp: torch.Tensor | None = None,
+                  stream=None):
+    """Q int32 [K/8, N], s fp16 [K/g, N], zero points z uint8 [K/g, N] (0..15) -> the zero-point buffer."""
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    if g <= 0 or K % g or g == K:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_prepack_zp")
+    _tensor(s, torch.float16, "s", shape=(K // g, N))
+    _tensor(z, torch.uint8, "z", shape=(K // g, N))
+    nbytes = wq_prepacked_bytes_zp(K, N, g)
+    if nbytes == 0:
+        raise WqError(WQ_ERR_INVALID_ARG if K % 128 == 0 else WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack_zp")
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Q=Q, s=s, z=z, Wp=Wp)
+    if Wp is None:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack_zp(_ptr(Q), _ptr(s), _ptr(z), K, N, g, _ptr(Wp), _stream(stream)), "wq_prepack_zp")
+    return Wp
+
+
+def wq_unpack_zp(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
+    """Inverse of wq_prepack_zp: (Q int32 [K/8, N], s fp16 [K/g, N], z uint8 [K/g, N])."""
+    if g <= 0 or K <= 0 or K % g or g == K:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_unpack_zp")
+    nbytes = wq_prepacked_bytes_zp(K, N, g)
+    if nbytes == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_unpack_zp")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Wp=Wp)
+    Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
+    s = torch.empty((K // g, N), dtype=torch.float16, device=Wp.device)
+    z = torch.empty((K // g, N), dtype=torch.uint8, device=Wp.device)
+    _check(lib.wq_unpack_zp(_ptr(Wp), K, N, g, _ptr(Q), _ptr(s), _ptr(z), _stream(stream)), "wq_unpack_zp")
+    return Q, s, z
+
+
+def wq_gemm_w4a16_zp(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor | None = None, stream=None):
+    """Y fp16 [M, N] = A fp16 [M, K] . ((q - z) * s), from the zero-point buffer."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    if g <= 0 or K % g or g == K:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_gemm_w4a16_zp")
+    nbytes = wq_prepacked_bytes_zp(K, N, g)
+    if nbytes == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_gemm_w4a16_zp")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    _on_one_cuda_device(A=A, Wp=Wp, Y=Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.wq_gemm_w4a16_zp(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)), "wq_gemm_w4a16_zp")
+    return Y
+
+
+def wq_quantize_act(A: torch.Tensor, A_q: torch.Tensor | None = None, sa: torch.Tensor | None = None, stream=None,
+                    bits: int = 8):
+    """fp16 A [M, K] -> (int8 codes [M, K], fp32 per-token scales [M]): symmetric, 127 levels
+    each side for bits = 8, 7 for bits = 4 (codes held one per int8)."""
     M, K = _matrix(A, "A")
     _tensor(A, torch.float16, "A")
     if A_q is not None:
@@ -286,14 +354,15 @@ def wq_quantize_act(A: torch.Tensor, A_q: torch.Tensor | None = None, sa: torch.
         A_q = torch.empty((M, K), dtype=torch.int8, device=A.device)
     if sa is None:
         sa = torch.empty((M,), dtype=torch.float32, device=A.device)
-    _check(lib.wq_quantize_act(_ptr(A), M, K, _ptr(A_q), _ptr(sa), _stream(stream)), "wq_quantize_act")
+    _check(lib.wq_quantize_act(_ptr(A), M, K, bits, _ptr(A_q), _ptr(sa), _stream(stream)), "wq_quantize_act")
     return A_q, sa
 
 
 def wq_gemm_w4a8_fp16act(A: torch.Tensor, Wp: torch.Tensor, sw: torch.Tensor, N: int,
                          Y: torch.Tensor | None = None, acc_out: torch.Tensor | None = None,
-                         sa_out: torch.Tensor | None = None, stream=None):
-    """W4A8 on fp16 activations: per-token quantisation of A [M, K] then the W4A8 layer, one call."""
+                         sa_out: torch.Tensor | None = None, stream=None, act_bits: int = 8):
+    """The layer on fp16 activations: per-token quantisation of A [M, K] to act_bits (8: W4A8,
+    4: W4A4) then the layer on the int8 tensor cores, one call."""
     M, K = _matrix(A, "A")
     _tensor(A, torch.float16, "A")
     _tensor(sw, torch.float32, "sw", shape=(N,))
@@ -308,7 +377,7 @@ def wq_gemm_w4a8_fp16act(A: torch.Tensor, Wp: torch.Tensor, sw: torch.Tensor, N:
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _check(lib.wq_gemm_w4a8_fp16act(_ptr(A), _ptr(Wp), _ptr(sw), _ptr(Y), _ptr(acc_out), _ptr(sa_out), M, N, K,
-                                    _stream(stream)), "wq_gemm_w4a8_fp16act")
+                                    act_bits, _stream(stream)), "wq_gemm_w4a8_fp16act")
     return Y
 
 

@@ -133,13 +133,14 @@ size_t workspace_bytes_for(const Plan& pl) {
     return 4096 + static_cast<size_t>(pl.grid) * pl.tile_m * kTileN * 4;
 }
 
+// kind 0: W4A16; 1: W4A8; 3: W4A16 with a zero point per group (g < K).
 int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* pl) {
     int mode;
     int slots = 0;
-    if (kind == 0) {
+    if (kind == 0 || kind == 3) {
         slots = scale_slots(K, g);
-        if (slots < 0) return WQ_ERR_INVALID_ARG;
-        mode = slots > 0 ? kModeGroup : kModeChannel;
+        if (slots < 0 || (kind == 3 && slots == 0)) return WQ_ERR_INVALID_ARG;
+        mode = kind == 3 ? kModeGroupZP : (slots > 0 ? kModeGroup : kModeChannel);
     } else {
         mode = kModeW4A8;
     }
@@ -188,12 +189,13 @@ size_t act_quant_bytes(int M, int K) {
 // scales go to sa_out when given, else to the workspace).
 int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y,
              int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream, const uint16_t* A_fp16 = nullptr,
-             float* sa_out = nullptr) {
+             float* sa_out = nullptr, int act_bits = 8) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M < 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if (kind == 0 && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if ((kind == 0 || kind == 3) && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (kind == 3 && scale_slots(K, g) == 0) return WQ_ERR_INVALID_ARG;
     if (kind == 1 && K > kMaxKW4A8) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (!Wp) return WQ_ERR_INVALID_ARG;
     if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
@@ -225,7 +227,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
         float* sq = sa_out ? sa_out
                            : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + gemm_ws +
                                                       (static_cast<size_t>(M) * K + 255) / 256 * 256);
-        if (launch_quantize_act(A_fp16, M, K, Aq, sq, stream) != 0) {
+        if (launch_quantize_act(A_fp16, M, K, act_bits, Aq, sq, stream) != 0) {
             cudaGetLastError();
             return WQ_ERR_CUDA;
         }
@@ -261,11 +263,13 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.chunk = pl.chunk;
     a.act_slot = pl.act_slot;
     a.blob_bytes = pl.blob_bytes;
-    a.group_rows = (kind == 0 && g < kTileK) ? g : kTileK;
+    a.group_rows = ((kind == 0 || kind == 3) && g < kTileK) ? g : kTileK;
     a.small = pl.small ? 1 : 0;
-    // large tiles round (q - 8) * s to fp16 in the dequant; small tiles apply a group scale of
+    // large tiles round (q - z) * s to fp16 in the dequant; small tiles apply a group scale of
     // g >= 128 to each k-block's fp32 partial instead (g = 32, 64 stay in the dequant)
-    a.scale_in_dequant = (pl.mode == kModeGroup && (!pl.small || g < kTileK)) ? 1 : 0;
+    a.scale_in_dequant =
+        ((pl.mode == kModeGroup || pl.mode == kModeGroupZP) && (!pl.small || g < kTileK)) ? 1 : 0;
+    a.zp_offset = (pl.mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16(scale_slots(K, g))) : 0;
     a.units = pl.units;
     a.grid = pl.grid;
     a.timeout_ns = g_timeout_ns;
@@ -410,7 +414,7 @@ int wq_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* W
     DeviceState* d = nullptr;
     rc = require_device(&dev, &d, st, true);
     if (rc) return rc;
-    if (launch_prepack(Q, s, K, N, g, Wp, st) != 0) {
+    if (launch_prepack(Q, s, nullptr, K, N, g, Wp, st) != 0) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -445,7 +449,7 @@ int wq_unpack(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_o
     DeviceState* d = nullptr;
     rc = require_device(&dev, &d, st, true);
     if (rc) return rc;
-    if (launch_unpack(Wp, K, N, g, Q_out, s_out, st) != 0) {
+    if (launch_unpack(Wp, K, N, g, Q_out, s_out, nullptr, st) != 0) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -472,13 +476,62 @@ int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, 
     return run_gemm(0, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
 }
 
+size_t wq_prepacked_bytes_zp(int K, int N, int g) {
+    if (!shape_ok(K, N)) return 0;
+    const int slots = scale_slots(K, g);
+    if (slots <= 0) return 0;
+    return static_cast<size_t>(n_tiles(N)) * (K / kTileK) * blob_bytes_w4a16_zp(slots);
+}
+
+int wq_prepack_zp(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K, int N, int g, void* Wp, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) <= 0) return WQ_ERR_INVALID_ARG;
+    if (!s || !z) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s, 16) || !aligned(z, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_prepack(Q, s, z, K, N, g, Wp, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_unpack_zp(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, uint8_t* z_out, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q_out, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) <= 0) return WQ_ERR_INVALID_ARG;
+    if (!s_out || !z_out) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s_out, 16) || !aligned(z_out, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_unpack(Wp, K, N, g, Q_out, s_out, z_out, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16_zp(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g, void* stream) {
+    return run_gemm(3, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
+}
+
 int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
                  int M, int N, int K, void* stream) {
     return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
 }
 
-int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, void* stream) {
-    if (K <= 0 || M < 0) return WQ_ERR_INVALID_ARG;
+int wq_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* A_q, float* sa, void* stream) {
+    if (K <= 0 || M < 0 || (bits != 4 && bits != 8)) return WQ_ERR_INVALID_ARG;
     if (K % 8 || M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (M == 0) return WQ_OK;
     if (!A || !A_q || !sa) return WQ_ERR_INVALID_ARG;
@@ -489,7 +542,7 @@ int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, voi
     DeviceState* d = nullptr;
     int rc = require_device(&dev, &d, st, true);
     if (rc) return rc;
-    if (launch_quantize_act(A, M, K, A_q, sa, st) != 0) {
+    if (launch_quantize_act(A, M, K, bits, A_q, sa, st) != 0) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -497,20 +550,21 @@ int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, voi
 }
 
 int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
-                         float* sa_out, int M, int N, int K, void* stream) {
-    if (M > 0 && !A) return WQ_ERR_INVALID_ARG;
+                         float* sa_out, int M, int N, int K, int act_bits, void* stream) {
+    if ((M > 0 && !A) || (act_bits != 4 && act_bits != 8)) return WQ_ERR_INVALID_ARG;
     return run_gemm(1, nullptr, nullptr, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream), A,
-                    sa_out);
+                    sa_out, act_bits);
 }
 
 size_t wq_workspace_bytes(int kind, int M, int N, int K) {
-    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 2) return 0;
+    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 3) return 0;
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
     DeviceState* d = device_state(&dev);
     if (!d || !d->supported) return 0;
     Plan pl;
-    if (plan_for(kind == 0 ? 0 : 1, M, N, K, kind == 0 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
+    const bool w4a16 = kind == 0 || kind == 3;  // the zero-point layer plans like the W4A16 one
+    if (plan_for(w4a16 ? 0 : 1, M, N, K, w4a16 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
     if (kind == 2) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_quant_bytes(M, K);
     return workspace_bytes_for(pl);
 }

@@ -71,6 +71,9 @@ struct Ctl {
     unsigned long long timeout_ns;
 };
 
+// Modes with group scales in the blob (symmetric, or with a zero point per group).
+__host__ __device__ constexpr bool is_group(int mode) { return mode == kModeGroup || mode == kModeGroupZP; }
+
 __device__ __forceinline__ void raise_error(const Ctl& c, int code) {
     *c.abort_flag = 1;
     atomicCAS(c.status, 0, code);
@@ -178,6 +181,14 @@ struct ChunkBar {
 // (w & 0x000F000F) | 0x64006400 is the fp16 pair (1024 + q_lo, 1024 + q_hi) exactly;
 // subtracting 1032 leaves q - 8 exactly. A nibble in bits 4..7 of a half gives 1024 + 16q;
 // (1024 + 16q)/16 - 72 = q - 8, again exact in one fused multiply-add.
+// With a zero point z per group (asymmetric groups) the two constants become 1024 + z and
+// -(64 + z): (1024 + q) - (1024 + z) and (1024 + 16q)/16 - (64 + z) are q - z, exact.
+__device__ __forceinline__ __half2 half2_bits(uint32_t v) { return *reinterpret_cast<const __half2*>(&v); }
+// The constants of zero point z (0..15): 0x6400 + z is 1024 + z (units of 1 in [1024, 2048)),
+// 0xD400 + 16z is -(64 + z) (units of 1/16 in [64, 128)).
+__device__ __forceinline__ uint32_t zp_lo(uint32_t z) { return (0x6400u + z) * 0x10001u; }
+__device__ __forceinline__ uint32_t zp_hi(uint32_t z) { return (0xD400u + (z << 4)) * 0x10001u; }
+
 __device__ __forceinline__ void dequant_word_f16(uint32_t x, __half2 s, bool scaled, uint32_t* out) {
     const uint32_t kMagic = 0x64006400u;
     const __half2 k1032 = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
@@ -193,6 +204,32 @@ __device__ __forceinline__ void dequant_word_f16(uint32_t x, __half2 s, bool sca
     __half2 h2 = __hsub2(*reinterpret_cast<const __half2*>(&u2), k1032);
     __half2 h3 = __hfma2(*reinterpret_cast<const __half2*>(&u3), kSixteenth, kMinus72);
     if (scaled) {  // one round-to-nearest of (q - 8) * s per weight
+        h0 = __hmul2(h0, s);
+        h1 = __hmul2(h1, s);
+        h2 = __hmul2(h2, s);
+        h3 = __hmul2(h3, s);
+    }
+    out[0] = *reinterpret_cast<uint32_t*>(&h0);
+    out[1] = *reinterpret_cast<uint32_t*>(&h1);
+    out[2] = *reinterpret_cast<uint32_t*>(&h2);
+    out[3] = *reinterpret_cast<uint32_t*>(&h3);
+}
+
+// The same with the zero point's constants klo = zp_lo(z), khi = zp_hi(z): q - z exactly.
+__device__ __forceinline__ void dequant_word_f16_zp(uint32_t x, __half2 s, bool scaled, uint32_t klo, uint32_t khi,
+                                                    uint32_t* out) {
+    const uint32_t kMagic = 0x64006400u;
+    const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+    const uint32_t x8 = x >> 8;
+    const uint32_t u0 = lop3_and_or(x, 0x000F000Fu, kMagic);
+    const uint32_t u1 = lop3_and_or(x, 0x00F000F0u, kMagic);
+    const uint32_t u2 = lop3_and_or(x8, 0x000F000Fu, kMagic);
+    const uint32_t u3 = lop3_and_or(x8, 0x00F000F0u, kMagic);
+    __half2 h0 = __hsub2(*reinterpret_cast<const __half2*>(&u0), half2_bits(klo));
+    __half2 h1 = __hfma2(*reinterpret_cast<const __half2*>(&u1), kSixteenth, half2_bits(khi));
+    __half2 h2 = __hsub2(*reinterpret_cast<const __half2*>(&u2), half2_bits(klo));
+    __half2 h3 = __hfma2(*reinterpret_cast<const __half2*>(&u3), kSixteenth, half2_bits(khi));
+    if (scaled) {
         h0 = __hmul2(h0, s);
         h1 = __hmul2(h1, s);
         h2 = __hmul2(h2, s);
@@ -373,15 +410,20 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
                 const uint32_t a = iter % kASlots, aph = (iter / kASlots) & 1;
                 uint4 w0 = make_uint4(0, 0, 0, 0), w1 = make_uint4(0, 0, 0, 0);
                 uint16_t sc0 = 0, sc1 = 0;
+                uint32_t z0 = 8, z1 = 8;
                 if (ok) {
                     const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
                     const uint4* words = reinterpret_cast<const uint4*>(blob);
                     w0 = words[(half * 2 + 0) * kTileN + row];
                     w1 = words[(half * 2 + 1) * kTileN + row];
-                    if (MODE == kModeGroup && p.scale_in_dequant) {
+                    if (is_group(MODE) && p.scale_in_dequant) {
                         const uint16_t* sc = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
                         sc0 = sc[u0 * kTileN + row];
                         sc1 = sc[u1 * kTileN + row];
+                    }
+                    if (MODE == kModeGroupZP) {
+                        z0 = blob[p.zp_offset + u0 * kTileN + row];
+                        z1 = blob[p.zp_offset + u1 * kTileN + row];
                     }
                 }
                 __syncwarp();
@@ -399,7 +441,13 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
                         uint32_t out[32];
                         const __half2 s0 = __half2half2(__ushort_as_half(sc0));
                         const __half2 s1 = __half2half2(__ushort_as_half(sc1));
-                        if (MODE == kModeGroup && p.scale_in_dequant) {
+                        if (MODE == kModeGroupZP) {
+                            const uint32_t lo0 = zp_lo(z0), hi0 = zp_hi(z0), lo1 = zp_lo(z1), hi1 = zp_hi(z1);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                dequant_word_f16_zp(wv[i], i < 4 ? s0 : s1, true, i < 4 ? lo0 : lo1, i < 4 ? hi0 : hi1,
+                                                    out + 4 * i);
+                        } else if (MODE == kModeGroup && p.scale_in_dequant) {
 #pragma unroll
                             for (int i = 0; i < 8; ++i) dequant_word_f16(wv[i], i < 4 ? s0 : s1, true, out + 4 * i);
                         } else {
@@ -800,7 +848,7 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
                                    const Ctl& ctl, long long beg, long long end) {
     constexpr int kSlotCols = (MODE == kModeW4A8) ? 32 : 64;  // 128 k of fp16 or int8 per lane
     constexpr int H = TM / 4;
-    constexpr bool kScaleAtAdd = (MODE == kModeGroup) && !kScaled;
+    constexpr bool kScaleAtAdd = is_group(MODE) && !kScaled;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3;
     const uint32_t r = static_cast<uint32_t>(warp >> 2);
@@ -837,6 +885,7 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
                 uint4 w[4];
                 uint16_t sc[4] = {0, 0, 0, 0};
                 uint16_t sc_add = 0;
+                uint8_t zq[MODE == kModeGroupZP ? 4 : 1] = {8};  // asymmetric groups: each 32-row block's zero
                 if (ok) {
 #pragma unroll
                     for (int hv = 0; hv < (kSplitLoad ? 2 : 4); ++hv) w[hv] = words[hv * kTileN + row];
@@ -845,6 +894,15 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
                         for (int hv = 0; hv < 4; ++hv) sc[hv] = scs[((32 * hv) / p.group_rows) * kTileN + row];
                     }
                     if (kScaleAtAdd) sc_add = scs[row];
+                    if constexpr (MODE == kModeGroupZP) {
+                        if (kScaled) {
+#pragma unroll
+                            for (int hv = 0; hv < 4; ++hv)
+                                zq[hv] = blob[p.zp_offset + ((32 * hv) / p.group_rows) * kTileN + row];
+                        } else {
+                            zq[0] = zq[1] = zq[2] = zq[3] = blob[p.zp_offset + row];
+                        }
+                    }
                 }
                 if (!kSplitLoad) {
                     __syncwarp();
@@ -876,9 +934,18 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
 #pragma unroll
                             for (int q2 = 0; q2 < 2; ++q2) {  // 16 registers per store keeps the live set small
                                 uint32_t out[16];
+                                if constexpr (MODE == kModeGroupZP) {
+                                    const uint32_t zz = zq[2 * h + q2];
+                                    const uint32_t klo = zp_lo(zz), khi = zp_hi(zz);
 #pragma unroll
-                                for (int k = 0; k < 4; ++k)
-                                    dequant_word_f16(wv[4 * q2 + k], q2 == 0 ? s0 : s1, kScaled, out + 4 * k);
+                                    for (int k = 0; k < 4; ++k)
+                                        dequant_word_f16_zp(wv[4 * q2 + k], q2 == 0 ? s0 : s1, kScaled, klo, khi,
+                                                            out + 4 * k);
+                                } else {
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k)
+                                        dequant_word_f16(wv[4 * q2 + k], q2 == 0 ? s0 : s1, kScaled, out + 4 * k);
+                                }
                                 tmem_st_x16(slot_addr + h * 32 + q2 * 16, out);
                             }
                         }
@@ -1056,7 +1123,7 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
 
     if (warp < kDqWarpsS) {
-        if constexpr (MODE == kModeGroup) {
+        if constexpr (is_group(MODE)) {
             if (p.scale_in_dequant)
                 dequant_role_small<MODE, TM, true>(p, wring, bars, tmem, ctl, beg, end);
             else
@@ -1098,7 +1165,9 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->threads = pl->small ? kThreadsSmall : kThreadsLarge;
     pl->issuers = pl->small ? kMaxIssuers : (tm <= 64 ? 4 : (tm <= 128 ? 2 : 1));
     pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;
-    pl->blob_bytes = (mode == kModeGroup) ? static_cast<int>(blob_bytes_w4a16(slots)) : kCodeBytes;
+    pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
+                     : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
+                                              : kCodeBytes;
     const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */;
     int s = budget / (pl->act_slot + pl->blob_bytes);
     if (s > kMaxSlots) s = kMaxSlots;
@@ -1129,6 +1198,9 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeChannel, 32>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 32>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeGroupZP>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 16>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 32>, max_dynamic_smem);
     return e;
 }
 
@@ -1165,6 +1237,7 @@ cudaError_t launch_gemm(int mode, const ActMaps& maps, const GemmArgs& args, con
     switch (mode) {
         case kModeGroup: return launch_mode<kModeGroup>(maps, args, plan, stream);
         case kModeChannel: return launch_mode<kModeChannel>(maps, args, plan, stream);
+        case kModeGroupZP: return launch_mode<kModeGroupZP>(maps, args, plan, stream);
         default: return launch_mode<kModeW4A8>(maps, args, plan, stream);
     }
 }

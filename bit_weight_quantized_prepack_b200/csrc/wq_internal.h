@@ -30,6 +30,7 @@ struct GemmArgs {
     int group_rows;            // W4A16 grouped: rows per scale slot, min(g, 128)
     int small;                 // 1: per-k-block partials summed by the dequant warps (tile_m <= 32)
     int scale_in_dequant;      // 1: the dequant multiplies by the group scale (fp16 weights)
+    int zp_offset;             // asymmetric groups: byte offset of the zero points within a blob
     long long units;           // tiles * k_blocks
     int grid;
     unsigned long long timeout_ns;
@@ -56,10 +57,11 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem);
 cudaError_t launch_gemm(int mode, const ActMaps& maps, const GemmArgs& args, const Plan& plan,
                         cudaStream_t stream);
 
-int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, cudaStream_t st);
+int launch_prepack(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K, int N, int g, void* Wp,
+                   cudaStream_t st);
 int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t st);
-int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st);
+int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* z, cudaStream_t st);
 int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st);
-int launch_quantize_act(const uint16_t* A, int M, int K, int8_t* Aq, float* sa, cudaStream_t st);
+int launch_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* Aq, float* sa, cudaStream_t st);
 
 }  // namespace wq

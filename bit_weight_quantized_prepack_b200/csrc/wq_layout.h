@@ -14,6 +14,9 @@
 //   NT*128 entries, then to 16 bytes) follows the last blob.
 //   Columns past N hold code 8 and scale 0: zero weights.
 // Prepacked W4A8 buffer: the same blobs, codes only, with the W4A8 nibble order.
+// Prepacked W4A16 buffer with zero points (g < K): each blob is the W4A16 blob followed by
+//   `slots` rows of 128 uint8 zero points z (0..15), laid out like the scale rows; padded
+//   columns hold zero point 8 (and scale 0).
 //
 // Nibble orders. Within a word the W4A16 order puts codes (2p, 2p+1) at nibble positions
 // (p, p+4) for p = 0..3, so that masking 0x000F000F (p = 0) or 0x00F000F0 (p = 1) of the
@@ -54,7 +57,7 @@ constexpr int kASlots = 4;                    // dequantised weight tiles in ten
 constexpr int kTmemCols = 512;
 constexpr int kTmemAOffset = 256;             // accumulators in columns [0, 256), A slots above
 
-enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2 };
+enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2, kModeGroupZP = 3 };
 
 // Scale rows per blob for W4A16; 0 means per-column scales (g == K); -1 unsupported.
 inline int scale_slots(int K, int g) {
@@ -70,6 +73,9 @@ inline bool shape_ok(int K, int N) { return K > 0 && K % kTileK == 0 && N > 0 &&
 inline int n_tiles(int N) { return (N + kTileN - 1) / kTileN; }
 
 inline size_t blob_bytes_w4a16(int slots) { return kCodeBytes + 2u * kTileN * static_cast<size_t>(slots); }
+
+// Asymmetric groups: the W4A16 blob followed by `slots` rows of 128 uint8 zero points.
+inline size_t blob_bytes_w4a16_zp(int slots) { return blob_bytes_w4a16(slots) + static_cast<size_t>(kTileN) * slots; }
 
 inline size_t channel_tail_bytes(int N) { return ((2u * n_tiles(N) * kTileN) + 15u) / 16u * 16u; }
 

@@ -1,5 +1,5 @@
-// The layout pass: reorder 4-bit codes and group scales into the blobs the GEMM streams,
-// and its inverse (a test aid). Layout: see wq_layout.h.
+// The layout pass: reorder 4-bit codes, group scales and (asymmetric groups) zero points into
+// the blobs the GEMM streams, and its inverse (a test aid). Layout: see wq_layout.h.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -103,6 +103,36 @@ __global__ void unpack_scales_kernel(const uint8_t* __restrict__ wp, int N, int 
     s[(row0 / g) * N + n] = reinterpret_cast<const uint16_t*>(wp + blob * blob_bytes + kCodeBytes)[u * kTileN + r];
 }
 
+// One thread per (blob, slot, r): copy one zero point into the blob's zero rows (asymmetric groups).
+__global__ void prepack_zeros_kernel(const uint8_t* __restrict__ z, int N, int KT, int g, int slots, long long total,
+                                     uint8_t* __restrict__ wp, size_t blob_bytes, size_t zoff) {
+    long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int u = static_cast<int>((idx / kTileN) % slots);
+    const long long blob = idx / (static_cast<long long>(slots) * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const long long n = nt * kTileN + r;
+    const long long grp = (static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g) / g;
+    wp[blob * blob_bytes + zoff + u * kTileN + r] = (n < N) ? z[grp * N + n] : static_cast<uint8_t>(8);
+}
+
+__global__ void unpack_zeros_kernel(const uint8_t* __restrict__ wp, int N, int KT, int g, int slots, long long total,
+                                    uint8_t* __restrict__ z, size_t blob_bytes, size_t zoff) {
+    long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int u = static_cast<int>((idx / kTileN) % slots);
+    const long long blob = idx / (static_cast<long long>(slots) * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const long long n = nt * kTileN + r;
+    const long long row0 = static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g;
+    if (n >= N || row0 % g != 0) return;  // a group larger than a blob is written by its first blob only
+    z[(row0 / g) * N + n] = wp[blob * blob_bytes + zoff + u * kTileN + r];
+}
+
 __global__ void channel_tail_kernel(const uint16_t* __restrict__ s, int N, int padded, int tail_elems,
                                     uint16_t* __restrict__ tail) {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -119,10 +149,12 @@ static inline unsigned blocks_for(long long total, int threads) {
     return static_cast<unsigned>((total + threads - 1) / threads);
 }
 
-int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, cudaStream_t st) {
+int launch_prepack(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K, int N, int g, void* Wp,
+                   cudaStream_t st) {
     const int slots = scale_slots(K, g);
     const int KT = K / kTileK, NT = n_tiles(N);
-    const size_t blob = slots > 0 ? blob_bytes_w4a16(slots) : static_cast<size_t>(kCodeBytes);
+    const size_t blob = slots > 0 ? (z ? blob_bytes_w4a16_zp(slots) : blob_bytes_w4a16(slots))
+                                  : static_cast<size_t>(kCodeBytes);
     uint8_t* wp = static_cast<uint8_t*>(Wp);
     const long long nblob = static_cast<long long>(NT) * KT;
     const long long tc = nblob * 4 * kTileN;
@@ -131,6 +163,9 @@ int launch_prepack(const int32_t* Q, const uint16_t* s, int K, int N, int g, voi
     if (slots > 0) {
         const long long ts = nblob * slots * kTileN;
         prepack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(s, N, KT, g, slots, ts, wp, blob);
+        if (z)
+            prepack_zeros_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(z, N, KT, g, slots, ts, wp, blob,
+                                                                       blob_bytes_w4a16(slots));
     } else {
         const int tail_elems = static_cast<int>(channel_tail_bytes(N) / 2);
         channel_tail_kernel<<<blocks_for(tail_elems, 256), 256, 0, st>>>(
@@ -147,10 +182,11 @@ int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t s
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
-int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st) {
+int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* z, cudaStream_t st) {
     const int slots = scale_slots(K, g);
     const int KT = K / kTileK, NT = n_tiles(N);
-    const size_t blob = slots > 0 ? blob_bytes_w4a16(slots) : static_cast<size_t>(kCodeBytes);
+    const size_t blob = slots > 0 ? (z ? blob_bytes_w4a16_zp(slots) : blob_bytes_w4a16(slots))
+                                  : static_cast<size_t>(kCodeBytes);
     const uint8_t* wp = static_cast<const uint8_t*>(Wp);
     const long long nblob = static_cast<long long>(NT) * KT;
     const long long tc = nblob * 4 * kTileN;
@@ -159,6 +195,9 @@ int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, 
     if (slots > 0) {
         const long long ts = nblob * slots * kTileN;
         unpack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, s, blob);
+        if (z)
+            unpack_zeros_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, z, blob,
+                                                                      blob_bytes_w4a16(slots));
     } else {
         channel_untail_kernel<<<blocks_for(N, 256), 256, 0, st>>>(
             reinterpret_cast<const uint16_t*>(wp + nblob * blob), N, s);

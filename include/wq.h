@@ -110,6 +110,27 @@ WQ_API int wq_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q_out, void* st
 WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
                   int M, int N, int K, int g, void* stream);
 
+/* ---------------------------------------------------------------- asymmetric groups
+ * The layer with a zero point per group and column: W[k,n] = (q[k,n] - z[k/g, n]) * s[k/g, n]
+ * ("Atom: Low-bit Quantization for Efficient and Accurate LLM Serving", method: fine-grained
+ * group quantisation, read with the GPTQ-style 4-bit zero point that the pages leave open;
+ * z = 8 everywhere is the symmetric layer). z is uint8 [K/g, N] with values 0..15, 16-byte
+ * aligned (a value above 15 is stored as given and gives wrong weights, never an access out
+ * of bounds); g must be below K (32, 64, 128 or a multiple of 128 dividing K).
+ * wq_prepacked_bytes_zp: the size of the prepacked buffer, or 0 when unsupported; each blob
+ * is the W4A16 blob followed by its groups' uint8 zero points (columns padded with z = 8 and
+ * s = 0). wq_prepack_zp / wq_unpack_zp: the layout pass and its inverse (test aid), as
+ * wq_prepack / wq_unpack. wq_gemm_w4a16_zp: as wq_gemm_w4a16, on the zero-point buffer; the
+ * weight (q - z) * s is exact before its one fp16 rounding (none for group scales of
+ * g >= 128 on M <= 32, where the scale multiplies each k-block's fp32 partial). */
+WQ_API size_t wq_prepacked_bytes_zp(int K, int N, int g);
+WQ_API int wq_prepack_zp(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K, int N, int g, void* Wp,
+                 void* stream);
+WQ_API int wq_unpack_zp(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, uint8_t* z_out,
+                 void* stream);
+WQ_API int wq_gemm_w4a16_zp(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g,
+                 void* stream);
+
 /* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
  * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
  * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
@@ -119,24 +140,27 @@ WQ_API int wq_gemm_w4a16(const uint16_t* A, const void* Wp, uint16_t* Y,
 WQ_API int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw,
                  uint16_t* Y, int32_t* acc_out, int M, int N, int K, void* stream);
 
-/* Per-token activation quantisation, the step before the W4A8 layer ("Atom: Low-bit
- * Quantization for Efficient and Accurate LLM Serving", method: quantisation parameters of
- * the activations computed from them at inference time, one scale per token). For each row m
- * of the fp16 activations A [M, K]: amax = max_k |A[m,k]|, inv = 127 / amax and
- * sa[m] = amax / 127 (fp32 divisions, round to nearest), A_q[m,k] = round-half-even(A[m,k]
- * * inv) (fp32 product, round to nearest) clamped to [-127, 127]; a row of zeros gives codes 0
- * and sa[m] = 0. A must be finite. A_q int8 [M, K] and sa fp32 [M] are caller-owned device
- * memory. K a positive multiple of 8, 0 <= M <= 2^24; A and A_q 16-byte aligned, sa 4-byte. */
-WQ_API int wq_quantize_act(const uint16_t* A, int M, int K, int8_t* A_q, float* sa, void* stream);
+/* Per-token activation quantisation, the step before the layer on int8 tensor cores ("Atom:
+ * Low-bit Quantization for Efficient and Accurate LLM Serving", method: quantisation
+ * parameters of the activations computed from them at inference time, one scale per token;
+ * 8-bit activations for W4A8, 4-bit for W4A4). With L = 127 (bits = 8) or 7 (bits = 4), for
+ * each row m of the fp16 activations A [M, K]: amax = max_k |A[m,k]|, inv = L / amax and
+ * sa[m] = amax / L (fp32 divisions, round to nearest), A_q[m,k] = round-half-even(A[m,k] *
+ * inv) (fp32 product, round to nearest) clamped to [-L, L]; a row of zeros gives codes 0 and
+ * sa[m] = 0. 4-bit codes are stored one per int8 (unpacked: tcgen05 has no 4-bit integer
+ * MMA). A must be finite. A_q int8 [M, K] and sa fp32 [M] are caller-owned device memory.
+ * K a positive multiple of 8, 0 <= M <= 2^24; A and A_q 16-byte aligned, sa 4-byte. */
+WQ_API int wq_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* A_q, float* sa, void* stream);
 
-/* The W4A8 layer on fp16 activations: wq_quantize_act into the stream's workspace, then
- * wq_gemm_w4a8 on the codes and scales, in one call (two launches on `stream`; the layer's
- * kernel starts streaming weights while the quantisation finishes, and reads the codes only
- * after it). Y, acc_out and the constraints are those of wq_gemm_w4a8; sa_out (fp32 [M],
- * nullable) receives the per-token scales. The workspace must hold
- * wq_workspace_bytes(2, M, N, K) bytes (it grows on first use, or by wq_workspace_reserve). */
+/* The layer on fp16 activations quantised per token to act_bits = 8 (W4A8) or 4 (W4A4):
+ * wq_quantize_act into the stream's workspace, then wq_gemm_w4a8 on the codes and scales, in
+ * one call (two launches on `stream`; the layer's kernel sets up and prefetches its first
+ * weight blobs while the quantisation finishes, and reads the codes only after it). Y,
+ * acc_out and the constraints are those of wq_gemm_w4a8; sa_out (fp32 [M], nullable)
+ * receives the per-token scales. The workspace must hold wq_workspace_bytes(2, M, N, K)
+ * bytes (it grows on first use, or by wq_workspace_reserve). */
 WQ_API int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uint16_t* Y,
-                 int32_t* acc_out, float* sa_out, int M, int N, int K, void* stream);
+                 int32_t* acc_out, float* sa_out, int M, int N, int K, int act_bits, void* stream);
 
 /* W4A16 without any allocation. No counterpart in the paper: it exists for callers that
  * cannot allocate device memory when they run the layer (an engine that gave all free
@@ -165,8 +189,8 @@ WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
                   int M, int N, int K, int g, void* stream);
 
 /* ---------------------------------------------------------------- workspace and status
- * Bytes of library workspace one call of the given kind and shape needs
- * (kind 0 = W4A16, 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act). */
+ * Bytes of library workspace one call of the given kind and shape needs (kind 0 = W4A16,
+ * 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act, 3 = wq_gemm_w4a16_zp). */
 WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it

@@ -11,7 +11,7 @@ import bit_weight_quantized_prepack_b200 as wq
 class _Recorder:
     """Stands in for the loaded library: records every entry point called, except the pure size
     queries, which it forwards to the real library."""
-    PURE = {"wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_status_string"}
+    PURE = {"wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepacked_bytes_zp", "wq_status_string"}
 
     def __init__(self, real):
         self.real, self.calls = real, []
@@ -109,4 +109,19 @@ def test_prepack_and_unpack_refuse_wrong_sizes(rec):
         wq.wq_unpack(torch.zeros(16, dtype=torch.uint8), K, N, g)
     with pytest.raises(ValueError):
         wq.wq_unpack_w4a8(torch.zeros(16, dtype=torch.uint8), K, N)
+    assert rec.calls == []
+
+
+def test_zero_point_calls_refuse_wrong_sizes(rec):
+    Q = torch.zeros((K // 8, N), dtype=torch.int32)
+    s = torch.zeros((K // g, N), dtype=torch.float16)
+    with pytest.raises(ValueError):  # z must be [K/g, N]
+        wq.wq_prepack_zp(Q, s, torch.zeros((K // g, N + 8), dtype=torch.uint8), g)
+    with pytest.raises(TypeError):  # z must be uint8
+        wq.wq_prepack_zp(Q, s, torch.zeros((K // g, N), dtype=torch.int32), g)
+    with pytest.raises(wq.WqError):  # zero points need g < K
+        wq.wq_prepack_zp(Q, torch.zeros((1, N), dtype=torch.float16), torch.zeros((1, N), dtype=torch.uint8), K)
+    with pytest.raises(ValueError):  # the zero-point buffer is larger than the symmetric one
+        wq.wq_gemm_w4a16_zp(torch.zeros((M, K), dtype=torch.float16),
+                            torch.zeros(wq.wq_prepacked_bytes(K, N, g), dtype=torch.uint8), N, g)
     assert rec.calls == []
