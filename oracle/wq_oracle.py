@@ -43,6 +43,8 @@ import numpy as np
 __all__ = [
     "unpack_codes", "dequant", "w4a16", "w4a16_absdot", "w4a16_entry",
     "tolerance", "w4a8_acc", "w4a8", "w4a8_absdot", "quantize_act",
+    "dequant_gidx", "w4a16_gidx", "w4a16_gidx_absdot", "act_order_perm", "pack_codes", "reorder_rows",
+    "prepack_w4a16_act_order",
     "dequant_zp", "w4a16_zp", "w4a16_zp_absdot", "prepack_w4a16_zp", "prepacked_bytes_w4a16_zp", "unprepack_w4a16_zp",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
@@ -151,6 +153,90 @@ def w4a8_absdot(A: np.ndarray, sa: np.ndarray, Q: np.ndarray, sw: np.ndarray, ch
         wq = np.abs(unpack_codes(np.asarray(Q)[:, n0:n1]).astype(np.float64) - ZERO_POINT)
         out[:, n0:n1] = A64 @ wq
     return out * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+
+
+# --------------------------------------------------------------------------
+# act order: groups that are not contiguous along K
+# --------------------------------------------------------------------------
+def dequant_gidx(q: np.ndarray, s: np.ndarray, z, g_idx: np.ndarray) -> np.ndarray:
+    """``W[k,n] = (q[k,n] - z[g_idx[k], n]) * s[g_idx[k], n]`` in float64 (exact).
+
+    Group quantisation whose groups are not runs of consecutive rows: row ``k`` belongs to
+    group ``g_idx[k]`` (the "act order" of GPTQ-style checkpoints, where the rows were
+    quantised in an order of decreasing activation importance and each run of ``g`` rows in
+    that order shares one scale and zero point). The pages fix groups only as "fine-grained"
+    (Atom, method); this reading keeps their per-group scale and zero point and lets the rows
+    of a group lie anywhere. ``z = None`` is the fixed zero point 8.
+    """
+    g_idx = np.asarray(g_idx)
+    zz = ZERO_POINT if z is None else np.asarray(z, dtype=np.float64)[g_idx, :]
+    return (q.astype(np.float64) - zz) * np.asarray(s, dtype=np.float64)[g_idx, :]
+
+
+def w4a16_gidx(A: np.ndarray, Q: np.ndarray, s: np.ndarray, z, g_idx: np.ndarray, chunk: int = 4096) -> np.ndarray:
+    """``Y = A . W`` with ``W = dequant_gidx(...)``, in float64, chunked along N."""
+    A64 = np.asarray(A, dtype=np.float64)
+    N = np.asarray(Q).shape[1]
+    Y = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        zc = None if z is None else np.asarray(z)[:, n0:n1]
+        Y[:, n0:n1] = A64 @ dequant_gidx(unpack_codes(np.asarray(Q)[:, n0:n1]), np.asarray(s)[:, n0:n1], zc, g_idx)
+    return Y
+
+
+def w4a16_gidx_absdot(A: np.ndarray, Q: np.ndarray, s: np.ndarray, z, g_idx: np.ndarray,
+                      chunk: int = 4096) -> np.ndarray:
+    """``sum_k |A[m,k] * W[k,n]|`` for the act-order weights."""
+    A64 = np.abs(np.asarray(A, dtype=np.float64))
+    N = np.asarray(Q).shape[1]
+    out = np.empty((A64.shape[0], N), dtype=np.float64)
+    for n0 in range(0, N, chunk):
+        n1 = min(N, n0 + chunk)
+        zc = None if z is None else np.asarray(z)[:, n0:n1]
+        out[:, n0:n1] = A64 @ np.abs(dequant_gidx(unpack_codes(np.asarray(Q)[:, n0:n1]), np.asarray(s)[:, n0:n1],
+                                                  zc, g_idx))
+    return out
+
+
+def act_order_perm(g_idx: np.ndarray, g: int) -> np.ndarray:
+    """The row order that makes the groups contiguous: ``perm`` with ``g_idx[perm[i]] == i // g``.
+
+    Rows are sorted by group, keeping their order inside a group. Every group must hold
+    exactly ``g`` rows (as it does when the groups are runs of ``g`` rows of some order);
+    otherwise no such ``perm`` exists and ``ValueError`` is raised.
+    """
+    g_idx = np.asarray(g_idx)
+    K = g_idx.shape[0]
+    if g <= 0 or K % g:
+        raise ValueError("g must divide K")
+    perm = np.argsort(g_idx, kind="stable")
+    if not np.array_equal(g_idx[perm], np.arange(K) // g):
+        raise ValueError("every group must hold exactly g rows")
+    return perm
+
+
+def pack_codes(q: np.ndarray) -> np.ndarray:
+    """``Q[K/8, N]`` int32 from codes ``q[K, N]``: code ``8i + j`` in bits ``4j .. 4j+3`` of ``Q[i]``."""
+    K, N = q.shape
+    q32 = np.asarray(q, dtype=np.uint32).reshape(K // 8, 8, N)
+    word = np.zeros((K // 8, N), dtype=np.uint32)
+    for j in range(8):
+        word |= q32[:, j, :] << np.uint32(4 * j)
+    return word.view(np.int32)
+
+
+def reorder_rows(Q: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """The packed codes of the weight whose row ``i`` is row ``perm[i]`` of ``Q``'s weight."""
+    return pack_codes(unpack_codes(Q)[np.asarray(perm)])
+
+
+def prepack_w4a16_act_order(Q: np.ndarray, s: np.ndarray, z, perm: np.ndarray, g: int) -> np.ndarray:
+    """The prepacked buffer of an act-order weight: its rows taken in the order ``perm`` (so that
+    group ``i // g`` holds rows ``i``), then the contiguous-group layout (with zero points when
+    ``z`` is given). The layer then reads the activations in the same order."""
+    Qr = reorder_rows(Q, perm)
+    return prepack_w4a16(Qr, s, g) if z is None else prepack_w4a16_zp(Qr, s, z, g)
 
 
 # --------------------------------------------------------------------------

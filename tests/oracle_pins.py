@@ -16,6 +16,9 @@ with the fact it is pinned to:
   and exact rational bounds;
 * asymmetric groups (zero points): hand-worked layers (``tests/golden/zp_examples.txt``),
   exact rational brute force, and zero point 8 reproducing the symmetric layer;
+* act order (groups not contiguous along K): hand-worked layers, row orders and reordered
+  words (``tests/golden/act_order_examples.txt``), exact rational brute force, contiguous
+  groups reproducing the grouped layers, and the reordering identity the library relies on;
 * the prepacked layout: single codes and scales placed by hand-worked byte
   offsets (``tests/golden/blob_layout.txt``), independent of the oracle's own
   inverse of its layout.
@@ -396,10 +399,118 @@ def pin_zp_eight_is_symmetric(o):
     assert np.array_equal(o.w4a16_zp(d["A"], d["Q"], d["s"], z, 64), o.w4a16(d["A"], d["Q"], d["s"], 64))
 
 
+# ---------------------------------------------------------------- act order
+def golden_act_order(kind):
+    out = []
+    for line in _rows("act_order_examples.txt"):
+        parts = [p.strip() for p in line.split("|")]
+        if parts[0] != kind:
+            continue
+        if kind == "layer":
+            words, scales, zeros, gidx, acts, expect = parts[1:]
+            out.append({"Q": np.array([int(w, 16) for w in words.split()], np.uint32).view(np.int32).reshape(-1, 1),
+                        "s": np.array([float(x) for x in scales.split()], np.float16).reshape(-1, 1),
+                        "z": None if zeros == "-" else np.array([int(x) for x in zeros.split()], np.uint8).reshape(-1, 1),
+                        "g_idx": np.array([int(x) for x in gidx.split()]),
+                        "A": np.array([float(x) for x in acts.split()], np.float16).reshape(1, -1),
+                        "y": float(expect)})
+        elif kind == "perm":
+            g, gidx, perm = parts[1:]
+            out.append((int(g), np.array([int(x) for x in gidx.split()]), [int(x) for x in perm.split()]))
+        else:
+            words, perm, expect = parts[1:]
+            out.append((np.array([int(w, 16) for w in words.split()], np.uint32).view(np.int32).reshape(-1, 1),
+                        np.array([int(x) for x in perm.split()]), [int(w, 16) for w in expect.split()]))
+    return out
+
+
+def pin_act_order_golden(o):
+    for ex in golden_act_order("layer"):
+        y = o.w4a16_gidx(ex["A"], ex["Q"], ex["s"], ex["z"], ex["g_idx"])
+        assert y.shape == (1, 1) and y[0, 0] == ex["y"], (y, ex["y"])
+    for g, gidx, perm in golden_act_order("perm"):
+        assert o.act_order_perm(gidx, g).tolist() == perm
+    for Q, perm, words in golden_act_order("reorder"):
+        assert o.reorder_rows(Q, perm).view(np.uint32)[:, 0].tolist() == words
+
+
+def pin_act_order_unequal_groups_refused(o):
+    for g, gidx in [(2, [0, 0, 0, 1]), (2, [0, 1, 2, 2]), (3, [0, 0, 1, 1])]:
+        try:
+            o.act_order_perm(np.array(gidx), g)
+        except ValueError:
+            continue
+        raise AssertionError(f"g_idx {gidx} with g = {g} has no contiguous order but was accepted")
+
+
+def _random_gidx(rng, K, g):
+    return rng.permutation(np.arange(K) // g)
+
+
+def pin_act_order_bruteforce(o):
+    # exact rationals from the raw codes of the generator; groups scattered at random along K
+    for (M, K, N, g, zp, seed) in [(3, 64, 5, 16, True, 1), (2, 48, 7, 8, False, 2), (1, 128, 9, 32, True, 4)]:
+        d = synth.w4a16_inputs(K, N, g, M, seed=seed)
+        rng = np.random.default_rng(seed + 200)
+        gidx = _random_gidx(rng, K, g)
+        z = rng.integers(0, 16, (K // g, N)).astype(np.uint8) if zp else None
+        y = o.w4a16_gidx(d["A"], d["Q"], d["s"], z, gidx)
+        ad = o.w4a16_gidx_absdot(d["A"], d["Q"], d["s"], z, gidx)
+        assert y.shape == (M, N)
+        for m in range(M):
+            for n in range(N):
+                exact = Fraction(0)
+                absdot = Fraction(0)
+                for k in range(K):
+                    zk = 8 if z is None else int(z[gidx[k], n])
+                    t = Fraction(float(d["A"][m, k])) * (int(d["q"][k, n]) - zk) * Fraction(float(d["s"][gidx[k], n]))
+                    exact += t
+                    absdot += abs(t)
+                assert abs(Fraction(float(y[m, n])) - exact) <= Fraction(K * 2.0 ** -52) * absdot + Fraction(1e-300)
+                assert abs(Fraction(float(ad[m, n])) - absdot) <= Fraction(K * 2.0 ** -52) * absdot + Fraction(1e-300)
+
+
+def pin_act_order_contiguous_is_grouped(o):
+    # g_idx = k // g is the grouped layer, bit for bit (same weights, same product)
+    d = synth.w4a16_inputs(256, 40, 64, 3, seed=15)
+    z = np.random.default_rng(15).integers(0, 16, (4, 40)).astype(np.uint8)
+    gidx = np.arange(256) // 64
+    assert np.array_equal(o.w4a16_gidx(d["A"], d["Q"], d["s"], z, gidx), o.w4a16_zp(d["A"], d["Q"], d["s"], z, 64))
+    assert np.array_equal(o.w4a16_gidx(d["A"], d["Q"], d["s"], None, gidx), o.w4a16(d["A"], d["Q"], d["s"], 64))
+
+
+def pin_act_order_reordering_identity(o):
+    # taking the weight's rows and the activations' columns in the order perm turns scattered
+    # groups into contiguous ones and leaves y unchanged (up to the order of the fp64 sums)
+    for (M, K, N, g, zp, seed) in [(4, 512, 24, 128, True, 21), (3, 256, 16, 32, False, 22), (2, 384, 8, 64, True, 23)]:
+        d = synth.w4a16_inputs(K, N, g, M, seed=seed)
+        rng = np.random.default_rng(seed)
+        gidx = _random_gidx(rng, K, g)
+        z = rng.integers(0, 16, (K // g, N)).astype(np.uint8) if zp else None
+        perm = o.act_order_perm(gidx, g)
+        assert sorted(perm.tolist()) == list(range(K))
+        assert np.array_equal(gidx[perm], np.arange(K) // g)
+        y = o.w4a16_gidx(d["A"], d["Q"], d["s"], z, gidx)
+        ad = o.w4a16_gidx_absdot(d["A"], d["Q"], d["s"], z, gidx)
+        Qr = o.reorder_rows(d["Q"], perm)
+        assert np.array_equal(o.unpack_codes(Qr), d["q"][perm])
+        Ar = d["A"][:, perm]
+        yr = o.w4a16(Ar, Qr, d["s"], g) if z is None else o.w4a16_zp(Ar, Qr, d["s"], z, g)
+        assert np.all(np.abs(yr - y) <= 1e-12 * ad)
+
+
+def pin_pack_codes(o):
+    d = synth.w4a16_inputs(64, 12, 64, 1, seed=16)
+    assert np.array_equal(o.pack_codes(d["q"]), d["Q"])
+    assert np.array_equal(o.pack_codes(o.unpack_codes(d["Q"])), d["Q"])
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
     pin_row_permutation, pin_linearity, pin_tolerance_formula, pin_bruteforce_w4a8, pin_w4a8_extremes,
     pin_blob_layout_golden, pin_act_quant_golden, pin_act_quant_bounds, pin_zp_golden, pin_zp_bruteforce,
-    pin_zp_eight_is_symmetric,
+    pin_zp_eight_is_symmetric, pin_act_order_golden, pin_act_order_unequal_groups_refused,
+    pin_act_order_bruteforce, pin_act_order_contiguous_is_grouped, pin_act_order_reordering_identity,
+    pin_pack_codes,
 ]

@@ -157,7 +157,37 @@ def _mut_zp_sign(mp):
     mp.setattr(O, "dequant_zp", dequant_zp)
 
 
-MUTATIONS = [_mut_zp_ignored, _mut_zp_sign, _mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
+def _mut_gidx_ignored(mp):
+    def dequant_gidx(q, s, z, g_idx):  # groups read as contiguous runs instead of g_idx
+        G = np.asarray(s).shape[0]
+        grp = np.arange(q.shape[0]) // (q.shape[0] // G)
+        zz = 8 if z is None else np.asarray(z, np.float64)[grp, :]
+        return (q.astype(np.float64) - zz) * np.asarray(s, np.float64)[grp, :]
+    mp.setattr(O, "dequant_gidx", dequant_gidx)
+
+
+def _mut_gidx_zero_contiguous(mp):
+    def dequant_gidx(q, s, z, g_idx):  # the scale follows g_idx, the zero point does not
+        G = np.asarray(s).shape[0]
+        grp = np.arange(q.shape[0]) // (q.shape[0] // G)
+        zz = 8 if z is None else np.asarray(z, np.float64)[grp, :]
+        return (q.astype(np.float64) - zz) * np.asarray(s, np.float64)[np.asarray(g_idx), :]
+    mp.setattr(O, "dequant_gidx", dequant_gidx)
+
+
+def _mut_perm_inverse(mp):
+    real = O.act_order_perm
+    mp.setattr(O, "act_order_perm", lambda g_idx, g: np.argsort(real(g_idx, g)))
+
+
+def _mut_reorder_within_word(mp):
+    def reorder_rows(Q, perm):  # the order applied to whole words, codes kept inside them
+        q = O.unpack_codes(Q)
+        return O.pack_codes(q.reshape(-1, 8, q.shape[1])[np.asarray(perm)[::8] // 8].reshape(q.shape))
+    mp.setattr(O, "reorder_rows", reorder_rows)
+
+
+MUTATIONS = [_mut_gidx_ignored, _mut_gidx_zero_contiguous, _mut_perm_inverse, _mut_reorder_within_word, _mut_zp_ignored, _mut_zp_sign, _mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
              _mut_k_reversed, _mut_sign_flipped, _mut_w4a8_no_zero_point, _mut_w4a8_sw_dropped,
              _mut_absdot_signed, _mut_tolerance_rel_dropped]
 
