@@ -20,6 +20,7 @@ __all__ = [
     "wq_unpack", "wq_unpack_w4a8", "wq_gemm_w4a16", "wq_gemm_w4a16_noalloc", "wq_gemm_w4a8",
     "wq_quantize_act", "wq_gemm_w4a8_fp16act",
     "wq_prepacked_bytes_zp", "wq_prepack_zp", "wq_unpack_zp", "wq_gemm_w4a16_zp",
+    "wq_prepack_act_order", "wq_permute_act", "wq_gemm_w4a16_act_order",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
@@ -67,6 +68,9 @@ def _load():
         "wq_prepack_zp": (I, [P, P, P, I, I, I, P, P]),
         "wq_unpack_zp": (I, [P, I, I, I, P, P, P, P]),
         "wq_gemm_w4a16_zp": (I, [P, P, P, I, I, I, I, P]),
+        "wq_prepack_act_order": (I, [P, P, P, P, I, I, I, P, P]),
+        "wq_permute_act": (I, [P, P, I, I, P, P]),
+        "wq_gemm_w4a16_act_order": (I, [P, P, P, P, I, I, I, I, I, P]),
         "wq_gemm_w4a8_fp16act": (I, [P, P, P, P, P, P, I, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
@@ -336,6 +340,77 @@ def wq_gemm_w4a16_zp(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _check(lib.wq_gemm_w4a16_zp(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)), "wq_gemm_w4a16_zp")
+    return Y
+
+
+def wq_prepack_act_order(Q: torch.Tensor, s: torch.Tensor, perm: torch.Tensor, g: int, z: torch.Tensor | None = None,
+                         Wp: torch.Tensor | None = None, stream=None):
+    """Act order: Q int32 [K/8, N] in the checkpoint's row order, s fp16 [K/g, N] and optional zero
+    points z uint8 [K/g, N] by group, perm int32 [K] with g_idx[perm[i]] == i // g (for example
+    ``torch.argsort(g_idx, stable=True)``) -> the buffer of the reordered weight (the zero-point
+    layout when z is given). Synchronises the stream (perm is checked on the host)."""
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    if g <= 0 or K % g or (z is not None and g == K):
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_prepack_act_order")
+    _tensor(s, torch.float16, "s", shape=(K // g, N))
+    _tensor(perm, torch.int32, "perm", shape=(K,))
+    if z is not None:
+        _tensor(z, torch.uint8, "z", shape=(K // g, N))
+        nbytes = wq_prepacked_bytes_zp(K, N, g)
+        if nbytes == 0:
+            raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_prepack_act_order")
+    else:
+        nbytes = _prepacked_size(K, N, g, "wq_prepack_act_order")
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Q=Q, s=s, z=z, perm=perm, Wp=Wp)
+    if Wp is None:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack_act_order(_ptr(Q), _ptr(s), _ptr(z), _ptr(perm), K, N, g, _ptr(Wp), _stream(stream)),
+           "wq_prepack_act_order")
+    return Wp
+
+
+def wq_permute_act(A: torch.Tensor, perm: torch.Tensor, A_out: torch.Tensor | None = None, stream=None):
+    """A_out fp16 [M, K] = A[:, perm] (perm int32 [K]); an index outside [0, K) gives 0 and is
+    reported by wq_get_device_status."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    _tensor(perm, torch.int32, "perm", shape=(K,))
+    if A_out is not None:
+        _tensor(A_out, torch.float16, "A_out", shape=(M, K))
+    _on_one_cuda_device(A=A, perm=perm, A_out=A_out)
+    if A_out is None:
+        A_out = torch.empty((M, K), dtype=torch.float16, device=A.device)
+    _check(lib.wq_permute_act(_ptr(A), _ptr(perm), M, K, _ptr(A_out), _stream(stream)), "wq_permute_act")
+    return A_out
+
+
+def wq_gemm_w4a16_act_order(A: torch.Tensor, perm: torch.Tensor, Wp: torch.Tensor, N: int, g: int,
+                            zero_points: bool = False, Y: torch.Tensor | None = None, stream=None):
+    """Y fp16 [M, N] = A[:, perm] . W_reordered from a wq_prepack_act_order buffer (with zero
+    points when ``zero_points``): the activations are gathered and the layer run in one call."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    _tensor(perm, torch.int32, "perm", shape=(K,))
+    if g <= 0 or K % g or (zero_points and g == K):
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_gemm_w4a16_act_order")
+    if zero_points:
+        nbytes = wq_prepacked_bytes_zp(K, N, g)
+        if nbytes == 0:
+            raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_gemm_w4a16_act_order")
+    else:
+        nbytes = _prepacked_size(K, N, g, "wq_gemm_w4a16_act_order")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    _on_one_cuda_device(A=A, perm=perm, Wp=Wp, Y=Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.wq_gemm_w4a16_act_order(_ptr(A), _ptr(perm), _ptr(Wp), _ptr(Y), M, N, K, g, int(bool(zero_points)),
+                                       _stream(stream)), "wq_gemm_w4a16_act_order")
     return Y
 
 

@@ -8,6 +8,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <vector>
 #include <utility>
 
 #include "wq.h"
@@ -184,12 +185,23 @@ size_t act_quant_bytes(int M, int K) {
     return ((static_cast<size_t>(M) * K + 255) / 256) * 256 + ((static_cast<size_t>(M) * 4 + 255) / 256) * 256;
 }
 
-// The W4A16 (kind 0) or W4A8 (kind 1) layer. A_fp16 (W4A8 only, may be null): fp16
-// activations that are first quantised per token into the workspace (the codes replace A, the
-// scales go to sa_out when given, else to the workspace).
+// Bytes of the gathered activations the act-order call keeps in the workspace after the
+// stream-K part: fp16 [M, K], 256-byte aligned.
+size_t act_perm_bytes(int M, int K) { return ((static_cast<size_t>(M) * K * 2 + 255) / 256) * 256; }
+
+// Act-order gathers launch M * ceil(K / 2048) CTAs; the grid must stay below 2^31.
+bool perm_grid_ok(int M, int K) {
+    return static_cast<long long>(M) * ((K / 8 + 255) / 256) < (1LL << 31) - 1;
+}
+
+// The W4A16 (kind 0), W4A8 (kind 1) or zero-point (kind 3) layer. A_fp16 (W4A8 only, may be
+// null): fp16 activations that are first quantised per token into the workspace (the codes
+// replace A, the scales go to sa_out when given, else to the workspace). perm (kinds 0 and 3,
+// may be null): act order; A's columns are first gathered in the order perm into the
+// workspace, which then replaces A.
 int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y,
              int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream, const uint16_t* A_fp16 = nullptr,
-             float* sa_out = nullptr, int act_bits = 8) {
+             float* sa_out = nullptr, int act_bits = 8, const int32_t* perm = nullptr) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M < 0) return WQ_ERR_INVALID_ARG;
@@ -209,6 +221,8 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     }
     if (!aligned(Y, 16) || (acc_out && !aligned(acc_out, 16))) return WQ_ERR_MISALIGNED;
     if (kind == 1 && !aligned(sw, 4)) return WQ_ERR_MISALIGNED;
+    if (perm && !aligned(perm, 16)) return WQ_ERR_MISALIGNED;
+    if (perm && !perm_grid_ok(M, K)) return WQ_ERR_UNSUPPORTED_SHAPE;
 
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
@@ -220,8 +234,17 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     if (rc) return rc;
     void* ws = nullptr;
     const size_t gemm_ws = (workspace_bytes_for(pl) + 255) / 256 * 256;
-    rc = get_workspace(dev, stream, gemm_ws + (A_fp16 ? act_quant_bytes(M, K) : 0), &ws);
+    rc = get_workspace(dev, stream,
+                       gemm_ws + (A_fp16 ? act_quant_bytes(M, K) : 0) + (perm ? act_perm_bytes(M, K) : 0), &ws);
     if (rc) return rc;
+    if (perm) {
+        uint16_t* Ap = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + gemm_ws);
+        if (launch_permute_act(static_cast<const uint16_t*>(A), perm, M, K, Ap, d->status, stream) != 0) {
+            cudaGetLastError();
+            return WQ_ERR_CUDA;
+        }
+        A = Ap;
+    }
     if (A_fp16) {
         int8_t* Aq = reinterpret_cast<int8_t*>(static_cast<uint8_t*>(ws) + gemm_ws);
         float* sq = sa_out ? sa_out
@@ -525,6 +548,78 @@ int wq_gemm_w4a16_zp(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int 
     return run_gemm(3, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
 }
 
+int wq_prepack_act_order(const int32_t* Q, const uint16_t* s, const uint8_t* z, const int32_t* perm, int K, int N,
+                         int g, void* Wp, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    const int slots = scale_slots(K, g);
+    if (slots < 0 || (z && slots == 0)) return WQ_ERR_INVALID_ARG;
+    if (!s || !perm) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s, 16) || !aligned(perm, 16) || (z && !aligned(z, 16))) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    // perm must be a permutation of 0..K-1: checked on the host (once per weight), so the
+    // reordering kernel never reads outside Q
+    std::vector<int32_t> h(static_cast<size_t>(K));
+    if (cudaMemcpyAsync(h.data(), perm, h.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    std::vector<char> seen(static_cast<size_t>(K), 0);
+    for (int32_t r : h) {
+        if (r < 0 || r >= K || seen[r]) return WQ_ERR_INVALID_ARG;
+        seen[r] = 1;
+    }
+    void* Qp = nullptr;
+    if (cudaMallocAsync(&Qp, static_cast<size_t>(K / 8) * N * sizeof(int32_t), st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_NO_MEMORY;
+    }
+    rc = WQ_OK;
+    if (launch_permute_codes(Q, perm, K, N, static_cast<int32_t*>(Qp), st) != 0 ||
+        launch_prepack(static_cast<const int32_t*>(Qp), s, z, K, N, g, Wp, st) != 0) {
+        cudaGetLastError();
+        rc = WQ_ERR_CUDA;
+    }
+    if (cudaFreeAsync(Qp, st) != cudaSuccess) {
+        cudaGetLastError();
+        rc = WQ_ERR_CUDA;
+    }
+    return rc;
+}
+
+int wq_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, uint16_t* A_out, void* stream) {
+    if (K <= 0 || M < 0) return WQ_ERR_INVALID_ARG;
+    if (K % 8 || M > (1 << 24) || !perm_grid_ok(M, K)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return WQ_OK;
+    if (!A || !perm || !A_out) return WQ_ERR_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(perm, 16) || !aligned(A_out, 16)) return WQ_ERR_MISALIGNED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    int rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_permute_act(A, perm, M, K, A_out, d->status, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16_act_order(const uint16_t* A, const int32_t* perm, const void* Wp, uint16_t* Y, int M, int N,
+                            int K, int g, int zero_points, void* stream) {
+    if (M > 0 && (!A || !perm)) return WQ_ERR_INVALID_ARG;
+    if (zero_points != 0 && zero_points != 1) return WQ_ERR_INVALID_ARG;
+    return run_gemm(zero_points ? 3 : 0, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g,
+                    static_cast<cudaStream_t>(stream), nullptr, nullptr, 8, perm);
+}
+
 int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
                  int M, int N, int K, void* stream) {
     return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
@@ -557,15 +652,16 @@ int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uin
 }
 
 size_t wq_workspace_bytes(int kind, int M, int N, int K) {
-    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 3) return 0;
+    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 4) return 0;
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
     DeviceState* d = device_state(&dev);
     if (!d || !d->supported) return 0;
     Plan pl;
-    const bool w4a16 = kind == 0 || kind == 3;  // the zero-point layer plans like the W4A16 one
+    const bool w4a16 = kind == 0 || kind == 3 || kind == 4;  // these plan like the W4A16 layer
     if (plan_for(w4a16 ? 0 : 1, M, N, K, w4a16 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
     if (kind == 2) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_quant_bytes(M, K);
+    if (kind == 4) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_perm_bytes(M, K);
     return workspace_bytes_for(pl);
 }
 

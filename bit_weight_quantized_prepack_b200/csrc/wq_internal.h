@@ -63,5 +63,8 @@ int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t s
 int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* z, cudaStream_t st);
 int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st);
 int launch_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* Aq, float* sa, cudaStream_t st);
+int launch_permute_codes(const int32_t* Q, const int32_t* perm, int K, int N, int32_t* Qp, cudaStream_t st);
+int launch_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, uint16_t* Ap, int* status,
+                       cudaStream_t st);
 
 }  // namespace wq

@@ -131,6 +131,34 @@ WQ_API int wq_unpack_zp(const void* Wp, int K, int N, int g, int32_t* Q_out, uin
 WQ_API int wq_gemm_w4a16_zp(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g,
                  void* stream);
 
+/* ---------------------------------------------------------------- act order
+ * Groups whose rows are scattered along K: row k belongs to group g_idx[k] (GPTQ-style
+ * act-order checkpoints; "Atom: Low-bit Quantization for Efficient and Accurate LLM Serving",
+ * method: one scale, and zero point, per fine-grained group, read with the rows of a group
+ * placed anywhere). With perm int32 [K] a permutation of 0..K-1 such that
+ * g_idx[perm[i]] == i / g (every group holds exactly g rows; the rows sorted by group, e.g. a
+ * stable argsort of g_idx), y = sum_i A[m, perm[i]] * W[perm[i], n] is the grouped layer on the
+ * reordered weight and the gathered activations.
+ * wq_prepack_act_order: Q int32 [K/8, N] in the checkpoint's row order, s fp16 [K/g, N] and
+ * z uint8 [K/g, N] (nullable: the fixed zero point 8) indexed by group -> Wp of
+ * wq_prepacked_bytes(K, N, g) bytes (z NULL) or wq_prepacked_bytes_zp(K, N, g) bytes. perm is
+ * copied to the host and checked to be a permutation (WQ_ERR_INVALID_ARG otherwise); the call
+ * synchronises `stream` and allocates a K/2 * N byte temporary with cudaMallocAsync
+ * (WQ_ERR_NO_MEMORY when that fails). Run once per weight.
+ * wq_permute_act: A_out fp16 [M, K] = A[:, perm], caller-owned, 16-byte aligned like A and perm;
+ * K a positive multiple of 8. An entry of perm outside [0, K) is never dereferenced: its
+ * element becomes 0 and the device status word records WQ_ERR_INVALID_ARG
+ * (wq_get_device_status reports and clears it).
+ * wq_gemm_w4a16_act_order: wq_permute_act into the stream's workspace, then wq_gemm_w4a16
+ * (zero_points 0) or wq_gemm_w4a16_zp (zero_points 1) on the act-order buffer, in one call (two
+ * launches; the layer's kernel sets up while the gather finishes). The workspace must hold
+ * wq_workspace_bytes(4, M, N, K) before the call is captured in a CUDA graph. */
+WQ_API int wq_prepack_act_order(const int32_t* Q, const uint16_t* s, const uint8_t* z, const int32_t* perm,
+                 int K, int N, int g, void* Wp, void* stream);
+WQ_API int wq_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, uint16_t* A_out, void* stream);
+WQ_API int wq_gemm_w4a16_act_order(const uint16_t* A, const int32_t* perm, const void* Wp, uint16_t* Y,
+                 int M, int N, int K, int g, int zero_points, void* stream);
+
 /* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
  * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
  * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
@@ -190,7 +218,8 @@ WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
 
 /* ---------------------------------------------------------------- workspace and status
  * Bytes of library workspace one call of the given kind and shape needs (kind 0 = W4A16,
- * 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act, 3 = wq_gemm_w4a16_zp). */
+ * 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act, 3 = wq_gemm_w4a16_zp,
+ * 4 = wq_gemm_w4a16_act_order). */
 WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it

@@ -125,3 +125,22 @@ def test_zero_point_calls_refuse_wrong_sizes(rec):
         wq.wq_gemm_w4a16_zp(torch.zeros((M, K), dtype=torch.float16),
                             torch.zeros(wq.wq_prepacked_bytes(K, N, g), dtype=torch.uint8), N, g)
     assert rec.calls == []
+
+
+def test_act_order_calls_refuse_wrong_sizes(rec):
+    Q = torch.zeros((K // 8, N), dtype=torch.int32)
+    s = torch.zeros((K // g, N), dtype=torch.float16)
+    perm = torch.arange(K, dtype=torch.int32)
+    with pytest.raises(ValueError):  # perm must be [K]
+        wq.wq_prepack_act_order(Q, s, perm[:-8], g)
+    with pytest.raises(TypeError):  # perm must be int32
+        wq.wq_prepack_act_order(Q, s, perm.long(), g)
+    with pytest.raises(ValueError):  # z must be [K/g, N]
+        wq.wq_prepack_act_order(Q, s, perm, g, z=torch.zeros((K // g + 1, N), dtype=torch.uint8))
+    A = torch.zeros((M, K), dtype=torch.float16)
+    with pytest.raises(ValueError):
+        wq.wq_permute_act(A, perm, A_out=torch.zeros((M, K + 8), dtype=torch.float16))
+    with pytest.raises(ValueError):  # the zero-point buffer is larger than the symmetric one
+        wq.wq_gemm_w4a16_act_order(A, perm, torch.zeros(wq.wq_prepacked_bytes(K, N, g), dtype=torch.uint8), N, g,
+                                   zero_points=True)
+    assert rec.calls == []
