@@ -153,7 +153,9 @@ int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* p
 // split into swizzle-wide pieces: dims {64 fp16 or 128 int8, M, K/piece}, strides {K*elem (rows),
 // piece bytes}; a box of {piece, tile_m, c*pieces_per_kblock} lands in shared memory as
 // [piece index][row][128 bytes], the K-major 128-byte-swizzled layout the MMA reads.
-int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_m, int chunk, bool int8) {
+// Unswizzled (swizzle false: the matrix-vector kernel) the box lands as [piece][row][64 fp16].
+int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_m, int chunk, bool int8,
+                           bool swizzle = true) {
     const int piece = int8 ? 128 : 64;                 // elements per 128-byte row
     const int per_kblock = kTileK / piece;             // 1 (int8) or 2 (fp16)
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(piece), static_cast<cuuint64_t>(M),
@@ -166,7 +168,8 @@ int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_
                                    static_cast<cuuint32_t>(c * per_kblock)};
         CUresult r = g_encode(&maps->m[c - 1], int8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                               const_cast<void*>(A), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return WQ_ERR_CUDA;
     }
@@ -258,7 +261,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
         sa = sq;
     }
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1);
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1, !pl.gemv);
     if (rc) return rc;
 
     GemmArgs a;
@@ -801,7 +804,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     if (rc) return rc;
     if (workspace_bytes_for(pl) > kNoAllocStatusOffset) return WQ_ERR_SCRATCH_LIMIT;
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false);
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false, !pl.gemv);
     if (rc) return rc;
     // the scratch keeps whatever the last call left; the publish flags must start at zero
     if (cudaMemsetAsync(d->scratch, 0, static_cast<size_t>(pl.grid) * sizeof(int), st) != cudaSuccess) {

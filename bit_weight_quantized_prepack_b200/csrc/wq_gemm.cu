@@ -1148,11 +1148,266 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     }
 }
 
+// ------------------------------------------------------------------ matrix-vector tiles
+// At M <= 4 a k-block's product is 128 x 128 x M multiply-adds: too little to amortise the
+// tensor-memory chain of the small-tile kernel (dequantise into tensor memory, issue, wait,
+// read the partial back), whose per-k-block cost, not HBM, bounds that kernel at M = 1.
+// Here the dequantised weights never leave registers: each thread multiplies its codes with
+// the activations in fp32 on the CUDA cores.
+//
+// Roles (576 threads): warps 0..15 consume every k-block of the walk; warp w owns weight
+// column row = 32 (w % 4) + lane of the tile and k-block rows 32 hv .. 32 hv + 31, hv = w / 4
+// (its four code words are one 16-byte load, its activations four 16-byte broadcast loads);
+// warp 16 streams the weight blobs and warp 17 the activation rows (one unswizzled tile copy,
+// TM rows of 128 k per k-block) into the same shared-memory ring as the other kernels.
+// Per k-block a thread turns each word into four fp16 pairs of exact (q - z) values (the
+// magic-number conversion), multiplies them with the fp16 activations in fp32 (a mixed
+// f16 x f16 + f32 fused multiply-add: the product of an fp16 and a 4-bit integer is exact in
+// fp32) and adds s * sum into its fp32 accumulators: one scale per thread and k-block for
+// g >= 32, and none for per-column scales (the epilogue applies those). At a segment's end
+// the four row blocks of a column are summed in a fixed order through shared memory and
+// warps 0..3 run the stream-K epilogue of the other kernels (publish, or fix-up and store).
+
+// lo += a.x * w.x and hi += a.y * w.y for two fp16 pairs, in fp32 (one rounding per add)
+__device__ __forceinline__ void fma_f16x2_f32(uint32_t a2, uint32_t w2, float& lo, float& hi) {
+    asm("{\n\t.reg .f16 al, ah, wl, wh;\n\tmov.b32 {al, ah}, %2;\n\tmov.b32 {wl, wh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, al, wl, %0;\n\tfma.rn.f32.f16 %1, ah, wh, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(a2), "r"(w2));
+}
+
+// Epilogue of a matrix-vector tile: thread (quarter, lane) of warps 0..3 holds in v the complete
+// sums of output column n = tile*128 + 32 quarter + lane for rows 0 .. TM - 1 (only rows below
+// M are live). The stream-K protocol is that of the small tiles: a contributor writes its
+// partial and releases its flag; the owner waits for its contributors' flags and adds their
+// partials in descending CTA order.
+template <int MODE, int TM>
+__device__ void epilogue_gemv(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, float (&v)[TM], bool ok,
+                              int quarter, int lane) {
+    const int row = quarter * 32 + lane;
+    const int n = seg.tile * kTileN + row;  // one m-tile: tile index = n-tile index
+    const int live = p.M < TM ? p.M : TM;
+    const bool leader = threadIdx.x == 0;
+    const int me = static_cast<int>(blockIdx.x);
+    if (!seg.owner) {
+        float* part = p.ws_partial + static_cast<size_t>(me) * TM * kTileN;
+        if (ok) {
+#pragma unroll
+            for (int m = 0; m < TM; ++m)
+                if (m < live) part[m * kTileN + row] = v[m];
+        }
+        __threadfence();
+        named_barrier_sync(2, 4 * 32);
+        if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
+        return;
+    }
+    int c_last = me;  // contributors are CTAs c_last .. me - 1
+    if (!seg.whole) {
+        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        const int ncontrib = me - c_last;
+        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
+            bool good = true;
+            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
+            ok = __all_sync(0xffffffffu, good) && ok;
+        }
+        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
+        if (ok) {
+            constexpr int kBatch = 4;
+            for (int j = 0; j < ncontrib; j += kBatch) {
+                float w[kBatch][TM];
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const float* part = p.ws_partial + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
+#pragma unroll
+                    for (int m = 0; m < TM; ++m)
+                        w[b][m] = (j + b < ncontrib && m < live) ? __ldcg(part + m * kTileN + row) : 0.0f;
+                }
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b)
+                    if (j + b < ncontrib) {
+#pragma unroll
+                        for (int m = 0; m < TM; ++m) v[m] += w[b][m];
+                    }
+            }
+        }
+    }
+    if (ok && n < p.N) {
+        const float s_col = (MODE == kModeChannel) ? __half2float(__ushort_as_half(p.s_chan[n])) : 1.0f;
+#pragma unroll
+        for (int m = 0; m < TM; ++m)
+            if (m < live) {
+                const float y = (MODE == kModeChannel) ? v[m] * s_col : v[m];
+                p.y[static_cast<size_t>(m) * p.N + n] = __half_as_ushort(__float2half_rn(y));
+            }
+    }
+    if (!seg.whole) {
+        named_barrier_sync(2, 4 * 32);  // every epilogue warp has read the partials
+        if (leader && !*ctl.abort_flag)
+            for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;
+    }
+}
+
+// Consumer warp of a matrix-vector tile (warps 0..15). red: 2 x 4 x TM x 128 floats of shared
+// memory, one half per segment parity, for the sum over the four row blocks.
+template <int MODE, int TM>
+__device__ void gemv_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
+                          const Ctl& ctl, long long beg, long long end) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, hv = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const int gslot = (32 * hv) / p.group_rows;  // scale / zero slot of this thread's 32 rows
+    // activations of rows 32 hv .. +31: piece hv / 2 of the k-block, half hv % 2 of its 64 k
+    const int act_off = (hv >> 1) * TM * 128 + (hv & 1) * 64;
+    ChunkBar cb;
+    int pos = 0;
+    uint32_t seg_no = 0;
+    bool ok = true;
+    SegCursor seg(beg, end, p.k_blocks);
+    while (seg.next()) {
+        float acc[TM];
+#pragma unroll
+        for (int m = 0; m < TM; ++m) acc[m] = 0.0f;
+        for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const uint32_t fb = cb.bar, fpar = cb.parity;
+            cb.next();
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
+            for (int t = 0; t < c; ++t) {
+                const int s = pos + t;
+                const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                float sc = 1.0f;
+                uint32_t z = 8;
+                if (ok) {
+                    w = reinterpret_cast<const uint4*>(blob)[hv * kTileN + row];
+                    if (is_group(MODE))
+                        sc = __half2float(
+                            __ushort_as_half(reinterpret_cast<const uint16_t*>(blob + kCodeBytes)[gslot * kTileN + row]));
+                    if (MODE == kModeGroupZP) z = blob[p.zp_offset + gslot * kTileN + row];
+                }
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);  // codes, scale and zero are in registers
+                if (ok) {
+                    const uint4* act = reinterpret_cast<const uint4*>(aring + static_cast<size_t>(s) * p.act_slot + act_off);
+                    const uint32_t klo = zp_lo(z), khi = zp_hi(z);
+                    float lo[TM], hi[TM];
+#pragma unroll
+                    for (int m = 0; m < TM; ++m) lo[m] = hi[m] = 0.0f;
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {  // word i: rows 8i .. 8i + 7 of the 32
+                        uint32_t d[4];             // fp16 pairs (q - z) of rows (8i+2k, 8i+2k+1)
+                        dequant_word_f16_zp(wv[i], __half2half2(__ushort_as_half(0x3C00)), false, klo, khi, d);
+#pragma unroll
+                        for (int m = 0; m < TM; ++m) {
+                            const uint4 a = act[m * 8 + i];  // activation row m, the same 8 k (broadcast)
+                            const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) fma_f16x2_f32(av[k], d[k], lo[m], hi[m]);
+                        }
+                    }
+#pragma unroll
+                    for (int m = 0; m < TM; ++m) acc[m] = fmaf(sc, lo[m] + hi[m], acc[m]);
+                }
+                __syncwarp();
+                if (ok && lane == 0) mbar_arrive(&b.empty_a[s]);  // every activation load has completed
+            }
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+        }
+        // the four row blocks of each column, summed in the order hv = 0..3
+        float* rb = red + (seg_no & 1u) * 4 * TM * kTileN;
+#pragma unroll
+        for (int m = 0; m < TM; ++m) rb[(hv * TM + m) * kTileN + row] = acc[m];
+        named_barrier_sync(1, kGemvWarps * 32);
+        ++seg_no;
+        if (hv == 0) {
+            ok = ok && !*ctl.abort_flag;
+            float v[TM];
+#pragma unroll
+            for (int m = 0; m < TM; ++m) {
+                v[m] = rb[m * kTileN + row];
+#pragma unroll
+                for (int h = 1; h < 4; ++h) v[m] += rb[(h * TM + m) * kTileN + row];
+            }
+            epilogue_gemv<MODE, TM>(p, ctl, seg, v, ok, quarter, lane);
+        }
+    }
+}
+
+template <int MODE, int TM>
+__global__ void __launch_bounds__(kThreadsGemv, 1) wq_gemv(const __grid_constant__ ActMaps maps, const GemmArgs p) {
+    extern __shared__ uint8_t smem_dyn[];
+    __shared__ Barriers bars;
+    __shared__ int abort_flag;
+
+    uint8_t* aring = align_ring(smem_dyn);
+    uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
+    float* red = reinterpret_cast<float*>(wring + static_cast<size_t>(p.slots) * p.blob_bytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const long long beg = unit_start(blockIdx.x, p.units, p.grid);
+    const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
+    if (threadIdx.x == 0) griddep_launch_dependents();
+    if (warp == kWeightWarpV && lane == 0) prefetch_first_blobs(p, beg, end);
+    if (warp == 0) {
+        for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
+        for (int s = lane; s < p.slots; s += 32) {
+            mbar_init(&bars.empty_w[s], kGemvWarps);  // every consumer warp reads every k-block
+            mbar_init(&bars.empty_a[s], kGemvWarps);
+        }
+        if (lane == 0) abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kActWarpV && lane == 0)
+        for (int c = 0; c < p.chunk; ++c) prefetch_tensor_map(&maps.m[c]);
+    __syncthreads();
+
+    const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
+    if (warp < kGemvWarps) {
+        gemv_role<MODE, TM>(p, aring, wring, bars, red, ctl, beg, end);
+    } else if (warp == kWeightWarpV) {
+        if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
+    } else {
+        if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
+    }
+}
+
 // ------------------------------------------------------------------ host side
+// Bytes of the matrix-vector kernel's row-block sums (after the ring in dynamic shared memory).
+static int gemv_red_bytes(int tm) { return 2 * 4 * tm * kTileN * 4; }
+
 int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl) {
     pl->mode = mode;
     pl->k_blocks = K / kTileK;
     pl->n_tiles = n_tiles(N);
+    pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
+                     : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
+                                              : kCodeBytes;
+    pl->gemv = mode != kModeW4A8 && M <= kGemvMaxM;
+    if (pl->gemv) {
+        const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
+        pl->tile_m = tm;
+        pl->m_tiles = 1;
+        pl->small = false;
+        pl->threads = kThreadsGemv;
+        pl->issuers = 0;
+        pl->act_slot = tm * 256;  // TM rows x 128 fp16, unswizzled
+        const int budget = smem_optin - 2048 - 1024 - gemv_red_bytes(tm);
+        int s = budget / (pl->act_slot + pl->blob_bytes);
+        if (s > kMaxSlots) s = kMaxSlots;
+        if (s < 2) return -1;
+        pl->slots = s;
+        int c = s / 2;
+        if (c > kMaxChunk) c = kMaxChunk;
+        pl->chunk = c;
+        pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + gemv_red_bytes(tm);
+        pl->units = static_cast<long long>(pl->n_tiles) * pl->k_blocks;
+        pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
+        return 0;
+    }
     int mt = (M + kMaxTileM - 1) / kMaxTileM;
     if (mt < 1) mt = 1;
     int tm = (M + mt - 1) / mt;
@@ -1165,9 +1420,6 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->threads = pl->small ? kThreadsSmall : kThreadsLarge;
     pl->issuers = pl->small ? kMaxIssuers : (tm <= 64 ? 4 : (tm <= 128 ? 2 : 1));
     pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;
-    pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
-                     : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
-                                              : kCodeBytes;
     const int budget = smem_optin - 2048 /* static shared memory */ - 1024 /* alignment slack */;
     int s = budget / (pl->act_slot + pl->blob_bytes);
     if (s > kMaxSlots) s = kMaxSlots;
@@ -1201,6 +1453,15 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeGroupZP>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 32>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 4>, max_dynamic_smem);
     return e;
 }
 
@@ -1228,6 +1489,13 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
 
 template <int MODE>
 static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
+    if constexpr (MODE != kModeW4A8) {
+        if (plan.gemv) {
+            if (plan.tile_m == 1) return launch_kernel(wq_gemv<MODE, 1>, maps, args, plan, st);
+            if (plan.tile_m == 2) return launch_kernel(wq_gemv<MODE, 2>, maps, args, plan, st);
+            return launch_kernel(wq_gemv<MODE, 4>, maps, args, plan, st);
+        }
+    }
     if (!plan.small) return launch_kernel(wq_gemm_large<MODE>, maps, args, plan, st);
     if (plan.tile_m == 16) return launch_kernel(wq_gemm_small<MODE, 16>, maps, args, plan, st);
     return launch_kernel(wq_gemm_small<MODE, 32>, maps, args, plan, st);

@@ -1,12 +1,21 @@
 """CPU tests of the launch planner through wq_plan_for (host arithmetic, no GPU): for a B200's
 148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
 cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
-work."""
+work. W4A16 calls of at most 4 rows get the matrix-vector plan: one tile of 1, 2 or 4 rows,
+576 threads, and the row-block sums in shared memory after the ring."""
 import itertools
 
 import pytest
 
 SMS, SMEM = 148, 232448
+
+
+def _gemv(kind, M):
+    return kind == 0 and M <= 4
+
+
+def _red(p):  # bytes of the matrix-vector kernel's row-block sums
+    return 2 * 4 * p["tile_m"] * 128 * 4
 
 
 @pytest.fixture(scope="module")
@@ -28,7 +37,10 @@ def test_plan_invariants(wq, K, N, kind, g):
     for M in MS:
         p = wq.wq_plan_for(kind, M, N, K, g, SMS, SMEM)
         tm = p["tile_m"]
-        assert tm % 16 == 0 and 16 <= tm <= 256, (M, p)
+        if _gemv(kind, M):
+            assert tm == {1: 1, 2: 2, 3: 4, 4: 4}[M], (M, p)
+        else:
+            assert tm % 16 == 0 and 16 <= tm <= 256, (M, p)
         assert p["m_tiles"] == -(-M // tm), (M, p)                     # the tiles cover M ...
         assert (p["m_tiles"] - 1) * tm < M, (M, p)                      # ... with no empty tile
         assert p["n_tiles"] == -(-N // 128) and p["k_blocks"] == K // 128
@@ -37,9 +49,10 @@ def test_plan_invariants(wq, K, N, kind, g):
         assert 2 <= p["stages"] <= 32
         act = tm * (256 if kind == 0 else 128)
         blob = 8192 + (256 * (128 // min(g, 128)) if kind == 0 and g < K else 0)
-        assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024     # ring + alignment slack
+        red = _red(p) if _gemv(kind, M) else 0
+        assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024 + red  # ring + alignment slack
         assert p["smem_bytes"] + 2048 <= SMEM                           # room for the static barriers
-        assert p["threads"] == 704
+        assert p["threads"] == (576 if _gemv(kind, M) else 704)
 
 
 def test_plan_uses_the_largest_ring_that_fits(wq):
@@ -47,7 +60,7 @@ def test_plan_uses_the_largest_ring_that_fits(wq):
         p = wq.wq_plan_for(kind, M, 4096, 4096, 128 if kind == 0 else 4096, SMS, SMEM)
         act = p["tile_m"] * (256 if kind == 0 else 128)
         blob = 8192 + (256 if kind == 0 else 0)
-        more = (p["stages"] + 1) * (act + blob) + 1024
+        more = (p["stages"] + 1) * (act + blob) + 1024 + (_red(p) if _gemv(kind, M) else 0)
         assert p["stages"] == 32 or more + 2048 > SMEM, p
 
 

@@ -16,12 +16,13 @@ def _wq():
     return wq
 
 
-def test_expired_wait_reports_timeout_and_context_survives():
+@pytest.mark.parametrize("M", [1, 16])  # the matrix-vector and the small-tile kernel
+def test_expired_wait_reports_timeout_and_context_survives(M):
     # CTA 0 holds the first k-blocks of tile 0 and skips publishing its partial, so the CTA
     # that finishes tile 0 waits on a flag nothing sets. With a 20 ms limit the wait expires,
     # the call reports WQ_ERR_TIMEOUT, and the next call is correct.
     wq = _wq()
-    K, N, g, M = 4096, 4096, 128, 1
+    K, N, g = 4096, 4096, 128
     plan = wq.wq_plan(0, M, N, K, g)
     assert plan["units"] > plan["grid"] > 1 and plan["units"] % plan["grid"] != 0
     d = synth.w4a16_inputs(K, N, g, M, seed=3)
@@ -82,21 +83,22 @@ def test_capture_without_reserved_workspace_is_refused():
 
 
 def test_two_streams_concurrently():
-    # Two layers of different shapes and kernels (16-row and large tiles) on two streams, 50
-    # rounds: the kernels may run side by side and their CTAs start in any order and residency.
-    # A split tile is finished by whichever CTA takes its last ticket, so no CTA waits for
-    # another; every round must report WQ_OK and match the oracle.
+    # Three layers of different shapes and kernels (matrix-vector, 16-row and large tiles) on
+    # three streams, 50 rounds: the kernels may run side by side, so a stream-K owner may find
+    # the CTAs it waits for not yet resident; its waits are bounded and no round may time out.
+    # Every round must report WQ_OK and match the oracle.
     import oracle
     from wq_check import compare, half_bits_to_f64
     wq = _wq()
     K, g = 4096, 128
-    cases = [synth.w4a16_inputs(K, 4096, g, 3, seed=6), synth.w4a16_inputs(K, 2048, g, 40, seed=7)]
+    cases = [synth.w4a16_inputs(K, 4096, g, 3, seed=6), synth.w4a16_inputs(K, 2048, g, 40, seed=7),
+             synth.w4a16_inputs(K, 3072, g, 16, seed=8)]
     refs = [(oracle.w4a16(d["A"], d["Q"], d["s"], g), oracle.w4a16_absdot(d["A"], d["Q"], d["s"], g)) for d in cases]
     dev = [(to_dev(d["A"]), wq.wq_prepack(to_dev(d["Q"]), to_dev(d["s"]), g)) for d in cases]
     torch.cuda.synchronize()
-    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    streams = [torch.cuda.Stream() for _ in cases]
     for it in range(50):
-        outs = [None, None]
+        outs = [None] * len(cases)
         for i, (st, (A, Wp)) in enumerate(zip(streams, dev)):
             with torch.cuda.stream(st):
                 outs[i] = wq.wq_gemm_w4a16(A, Wp, cases[i]["N"], g, stream=st)
