@@ -797,3 +797,127 @@ def simulate_ring(units, grid, kbs, slots, na, rng=None, ctas_only=None):
                 moved = True
     stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
     return problems + stuck
+
+
+# ---------------------------------------------------------------------------- matrix-vector tiles
+RED_BUFFERS = 2  # the matrix-vector kernel's row-block sums: one buffer per segment parity
+
+
+def _roles_gemv(cta, units, grid, kbs, chunk, slots, B):
+    """The matrix-vector kernel: 16 consumer warps (row block hv = w / 4, lane quarter w % 4)
+    all read every k-block (empty_w and empty_a count 16 arrivals); at a segment's end each
+    writes its sums into buffer (segment mod RED_BUFFERS), meets the others at a 16-warp
+    barrier, and warps 0..3 (hv = 0) read the four row blocks and run the stream-K epilogue
+    (a 4-warp barrier). Besides barrier operations the roles report ("red_write", segment)
+    and ("red_read", segment): a write into a buffer whose previous segment has not been read
+    by all four epilogue warps is a race."""
+    beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
+
+    def consumer(w):
+        seg_no = 0
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                yield ("red_write", seg_no)
+                yield ("nbar", "red", 16)
+                if w < 4:
+                    yield ("red_read", seg_no)
+                    tile, kb_lo, kb_hi, owner, whole = seg
+                    if not owner:
+                        yield ("nbar", "epi", 4)
+                        if w == 0:
+                            yield ("flag_set", cta)
+                    elif not whole:
+                        for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                            yield ("flag_wait", cc)
+                        yield ("nbar", "epi", 4)
+                seg_no += 1
+                continue
+            yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
+            for t in range(c):
+                yield ("arrive", B["empty_w"][pos + t])
+                yield ("arrive", B["empty_a"][pos + t])
+
+    def producer(which):
+        uses = [0] * slots
+        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
+            if pos is None:
+                continue
+            for t in range(c):
+                yield ("wait", B[which][pos + t], uses[pos + t], it0 + t)
+                uses[pos + t] += 1
+            yield ("arrive", B["full"][ch % NCB])
+
+    roles = {f"cw{w}": consumer(w) for w in range(16)}
+    roles["prod_w"] = producer("empty_w")
+    roles["prod_a"] = producer("empty_a")
+    return roles
+
+
+def simulate_gemv(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
+    """Like simulate, for the matrix-vector kernel; problems also include ("race", cta, segment)
+    for a row-block sum overwritten before the epilogue warps read it."""
+    flags = {}
+    if ctas_only is not None:
+        flags = {c: 1 for c in range(grid) if c not in ctas_only}
+    ctas = []
+    for cta in (range(grid) if ctas_only is None else ctas_only):
+        B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
+             "empty_w": [Bar(16, f"empty_w{s}") for s in range(slots)],
+             "empty_a": [Bar(16, f"empty_a{s}") for s in range(slots)]}
+        roles = _roles_gemv(cta, units, grid, kbs, chunk, slots, B)
+        ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
+                     "nbar": defaultdict(list), "reads": defaultdict(int)})
+    problems = []
+    moved = True
+    while moved:
+        moved = False
+        order = [(st, name) for st in ctas for name in st["roles"]]
+        if rng is not None:
+            rng.shuffle(order)
+        for st, name in order:
+            gen = st["roles"][name]
+            steps = 0
+            while name not in st["done"]:
+                if rng is not None and steps >= rng.randint(1, 4):
+                    moved = True
+                    break
+                steps += 1
+                op = st["cur"][name]
+                if op is None:
+                    try:
+                        op = st["cur"][name] = next(gen)
+                    except StopIteration:
+                        st["done"].add(name)
+                        break
+                kind = op[0]
+                if kind == "wait":
+                    if not op[1].ready(op[2]):
+                        break
+                    if op[1].phase != op[2]:
+                        problems.append(("alias", st["cta"], name, op[1].name, op[2], op[1].phase))
+                elif kind == "flag_wait":
+                    if not flags.get(op[1]):
+                        break
+                elif kind == "arrive":
+                    op[1].arrive()
+                elif kind == "flag_set":
+                    flags[op[1]] = 1
+                elif kind == "red_read":
+                    st["reads"][op[1]] += 1
+                elif kind == "red_write":
+                    prev = op[1] - RED_BUFFERS  # the segment that last used this buffer
+                    if prev >= 0 and st["reads"][prev] < 4:
+                        problems.append(("race", st["cta"], prev))
+                elif kind == "nbar":
+                    waiting = st["nbar"][op[1]]
+                    if name not in waiting:
+                        waiting.append(name)
+                    if len(waiting) < op[2]:
+                        break
+                    for other in waiting:
+                        st["cur"][other] = None
+                    st["nbar"][op[1]] = []
+                st["cur"][name] = None
+                moved = True
+    stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
+    return problems + stuck
