@@ -130,6 +130,15 @@ int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
 }
 
 // Layout of a workspace: flags [grid] int32 at offset 0, partial tiles from offset 4096 on.
+// 1 when the dequant multiplies the group scale into the fp16 weight (one rounding per weight):
+// large tiles always; small tiles for g = 32, 64 (g >= 128 scales each k-block's fp32 partial);
+// register-operand tiles for g = 32 (g >= 64 scales each k-block's fp32 sum).
+int scale_in_dequant(const Plan& pl, int g) {
+    if (pl.mode != kModeGroup && pl.mode != kModeGroupZP) return 0;
+    if (pl.rf) return g < 64 ? 1 : 0;
+    return (!pl.small || g < kTileK) ? 1 : 0;
+}
+
 size_t workspace_bytes_for(const Plan& pl) {
     return 4096 + static_cast<size_t>(pl.grid) * pl.tile_m * kTileN * 4;
 }
@@ -153,7 +162,7 @@ int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* p
 // split into swizzle-wide pieces: dims {64 fp16 or 128 int8, M, K/piece}, strides {K*elem (rows),
 // piece bytes}; a box of {piece, tile_m, c*pieces_per_kblock} lands in shared memory as
 // [piece index][row][128 bytes], the K-major 128-byte-swizzled layout the MMA reads.
-// Unswizzled (swizzle false: the matrix-vector kernel) the box lands as [piece][row][64 fp16].
+// Unswizzled (swizzle false: the register-operand kernel) the box lands as [piece][row][64 fp16].
 int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_m, int chunk, bool int8,
                            bool swizzle = true) {
     const int piece = int8 ? 128 : 64;                 // elements per 128-byte row
@@ -261,7 +270,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
         sa = sq;
     }
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1, !pl.gemv);
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1, !pl.rf);
     if (rc) return rc;
 
     GemmArgs a;
@@ -291,10 +300,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.blob_bytes = pl.blob_bytes;
     a.group_rows = ((kind == 0 || kind == 3) && g < kTileK) ? g : kTileK;
     a.small = pl.small ? 1 : 0;
-    // large tiles round (q - z) * s to fp16 in the dequant; small tiles apply a group scale of
-    // g >= 128 to each k-block's fp32 partial instead (g = 32, 64 stay in the dequant)
-    a.scale_in_dequant =
-        ((pl.mode == kModeGroup || pl.mode == kModeGroupZP) && (!pl.small || g < kTileK)) ? 1 : 0;
+    a.scale_in_dequant = scale_in_dequant(pl, g);
     a.zp_offset = (pl.mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16(scale_slots(K, g))) : 0;
     a.units = pl.units;
     a.grid = pl.grid;
@@ -804,7 +810,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     if (rc) return rc;
     if (workspace_bytes_for(pl) > kNoAllocStatusOffset) return WQ_ERR_SCRATCH_LIMIT;
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false, !pl.gemv);
+    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false, !pl.rf);
     if (rc) return rc;
     // the scratch keeps whatever the last call left; the publish flags must start at zero
     if (cudaMemsetAsync(d->scratch, 0, static_cast<size_t>(pl.grid) * sizeof(int), st) != cudaSuccess) {
@@ -837,7 +843,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     a.blob_bytes = pl.blob_bytes;
     a.group_rows = g < kTileK ? g : kTileK;
     a.small = pl.small ? 1 : 0;
-    a.scale_in_dequant = (pl.mode == kModeGroup && (!pl.small || g < kTileK)) ? 1 : 0;
+    a.scale_in_dequant = scale_in_dequant(pl, g);
     a.units = pl.units;
     a.grid = pl.grid;
     a.timeout_ns = g_timeout_ns;

@@ -1148,42 +1148,46 @@ __global__ void __launch_bounds__(kThreadsSmall, 1)
     }
 }
 
-// ------------------------------------------------------------------ matrix-vector tiles
-// At M <= 4 a k-block's product is 128 x 128 x M multiply-adds: too little to amortise the
-// tensor-memory chain of the small-tile kernel (dequantise into tensor memory, issue, wait,
-// read the partial back), whose per-k-block cost, not HBM, bounds that kernel at M = 1.
-// Here the dequantised weights never leave registers: each thread multiplies its codes with
-// the activations in fp32 on the CUDA cores.
+// ------------------------------------------------------------------ register-operand tiles
+// At M <= 8 a k-block's product is 128 x 128 x M multiply-adds: too little to amortise the
+// tensor-memory chain of the small-tile kernel (dequantise into tensor memory, hand the slot
+// to an issuing thread, wait for its MMAs, read the partial back), whose per-k-block cost, not
+// HBM, bounds that kernel at small M. Here every warp multiplies the weights it has just
+// dequantised, from its own registers, with the warp-level tensor-core instruction
+// (mma.sync m16n8k16, fp16 operands, fp32 accumulation): no cross-warp chain, no tensor memory.
 //
-// Roles (576 threads): warps 0..15 consume every k-block of the walk; warp w owns weight
-// column row = 32 (w % 4) + lane of the tile and k-block rows 32 hv .. 32 hv + 31, hv = w / 4
-// (its four code words are one 16-byte load, its activations four 16-byte broadcast loads);
-// warp 16 streams the weight blobs and warp 17 the activation rows (one unswizzled tile copy,
-// TM rows of 128 k per k-block) into the same shared-memory ring as the other kernels.
-// Per k-block a thread turns each word into four fp16 pairs of exact (q - z) values (the
-// magic-number conversion), multiplies them with the fp16 activations in fp32 (a mixed
-// f16 x f16 + f32 fused multiply-add: the product of an fp16 and a 4-bit integer is exact in
-// fp32) and adds s * sum into its fp32 accumulators: one scale per thread and k-block for
-// g >= 32, and none for per-column scales (the epilogue applies those). At a segment's end
-// the four row blocks of a column are summed in a fixed order through shared memory and
-// warps 0..3 run the stream-K epilogue of the other kernels (publish, or fix-up and store).
+// Roles (576 threads): warps 0..15 consume every k-block of the walk. Warp w owns 16 weight
+// columns 16 (w mod 8) + {0..7, 8..15} and the 64 rows 64 (w / 8) .. + 63 of each k-block (two
+// 32-row blocks A and B); warp 16 streams the weight blobs and warp 17 the activation rows
+// (unswizzled, TM rows of 128 k per k-block) into the shared-memory ring of the other kernels.
+// Lane (g, q) = (lane / 4, lane % 4) loads word q of its two columns g, g + 8 in blocks A and
+// B: four 32-bit loads, 8 rows each. Each word becomes four fp16 pairs of exact (q - z) (the
+// magic-number conversion); pair s of the four words is exactly the lane's A fragment of the
+// s-th MMA (rows = columns g, g + 8; k = the pair's two rows, block A in k 0..7, block B in
+// k 8..15), and pair s of the lane's activation words (rows 8q .. 8q + 7 of blocks A and B of
+// activation row g) its B fragment. The MMA's k order is a permutation of the 64 rows, the
+// same for both operands. The four MMAs of a k-block accumulate in fp32; the group scale
+// multiplies the k-block's sum (acc += s * D) for g >= 64, or the fp16 weight (g = 32, one
+// rounding per weight as in the other kernels); per-column scales wait for the epilogue.
+// At a segment's end the two row halves of each column are summed through shared memory (two
+// buffers by segment parity) and warps 0..3 run the stream-K epilogue of the small tiles.
 
-// lo += a.x * w.x and hi += a.y * w.y for two fp16 pairs, in fp32 (one rounding per add)
-__device__ __forceinline__ void fma_f16x2_f32(uint32_t a2, uint32_t w2, float& lo, float& hi) {
-    asm("{\n\t.reg .f16 al, ah, wl, wh;\n\tmov.b32 {al, ah}, %2;\n\tmov.b32 {wl, wh}, %3;\n\t"
-        "fma.rn.f32.f16 %0, al, wl, %0;\n\tfma.rn.f32.f16 %1, ah, wh, %1;\n\t}"
-        : "+f"(lo), "+f"(hi)
-        : "r"(a2), "r"(w2));
+__device__ __forceinline__ void mma_m16n8k16_f16_f32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Epilogue of a matrix-vector tile: thread (quarter, lane) of warps 0..3 holds in v the complete
-// sums of output column n = tile*128 + 32 quarter + lane for rows 0 .. TM - 1 (only rows below
-// M are live). The stream-K protocol is that of the small tiles: a contributor writes its
-// partial and releases its flag; the owner waits for its contributors' flags and adds their
-// partials in descending CTA order.
+// Epilogue of a register-operand tile: thread (quarter, lane) of warps 0..3 holds in v the
+// complete sums of output column n = tile*128 + 32 quarter + lane for rows 0 .. TM - 1 (only
+// rows below M are live). The stream-K protocol is that of the small tiles: a contributor
+// writes its partial and releases its flag; the owner waits for its contributors' flags and
+// adds their partials in descending CTA order.
 template <int MODE, int TM>
-__device__ void epilogue_gemv(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, float (&v)[TM], bool ok,
-                              int quarter, int lane) {
+__device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, float (&v)[TM], bool ok,
+                            int quarter, int lane) {
     const int row = quarter * 32 + lane;
     const int n = seg.tile * kTileN + row;  // one m-tile: tile index = n-tile index
     const int live = p.M < TM ? p.M : TM;
@@ -1213,7 +1217,7 @@ __device__ void epilogue_gemv(const GemmArgs& p, const Ctl& ctl, const SegCursor
         }
         __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
         if (ok) {
-            constexpr int kBatch = 4;
+            constexpr int kBatch = TM <= 2 ? 4 : 2;
             for (int j = 0; j < ncontrib; j += kBatch) {
                 float w[kBatch][TM];
 #pragma unroll
@@ -1248,26 +1252,35 @@ __device__ void epilogue_gemv(const GemmArgs& p, const Ctl& ctl, const SegCursor
     }
 }
 
-// Consumer warp of a matrix-vector tile (warps 0..15). red: 2 x 4 x TM x 128 floats of shared
-// memory, one half per segment parity, for the sum over the four row blocks.
-template <int MODE, int TM>
-__device__ void gemv_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
-                          const Ctl& ctl, long long beg, long long end) {
+// Consumer warp of a register-operand tile (warps 0..15). kScaled: the group scale multiplies
+// the fp16 weight (g = 32, where the two row blocks of a warp fall in different groups);
+// otherwise the k-block's fp32 sum is scaled (g >= 64), or not at all (per-column scales).
+// red: 2 x 2 x TM x 128 floats of shared memory (segment parity, row half, row, column).
+template <int MODE, int TM, bool kScaled>
+__device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
+                        const Ctl& ctl, long long beg, long long end) {
+    constexpr bool kScaleSum = is_group(MODE) && !kScaled;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quarter = warp & 3, hv = warp >> 2;
-    const int row = quarter * 32 + lane;
-    const int gslot = (32 * hv) / p.group_rows;  // scale / zero slot of this thread's 32 rows
-    // activations of rows 32 hv .. +31: piece hv / 2 of the k-block, half hv % 2 of its 64 k
-    const int act_off = (hv >> 1) * TM * 128 + (hv & 1) * 64;
+    const int g = lane >> 2, q = lane & 3;
+    const int half = warp >> 3;                    // rows 64 half .. + 63: blocks A = 2 half, B = 2 half + 1
+    const int col0 = 16 * (warp & 7) + g;          // this lane's columns col0, col0 + 8
+    const int hvA = 2 * half, hvB = 2 * half + 1;
+    // 32-bit word indices of word q of (column, block) in a blob
+    const int wA0 = (hvA * kTileN + col0) * 4 + q, wA1 = wA0 + 8 * 4;
+    const int wB0 = (hvB * kTileN + col0) * 4 + q, wB1 = wB0 + 8 * 4;
+    const int uA = (32 * hvA) / p.group_rows, uB = (32 * hvB) / p.group_rows;  // scale / zero slots
+    // activation row g (rows past TM read the last one: those MMA columns are not used), words
+    // of rows 8q .. 8q + 7 of blocks A and B
+    const int arow = g < TM ? g : TM - 1;
+    const int aoffA = (hvA >> 1) * TM * 128 + arow * 128 + (hvA & 1) * 64 + 16 * q;
+    const int aoffB = (hvB >> 1) * TM * 128 + arow * 128 + (hvB & 1) * 64 + 16 * q;
     ChunkBar cb;
     int pos = 0;
     uint32_t seg_no = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
-        float acc[TM];
-#pragma unroll
-        for (int m = 0; m < TM; ++m) acc[m] = 0.0f;
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // D fragment: columns col0, col0 + 8 x rows 2q, 2q + 1
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
             const uint32_t fb = cb.bar, fpar = cb.parity;
@@ -1276,69 +1289,99 @@ __device__ void gemv_role(const GemmArgs& p, const uint8_t* aring, const uint8_t
             for (int t = 0; t < c; ++t) {
                 const int s = pos + t;
                 const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
-                uint4 w = make_uint4(0, 0, 0, 0);
-                float sc = 1.0f;
-                uint32_t z = 8;
+                const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
+                const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+                uint32_t w[4] = {0, 0, 0, 0};          // (col0, A), (col0 + 8, A), (col0, B), (col0 + 8, B)
+                uint16_t sc[4] = {0x3C00, 0x3C00, 0x3C00, 0x3C00};
+                uint32_t z[4] = {8, 8, 8, 8};
+                uint4 actA = make_uint4(0, 0, 0, 0), actB = make_uint4(0, 0, 0, 0);
                 if (ok) {
-                    w = reinterpret_cast<const uint4*>(blob)[hv * kTileN + row];
-                    if (is_group(MODE))
-                        sc = __half2float(
-                            __ushort_as_half(reinterpret_cast<const uint16_t*>(blob + kCodeBytes)[gslot * kTileN + row]));
-                    if (MODE == kModeGroupZP) z = blob[p.zp_offset + gslot * kTileN + row];
+                    w[0] = words[wA0];
+                    w[1] = words[wA1];
+                    w[2] = words[wB0];
+                    w[3] = words[wB1];
+                    if (is_group(MODE)) {
+                        sc[0] = scs[uA * kTileN + col0];
+                        sc[1] = scs[uA * kTileN + col0 + 8];
+                        sc[2] = scs[uB * kTileN + col0];
+                        sc[3] = scs[uB * kTileN + col0 + 8];
+                    }
+                    if (MODE == kModeGroupZP) {
+                        z[0] = blob[p.zp_offset + uA * kTileN + col0];
+                        z[1] = blob[p.zp_offset + uA * kTileN + col0 + 8];
+                        z[2] = blob[p.zp_offset + uB * kTileN + col0];
+                        z[3] = blob[p.zp_offset + uB * kTileN + col0 + 8];
+                    }
+                    const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
+                    actA = *reinterpret_cast<const uint4*>(act + aoffA);
+                    actB = *reinterpret_cast<const uint4*>(act + aoffB);
                 }
                 __syncwarp();
-                if (ok && lane == 0) mbar_arrive(&b.empty_w[s]);  // codes, scale and zero are in registers
+                if (ok && lane == 0) {
+                    mbar_arrive(&b.empty_w[s]);
+                    mbar_arrive(&b.empty_a[s]);
+                }
                 if (ok) {
-                    const uint4* act = reinterpret_cast<const uint4*>(aring + static_cast<size_t>(s) * p.act_slot + act_off);
-                    const uint32_t klo = zp_lo(z), khi = zp_hi(z);
-                    float lo[TM], hi[TM];
+                    uint32_t d[4][4];  // d[word][pair s]
 #pragma unroll
-                    for (int m = 0; m < TM; ++m) lo[m] = hi[m] = 0.0f;
-                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                    for (int j = 0; j < 4; ++j)
+                        dequant_word_f16_zp(w[j], __half2half2(__ushort_as_half(sc[j])), kScaled, zp_lo(z[j]),
+                                            zp_hi(z[j]), d[j]);
+                    const uint32_t bA[4] = {actA.x, actA.y, actA.z, actA.w};
+                    const uint32_t bB[4] = {actB.x, actB.y, actB.z, actB.w};
+                    if constexpr (kScaleSum) {
+                        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {  // word i: rows 8i .. 8i + 7 of the 32
-                        uint32_t d[4];             // fp16 pairs (q - z) of rows (8i+2k, 8i+2k+1)
-                        dequant_word_f16_zp(wv[i], __half2half2(__ushort_as_half(0x3C00)), false, klo, khi, d);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t a[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
+                            mma_m16n8k16_f16_f32(part, a, bA[k], bB[k]);
+                        }
+                        // one group per warp and k-block (g >= 64): blocks A and B share the scale
+                        const float s0 = __half2float(__ushort_as_half(sc[0]));
+                        const float s1 = __half2float(__ushort_as_half(sc[1]));
+                        acc[0] = fmaf(s0, part[0], acc[0]);
+                        acc[1] = fmaf(s0, part[1], acc[1]);
+                        acc[2] = fmaf(s1, part[2], acc[2]);
+                        acc[3] = fmaf(s1, part[3], acc[3]);
+                    } else {
 #pragma unroll
-                        for (int m = 0; m < TM; ++m) {
-                            const uint4 a = act[m * 8 + i];  // activation row m, the same 8 k (broadcast)
-                            const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) fma_f16x2_f32(av[k], d[k], lo[m], hi[m]);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t a[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
+                            mma_m16n8k16_f16_f32(acc, a, bA[k], bB[k]);
                         }
                     }
-#pragma unroll
-                    for (int m = 0; m < TM; ++m) acc[m] = fmaf(sc, lo[m] + hi[m], acc[m]);
                 }
-                __syncwarp();
-                if (ok && lane == 0) mbar_arrive(&b.empty_a[s]);  // every activation load has completed
             }
             kb += c;
             pos += c;
             if (pos == p.slots) pos = 0;
         }
-        // the four row blocks of each column, summed in the order hv = 0..3
-        float* rb = red + (seg_no & 1u) * 4 * TM * kTileN;
+        // the two row halves of each column, summed in the order half = 0, 1
+        float* rb = red + (seg_no & 1u) * 2 * TM * kTileN + half * TM * kTileN;
 #pragma unroll
-        for (int m = 0; m < TM; ++m) rb[(hv * TM + m) * kTileN + row] = acc[m];
-        named_barrier_sync(1, kGemvWarps * 32);
-        ++seg_no;
-        if (hv == 0) {
+        for (int j = 0; j < 2; ++j) {
+            const int m = 2 * q + j;
+            if (m < TM) {
+                rb[m * kTileN + col0] = acc[j];
+                rb[m * kTileN + col0 + 8] = acc[2 + j];
+            }
+        }
+        named_barrier_sync(1, kRfWarps * 32);
+        if (warp < 4) {
             ok = ok && !*ctl.abort_flag;
+            const float* r0 = red + (seg_no & 1u) * 2 * TM * kTileN;
+            const int col = warp * 32 + lane;
             float v[TM];
 #pragma unroll
-            for (int m = 0; m < TM; ++m) {
-                v[m] = rb[m * kTileN + row];
-#pragma unroll
-                for (int h = 1; h < 4; ++h) v[m] += rb[(h * TM + m) * kTileN + row];
-            }
-            epilogue_gemv<MODE, TM>(p, ctl, seg, v, ok, quarter, lane);
+            for (int m = 0; m < TM; ++m) v[m] = r0[m * kTileN + col] + r0[(TM + m) * kTileN + col];
+            epilogue_rf<MODE, TM>(p, ctl, seg, v, ok, warp, lane);
         }
+        ++seg_no;
     }
 }
 
 template <int MODE, int TM>
-__global__ void __launch_bounds__(kThreadsGemv, 1) wq_gemv(const __grid_constant__ ActMaps maps, const GemmArgs p) {
+__global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constant__ ActMaps maps, const GemmArgs p) {
     extern __shared__ uint8_t smem_dyn[];
     __shared__ Barriers bars;
     __shared__ int abort_flag;
@@ -1351,24 +1394,27 @@ __global__ void __launch_bounds__(kThreadsGemv, 1) wq_gemv(const __grid_constant
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
     if (threadIdx.x == 0) griddep_launch_dependents();
-    if (warp == kWeightWarpV && lane == 0) prefetch_first_blobs(p, beg, end);
+    if (warp == kWeightWarpR && lane == 0) prefetch_first_blobs(p, beg, end);
     if (warp == 0) {
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
         for (int s = lane; s < p.slots; s += 32) {
-            mbar_init(&bars.empty_w[s], kGemvWarps);  // every consumer warp reads every k-block
-            mbar_init(&bars.empty_a[s], kGemvWarps);
+            mbar_init(&bars.empty_w[s], kRfWarps);  // every consumer warp reads every k-block
+            mbar_init(&bars.empty_a[s], kRfWarps);
         }
         if (lane == 0) abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == kActWarpV && lane == 0)
+    if (warp == kActWarpR && lane == 0)
         for (int c = 0; c < p.chunk; ++c) prefetch_tensor_map(&maps.m[c]);
     __syncthreads();
 
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
-    if (warp < kGemvWarps) {
-        gemv_role<MODE, TM>(p, aring, wring, bars, red, ctl, beg, end);
-    } else if (warp == kWeightWarpV) {
+    if (warp < kRfWarps) {
+        if (is_group(MODE) && p.scale_in_dequant)
+            rf_role<MODE, TM, true>(p, aring, wring, bars, red, ctl, beg, end);
+        else
+            rf_role<MODE, TM, false>(p, aring, wring, bars, red, ctl, beg, end);
+    } else if (warp == kWeightWarpR) {
         if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
@@ -1376,8 +1422,8 @@ __global__ void __launch_bounds__(kThreadsGemv, 1) wq_gemv(const __grid_constant
 }
 
 // ------------------------------------------------------------------ host side
-// Bytes of the matrix-vector kernel's row-block sums (after the ring in dynamic shared memory).
-static int gemv_red_bytes(int tm) { return 2 * 4 * tm * kTileN * 4; }
+// Bytes of the register-operand kernel's row-half sums (after the ring in dynamic shared memory).
+static int rf_red_bytes(int tm) { return 2 * 2 * tm * kTileN * 4; }
 
 int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl) {
     pl->mode = mode;
@@ -1386,16 +1432,16 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
                      : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
                                               : kCodeBytes;
-    pl->gemv = mode != kModeW4A8 && M <= kGemvMaxM;
-    if (pl->gemv) {
-        const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
+    pl->rf = mode != kModeW4A8 && M <= kRfMaxM;
+    if (pl->rf) {
+        const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
         pl->tile_m = tm;
         pl->m_tiles = 1;
         pl->small = false;
-        pl->threads = kThreadsGemv;
+        pl->threads = kThreadsRf;
         pl->issuers = 0;
         pl->act_slot = tm * 256;  // TM rows x 128 fp16, unswizzled
-        const int budget = smem_optin - 2048 - 1024 - gemv_red_bytes(tm);
+        const int budget = smem_optin - 2048 - 1024 - rf_red_bytes(tm);
         int s = budget / (pl->act_slot + pl->blob_bytes);
         if (s > kMaxSlots) s = kMaxSlots;
         if (s < 2) return -1;
@@ -1403,7 +1449,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
         int c = s / 2;
         if (c > kMaxChunk) c = kMaxChunk;
         pl->chunk = c;
-        pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + gemv_red_bytes(tm);
+        pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + rf_red_bytes(tm);
         pl->units = static_cast<long long>(pl->n_tiles) * pl->k_blocks;
         pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
         return 0;
@@ -1453,15 +1499,18 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeGroupZP>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 32>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 1>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 2>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroup, 4>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 1>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 2>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeChannel, 4>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 1>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 2>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemv<kModeGroupZP, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 8>, max_dynamic_smem);
     return e;
 }
 
@@ -1490,10 +1539,11 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
 template <int MODE>
 static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
     if constexpr (MODE != kModeW4A8) {
-        if (plan.gemv) {
-            if (plan.tile_m == 1) return launch_kernel(wq_gemv<MODE, 1>, maps, args, plan, st);
-            if (plan.tile_m == 2) return launch_kernel(wq_gemv<MODE, 2>, maps, args, plan, st);
-            return launch_kernel(wq_gemv<MODE, 4>, maps, args, plan, st);
+        if (plan.rf) {
+            if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1>, maps, args, plan, st);
+            if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2>, maps, args, plan, st);
+            if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4>, maps, args, plan, st);
+            return launch_kernel(wq_gemm_rf<MODE, 8>, maps, args, plan, st);
         }
     }
     if (!plan.small) return launch_kernel(wq_gemm_large<MODE>, maps, args, plan, st);

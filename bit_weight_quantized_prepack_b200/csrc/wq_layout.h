@@ -50,12 +50,12 @@ constexpr int kASlotsS = 4;                   // dequantised k-blocks in tensor 
 constexpr int kSmallTileMax = 32;             // tiles of at most this many rows use per-k-block partials
 constexpr int kTmemAOffsetS = 256;            // small tiles: 2 partials per residue in [0, 256), 4 A slots above
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
-// matrix-vector tiles (M <= kGemvMaxM): CUDA-core dot products, no tensor memory
-constexpr int kGemvMaxM = 4;                  // activation rows handled without the tensor cores
-constexpr int kGemvWarps = 16;                // 4 row blocks of 32 x 4 lane quarters of 32 columns
-constexpr int kWeightWarpV = kGemvWarps;      // warp 16
-constexpr int kActWarpV = kGemvWarps + 1;     // warp 17
-constexpr int kThreadsGemv = (kActWarpV + 1) * 32;  // 576
+// register-operand tiles (M <= kRfMaxM): warp-level MMAs on weights dequantised in registers
+constexpr int kRfMaxM = 8;                  // activation rows of one m16n8k16 MMA
+constexpr int kRfWarps = 16;                // 8 column groups of 16 x 2 row halves of 64
+constexpr int kWeightWarpR = kRfWarps;      // warp 16
+constexpr int kActWarpR = kRfWarps + 1;     // warp 17
+constexpr int kThreadsRf = (kActWarpR + 1) * 32;  // 576
 constexpr int kMaxSlots = 32;                 // shared-memory ring slots (one k-block each)
 constexpr int kMaxChunk = 4;                  // k-blocks moved by one copy
 constexpr int kChunkBars = kMaxSlots + 1;     // chunk barriers: more than ring slots

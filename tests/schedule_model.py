@@ -799,18 +799,18 @@ def simulate_ring(units, grid, kbs, slots, na, rng=None, ctas_only=None):
     return problems + stuck
 
 
-# ---------------------------------------------------------------------------- matrix-vector tiles
-RED_BUFFERS = 2  # the matrix-vector kernel's row-block sums: one buffer per segment parity
+# ---------------------------------------------------------------------------- register-operand tiles
+RED_BUFFERS = 2  # the register-operand kernel's row-half sums: one buffer per segment parity
 
 
-def _roles_gemv(cta, units, grid, kbs, chunk, slots, B):
-    """The matrix-vector kernel: 16 consumer warps (row block hv = w / 4, lane quarter w % 4)
-    all read every k-block (empty_w and empty_a count 16 arrivals); at a segment's end each
-    writes its sums into buffer (segment mod RED_BUFFERS), meets the others at a 16-warp
-    barrier, and warps 0..3 (hv = 0) read the four row blocks and run the stream-K epilogue
-    (a 4-warp barrier). Besides barrier operations the roles report ("red_write", segment)
-    and ("red_read", segment): a write into a buffer whose previous segment has not been read
-    by all four epilogue warps is a race."""
+def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
+    """The register-operand kernel: 16 consumer warps (column group w % 8, row half w / 8) all
+    read every k-block (empty_w and empty_a count 16 arrivals); at a segment's end each writes
+    its sums into buffer (segment mod RED_BUFFERS), meets the others at a 16-warp barrier, and
+    warps 0..3 read both row halves and run the stream-K epilogue (a 4-warp barrier). Besides
+    barrier operations the roles report ("red_write", segment) and ("red_read", segment): a
+    write into a buffer whose previous segment has not been read by all four epilogue warps is
+    a race."""
     beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
 
     def consumer(w):
@@ -853,9 +853,9 @@ def _roles_gemv(cta, units, grid, kbs, chunk, slots, B):
     return roles
 
 
-def simulate_gemv(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
-    """Like simulate, for the matrix-vector kernel; problems also include ("race", cta, segment)
-    for a row-block sum overwritten before the epilogue warps read it."""
+def simulate_rf(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
+    """Like simulate, for the register-operand kernel; problems also include ("race", cta,
+    segment) for a row-half sum overwritten before the epilogue warps read it."""
     flags = {}
     if ctas_only is not None:
         flags = {c: 1 for c in range(grid) if c not in ctas_only}
@@ -864,7 +864,7 @@ def simulate_gemv(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
         B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
              "empty_w": [Bar(16, f"empty_w{s}") for s in range(slots)],
              "empty_a": [Bar(16, f"empty_a{s}") for s in range(slots)]}
-        roles = _roles_gemv(cta, units, grid, kbs, chunk, slots, B)
+        roles = _roles_rf(cta, units, grid, kbs, chunk, slots, B)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
                      "nbar": defaultdict(list), "reads": defaultdict(int)})
     problems = []

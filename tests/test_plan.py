@@ -1,8 +1,8 @@
 """CPU tests of the launch planner through wq_plan_for (host arithmetic, no GPU): for a B200's
 148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
 cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
-work. W4A16 calls of at most 4 rows get the matrix-vector plan: one tile of 1, 2 or 4 rows,
-576 threads, and the row-block sums in shared memory after the ring."""
+work. W4A16 calls of at most 8 rows get the register-operand plan: one tile of 1, 2, 4 or 8
+rows, 576 threads, and the row-half sums in shared memory after the ring."""
 import itertools
 
 import pytest
@@ -10,12 +10,12 @@ import pytest
 SMS, SMEM = 148, 232448
 
 
-def _gemv(kind, M):
-    return kind == 0 and M <= 4
+def _rf(kind, M):
+    return kind == 0 and M <= 8
 
 
-def _red(p):  # bytes of the matrix-vector kernel's row-block sums
-    return 2 * 4 * p["tile_m"] * 128 * 4
+def _red(p):  # bytes of the register-operand kernel's row-half sums
+    return 2 * 2 * p["tile_m"] * 128 * 4
 
 
 @pytest.fixture(scope="module")
@@ -37,8 +37,8 @@ def test_plan_invariants(wq, K, N, kind, g):
     for M in MS:
         p = wq.wq_plan_for(kind, M, N, K, g, SMS, SMEM)
         tm = p["tile_m"]
-        if _gemv(kind, M):
-            assert tm == {1: 1, 2: 2, 3: 4, 4: 4}[M], (M, p)
+        if _rf(kind, M):
+            assert tm == {1: 1, 2: 2, 3: 4, 4: 4, 5: 8, 6: 8, 7: 8, 8: 8}[M], (M, p)
         else:
             assert tm % 16 == 0 and 16 <= tm <= 256, (M, p)
         assert p["m_tiles"] == -(-M // tm), (M, p)                     # the tiles cover M ...
@@ -49,10 +49,10 @@ def test_plan_invariants(wq, K, N, kind, g):
         assert 2 <= p["stages"] <= 32
         act = tm * (256 if kind == 0 else 128)
         blob = 8192 + (256 * (128 // min(g, 128)) if kind == 0 and g < K else 0)
-        red = _red(p) if _gemv(kind, M) else 0
+        red = _red(p) if _rf(kind, M) else 0
         assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024 + red  # ring + alignment slack
         assert p["smem_bytes"] + 2048 <= SMEM                           # room for the static barriers
-        assert p["threads"] == (576 if _gemv(kind, M) else 704)
+        assert p["threads"] == (576 if _rf(kind, M) else 704)
 
 
 def test_plan_uses_the_largest_ring_that_fits(wq):
@@ -60,7 +60,7 @@ def test_plan_uses_the_largest_ring_that_fits(wq):
         p = wq.wq_plan_for(kind, M, 4096, 4096, 128 if kind == 0 else 4096, SMS, SMEM)
         act = p["tile_m"] * (256 if kind == 0 else 128)
         blob = 8192 + (256 if kind == 0 else 0)
-        more = (p["stages"] + 1) * (act + blob) + 1024 + (_red(p) if _gemv(kind, M) else 0)
+        more = (p["stages"] + 1) * (act + blob) + 1024 + (_red(p) if _rf(kind, M) else 0)
         assert p["stages"] == 32 or more + 2048 > SMEM, p
 
 

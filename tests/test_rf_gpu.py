@@ -1,8 +1,9 @@
-"""GPU parity of the matrix-vector kernel (W4A16 calls of at most 4 rows: CUDA-core dot
-products in fp32, no tensor memory) against the fp64 oracle: every scale mode (groups of
-32, 64, 128 and 256 rows, one scale per column, zero points), every tile height (1, 2, 4 rows,
-rows past M zero), ragged N, stream-K splits from whole tiles to 32 CTAs per tile, the full
-layer sizes, bitwise determinism, and identity activations reproducing (q - 8) * s."""
+"""GPU parity of the register-operand kernel (W4A16 calls of at most 8 rows: weights
+dequantised in registers feed warp-level m16n8k16 MMAs, no tensor memory) against the fp64
+oracle: every scale mode (groups of 32, 64, 128 and 256 rows, one scale per column, zero
+points), every tile height (1, 2, 4, 8 rows, rows past M zero), ragged N, stream-K splits from
+whole tiles to 32 CTAs per tile, the full layer sizes, bitwise determinism, and identity
+activations reproducing (q - 8) * s."""
 import numpy as np
 import pytest
 import torch
@@ -25,10 +26,10 @@ def _wq():
 SHAPES = [(128, 8), (4096, 264), (4096, 4096), (11008, 392)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("K,N", SHAPES)
 @pytest.mark.parametrize("g", [32, 64, 128, 256, "K"])
-def test_gemv_vs_oracle(M, K, N, g):
+def test_rf_vs_oracle(M, K, N, g):
     wq = _wq()
     g = K if g == "K" else g
     if K % g:
@@ -40,12 +41,12 @@ def test_gemv_vs_oracle(M, K, N, g):
     Y = wq.wq_gemm_w4a16(to_dev(d["A"]), Wp, N, g)
     torch.cuda.synchronize()
     assert wq.wq_get_device_status() == wq.WQ_OK
-    check_w4a16_full(d, Y, f"gemv K={K} N={N} g={g} M={M}")
+    check_w4a16_full(d, Y, f"rf K={K} N={N} g={g} M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 2, 4])
+@pytest.mark.parametrize("M", [1, 2, 4, 7])
 @pytest.mark.parametrize("K,N,g", [(4096, 264, 64), (4096, 4096, 128), (11008, 392, 32), (2048, 136, 256)])
-def test_gemv_zero_points_vs_oracle(M, K, N, g):
+def test_rf_zero_points_vs_oracle(M, K, N, g):
     wq = _wq()
     d = synth.w4a16_inputs(K, N, g, M, seed=K + M)
     z = np.random.default_rng(K + N).integers(0, 16, (K // g, N)).astype(np.uint8)
@@ -54,13 +55,13 @@ def test_gemv_zero_points_vs_oracle(M, K, N, g):
     torch.cuda.synchronize()
     assert wq.wq_get_device_status() == wq.WQ_OK
     compare(half_bits_to_f64(Y), oracle.w4a16_zp(d["A"], d["Q"], d["s"], z, g),
-            oracle.w4a16_zp_absdot(d["A"], d["Q"], d["s"], z, g), f"gemv zp K={K} N={N} g={g} M={M}")
+            oracle.w4a16_zp_absdot(d["A"], d["Q"], d["s"], z, g), f"rf zp K={K} N={N} g={g} M={M}")
 
 
 @pytest.mark.parametrize("K,N,g", [(4096, 12288, 128), (4096, 22016, 128), (11008, 4096, 128), (8192, 57344, 128),
                                    (8192, 57344, 8192), (28672, 8192, 128)])
-@pytest.mark.parametrize("M", [1, 2])
-def test_gemv_full_layer_sizes_sampled(K, N, g, M):
+@pytest.mark.parametrize("M", [1, 2, 8])
+def test_rf_full_layer_sizes_sampled(K, N, g, M):
     # the bench's launch configuration at full size; the oracle computes sampled columns
     wq = _wq()
     d = synth.w4a16_inputs(K, N, g, M, seed=N + M)
@@ -68,10 +69,10 @@ def test_gemv_full_layer_sizes_sampled(K, N, g, M):
     Y = wq.wq_gemm_w4a16(to_dev(d["A"]), Wp, N, g)
     torch.cuda.synchronize()
     assert wq.wq_get_device_status() == wq.WQ_OK
-    check_w4a16_cols(d, Y, sample_cols(N, 96, seed=M), what=f"gemv full K={K} N={N} g={g} M={M}")
+    check_w4a16_cols(d, Y, sample_cols(N, 96, seed=M), what=f"rf full K={K} N={N} g={g} M={M}")
 
 
-def test_gemv_is_deterministic():
+def test_rf_is_deterministic():
     wq = _wq()
     K, N, g, M = 4096, 4096, 128, 2
     d = synth.w4a16_inputs(K, N, g, M, seed=11)
@@ -81,10 +82,11 @@ def test_gemv_is_deterministic():
         assert torch.equal(wq.wq_gemm_w4a16(A, Wp, N, g).view(torch.int16), Y0.view(torch.int16))
 
 
-@pytest.mark.parametrize("K,g", [(128, 32), (256, 128), (512, 256)])
-def test_gemv_identity_rows_reproduce_weights(K, g):
-    # rows e_k, four at a time (M = 4): y[m, n] = (q[k, n] - 8) * s[k // g, n], exact in fp32, then
-    # one fp16 rounding, the same as the weight's own
+@pytest.mark.parametrize("K,g", [(128, 32), (256, 64), (256, 128), (512, 256)])
+def test_rf_identity_rows_reproduce_weights(K, g):
+    # rows e_k, four at a time (M = 4): y[m, n] = (q[k, n] - 8) * s[k // g, n] (for g = 32 the
+    # weight rounded to fp16 once, otherwise exact in fp32), then one fp16 rounding: either way
+    # the weight's own fp16 value
     wq = _wq()
     N = 136
     d = synth.w4a16_inputs(K, N, g, 1, seed=K + g)

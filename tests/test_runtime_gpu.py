@@ -16,7 +16,7 @@ def _wq():
     return wq
 
 
-@pytest.mark.parametrize("M", [1, 16])  # the matrix-vector and the small-tile kernel
+@pytest.mark.parametrize("M", [1, 16])  # the register-operand and the small-tile kernel
 def test_expired_wait_reports_timeout_and_context_survives(M):
     # CTA 0 holds the first k-blocks of tile 0 and skips publishing its partial, so the CTA
     # that finishes tile 0 waits on a flag nothing sets. With a 20 ms limit the wait expires,
@@ -83,7 +83,7 @@ def test_capture_without_reserved_workspace_is_refused():
 
 
 def test_two_streams_concurrently():
-    # Three layers of different shapes and kernels (matrix-vector, 16-row and large tiles) on
+    # Three layers of different shapes and kernels (register-operand, 16-row and large tiles) on
     # three streams, 50 rounds: the kernels may run side by side, so a stream-K owner may find
     # the CTAs it waits for not yet resident; its waits are bounded and no round may time out.
     # Every round must report WQ_OK and match the oracle.

@@ -389,10 +389,10 @@ def test_ring_model_catches_planted_mistake(na, flag, value, monkeypatch):
     assert _ring_problems_everywhere(na=na), f"{flag} = {value} went unnoticed at {na} slots"
 
 
-# ---------------------------------------------------------------------------- matrix-vector tiles
-_GEMV_BIASES = {
+# ---------------------------------------------------------------------------- register-operand tiles
+_RF_BIASES = {
     "consumers-first": lambda n: n.startswith("cw"), "producers-first": lambda n: n.startswith("prod"),
-    "row-blocks-1-3-first": lambda n: n.startswith("cw") and int(n[2:]) >= 4,   # run a segment ahead
+    "non-epilogue-warps-first": lambda n: n.startswith("cw") and int(n[2:]) >= 4,  # run a segment ahead
     "epilogue-warps-first": lambda n: n in ("cw0", "cw1", "cw2", "cw3"),
     "one-consumer-first": lambda n: n == "cw7", "one-consumer-last": lambda n: n != "cw0",
 }
@@ -400,24 +400,24 @@ _GEMV_BIASES = {
 
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 264), (11008, 4096), (4096, 22016), (128, 8), (384, 1000)])
 @pytest.mark.parametrize("slots", [2, 5, 13, 25])
-def test_gemv_no_alias_deadlock_or_race(K, N, slots):
-    # every consumer warp reads every k-block; the row-block sums alternate between two
-    # buffers by segment, so a warp that runs a segment ahead never overwrites sums the
-    # epilogue warps have not read
+def test_rf_no_alias_deadlock_or_race(K, N, slots):
+    # every consumer warp reads every k-block; the row-half sums alternate between two buffers
+    # by segment, so a warp that runs a segment ahead never overwrites sums the epilogue warps
+    # have not read
     import random
-    from schedule_model import simulate_gemv
+    from schedule_model import simulate_rf
     units, grid, kbs = _plan(K, N)
     chunk = max(1, min(4, slots // 2))
-    assert not simulate_gemv(units, grid, kbs, chunk, slots)
+    assert not simulate_rf(units, grid, kbs, chunk, slots)
     for cta in sorted({0, 1, grid // 2, grid - 1}):
-        for name, first in _GEMV_BIASES.items():
-            problems = simulate_gemv(units, grid, kbs, chunk, slots, rng=_Biased(first, cta), ctas_only=[cta])
+        for name, first in _RF_BIASES.items():
+            problems = simulate_rf(units, grid, kbs, chunk, slots, rng=_Biased(first, cta), ctas_only=[cta])
             assert not problems, (name, cta, problems[:3])
-        problems = simulate_gemv(units, grid, kbs, chunk, slots, rng=random.Random(cta), ctas_only=[cta])
+        problems = simulate_rf(units, grid, kbs, chunk, slots, rng=random.Random(cta), ctas_only=[cta])
         assert not problems, ("random", cta, problems[:3])
 
 
-def test_gemv_model_catches_a_single_sum_buffer():
+def test_rf_model_catches_a_single_sum_buffer():
     # with one buffer a consumer warp that has finished its next segment overwrites the sums
     # while the epilogue warps may still be reading them
     import schedule_model as sm
@@ -427,8 +427,8 @@ def test_gemv_model_catches_a_single_sum_buffer():
     try:
         races = []
         for cta in range(8):
-            for name, first in _GEMV_BIASES.items():
-                races += [p for p in sm.simulate_gemv(units, grid, kbs, 4, 13, rng=_Biased(first, cta), ctas_only=[cta])
+            for name, first in _RF_BIASES.items():
+                races += [p for p in sm.simulate_rf(units, grid, kbs, 4, 13, rng=_Biased(first, cta), ctas_only=[cta])
                           if p[0] == "race"]
     finally:
         sm.RED_BUFFERS = saved

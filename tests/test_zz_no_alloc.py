@@ -34,9 +34,10 @@ def _c_abi(wq, A, Wp, Y, N, g):
                                         ctypes.c_void_p(Y.data_ptr()), M, N, K, g, stream)
 
 
-# (K, N, g, M): 16-row tile; 32-row tile; a 48-row large tile; per-column scales on 16- and 32-row tiles
+# (K, N, g, M): 16-row tile; 32-row tile; a 48-row large tile; per-column scales on the
+# register-operand kernel (M = 3), 16- and 32-row tiles; the register-operand kernel at M = 1
 CASES = [(4096, 1032, 128, 5), (1024, 1032, 128, 28), (2048, 2056, 64, 40), (2048, 520, 2048, 3),
-         (1024, 264, 1024, 24)]
+         (2048, 520, 2048, 12), (1024, 264, 1024, 24), (4096, 1032, 64, 1)]
 
 
 @pytest.mark.parametrize("K,N,g,M", CASES)
