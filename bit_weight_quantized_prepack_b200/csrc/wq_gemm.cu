@@ -1252,131 +1252,198 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
     }
 }
 
-// Consumer warp of a register-operand tile (warps 0..15). kScaled: the group scale multiplies
-// the fp16 weight (g = 32, where the two row blocks of a warp fall in different groups);
-// otherwise the k-block's fp32 sum is scaled (g >= 64), or not at all (per-column scales).
-// red: 2 x 2 x TM x 128 floats of shared memory (segment parity, row half, row, column).
-template <int MODE, int TM, bool kScaled>
+// How the register-operand consumer applies the group scale.
+enum RfScale : int {
+    kRfScaleNone = 0,     // per-column scales: the epilogue multiplies
+    kRfScaleWeight = 1,   // g = 32: the fp16 weight (one rounding per weight)
+    kRfScalePair = 2,     // g = 64: each 64-row pair's fp32 sum
+    kRfScaleBlock = 3,    // g >= 128: each k-block's fp32 sum
+};
+
+// Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
+// k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
+// of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
+// 32 cg + 16 tau + g and + 8, tau = 0, 1) and two 64-row pairs (blocks A = 2p, B = 2p + 1).
+// red: 4 x TM x 128 floats of shared memory (residue, row, column).
+template <int MODE, int TM, int SCALE>
 __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
                         const Ctl& ctl, long long beg, long long end) {
-    constexpr bool kScaleSum = is_group(MODE) && !kScaled;
+    constexpr int NB = (TM + 7) / 8;  // MMAs of 8 activation rows per k-step
+    constexpr bool kScaled = SCALE == kRfScaleWeight;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t r = static_cast<uint32_t>(warp >> 2);
+    const int cg = warp & 3;
     const int g = lane >> 2, q = lane & 3;
-    const int half = warp >> 3;                    // rows 64 half .. + 63: blocks A = 2 half, B = 2 half + 1
-    const int col0 = 16 * (warp & 7) + g;          // this lane's columns col0, col0 + 8
-    const int hvA = 2 * half, hvB = 2 * half + 1;
-    // 32-bit word indices of word q of (column, block) in a blob
-    const int wA0 = (hvA * kTileN + col0) * 4 + q, wA1 = wA0 + 8 * 4;
-    const int wB0 = (hvB * kTileN + col0) * 4 + q, wB1 = wB0 + 8 * 4;
-    const int uA = (32 * hvA) / p.group_rows, uB = (32 * hvB) / p.group_rows;  // scale / zero slots
-    // activation row g (rows past TM read the last one: those MMA columns are not used), words
-    // of rows 8q .. 8q + 7 of blocks A and B
-    const int arow = g < TM ? g : TM - 1;
-    const int aoffA = (hvA >> 1) * TM * 128 + arow * 128 + (hvA & 1) * 64 + 16 * q;
-    const int aoffB = (hvB >> 1) * TM * 128 + arow * 128 + (hvB & 1) * 64 + 16 * q;
+    const int colb = 32 * cg + g;  // columns colb + 16 tau + 8 j
+    int aoff[NB];                  // activation row 8 nb + g (clamped to TM - 1), rows 8q .. 8q + 7 of block A of pair 0
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const int arow = 8 * nb + g < TM ? 8 * nb + g : TM - 1;
+        aoff[nb] = arow * 128 + 16 * q;
+    }
     ChunkBar cb;
+    uint32_t iter = 0;
     int pos = 0;
-    uint32_t seg_no = 0;
     bool ok = true;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // D fragment: columns col0, col0 + 8 x rows 2q, 2q + 1
+        float acc[2][NB][4];  // [tau][nb]: columns colb + 16 tau + {0, 8} x rows 8 nb + 2q + {0, 1}
+#pragma unroll
+        for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) acc[tau][nb][0] = acc[tau][nb][1] = acc[tau][nb][2] = acc[tau][nb][3] = 0.0f;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
             const uint32_t fb = cb.bar, fpar = cb.parity;
             cb.next();
-            if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
-            for (int t = 0; t < c; ++t) {
-                const int s = pos + t;
+            if (chunk_has(iter, c, 4, r)) {
+                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
+                const int s = pos + static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block
                 const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
                 const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
                 const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
-                uint32_t w[4] = {0, 0, 0, 0};          // (col0, A), (col0 + 8, A), (col0, B), (col0 + 8, B)
-                uint16_t sc[4] = {0x3C00, 0x3C00, 0x3C00, 0x3C00};
-                uint32_t z[4] = {8, 8, 8, 8};
-                uint4 actA = make_uint4(0, 0, 0, 0), actB = make_uint4(0, 0, 0, 0);
+                const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
+                uint32_t w[2][2][2][2];  // [pair][block A/B][tau][j]
                 if (ok) {
-                    w[0] = words[wA0];
-                    w[1] = words[wA1];
-                    w[2] = words[wB0];
-                    w[3] = words[wB1];
-                    if (is_group(MODE)) {
-                        sc[0] = scs[uA * kTileN + col0];
-                        sc[1] = scs[uA * kTileN + col0 + 8];
-                        sc[2] = scs[uB * kTileN + col0];
-                        sc[3] = scs[uB * kTileN + col0 + 8];
-                    }
-                    if (MODE == kModeGroupZP) {
-                        z[0] = blob[p.zp_offset + uA * kTileN + col0];
-                        z[1] = blob[p.zp_offset + uA * kTileN + col0 + 8];
-                        z[2] = blob[p.zp_offset + uB * kTileN + col0];
-                        z[3] = blob[p.zp_offset + uB * kTileN + col0 + 8];
-                    }
-                    const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
-                    actA = *reinterpret_cast<const uint4*>(act + aoffA);
-                    actB = *reinterpret_cast<const uint4*>(act + aoffB);
-                }
-                __syncwarp();
-                if (ok && lane == 0) {
-                    mbar_arrive(&b.empty_w[s]);
-                    mbar_arrive(&b.empty_a[s]);
-                }
-                if (ok) {
-                    uint32_t d[4][4];  // d[word][pair s]
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        dequant_word_f16_zp(w[j], __half2half2(__ushort_as_half(sc[j])), kScaled, zp_lo(z[j]),
-                                            zp_hi(z[j]), d[j]);
-                    const uint32_t bA[4] = {actA.x, actA.y, actA.z, actA.w};
-                    const uint32_t bB[4] = {actB.x, actB.y, actB.z, actB.w};
-                    if constexpr (kScaleSum) {
-                        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t a[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
-                            mma_m16n8k16_f16_f32(part, a, bA[k], bB[k]);
+                        for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+                            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                                for (int j = 0; j < 2; ++j)
+                                    w[pp][bb][tau][j] = words[((2 * pp + bb) * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
+                }
+                uint16_t scb[2][2] = {{0x3C00, 0x3C00}, {0x3C00, 0x3C00}};  // kRfScaleBlock: [tau][j]
+                if (ok && SCALE == kRfScaleBlock) {
+#pragma unroll
+                    for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) scb[tau][j] = scs[colb + 16 * tau + 8 * j];
+                }
+                float part[2][NB][4];
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {  // 64-row pair pp: blocks 2pp (k 0..7 of each MMA) and 2pp + 1 (k 8..15)
+                    uint16_t sc[2][2][2] = {{{0x3C00, 0x3C00}, {0x3C00, 0x3C00}}, {{0x3C00, 0x3C00}, {0x3C00, 0x3C00}}};
+                    uint32_t z[2][2][2] = {{{8, 8}, {8, 8}}, {{8, 8}, {8, 8}}};  // [block][tau][j]
+                    if (ok && (SCALE == kRfScaleWeight || SCALE == kRfScalePair || MODE == kModeGroupZP)) {
+#pragma unroll
+                        for (int bb = 0; bb < 2; ++bb) {
+                            const int u = (32 * (2 * pp + bb)) / p.group_rows;
+#pragma unroll
+                            for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                                for (int j = 0; j < 2; ++j) {
+                                    const int col = colb + 16 * tau + 8 * j;
+                                    if (SCALE == kRfScaleWeight || SCALE == kRfScalePair) sc[bb][tau][j] = scs[u * kTileN + col];
+                                    if (MODE == kModeGroupZP) z[bb][tau][j] = blob[p.zp_offset + u * kTileN + col];
+                                }
                         }
-                        // one group per warp and k-block (g >= 64): blocks A and B share the scale
-                        const float s0 = __half2float(__ushort_as_half(sc[0]));
-                        const float s1 = __half2float(__ushort_as_half(sc[1]));
-                        acc[0] = fmaf(s0, part[0], acc[0]);
-                        acc[1] = fmaf(s0, part[1], acc[1]);
-                        acc[2] = fmaf(s1, part[2], acc[2]);
-                        acc[3] = fmaf(s1, part[3], acc[3]);
-                    } else {
+                    }
+                    uint4 actA[NB], actB[NB];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t a[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
-                            mma_m16n8k16_f16_f32(acc, a, bA[k], bB[k]);
+                    for (int nb = 0; nb < NB; ++nb) {
+                        actA[nb] = ok ? *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb]) : make_uint4(0, 0, 0, 0);
+                        actB[nb] = ok ? *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb] + 64)
+                                      : make_uint4(0, 0, 0, 0);
+                    }
+                    if (pp == 1) {  // the last reads of this ring slot are in flight or done
+                        __syncwarp();
+                        if (ok && lane == 0) {
+                            mbar_arrive(&b.empty_w[s]);
+                            mbar_arrive(&b.empty_a[s]);
+                        }
+                    }
+                    if (ok) {
+#pragma unroll
+                        for (int tau = 0; tau < 2; ++tau) {
+                            uint32_t d[4][4];  // fragment register order: (A, j0), (A, j1), (B, j0), (B, j1); pair s
+#pragma unroll
+                            for (int bb = 0; bb < 2; ++bb)
+#pragma unroll
+                                for (int j = 0; j < 2; ++j) {
+                                    const uint32_t zz = z[bb][tau][j];
+                                    dequant_word_f16_zp(w[pp][bb][tau][j], __half2half2(__ushort_as_half(sc[bb][tau][j])),
+                                                        kScaled, zp_lo(zz), zp_hi(zz), d[2 * bb + j]);
+                                }
+#pragma unroll
+                            for (int nb = 0; nb < NB; ++nb) {
+                                const uint32_t bA[4] = {actA[nb].x, actA[nb].y, actA[nb].z, actA[nb].w};
+                                const uint32_t bB[4] = {actB[nb].x, actB[nb].y, actB[nb].z, actB[nb].w};
+                                float* dst = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau][nb] : acc[tau][nb];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const uint32_t afrag[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
+                                    float (&dd)[4] = *reinterpret_cast<float (*)[4]>(dst);
+                                    mma_m16n8k16_f16_f32(dd, afrag, bA[k], bB[k]);
+                                }
+                                if (SCALE == kRfScalePair) {  // both blocks of the pair share the group
+                                    const float s0 = __half2float(__ushort_as_half(sc[0][tau][0]));
+                                    const float s1 = __half2float(__ushort_as_half(sc[0][tau][1]));
+                                    acc[tau][nb][0] = fmaf(s0, part[tau][nb][0], acc[tau][nb][0]);
+                                    acc[tau][nb][1] = fmaf(s0, part[tau][nb][1], acc[tau][nb][1]);
+                                    acc[tau][nb][2] = fmaf(s1, part[tau][nb][2], acc[tau][nb][2]);
+                                    acc[tau][nb][3] = fmaf(s1, part[tau][nb][3], acc[tau][nb][3]);
+                                    part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
+                                }
+                            }
+                        }
+                    }
+                }
+                if (ok && SCALE == kRfScaleBlock) {  // one group for the whole k-block
+#pragma unroll
+                    for (int tau = 0; tau < 2; ++tau) {
+                        const float s0 = __half2float(__ushort_as_half(scb[tau][0]));
+                        const float s1 = __half2float(__ushort_as_half(scb[tau][1]));
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            acc[tau][nb][0] = fmaf(s0, part[tau][nb][0], acc[tau][nb][0]);
+                            acc[tau][nb][1] = fmaf(s0, part[tau][nb][1], acc[tau][nb][1]);
+                            acc[tau][nb][2] = fmaf(s1, part[tau][nb][2], acc[tau][nb][2]);
+                            acc[tau][nb][3] = fmaf(s1, part[tau][nb][3], acc[tau][nb][3]);
                         }
                     }
                 }
             }
+            iter += c;
             kb += c;
             pos += c;
             if (pos == p.slots) pos = 0;
         }
-        // the two row halves of each column, summed in the order half = 0, 1
-        float* rb = red + (seg_no & 1u) * 2 * TM * kTileN + half * TM * kTileN;
+        // the residues' sums of each column, added in the order r = 0..3 by warps 0..3
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int m = 2 * q + j;
-            if (m < TM) {
-                rb[m * kTileN + col0] = acc[j];
-                rb[m * kTileN + col0 + 8] = acc[2 + j];
+        for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int m = 8 * nb + 2 * q + jj;
+                    if (m < TM) {
+                        red[(r * TM + m) * kTileN + colb + 16 * tau] = acc[tau][nb][jj];
+                        red[(r * TM + m) * kTileN + colb + 16 * tau + 8] = acc[tau][nb][2 + jj];
+                    }
+                }
+        named_barrier_sync(1, kRfWarps * 32);
+        float v[TM];
+        if (warp < 4) {
+            const int col = warp * 32 + lane;
+#pragma unroll
+            for (int m = 0; m < TM; ++m) {
+                v[m] = red[m * kTileN + col];
+#pragma unroll
+                for (int rr = 1; rr < 4; ++rr) v[m] += red[(rr * TM + m) * kTileN + col];
             }
         }
-        named_barrier_sync(1, kRfWarps * 32);
+        named_barrier_sync(1, kRfWarps * 32);  // the sums are read: the next segment may write them
         if (warp < 4) {
             ok = ok && !*ctl.abort_flag;
-            const float* r0 = red + (seg_no & 1u) * 2 * TM * kTileN;
-            const int col = warp * 32 + lane;
-            float v[TM];
-#pragma unroll
-            for (int m = 0; m < TM; ++m) v[m] = r0[m * kTileN + col] + r0[(TM + m) * kTileN + col];
             epilogue_rf<MODE, TM>(p, ctl, seg, v, ok, warp, lane);
         }
-        ++seg_no;
     }
 }
 
@@ -1398,8 +1465,8 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
     if (warp == 0) {
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
         for (int s = lane; s < p.slots; s += 32) {
-            mbar_init(&bars.empty_w[s], kRfWarps);  // every consumer warp reads every k-block
-            mbar_init(&bars.empty_a[s], kRfWarps);
+            mbar_init(&bars.empty_w[s], 4);  // the k-block's residue: 4 column-group warps
+            mbar_init(&bars.empty_a[s], 4);
         }
         if (lane == 0) abort_flag = 0;
         fence_barrier_init();
@@ -1410,10 +1477,16 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
 
     const Ctl ctl{&abort_flag, p.status, p.timeout_ns};
     if (warp < kRfWarps) {
-        if (is_group(MODE) && p.scale_in_dequant)
-            rf_role<MODE, TM, true>(p, aring, wring, bars, red, ctl, beg, end);
-        else
-            rf_role<MODE, TM, false>(p, aring, wring, bars, red, ctl, beg, end);
+        if constexpr (is_group(MODE)) {
+            if (p.scale_in_dequant)
+                rf_role<MODE, TM, kRfScaleWeight>(p, aring, wring, bars, red, ctl, beg, end);
+            else if (p.group_rows < kTileK)
+                rf_role<MODE, TM, kRfScalePair>(p, aring, wring, bars, red, ctl, beg, end);
+            else
+                rf_role<MODE, TM, kRfScaleBlock>(p, aring, wring, bars, red, ctl, beg, end);
+        } else {
+            rf_role<MODE, TM, kRfScaleNone>(p, aring, wring, bars, red, ctl, beg, end);
+        }
     } else if (warp == kWeightWarpR) {
         if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
@@ -1422,8 +1495,8 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
 }
 
 // ------------------------------------------------------------------ host side
-// Bytes of the register-operand kernel's row-half sums (after the ring in dynamic shared memory).
-static int rf_red_bytes(int tm) { return 2 * 2 * tm * kTileN * 4; }
+// Bytes of the register-operand kernel's residue sums (after the ring in dynamic shared memory).
+static int rf_red_bytes(int tm) { return 4 * tm * kTileN * 4; }
 
 int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl) {
     pl->mode = mode;
@@ -1434,7 +1507,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
                                               : kCodeBytes;
     pl->rf = mode != kModeW4A8 && M <= kRfMaxM;
     if (pl->rf) {
-        const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8));
+        const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : (M <= 8 ? 8 : (M <= 16 ? 16 : 32))));
         pl->tile_m = tm;
         pl->m_tiles = 1;
         pl->small = false;
@@ -1511,6 +1584,16 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 8>, max_dynamic_smem);
+    if constexpr (kRfMaxM > 8) {
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 16>, max_dynamic_smem);
+    }
+    if constexpr (kRfMaxM > 16) {
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 32>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 32>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 32>, max_dynamic_smem);
+    }
     return e;
 }
 
@@ -1543,6 +1626,12 @@ static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const 
             if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1>, maps, args, plan, st);
             if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2>, maps, args, plan, st);
             if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4>, maps, args, plan, st);
+            if constexpr (kRfMaxM > 8) {
+                if (plan.tile_m == 16) return launch_kernel(wq_gemm_rf<MODE, 16>, maps, args, plan, st);
+            }
+            if constexpr (kRfMaxM > 16) {
+                if (plan.tile_m == 32) return launch_kernel(wq_gemm_rf<MODE, 32>, maps, args, plan, st);
+            }
             return launch_kernel(wq_gemm_rf<MODE, 8>, maps, args, plan, st);
         }
     }

@@ -800,20 +800,24 @@ def simulate_ring(units, grid, kbs, slots, na, rng=None, ctas_only=None):
 
 
 # ---------------------------------------------------------------------------- register-operand tiles
-RED_BUFFERS = 2  # the register-operand kernel's row-half sums: one buffer per segment parity
+RED_SECOND_BARRIER = True  # the residue sums: one buffer, a second barrier once they are read
 
 
 def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
-    """The register-operand kernel: 16 consumer warps (column group w % 8, row half w / 8) all
-    read every k-block (empty_w and empty_a count 16 arrivals); at a segment's end each writes
-    its sums into buffer (segment mod RED_BUFFERS), meets the others at a 16-warp barrier, and
-    warps 0..3 read both row halves and run the stream-K epilogue (a 4-warp barrier). Besides
-    barrier operations the roles report ("red_write", segment) and ("red_read", segment): a
-    write into a buffer whose previous segment has not been read by all four epilogue warps is
-    a race."""
+    """The register-operand kernel: 16 consumer warps in 4 residues (walk index mod 4) x 4 column
+    groups; the 4 warps of a k-block's residue read it (empty_w and empty_a count 4 arrivals).
+    At a segment's end every warp writes its sums into the one buffer, all meet at a 16-warp
+    barrier, warps 0..3 read the four residues' sums, all meet again (RED_SECOND_BARRIER) and
+    warps 0..3 run the stream-K epilogue (a 4-warp barrier). Besides barrier operations the
+    roles report ("red_write", segment) and ("red_read", segment): a write while the previous
+    segment's sums have not been read by all four epilogue warps is a race."""
     beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
 
+    def has(it0, c, residue):
+        return ((residue + 4 - it0 % 4) % 4) < c
+
     def consumer(w):
+        residue = w >> 2
         seg_no = 0
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
@@ -821,6 +825,9 @@ def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
                 yield ("nbar", "red", 16)
                 if w < 4:
                     yield ("red_read", seg_no)
+                if RED_SECOND_BARRIER:
+                    yield ("nbar", "red", 16)
+                if w < 4:
                     tile, kb_lo, kb_hi, owner, whole = seg
                     if not owner:
                         yield ("nbar", "epi", 4)
@@ -832,10 +839,13 @@ def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
                         yield ("nbar", "epi", 4)
                 seg_no += 1
                 continue
+            if not has(it0, c, residue):
+                continue
             yield ("wait", B["full"][ch % NCB], ch // NCB + 1, it0)
             for t in range(c):
-                yield ("arrive", B["empty_w"][pos + t])
-                yield ("arrive", B["empty_a"][pos + t])
+                if (it0 + t) % 4 == residue:
+                    yield ("arrive", B["empty_w"][pos + t])
+                    yield ("arrive", B["empty_a"][pos + t])
 
     def producer(which):
         uses = [0] * slots
@@ -855,15 +865,15 @@ def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
 
 def simulate_rf(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
     """Like simulate, for the register-operand kernel; problems also include ("race", cta,
-    segment) for a row-half sum overwritten before the epilogue warps read it."""
+    segment) for a residue sum overwritten before the epilogue warps read it."""
     flags = {}
     if ctas_only is not None:
         flags = {c: 1 for c in range(grid) if c not in ctas_only}
     ctas = []
     for cta in (range(grid) if ctas_only is None else ctas_only):
         B = {"full": [Bar(2, f"full{k}") for k in range(NCB)],
-             "empty_w": [Bar(16, f"empty_w{s}") for s in range(slots)],
-             "empty_a": [Bar(16, f"empty_a{s}") for s in range(slots)]}
+             "empty_w": [Bar(4, f"empty_w{s}") for s in range(slots)],
+             "empty_a": [Bar(4, f"empty_a{s}") for s in range(slots)]}
         roles = _roles_rf(cta, units, grid, kbs, chunk, slots, B)
         ctas.append({"cta": cta, "roles": roles, "cur": dict.fromkeys(roles), "done": set(),
                      "nbar": defaultdict(list), "reads": defaultdict(int)})
@@ -905,7 +915,7 @@ def simulate_rf(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
                 elif kind == "red_read":
                     st["reads"][op[1]] += 1
                 elif kind == "red_write":
-                    prev = op[1] - RED_BUFFERS  # the segment that last used this buffer
+                    prev = op[1] - 1  # the segment that last used the buffer
                     if prev >= 0 and st["reads"][prev] < 4:
                         problems.append(("race", st["cta"], prev))
                 elif kind == "nbar":

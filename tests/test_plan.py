@@ -2,7 +2,7 @@
 148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
 cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
 work. W4A16 calls of at most 8 rows get the register-operand plan: one tile of 1, 2, 4 or 8
-rows, 576 threads, and the row-half sums in shared memory after the ring."""
+rows, 576 threads, and the residue sums in shared memory after the ring."""
 import itertools
 
 import pytest
@@ -14,8 +14,8 @@ def _rf(kind, M):
     return kind == 0 and M <= 8
 
 
-def _red(p):  # bytes of the register-operand kernel's row-half sums
-    return 2 * 2 * p["tile_m"] * 128 * 4
+def _red(p):  # bytes of the register-operand kernel's residue sums
+    return 4 * p["tile_m"] * 128 * 4
 
 
 @pytest.fixture(scope="module")

@@ -393,6 +393,7 @@ def test_ring_model_catches_planted_mistake(na, flag, value, monkeypatch):
 _RF_BIASES = {
     "consumers-first": lambda n: n.startswith("cw"), "producers-first": lambda n: n.startswith("prod"),
     "non-epilogue-warps-first": lambda n: n.startswith("cw") and int(n[2:]) >= 4,  # run a segment ahead
+    "one-residue-first": lambda n: n in ("cw12", "cw13", "cw14", "cw15"),
     "epilogue-warps-first": lambda n: n in ("cw0", "cw1", "cw2", "cw3"),
     "one-consumer-first": lambda n: n == "cw7", "one-consumer-last": lambda n: n != "cw0",
 }
@@ -401,9 +402,9 @@ _RF_BIASES = {
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 264), (11008, 4096), (4096, 22016), (128, 8), (384, 1000)])
 @pytest.mark.parametrize("slots", [2, 5, 13, 25])
 def test_rf_no_alias_deadlock_or_race(K, N, slots):
-    # every consumer warp reads every k-block; the row-half sums alternate between two buffers
-    # by segment, so a warp that runs a segment ahead never overwrites sums the epilogue warps
-    # have not read
+    # a k-block is read by its residue's 4 warps; the residue sums share one buffer, and a second
+    # barrier after the epilogue warps have read them keeps a warp that runs a segment ahead
+    # from overwriting them
     import random
     from schedule_model import simulate_rf
     units, grid, kbs = _plan(K, N)
@@ -417,13 +418,13 @@ def test_rf_no_alias_deadlock_or_race(K, N, slots):
         assert not problems, ("random", cta, problems[:3])
 
 
-def test_rf_model_catches_a_single_sum_buffer():
-    # with one buffer a consumer warp that has finished its next segment overwrites the sums
-    # while the epilogue warps may still be reading them
+def test_rf_model_catches_a_missing_second_barrier():
+    # without the second barrier a consumer warp that has finished its next segment overwrites
+    # the sums while the epilogue warps may still be reading them
     import schedule_model as sm
     units, grid, kbs = _plan(4096, 22016)  # several segments per CTA
-    saved = sm.RED_BUFFERS
-    sm.RED_BUFFERS = 1
+    saved = sm.RED_SECOND_BARRIER
+    sm.RED_SECOND_BARRIER = False
     try:
         races = []
         for cta in range(8):
@@ -431,5 +432,5 @@ def test_rf_model_catches_a_single_sum_buffer():
                 races += [p for p in sm.simulate_rf(units, grid, kbs, 4, 13, rng=_Biased(first, cta), ctas_only=[cta])
                           if p[0] == "race"]
     finally:
-        sm.RED_BUFFERS = saved
+        sm.RED_SECOND_BARRIER = saved
     assert races
