@@ -526,10 +526,11 @@ def run_ours(args, rank, world, local_rank):
                                    "speedup_vs_fp16_bound": round(fp16_bound_time(1, 4096, 4096, hbm_gbs) / t, 2)})
 
     # ---------------------------------------------------------- the dominant kernel's roofline
-    # The calls at M <= 16 run the 16-row small-tile kernel, the largest share of the step's device
-    # time. They are captured in their own graph, in the step's order and weight copies, and timed
-    # like the step (events on the launching stream around whole replays).
-    dom_ms = [M for M in M_SWEEP if M <= 16]
+    # The calls whose plan is the register-operand kernel (576 threads: the small M of decoding)
+    # take the largest share of the step's device time. They are captured in their own graph, in
+    # the step's order and weight copies, and timed like the step (events on the launching stream
+    # around whole replays).
+    dom_ms = [M for M in M_SWEEP if wq.wq_plan(0, M, LAYERS[0][1], LAYERS[0][0], G)["threads"] == 576]
     dom_calls = [(mi, M, L) for mi, M in enumerate(M_SWEEP) if M in dom_ms for L in layers]
     gd = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -575,13 +576,14 @@ def run_ours(args, rank, world, local_rank):
                                   "bytes / measured copy bandwidth, flops / measured bf16 peak), over the step's "
                                   "device time (M = 64 and 128 are past the ridge, so a pure bandwidth fraction "
                                   "of the whole step would understate them)"},
-        "roofline": {"bound": "hbm", "kernel": "wq_gemm_small<fp16 groups, 16-row tiles> (the step's M <= 16 calls)",
+        "roofline": {"bound": "hbm", "kernel": f"wq_gemm_rf<fp16 groups> (register-operand tiles: the step's "
+                                                f"M = {', '.join(map(str, dom_ms))} calls)",
                      "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(achieved / hbm_gbs, 3), "traffic": traffic,
                      "traffic_algo_bytes": round(b_dom),
                      "launch_us": round(t_dom * 1e6, 2),
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth), of measured",
-                     "note": f"achieved = average algorithmic bytes per launch of the {len(dom_calls)} M <= 16 calls "
+                     "note": f"achieved = average algorithmic bytes per launch of the {len(dom_calls)} calls "
                              f"(weights + scales + A + Y) / their average launch duration, CUDA events over "
                              f"{dom_reps} replays of a graph holding just those calls in the step's order"},
         "c1_4096x4096_M1": c1_row,

@@ -1260,6 +1260,51 @@ enum RfScale : int {
     kRfScaleBlock = 3,    // g >= 128: each k-block's fp32 sum
 };
 
+// Pair s (rows 2s, 2s + 1 of the word's 8) of a code word as fp16 (q - z), with the constants
+// klo = zp_lo(z), khi = zp_hi(z) and x8 = x >> 8; times the fp16 scale sc when kScaled. The
+// four pairs of a word are dequant_word_f16_zp's four outputs, one at a time, so that the
+// register-operand consumer builds each MMA's A fragment from the same pair of four words.
+template <int S, bool kScaled>
+__device__ __forceinline__ uint32_t pair_f16(uint32_t x, uint32_t x8, uint32_t klo, uint32_t khi, __half2 sc) {
+    const uint32_t kMagic = 0x64006400u;
+    const __half2 kSixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));
+    __half2 h;
+    if constexpr (S == 0) {
+        const uint32_t u = lop3_and_or(x, 0x000F000Fu, kMagic);
+        h = __hsub2(half2_bits(u), half2_bits(klo));
+    } else if constexpr (S == 1) {
+        const uint32_t u = lop3_and_or(x, 0x00F000F0u, kMagic);
+        h = __hfma2(half2_bits(u), kSixteenth, half2_bits(khi));
+    } else if constexpr (S == 2) {
+        const uint32_t u = lop3_and_or(x8, 0x000F000Fu, kMagic);
+        h = __hsub2(half2_bits(u), half2_bits(klo));
+    } else {
+        const uint32_t u = lop3_and_or(x8, 0x00F000F0u, kMagic);
+        h = __hfma2(half2_bits(u), kSixteenth, half2_bits(khi));
+    }
+    if constexpr (kScaled) h = __hmul2(h, sc);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The four MMAs (pairs s = 0..3) of one row tile and one 64-row pair: A fragment of MMA s =
+// pair s of the words (block A, column j = 0), (A, 1), (B, 0), (B, 1); B fragment = pair s of the
+// activation words of blocks A and B.
+template <int S, bool kScaled, int NB>
+__device__ __forceinline__ void rf_mma_pair(const uint32_t (&x)[4], const uint32_t (&x8)[4], const uint32_t (&klo)[4],
+                                            const uint32_t (&khi)[4], const __half2 (&sc)[4], const uint4 (&actA)[NB],
+                                            const uint4 (&actB)[NB], float (&d)[NB][4]) {
+    const uint32_t afrag[4] = {pair_f16<S, kScaled>(x[0], x8[0], klo[0], khi[0], sc[0]),
+                               pair_f16<S, kScaled>(x[1], x8[1], klo[1], khi[1], sc[1]),
+                               pair_f16<S, kScaled>(x[2], x8[2], klo[2], khi[2], sc[2]),
+                               pair_f16<S, kScaled>(x[3], x8[3], klo[3], khi[3], sc[3])};
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        const uint32_t bA = S == 0 ? actA[nb].x : (S == 1 ? actA[nb].y : (S == 2 ? actA[nb].z : actA[nb].w));
+        const uint32_t bB = S == 0 ? actB[nb].x : (S == 1 ? actB[nb].y : (S == 2 ? actB[nb].z : actB[nb].w));
+        mma_m16n8k16_f16_f32(d[nb], afrag, bA, bB);
+    }
+}
+
 // Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
 // k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
 // of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
@@ -1270,6 +1315,7 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                         const Ctl& ctl, long long beg, long long end) {
     constexpr int NB = (TM + 7) / 8;  // MMAs of 8 activation rows per k-step
     constexpr bool kScaled = SCALE == kRfScaleWeight;
+    constexpr bool kPerBlock = SCALE == kRfScaleWeight || SCALE == kRfScalePair || MODE == kModeGroupZP;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t r = static_cast<uint32_t>(warp >> 2);
     const int cg = warp & 3;
@@ -1295,125 +1341,117 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
             const uint32_t fb = cb.bar, fpar = cb.parity;
+            const int s = pos + static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block, if any
+            const bool mine = chunk_has(iter, c, 4, r);
             cb.next();
-            if (chunk_has(iter, c, 4, r)) {
-                if (ok) ok = __all_sync(0xffffffffu, wait_bar(&b.full[fb], fpar, ctl));
-                const int s = pos + static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block
-                const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
-                const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
-                const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
-                const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
-                uint32_t w[2][2][2][2];  // [pair][block A/B][tau][j]
-                if (ok) {
+            iter += c;
+            kb += c;
+            pos += c;
+            if (pos == p.slots) pos = 0;
+            if (!mine) continue;
+            ok = __all_sync(0xffffffffu, ok && wait_bar(&b.full[fb], fpar, ctl));
+            if (!ok) continue;  // an expired wait: the CTA winds down (nothing more is read or released)
+            const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
+            const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
+            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+            const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
+            uint32_t w[2][2][2][2];  // [pair][block A/B][tau][j]
 #pragma unroll
-                    for (int pp = 0; pp < 2; ++pp)
+            for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
-                        for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-                            for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-                                for (int j = 0; j < 2; ++j)
-                                    w[pp][bb][tau][j] = words[((2 * pp + bb) * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
-                }
-                uint16_t scb[2][2] = {{0x3C00, 0x3C00}, {0x3C00, 0x3C00}};  // kRfScaleBlock: [tau][j]
-                if (ok && SCALE == kRfScaleBlock) {
+                for (int bb = 0; bb < 2; ++bb)
 #pragma unroll
                     for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) scb[tau][j] = scs[colb + 16 * tau + 8 * j];
-                }
-                float part[2][NB][4];
+                        for (int j = 0; j < 2; ++j)
+                            w[pp][bb][tau][j] = words[((2 * pp + bb) * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
+            float scb[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // kRfScaleBlock: [tau][j]
+            if (SCALE == kRfScaleBlock) {
 #pragma unroll
                 for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
+                    for (int j = 0; j < 2; ++j) scb[tau][j] = __half2float(__ushort_as_half(scs[colb + 16 * tau + 8 * j]));
+            }
+            float part[2][NB][4];
 #pragma unroll
-                for (int pp = 0; pp < 2; ++pp) {  // 64-row pair pp: blocks 2pp (k 0..7 of each MMA) and 2pp + 1 (k 8..15)
-                    uint16_t sc[2][2][2] = {{{0x3C00, 0x3C00}, {0x3C00, 0x3C00}}, {{0x3C00, 0x3C00}, {0x3C00, 0x3C00}}};
-                    uint32_t z[2][2][2] = {{{8, 8}, {8, 8}}, {{8, 8}, {8, 8}}};  // [block][tau][j]
-                    if (ok && (SCALE == kRfScaleWeight || SCALE == kRfScalePair || MODE == kModeGroupZP)) {
+            for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                        for (int bb = 0; bb < 2; ++bb) {
-                            const int u = (32 * (2 * pp + bb)) / p.group_rows;
+                for (int nb = 0; nb < NB; ++nb) part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
 #pragma unroll
-                            for (int tau = 0; tau < 2; ++tau)
+            for (int pp = 0; pp < 2; ++pp) {  // 64-row pair pp: blocks 2pp (k 0..7 of each MMA) and 2pp + 1 (k 8..15)
+                __half2 sc[2][4];    // [tau][fragment register]
+                uint32_t klo[2][4], khi[2][4];
 #pragma unroll
-                                for (int j = 0; j < 2; ++j) {
-                                    const int col = colb + 16 * tau + 8 * j;
-                                    if (SCALE == kRfScaleWeight || SCALE == kRfScalePair) sc[bb][tau][j] = scs[u * kTileN + col];
-                                    if (MODE == kModeGroupZP) z[bb][tau][j] = blob[p.zp_offset + u * kTileN + col];
-                                }
-                        }
+                for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                    for (int f = 0; f < 4; ++f) {
+                        sc[tau][f] = __half2half2(__ushort_as_half(0x3C00));
+                        klo[tau][f] = zp_lo(8);
+                        khi[tau][f] = zp_hi(8);
                     }
-                    uint4 actA[NB], actB[NB];
+                if (kPerBlock) {
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        actA[nb] = ok ? *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb]) : make_uint4(0, 0, 0, 0);
-                        actB[nb] = ok ? *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb] + 64)
-                                      : make_uint4(0, 0, 0, 0);
-                    }
-                    if (pp == 1) {  // the last reads of this ring slot are in flight or done
-                        __syncwarp();
-                        if (ok && lane == 0) {
-                            mbar_arrive(&b.empty_w[s]);
-                            mbar_arrive(&b.empty_a[s]);
-                        }
-                    }
-                    if (ok) {
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const int u = (32 * (2 * pp + bb)) / p.group_rows;
 #pragma unroll
-                        for (int tau = 0; tau < 2; ++tau) {
-                            uint32_t d[4][4];  // fragment register order: (A, j0), (A, j1), (B, j0), (B, j1); pair s
+                        for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                            for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-                                for (int j = 0; j < 2; ++j) {
-                                    const uint32_t zz = z[bb][tau][j];
-                                    dequant_word_f16_zp(w[pp][bb][tau][j], __half2half2(__ushort_as_half(sc[bb][tau][j])),
-                                                        kScaled, zp_lo(zz), zp_hi(zz), d[2 * bb + j]);
-                                }
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb) {
-                                const uint32_t bA[4] = {actA[nb].x, actA[nb].y, actA[nb].z, actA[nb].w};
-                                const uint32_t bB[4] = {actB[nb].x, actB[nb].y, actB[nb].z, actB[nb].w};
-                                float* dst = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau][nb] : acc[tau][nb];
-#pragma unroll
-                                for (int k = 0; k < 4; ++k) {
-                                    const uint32_t afrag[4] = {d[0][k], d[1][k], d[2][k], d[3][k]};
-                                    float (&dd)[4] = *reinterpret_cast<float (*)[4]>(dst);
-                                    mma_m16n8k16_f16_f32(dd, afrag, bA[k], bB[k]);
-                                }
-                                if (SCALE == kRfScalePair) {  // both blocks of the pair share the group
-                                    const float s0 = __half2float(__ushort_as_half(sc[0][tau][0]));
-                                    const float s1 = __half2float(__ushort_as_half(sc[0][tau][1]));
-                                    acc[tau][nb][0] = fmaf(s0, part[tau][nb][0], acc[tau][nb][0]);
-                                    acc[tau][nb][1] = fmaf(s0, part[tau][nb][1], acc[tau][nb][1]);
-                                    acc[tau][nb][2] = fmaf(s1, part[tau][nb][2], acc[tau][nb][2]);
-                                    acc[tau][nb][3] = fmaf(s1, part[tau][nb][3], acc[tau][nb][3]);
-                                    part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
+                            for (int j = 0; j < 2; ++j) {
+                                const int col = colb + 16 * tau + 8 * j;
+                                if (SCALE == kRfScaleWeight || SCALE == kRfScalePair)
+                                    sc[tau][2 * bb + j] = __half2half2(__ushort_as_half(scs[u * kTileN + col]));
+                                if (MODE == kModeGroupZP) {
+                                    const uint32_t zz = blob[p.zp_offset + u * kTileN + col];
+                                    klo[tau][2 * bb + j] = zp_lo(zz);
+                                    khi[tau][2 * bb + j] = zp_hi(zz);
                                 }
                             }
-                        }
                     }
                 }
-                if (ok && SCALE == kRfScaleBlock) {  // one group for the whole k-block
+                uint4 actA[NB], actB[NB];
 #pragma unroll
-                    for (int tau = 0; tau < 2; ++tau) {
-                        const float s0 = __half2float(__ushort_as_half(scb[tau][0]));
-                        const float s1 = __half2float(__ushort_as_half(scb[tau][1]));
+                for (int nb = 0; nb < NB; ++nb) {
+                    actA[nb] = *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb]);
+                    actB[nb] = *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb] + 64);
+                }
+                if (pp == 1) {  // the last reads of this ring slot are issued: release it
+                    __syncwarp();
+                    mbar_arrive_if(&b.empty_w[s], lane == 0);
+                    mbar_arrive_if(&b.empty_a[s], lane == 0);
+                }
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau) {
+                    const uint32_t x[4] = {w[pp][0][tau][0], w[pp][0][tau][1], w[pp][1][tau][0], w[pp][1][tau][1]};
+                    const uint32_t x8[4] = {x[0] >> 8, x[1] >> 8, x[2] >> 8, x[3] >> 8};
+                    float (&dst)[NB][4] = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau] : acc[tau];
+                    rf_mma_pair<0, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
+                    rf_mma_pair<1, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
+                    rf_mma_pair<2, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
+                    rf_mma_pair<3, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
+                    if (SCALE == kRfScalePair) {  // both blocks of the pair share the group
+                        const float s0 = __low2float(sc[tau][0]), s1 = __low2float(sc[tau][1]);
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb) {
                             acc[tau][nb][0] = fmaf(s0, part[tau][nb][0], acc[tau][nb][0]);
                             acc[tau][nb][1] = fmaf(s0, part[tau][nb][1], acc[tau][nb][1]);
                             acc[tau][nb][2] = fmaf(s1, part[tau][nb][2], acc[tau][nb][2]);
                             acc[tau][nb][3] = fmaf(s1, part[tau][nb][3], acc[tau][nb][3]);
+                            part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
                         }
                     }
                 }
             }
-            iter += c;
-            kb += c;
-            pos += c;
-            if (pos == p.slots) pos = 0;
+            if (SCALE == kRfScaleBlock) {  // one group for the whole k-block
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        acc[tau][nb][0] = fmaf(scb[tau][0], part[tau][nb][0], acc[tau][nb][0]);
+                        acc[tau][nb][1] = fmaf(scb[tau][0], part[tau][nb][1], acc[tau][nb][1]);
+                        acc[tau][nb][2] = fmaf(scb[tau][1], part[tau][nb][2], acc[tau][nb][2]);
+                        acc[tau][nb][3] = fmaf(scb[tau][1], part[tau][nb][3], acc[tau][nb][3]);
+                    }
+            }
         }
         // the residues' sums of each column, added in the order r = 0..3 by warps 0..3
 #pragma unroll
