@@ -298,7 +298,8 @@ __device__ void epilogue(const GemmArgs& p, Barriers& b, uint32_t tmem, const Ct
                 for (int j = 0; j < 8; ++j) part[static_cast<size_t>(c_begin + c + j) * kTileN + row] = v[j];
             }
         }
-        __threadfence();
+        // the barrier orders every thread's partial stores before the leader's release of the flag
+        // (the release is cumulative), so no thread needs a GPU-scope fence of its own
         tc_fence_before();
         named_barrier_sync(1, kNumDqWarps * 32);  // also: every warp has read the accumulators
         if (threadIdx.x == 0 && ok && !*ctl.abort_flag && static_cast<int>(blockIdx.x) != p.skip_publish)
@@ -764,7 +765,7 @@ __device__ void epilogue_small(const GemmArgs& p, const Ctl& ctl, const SegCurso
             for (int c = 0; c < H; ++c)
                 if (c < live) part[static_cast<size_t>(r0 + c) * kTileN + row] = v[c];
         }
-        __threadfence();
+        // the barrier orders every thread's partial stores before the leader's (cumulative) release
         named_barrier_sync(2, kDqWarpsS * 32);
         if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
         return;
@@ -1200,7 +1201,7 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
             for (int m = 0; m < TM; ++m)
                 if (m < live) part[m * kTileN + row] = v[m];
         }
-        __threadfence();
+        // the barrier orders every thread's partial stores before the leader's (cumulative) release
         named_barrier_sync(2, 4 * 32);
         if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
         return;
