@@ -148,11 +148,15 @@ struct SegCursor {
 };
 
 // Length of the chunk that starts at k-block kb of a segment ending at kb_hi, at ring slot pos:
-// at most `chunk` k-blocks, never past the segment, never wrapping the ring.
-__device__ __forceinline__ int chunk_len(int chunk, int kb, int kb_hi, int pos, int slots) {
+// at most `chunk` k-blocks, never past the segment, never wrapping the ring. The CTA's first
+// chunk (first: walk index 0) is one k-block: every CTA asks for its first chunk at the same
+// moment, when the grid dependency resolves, and the smaller it is the sooner the consumers
+// start (the rest streams in behind it).
+__device__ __forceinline__ int chunk_len(int chunk, int kb, int kb_hi, int pos, int slots, bool first) {
     int c = kb_hi - kb + 1;
     if (c > chunk) c = chunk;
     if (c > slots - pos) c = slots - pos;
+    if (first && c > 1) c = 1;
     return c;
 }
 
@@ -400,7 +404,7 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, iter == 0);
             const uint32_t fb = cb.bar, fpar = cb.parity;
             cb.next();
             const bool mine = ((residue + kDqResidues - iter % kDqResidues) % kDqResidues) < static_cast<uint32_t>(c);
@@ -492,7 +496,7 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
         const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
         const uint8_t* wtile = p.wp + static_cast<size_t>(nt) * p.k_blocks * p.blob_bytes;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, ch == 0);
             for (int t = 0; t < c; ++t) {
                 const int s = pos + t;
                 if (ok && ch >= first_pass_chunks)  // a slot's first use needs no wait
@@ -548,7 +552,7 @@ __device__ void issuer_role(int q, const GemmArgs& p, const uint8_t* aring, Barr
     while (seg.next()) {
         bool first = true;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, iter == 0);
             if (ok) ok = wait_bar(&b.full[cb.bar], cb.parity, ctl);
             cb.next();
             for (int t = 0; t < c; ++t, ++iter) {
@@ -870,7 +874,7 @@ __device__ void dequant_role_small(const GemmArgs& p, const uint8_t* wring, Barr
         bool pending = false;                      // a k-block of this segment whose partial is not added yet
         float sc_pending = 1.0f;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, iter == 0);
             const uint32_t fb = cb.bar, fpar = cb.parity;
             cb.next();
             if (chunk_has(iter, c, 4, r)) {
@@ -1034,7 +1038,7 @@ __device__ void issuer_role_small(int r, const GemmArgs& p, const uint8_t* aring
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, iter == 0);
             const uint32_t fb = cb.bar, fpar = cb.parity;
             cb.next();
             if (chunk_has(iter, c, 4, static_cast<uint32_t>(r))) {
@@ -1181,13 +1185,21 @@ __device__ __forceinline__ void mma_m16n8k16_f16_f32(float (&d)[4], const uint32
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_m16n8k32_s8_s32(uint32_t (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // Epilogue of a register-operand tile: thread (quarter, lane) of warps 0..3 holds in v the
 // complete sums of output column n = tile*128 + 32 quarter + lane for rows 0 .. TM - 1 (only
 // rows below M are live). The stream-K protocol is that of the small tiles: a contributor
 // writes its partial and releases its flag; the owner waits for its contributors' flags and
 // adds their partials in descending CTA order.
 template <int MODE, int TM>
-__device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, float (&v)[TM], bool ok,
+__device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM], bool ok,
                             int quarter, int lane) {
     const int row = quarter * 32 + lane;
     const int n = seg.tile * kTileN + row;  // one m-tile: tile index = n-tile index
@@ -1195,7 +1207,7 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
     const bool leader = threadIdx.x == 0;
     const int me = static_cast<int>(blockIdx.x);
     if (!seg.owner) {
-        float* part = p.ws_partial + static_cast<size_t>(me) * TM * kTileN;
+        uint32_t* part = reinterpret_cast<uint32_t*>(p.ws_partial) + static_cast<size_t>(me) * TM * kTileN;
         if (ok) {
 #pragma unroll
             for (int m = 0; m < TM; ++m)
@@ -1220,30 +1232,42 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
         if (ok) {
             constexpr int kBatch = TM <= 2 ? 4 : 2;
             for (int j = 0; j < ncontrib; j += kBatch) {
-                float w[kBatch][TM];
+                uint32_t w[kBatch][TM];
 #pragma unroll
                 for (int b = 0; b < kBatch; ++b) {
-                    const float* part = p.ws_partial + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
+                    const uint32_t* part =
+                        reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
 #pragma unroll
-                    for (int m = 0; m < TM; ++m)
-                        w[b][m] = (j + b < ncontrib && m < live) ? __ldcg(part + m * kTileN + row) : 0.0f;
+                    for (int m = 0; m < TM; ++m) w[b][m] = (j + b < ncontrib && m < live) ? __ldcg(part + m * kTileN + row) : 0u;
                 }
 #pragma unroll
                 for (int b = 0; b < kBatch; ++b)
                     if (j + b < ncontrib) {
 #pragma unroll
-                        for (int m = 0; m < TM; ++m) v[m] += w[b][m];
+                        for (int m = 0; m < TM; ++m)
+                            v[m] = (MODE == kModeW4A8)
+                                       ? static_cast<uint32_t>(static_cast<int32_t>(v[m]) + static_cast<int32_t>(w[b][m]))
+                                       : __float_as_uint(__uint_as_float(v[m]) + __uint_as_float(w[b][m]));
                     }
             }
         }
     }
     if (ok && n < p.N) {
         const float s_col = (MODE == kModeChannel) ? __half2float(__ushort_as_half(p.s_chan[n])) : 1.0f;
+        const float sw_col = (MODE == kModeW4A8) ? p.sw[n] : 0.0f;
 #pragma unroll
         for (int m = 0; m < TM; ++m)
             if (m < live) {
-                const float y = (MODE == kModeChannel) ? v[m] * s_col : v[m];
-                p.y[static_cast<size_t>(m) * p.N + n] = __half_as_ushort(__float2half_rn(y));
+                const size_t o = static_cast<size_t>(m) * p.N + n;
+                float y;
+                if (MODE == kModeW4A8) {
+                    const int32_t acc = static_cast<int32_t>(v[m]) >> 4;  // the codes were 16 (q - 8)
+                    if (p.acc_out) p.acc_out[o] = acc;
+                    y = (static_cast<float>(acc) * p.sa[m]) * sw_col;
+                } else {
+                    y = (MODE == kModeChannel) ? __uint_as_float(v[m]) * s_col : __uint_as_float(v[m]);
+                }
+                p.y[o] = __half_as_ushort(__float2half_rn(y));
             }
     }
     if (!seg.whole) {
@@ -1306,6 +1330,28 @@ __device__ __forceinline__ void rf_mma_pair(const uint32_t (&x)[4], const uint32
     }
 }
 
+// W4A8: the two MMAs (k = 32 each) of one row tile and one 64-row pair. Word q of a column in a
+// block holds rows 8q .. 8q + 7; dequant_word_i8 gives them as int8 16 (q - 8) in two registers
+// (rows 8q + 4s .. + 3, s = 0, 1), and MMA s takes register s of the block A words as its k 0..15
+// quarter-rows and of the block B words as k 16..31, with the matching activation registers.
+template <int NB>
+__device__ __forceinline__ void rf_mma_pair_i8(const uint32_t (&x)[4], const uint2 (&actA)[NB], const uint2 (&actB)[NB],
+                                               uint32_t (&d)[NB][4]) {
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int f = 0; f < 4; ++f) {
+        uint32_t o[2];
+        dequant_word_i8(x[f], o);
+        lo[f] = o[0];
+        hi[f] = o[1];
+    }
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+        mma_m16n8k32_s8_s32(d[nb], lo, actA[nb].x, actB[nb].x);
+        mma_m16n8k32_s8_s32(d[nb], hi, actA[nb].y, actB[nb].y);
+    }
+}
+
 // Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
 // k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
 // of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
@@ -1335,12 +1381,16 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         float acc[2][NB][4];  // [tau][nb]: columns colb + 16 tau + {0, 8} x rows 8 nb + 2q + {0, 1}
+        uint32_t iacc[2][NB][4];  // W4A8: the same, exact int32
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) acc[tau][nb][0] = acc[tau][nb][1] = acc[tau][nb][2] = acc[tau][nb][3] = 0.0f;
+            for (int nb = 0; nb < NB; ++nb) {
+                acc[tau][nb][0] = acc[tau][nb][1] = acc[tau][nb][2] = acc[tau][nb][3] = 0.0f;
+                iacc[tau][nb][0] = iacc[tau][nb][1] = iacc[tau][nb][2] = iacc[tau][nb][3] = 0u;
+            }
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
-            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots);
+            const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, iter == 0);
             const uint32_t fb = cb.bar, fpar = cb.parity;
             const int s = pos + static_cast<int>((r + 4 - iter % 4) % 4);  // this residue's k-block, if any
             const bool mine = chunk_has(iter, c, 4, r);
@@ -1356,6 +1406,34 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
             const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
             const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
+            if constexpr (MODE == kModeW4A8) {
+                // int8 activation rows of 128 bytes: row arow, block hv, word q at arow*128 + 32 hv + 8q
+                uint32_t x[2][2][4];  // [pair][tau][fragment register]: (A, j0), (A, j1), (B, j0), (B, j1)
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                    for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                        for (int f = 0; f < 4; ++f)
+                            x[pp][tau][f] = words[((2 * pp + (f >> 1)) * kTileN + colb + 16 * tau + 8 * (f & 1)) * 4 + q];
+                uint2 actA[2][NB], actB[2][NB];
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        const int base = (aoff[nb] - 16 * q) + 64 * pp + 8 * q;  // row offset + pair + word
+                        actA[pp][nb] = *reinterpret_cast<const uint2*>(act + base);
+                        actB[pp][nb] = *reinterpret_cast<const uint2*>(act + base + 32);
+                    }
+                __syncwarp();
+                mbar_arrive_if(&b.empty_w[s], lane == 0);
+                mbar_arrive_if(&b.empty_a[s], lane == 0);
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+                    for (int tau = 0; tau < 2; ++tau) rf_mma_pair_i8<NB>(x[pp][tau], actA[pp], actB[pp], iacc[tau]);
+                continue;
+            }
             uint32_t w[2][2][2][2];  // [pair][block A/B][tau][j]
 #pragma unroll
             for (int pp = 0; pp < 2; ++pp)
@@ -1463,19 +1541,27 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                 for (int jj = 0; jj < 2; ++jj) {
                     const int m = 8 * nb + 2 * q + jj;
                     if (m < TM) {
-                        red[(r * TM + m) * kTileN + colb + 16 * tau] = acc[tau][nb][jj];
-                        red[(r * TM + m) * kTileN + colb + 16 * tau + 8] = acc[tau][nb][2 + jj];
+                        uint32_t* rw = reinterpret_cast<uint32_t*>(red);
+                        rw[(r * TM + m) * kTileN + colb + 16 * tau] =
+                            MODE == kModeW4A8 ? iacc[tau][nb][jj] : __float_as_uint(acc[tau][nb][jj]);
+                        rw[(r * TM + m) * kTileN + colb + 16 * tau + 8] =
+                            MODE == kModeW4A8 ? iacc[tau][nb][2 + jj] : __float_as_uint(acc[tau][nb][2 + jj]);
                     }
                 }
         named_barrier_sync(1, kRfWarps * 32);
-        float v[TM];
+        uint32_t v[TM];
         if (warp < 4) {
             const int col = warp * 32 + lane;
+            const uint32_t* rw = reinterpret_cast<const uint32_t*>(red);
 #pragma unroll
             for (int m = 0; m < TM; ++m) {
-                v[m] = red[m * kTileN + col];
+                v[m] = rw[m * kTileN + col];
 #pragma unroll
-                for (int rr = 1; rr < 4; ++rr) v[m] += red[(rr * TM + m) * kTileN + col];
+                for (int rr = 1; rr < 4; ++rr) {
+                    const uint32_t x = rw[(rr * TM + m) * kTileN + col];
+                    v[m] = (MODE == kModeW4A8) ? static_cast<uint32_t>(static_cast<int32_t>(v[m]) + static_cast<int32_t>(x))
+                                               : __float_as_uint(__uint_as_float(v[m]) + __uint_as_float(x));
+                }
             }
         }
         named_barrier_sync(1, kRfWarps * 32);  // the sums are read: the next segment may write them
@@ -1544,7 +1630,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
                      : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
                                               : kCodeBytes;
-    pl->rf = mode != kModeW4A8 && M <= kRfMaxM;
+    pl->rf = M <= kRfMaxM;
     if (pl->rf) {
         const int tm = M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : (M <= 8 ? 8 : (M <= 16 ? 16 : 32))));
         pl->tile_m = tm;
@@ -1552,7 +1638,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
         pl->small = false;
         pl->threads = kThreadsRf;
         pl->issuers = 0;
-        pl->act_slot = tm * 256;  // TM rows x 128 fp16, unswizzled
+        pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;  // TM rows x 128 int8 or fp16, unswizzled
         const int budget = smem_optin - 2048 - 1024 - rf_red_bytes(tm);
         int s = budget / (pl->act_slot + pl->blob_bytes);
         if (s > kMaxSlots) s = kMaxSlots;
@@ -1623,6 +1709,10 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 8>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 1>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 2>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 4>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 8>, max_dynamic_smem);
     if constexpr (kRfMaxM > 8) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16>, max_dynamic_smem);
@@ -1660,7 +1750,7 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
 
 template <int MODE>
 static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
-    if constexpr (MODE != kModeW4A8) {
+    {
         if (plan.rf) {
             if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1>, maps, args, plan, st);
             if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2>, maps, args, plan, st);

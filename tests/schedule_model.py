@@ -88,6 +88,9 @@ def segments(beg, end, kbs):
         it = lo - 1
 
 
+FIRST_CHUNK = 1  # the CTA's first chunk is one k-block (the kernels' chunk_len)
+
+
 def chunks(beg, end, kbs, chunk, slots):
     pos = it = ch = 0
     for seg in segments(beg, end, kbs):
@@ -95,6 +98,8 @@ def chunks(beg, end, kbs, chunk, slots):
         kb = kb_lo
         while kb <= kb_hi:
             c = min(chunk, kb_hi - kb + 1, slots - pos)
+            if ch == 0:
+                c = min(c, FIRST_CHUNK)
             yield seg, pos, c, it, ch
             ch += 1
             it += c

@@ -1,8 +1,8 @@
 """CPU tests of the launch planner through wq_plan_for (host arithmetic, no GPU): for a B200's
 148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
 cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
-work. W4A16 calls of at most 8 rows get the register-operand plan: one tile of 1, 2, 4 or 8
-rows, 576 threads, and the residue sums in shared memory after the ring."""
+work. Calls of at most 8 rows (W4A16 and W4A8) get the register-operand plan: one tile of 1, 2,
+4 or 8 rows, 576 threads, and the residue sums in shared memory after the ring."""
 import itertools
 
 import pytest
@@ -11,7 +11,7 @@ SMS, SMEM = 148, 232448
 
 
 def _rf(kind, M):
-    return kind == 0 and M <= 8
+    return M <= 8
 
 
 def _red(p):  # bytes of the register-operand kernel's residue sums

@@ -95,3 +95,69 @@ def test_rf_identity_rows_reproduce_weights(K, g):
     W = np.concatenate([wq.wq_gemm_w4a16(to_dev(eye[k:k + 4]), Wp, N, g).cpu().numpy() for k in range(0, K, 4)])
     exp = ((d["q"].astype(np.float32) - 8) * d["s"][np.arange(K) // g].astype(np.float32)).astype(np.float16)
     assert np.array_equal(W.view(np.uint16), exp.view(np.uint16))
+
+
+# ---------------------------------------------------------------- W4A8 on the register-operand kernel
+def _w4a8(d, with_acc=True):
+    wq = _wq()
+    M, N = d["M"], d["N"]
+    Wp = wq.wq_prepack_w4a8(to_dev(d["Q"]))
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda") if with_acc else None
+    Y = wq.wq_gemm_w4a8(to_dev(d["A"]), to_dev(d["sa"]), Wp, to_dev(d["sw"]), N, acc_out=acc)
+    torch.cuda.synchronize()
+    assert wq.wq_get_device_status() == wq.WQ_OK
+    return Y, acc
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("K,N", [(128, 8), (4096, 264), (4096, 4096), (11008, 392)])
+def test_rf_w4a8_exact_acc(M, K, N):
+    wq = _wq()
+    assert wq.wq_plan(1, M, N, K, K)["threads"] == 576
+    d = synth.w4a8_inputs(K, N, M, seed=K + N + M)
+    Y, acc = _w4a8(d)
+    acc_ref, y_ref = oracle.w4a8(d["A"], d["sa"], d["Q"], d["sw"])
+    got = acc.cpu().numpy().astype(np.int64)
+    assert np.array_equal(got, acc_ref), f"{int((got != acc_ref).sum())} accumulators differ"
+    compare(half_bits_to_f64(Y), y_ref, oracle.w4a8_absdot(d["A"], d["sa"], d["Q"], d["sw"]), f"rf w4a8 {K}x{N} M={M}")
+
+
+def test_rf_w4a8_extremes():
+    # a = -128 (the int8 minimum) against codes 0 and 15 over K = 16384, and a = 127: the largest sums
+    K, N, M = 16384, 256, 2
+    d = synth.w4a8_inputs(K, N, M, seed=1)
+    q = np.zeros((K, N), np.uint8)
+    q[:, N // 2:] = 15
+    d["Q"] = synth.pack_q(q)
+    d["A"] = np.stack([np.full(K, -128, np.int8), np.full(K, 127, np.int8)])
+    _, acc = _w4a8(d)
+    got = acc.cpu().numpy()
+    assert np.all(got[0, : N // 2] == 8 * 128 * K) and np.all(got[0, N // 2:] == -7 * 128 * K)
+    assert np.all(got[1, : N // 2] == -8 * 127 * K) and np.all(got[1, N // 2:] == 7 * 127 * K)
+
+
+@pytest.mark.parametrize("K,N", [(4096, 11008), (11008, 4096)])
+@pytest.mark.parametrize("M", [1, 8])
+def test_rf_w4a8_full_sizes_sampled(K, N, M):
+    d = synth.w4a8_inputs(K, N, M, seed=N + M)
+    Y, acc = _w4a8(d)
+    cols = sample_cols(N, 96, seed=M)
+    acc_ref = oracle.w4a8_acc(d["A"], d["Q"][:, cols])
+    assert np.array_equal(acc.cpu().numpy()[:, cols].astype(np.int64), acc_ref)
+
+
+@pytest.mark.parametrize("M,bits", [(1, 8), (4, 8), (8, 4)])
+def test_rf_w4a8_on_fp16_activations(M, bits):
+    # the one-call quantise-then-multiply path on the register-operand kernel: accumulators
+    # bit-exact against the oracle's quantiser and exact integer sums
+    wq = _wq()
+    K, N = 4096, 1032
+    rng = np.random.default_rng(M + bits)
+    A = rng.standard_normal((M, K)).astype(np.float16)
+    d = synth.w4a8_inputs(K, N, M, seed=M)
+    Wp = wq.wq_prepack_w4a8(to_dev(d["Q"]))
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    wq.wq_gemm_w4a8_fp16act(to_dev(A), Wp, to_dev(d["sw"]), N, acc_out=acc, act_bits=bits)
+    torch.cuda.synchronize()
+    q, sa = oracle.quantize_act(A, bits=bits)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.w4a8_acc(q, d["Q"]))
