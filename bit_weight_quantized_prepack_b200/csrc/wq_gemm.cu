@@ -1193,62 +1193,14 @@ __device__ __forceinline__ void mma_m16n8k32_s8_s32(uint32_t (&d)[4], const uint
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Raw 32-bit sum: int32 for W4A8, fp32 otherwise.
-template <int MODE>
-__device__ __forceinline__ uint32_t add_raw(uint32_t a, uint32_t b) {
-    return (MODE == kModeW4A8) ? static_cast<uint32_t>(static_cast<int32_t>(a) + static_cast<int32_t>(b))
-                               : __float_as_uint(__uint_as_float(a) + __uint_as_float(b));
-}
-
-// Contributors' partials of a register-operand tile that this CTA finishes (owner, not whole):
-// thread (quarter, lane) of warps 0..3 waits for the contributing CTAs' flags (one per lane)
-// and sums their partials of column 32 quarter + lane, rows 0 .. TM - 1, in descending CTA
-// order into pre. Warps 0..3 call it as soon as their own k-blocks of the segment are done, so
-// that the loads overlap the other residues' last k-blocks.
-template <int MODE, int TM>
-__device__ void rf_gather(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&pre)[TM], bool& ok,
-                          int quarter, int lane) {
-    const int row = quarter * 32 + lane;
-    const int live = p.M < TM ? p.M : TM;
-    const int me = static_cast<int>(blockIdx.x);
-    const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
-    const int c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
-    const int ncontrib = me - c_last;
-    for (int j0 = 0; j0 < ncontrib; j0 += 32) {
-        bool good = true;
-        if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
-        ok = __all_sync(0xffffffffu, good) && ok;
-    }
-    __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
-    if (!ok) return;
-    constexpr int kBatch = TM <= 2 ? 4 : 2;
-    for (int j = 0; j < ncontrib; j += kBatch) {
-        uint32_t w[kBatch][TM];
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const uint32_t* part =
-                reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
-#pragma unroll
-            for (int m = 0; m < TM; ++m) w[b][m] = (j + b < ncontrib && m < live) ? __ldcg(part + m * kTileN + row) : 0u;
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b)
-            if (j + b < ncontrib) {
-#pragma unroll
-                for (int m = 0; m < TM; ++m) pre[m] = add_raw<MODE>(pre[m], w[b][m]);
-            }
-    }
-}
-
 // Epilogue of a register-operand tile: thread (quarter, lane) of warps 0..3 holds in v the
-// sums of output column n = tile*128 + 32 quarter + lane over this CTA's k-blocks, rows
-// 0 .. TM - 1 (only rows below M are live), and in pre the contributors' sums (owner, not
-// whole; rf_gather). The stream-K protocol is that of the small tiles: a contributor writes
-// its partial and releases its flag; the owner adds the contributors' partials (fixed order)
-// and stores the tile, then clears their flags.
+// complete sums of output column n = tile*128 + 32 quarter + lane for rows 0 .. TM - 1 (only
+// rows below M are live). The stream-K protocol is that of the small tiles: a contributor
+// writes its partial and releases its flag; the owner waits for its contributors' flags and
+// adds their partials in descending CTA order.
 template <int MODE, int TM>
-__device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM],
-                            const uint32_t (&pre)[TM], bool ok, int quarter, int lane) {
+__device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& seg, uint32_t (&v)[TM], bool ok,
+                            int quarter, int lane) {
     const int row = quarter * 32 + lane;
     const int n = seg.tile * kTileN + row;  // one m-tile: tile index = n-tile index
     const int live = p.M < TM ? p.M : TM;
@@ -1266,9 +1218,39 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
         if (leader && ok && !*ctl.abort_flag && me != p.skip_publish) st_release_gpu(&p.ws_flags[me], 1);
         return;
     }
+    int c_last = me;  // contributors are CTAs c_last .. me - 1
     if (!seg.whole) {
+        const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
+        c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        const int ncontrib = me - c_last;
+        for (int j0 = 0; j0 < ncontrib; j0 += 32) {
+            bool good = true;
+            if (ok && j0 + lane < ncontrib) good = wait_flag(&p.ws_flags[me - 1 - j0 - lane], ctl);
+            ok = __all_sync(0xffffffffu, good) && ok;
+        }
+        __syncwarp();  // the polling lanes' acquires order the whole warp's loads below
+        if (ok) {
+            constexpr int kBatch = TM <= 2 ? 4 : 2;
+            for (int j = 0; j < ncontrib; j += kBatch) {
+                uint32_t w[kBatch][TM];
 #pragma unroll
-        for (int m = 0; m < TM; ++m) v[m] = add_raw<MODE>(v[m], pre[m]);
+                for (int b = 0; b < kBatch; ++b) {
+                    const uint32_t* part =
+                        reinterpret_cast<const uint32_t*>(p.ws_partial) + static_cast<size_t>(me - 1 - j - b) * TM * kTileN;
+#pragma unroll
+                    for (int m = 0; m < TM; ++m) w[b][m] = (j + b < ncontrib && m < live) ? __ldcg(part + m * kTileN + row) : 0u;
+                }
+#pragma unroll
+                for (int b = 0; b < kBatch; ++b)
+                    if (j + b < ncontrib) {
+#pragma unroll
+                        for (int m = 0; m < TM; ++m)
+                            v[m] = (MODE == kModeW4A8)
+                                       ? static_cast<uint32_t>(static_cast<int32_t>(v[m]) + static_cast<int32_t>(w[b][m]))
+                                       : __float_as_uint(__uint_as_float(v[m]) + __uint_as_float(w[b][m]));
+                    }
+            }
+        }
     }
     if (ok && n < p.N) {
         const float s_col = (MODE == kModeChannel) ? __half2float(__ushort_as_half(p.s_chan[n])) : 1.0f;
@@ -1290,11 +1272,8 @@ __device__ void epilogue_rf(const GemmArgs& p, const Ctl& ctl, const SegCursor& 
     }
     if (!seg.whole) {
         named_barrier_sync(2, 4 * 32);  // every epilogue warp has read the partials
-        if (leader && !*ctl.abort_flag) {
-            const long long tbase = static_cast<long long>(seg.tile) * p.k_blocks;
-            const int c_last = static_cast<int>(((tbase + 1) * p.grid + p.units - 1) / p.units) - 1;
+        if (leader && !*ctl.abort_flag)
             for (int cc = me - 1; cc >= c_last; --cc) p.ws_flags[cc] = 0;
-        }
     }
 }
 
@@ -1553,12 +1532,6 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                     }
             }
         }
-        // warps 0..3 fetch the contributors' partials of a tile this CTA finishes while the other
-        // residues may still be on their last k-blocks
-        uint32_t pre[TM];
-#pragma unroll
-        for (int m = 0; m < TM; ++m) pre[m] = 0u;
-        if (warp < 4 && seg.owner && !seg.whole) rf_gather<MODE, TM>(p, ctl, seg, pre, ok, warp, lane);
         // the residues' sums of each column, added in the order r = 0..3 by warps 0..3
 #pragma unroll
         for (int tau = 0; tau < 2; ++tau)
@@ -1584,13 +1557,17 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             for (int m = 0; m < TM; ++m) {
                 v[m] = rw[m * kTileN + col];
 #pragma unroll
-                for (int rr = 1; rr < 4; ++rr) v[m] = add_raw<MODE>(v[m], rw[(rr * TM + m) * kTileN + col]);
+                for (int rr = 1; rr < 4; ++rr) {
+                    const uint32_t x = rw[(rr * TM + m) * kTileN + col];
+                    v[m] = (MODE == kModeW4A8) ? static_cast<uint32_t>(static_cast<int32_t>(v[m]) + static_cast<int32_t>(x))
+                                               : __float_as_uint(__uint_as_float(v[m]) + __uint_as_float(x));
+                }
             }
         }
         named_barrier_sync(1, kRfWarps * 32);  // the sums are read: the next segment may write them
         if (warp < 4) {
             ok = ok && !*ctl.abort_flag;
-            epilogue_rf<MODE, TM>(p, ctl, seg, v, pre, ok, warp, lane);
+            epilogue_rf<MODE, TM>(p, ctl, seg, v, ok, warp, lane);
         }
     }
 }

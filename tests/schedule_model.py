@@ -811,10 +811,9 @@ RED_SECOND_BARRIER = True  # the residue sums: one buffer, a second barrier once
 def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
     """The register-operand kernel: 16 consumer warps in 4 residues (walk index mod 4) x 4 column
     groups; the 4 warps of a k-block's residue read it (empty_w and empty_a count 4 arrivals).
-    At a segment's end warps 0..3 of an owner that is not whole first wait for the contributors'
-    flags (and load their partials), every warp writes its sums into the one buffer, all meet at
-    a 16-warp barrier, warps 0..3 read the four residues' sums, all meet again
-    (RED_SECOND_BARRIER) and warps 0..3 run the stream-K epilogue (a 4-warp barrier). Besides barrier operations the
+    At a segment's end every warp writes its sums into the one buffer, all meet at a 16-warp
+    barrier, warps 0..3 read the four residues' sums, all meet again (RED_SECOND_BARRIER) and
+    warps 0..3 run the stream-K epilogue (a 4-warp barrier). Besides barrier operations the
     roles report ("red_write", segment) and ("red_read", segment): a write while the previous
     segment's sums have not been read by all four epilogue warps is a race."""
     beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
@@ -827,10 +826,6 @@ def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
         seg_no = 0
         for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
             if pos is None:
-                tile, kb_lo, kb_hi, owner, whole = seg
-                if w < 4 and owner and not whole:  # the contributors' partials, before the residue barrier
-                    for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
-                        yield ("flag_wait", cc)
                 yield ("red_write", seg_no)
                 yield ("nbar", "red", 16)
                 if w < 4:
@@ -838,11 +833,14 @@ def _roles_rf(cta, units, grid, kbs, chunk, slots, B):
                 if RED_SECOND_BARRIER:
                     yield ("nbar", "red", 16)
                 if w < 4:
+                    tile, kb_lo, kb_hi, owner, whole = seg
                     if not owner:
                         yield ("nbar", "epi", 4)
                         if w == 0:
                             yield ("flag_set", cta)
                     elif not whole:
+                        for cc in range(cta - 1, first_contributor(tile * kbs, units, grid) - 1, -1):
+                            yield ("flag_wait", cc)
                         yield ("nbar", "epi", 4)
                 seg_no += 1
                 continue
