@@ -50,9 +50,13 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 # DRAM traffic per launch of the dominant kernel (dram__bytes_read.sum + dram__bytes_write.sum
-# from one ncu capture of a few of its launches in this workload), valid for the kernel sources
-# whose hash is recorded with it and reported as null once they change.
-TRAFFIC = {"kernel_sha": None, "bytes_per_launch": None, "algo_bytes_per_launch": None}
+# from ncu captures of single launches on one layer of the set, scaled to this workload's launches
+# by their algorithmic bytes), valid for the kernel sources whose hash is recorded with it and
+# reported as null once they change.
+TRAFFIC = {"kernel_sha": "ca0ab7d8f02ace0f", "bytes_per_launch": 26140537, "algo_bytes_per_launch": 26210784,
+           "how": "dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant kernel on the "
+                  "4096x22016 layer at M = 1 and M = 8 (1.0005 and 0.9942 of their algorithmic bytes), the mean "
+                  "ratio times this workload's average algorithmic bytes per launch of that kernel"}
 
 
 def kernel_sha() -> str:
@@ -530,7 +534,16 @@ def run_ours(args, rank, world, local_rank):
     # take the largest share of the step's device time. They are captured in their own graph, in
     # the step's order and weight copies, and timed like the step (events on the launching stream
     # around whole replays).
-    dom_ms = [M for M in M_SWEEP if wq.wq_plan(0, M, LAYERS[0][1], LAYERS[0][0], G)["threads"] == 576]
+    def family(M):
+        pl = wq.wq_plan(0, M, LAYERS[0][1], LAYERS[0][0], G)
+        if pl["threads"] == 576:
+            return "wq_gemm_rf<fp16 groups> (register-operand tiles)"
+        return f"wq_gemm_small<fp16 groups, {pl['tile_m']}-row tiles>" if pl["tile_m"] <= 32 else "wq_gemm_large<fp16 groups>"
+
+    dom_ms = sorted({M for M in M_SWEEP if wq.wq_plan(0, M, LAYERS[0][1], LAYERS[0][0], G)["threads"] == 576})
+    if not dom_ms:  # a single-layer case (--case) whose M runs another kernel: that kernel is the one timed
+        dom_ms = sorted(set(M_SWEEP))
+    dom_kernel = family(dom_ms[0])
     dom_calls = [(mi, M, L) for mi, M in enumerate(M_SWEEP) if M in dom_ms for L in layers]
     gd = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -576,10 +589,10 @@ def run_ours(args, rank, world, local_rank):
                                   "bytes / measured copy bandwidth, flops / measured bf16 peak), over the step's "
                                   "device time (M = 64 and 128 are past the ridge, so a pure bandwidth fraction "
                                   "of the whole step would understate them)"},
-        "roofline": {"bound": "hbm", "kernel": f"wq_gemm_rf<fp16 groups> (register-operand tiles: the step's "
-                                                f"M = {', '.join(map(str, dom_ms))} calls)",
+        "roofline": {"bound": "hbm", "kernel": f"{dom_kernel}: the step's M = {', '.join(map(str, dom_ms))} calls",
                      "achieved": round(achieved, 1), "peak": hbm_gbs, "unit": "GB/s",
                      "frac": round(achieved / hbm_gbs, 3), "traffic": traffic,
+                     "traffic_how": TRAFFIC["how"] if traffic is not None else None,
                      "traffic_algo_bytes": round(b_dom),
                      "launch_us": round(t_dom * 1e6, 2),
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth), of measured",
