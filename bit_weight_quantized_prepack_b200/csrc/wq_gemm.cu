@@ -1311,51 +1311,48 @@ __device__ __forceinline__ uint32_t pair_f16(uint32_t x, uint32_t x8, uint32_t k
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// The four MMAs (pairs s = 0..3) of one row tile and one 64-row pair: A fragment of MMA s =
-// pair s of the words (block A, column j = 0), (A, 1), (B, 0), (B, 1); B fragment = pair s of the
-// activation words of blocks A and B.
-template <int S, bool kScaled, int NB>
-__device__ __forceinline__ void rf_mma_pair(const uint32_t (&x)[4], const uint32_t (&x8)[4], const uint32_t (&klo)[4],
-                                            const uint32_t (&khi)[4], const __half2 (&sc)[4], const uint4 (&actA)[NB],
-                                            const uint4 (&actB)[NB], float (&d)[NB][4]) {
-    const uint32_t afrag[4] = {pair_f16<S, kScaled>(x[0], x8[0], klo[0], khi[0], sc[0]),
-                               pair_f16<S, kScaled>(x[1], x8[1], klo[1], khi[1], sc[1]),
-                               pair_f16<S, kScaled>(x[2], x8[2], klo[2], khi[2], sc[2]),
-                               pair_f16<S, kScaled>(x[3], x8[3], klo[3], khi[3], sc[3])};
+// The two MMAs (t = 0, 1) of one row tile (columns c, c + 8 of lane (g, q): word x0 of column c,
+// x1 of column c + 8, rows 8q .. 8q + 7 of a 32-row block) and one block. MMA t takes rows
+// 8q + 4t .. 8q + 4t + 3 of each lane: its A fragment is pairs 2t and 2t + 1 of the two words
+// (fragment k 2q, 2q + 1 and 2q + 8, 2q + 9), its B fragment pairs 2t and 2t + 1 of the lane's
+// activation word of the same rows, two adjacent registers of one 16-byte load. The MMA's k order
+// is a permutation of the block's rows, the same for both operands.
+template <bool kScaled, int NB>
+__device__ __forceinline__ void rf_mma_block(uint32_t x0, uint32_t x1, uint32_t klo0, uint32_t khi0, uint32_t klo1,
+                                             uint32_t khi1, __half2 sc0, __half2 sc1, const uint4 (&act)[NB],
+                                             float (&d)[NB][4]) {
+    const uint32_t x80 = x0 >> 8, x81 = x1 >> 8;
+    {
+        const uint32_t afrag[4] = {pair_f16<0, kScaled>(x0, x80, klo0, khi0, sc0), pair_f16<0, kScaled>(x1, x81, klo1, khi1, sc1),
+                                   pair_f16<1, kScaled>(x0, x80, klo0, khi0, sc0), pair_f16<1, kScaled>(x1, x81, klo1, khi1, sc1)};
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        const uint32_t bA = S == 0 ? actA[nb].x : (S == 1 ? actA[nb].y : (S == 2 ? actA[nb].z : actA[nb].w));
-        const uint32_t bB = S == 0 ? actB[nb].x : (S == 1 ? actB[nb].y : (S == 2 ? actB[nb].z : actB[nb].w));
-        mma_m16n8k16_f16_f32(d[nb], afrag, bA, bB);
+        for (int nb = 0; nb < NB; ++nb) mma_m16n8k16_f16_f32(d[nb], afrag, act[nb].x, act[nb].y);
+    }
+    {
+        const uint32_t afrag[4] = {pair_f16<2, kScaled>(x0, x80, klo0, khi0, sc0), pair_f16<2, kScaled>(x1, x81, klo1, khi1, sc1),
+                                   pair_f16<3, kScaled>(x0, x80, klo0, khi0, sc0), pair_f16<3, kScaled>(x1, x81, klo1, khi1, sc1)};
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_m16n8k16_f16_f32(d[nb], afrag, act[nb].z, act[nb].w);
     }
 }
 
-// W4A8: the two MMAs (k = 32 each) of one row tile and one 64-row pair. Word q of a column in a
-// block holds rows 8q .. 8q + 7; dequant_word_i8 gives them as int8 16 (q - 8) in two registers
-// (rows 8q + 4s .. + 3, s = 0, 1), and MMA s takes register s of the block A words as its k 0..15
-// quarter-rows and of the block B words as k 16..31, with the matching activation registers.
+// W4A8: the MMA (k = 32) of one row tile and one 32-row block. dequant_word_i8 gives a word's
+// rows 8q .. 8q + 3 and 8q + 4 .. 8q + 7 as int8 16 (q - 8) in two registers: fragment k 4q .. 4q + 3
+// and 4q + 16 .. 4q + 19; the activation word (8 int8 of the same rows) is the B fragment.
 template <int NB>
-__device__ __forceinline__ void rf_mma_pair_i8(const uint32_t (&x)[4], const uint2 (&actA)[NB], const uint2 (&actB)[NB],
-                                               uint32_t (&d)[NB][4]) {
-    uint32_t lo[4], hi[4];
+__device__ __forceinline__ void rf_mma_block_i8(uint32_t x0, uint32_t x1, const uint2 (&act)[NB], uint32_t (&d)[NB][4]) {
+    uint32_t o0[2], o1[2];
+    dequant_word_i8(x0, o0);
+    dequant_word_i8(x1, o1);
+    const uint32_t afrag[4] = {o0[0], o1[0], o0[1], o1[1]};
 #pragma unroll
-    for (int f = 0; f < 4; ++f) {
-        uint32_t o[2];
-        dequant_word_i8(x[f], o);
-        lo[f] = o[0];
-        hi[f] = o[1];
-    }
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        mma_m16n8k32_s8_s32(d[nb], lo, actA[nb].x, actB[nb].x);
-        mma_m16n8k32_s8_s32(d[nb], hi, actA[nb].y, actB[nb].y);
-    }
+    for (int nb = 0; nb < NB; ++nb) mma_m16n8k32_s8_s32(d[nb], afrag, act[nb].x, act[nb].y);
 }
 
 // Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
 // k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
 // of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
-// 32 cg + 16 tau + g and + 8, tau = 0, 1) and two 64-row pairs (blocks A = 2p, B = 2p + 1).
+// 32 cg + 16 tau + g and + 8, tau = 0, 1) in each of the four 32-row blocks.
 // red: 4 x TM x 128 floats of shared memory (residue, row, column).
 template <int MODE, int TM, int SCALE>
 __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
@@ -1406,44 +1403,31 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
             const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
             const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
+            uint32_t w[4][2][2];  // [block hv][tau][j]: word q of column colb + 16 tau + 8 j
+#pragma unroll
+            for (int hv = 0; hv < 4; ++hv)
+#pragma unroll
+                for (int tau = 0; tau < 2; ++tau)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) w[hv][tau][j] = words[(hv * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
             if constexpr (MODE == kModeW4A8) {
                 // int8 activation rows of 128 bytes: row arow, block hv, word q at arow*128 + 32 hv + 8q
-                uint32_t x[2][2][4];  // [pair][tau][fragment register]: (A, j0), (A, j1), (B, j0), (B, j1)
 #pragma unroll
-                for (int pp = 0; pp < 2; ++pp)
+                for (int hv = 0; hv < 4; ++hv) {
+                    uint2 a8[NB];
 #pragma unroll
-                    for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-                        for (int f = 0; f < 4; ++f)
-                            x[pp][tau][f] = words[((2 * pp + (f >> 1)) * kTileN + colb + 16 * tau + 8 * (f & 1)) * 4 + q];
-                uint2 actA[2][NB], actB[2][NB];
-#pragma unroll
-                for (int pp = 0; pp < 2; ++pp)
-#pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        const int base = (aoff[nb] - 16 * q) + 64 * pp + 8 * q;  // row offset + pair + word
-                        actA[pp][nb] = *reinterpret_cast<const uint2*>(act + base);
-                        actB[pp][nb] = *reinterpret_cast<const uint2*>(act + base + 32);
+                    for (int nb = 0; nb < NB; ++nb)
+                        a8[nb] = *reinterpret_cast<const uint2*>(act + (aoff[nb] - 16 * q) + 32 * hv + 8 * q);
+                    if (hv == 3) {  // the last reads of this ring slot are issued: release it
+                        __syncwarp();
+                        mbar_arrive_if(&b.empty_w[s], lane == 0);
+                        mbar_arrive_if(&b.empty_a[s], lane == 0);
                     }
-                __syncwarp();
-                mbar_arrive_if(&b.empty_w[s], lane == 0);
-                mbar_arrive_if(&b.empty_a[s], lane == 0);
 #pragma unroll
-                for (int pp = 0; pp < 2; ++pp)
-#pragma unroll
-                    for (int tau = 0; tau < 2; ++tau) rf_mma_pair_i8<NB>(x[pp][tau], actA[pp], actB[pp], iacc[tau]);
+                    for (int tau = 0; tau < 2; ++tau) rf_mma_block_i8<NB>(w[hv][tau][0], w[hv][tau][1], a8, iacc[tau]);
+                }
                 continue;
             }
-            uint32_t w[2][2][2][2];  // [pair][block A/B][tau][j]
-#pragma unroll
-            for (int pp = 0; pp < 2; ++pp)
-#pragma unroll
-                for (int bb = 0; bb < 2; ++bb)
-#pragma unroll
-                    for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-                        for (int j = 0; j < 2; ++j)
-                            w[pp][bb][tau][j] = words[((2 * pp + bb) * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
             float scb[2][2] = {{1.0f, 1.0f}, {1.0f, 1.0f}};  // kRfScaleBlock: [tau][j]
             if (SCALE == kRfScaleBlock) {
 #pragma unroll
@@ -1457,57 +1441,48 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) part[tau][nb][0] = part[tau][nb][1] = part[tau][nb][2] = part[tau][nb][3] = 0.0f;
 #pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {  // 64-row pair pp: blocks 2pp (k 0..7 of each MMA) and 2pp + 1 (k 8..15)
-                __half2 sc[2][4];    // [tau][fragment register]
-                uint32_t klo[2][4], khi[2][4];
+            for (int hv = 0; hv < 4; ++hv) {  // 32-row block hv
+                __half2 sc[2][2];    // [tau][j]
+                uint32_t klo[2][2], khi[2][2];
 #pragma unroll
                 for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                    for (int f = 0; f < 4; ++f) {
-                        sc[tau][f] = __half2half2(__ushort_as_half(0x3C00));
-                        klo[tau][f] = zp_lo(8);
-                        khi[tau][f] = zp_hi(8);
+                    for (int j = 0; j < 2; ++j) {
+                        sc[tau][j] = __half2half2(__ushort_as_half(0x3C00));
+                        klo[tau][j] = zp_lo(8);
+                        khi[tau][j] = zp_hi(8);
                     }
                 if (kPerBlock) {
+                    const int u = (32 * hv) / p.group_rows;
 #pragma unroll
-                    for (int bb = 0; bb < 2; ++bb) {
-                        const int u = (32 * (2 * pp + bb)) / p.group_rows;
+                    for (int tau = 0; tau < 2; ++tau)
 #pragma unroll
-                        for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-                            for (int j = 0; j < 2; ++j) {
-                                const int col = colb + 16 * tau + 8 * j;
-                                if (SCALE == kRfScaleWeight || SCALE == kRfScalePair)
-                                    sc[tau][2 * bb + j] = __half2half2(__ushort_as_half(scs[u * kTileN + col]));
-                                if (MODE == kModeGroupZP) {
-                                    const uint32_t zz = blob[p.zp_offset + u * kTileN + col];
-                                    klo[tau][2 * bb + j] = zp_lo(zz);
-                                    khi[tau][2 * bb + j] = zp_hi(zz);
-                                }
+                        for (int j = 0; j < 2; ++j) {
+                            const int col = colb + 16 * tau + 8 * j;
+                            if (SCALE == kRfScaleWeight || SCALE == kRfScalePair)
+                                sc[tau][j] = __half2half2(__ushort_as_half(scs[u * kTileN + col]));
+                            if (MODE == kModeGroupZP) {
+                                const uint32_t zz = blob[p.zp_offset + u * kTileN + col];
+                                klo[tau][j] = zp_lo(zz);
+                                khi[tau][j] = zp_hi(zz);
                             }
-                    }
+                        }
                 }
-                uint4 actA[NB], actB[NB];
+                uint4 a16[NB];  // activation row 8 nb + g, rows 8q .. 8q + 7 of block hv
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    actA[nb] = *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb]);
-                    actB[nb] = *reinterpret_cast<const uint4*>(act + pp * TM * 128 + aoff[nb] + 64);
-                }
-                if (pp == 1) {  // the last reads of this ring slot are issued: release it
+                for (int nb = 0; nb < NB; ++nb)
+                    a16[nb] = *reinterpret_cast<const uint4*>(act + (hv >> 1) * TM * 128 + aoff[nb] + (hv & 1) * 64);
+                if (hv == 3) {  // the last reads of this ring slot are issued: release it
                     __syncwarp();
                     mbar_arrive_if(&b.empty_w[s], lane == 0);
                     mbar_arrive_if(&b.empty_a[s], lane == 0);
                 }
 #pragma unroll
                 for (int tau = 0; tau < 2; ++tau) {
-                    const uint32_t x[4] = {w[pp][0][tau][0], w[pp][0][tau][1], w[pp][1][tau][0], w[pp][1][tau][1]};
-                    const uint32_t x8[4] = {x[0] >> 8, x[1] >> 8, x[2] >> 8, x[3] >> 8};
                     float (&dst)[NB][4] = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau] : acc[tau];
-                    rf_mma_pair<0, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
-                    rf_mma_pair<1, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
-                    rf_mma_pair<2, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
-                    rf_mma_pair<3, kScaled, NB>(x, x8, klo[tau], khi[tau], sc[tau], actA, actB, dst);
-                    if (SCALE == kRfScalePair) {  // both blocks of the pair share the group
+                    rf_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], klo[tau][0], khi[tau][0], klo[tau][1],
+                                              khi[tau][1], sc[tau][0], sc[tau][1], a16, dst);
+                    if (SCALE == kRfScalePair && (hv & 1)) {  // the 64-row pair (blocks hv - 1, hv) shares a group
                         const float s0 = __low2float(sc[tau][0]), s1 = __low2float(sc[tau][1]);
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb) {
