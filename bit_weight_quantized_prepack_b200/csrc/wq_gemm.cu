@@ -1663,14 +1663,10 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
     cudaError_t e = allow_smem(wq_gemm_large<kModeGroup>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeChannel>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeW4A8>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroup, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroup, 32>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeChannel, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeChannel, 32>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeW4A8, 32>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_large<kModeGroupZP>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 16>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_small<kModeGroupZP, 32>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1>, max_dynamic_smem);
     if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2>, max_dynamic_smem);
@@ -1692,11 +1688,13 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 16>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 16>, max_dynamic_smem);
     }
     if constexpr (kRfMaxM > 16) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 32>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 32>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 32>, max_dynamic_smem);
+        if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 32>, max_dynamic_smem);
     }
     return e;
 }
@@ -1740,7 +1738,8 @@ static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const 
         }
     }
     if (!plan.small) return launch_kernel(wq_gemm_large<MODE>, maps, args, plan, st);
-    if (plan.tile_m == 16) return launch_kernel(wq_gemm_small<MODE, 16>, maps, args, plan, st);
+    // M <= 16 runs the register-operand kernel, so a small tile here is always 32 rows (M = 17..32)
+    if (plan.tile_m != 32) return cudaErrorInvalidConfiguration;
     return launch_kernel(wq_gemm_small<MODE, 32>, maps, args, plan, st);
 }
 

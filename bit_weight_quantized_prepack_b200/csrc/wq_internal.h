@@ -48,7 +48,7 @@ struct Plan {
     long long units;
     int grid, issuers, slots, chunk, act_slot, blob_bytes, smem_bytes, threads;
     bool small;
-    bool rf;    // M <= kRfMaxM (not W4A8): the register-operand kernel, unswizzled activation slots
+    bool rf;    // M <= kRfMaxM: the register-operand kernel, unswizzled activation slots
 };
 
 int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan);

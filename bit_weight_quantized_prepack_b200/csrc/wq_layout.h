@@ -51,7 +51,7 @@ constexpr int kSmallTileMax = 32;             // tiles of at most this many rows
 constexpr int kTmemAOffsetS = 256;            // small tiles: 2 partials per residue in [0, 256), 4 A slots above
 constexpr int kMaxTileM = 256;                // activation rows per tile = tcgen05 N extent
 // register-operand tiles (M <= kRfMaxM): warp-level MMAs on weights dequantised in registers
-constexpr int kRfMaxM = 8;                  // activation rows of one m16n8k16 MMA
+constexpr int kRfMaxM = 16;                 // activation rows of two m16n8k16 MMAs
 constexpr int kRfWarps = 16;                // 8 column groups of 16 x 2 row halves of 64
 constexpr int kWeightWarpR = kRfWarps;      // warp 16
 constexpr int kActWarpR = kRfWarps + 1;     // warp 17

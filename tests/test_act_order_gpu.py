@@ -49,7 +49,7 @@ def test_permute_act_bitwise(M, K):
     assert np.array_equal(out.cpu().numpy().view(np.uint16), A[:, perm].view(np.uint16))
 
 
-# 16-row and 32-row small tiles, large tiles, ragged N, group sizes below, at and above 128
+# register-operand tiles, 32-row small tiles, large tiles, ragged N, group sizes below, at and above 128
 CASES = [(1024, 264, 128, 1, False), (1024, 264, 128, 1, True), (512, 392, 64, 5, True), (384, 136, 32, 16, False),
          (1024, 1024, 128, 33, True), (2048, 256, 256, 17, False), (1024, 640, 32, 300, True),
          (4096, 4096, 128, 8, True)]

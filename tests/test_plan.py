@@ -1,8 +1,8 @@
 """CPU tests of the launch planner through wq_plan_for (host arithmetic, no GPU): for a B200's
 148 SMs and 227 KB of opt-in shared memory, every supported shape gets a plan whose tiles
 cover M, whose ring and barriers fit shared memory, and whose stream-K split gives every CTA
-work. Calls of at most 8 rows (W4A16 and W4A8) get the register-operand plan: one tile of 1, 2,
-4 or 8 rows, 576 threads, and the residue sums in shared memory after the ring."""
+work. Calls of at most 16 rows (W4A16 and W4A8) get the register-operand plan: one tile of 1, 2,
+4, 8 or 16 rows, 576 threads, and the residue sums in shared memory after the ring."""
 import itertools
 
 import pytest
@@ -11,7 +11,7 @@ SMS, SMEM = 148, 232448
 
 
 def _rf(kind, M):
-    return M <= 8
+    return M <= 16
 
 
 def _red(p):  # bytes of the register-operand kernel's residue sums
@@ -38,7 +38,7 @@ def test_plan_invariants(wq, K, N, kind, g):
         p = wq.wq_plan_for(kind, M, N, K, g, SMS, SMEM)
         tm = p["tile_m"]
         if _rf(kind, M):
-            assert tm == {1: 1, 2: 2, 3: 4, 4: 4, 5: 8, 6: 8, 7: 8, 8: 8}[M], (M, p)
+            assert tm == (1 if M == 1 else 2 if M == 2 else 4 if M <= 4 else 8 if M <= 8 else 16), (M, p)
         else:
             assert tm % 16 == 0 and 16 <= tm <= 256, (M, p)
         assert p["m_tiles"] == -(-M // tm), (M, p)                     # the tiles cover M ...

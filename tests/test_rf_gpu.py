@@ -1,7 +1,7 @@
-"""GPU parity of the register-operand kernel (W4A16 calls of at most 8 rows: weights
+"""GPU parity of the register-operand kernel (calls of at most 16 rows: weights
 dequantised in registers feed warp-level m16n8k16 MMAs, no tensor memory) against the fp64
 oracle: every scale mode (groups of 32, 64, 128 and 256 rows, one scale per column, zero
-points), every tile height (1, 2, 4, 8 rows, rows past M zero), ragged N, stream-K splits from
+points), every tile height (1, 2, 4, 8, 16 rows, rows past M zero), ragged N, stream-K splits from
 whole tiles to 32 CTAs per tile, the full layer sizes, bitwise determinism, and identity
 activations reproducing (q - 8) * s."""
 import numpy as np
@@ -26,7 +26,7 @@ def _wq():
 SHAPES = [(128, 8), (4096, 264), (4096, 4096), (11008, 392)]
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16])
 @pytest.mark.parametrize("K,N", SHAPES)
 @pytest.mark.parametrize("g", [32, 64, 128, 256, "K"])
 def test_rf_vs_oracle(M, K, N, g):
@@ -44,7 +44,7 @@ def test_rf_vs_oracle(M, K, N, g):
     check_w4a16_full(d, Y, f"rf K={K} N={N} g={g} M={M}")
 
 
-@pytest.mark.parametrize("M", [1, 2, 4, 7])
+@pytest.mark.parametrize("M", [1, 2, 4, 7, 13])
 @pytest.mark.parametrize("K,N,g", [(4096, 264, 64), (4096, 4096, 128), (11008, 392, 32), (2048, 136, 256)])
 def test_rf_zero_points_vs_oracle(M, K, N, g):
     wq = _wq()
@@ -60,7 +60,7 @@ def test_rf_zero_points_vs_oracle(M, K, N, g):
 
 @pytest.mark.parametrize("K,N,g", [(4096, 12288, 128), (4096, 22016, 128), (11008, 4096, 128), (8192, 57344, 128),
                                    (8192, 57344, 8192), (28672, 8192, 128)])
-@pytest.mark.parametrize("M", [1, 2, 8])
+@pytest.mark.parametrize("M", [1, 2, 8, 16])
 def test_rf_full_layer_sizes_sampled(K, N, g, M):
     # the bench's launch configuration at full size; the oracle computes sampled columns
     wq = _wq()
@@ -109,7 +109,7 @@ def _w4a8(d, with_acc=True):
     return Y, acc
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 11, 16])
 @pytest.mark.parametrize("K,N", [(128, 8), (4096, 264), (4096, 4096), (11008, 392)])
 def test_rf_w4a8_exact_acc(M, K, N):
     wq = _wq()
@@ -125,7 +125,7 @@ def test_rf_w4a8_exact_acc(M, K, N):
 def test_rf_w4a8_extremes():
     # a = -128 (the int8 minimum) against codes 0 and 15 over K = 16384, and a = 127: the largest sums
     K, N, M = 16384, 256, 2
-    d = synth.w4a8_inputs(K, N, M, seed=1)
+    d = synth.w4a8_inputs(K, N, M, seed=1)  # two rows: the register-operand kernel's 2-row tile
     q = np.zeros((K, N), np.uint8)
     q[:, N // 2:] = 15
     d["Q"] = synth.pack_q(q)
@@ -137,7 +137,7 @@ def test_rf_w4a8_extremes():
 
 
 @pytest.mark.parametrize("K,N", [(4096, 11008), (11008, 4096)])
-@pytest.mark.parametrize("M", [1, 8])
+@pytest.mark.parametrize("M", [1, 8, 16])
 def test_rf_w4a8_full_sizes_sampled(K, N, M):
     d = synth.w4a8_inputs(K, N, M, seed=N + M)
     Y, acc = _w4a8(d)
@@ -146,7 +146,7 @@ def test_rf_w4a8_full_sizes_sampled(K, N, M):
     assert np.array_equal(acc.cpu().numpy()[:, cols].astype(np.int64), acc_ref)
 
 
-@pytest.mark.parametrize("M,bits", [(1, 8), (4, 8), (8, 4)])
+@pytest.mark.parametrize("M,bits", [(1, 8), (4, 8), (8, 4), (16, 8)])
 def test_rf_w4a8_on_fp16_activations(M, bits):
     # the one-call quantise-then-multiply path on the register-operand kernel: accumulators
     # bit-exact against the oracle's quantiser and exact integer sums

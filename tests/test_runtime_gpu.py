@@ -16,7 +16,7 @@ def _wq():
     return wq
 
 
-@pytest.mark.parametrize("M", [1, 16])  # the register-operand and the small-tile kernel
+@pytest.mark.parametrize("M", [1, 24])  # the register-operand and the small-tile kernel
 def test_expired_wait_reports_timeout_and_context_survives(M):
     # CTA 0 holds the first k-blocks of tile 0 and skips publishing its partial, so the CTA
     # that finishes tile 0 waits on a flag nothing sets. With a 20 ms limit the wait expires,
@@ -83,7 +83,7 @@ def test_capture_without_reserved_workspace_is_refused():
 
 
 def test_two_streams_concurrently():
-    # Three layers of different shapes and kernels (register-operand, 16-row and large tiles) on
+    # Three layers of different shapes and kernels (register-operand, 32-row and large tiles) on
     # three streams, 50 rounds: the kernels may run side by side, so a stream-K owner may find
     # the CTAs it waits for not yet resident; its waits are bounded and no round may time out.
     # Every round must report WQ_OK and match the oracle.
@@ -92,7 +92,7 @@ def test_two_streams_concurrently():
     wq = _wq()
     K, g = 4096, 128
     cases = [synth.w4a16_inputs(K, 4096, g, 3, seed=6), synth.w4a16_inputs(K, 2048, g, 40, seed=7),
-             synth.w4a16_inputs(K, 3072, g, 16, seed=8)]
+             synth.w4a16_inputs(K, 3072, g, 24, seed=8)]
     refs = [(oracle.w4a16(d["A"], d["Q"], d["s"], g), oracle.w4a16_absdot(d["A"], d["Q"], d["s"], g)) for d in cases]
     dev = [(to_dev(d["A"]), wq.wq_prepack(to_dev(d["Q"]), to_dev(d["s"]), g)) for d in cases]
     torch.cuda.synchronize()

@@ -36,7 +36,7 @@ def test_prepack_zp_matches_oracle_bytes_and_roundtrips(K, N, g):
     assert np.array_equal(s.cpu().numpy().view(np.uint16), d["s"].view(np.uint16))
 
 
-# 16-row and 32-row small tiles, large tiles, several m-tiles; group sizes below, at and above 128
+# register-operand tiles, 32-row small tiles, large tiles, several m-tiles; group sizes below, at and above 128
 CASES = [(1024, 264, 128, 1), (512, 392, 64, 5), (384, 136, 32, 16), (1024, 1024, 128, 17), (2048, 256, 256, 33),
          (1024, 512, 32, 100), (512, 640, 128, 300), (4096, 4096, 128, 16)]
 

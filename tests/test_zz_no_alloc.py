@@ -10,7 +10,7 @@ The test calls the entry point through the C ABI (ctypes, raw device pointers) t
 row with different activations, so that the second call runs on the scratch the first one
 left behind. Each output is compared with the fp64 oracle within the parity tolerance of the
 other tests and, since both entry points run the same deterministic kernels, bit for bit with
-the regular entry point on the same inputs. The cases cover 16-row tiles, 32-row tiles, a
+the regular entry point on the same inputs. The cases cover register-operand tiles, 32-row tiles, a
 large tile and per-column scales (g = K). The test also checks that the second call leaves
 the device's free memory unchanged, that a call needing more scratch than the array holds is
 refused without a launch, and that an expired device-side wait of the fixed-scratch call is
@@ -34,10 +34,10 @@ def _c_abi(wq, A, Wp, Y, N, g):
                                         ctypes.c_void_p(Y.data_ptr()), M, N, K, g, stream)
 
 
-# (K, N, g, M): 16-row tile; 32-row tile; a 48-row large tile; per-column scales on the
-# register-operand kernel (M = 3), 16- and 32-row tiles; the register-operand kernel at M = 1
-CASES = [(4096, 1032, 128, 5), (1024, 1032, 128, 28), (2048, 2056, 64, 40), (2048, 520, 2048, 3),
-         (2048, 520, 2048, 12), (1024, 264, 1024, 24), (4096, 1032, 64, 1)]
+# (K, N, g, M): register-operand tiles (M = 5, 12); 32-row tiles; a 48-row large tile; per-column
+# scales on the register-operand kernel (M = 3) and 32-row tiles; g = 64 at M = 1
+CASES = [(4096, 1032, 128, 5), (4096, 1032, 128, 12), (1024, 1032, 128, 28), (2048, 2056, 64, 40),
+         (2048, 520, 2048, 3), (1024, 264, 1024, 24), (4096, 1032, 64, 1)]
 
 
 @pytest.mark.parametrize("K,N,g,M", CASES)
