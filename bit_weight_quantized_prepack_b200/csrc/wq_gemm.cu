@@ -5,14 +5,21 @@
 // sizes 1..128 through asynchronous memory access, task scheduling, pipelining and bespoke
 // quantisation support; hide the dequantisation ("Enabling Fast 2-bit LLM on GPUs: Memory
 // Alignment and Asynchronous Dequantization", Abstract: dequantisation otherwise takes more
-// than half of the run time). How this kernel does it on B200:
+// than half of the run time). How these kernels do it on B200 (three families, picked by the
+// number of activation rows M; all share the prepacked layout, the stream-K walk, the producers
+// and the shared-memory ring):
 //
-//   * The weights are the MMA's M operand (128 output columns per tile) and the activations
-//     its N operand (tile_m rows, 16..256), so even M = 1 uses a legal tcgen05 shape.
+//   * M <= 16: the register-operand kernel (wq_gemm_rf, at the end of this file): every warp
+//     dequantises its share of each k-block into registers and multiplies it with the
+//     warp-level MMA (mma.sync), no tensor memory and no hand-off between warps. At so few rows
+//     the tensor-memory chain below costs more per k-block than the arithmetic.
+//   * M = 17..32 (small tiles) and M > 32 (large tiles): the tcgen05 kernels described next.
+//     The weights are the MMA's M operand (128 output columns per tile) and the activations
+//     its N operand (tile_m rows, 32..256).
 //   * One persistent CTA per SM walks a contiguous range of (tile, k-block) units (stream-K).
 //     A tile split between CTAs is finished by the CTA holding its last k-block, which adds
 //     the other CTAs' partial sums in a fixed order: results are deterministic.
-//   * Warp roles per CTA (704 threads in both designs):
+//   * Warp roles per CTA of the tcgen05 kernels (704 threads in both designs):
 //       warp 20     weight producer: one bulk copy moves up to 4 consecutive blobs (codes +
 //                   scales of 4 k-blocks, contiguous in HBM by construction of the prepack);
 //       warp 21     activation producer: one 3-D tensor copy moves the same k-blocks of the
@@ -25,7 +32,7 @@
 //                   k-blocks per lane quarter are in flight at once;
 //       warps 16..19 MMA issuers (one elected thread each).
 //     Two ways to split the work, by tile height:
-//       small tiles (tile_m <= 32, the memory-bound decode regime): 4 residues; issuer r owns
+//       small tiles (tile_m = 32): 4 residues; issuer r owns
 //                   every fourth k-block and writes each k-block's product into a fresh
 //                   partial in tensor memory (two buffers per residue, used in turn), which
 //                   the dequant warps of residue r add in fp32 registers (applying the group
@@ -40,7 +47,8 @@
 //     ~75-85 cycles whatever the shape, and one issuing bulk copies gets one copy per ~270 ns;
 //     several issuing warps and copies of 16-33 KB take both costs off the critical path.
 //     At small M each residue's k-block is a chain (dequant into the A slot, MMA issue,
-//     completion, next dequant) whose length, with four chains per SM, sets the ceiling.
+//     completion, next dequant) whose length, with four chains per SM, sets the ceiling: the
+//     reason the register-operand kernel takes M <= 16.
 //   * Every wait is bounded by a global-timer limit; an expired wait records WQ_ERR_TIMEOUT
 //     and the CTA winds down (drains its copies and MMAs, frees tensor memory) instead of
 //     hanging.

@@ -242,13 +242,14 @@ WQ_API int wq_get_device_status(void* stream);
  * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8. */
 typedef struct {
     int grid;         /* persistent CTAs launched (<= number of SMs) */
-    int tile_m;       /* activation rows per tile (the MMA's N extent) */
+    int tile_m;       /* activation rows per tile: 1, 2, 4, 8 or 16 for the register-operand kernel
+                         (M <= 16), else the tcgen05 MMA's N extent (32..256) */
     int m_tiles;      /* tiles along M */
     int n_tiles;      /* tiles of 128 columns along N */
     int k_blocks;     /* blocks of 128 rows along K */
     int stages;       /* shared-memory pipeline depth */
     int smem_bytes;   /* dynamic shared memory per CTA */
-    int threads;      /* threads per CTA */
+    int threads;      /* threads per CTA: 576 for the register-operand kernel, 704 otherwise */
     long long units;  /* (tile, k-block) work units split across the CTAs */
 } wq_plan_t;
 WQ_API int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan);
