@@ -107,3 +107,41 @@ def test_two_streams_concurrently():
             assert wq.wq_get_device_status(st) == wq.WQ_OK, f"round {it}"
         for (y_ref, ad), Y in zip(refs, outs):
             compare(half_bits_to_f64(Y), y_ref, ad, f"two streams, round {it}")
+
+
+@pytest.mark.parametrize("M", [3, 24])  # register-operand and 32-row tiles
+def test_graph_capture_of_the_one_call_entry_points(M):
+    # the act-order layer (gather + layer) and W4A8 on fp16 activations (quantise + layer) keep
+    # their intermediate buffers in the stream's workspace: with the workspace of their kind
+    # reserved, a captured call replays the eager call bit for bit
+    import oracle
+    wq = _wq()
+    K, N, g = 2048, 1032, 128
+    d = synth.w4a16_inputs(K, N, g, M, seed=M)
+    rng = np.random.default_rng(M)
+    gidx = rng.permutation(np.arange(K) // g)
+    perm = to_dev(oracle.act_order_perm(gidx, g).astype(np.int32))
+    A = to_dev(d["A"])
+    Wa = wq.wq_prepack_act_order(to_dev(d["Q"]), to_dev(d["s"]), perm, g)
+    W8 = wq.wq_prepack_w4a8(to_dev(d["Q"]))
+    sw = to_dev(np.full(N, 0.01, np.float32))
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    Y1 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    Y2 = torch.empty((M, N), dtype=torch.float16, device="cuda")
+    with torch.cuda.stream(s):
+        wq.wq_workspace_reserve(max(wq.wq_workspace_bytes(4, M, N, K), wq.wq_workspace_bytes(2, M, N, K)), stream=s)
+        E1 = wq.wq_gemm_w4a16_act_order(A, perm, Wa, N, g, stream=s)
+        E2 = wq.wq_gemm_w4a8_fp16act(A, W8, sw, N, stream=s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            wq.wq_gemm_w4a16_act_order(A, perm, Wa, N, g, Y=Y1, stream=s)
+            wq.wq_gemm_w4a8_fp16act(A, W8, sw, N, Y=Y2, stream=s)
+    for _ in range(3):
+        Y1.zero_()
+        Y2.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(Y1.view(torch.int16), E1.view(torch.int16))
+        assert torch.equal(Y2.view(torch.int16), E2.view(torch.int16))
+    assert wq.wq_get_device_status(s) == wq.WQ_OK
