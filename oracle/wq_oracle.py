@@ -19,6 +19,19 @@ What it computes, and where that comes from:
   (Atom, dynamic activation quantisation) and a per-channel weight scale:
   ``Y[m,n] = sa[m] * sw[n] * sum_k A[m,k] * (q[k,n] - 8)``.
 
+Around the layer (each function's docstring gives its reading of the pages):
+
+* per-token activation quantisation (``quantize_act``; Atom, method: dynamic
+  activation quantisation), 8-bit for W4A8 and 4-bit for W4A4 numerics;
+* asymmetric groups (``dequant_zp``, ``w4a16_zp``): a 4-bit zero point per group
+  and column instead of the fixed 8;
+* act order (``dequant_gidx``, ``w4a16_gidx``, ``act_order_perm``,
+  ``reorder_rows``): groups whose rows are scattered along K by ``g_idx``.
+
+Every function here is pinned by ``tests/oracle_pins.py`` (hand-worked golden
+values, exact rational brute force, closed forms and invariants); none is
+"parity unpinned".
+
 The pages do not fix the packing of the codes; the reading used here is the
 plainest one for "8 codes per int32" of a K x N weight: ``Q`` is ``[K/8, N]``
 and code ``k = 8*i + j`` of column ``n`` sits in bits ``4j .. 4j+3`` of
