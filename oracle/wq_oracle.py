@@ -26,7 +26,9 @@ Around the layer (each function's docstring gives its reading of the pages):
 * asymmetric groups (``dequant_zp``, ``w4a16_zp``): a 4-bit zero point per group
   and column instead of the fixed 8;
 * act order (``dequant_gidx``, ``w4a16_gidx``, ``act_order_perm``,
-  ``reorder_rows``): groups whose rows are scattered along K by ``g_idx``.
+  ``reorder_rows``): groups whose rows are scattered along K by ``g_idx``;
+* 2:4 sparse weights (``is_sparse24``, ``prepack_w4a16_sparse24``): the layer is
+  ``w4a16`` of the pruned weight; only the prepacked format differs.
 
 Every function here is pinned by ``tests/oracle_pins.py`` (hand-worked golden
 values, exact rational brute force, closed forms and invariants); none is
@@ -60,6 +62,8 @@ __all__ = [
     "prepack_w4a16_act_order",
     "dequant_zp", "w4a16_zp", "w4a16_zp_absdot", "prepack_w4a16_zp", "prepacked_bytes_w4a16_zp", "unprepack_w4a16_zp",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
+    "SPARSE_GROUP_ORDER", "is_sparse24", "prepacked_bytes_w4a16_sparse24", "prepack_w4a16_sparse24",
+    "unprepack_w4a16_sparse24",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
 ]
 
@@ -525,3 +529,139 @@ def unprepack_w4a16_zp(Wp: np.ndarray, K: int, N: int, g: int):
     z = np.zeros((K // g, nt * TILE_N), dtype=np.uint8)
     z[krow // g] = zz
     return q, s, z[:, :N]
+
+
+# --------------------------------------------------------------------------
+# 2:4 sparse weights (the library's prepacked format for them)
+# --------------------------------------------------------------------------
+# A 2:4 sparse weight has, in every run of 4 consecutive rows of a column (a pruning group,
+# rows 4i .. 4i+3), at most 2 codes other than 8 (weight 0). The layer is the W4A16 layer of
+# that weight (``w4a16``): sparsity changes the storage, not the result. ("MARLIN:
+# Mixed-Precision Auto-Regressive Parallel Inference on Large Language Models", Abstract: the
+# kernel extends to NVIDIA 2:4 sparsity; the format below is this library's own.)
+#
+# Blob (nt, kt) of a 128-column tile and a 128-row k-block: 4096 bytes of code words, 2048 bytes
+# of metadata words, then the group scales as in the dense blob (``slots`` rows of 128 fp16).
+# Within the k-block, 32-row block b (rows 32b .. 32b+31) holds pruning groups pg = 0..7; the
+# sparse MMA's group j of the block is pruning group SPARSE_GROUP_ORDER[j]. Column c of the tile
+# is in row tile rt = c // 16, with g = c % 8 and half = (c % 16) // 8.
+#   code word (b*8 + rt)*32 + 4g + q holds the kept codes of MMA groups q and q+4 of the two
+#     columns 16rt + g (half 0) and 16rt + g + 8 (half 1): nibble
+#     (half + 2*(j >= 4)) + 4*kept_index, kept_index 0 for the lower kept row, 1 for the higher;
+#   metadata word ((b*8 + rt)*8 + g)*2 + h holds, at nibble (j % 4) + 4*half for MMA group
+#     j = 4h .. 4h+3, the kept rows' positions in the group: bits 0-1 the lower, bits 2-3 the
+#     higher.
+# The kept rows of a group are its rows whose code is not 8, made up to two with the lowest
+# remaining rows (code 8).
+SPARSE_GROUP_ORDER = (0, 4, 1, 5, 2, 6, 3, 7)  # MMA group j -> pruning group of the 32-row block
+
+
+def is_sparse24(q: np.ndarray) -> bool:
+    """True when every run of 4 rows (4i .. 4i+3) of every column has at most 2 codes other than 8."""
+    q = np.asarray(q)
+    K, N = q.shape
+    return K % 4 == 0 and bool(((q.reshape(K // 4, 4, N) != ZERO_POINT).sum(axis=1) <= 2).all())
+
+
+def _kept_rows(col_group: np.ndarray):
+    """The two kept positions (ascending) of a pruning group's 4 codes."""
+    keep = [p for p in range(4) if col_group[p] != ZERO_POINT]
+    for p in range(4):
+        if len(keep) == 2:
+            break
+        if p not in keep:
+            keep.append(p)
+    return sorted(keep)
+
+
+def prepacked_bytes_w4a16_sparse24(K: int, N: int, g: int) -> int:
+    _check_kn(K, N)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    slots = _group_slots(K, g)
+    blob = 4096 + 2048 + 2 * TILE_N * slots
+    tail = 0 if slots else ((2 * nt * TILE_N + 15) // 16) * 16
+    return nt * kt * blob + tail
+
+
+def prepack_w4a16_sparse24(Q: np.ndarray, s: np.ndarray, g: int) -> np.ndarray:
+    """The 2:4 sparse prepacked buffer as bytes, following the layout above (loops over the
+    documented indices, one code at a time)."""
+    q = unpack_codes(Q)
+    K, N = q.shape
+    if not is_sparse24(q):
+        raise ValueError("not 2:4 sparse")
+    slots = _group_slots(K, g)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    qp = np.full((K, nt * TILE_N), ZERO_POINT, dtype=np.uint8)
+    qp[:, :N] = q
+    blob_bytes = 4096 + 2048 + 2 * TILE_N * slots
+    out = np.zeros(prepacked_bytes_w4a16_sparse24(K, N, g), dtype=np.uint8)
+    sp = np.zeros((np.asarray(s).shape[0], nt * TILE_N), dtype=np.float16)
+    sp[:, :N] = np.asarray(s, dtype=np.float16)
+    for n_t in range(nt):
+        for k_t in range(kt):
+            codes = np.zeros(1024, dtype=np.uint32)
+            meta = np.zeros(512, dtype=np.uint32)
+            for c in range(TILE_N):
+                col = n_t * TILE_N + c
+                rt, gg, half = c // 16, c % 8, (c % 16) // 8
+                for b in range(4):
+                    for j in range(8):
+                        pg = SPARSE_GROUP_ORDER[j]
+                        r0 = k_t * TILE_K + 32 * b + 4 * pg
+                        keep = _kept_rows(qp[r0:r0 + 4, col])
+                        qq = j % 4
+                        w = (b * 8 + rt) * 32 + 4 * gg + qq
+                        for ki, pos in enumerate(keep):
+                            nib = half + 2 * (j >= 4) + 4 * ki
+                            codes[w] |= np.uint32(int(qp[r0 + pos, col]) << (4 * nib))
+                        mw = ((b * 8 + rt) * 8 + gg) * 2 + j // 4
+                        meta[mw] |= np.uint32((keep[0] | (keep[1] << 2)) << (4 * ((j % 4) + 4 * half)))
+            start = (n_t * kt + k_t) * blob_bytes
+            out[start:start + 4096] = codes.view(np.uint8)
+            out[start + 4096:start + 6144] = meta.view(np.uint8)
+            for u in range(slots):
+                grp = (k_t * TILE_K + u * g) // g
+                out[start + 6144 + 256 * u:start + 6144 + 256 * (u + 1)] = \
+                    sp[grp, n_t * TILE_N:(n_t + 1) * TILE_N].view(np.uint8)
+    if not slots:
+        tail = nt * kt * blob_bytes
+        out[tail:tail + 2 * nt * TILE_N] = sp[0].view(np.uint8)
+    return out
+
+
+def unprepack_w4a16_sparse24(Wp: np.ndarray, K: int, N: int, g: int):
+    """Inverse of ``prepack_w4a16_sparse24``: ``(q[K,N] uint8, s[K/g, N] fp16)``, pruned rows as 8."""
+    slots = _group_slots(K, g)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    Wp = np.asarray(Wp, dtype=np.uint8)
+    blob_bytes = 4096 + 2048 + 2 * TILE_N * slots
+    q = np.full((K, nt * TILE_N), ZERO_POINT, dtype=np.uint8)
+    s = np.zeros((K // g, nt * TILE_N), dtype=np.float16)
+    for n_t in range(nt):
+        for k_t in range(kt):
+            start = (n_t * kt + k_t) * blob_bytes
+            codes = Wp[start:start + 4096].copy().view(np.uint32)
+            meta = Wp[start + 4096:start + 6144].copy().view(np.uint32)
+            for c in range(TILE_N):
+                col = n_t * TILE_N + c
+                rt, gg, half = c // 16, c % 8, (c % 16) // 8
+                for b in range(4):
+                    for j in range(8):
+                        pg = SPARSE_GROUP_ORDER[j]
+                        r0 = k_t * TILE_K + 32 * b + 4 * pg
+                        mw = ((b * 8 + rt) * 8 + gg) * 2 + j // 4
+                        m = (int(meta[mw]) >> (4 * ((j % 4) + 4 * half))) & 0xF
+                        keep = (m & 3, m >> 2)
+                        w = (b * 8 + rt) * 32 + 4 * gg + j % 4
+                        for ki, pos in enumerate(keep):
+                            nib = half + 2 * (j >= 4) + 4 * ki
+                            q[r0 + pos, col] = (int(codes[w]) >> (4 * nib)) & 0xF
+            for u in range(slots):
+                grp = (k_t * TILE_K + u * g) // g
+                s[grp, n_t * TILE_N:(n_t + 1) * TILE_N] = \
+                    Wp[start + 6144 + 256 * u:start + 6144 + 256 * (u + 1)].copy().view(np.float16)
+    if not slots:
+        tail = nt * kt * blob_bytes
+        s = Wp[tail:tail + 2 * nt * TILE_N].copy().view(np.float16)[None, :]
+    return q[:, :N], s[:, :N]

@@ -30,7 +30,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["pack_q", "w4a16_inputs", "w4a8_inputs"]
+__all__ = ["pack_q", "w4a16_inputs", "w4a8_inputs", "w4a16_sparse24_inputs"]
 
 
 def pack_q(q: np.ndarray) -> np.ndarray:
@@ -69,3 +69,19 @@ def w4a8_inputs(K: int, N: int, M: int, seed: int = 0) -> dict:
     A = rng.integers(-127, 128, size=(M, K), dtype=np.int8)
     sa = (0.01 + 0.05 * np.abs(rng.standard_normal(M))).astype(np.float32)
     return {"q": q, "Q": pack_q(q), "sw": sw, "A": A, "sa": sa, "K": K, "N": N, "M": M}
+
+
+def w4a16_sparse24_inputs(K: int, N: int, g: int, M: int, seed: int = 0) -> dict:
+    """The inputs of ``w4a16_inputs`` with the codes pruned 2:4: in every run of 4 rows
+    (4i .. 4i+3) of every column, two rows drawn uniformly keep their code and the other two
+    get code 8 (a zero weight). The pattern is drawn after the activations."""
+    d = w4a16_inputs(K, N, g, M, seed=seed)
+    rng = np.random.default_rng(seed + 1)
+    q = d["q"].reshape(K // 4, 4, N).copy()
+    keep = np.argsort(rng.random((K // 4, 4, N)), axis=1)[:, :2, :]  # two distinct rows per group
+    mask = np.zeros((K // 4, 4, N), dtype=bool)
+    np.put_along_axis(mask, keep, True, axis=1)
+    q[~mask] = 8
+    q = q.reshape(K, N)
+    d.update(q=q, Q=pack_q(q))
+    return d

@@ -30,6 +30,7 @@ import os
 from fractions import Fraction
 
 import numpy as np
+import pytest
 
 import synth
 
@@ -505,6 +506,75 @@ def pin_pack_codes(o):
     assert np.array_equal(o.pack_codes(o.unpack_codes(d["Q"])), d["Q"])
 
 
+# ---------------------------------------------------------------- 2:4 sparse prepacked layout
+def golden_sparse24():
+    out = []
+    for line in _rows("sparse24_layout.txt"):
+        parts = [p.strip() for p in line.split("|")]
+        K, N, g = (int(x) for x in parts[1].split())
+        a, b = (int(x) for x in parts[2].split())
+        offs = [int(x) for x in parts[3].split()]
+        vals = [int(x, 16) for x in parts[4].split()] if len(parts) > 4 else None
+        out.append((parts[0], K, N, g, a, b, offs, vals))
+    return out
+
+
+def pin_sparse24_layout_golden(o):
+    # one code 3 among 8s (its code byte and, where the kept rows move, its metadata byte) or one
+    # scale among zeros: exactly the bytes the hand-worked table names change, to its values
+    bases = {}
+    for what, K, N, g, a, b, offs, vals in golden_sparse24():
+        q = np.full((K, N), 8, np.uint8)
+        s = np.zeros((K // g, N), np.float16)
+        if (K, N, g) not in bases:
+            bases[K, N, g] = o.prepack_w4a16_sparse24(synth.pack_q(q), s, g)
+        base = bases[K, N, g]
+        assert np.all(base[:4096] == 0x88) and np.all(base[4096:6144] == 0x44)
+        if what == "code":
+            q[a, b] = 3
+            Wp = o.prepack_w4a16_sparse24(synth.pack_q(q), s, g)
+            diff = np.nonzero(Wp != base)[0].tolist()
+            assert diff == offs, (K, N, g, a, b, diff, offs)
+            assert [int(Wp[x]) for x in offs] == vals, (a, b, [hex(int(Wp[x])) for x in offs])
+        else:
+            s[a, b] = np.array([_SCALE_BITS], np.uint16).view(np.float16)[0]
+            Wp = o.prepack_w4a16_sparse24(synth.pack_q(q), s, g)
+            diff = np.nonzero(Wp != base)[0].tolist()
+            assert diff == sorted(x for off in offs for x in (off, off + 1)), (K, N, g, a, b, diff, offs)
+            for off in offs:
+                assert int(Wp[off]) | (int(Wp[off + 1]) << 8) == _SCALE_BITS
+
+
+def pin_sparse24_two_kept_codes(o):
+    # both kept rows of one group non-zero, at positions 2 and 3 (the worked example's column
+    # and group): code byte 3164 takes pos 2 in its low half, byte 3166 pos 3; metadata 2 | 3 << 2
+    q = np.full((384, 296), 8, np.uint8)
+    q[118, 5], q[119, 5] = 5, 3
+    s = np.zeros((3, 296), np.float16)
+    Wp = o.prepack_w4a16_sparse24(synth.pack_q(q), s, 128)
+    base = o.prepack_w4a16_sparse24(synth.pack_q(np.full((384, 296), 8, np.uint8)), s, 128)
+    assert np.nonzero(Wp != base)[0].tolist() == [3164, 3166, 5673]
+    assert [int(Wp[x]) for x in (3164, 3166, 5673)] == [0x85, 0x83, 0xE4]
+
+
+def pin_sparse24_definition(o):
+    # is_sparse24 against its definition, brute force over every 4-row pattern of one column
+    for bits in range(16):
+        q = np.full((8, 1), 8, np.uint8)
+        for p in range(4):
+            if bits >> p & 1:
+                q[4 + p, 0] = 1 + p
+        assert o.is_sparse24(q) == (bin(bits).count("1") <= 2)
+    assert not o.is_sparse24(np.full((6, 1), 8, np.uint8))  # K not a multiple of 4
+    q = np.full((128, 8), 8, np.uint8)
+    q[0:3, 2] = 1
+    with pytest.raises(ValueError):
+        o.prepack_w4a16_sparse24(synth.pack_q(q), np.zeros((1, 8), np.float16), 128)
+    d = synth.w4a16_sparse24_inputs(256, 24, 64, 1, seed=3)
+    nz = (d["q"].reshape(64, 4, 24) != 8).sum(axis=1)
+    assert o.is_sparse24(d["q"]) and nz.max() <= 2
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
@@ -512,5 +582,5 @@ ALL_PINS = [
     pin_blob_layout_golden, pin_act_quant_golden, pin_act_quant_bounds, pin_zp_golden, pin_zp_bruteforce,
     pin_zp_eight_is_symmetric, pin_act_order_golden, pin_act_order_unequal_groups_refused,
     pin_act_order_bruteforce, pin_act_order_contiguous_is_grouped, pin_act_order_reordering_identity,
-    pin_pack_codes,
+    pin_pack_codes, pin_sparse24_layout_golden, pin_sparse24_two_kept_codes, pin_sparse24_definition,
 ]

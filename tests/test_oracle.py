@@ -6,7 +6,7 @@ import oracle
 import synth
 from oracle import wq_oracle as O
 
-from oracle_pins import ALL_PINS, pin_blob_layout_golden
+from oracle_pins import ALL_PINS, pin_blob_layout_golden, pin_sparse24_layout_golden
 
 
 
@@ -311,6 +311,48 @@ def test_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeypatch):
     # ... and the hand-worked byte offsets catch it
     with pytest.raises(AssertionError):
         pin_blob_layout_golden(O)
+
+
+@pytest.mark.parametrize("K,N,g", [(128, 128, 128), (256, 200, 64), (384, 136, 32), (512, 8, 256), (256, 40, 256)])
+def test_prepack_sparse24_roundtrip(K, N, g):
+    d = synth.w4a16_sparse24_inputs(K, N, g, 1, seed=K + N + g)
+    Wp = O.prepack_w4a16_sparse24(d["Q"], d["s"], g)
+    assert Wp.nbytes == O.prepacked_bytes_w4a16_sparse24(K, N, g)
+    q, s = O.unprepack_w4a16_sparse24(Wp, K, N, g)
+    assert np.array_equal(q, d["q"])
+    assert np.array_equal(s.view(np.uint16), d["s"].view(np.uint16))
+
+
+def test_prepack_sparse24_padding_is_zero_weight():
+    d = synth.w4a16_sparse24_inputs(256, 72, 64, 1, seed=2)
+    q, s = O.unprepack_w4a16_sparse24(O.prepack_w4a16_sparse24(d["Q"], d["s"], 64), 256, 128, 64)
+    assert np.all(q[:, 72:] == 8) and np.all(s[:, 72:] == 0)
+
+
+# Sparse layout mistakes made in both directions: the round trip passes, the offsets catch them.
+def _mut_sparse_group_order_plain(mp):
+    mp.setattr(O, "SPARSE_GROUP_ORDER", tuple(range(8)))
+
+
+def _mut_sparse_fill_highest(mp):
+    def kept_rows(col_group):
+        keep = [p for p in range(4) if col_group[p] != 8]
+        for p in (3, 2, 1, 0):
+            if len(keep) == 2:
+                break
+            if p not in keep:
+                keep.append(p)
+        return sorted(keep)
+    mp.setattr(O, "_kept_rows", kept_rows)
+
+
+@pytest.mark.parametrize("mutate", [_mut_sparse_group_order_plain, _mut_sparse_fill_highest],
+                         ids=lambda f: f.__name__[5:])
+def test_sparse_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeypatch):
+    mutate(monkeypatch)
+    test_prepack_sparse24_roundtrip(256, 200, 64)
+    with pytest.raises(AssertionError):
+        pin_sparse24_layout_golden(O)
 
 
 def test_package_reexports():
