@@ -62,7 +62,7 @@ __all__ = [
     "prepack_w4a16_act_order",
     "dequant_zp", "w4a16_zp", "w4a16_zp_absdot", "prepack_w4a16_zp", "prepacked_bytes_w4a16_zp", "unprepack_w4a16_zp",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
-    "SPARSE_GROUP_ORDER", "is_sparse24", "prepacked_bytes_w4a16_sparse24", "prepack_w4a16_sparse24",
+    "is_sparse24", "prepacked_bytes_w4a16_sparse24", "prepack_w4a16_sparse24",
     "unprepack_w4a16_sparse24",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
 ]
@@ -542,18 +542,25 @@ def unprepack_w4a16_zp(Wp: np.ndarray, K: int, N: int, g: int):
 #
 # Blob (nt, kt) of a 128-column tile and a 128-row k-block: 4096 bytes of code words, 2048 bytes
 # of metadata words, then the group scales as in the dense blob (``slots`` rows of 128 fp16).
-# Within the k-block, 32-row block b (rows 32b .. 32b+31) holds pruning groups pg = 0..7; the
-# sparse MMA's group j of the block is pruning group SPARSE_GROUP_ORDER[j]. Column c of the tile
-# is in row tile rt = c // 16, with g = c % 8 and half = (c % 16) // 8.
-#   code word (b*8 + rt)*32 + 4g + q holds the kept codes of MMA groups q and q+4 of the two
-#     columns 16rt + g (half 0) and 16rt + g + 8 (half 1): nibble
-#     (half + 2*(j >= 4)) + 4*kept_index, kept_index 0 for the lower kept row, 1 for the higher;
-#   metadata word ((b*8 + rt)*8 + g)*2 + h holds, at nibble (j % 4) + 4*half for MMA group
-#     j = 4h .. 4h+3, the kept rows' positions in the group: bits 0-1 the lower, bits 2-3 the
-#     higher.
+# Within the k-block, 32-row block b (rows 32b .. 32b+31) holds pruning groups j = 0..7. Column
+# c of the tile is in row tile rt = c // 16, with g = c % 8 and half = (c % 16) // 8.
+#   code word (b*8 + rt)*32 + 4g + (j % 4) holds the kept codes of groups j and j+4 of the two
+#     columns 16rt + g (half 0) and 16rt + g + 8 (half 1) (``_sparse_code_nibble``);
+#   metadata word ((b*8 + rt)*8 + g)*2 + j // 4 holds each group's two kept positions, bits 0-1
+#     the lower, bits 2-3 the higher (``_sparse_meta_place``).
 # The kept rows of a group are its rows whose code is not 8, made up to two with the lowest
 # remaining rows (code 8).
-SPARSE_GROUP_ORDER = (0, 4, 1, 5, 2, 6, 3, 7)  # MMA group j -> pruning group of the 32-row block
+
+
+def _sparse_code_nibble(half: int, j: int, kept_index: int) -> int:
+    """Nibble of a code word that holds kept code ``kept_index`` (0 lower, 1 higher row) of
+    group j of the column in ``half``."""
+    return half + 2 * (j >= 4) + 4 * kept_index
+
+
+def _sparse_meta_place(b: int, rt: int, g: int, half: int, j: int):
+    """(word, nibble) of the metadata of group j of column 16rt + 8half + g in 32-row block b."""
+    return ((b * 8 + rt) * 8 + g) * 2 + j // 4, (j % 4) + 4 * half
 
 
 def is_sparse24(q: np.ndarray) -> bool:
@@ -607,16 +614,13 @@ def prepack_w4a16_sparse24(Q: np.ndarray, s: np.ndarray, g: int) -> np.ndarray:
                 rt, gg, half = c // 16, c % 8, (c % 16) // 8
                 for b in range(4):
                     for j in range(8):
-                        pg = SPARSE_GROUP_ORDER[j]
-                        r0 = k_t * TILE_K + 32 * b + 4 * pg
+                        r0 = k_t * TILE_K + 32 * b + 4 * j
                         keep = _kept_rows(qp[r0:r0 + 4, col])
-                        qq = j % 4
-                        w = (b * 8 + rt) * 32 + 4 * gg + qq
+                        w = (b * 8 + rt) * 32 + 4 * gg + j % 4
                         for ki, pos in enumerate(keep):
-                            nib = half + 2 * (j >= 4) + 4 * ki
-                            codes[w] |= np.uint32(int(qp[r0 + pos, col]) << (4 * nib))
-                        mw = ((b * 8 + rt) * 8 + gg) * 2 + j // 4
-                        meta[mw] |= np.uint32((keep[0] | (keep[1] << 2)) << (4 * ((j % 4) + 4 * half)))
+                            codes[w] |= np.uint32(int(qp[r0 + pos, col]) << (4 * _sparse_code_nibble(half, j, ki)))
+                        mw, mn = _sparse_meta_place(b, rt, gg, half, j)
+                        meta[mw] |= np.uint32((keep[0] | (keep[1] << 2)) << (4 * mn))
             start = (n_t * kt + k_t) * blob_bytes
             out[start:start + 4096] = codes.view(np.uint8)
             out[start + 4096:start + 6144] = meta.view(np.uint8)
@@ -648,15 +652,12 @@ def unprepack_w4a16_sparse24(Wp: np.ndarray, K: int, N: int, g: int):
                 rt, gg, half = c // 16, c % 8, (c % 16) // 8
                 for b in range(4):
                     for j in range(8):
-                        pg = SPARSE_GROUP_ORDER[j]
-                        r0 = k_t * TILE_K + 32 * b + 4 * pg
-                        mw = ((b * 8 + rt) * 8 + gg) * 2 + j // 4
-                        m = (int(meta[mw]) >> (4 * ((j % 4) + 4 * half))) & 0xF
-                        keep = (m & 3, m >> 2)
+                        r0 = k_t * TILE_K + 32 * b + 4 * j
+                        mw, mn = _sparse_meta_place(b, rt, gg, half, j)
+                        m = (int(meta[mw]) >> (4 * mn)) & 0xF
                         w = (b * 8 + rt) * 32 + 4 * gg + j % 4
-                        for ki, pos in enumerate(keep):
-                            nib = half + 2 * (j >= 4) + 4 * ki
-                            q[r0 + pos, col] = (int(codes[w]) >> (4 * nib)) & 0xF
+                        for ki, pos in enumerate((m & 3, m >> 2)):
+                            q[r0 + pos, col] = (int(codes[w]) >> (4 * _sparse_code_nibble(half, j, ki))) & 0xF
             for u in range(slots):
                 grp = (k_t * TILE_K + u * g) // g
                 s[grp, n_t * TILE_N:(n_t + 1) * TILE_N] = \

@@ -547,14 +547,15 @@ def pin_sparse24_layout_golden(o):
 
 def pin_sparse24_two_kept_codes(o):
     # both kept rows of one group non-zero, at positions 2 and 3 (the worked example's column
-    # and group): code byte 3164 takes pos 2 in its low half, byte 3166 pos 3; metadata 2 | 3 << 2
+    # and group): nibble 2 (byte 3157, low half) takes pos 2, nibble 6 (byte 3159) pos 3;
+    # metadata 2 | 3 << 2
     q = np.full((384, 296), 8, np.uint8)
     q[118, 5], q[119, 5] = 5, 3
     s = np.zeros((3, 296), np.float16)
     Wp = o.prepack_w4a16_sparse24(synth.pack_q(q), s, 128)
     base = o.prepack_w4a16_sparse24(synth.pack_q(np.full((384, 296), 8, np.uint8)), s, 128)
-    assert np.nonzero(Wp != base)[0].tolist() == [3164, 3166, 5673]
-    assert [int(Wp[x]) for x in (3164, 3166, 5673)] == [0x85, 0x83, 0xE4]
+    assert np.nonzero(Wp != base)[0].tolist() == [3157, 3159, 5676]
+    assert [int(Wp[x]) for x in (3157, 3159, 5676)] == [0x85, 0x83, 0xE4]
 
 
 def pin_sparse24_definition(o):

@@ -330,8 +330,13 @@ def test_prepack_sparse24_padding_is_zero_weight():
 
 
 # Sparse layout mistakes made in both directions: the round trip passes, the offsets catch them.
-def _mut_sparse_group_order_plain(mp):
-    mp.setattr(O, "SPARSE_GROUP_ORDER", tuple(range(8)))
+def _mut_sparse_code_nibble_bits_swapped(mp):
+    mp.setattr(O, "_sparse_code_nibble", lambda half, j, ki: 2 * half + (j >= 4) + 4 * ki)
+
+
+def _mut_sparse_meta_half_and_word_swapped(mp):
+    mp.setattr(O, "_sparse_meta_place",
+               lambda b, rt, g, half, j: (((b * 8 + rt) * 8 + g) * 2 + half, (j % 4) + 4 * (j // 4)))
 
 
 def _mut_sparse_fill_highest(mp):
@@ -346,7 +351,8 @@ def _mut_sparse_fill_highest(mp):
     mp.setattr(O, "_kept_rows", kept_rows)
 
 
-@pytest.mark.parametrize("mutate", [_mut_sparse_group_order_plain, _mut_sparse_fill_highest],
+@pytest.mark.parametrize("mutate", [_mut_sparse_code_nibble_bits_swapped, _mut_sparse_meta_half_and_word_swapped,
+                                    _mut_sparse_fill_highest],
                          ids=lambda f: f.__name__[5:])
 def test_sparse_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeypatch):
     mutate(monkeypatch)
