@@ -21,17 +21,19 @@ __all__ = [
     "wq_quantize_act", "wq_gemm_w4a8_fp16act",
     "wq_prepacked_bytes_zp", "wq_prepack_zp", "wq_unpack_zp", "wq_gemm_w4a16_zp",
     "wq_prepack_act_order", "wq_permute_act", "wq_gemm_w4a16_act_order",
+    "wq_prepacked_bytes_sparse24", "wq_prepack_sparse24", "wq_unpack_sparse24", "wq_gemm_w4a16_sparse24",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
     "WQ_ERR_UNSUPPORTED_DEVICE", "WQ_ERR_CUDA", "WQ_ERR_TIMEOUT", "WQ_ERR_NO_MEMORY", "WQ_ERR_CAPTURING",
-    "WQ_ERR_SCRATCH_LIMIT",
+    "WQ_ERR_SCRATCH_LIMIT", "WQ_ERR_NOT_SPARSE",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
 
 (WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_UNSUPPORTED_SHAPE, WQ_ERR_MISALIGNED, WQ_ERR_UNSUPPORTED_DEVICE,
- WQ_ERR_CUDA, WQ_ERR_TIMEOUT, WQ_ERR_NO_MEMORY, WQ_ERR_CAPTURING, WQ_ERR_SCRATCH_LIMIT) = range(10)
+ WQ_ERR_CUDA, WQ_ERR_TIMEOUT, WQ_ERR_NO_MEMORY, WQ_ERR_CAPTURING, WQ_ERR_SCRATCH_LIMIT,
+ WQ_ERR_NOT_SPARSE) = range(11)
 
 
 class WqError(RuntimeError):
@@ -72,6 +74,10 @@ def _load():
         "wq_permute_act": (I, [P, P, I, I, P, P]),
         "wq_gemm_w4a16_act_order": (I, [P, P, P, P, I, I, I, I, I, P]),
         "wq_gemm_w4a8_fp16act": (I, [P, P, P, P, P, P, I, I, I, I, P]),
+        "wq_prepacked_bytes_sparse24": (Z, [I, I, I]),
+        "wq_prepack_sparse24": (I, [P, P, I, I, I, P, P]),
+        "wq_unpack_sparse24": (I, [P, I, I, I, P, P, P]),
+        "wq_gemm_w4a16_sparse24": (I, [P, P, P, I, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
         "wq_get_device_status": (I, [P]),
@@ -411,6 +417,63 @@ def wq_gemm_w4a16_act_order(A: torch.Tensor, perm: torch.Tensor, Wp: torch.Tenso
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _check(lib.wq_gemm_w4a16_act_order(_ptr(A), _ptr(perm), _ptr(Wp), _ptr(Y), M, N, K, g, int(bool(zero_points)),
                                        _stream(stream)), "wq_gemm_w4a16_act_order")
+    return Y
+
+
+def wq_prepacked_bytes_sparse24(K: int, N: int, g: int) -> int:
+    return lib.wq_prepacked_bytes_sparse24(K, N, g)
+
+
+def _sparse_size(K, N, g, where):
+    if g <= 0 or K <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, where)
+    n = wq_prepacked_bytes_sparse24(K, N, g)
+    if n == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE if K % 128 == 0 else WQ_ERR_INVALID_ARG, where)
+    return n
+
+
+def wq_prepack_sparse24(Q: torch.Tensor, s: torch.Tensor, g: int, Wp: torch.Tensor | None = None, stream=None):
+    """Q int32 [K/8, N] of 2:4 sparse codes (at most 2 of every 4 rows 4i..4i+3 differ from 8),
+    s fp16 [K/g, N] -> the sparse buffer. Raises WqError(WQ_ERR_NOT_SPARSE) otherwise; the
+    call synchronises the stream."""
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    nbytes = _sparse_size(K, N, g, "wq_prepack_sparse24")
+    _tensor(s, torch.float16, "s", shape=(K // g, N))
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    _on_one_cuda_device(Q=Q, s=s, Wp=Wp)
+    if Wp is None:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack_sparse24(_ptr(Q), _ptr(s), K, N, g, _ptr(Wp), _stream(stream)), "wq_prepack_sparse24")
+    return Wp
+
+
+def wq_unpack_sparse24(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
+    """Inverse of wq_prepack_sparse24: (Q int32 [K/8, N] with pruned codes 8, s fp16 [K/g, N])."""
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_sparse_size(K, N, g, "wq_unpack_sparse24"))
+    _on_one_cuda_device(Wp=Wp)
+    Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
+    s = torch.empty((K // g, N), dtype=torch.float16, device=Wp.device)
+    _check(lib.wq_unpack_sparse24(_ptr(Wp), K, N, g, _ptr(Q), _ptr(s), _stream(stream)), "wq_unpack_sparse24")
+    return Q, s
+
+
+def wq_gemm_w4a16_sparse24(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor | None = None,
+                           stream=None):
+    """Y fp16 [M, N] = A fp16 [M, K] . dequant(Wp) for a 2:4 sparse buffer, M <= 16."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=_sparse_size(K, N, g, "wq_gemm_w4a16_sparse24"))
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    _on_one_cuda_device(A=A, Wp=Wp, Y=Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.wq_gemm_w4a16_sparse24(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)),
+           "wq_gemm_w4a16_sparse24")
     return Y
 
 

@@ -34,6 +34,7 @@ struct DeviceState {
     int num_sms = 0;
     int smem_optin = 0;
     int* status = nullptr;  // device status word
+    int* check = nullptr;   // 2:4 sparse layout pass: set when a group has more than two weights
 };
 std::map<int, DeviceState> g_devices;
 
@@ -67,6 +68,7 @@ DeviceState* device_state(int* dev_out) {
     if (d.supported) {
         if (cudaMalloc(&d.status, sizeof(int)) != cudaSuccess) return nullptr;
         if (cudaMemset(d.status, 0, sizeof(int)) != cudaSuccess) return nullptr;
+        if (cudaMalloc(&d.check, sizeof(int)) != cudaSuccess) return nullptr;
         if (configure_gemm_kernels(d.smem_optin - 2048) != cudaSuccess) return nullptr;
     }
     if (!g_encode) {
@@ -143,18 +145,20 @@ size_t workspace_bytes_for(const Plan& pl) {
     return 4096 + static_cast<size_t>(pl.grid) * pl.tile_m * kTileN * 4;
 }
 
-// kind 0: W4A16; 1: W4A8; 3: W4A16 with a zero point per group (g < K).
+// kind 0: W4A16; 1: W4A8; 3: W4A16 with a zero point per group (g < K); 5: 2:4 sparse W4A16
+// (M <= kRfMaxM).
 int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* pl) {
     int mode;
     int slots = 0;
-    if (kind == 0 || kind == 3) {
+    if (kind == 0 || kind == 3 || kind == 5) {
         slots = scale_slots(K, g);
         if (slots < 0 || (kind == 3 && slots == 0)) return WQ_ERR_INVALID_ARG;
         mode = kind == 3 ? kModeGroupZP : (slots > 0 ? kModeGroup : kModeChannel);
     } else {
         mode = kModeW4A8;
     }
-    if (make_plan(mode, M, N, K, slots, d.num_sms, d.smem_optin, pl) != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (kind == 5 && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (make_plan(mode, M, N, K, slots, d.num_sms, d.smem_optin, pl, kind == 5) != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
     return WQ_OK;
 }
 
@@ -162,7 +166,8 @@ int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* p
 // split into swizzle-wide pieces: dims {64 fp16 or 128 int8, M, K/piece}, strides {K*elem (rows),
 // piece bytes}; a box of {piece, tile_m, c*pieces_per_kblock} lands in shared memory as
 // [piece index][row][128 bytes], the K-major 128-byte-swizzled layout the MMA reads.
-// Unswizzled (swizzle false: the register-operand kernel) the box lands as [piece][row][64 fp16].
+// Unswizzled (swizzle false: the register-operand kernel on dense weights) the box lands as
+// [piece][row][64 fp16]. tile_m is the box's row count (rows past M read as zeros).
 int encode_activation_maps(ActMaps* maps, const void* A, int M, int K, int tile_m, int chunk, bool int8,
                            bool swizzle = true) {
     const int piece = int8 ? 128 : 64;                 // elements per 128-byte row
@@ -206,7 +211,7 @@ bool perm_grid_ok(int M, int K) {
     return static_cast<long long>(M) * ((K / 8 + 255) / 256) < (1LL << 31) - 1;
 }
 
-// The W4A16 (kind 0), W4A8 (kind 1) or zero-point (kind 3) layer. A_fp16 (W4A8 only, may be
+// The W4A16 (kind 0), W4A8 (kind 1), zero-point (kind 3) or 2:4 sparse W4A16 (kind 5) layer. A_fp16 (W4A8 only, may be
 // null): fp16 activations that are first quantised per token into the workspace (the codes
 // replace A, the scales go to sa_out when given, else to the workspace). perm (kinds 0 and 3,
 // may be null): act order; A's columns are first gathered in the order perm into the
@@ -218,8 +223,9 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     if (rc) return rc;
     if (M < 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if ((kind == 0 || kind == 3) && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if ((kind == 0 || kind == 3 || kind == 5) && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
     if (kind == 3 && scale_slots(K, g) == 0) return WQ_ERR_INVALID_ARG;
+    if (kind == 5 && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (kind == 1 && K > kMaxKW4A8) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (!Wp) return WQ_ERR_INVALID_ARG;
     if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
@@ -270,7 +276,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
         sa = sq;
     }
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, kind == 1, !pl.rf);
+    rc = encode_activation_maps(&maps, A, M, K, pl.act_rows, pl.chunk, kind == 1, !pl.rf || pl.sparse);
     if (rc) return rc;
 
     GemmArgs a;
@@ -278,7 +284,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.wp = static_cast<const uint8_t*>(Wp);
     a.s_chan = (pl.mode == kModeChannel)
                    ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
-                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * kCodeBytes)
+                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * pl.blob_bytes)
                    : nullptr;
     a.sa = sa;
     a.sw = sw;
@@ -298,7 +304,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.chunk = pl.chunk;
     a.act_slot = pl.act_slot;
     a.blob_bytes = pl.blob_bytes;
-    a.group_rows = ((kind == 0 || kind == 3) && g < kTileK) ? g : kTileK;
+    a.group_rows = ((kind == 0 || kind == 3 || kind == 5) && g < kTileK) ? g : kTileK;
     a.small = pl.small ? 1 : 0;
     a.scale_in_dequant = scale_in_dequant(pl, g);
     a.zp_offset = (pl.mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16(scale_slots(K, g))) : 0;
@@ -404,13 +410,16 @@ const char* wq_status_string(int status) {
         case WQ_OK: return "WQ_OK";
         case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG: null pointer, negative size or unsupported group size";
         case WQ_ERR_UNSUPPORTED_SHAPE:
-            return "WQ_ERR_UNSUPPORTED_SHAPE: K must be a multiple of 128, N a multiple of 8, M at most 2^24";
+            return "WQ_ERR_UNSUPPORTED_SHAPE: K must be a multiple of 128, N a multiple of 8, M at most 2^24 "
+                   "(2:4 sparse weights: M at most 16)";
         case WQ_ERR_MISALIGNED: return "WQ_ERR_MISALIGNED: a pointer breaks the alignment rule";
         case WQ_ERR_UNSUPPORTED_DEVICE: return "WQ_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (sm_100a)";
         case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or kernel launch failed";
         case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT: a device-side wait expired";
         case WQ_ERR_NO_MEMORY: return "WQ_ERR_NO_MEMORY: workspace allocation failed";
         case WQ_ERR_CAPTURING: return "WQ_ERR_CAPTURING: reserve the workspace before capturing the stream";
+        case WQ_ERR_NOT_SPARSE:
+            return "WQ_ERR_NOT_SPARSE: a run of 4 weight rows holds more than 2 codes other than 8";
         case WQ_ERR_SCRATCH_LIMIT:
             return "WQ_ERR_SCRATCH_LIMIT: the call needs more stream-K scratch than the fixed array of "
                    "wq_gemm_w4a16_noalloc holds (use wq_gemm_w4a16)";
@@ -629,6 +638,64 @@ int wq_gemm_w4a16_act_order(const uint16_t* A, const int32_t* perm, const void* 
                     static_cast<cudaStream_t>(stream), nullptr, nullptr, 8, perm);
 }
 
+size_t wq_prepacked_bytes_sparse24(int K, int N, int g) {
+    if (!shape_ok(K, N)) return 0;
+    const int slots = scale_slots(K, g);
+    if (slots < 0) return 0;
+    const size_t nblob = static_cast<size_t>(n_tiles(N)) * (K / kTileK);
+    if (slots == 0) return nblob * blob_bytes_sp24(0) + channel_tail_bytes(N);
+    return nblob * blob_bytes_sp24(slots);
+}
+
+int wq_prepack_sparse24(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (!s) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return WQ_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return WQ_ERR_CAPTURING;  // the check below synchronises
+    int bad = 0;
+    if (cudaMemsetAsync(d->check, 0, sizeof(int), st) != cudaSuccess ||
+        launch_prepack_sp24(Q, s, K, N, g, Wp, d->check, st) != 0 ||
+        cudaMemcpyAsync(&bad, d->check, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return bad ? WQ_ERR_NOT_SPARSE : WQ_OK;
+}
+
+int wq_unpack_sparse24(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q_out, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if (!s_out) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s_out, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_unpack_sp24(Wp, K, N, g, Q_out, s_out, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16_sparse24(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g, void* stream) {
+    return run_gemm(5, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
+}
+
 int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
                  int M, int N, int K, void* stream) {
     return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
@@ -661,13 +728,14 @@ int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uin
 }
 
 size_t wq_workspace_bytes(int kind, int M, int N, int K) {
-    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 4) return 0;
+    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 5) return 0;
+    if (kind == 5 && M > kRfMaxM) return 0;
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
     DeviceState* d = device_state(&dev);
     if (!d || !d->supported) return 0;
     Plan pl;
-    const bool w4a16 = kind == 0 || kind == 3 || kind == 4;  // these plan like the W4A16 layer
+    const bool w4a16 = kind == 0 || kind == 3 || kind == 4 || kind == 5;  // these plan like the W4A16 layer
     if (plan_for(w4a16 ? 0 : 1, M, N, K, w4a16 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
     if (kind == 2) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_quant_bytes(M, K);
     if (kind == 4) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_perm_bytes(M, K);
@@ -726,13 +794,13 @@ int fill_plan(int kind, int M, int N, int K, int g, int num_sms, int smem_optin,
     if (rc) return rc;
     if (M <= 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if (kind != 0 && kind != 1) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1 && kind != 5) return WQ_ERR_INVALID_ARG;
     if (num_sms <= 0 || smem_optin <= 0) return WQ_ERR_INVALID_ARG;
     DeviceState d;
     d.num_sms = num_sms;
     d.smem_optin = smem_optin;
     Plan pl;
-    rc = plan_for(kind, M, N, K, kind == 0 ? g : K, d, &pl);
+    rc = plan_for(kind, M, N, K, kind == 1 ? K : g, d, &pl);
     if (rc) return rc;
     plan->grid = pl.grid;
     plan->tile_m = pl.tile_m;
@@ -752,7 +820,7 @@ int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M <= 0) return WQ_ERR_INVALID_ARG;
-    if (kind != 0 && kind != 1) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1 && kind != 5) return WQ_ERR_INVALID_ARG;
     int num_sms = 0, smem_optin = 0;
     {
         std::lock_guard<std::mutex> lock(g_mu);
@@ -810,7 +878,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     if (rc) return rc;
     if (workspace_bytes_for(pl) > kNoAllocStatusOffset) return WQ_ERR_SCRATCH_LIMIT;
     ActMaps maps;
-    rc = encode_activation_maps(&maps, A, M, K, pl.tile_m, pl.chunk, false, !pl.rf);
+    rc = encode_activation_maps(&maps, A, M, K, pl.act_rows, pl.chunk, false, !pl.rf);
     if (rc) return rc;
     // the scratch keeps whatever the last call left; the publish flags must start at zero
     if (cudaMemsetAsync(d->scratch, 0, static_cast<size_t>(pl.grid) * sizeof(int), st) != cudaSuccess) {
@@ -824,7 +892,7 @@ int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y, int M,
     a.wp = static_cast<const uint8_t*>(Wp);
     a.s_chan = (pl.mode == kModeChannel)
                    ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
-                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * kCodeBytes)
+                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * pl.blob_bytes)
                    : nullptr;
     a.y = Y;
     a.ws_flags = reinterpret_cast<int*>(d->scratch);

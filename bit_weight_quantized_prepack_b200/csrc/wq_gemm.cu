@@ -1357,15 +1357,56 @@ __device__ __forceinline__ void rf_mma_block_i8(uint32_t x0, uint32_t x1, const 
     for (int nb = 0; nb < NB; ++nb) mma_m16n8k32_s8_s32(d[nb], afrag, act[nb].x, act[nb].y);
 }
 
+// 2:4 sparse weights. The sparse warp MMA (m16n8k32, groups of 4 along k, 2 kept per group)
+// takes as A operand the kept values only: lane (g, q) holds, as four fp16 pairs, the two kept
+// values of group q of rows g and g + 8, then of group q + 4 of the same rows, which is the
+// order of the nibble pairs (0, 4), (1, 5), (2, 6), (3, 7) of one sparse code word: the word
+// dequantises straight into the operand. Its metadata (lanes q = 0, 1 of each quad, selector 0)
+// gives each group's two kept positions. The B operand is the dense 32 x 8 activation block:
+// lane (g, q) register r holds activation row g, k = 8r + 2q, 8r + 2q + 1, i.e. element
+// (g, 2q) of the 8 x 8 matrix at k = 8r: one ldmatrix.x4 per 8 activation rows.
+__device__ __forceinline__ void mma_sp_m16n8k32_f16_f32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[4],
+                                                        uint32_t e) {
+    asm volatile(
+        "mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9, %10, %11}, {%0, %1, %2, %3}, %12, 0x0;\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(e));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&d)[4], uint32_t saddr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+                 : "r"(saddr)
+                 : "memory");
+}
+
+// The sparse MMA of one row tile (sparse code word x, metadata e) and one 32-row block; sc0,
+// sc1: the fp16 scales of the tile's columns g and g + 8 when kScaled.
+template <bool kScaled, int NB>
+__device__ __forceinline__ void rf_sp_mma_block(uint32_t x, uint32_t e, __half2 sc0, __half2 sc1,
+                                                const uint32_t (&bf)[NB][4], float (&d)[NB][4]) {
+    const uint32_t x8 = x >> 8, klo = zp_lo(8), khi = zp_hi(8);
+    const uint32_t a[4] = {pair_f16<0, kScaled>(x, x8, klo, khi, sc0), pair_f16<1, kScaled>(x, x8, klo, khi, sc1),
+                           pair_f16<2, kScaled>(x, x8, klo, khi, sc0), pair_f16<3, kScaled>(x, x8, klo, khi, sc1)};
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) mma_sp_m16n8k32_f16_f32(d[nb], a, bf[nb], e);
+}
+
 // Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
 // k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
 // of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
 // 32 cg + 16 tau + g and + 8, tau = 0, 1) in each of the four 32-row blocks.
 // red: 4 x TM x 128 floats of shared memory (residue, row, column).
-template <int MODE, int TM, int SCALE>
+// SP: 2:4 sparse blobs. Lane (g, q) then reads, per 32-row block and row tile, one code word
+// and one metadata word, and the activation slot holds AR = max(TM, 8) rows in the 128-byte
+// swizzled layout of the copy engine (16-byte chunk c of row m at chunk c ^ (m mod 8)), so
+// that the eight rows of each 8 x 8 matrix of an ldmatrix fall in eight different banks.
+template <int MODE, int TM, int SCALE, bool SP>
 __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
                         const Ctl& ctl, long long beg, long long end) {
     constexpr int NB = (TM + 7) / 8;  // MMAs of 8 activation rows per k-step
+    constexpr int AR = (SP && TM < kSpMinActRows) ? kSpMinActRows : TM;  // activation rows per slot piece
     constexpr bool kScaled = SCALE == kRfScaleWeight;
     constexpr bool kPerBlock = SCALE == kRfScaleWeight || SCALE == kRfScalePair || MODE == kModeGroupZP;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1379,6 +1420,10 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
         const int arow = 8 * nb + g < TM ? 8 * nb + g : TM - 1;
         aoff[nb] = arow * 128 + 16 * q;
     }
+    // SP: lane l gives the address of row l mod 8 of matrix l / 8 (k = 8 (l / 8) of the block):
+    // activation row 8 nb + l mod 8, 16-byte chunk 4 (hv mod 2) + l / 8, swizzled
+    const int lrow = lane & 7, lmat = lane >> 3;
+    const uint32_t sw_off[2] = {static_cast<uint32_t>(((0 + lmat) ^ lrow) << 4), static_cast<uint32_t>(((4 + lmat) ^ lrow) << 4)};
     ChunkBar cb;
     uint32_t iter = 0;
     int pos = 0;
@@ -1409,15 +1454,23 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             if (!ok) continue;  // an expired wait: the CTA winds down (nothing more is read or released)
             const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
             const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
-            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + kCodeBytes);
+            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + (SP ? kSpHeadBytes : kCodeBytes));
             const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
             uint32_t w[4][2][2];  // [block hv][tau][j]: word q of column colb + 16 tau + 8 j
+                                  // SP: [hv][tau][0] code word, [hv][tau][1] metadata word of row tile 2 cg + tau
 #pragma unroll
             for (int hv = 0; hv < 4; ++hv)
 #pragma unroll
-                for (int tau = 0; tau < 2; ++tau)
+                for (int tau = 0; tau < 2; ++tau) {
+                    if constexpr (SP) {
+                        const int tile16 = hv * 8 + 2 * cg + tau;
+                        w[hv][tau][0] = words[tile16 * 32 + lane];
+                        w[hv][tau][1] = words[kSpCodeBytes / 4 + tile16 * 16 + 2 * g + (q & 1)];
+                    } else {
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) w[hv][tau][j] = words[(hv * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
+                        for (int j = 0; j < 2; ++j) w[hv][tau][j] = words[(hv * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
+                    }
+                }
             if constexpr (MODE == kModeW4A8) {
                 // int8 activation rows of 128 bytes: row arow, block hv, word q at arow*128 + 32 hv + 8q
 #pragma unroll
@@ -1476,10 +1529,17 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                             }
                         }
                 }
-                uint4 a16[NB];  // activation row 8 nb + g, rows 8q .. 8q + 7 of block hv
+                uint4 a16[NB];      // activation row 8 nb + g, rows 8q .. 8q + 7 of block hv
+                uint32_t bf[NB][4];  // SP: the B operands (activation rows 8 nb .. 8 nb + 7)
+                if constexpr (SP) {
+                    const uint32_t piece = smem_addr(act) + (hv >> 1) * AR * 128 + sw_off[hv & 1];
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
-                    a16[nb] = *reinterpret_cast<const uint4*>(act + (hv >> 1) * TM * 128 + aoff[nb] + (hv & 1) * 64);
+                    for (int nb = 0; nb < NB; ++nb) ldmatrix_x4(bf[nb], piece + (8 * nb + lrow) * 128);
+                } else {
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+                        a16[nb] = *reinterpret_cast<const uint4*>(act + (hv >> 1) * TM * 128 + aoff[nb] + (hv & 1) * 64);
+                }
                 if (hv == 3) {  // the last reads of this ring slot are issued: release it
                     __syncwarp();
                     mbar_arrive_if(&b.empty_w[s], lane == 0);
@@ -1488,8 +1548,11 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
 #pragma unroll
                 for (int tau = 0; tau < 2; ++tau) {
                     float (&dst)[NB][4] = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau] : acc[tau];
-                    rf_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], klo[tau][0], khi[tau][0], klo[tau][1],
-                                              khi[tau][1], sc[tau][0], sc[tau][1], a16, dst);
+                    if constexpr (SP)
+                        rf_sp_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], sc[tau][0], sc[tau][1], bf, dst);
+                    else
+                        rf_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], klo[tau][0], khi[tau][0], klo[tau][1],
+                                                  khi[tau][1], sc[tau][0], sc[tau][1], a16, dst);
                     if (SCALE == kRfScalePair && (hv & 1)) {  // the 64-row pair (blocks hv - 1, hv) shares a group
                         const float s0 = __low2float(sc[tau][0]), s1 = __low2float(sc[tau][1]);
 #pragma unroll
@@ -1555,7 +1618,7 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
     }
 }
 
-template <int MODE, int TM>
+template <int MODE, int TM, bool SP = false>
 __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constant__ ActMaps maps, const GemmArgs p) {
     extern __shared__ uint8_t smem_dyn[];
     __shared__ Barriers bars;
@@ -1587,13 +1650,13 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
     if (warp < kRfWarps) {
         if constexpr (is_group(MODE)) {
             if (p.scale_in_dequant)
-                rf_role<MODE, TM, kRfScaleWeight>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScaleWeight, SP>(p, aring, wring, bars, red, ctl, beg, end);
             else if (p.group_rows < kTileK)
-                rf_role<MODE, TM, kRfScalePair>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScalePair, SP>(p, aring, wring, bars, red, ctl, beg, end);
             else
-                rf_role<MODE, TM, kRfScaleBlock>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScaleBlock, SP>(p, aring, wring, bars, red, ctl, beg, end);
         } else {
-            rf_role<MODE, TM, kRfScaleNone>(p, aring, wring, bars, red, ctl, beg, end);
+            rf_role<MODE, TM, kRfScaleNone, SP>(p, aring, wring, bars, red, ctl, beg, end);
         }
     } else if (warp == kWeightWarpR) {
         if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
@@ -1606,11 +1669,14 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
 // Bytes of the register-operand kernel's residue sums (after the ring in dynamic shared memory).
 static int rf_red_bytes(int tm) { return 4 * tm * kTileN * 4; }
 
-int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl) {
+int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl, bool sparse) {
     pl->mode = mode;
     pl->k_blocks = K / kTileK;
     pl->n_tiles = n_tiles(N);
-    pl->blob_bytes = (mode == kModeGroup)     ? static_cast<int>(blob_bytes_w4a16(slots))
+    pl->sparse = sparse;
+    if (sparse && (M > kRfMaxM || (mode != kModeGroup && mode != kModeChannel))) return -1;
+    pl->blob_bytes = sparse                   ? static_cast<int>(blob_bytes_sp24(slots))
+                     : (mode == kModeGroup)   ? static_cast<int>(blob_bytes_w4a16(slots))
                      : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
                                               : kCodeBytes;
     pl->rf = M <= kRfMaxM;
@@ -1621,7 +1687,9 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
         pl->small = false;
         pl->threads = kThreadsRf;
         pl->issuers = 0;
-        pl->act_slot = (mode == kModeW4A8) ? tm * 128 : tm * 256;  // TM rows x 128 int8 or fp16, unswizzled
+        // TM rows x 128 int8 or fp16, unswizzled; sparse: at least 8 rows, swizzled
+        pl->act_rows = (sparse && tm < kSpMinActRows) ? kSpMinActRows : tm;
+        pl->act_slot = (mode == kModeW4A8) ? tm * 128 : pl->act_rows * 256;
         const int budget = smem_optin - 2048 - 1024 - rf_red_bytes(tm);
         int s = budget / (pl->act_slot + pl->blob_bytes);
         if (s > kMaxSlots) s = kMaxSlots;
@@ -1641,6 +1709,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
     tm = ((tm + 15) / 16) * 16;
     if (tm < 16) tm = 16;
     pl->tile_m = tm;
+    pl->act_rows = tm;
     pl->m_tiles = (M + tm - 1) / tm;
     if (pl->m_tiles < 1) pl->m_tiles = 1;
     pl->small = tm <= kSmallTileMax;
@@ -1698,6 +1767,16 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 16>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 16>, max_dynamic_smem);
     }
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 4, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 1, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 2, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 4, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16, true>, max_dynamic_smem);
     if constexpr (kRfMaxM > 16) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 32>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 32>, max_dynamic_smem);
@@ -1732,6 +1811,17 @@ static cudaError_t launch_kernel(Kernel k, const ActMaps& maps, const GemmArgs& 
 template <int MODE>
 static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const Plan& plan, cudaStream_t st) {
     {
+        if (plan.rf && plan.sparse) {
+            if constexpr (MODE == kModeGroup || MODE == kModeChannel) {
+                if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1, true>, maps, args, plan, st);
+                if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2, true>, maps, args, plan, st);
+                if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4, true>, maps, args, plan, st);
+                if (plan.tile_m == 8) return launch_kernel(wq_gemm_rf<MODE, 8, true>, maps, args, plan, st);
+                if (plan.tile_m == 16) return launch_kernel(wq_gemm_rf<MODE, 16, true>, maps, args, plan, st);
+            }
+            return cudaErrorInvalidConfiguration;
+        }
+        if (plan.sparse) return cudaErrorInvalidConfiguration;
         if (plan.rf) {
             if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1>, maps, args, plan, st);
             if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2>, maps, args, plan, st);

@@ -49,9 +49,12 @@ struct Plan {
     int grid, issuers, slots, chunk, act_slot, blob_bytes, smem_bytes, threads;
     bool small;
     bool rf;    // M <= kRfMaxM: the register-operand kernel, unswizzled activation slots
+    bool sparse;   // 2:4 sparse weights (register-operand kernel only; swizzled activation slots)
+    int act_rows;  // rows of one activation copy: tile_m, or at least kSpMinActRows when sparse
 };
 
-int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan);
+int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan,
+              bool sparse = false);
 
 cudaError_t configure_gemm_kernels(int max_dynamic_smem);
 
@@ -63,6 +66,9 @@ int launch_prepack(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K,
 int launch_prepack_w4a8(const int32_t* Q, int K, int N, void* Wp, cudaStream_t st);
 int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* z, cudaStream_t st);
 int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st);
+int launch_prepack_sp24(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, int* bad,
+                        cudaStream_t st);
+int launch_unpack_sp24(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st);
 int launch_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* Aq, float* sa, cudaStream_t st);
 int launch_permute_codes(const int32_t* Q, const int32_t* perm, int K, int N, int32_t* Qp, cudaStream_t st);
 int launch_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, uint16_t* Ap, int* status,

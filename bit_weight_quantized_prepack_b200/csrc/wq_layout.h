@@ -17,6 +17,20 @@
 // Prepacked W4A16 buffer with zero points (g < K): each blob is the W4A16 blob followed by
 //   `slots` rows of 128 uint8 zero points z (0..15), laid out like the scale rows; padded
 //   columns hold zero point 8 (and scale 0).
+// Prepacked 2:4 sparse W4A16 buffer (every run of 4 rows 4i .. 4i+3 of a column holds at most
+//   two codes other than 8): the blobs of the W4A16 buffer with the 8192 bytes of code words
+//   replaced by 4096 bytes of code words and 2048 bytes of metadata words (then the scale
+//   rows, or the column scales after the last blob for g == K). Within blob (nt, kt), 32-row
+//   block b < 4 holds pruning groups j < 8 (rows 32b + 4j .. + 3); column c of the tile is in
+//   row tile rt = c / 16, with gc = c % 8 and half = (c % 16) / 8:
+//     code word (b*8 + rt)*32 + 4gc + (j % 4), nibble half + 2*(j / 4) + 4i: kept code i
+//       (0: the lower kept row) of group j of column c;
+//     metadata word ((b*8 + rt)*8 + gc)*2 + j / 4, nibble (j % 4) + 4*half: the kept rows'
+//       positions in the group, bits 0-1 the lower, bits 2-3 the higher.
+//   The kept rows of a group are those whose code is not 8, made up to two with the lowest
+//   other rows. Code word 32*(b*8 + rt) + lane is exactly lane's A operand of the sparse warp
+//   MMA (m16n8k32, groups of 4 along k) for that row tile and block, and metadata word
+//   16*(b*8 + rt) + lane / 2 its metadata operand (lanes 4gc, 4gc + 1).
 //
 // Nibble orders. Within a word the W4A16 order puts codes (2p, 2p+1) at nibble positions
 // (p, p+4) for p = 0..3, so that masking 0x000F000F (p = 0) or 0x00F000F0 (p = 1) of the
@@ -63,6 +77,11 @@ constexpr int kASlots = 4;                    // dequantised weight tiles in ten
 constexpr int kTmemCols = 512;
 constexpr int kTmemAOffset = 256;             // accumulators in columns [0, 256), A slots above
 
+constexpr int kSpCodeBytes = 4096;           // 2:4 sparse blob: kept codes
+constexpr int kSpMetaBytes = 2048;           // then 2-bit positions of the kept codes
+constexpr int kSpHeadBytes = kSpCodeBytes + kSpMetaBytes;  // the scale rows start here
+constexpr int kSpMinActRows = 8;             // sparse: activation rows per slot (one 128-byte swizzle atom)
+
 enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2, kModeGroupZP = 3 };
 
 // Scale rows per blob for W4A16; 0 means per-column scales (g == K); -1 unsupported.
@@ -82,6 +101,9 @@ inline size_t blob_bytes_w4a16(int slots) { return kCodeBytes + 2u * kTileN * st
 
 // Asymmetric groups: the W4A16 blob followed by `slots` rows of 128 uint8 zero points.
 inline size_t blob_bytes_w4a16_zp(int slots) { return blob_bytes_w4a16(slots) + static_cast<size_t>(kTileN) * slots; }
+
+// 2:4 sparse W4A16: code and metadata words, then `slots` rows of 128 fp16 scales.
+inline size_t blob_bytes_sp24(int slots) { return kSpHeadBytes + 2u * kTileN * static_cast<size_t>(slots); }
 
 inline size_t channel_tail_bytes(int N) { return ((2u * n_tiles(N) * kTileN) + 15u) / 16u * 16u; }
 

@@ -1,5 +1,6 @@
 // The layout pass: reorder 4-bit codes, group scales and (asymmetric groups) zero points into
-// the blobs the GEMM streams, and its inverse (a test aid). Layout: see wq_layout.h.
+// the blobs the GEMM streams, and its inverse (a test aid); the same for 2:4 sparse weights
+// (kept codes and their positions). Layouts: see wq_layout.h.
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -74,7 +75,7 @@ __global__ void unpack_codes_kernel(const uint8_t* __restrict__ wp, int N, int K
 
 // One thread per (blob, slot, r): copy one scale into the blob's scale rows.
 __global__ void prepack_scales_kernel(const uint16_t* __restrict__ s, int N, int KT, int g, int slots,
-                                      long long total, uint8_t* __restrict__ wp, size_t blob_bytes) {
+                                      long long total, uint8_t* __restrict__ wp, size_t blob_bytes, int head) {
     long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
     if (idx >= total) return;
     const int r = static_cast<int>(idx % kTileN);
@@ -85,11 +86,11 @@ __global__ void prepack_scales_kernel(const uint16_t* __restrict__ s, int N, int
     const long long n = nt * kTileN + r;
     const long long grp = (static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g) / g;
     const uint16_t v = (n < N) ? s[grp * N + n] : static_cast<uint16_t>(0);
-    reinterpret_cast<uint16_t*>(wp + blob * blob_bytes + kCodeBytes)[u * kTileN + r] = v;
+    reinterpret_cast<uint16_t*>(wp + blob * blob_bytes + head)[u * kTileN + r] = v;
 }
 
 __global__ void unpack_scales_kernel(const uint8_t* __restrict__ wp, int N, int KT, int g, int slots,
-                                     long long total, uint16_t* __restrict__ s, size_t blob_bytes) {
+                                     long long total, uint16_t* __restrict__ s, size_t blob_bytes, int head) {
     long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
     if (idx >= total) return;
     const int r = static_cast<int>(idx % kTileN);
@@ -100,7 +101,7 @@ __global__ void unpack_scales_kernel(const uint8_t* __restrict__ wp, int N, int 
     const long long n = nt * kTileN + r;
     const long long row0 = static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g;
     if (n >= N || row0 % g != 0) return;  // a group larger than a blob is written by its first blob only
-    s[(row0 / g) * N + n] = reinterpret_cast<const uint16_t*>(wp + blob * blob_bytes + kCodeBytes)[u * kTileN + r];
+    s[(row0 / g) * N + n] = reinterpret_cast<const uint16_t*>(wp + blob * blob_bytes + head)[u * kTileN + r];
 }
 
 // One thread per (blob, slot, r): copy one zero point into the blob's zero rows (asymmetric groups).
@@ -162,7 +163,7 @@ int launch_prepack(const int32_t* Q, const uint16_t* s, const uint8_t* z, int K,
                                                                       wp, blob);
     if (slots > 0) {
         const long long ts = nblob * slots * kTileN;
-        prepack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(s, N, KT, g, slots, ts, wp, blob);
+        prepack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(s, N, KT, g, slots, ts, wp, blob, kCodeBytes);
         if (z)
             prepack_zeros_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(z, N, KT, g, slots, ts, wp, blob,
                                                                        blob_bytes_w4a16(slots));
@@ -194,7 +195,7 @@ int launch_unpack(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, 
                                                                      blob);
     if (slots > 0) {
         const long long ts = nblob * slots * kTileN;
-        unpack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, s, blob);
+        unpack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, s, blob, kCodeBytes);
         if (z)
             unpack_zeros_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, z, blob,
                                                                       blob_bytes_w4a16(slots));
@@ -210,6 +211,130 @@ int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st
     const long long tc = static_cast<long long>(NT) * KT * 4 * kTileN;
     unpack_codes_kernel<true><<<blocks_for(tc, 256), 256, 0, st>>>(static_cast<const uint8_t*>(Wp), N, KT, tc,
                                                                     reinterpret_cast<uint32_t*>(Q), kCodeBytes);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+// ------------------------------------------------------------------ 2:4 sparse weights
+// One thread per (blob, code word w < 1024): w = (b*8 + rt)*32 + lane, lane = 4gc + t. The
+// thread reads the four groups its word holds (groups t and t + 4 of columns 16rt + gc and
+// + 8), picks each group's kept rows, writes the word and ORs its metadata nibbles with those
+// of the quad's other lanes (t = 0..3), whose lanes 0 and 1 write the quad's two metadata
+// words. A group with more than two codes other than 8 sets *bad (its two lowest such codes
+// are kept). Launched in blocks of 256 over whole blobs, so a quad is always one warp's.
+__global__ void prepack_sp24_codes_kernel(const uint32_t* __restrict__ Q, int N, int KT, long long total,
+                                          uint8_t* __restrict__ wp, size_t blob_bytes, int* __restrict__ bad) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;  // total is a multiple of 1024: whole warps leave together
+    const int w = static_cast<int>(idx % 1024);
+    const long long blob = idx / 1024;
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const int b = w >> 8, rt = (w >> 5) & 7, gc = (w >> 2) & 7, t = w & 3;
+    uint32_t code = 0, meta[2] = {0u, 0u};
+    bool over = false;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const long long n = nt * kTileN + 16 * rt + 8 * half + gc;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const int j = t + 4 * x;                                                // group: rows 32b + 4j ..
+            const long long qrow = static_cast<long long>(kt) * 16 + 4 * b + (j >> 1);  // row of Q (8 codes)
+            const uint32_t src = (n < N) ? __ldg(Q + qrow * N + n) : 0x88888888u;
+            const uint32_t c4 = (src >> (16 * (j & 1))) & 0xFFFFu;  // the group's codes, position p at bits 4p
+            uint32_t nz = 0;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) nz |= (((c4 >> (4 * p)) & 0xFu) != 8u ? 1u : 0u) << p;
+            over = over || __popc(nz) > 2;
+            uint32_t keep = nz;
+#pragma unroll
+            for (int p = 0; p < 4; ++p)  // made up to two with the lowest rows of code 8
+                if (__popc(keep) < 2 && !((keep >> p) & 1u)) keep |= 1u << p;
+            const int p0 = __ffs(keep) - 1;
+            const int p1 = __ffs(keep & (keep - 1)) - 1;
+            code |= ((c4 >> (4 * p0)) & 0xFu) << (4 * (half + 2 * x));
+            code |= ((c4 >> (4 * p1)) & 0xFu) << (4 * (half + 2 * x + 4));
+            meta[x] |= static_cast<uint32_t>(p0 | (p1 << 2)) << (4 * (t + 4 * half));
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+        meta[x] |= __shfl_xor_sync(0xffffffffu, meta[x], 1);
+        meta[x] |= __shfl_xor_sync(0xffffffffu, meta[x], 2);
+    }
+    uint8_t* base = wp + blob * blob_bytes;
+    reinterpret_cast<uint32_t*>(base)[w] = code;
+    if (t < 2) reinterpret_cast<uint32_t*>(base + kSpCodeBytes)[((b * 8 + rt) * 8 + gc) * 2 + t] = meta[t];
+    if (over) *bad = 1;
+}
+
+// One thread per (blob, row i of Q within the k-block (8 codes), column r): rebuilds the 8
+// codes (pruned rows as 8) from the code and metadata words of their two groups.
+__global__ void unpack_sp24_codes_kernel(const uint8_t* __restrict__ wp, int N, int KT, long long total,
+                                         uint32_t* __restrict__ Q, size_t blob_bytes) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int i = static_cast<int>((idx / kTileN) % 16);
+    const long long blob = idx / (16 * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const long long n = nt * kTileN + r;
+    if (n >= N) return;
+    const uint8_t* base = wp + blob * blob_bytes;
+    const uint32_t* code = reinterpret_cast<const uint32_t*>(base);
+    const uint32_t* meta = reinterpret_cast<const uint32_t*>(base + kSpCodeBytes);
+    const int b = i >> 2, rt = r >> 4, half = (r >> 3) & 1, gc = r & 7;
+    uint32_t out = 0x88888888u;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int j = 2 * (i & 3) + e;  // group j: rows 32b + 4j .. = codes 4e .. 4e + 3 of this Q word
+        const uint32_t m = (meta[((b * 8 + rt) * 8 + gc) * 2 + (j >> 2)] >> (4 * ((j & 3) + 4 * half))) & 0xFu;
+        const uint32_t cw = code[(b * 8 + rt) * 32 + 4 * gc + (j & 3)];
+        const int p0 = static_cast<int>(m & 3u), p1 = static_cast<int>(m >> 2);
+        const uint32_t c0 = (cw >> (4 * (half + 2 * (j >> 2)))) & 0xFu;
+        const uint32_t c1 = (cw >> (4 * (half + 2 * (j >> 2) + 4))) & 0xFu;
+        out = (out & ~(0xFu << (4 * (4 * e + p0)))) | (c0 << (4 * (4 * e + p0)));
+        out = (out & ~(0xFu << (4 * (4 * e + p1)))) | (c1 << (4 * (4 * e + p1)));
+    }
+    Q[(static_cast<long long>(kt) * 16 + i) * N + n] = out;
+}
+
+int launch_prepack_sp24(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, int* bad,
+                        cudaStream_t st) {
+    const int slots = scale_slots(K, g);
+    const int KT = K / kTileK, NT = n_tiles(N);
+    const size_t blob = blob_bytes_sp24(slots > 0 ? slots : 0);
+    uint8_t* wp = static_cast<uint8_t*>(Wp);
+    const long long nblob = static_cast<long long>(NT) * KT;
+    const long long tc = nblob * 1024;
+    prepack_sp24_codes_kernel<<<blocks_for(tc, 256), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(Q), N, KT, tc,
+                                                                    wp, blob, bad);
+    if (slots > 0) {
+        const long long ts = nblob * slots * kTileN;
+        prepack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(s, N, KT, g, slots, ts, wp, blob, kSpHeadBytes);
+    } else {
+        const int tail_elems = static_cast<int>(channel_tail_bytes(N) / 2);
+        channel_tail_kernel<<<blocks_for(tail_elems, 256), 256, 0, st>>>(
+            s, N, NT * kTileN, tail_elems, reinterpret_cast<uint16_t*>(wp + nblob * blob));
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_unpack_sp24(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st) {
+    const int slots = scale_slots(K, g);
+    const int KT = K / kTileK, NT = n_tiles(N);
+    const size_t blob = blob_bytes_sp24(slots > 0 ? slots : 0);
+    const uint8_t* wp = static_cast<const uint8_t*>(Wp);
+    const long long nblob = static_cast<long long>(NT) * KT;
+    const long long tc = nblob * 16 * kTileN;
+    unpack_sp24_codes_kernel<<<blocks_for(tc, 256), 256, 0, st>>>(wp, N, KT, tc, reinterpret_cast<uint32_t*>(Q), blob);
+    if (slots > 0) {
+        const long long ts = nblob * slots * kTileN;
+        unpack_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, s, blob, kSpHeadBytes);
+    } else {
+        channel_untail_kernel<<<blocks_for(N, 256), 256, 0, st>>>(
+            reinterpret_cast<const uint16_t*>(wp + nblob * blob), N, s);
+    }
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

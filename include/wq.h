@@ -62,7 +62,8 @@ typedef enum {
     WQ_ERR_TIMEOUT = 6,            /* a device-side bounded wait expired (see wq_get_device_status) */
     WQ_ERR_NO_MEMORY = 7,          /* the library could not allocate its workspace */
     WQ_ERR_CAPTURING = 8,          /* the workspace must grow while the stream is being captured */
-    WQ_ERR_SCRATCH_LIMIT = 9       /* wq_gemm_w4a16_noalloc: the plan needs more than its fixed scratch */
+    WQ_ERR_SCRATCH_LIMIT = 9,      /* wq_gemm_w4a16_noalloc: the plan needs more than its fixed scratch */
+    WQ_ERR_NOT_SPARSE = 10         /* wq_prepack_sparse24: the codes are not 2:4 sparse */
 } wq_status_t;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -159,6 +160,30 @@ WQ_API int wq_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, 
 WQ_API int wq_gemm_w4a16_act_order(const uint16_t* A, const int32_t* perm, const void* Wp, uint16_t* Y,
                  int M, int N, int K, int g, int zero_points, void* stream);
 
+/* ---------------------------------------------------------------- 2:4 sparse weights
+ * The W4A16 layer on a weight in which every run of 4 rows 4i .. 4i+3 of a column holds at
+ * most 2 codes other than 8 (2 of every 4 weights are zero): "MARLIN: Mixed-Precision
+ * Auto-Regressive Parallel Inference on Large Language Models", Abstract, names the kernel's
+ * extension to NVIDIA 2:4 sparsity and gives no format; the one here is this library's own.
+ * The buffer keeps the two kept codes of each run and their 2-bit positions: 3/4 of the
+ * dense buffer's code bytes. The result is the W4A16 layer of the same (pruned) weight.
+ * wq_prepacked_bytes_sparse24: size of the buffer, or 0 when the shape or g is unsupported
+ * (g as for wq_gemm_w4a16, g == K included).
+ * wq_prepack_sparse24: Q int32 [K/8, N] (pruned codes), s fp16 [K/g, N] -> Wp. Checks the
+ * pattern on the device and returns WQ_ERR_NOT_SPARSE when a run holds more than 2 codes
+ * other than 8 (Wp's content is then unspecified); the call therefore synchronises `stream`
+ * and returns WQ_ERR_CAPTURING while the stream is being captured. Run once per weight.
+ * wq_unpack_sparse24: the inverse (test aid): Q_out with the pruned codes as 8, s_out.
+ * wq_gemm_w4a16_sparse24: Y [M, N] = A . W as wq_gemm_w4a16 (same rounding: for g = 32 the
+ * fp16 weight is rounded once; for g >= 64 the scale multiplies each group's fp32 sum), for
+ * 0 <= M <= 16 (WQ_ERR_UNSUPPORTED_SHAPE above: the sparse warp MMA serves the decode-sized
+ * batches, where the weight bytes bound the layer). Workspace: wq_workspace_bytes(5, ...). */
+WQ_API size_t wq_prepacked_bytes_sparse24(int K, int N, int g);
+WQ_API int wq_prepack_sparse24(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, void* stream);
+WQ_API int wq_unpack_sparse24(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, void* stream);
+WQ_API int wq_gemm_w4a16_sparse24(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g,
+                 void* stream);
+
 /* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
  * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
  * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
@@ -219,7 +244,7 @@ WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
 /* ---------------------------------------------------------------- workspace and status
  * Bytes of library workspace one call of the given kind and shape needs (kind 0 = W4A16,
  * 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act, 3 = wq_gemm_w4a16_zp,
- * 4 = wq_gemm_w4a16_act_order). */
+ * 4 = wq_gemm_w4a16_act_order, 5 = wq_gemm_w4a16_sparse24 (0 for M > 16)). */
 WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it
@@ -239,7 +264,8 @@ WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
 WQ_API int wq_get_device_status(void* stream);
 
 /* ---------------------------------------------------------------- introspection and test hooks
- * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8. */
+ * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8, 5 = 2:4 sparse W4A16
+ * (M <= 16). */
 typedef struct {
     int grid;         /* persistent CTAs launched (<= number of SMs) */
     int tile_m;       /* activation rows per tile: 1, 2, 4, 8 or 16 for the register-operand kernel

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(wq):
 def test_version_and_status_strings(wq):
     assert wq.wq_version() >= 10000
     seen = set()
-    for st in range(9):
+    for st in range(11):
         s = wq.status_string(st)
         assert s.startswith("WQ_") and s not in seen
         seen.add(s)
@@ -55,6 +55,12 @@ def test_version_and_status_strings(wq):
 def test_prepacked_bytes_agree_with_oracle(wq, K, N, g):
     assert wq.wq_prepacked_bytes(K, N, g) == oracle.prepacked_bytes_w4a16(K, N, g)
     assert wq.wq_prepacked_bytes_w4a8(K, N) == oracle.prepacked_bytes_w4a8(K, N)
+
+
+@pytest.mark.parametrize("K,N,g", [(128, 8, 128), (384, 296, 128), (384, 296, 32), (4096, 4096, 4096),
+                                   (256, 200, 64), (1280, 520, 640)])
+def test_sparse_prepacked_bytes_agree_with_oracle(wq, K, N, g):
+    assert wq.wq_prepacked_bytes_sparse24(K, N, g) == oracle.prepacked_bytes_w4a16_sparse24(K, N, g)
 
 
 @pytest.mark.parametrize("K,N,g", [(100, 128, 100), (128, 12, 128), (0, 128, 128), (256, 128, 48),
@@ -93,6 +99,17 @@ def test_host_side_argument_checks(wq):
     assert L.wq_gemm_w4a16(good, good, odd, 1, 128, 128, 128, None) == wq.WQ_ERR_MISALIGNED
     assert L.wq_gemm_w4a8(good, P(0x10002), good, good, good, None, 1, 128, 128, None) == wq.WQ_ERR_MISALIGNED
     assert L.wq_prepack(odd, good, 128, 128, 128, good, None) == wq.WQ_ERR_MISALIGNED
+    # 2:4 sparse: the sparse warp MMA serves M <= 16; the same shape, group and pointer checks
+    assert L.wq_gemm_w4a16_sparse24(good, good, good, 17, 128, 128, 128, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
+    assert L.wq_gemm_w4a16_sparse24(good, good, good, 1, 128, 100, 128, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
+    assert L.wq_gemm_w4a16_sparse24(good, good, good, 1, 128, 256, 48, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_gemm_w4a16_sparse24(good, odd, good, 1, 128, 128, 128, None) == wq.WQ_ERR_MISALIGNED
+    assert L.wq_gemm_w4a16_sparse24(None, good, None, 0, 128, 128, 128, None) == wq.WQ_OK
+    assert L.wq_prepack_sparse24(good, good, 256, 128, 96, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_prepack_sparse24(odd, good, 128, 128, 128, good, None) == wq.WQ_ERR_MISALIGNED
+    assert L.wq_prepack_sparse24(good, None, 128, 128, 128, good, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_unpack_sparse24(good, 128, 128, 128, good, odd, None) == wq.WQ_ERR_MISALIGNED
+    assert wq.wq_prepacked_bytes_sparse24(256, 128, 96) == 0
     # an empty batch is a no-op that needs no activation or output pointer
     assert L.wq_gemm_w4a16(None, good, None, 0, 128, 128, 128, None) == wq.WQ_OK
     assert L.wq_gemm_w4a8(None, None, good, None, None, None, 0, 128, 128, None) == wq.WQ_OK

@@ -11,7 +11,8 @@ import bit_weight_quantized_prepack_b200 as wq
 class _Recorder:
     """Stands in for the loaded library: records every entry point called, except the pure size
     queries, which it forwards to the real library."""
-    PURE = {"wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepacked_bytes_zp", "wq_status_string"}
+    PURE = {"wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepacked_bytes_zp", "wq_prepacked_bytes_sparse24",
+            "wq_status_string"}
 
     def __init__(self, real):
         self.real, self.calls = real, []
@@ -143,4 +144,25 @@ def test_act_order_calls_refuse_wrong_sizes(rec):
     with pytest.raises(ValueError):  # the zero-point buffer is larger than the symmetric one
         wq.wq_gemm_w4a16_act_order(A, perm, torch.zeros(wq.wq_prepacked_bytes(K, N, g), dtype=torch.uint8), N, g,
                                    zero_points=True)
+    assert rec.calls == []
+
+
+def test_sparse_calls_refuse_wrong_sizes(rec):
+    Q = torch.zeros((K // 8, N), dtype=torch.int32)
+    with pytest.raises(ValueError):  # s must be [K/g, N]
+        wq.wq_prepack_sparse24(Q, torch.zeros((K // g + 1, N), dtype=torch.float16), g)
+    with pytest.raises(ValueError):  # caller-given Wp too small
+        wq.wq_prepack_sparse24(Q, torch.zeros((K // g, N), dtype=torch.float16), g,
+                               Wp=torch.zeros(wq.wq_prepacked_bytes_sparse24(K, N, g) - 16, dtype=torch.uint8))
+    with pytest.raises(wq.WqError):  # g does not divide K
+        wq.wq_prepack_sparse24(Q, torch.zeros((2, N), dtype=torch.float16), 96)
+    with pytest.raises(ValueError):  # the dense buffer is larger, the sparse one must hold its own size
+        wq.wq_gemm_w4a16_sparse24(torch.zeros((M, K), dtype=torch.float16),
+                                  torch.zeros(wq.wq_prepacked_bytes_sparse24(K, N, g) - 1, dtype=torch.uint8), N, g)
+    with pytest.raises(ValueError):
+        wq.wq_gemm_w4a16_sparse24(torch.zeros((M, K), dtype=torch.float16),
+                                  torch.zeros(wq.wq_prepacked_bytes_sparse24(K, N, g), dtype=torch.uint8), N, g,
+                                  Y=torch.zeros((M, N + 8), dtype=torch.float16))
+    with pytest.raises(ValueError):
+        wq.wq_unpack_sparse24(torch.zeros(16, dtype=torch.uint8), K, N, g)
     assert rec.calls == []

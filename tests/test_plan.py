@@ -55,6 +55,33 @@ def test_plan_invariants(wq, K, N, kind, g):
         assert p["threads"] == (576 if _rf(kind, M) else 704)
 
 
+@pytest.mark.parametrize("K,N", SHAPES)
+@pytest.mark.parametrize("g", [32, 64, 128, 256, None])
+def test_sparse_plan_invariants(wq, K, N, g):
+    # 2:4 sparse W4A16 (kind 5): the register-operand kernel only; activation slots of at
+    # least 8 rows (one 1024-byte swizzle atom per 64-column piece); blobs of 6144 bytes of
+    # codes and metadata plus the scale rows
+    g = K if g is None else g
+    if K % g:
+        pytest.skip("group size must divide K")
+    for M in [m for m in MS if m <= 16]:
+        p = wq.wq_plan_for(5, M, N, K, g, SMS, SMEM)
+        dense = wq.wq_plan_for(0, M, N, K, g, SMS, SMEM)
+        tm = p["tile_m"]
+        assert tm == dense["tile_m"] and p["grid"] == dense["grid"] and p["units"] == dense["units"]
+        assert p["threads"] == 576 and p["m_tiles"] == 1
+        act = max(tm, 8) * 256
+        blob = 6144 + (256 * (128 // min(g, 128)) if g < K else 0)
+        assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024 + _red(p)
+        assert p["smem_bytes"] + 2048 <= SMEM
+        more = (p["stages"] + 1) * (act + blob) + 1024 + _red(p)
+        assert p["stages"] == 32 or more + 2048 > SMEM
+    for M in (17, 32, 100):
+        with pytest.raises(wq.WqError) as e:
+            wq.wq_plan_for(5, M, N, K, g, SMS, SMEM)
+        assert e.value.status == wq.WQ_ERR_UNSUPPORTED_SHAPE
+
+
 def test_plan_uses_the_largest_ring_that_fits(wq):
     for M, kind in itertools.product([1, 16, 32, 64, 256], [0, 1]):
         p = wq.wq_plan_for(kind, M, 4096, 4096, 128 if kind == 0 else 4096, SMS, SMEM)
