@@ -257,6 +257,47 @@ def rows_70b(torch, wq, dev, stream, hbm_gbs, tflops):
     return out
 
 
+SPARSE_LAYERS = LAYERS + [(8192, 57344)]
+SPARSE_M = [1, 4, 16]
+
+
+def sparse_algo_bytes(M, K, N, g=G):
+    """Algorithmic bytes of one 2:4 sparse call: the kept codes (K/2 x N x 4 bits), their
+    positions (K/4 groups x N x 4 bits), the scales, A and Y."""
+    return K * N // 4 + K * N // 8 + 2 * (K // g) * N + 2 * M * K + 2 * M * N
+
+
+def rows_sparse24(torch, wq, dev, stream, hbm_gbs):
+    """2:4 sparse W4A16 (the Llama-7B layers and the 70B gate/up layer, g = 128, M in {1, 4, 16}):
+    the same pruned weight through the dense and the sparse buffer, each call back to back in a
+    CUDA graph over rotated copies (more than 3x L2 per rotation); per call: microseconds, GB/s
+    of the sparse call's own algorithmic bytes, its roofline fraction, and the dense call's time
+    over the sparse call's."""
+    out = {}
+    for K, N in SPARSE_LAYERS:
+        d = synth.w4a16_sparse24_inputs(K, N, G, max(SPARSE_M), seed=31)
+        Q, s = torch.from_numpy(d["Q"]).to(dev), torch.from_numpy(d["s"]).to(dev)
+        copies = int(min(12, max(2, -(-3 * 126_000_000 // (K * N * 3 // 8)))))
+        Wd = [wq.wq_prepack(Q, s, G) for _ in range(copies)]
+        Ws = [wq.wq_prepack_sparse24(Q, s, G) for _ in range(copies)]
+        A = torch.from_numpy(d["A"]).to(dev)
+        for M in SPARSE_M:
+            Am = A[:M].contiguous()
+            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            wq.wq_workspace_reserve(wq.wq_workspace_bytes(0, M, N, K), stream=stream)
+            td = _graph_time(torch, stream, lambda r: wq.wq_gemm_w4a16(Am, Wd[r % copies], N, G, Y=Y, stream=stream),
+                             2 * copies)
+            ts = _graph_time(torch, stream,
+                             lambda r: wq.wq_gemm_w4a16_sparse24(Am, Ws[r % copies], N, G, Y=Y, stream=stream),
+                             2 * copies)
+            b = sparse_algo_bytes(M, K, N)
+            out[f"{K}x{N}_M{M}"] = {"us": round(ts * 1e6, 2), "dense_us": round(td * 1e6, 2),
+                                   "gbs": round(b / ts / 1e9, 1), "roofline_frac": round(b / (hbm_gbs * 1e9) / ts, 3),
+                                   "speedup_vs_dense": round(td / ts, 3)}
+        del Wd, Ws, Q, s, A
+    return out
+
+
 def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
     """The compute-bound W4A16 sweep (K = N = 8192) and the W4A8 layers, each timed alone."""
     out = {"compute_sweep": {}, "w4a8": {}}
@@ -324,6 +365,7 @@ def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
     out["peaks"] = {"tensor_tflops": tflops, "int8_tops": int8_peak,
                     "note": "int8 peak = measured bf16 peak x the nominal 2x ratio"}
     out["layers_70b"] = rows_70b(torch, wq, dev, stream, hbm_gbs, tflops)
+    out["sparse24"] = rows_sparse24(torch, wq, dev, stream, hbm_gbs)
     return out
 
 
