@@ -28,7 +28,9 @@ Around the layer (each function's docstring gives its reading of the pages):
 * act order (``dequant_gidx``, ``w4a16_gidx``, ``act_order_perm``,
   ``reorder_rows``): groups whose rows are scattered along K by ``g_idx``;
 * 2:4 sparse weights (``is_sparse24``, ``prepack_w4a16_sparse24``): the layer is
-  ``w4a16`` of the pruned weight; only the prepacked format differs.
+  ``w4a16`` of the pruned weight; only the prepacked format differs;
+* mixed 2/4-bit weights (``dequant_mixed``, ``w4a16_mixed``, ``prepack_mixed``): a bit width
+  per aligned 32-row x 128-column block, zero point 2 or 8.
 
 Every function here is pinned by ``tests/oracle_pins.py`` (hand-worked golden
 values, exact rational brute force, closed forms and invariants); none is
@@ -62,7 +64,8 @@ __all__ = [
     "prepack_w4a16_act_order",
     "dequant_zp", "w4a16_zp", "w4a16_zp_absdot", "prepack_w4a16_zp", "prepacked_bytes_w4a16_zp", "unprepack_w4a16_zp",
     "TILE_N", "TILE_K", "prepack_w4a16", "prepack_w4a8",
-    "is_sparse24", "prepacked_bytes_w4a16_sparse24", "prepack_w4a16_sparse24",
+    "is_sparse24", "MIXED_BLOCK_ROWS", "mixed_zero_points", "dequant_mixed", "w4a16_mixed", "w4a16_mixed_absdot",
+    "prepacked_bytes_mixed", "prepack_mixed", "unprepack_mixed", "prepacked_bytes_w4a16_sparse24", "prepack_w4a16_sparse24",
     "unprepack_w4a16_sparse24",
     "prepacked_bytes_w4a16", "prepacked_bytes_w4a8", "unprepack_w4a16", "unprepack_w4a8",
 ]
@@ -666,3 +669,180 @@ def unprepack_w4a16_sparse24(Wp: np.ndarray, K: int, N: int, g: int):
         tail = nt * kt * blob_bytes
         s = Wp[tail:tail + 2 * nt * TILE_N].copy().view(np.float16)[None, :]
     return q[:, :N], s[:, :N]
+
+
+# --------------------------------------------------------------------------
+# Mixed 2/4-bit weights
+# --------------------------------------------------------------------------
+# "Enabling Fast 2-bit LLM on GPUs: Memory Alignment and Asynchronous Dequantization", Abstract:
+# most groups of weights are quantised to 2 bits and only the small fraction of groups with a
+# large range to 4 bits, the 4-bit groups placed with the GPU's memory alignment in mind.
+# Reading (the page gives no format): the bit width is chosen per aligned block of 32 rows
+# (32i .. 32i+31) and 128 columns (the n-tile), ``widths[K/32, ceil(N/128)]`` in {2, 4}; a
+# b-bit code q in 0 .. 2^b - 1 stands for q - 2^(b-1) (zero point 2 or 8) times the group
+# scale, ``W[k,n] = (q[k,n] - z(k,n)) * s[k // g, n]``. Codes of every width travel in the usual
+# 4-bit packing of Q.
+MIXED_BLOCK_ROWS = 32
+
+
+def mixed_zero_points(widths: np.ndarray, K: int, N: int) -> np.ndarray:
+    """z[K, N]: 2 in 2-bit blocks, 8 in 4-bit blocks."""
+    w = np.asarray(widths)
+    if w.shape != (K // MIXED_BLOCK_ROWS, -(-N // TILE_N)) or not np.isin(w, (2, 4)).all():
+        raise ValueError("widths must be [K/32, ceil(N/128)] with values 2 or 4")
+    per = np.repeat(np.repeat(w, MIXED_BLOCK_ROWS, axis=0), TILE_N, axis=1)[:, :N]
+    return np.where(per == 2, 2, 8).astype(np.int64)
+
+
+def dequant_mixed(q: np.ndarray, s: np.ndarray, g: int, widths: np.ndarray) -> np.ndarray:
+    """``W[k,n] = (q[k,n] - z[k,n]) * s[k // g, n]`` in float64, z from the block's width."""
+    K, N = q.shape
+    if K % g:
+        raise ValueError("g must divide K")
+    z = mixed_zero_points(widths, K, N)
+    if (q.astype(np.int64) >= 2 * z).any():
+        raise ValueError("a code does not fit its block's width")
+    return (q.astype(np.float64) - z) * np.asarray(s, dtype=np.float64)[np.arange(K) // g, :]
+
+
+def w4a16_mixed(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, widths: np.ndarray) -> np.ndarray:
+    """``Y = A . W`` in float64 for mixed 2/4-bit weights."""
+    return np.asarray(A, dtype=np.float64) @ dequant_mixed(unpack_codes(Q), s, g, widths)
+
+
+def w4a16_mixed_absdot(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, widths: np.ndarray) -> np.ndarray:
+    """``sum_k |A[m,k] * W[k,n]|`` for the tolerance of the mixed layer."""
+    return np.abs(np.asarray(A, dtype=np.float64)) @ np.abs(dequant_mixed(unpack_codes(Q), s, g, widths))
+
+
+# Prepacked mixed buffer (the library's own format):
+#   a table of NT*KT + 1 uint32 entries (padded to 16 bytes): entry nt*KT + kt = (byte offset of
+#     blob (nt, kt) / 16) << 4 | wbits, bit v of wbits set when 32-row block v of the blob is
+#     4-bit; the last entry = (end of the blobs / 16) << 4;
+#   for g == K the column scales (NT*128 fp16, padded to 16 bytes) right after the table;
+#   then the blobs, nt-major: blocks v = 0..3 (rows 32v .. of the k-block), each 2048 bytes
+#   (4-bit: word r*4 + i holds rows 32v + 8i + j of column r, code j at nibble
+#   NIBBLE_POS_W4A16[j], as in the dense blob) or 1024 bytes (2-bit: word rt*32 + 4gc + t holds
+#   rows 32v + 8t + r of columns 16rt + gc + 8j at the 2-bit field ``_mixed_field(r, j)``), then
+#   the ``slots`` rows of 128 fp16 group scales.
+def _mixed_field(r: int, j: int) -> int:
+    """2-bit field (bits 2f, 2f+1 of the word) of row 8t + r of column 16rt + gc + 8j."""
+    return r // 2 + 4 * j + 8 * (r % 2)
+
+
+def _mixed_table_bytes(nblob: int) -> int:
+    return ((nblob + 1) * 4 + 15) // 16 * 16
+
+
+def prepacked_bytes_mixed(K: int, N: int, g: int, widths: np.ndarray) -> int:
+    _check_kn(K, N)
+    nt, kt = -(-N // TILE_N), K // TILE_K
+    slots = _group_slots(K, g)
+    w = np.asarray(widths)
+    code = int(np.where(w == 4, 2048, 1024).sum())
+    tail = 0 if slots else ((2 * nt * TILE_N + 15) // 16) * 16
+    return _mixed_table_bytes(nt * kt) + tail + code + nt * kt * 2 * TILE_N * slots
+
+
+def prepack_mixed(Q: np.ndarray, s: np.ndarray, g: int, widths: np.ndarray) -> np.ndarray:
+    """The mixed 2/4-bit prepacked buffer as bytes, following the layout above (loops over the
+    documented indices)."""
+    q = unpack_codes(Q)
+    K, N = q.shape
+    dequant_mixed(q, np.zeros((K // g, N)), g, widths)  # checks the widths and the code ranges
+    w = np.asarray(widths)
+    slots = _group_slots(K, g)
+    nt_n, kt_n = -(-N // TILE_N), K // TILE_K
+    qp = np.full((K, nt_n * TILE_N), 0, dtype=np.uint8)
+    qp[:, :N] = q
+    for nt in range(nt_n):  # padded columns: the zero point of their block (weight 0)
+        for b in range(K // MIXED_BLOCK_ROWS):
+            if nt * TILE_N + TILE_N > N:
+                qp[32 * b:32 * b + 32, max(N, nt * TILE_N):(nt + 1) * TILE_N] = 2 if w[b, nt] == 2 else 8
+    sp = np.zeros((np.asarray(s).shape[0], nt_n * TILE_N), dtype=np.float16)
+    sp[:, :N] = np.asarray(s, dtype=np.float16)
+    nblob = nt_n * kt_n
+    head = _mixed_table_bytes(nblob) + (0 if slots else ((2 * nt_n * TILE_N + 15) // 16) * 16)
+    out = np.zeros(prepacked_bytes_mixed(K, N, g, w), dtype=np.uint8)
+    table = np.zeros(nblob + 1, dtype=np.uint32)
+    pos = head
+    for nt in range(nt_n):
+        for kt in range(kt_n):
+            wbits = sum(1 << v for v in range(4) if w[4 * kt + v, nt] == 4)
+            table[nt * kt_n + kt] = ((pos // 16) << 4) | wbits
+            for v in range(4):
+                r0 = kt * TILE_K + 32 * v
+                if w[4 * kt + v, nt] == 4:
+                    words = np.zeros(TILE_N * 4, dtype=np.uint32)
+                    for r in range(TILE_N):
+                        for i in range(4):
+                            for j in range(8):
+                                code = int(qp[r0 + 8 * i + j, nt * TILE_N + r])
+                                words[r * 4 + i] |= np.uint32(code << (4 * NIBBLE_POS_W4A16[j]))
+                else:
+                    words = np.zeros(256, dtype=np.uint32)
+                    for rt in range(8):
+                        for gc in range(8):
+                            for t in range(4):
+                                for j in range(2):
+                                    for r in range(8):
+                                        code = int(qp[r0 + 8 * t + r, nt * TILE_N + 16 * rt + gc + 8 * j])
+                                        words[rt * 32 + 4 * gc + t] |= np.uint32(code << (2 * _mixed_field(r, j)))
+                out[pos:pos + words.nbytes] = words.view(np.uint8)
+                pos += words.nbytes
+            for u in range(slots):
+                grp = (kt * TILE_K + u * g) // g
+                out[pos:pos + 256] = sp[grp, nt * TILE_N:(nt + 1) * TILE_N].view(np.uint8)
+                pos += 256
+    table[nblob] = (pos // 16) << 4
+    out[:table.nbytes] = table.view(np.uint8)
+    if not slots:
+        t0 = _mixed_table_bytes(nblob)
+        out[t0:t0 + 2 * nt_n * TILE_N] = sp[0].view(np.uint8)
+    assert pos == out.nbytes
+    return out
+
+
+def unprepack_mixed(Wp: np.ndarray, K: int, N: int, g: int):
+    """Inverse of ``prepack_mixed``: ``(q[K,N] uint8, s[K/g, N] fp16, widths[K/32, NT] uint8)``."""
+    Wp = np.asarray(Wp, dtype=np.uint8)
+    slots = _group_slots(K, g)
+    nt_n, kt_n = -(-N // TILE_N), K // TILE_K
+    nblob = nt_n * kt_n
+    table = Wp[:(nblob + 1) * 4].copy().view(np.uint32)
+    q = np.zeros((K, nt_n * TILE_N), dtype=np.uint8)
+    s = np.zeros((K // g, nt_n * TILE_N), dtype=np.float16)
+    widths = np.zeros((K // MIXED_BLOCK_ROWS, nt_n), dtype=np.uint8)
+    for nt in range(nt_n):
+        for kt in range(kt_n):
+            e = int(table[nt * kt_n + kt])
+            pos, wbits = (e >> 4) * 16, e & 0xF
+            for v in range(4):
+                r0 = kt * TILE_K + 32 * v
+                if (wbits >> v) & 1:
+                    widths[4 * kt + v, nt] = 4
+                    words = Wp[pos:pos + 2048].copy().view(np.uint32)
+                    for r in range(TILE_N):
+                        for i in range(4):
+                            for j in range(8):
+                                q[r0 + 8 * i + j, nt * TILE_N + r] = (int(words[r * 4 + i]) >> (4 * NIBBLE_POS_W4A16[j])) & 0xF
+                    pos += 2048
+                else:
+                    widths[4 * kt + v, nt] = 2
+                    words = Wp[pos:pos + 1024].copy().view(np.uint32)
+                    for rt in range(8):
+                        for gc in range(8):
+                            for t in range(4):
+                                for j in range(2):
+                                    for r in range(8):
+                                        q[r0 + 8 * t + r, nt * TILE_N + 16 * rt + gc + 8 * j] = \
+                                            (int(words[rt * 32 + 4 * gc + t]) >> (2 * _mixed_field(r, j))) & 0x3
+                    pos += 1024
+            for u in range(slots):
+                grp = (kt * TILE_K + u * g) // g
+                s[grp, nt * TILE_N:(nt + 1) * TILE_N] = Wp[pos:pos + 256].copy().view(np.float16)
+                pos += 256
+    if not slots:
+        t0 = _mixed_table_bytes(nblob)
+        s = Wp[t0:t0 + 2 * nt_n * TILE_N].copy().view(np.float16)[None, :]
+    return q[:, :N], s[:, :N], widths

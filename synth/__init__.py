@@ -30,7 +30,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["pack_q", "w4a16_inputs", "w4a8_inputs", "w4a16_sparse24_inputs"]
+__all__ = ["pack_q", "w4a16_inputs", "w4a8_inputs", "w4a16_sparse24_inputs", "w4a16_mixed_inputs"]
 
 
 def pack_q(q: np.ndarray) -> np.ndarray:
@@ -84,4 +84,18 @@ def w4a16_sparse24_inputs(K: int, N: int, g: int, M: int, seed: int = 0) -> dict
     q[~mask] = 8
     q = q.reshape(K, N)
     d.update(q=q, Q=pack_q(q))
+    return d
+
+
+def w4a16_mixed_inputs(K: int, N: int, g: int, M: int, seed: int = 0, frac4: float = 0.15) -> dict:
+    """The inputs of ``w4a16_inputs`` for mixed 2/4-bit weights: a width per block of 32 rows
+    and 128 columns, 4 with probability ``frac4`` and 2 otherwise (``widths`` uint8
+    [K/32, ceil(N/128)]); the codes of 2-bit blocks are the 4-bit draws reduced mod 4."""
+    d = w4a16_inputs(K, N, g, M, seed=seed)
+    rng = np.random.default_rng(seed + 2)
+    nt = -(-N // 128)
+    widths = np.where(rng.random((K // 32, nt)) < frac4, 4, 2).astype(np.uint8)
+    per = np.repeat(np.repeat(widths, 32, axis=0), 128, axis=1)[:, :N]
+    q = np.where(per == 2, d["q"] % 4, d["q"]).astype(np.uint8)
+    d.update(q=q, Q=pack_q(q), widths=widths)
     return d

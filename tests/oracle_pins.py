@@ -576,6 +576,94 @@ def pin_sparse24_definition(o):
     assert o.is_sparse24(d["q"]) and nz.max() <= 2
 
 
+# ---------------------------------------------------------------- mixed 2/4-bit weights
+MIXED_GOLDEN_WIDTHS = np.array([[2, 4], [4, 4], [2, 4], [2, 4], [2, 2], [2, 2], [2, 2], [2, 4]], np.uint8)
+
+
+def golden_mixed():
+    out = []
+    for line in _rows("mixed_layout.txt"):
+        parts = [p.strip() for p in line.split("|")]
+        K, N, g = (int(x) for x in parts[1].split())
+        ab = None if parts[2] == "-" else tuple(int(x) for x in parts[2].split())
+        offs = [int(x) for x in parts[3].split()]
+        vals = parts[4].split() if len(parts) > 4 else None
+        out.append((parts[0], K, N, g, ab, offs, vals))
+    return out
+
+
+def pin_mixed_layout_golden(o):
+    # the blob table, one code 3 among codes at their zero points, or one scale among zeros:
+    # exactly the bytes and values the hand-worked table names
+    W = MIXED_GOLDEN_WIDTHS
+    bases = {}
+    for what, K, N, g, ab, offs, vals in golden_mixed():
+        z = o.mixed_zero_points(W, K, N).astype(np.uint8)
+        s = np.zeros((K // g, N), np.float16)
+        if (K, N, g) not in bases:
+            bases[K, N, g] = o.prepack_mixed(synth.pack_q(z), s, g, W)
+        base = bases[K, N, g]
+        if what == "table":
+            assert base[:4 * len(offs)].view(np.uint32).tolist() == [int(v) for v in vals]
+            continue
+        q = z.copy()
+        if what == "code":
+            q[ab] = 3
+        else:
+            s[ab] = np.array([_SCALE_BITS], np.uint16).view(np.float16)[0]
+        Wp = o.prepack_mixed(synth.pack_q(q), s, g, W)
+        diff = np.nonzero(Wp != base)[0].tolist()
+        if what == "code":
+            assert diff == offs, (K, N, g, ab, diff, offs)
+            assert [int(Wp[x]) for x in offs] == [int(v, 16) for v in vals], (ab, [hex(int(Wp[x])) for x in offs])
+        else:
+            assert diff == sorted(x for off in offs for x in (off, off + 1)), (K, N, g, ab, diff, offs)
+            for off in offs:
+                assert int(Wp[off]) | (int(Wp[off + 1]) << 8) == _SCALE_BITS
+
+
+def pin_mixed_all_four_bit_is_w4a16(o):
+    # every block 4-bit: the layer is w4a16 bit for bit, and each blob is the dense blob
+    d = synth.w4a16_inputs(256, 200, 64, 3, seed=17)
+    W4 = np.full((256 // 32, 2), 4, np.uint8)
+    assert np.array_equal(o.w4a16_mixed(d["A"], d["Q"], d["s"], 64, W4), o.w4a16(d["A"], d["Q"], d["s"], 64))
+    mixed = o.prepack_mixed(d["Q"], d["s"], 64, W4)
+    dense = o.prepack_w4a16(d["Q"], d["s"], 64)
+    head = (4 * (2 * 2 + 1) + 15) // 16 * 16
+    assert np.array_equal(mixed[head:], dense)
+
+
+def pin_mixed_bruteforce(o):
+    # exact rational sums on a tiny mixed case (one block of each width per column tile)
+    rng = np.random.default_rng(19)
+    K, N, g, M = 64, 8, 32, 2
+    W = np.array([[2], [4]], np.uint8)
+    q = np.vstack([rng.integers(0, 4, (32, N)), rng.integers(0, 16, (32, N))]).astype(np.uint8)
+    s = (0.01 + 0.02 * rng.random((K // g, N))).astype(np.float16)
+    A = rng.standard_normal((M, K)).astype(np.float16)
+    y = o.w4a16_mixed(A, synth.pack_q(q), s, g, W)
+    for m in range(M):
+        for n in range(N):
+            ex = sum(Fraction(float(A[m, k])) * (int(q[k, n]) - (2 if k < 32 else 8)) * Fraction(float(s[k // g, n]))
+                     for k in range(K))
+            assert abs(Fraction(y[m, n]) - ex) <= abs(ex) * Fraction(1, 2 ** 40) + Fraction(1, 2 ** 60)
+
+
+def pin_mixed_two_bit_closed_form(o):
+    # every block 2-bit and every code 0: W = -2 s, so y = -2 sum_k a_k s[k // g]
+    d = synth.w4a16_inputs(128, 24, 32, 2, seed=23)
+    W2 = np.full((4, 1), 2, np.uint8)
+    y = o.w4a16_mixed(d["A"], synth.pack_q(np.zeros((128, 24), np.uint8)), d["s"], 32, W2)
+    want = -2.0 * (d["A"].astype(np.float64) @ d["s"].astype(np.float64)[np.arange(128) // 32])
+    assert np.allclose(y, want, rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):  # a 2-bit block holds codes 0..3 only
+        q = np.zeros((128, 24), np.uint8)
+        q[5, 3] = 4
+        o.w4a16_mixed(d["A"], synth.pack_q(q), d["s"], 32, W2)
+    with pytest.raises(ValueError):  # widths are 2 or 4
+        o.w4a16_mixed(d["A"], d["Q"], d["s"], 32, np.full((4, 1), 3, np.uint8))
+
+
 ALL_PINS = [
     pin_unpack_golden, pin_unpack_matches_generator, pin_hand_examples, pin_bruteforce_w4a16,
     pin_absdot, pin_identity_activation, pin_all_eight, pin_all_zero_codes, pin_scale_homogeneity,
@@ -584,4 +672,5 @@ ALL_PINS = [
     pin_zp_eight_is_symmetric, pin_act_order_golden, pin_act_order_unequal_groups_refused,
     pin_act_order_bruteforce, pin_act_order_contiguous_is_grouped, pin_act_order_reordering_identity,
     pin_pack_codes, pin_sparse24_layout_golden, pin_sparse24_two_kept_codes, pin_sparse24_definition,
+    pin_mixed_layout_golden, pin_mixed_all_four_bit_is_w4a16, pin_mixed_bruteforce, pin_mixed_two_bit_closed_form,
 ]

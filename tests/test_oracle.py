@@ -6,7 +6,7 @@ import oracle
 import synth
 from oracle import wq_oracle as O
 
-from oracle_pins import ALL_PINS, pin_blob_layout_golden, pin_sparse24_layout_golden
+from oracle_pins import ALL_PINS, pin_blob_layout_golden, pin_mixed_layout_golden, pin_sparse24_layout_golden
 
 
 
@@ -187,7 +187,12 @@ def _mut_reorder_within_word(mp):
     mp.setattr(O, "reorder_rows", reorder_rows)
 
 
-MUTATIONS = [_mut_gidx_ignored, _mut_gidx_zero_contiguous, _mut_perm_inverse, _mut_reorder_within_word, _mut_zp_ignored, _mut_zp_sign, _mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
+def _mut_mixed_two_bit_zero_one(mp):
+    real = O.mixed_zero_points
+    mp.setattr(O, "mixed_zero_points", lambda w, K, N: np.where(real(w, K, N) == 2, 1, 8))
+
+
+MUTATIONS = [_mut_mixed_two_bit_zero_one, _mut_gidx_ignored, _mut_gidx_zero_contiguous, _mut_perm_inverse, _mut_reorder_within_word, _mut_zp_ignored, _mut_zp_sign, _mut_act_4bit_8_levels, _mut_act_round_half_up, _mut_act_range_128, _mut_act_scale_per_tensor, _mut_zero_point, _mut_group_mod, _mut_group_off_by_one, _mut_scale_dropped, _mut_nibbles_reversed,
              _mut_k_reversed, _mut_sign_flipped, _mut_w4a8_no_zero_point, _mut_w4a8_sw_dropped,
              _mut_absdot_signed, _mut_tolerance_rel_dropped]
 
@@ -359,6 +364,35 @@ def test_sparse_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeyp
     test_prepack_sparse24_roundtrip(256, 200, 64)
     with pytest.raises(AssertionError):
         pin_sparse24_layout_golden(O)
+
+
+@pytest.mark.parametrize("K,N,g,frac4", [(128, 128, 128, 0.5), (256, 200, 64, 0.3), (384, 136, 32, 0.2),
+                                         (256, 40, 256, 0.5), (512, 8, 128, 1.0), (256, 136, 128, 0.0)])
+def test_prepack_mixed_roundtrip(K, N, g, frac4):
+    d = synth.w4a16_mixed_inputs(K, N, g, 1, seed=K + N + g, frac4=frac4)
+    Wp = O.prepack_mixed(d["Q"], d["s"], g, d["widths"])
+    assert Wp.nbytes == O.prepacked_bytes_mixed(K, N, g, d["widths"])
+    q, s, w = O.unprepack_mixed(Wp, K, N, g)
+    assert np.array_equal(q, d["q"]) and np.array_equal(w, d["widths"])
+    assert np.array_equal(s.view(np.uint16), d["s"].view(np.uint16))
+
+
+# Mixed layout mistakes made in both directions: the round trip passes, the offsets catch them.
+def _mut_mixed_field_halves_swapped(mp):
+    mp.setattr(O, "_mixed_field", lambda r, j: r // 2 + 8 * j + 4 * (r % 2))
+
+
+def _mut_mixed_table_padded_twice(mp):
+    mp.setattr(O, "_mixed_table_bytes", lambda nblob: ((nblob + 1) * 4 + 15) // 16 * 16 + 16)
+
+
+@pytest.mark.parametrize("mutate", [_mut_mixed_field_halves_swapped, _mut_mixed_table_padded_twice],
+                         ids=lambda f: f.__name__[5:])
+def test_mixed_layout_mistake_caught_only_by_the_golden_offsets(mutate, monkeypatch):
+    mutate(monkeypatch)
+    test_prepack_mixed_roundtrip(256, 200, 64, 0.3)
+    with pytest.raises(AssertionError):
+        pin_mixed_layout_golden(O)
 
 
 def test_package_reexports():
