@@ -22,6 +22,7 @@ __all__ = [
     "wq_prepacked_bytes_zp", "wq_prepack_zp", "wq_unpack_zp", "wq_gemm_w4a16_zp",
     "wq_prepack_act_order", "wq_permute_act", "wq_gemm_w4a16_act_order",
     "wq_prepacked_bytes_sparse24", "wq_prepack_sparse24", "wq_unpack_sparse24", "wq_gemm_w4a16_sparse24",
+    "wq_prepacked_bytes_mixed", "wq_prepack_mixed", "wq_unpack_mixed", "wq_gemm_w4a16_mixed",
     "wq_workspace_bytes", "wq_workspace_reserve", "wq_get_device_status", "wq_plan", "wq_plan_for",
     "wq_debug_set_wait_timeout_ns", "wq_debug_skip_publish",
     "WQ_OK", "WQ_ERR_INVALID_ARG", "WQ_ERR_UNSUPPORTED_SHAPE", "WQ_ERR_MISALIGNED",
@@ -78,6 +79,10 @@ def _load():
         "wq_prepack_sparse24": (I, [P, P, I, I, I, P, P]),
         "wq_unpack_sparse24": (I, [P, I, I, I, P, P, P]),
         "wq_gemm_w4a16_sparse24": (I, [P, P, P, I, I, I, I, P]),
+        "wq_prepacked_bytes_mixed": (Z, [I, I, I, ctypes.c_longlong]),
+        "wq_prepack_mixed": (I, [P, P, P, I, I, I, P, Z, P]),
+        "wq_unpack_mixed": (I, [P, I, I, I, P, P, P, P]),
+        "wq_gemm_w4a16_mixed": (I, [P, P, Z, P, I, I, I, I, P]),
         "wq_workspace_bytes": (Z, [I, I, I, I]),
         "wq_workspace_reserve": (I, [Z, P]),
         "wq_get_device_status": (I, [P]),
@@ -474,6 +479,71 @@ def wq_gemm_w4a16_sparse24(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y:
         Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
     _check(lib.wq_gemm_w4a16_sparse24(_ptr(A), _ptr(Wp), _ptr(Y), M, N, K, g, _stream(stream)),
            "wq_gemm_w4a16_sparse24")
+    return Y
+
+
+def wq_prepacked_bytes_mixed(K: int, N: int, g: int, n4: int) -> int:
+    return lib.wq_prepacked_bytes_mixed(K, N, g, n4)
+
+
+def wq_prepack_mixed(Q: torch.Tensor, s: torch.Tensor, widths: torch.Tensor, g: int, Wp: torch.Tensor | None = None,
+                     stream=None):
+    """Mixed 2/4-bit weights: Q int32 [K/8, N] (codes of 2-bit blocks 0..3), s fp16 [K/g, N],
+    widths uint8 [K/32, ceil(N/128)] of 2 or 4 -> the mixed buffer. Synchronises the stream."""
+    K8, N = _matrix(Q, "Q")
+    K = K8 * 8
+    _tensor(Q, torch.int32, "Q")
+    if g <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_prepack_mixed")
+    _tensor(s, torch.float16, "s", shape=(K // g, N))
+    _tensor(widths, torch.uint8, "widths", shape=(K // 32, -(-N // 128)))
+    _on_one_cuda_device(Q=Q, s=s, widths=widths, Wp=Wp)
+    nbytes = wq_prepacked_bytes_mixed(K, N, g, int((widths == 4).sum().item()))
+    if nbytes == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE if K % 128 == 0 else WQ_ERR_INVALID_ARG, "wq_prepack_mixed")
+    if Wp is not None:
+        _tensor(Wp, torch.uint8, "Wp", min_numel=nbytes)
+    else:
+        Wp = torch.empty(nbytes, dtype=torch.uint8, device=Q.device)
+    _check(lib.wq_prepack_mixed(_ptr(Q), _ptr(s), _ptr(widths), K, N, g, _ptr(Wp), Wp.numel(), _stream(stream)),
+           "wq_prepack_mixed")
+    return Wp
+
+
+def wq_unpack_mixed(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
+    """Inverse of wq_prepack_mixed: (Q int32 [K/8, N], s fp16 [K/g, N], widths uint8 [K/32, ceil(N/128)])."""
+    if g <= 0 or K <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_unpack_mixed")
+    least = wq_prepacked_bytes_mixed(K, N, g, 0)
+    if least == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_unpack_mixed")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=least)
+    _on_one_cuda_device(Wp=Wp)
+    Q = torch.empty((K // 8, N), dtype=torch.int32, device=Wp.device)
+    s = torch.empty((K // g, N), dtype=torch.float16, device=Wp.device)
+    widths = torch.empty((K // 32, -(-N // 128)), dtype=torch.uint8, device=Wp.device)
+    _check(lib.wq_unpack_mixed(_ptr(Wp), K, N, g, _ptr(Q), _ptr(s), _ptr(widths), _stream(stream)), "wq_unpack_mixed")
+    return Q, s, widths
+
+
+def wq_gemm_w4a16_mixed(A: torch.Tensor, Wp: torch.Tensor, N: int, g: int, Y: torch.Tensor | None = None,
+                        stream=None):
+    """Y fp16 [M, N] = A fp16 [M, K] . dequant(Wp) for a mixed 2/4-bit buffer, M <= 16."""
+    M, K = _matrix(A, "A")
+    _tensor(A, torch.float16, "A")
+    if g <= 0 or K % g:
+        raise WqError(WQ_ERR_INVALID_ARG, "wq_gemm_w4a16_mixed")
+    least = wq_prepacked_bytes_mixed(K, N, g, 0)
+    if least == 0:
+        raise WqError(WQ_ERR_UNSUPPORTED_SHAPE, "wq_gemm_w4a16_mixed")
+    _tensor(Wp, torch.uint8, "Wp", min_numel=least)
+    if Y is not None:
+        _tensor(Y, torch.float16, "Y", shape=(M, N))
+    _on_one_cuda_device(A=A, Wp=Wp, Y=Y)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=A.device)
+    _check(lib.wq_gemm_w4a16_mixed(_ptr(A), _ptr(Wp), Wp.numel(), _ptr(Y), M, N, K, g, _stream(stream)),
+           "wq_gemm_w4a16_mixed")
     return Y
 
 

@@ -145,20 +145,21 @@ size_t workspace_bytes_for(const Plan& pl) {
     return 4096 + static_cast<size_t>(pl.grid) * pl.tile_m * kTileN * 4;
 }
 
-// kind 0: W4A16; 1: W4A8; 3: W4A16 with a zero point per group (g < K); 5: 2:4 sparse W4A16
-// (M <= kRfMaxM).
+// kind 0: W4A16; 1: W4A8; 3: W4A16 with a zero point per group (g < K); 5: 2:4 sparse W4A16;
+// 6: mixed 2/4-bit W4A16 (5 and 6: M <= kRfMaxM).
 int plan_for(int kind, int M, int N, int K, int g, const DeviceState& d, Plan* pl) {
     int mode;
     int slots = 0;
-    if (kind == 0 || kind == 3 || kind == 5) {
+    if (kind == 0 || kind == 3 || kind == 5 || kind == 6) {
         slots = scale_slots(K, g);
         if (slots < 0 || (kind == 3 && slots == 0)) return WQ_ERR_INVALID_ARG;
         mode = kind == 3 ? kModeGroupZP : (slots > 0 ? kModeGroup : kModeChannel);
     } else {
         mode = kModeW4A8;
     }
-    if (kind == 5 && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if (make_plan(mode, M, N, K, slots, d.num_sms, d.smem_optin, pl, kind == 5) != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if ((kind == 5 || kind == 6) && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
+    const int fmt = kind == 5 ? 1 : (kind == 6 ? 2 : 0);
+    if (make_plan(mode, M, N, K, slots, d.num_sms, d.smem_optin, pl, fmt) != 0) return WQ_ERR_UNSUPPORTED_SHAPE;
     return WQ_OK;
 }
 
@@ -211,22 +212,24 @@ bool perm_grid_ok(int M, int K) {
     return static_cast<long long>(M) * ((K / 8 + 255) / 256) < (1LL << 31) - 1;
 }
 
-// The W4A16 (kind 0), W4A8 (kind 1), zero-point (kind 3) or 2:4 sparse W4A16 (kind 5) layer. A_fp16 (W4A8 only, may be
+// The W4A16 (kind 0), W4A8 (kind 1), zero-point (kind 3), 2:4 sparse (kind 5) or mixed 2/4-bit
+// (kind 6) layer. A_fp16 (W4A8 only, may be
 // null): fp16 activations that are first quantised per token into the workspace (the codes
 // replace A, the scales go to sa_out when given, else to the workspace). perm (kinds 0 and 3,
 // may be null): act order; A's columns are first gathered in the order perm into the
 // workspace, which then replaces A.
 int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y,
              int32_t* acc_out, int M, int N, int K, int g, cudaStream_t stream, const uint16_t* A_fp16 = nullptr,
-             float* sa_out = nullptr, int act_bits = 8, const int32_t* perm = nullptr) {
+             float* sa_out = nullptr, int act_bits = 8, const int32_t* perm = nullptr, size_t wp_bytes = 0) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M < 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if ((kind == 0 || kind == 3 || kind == 5) && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
+    if ((kind == 0 || kind == 3 || kind == 5 || kind == 6) && scale_slots(K, g) < 0) return WQ_ERR_INVALID_ARG;
     if (kind == 3 && scale_slots(K, g) == 0) return WQ_ERR_INVALID_ARG;
-    if (kind == 5 && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if ((kind == 5 || kind == 6) && M > kRfMaxM) return WQ_ERR_UNSUPPORTED_SHAPE;
     if (kind == 1 && K > kMaxKW4A8) return WQ_ERR_UNSUPPORTED_SHAPE;
+    if (kind == 6 && wp_bytes < wq_prepacked_bytes_mixed(K, N, g, 0)) return WQ_ERR_INVALID_ARG;
     if (!Wp) return WQ_ERR_INVALID_ARG;
     if (!aligned(Wp, 16)) return WQ_ERR_MISALIGNED;
     if (M == 0) return WQ_OK;
@@ -282,10 +285,13 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     GemmArgs a;
     std::memset(&a, 0, sizeof(a));
     a.wp = static_cast<const uint8_t*>(Wp);
-    a.s_chan = (pl.mode == kModeChannel)
-                   ? reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
-                                                       static_cast<size_t>(pl.n_tiles) * pl.k_blocks * pl.blob_bytes)
-                   : nullptr;
+    const long long nblob = static_cast<long long>(pl.n_tiles) * pl.k_blocks;
+    a.s_chan = (pl.mode != kModeChannel) ? nullptr
+               : reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(Wp) +
+                                                   (pl.mixed ? mixed_table_bytes(nblob)
+                                                             : static_cast<size_t>(nblob) * pl.blob_bytes));
+    a.mix_table = pl.mixed ? static_cast<const uint32_t*>(Wp) : nullptr;
+    a.wp_bytes = wp_bytes;
     a.sa = sa;
     a.sw = sw;
     a.y = Y;
@@ -304,7 +310,7 @@ int run_gemm(int kind, const void* A, const float* sa, const void* Wp, const flo
     a.chunk = pl.chunk;
     a.act_slot = pl.act_slot;
     a.blob_bytes = pl.blob_bytes;
-    a.group_rows = ((kind == 0 || kind == 3 || kind == 5) && g < kTileK) ? g : kTileK;
+    a.group_rows = ((kind == 0 || kind == 3 || kind == 5 || kind == 6) && g < kTileK) ? g : kTileK;
     a.small = pl.small ? 1 : 0;
     a.scale_in_dequant = scale_in_dequant(pl, g);
     a.zp_offset = (pl.mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16(scale_slots(K, g))) : 0;
@@ -411,7 +417,7 @@ const char* wq_status_string(int status) {
         case WQ_ERR_INVALID_ARG: return "WQ_ERR_INVALID_ARG: null pointer, negative size or unsupported group size";
         case WQ_ERR_UNSUPPORTED_SHAPE:
             return "WQ_ERR_UNSUPPORTED_SHAPE: K must be a multiple of 128, N a multiple of 8, M at most 2^24 "
-                   "(2:4 sparse weights: M at most 16)";
+                   "(2:4 sparse and mixed 2/4-bit weights: M at most 16)";
         case WQ_ERR_MISALIGNED: return "WQ_ERR_MISALIGNED: a pointer breaks the alignment rule";
         case WQ_ERR_UNSUPPORTED_DEVICE: return "WQ_ERR_UNSUPPORTED_DEVICE: needs compute capability 10.0 (sm_100a)";
         case WQ_ERR_CUDA: return "WQ_ERR_CUDA: a CUDA call or kernel launch failed";
@@ -696,6 +702,95 @@ int wq_gemm_w4a16_sparse24(const uint16_t* A, const void* Wp, uint16_t* Y, int M
     return run_gemm(5, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream));
 }
 
+size_t wq_prepacked_bytes_mixed(int K, int N, int g, long long n4) {
+    if (!shape_ok(K, N)) return 0;
+    const int slots = scale_slots(K, g);
+    if (slots < 0) return 0;
+    const long long nblob = static_cast<long long>(n_tiles(N)) * (K / kTileK);
+    if (n4 < 0 || n4 > 4 * nblob) return 0;
+    return mixed_table_bytes(nblob) + (slots ? 0 : channel_tail_bytes(N)) + static_cast<size_t>(4 * nblob + n4) * kMixBlock2 +
+           static_cast<size_t>(nblob) * 2 * kTileN * slots;
+}
+
+int wq_prepack_mixed(const int32_t* Q, const uint16_t* s, const uint8_t* widths, int K, int N, int g, void* Wp,
+                     size_t wp_bytes, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q, K, N, Wp, st);
+    if (rc) return rc;
+    const int slots = scale_slots(K, g);
+    if (slots < 0 || !s || !widths) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return WQ_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return WQ_ERR_CAPTURING;  // the widths are read on the host
+    const int KT = K / kTileK, NT = n_tiles(N);
+    const long long nblob = static_cast<long long>(NT) * KT;
+    std::vector<uint8_t> w(static_cast<size_t>(K / kMixBlockRows) * NT);
+    if (cudaMemcpyAsync(w.data(), widths, w.size(), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    // the blob table: each blob's offset (a prefix sum over the widths) and its widths
+    std::vector<uint32_t> table(static_cast<size_t>(nblob) + 1);
+    size_t pos = mixed_table_bytes(nblob) + (slots ? 0 : channel_tail_bytes(N));
+    for (int nt = 0; nt < NT; ++nt)
+        for (int kt = 0; kt < KT; ++kt) {
+            uint32_t wbits = 0;
+            for (int v = 0; v < 4; ++v) {
+                const uint8_t x = w[static_cast<size_t>(kt * 4 + v) * NT + nt];
+                if (x != 2 && x != 4) return WQ_ERR_INVALID_ARG;
+                if (x == 4) wbits |= 1u << v;
+            }
+            if (pos / 16 >= (1u << 28)) return WQ_ERR_UNSUPPORTED_SHAPE;  // 28 bits of offset per entry
+            table[static_cast<size_t>(nt) * KT + kt] = static_cast<uint32_t>(pos / 16) << 4 | wbits;
+            pos += static_cast<size_t>(kMixBlock2) * (4 + __builtin_popcount(wbits)) + 2 * kTileN * slots;
+        }
+    if (pos / 16 >= (1u << 28)) return WQ_ERR_UNSUPPORTED_SHAPE;
+    table[static_cast<size_t>(nblob)] = static_cast<uint32_t>(pos / 16) << 4;
+    if (pos > wp_bytes) return WQ_ERR_INVALID_ARG;  // the caller's buffer is smaller than the format needs
+    int bad = 0;
+    if (cudaMemcpyAsync(Wp, table.data(), table.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemsetAsync(d->check, 0, sizeof(int), st) != cudaSuccess ||
+        launch_prepack_mixed(Q, s, K, N, g, Wp, d->check, st) != 0 ||
+        cudaMemcpyAsync(&bad, d->check, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return bad ? WQ_ERR_INVALID_ARG : WQ_OK;
+}
+
+int wq_unpack_mixed(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, uint8_t* widths_out,
+                    void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = prepack_common_checks(Q_out, K, N, Wp, st);
+    if (rc) return rc;
+    if (scale_slots(K, g) < 0 || !s_out || !widths_out) return WQ_ERR_INVALID_ARG;
+    if (!aligned(s_out, 16)) return WQ_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    int dev = 0;
+    DeviceState* d = nullptr;
+    rc = require_device(&dev, &d, st, true);
+    if (rc) return rc;
+    if (launch_unpack_mixed(Wp, K, N, g, Q_out, s_out, widths_out, st) != 0) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
+    return WQ_OK;
+}
+
+int wq_gemm_w4a16_mixed(const uint16_t* A, const void* Wp, size_t wp_bytes, uint16_t* Y, int M, int N, int K, int g,
+                        void* stream) {
+    return run_gemm(6, A, nullptr, Wp, nullptr, Y, nullptr, M, N, K, g, static_cast<cudaStream_t>(stream), nullptr,
+                    nullptr, 8, nullptr, wp_bytes);
+}
+
 int wq_gemm_w4a8(const int8_t* A, const float* sa, const void* Wp, const float* sw, uint16_t* Y, int32_t* acc_out,
                  int M, int N, int K, void* stream) {
     return run_gemm(1, A, sa, Wp, sw, Y, acc_out, M, N, K, K, static_cast<cudaStream_t>(stream));
@@ -728,14 +823,14 @@ int wq_gemm_w4a8_fp16act(const uint16_t* A, const void* Wp, const float* sw, uin
 }
 
 size_t wq_workspace_bytes(int kind, int M, int N, int K) {
-    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 5) return 0;
-    if (kind == 5 && M > kRfMaxM) return 0;
+    if (!shape_ok(K, N) || M <= 0 || kind < 0 || kind > 6) return 0;
+    if ((kind == 5 || kind == 6) && M > kRfMaxM) return 0;
     std::lock_guard<std::mutex> lock(g_mu);
     int dev = 0;
     DeviceState* d = device_state(&dev);
     if (!d || !d->supported) return 0;
     Plan pl;
-    const bool w4a16 = kind == 0 || kind == 3 || kind == 4 || kind == 5;  // these plan like the W4A16 layer
+    const bool w4a16 = kind == 0 || kind >= 3;  // these plan like the W4A16 layer
     if (plan_for(w4a16 ? 0 : 1, M, N, K, w4a16 ? kTileK : K, *d, &pl) != WQ_OK) return 0;
     if (kind == 2) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_quant_bytes(M, K);
     if (kind == 4) return (workspace_bytes_for(pl) + 255) / 256 * 256 + act_perm_bytes(M, K);
@@ -794,7 +889,7 @@ int fill_plan(int kind, int M, int N, int K, int g, int num_sms, int smem_optin,
     if (rc) return rc;
     if (M <= 0) return WQ_ERR_INVALID_ARG;
     if (M > (1 << 24)) return WQ_ERR_UNSUPPORTED_SHAPE;
-    if (kind != 0 && kind != 1 && kind != 5) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1 && kind != 5 && kind != 6) return WQ_ERR_INVALID_ARG;
     if (num_sms <= 0 || smem_optin <= 0) return WQ_ERR_INVALID_ARG;
     DeviceState d;
     d.num_sms = num_sms;
@@ -820,7 +915,7 @@ int wq_plan(int kind, int M, int N, int K, int g, wq_plan_t* plan) {
     int rc = check_shape(K, N);
     if (rc) return rc;
     if (M <= 0) return WQ_ERR_INVALID_ARG;
-    if (kind != 0 && kind != 1 && kind != 5) return WQ_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1 && kind != 5 && kind != 6) return WQ_ERR_INVALID_ARG;
     int num_sms = 0, smem_optin = 0;
     {
         std::lock_guard<std::mutex> lock(g_mu);

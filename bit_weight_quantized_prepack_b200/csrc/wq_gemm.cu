@@ -71,6 +71,7 @@ struct Barriers {
     uint64_t aempty[kASlotsS];     // MMAs done with a tensor-memory slot
     uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
     uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
+    uint32_t wbits[kMaxSlots];     // mixed 2/4-bit: the widths of the blob in each weight slot
 };
 
 struct Ctl {
@@ -485,7 +486,7 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
 }
 
 // Weight producer (kWeightWarp, one thread) or activation producer (kActWarp, one thread).
-template <int MODE, bool kWeights>
+template <int MODE, bool kWeights, bool kMix = false>
 __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* aring, uint8_t* wring, Barriers& b,
                               const Ctl& ctl, long long beg, long long end) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
@@ -513,7 +514,37 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
             }
             if (ok) {
                 uint64_t* fbar = &b.full[cb.bar];
-                if (kWeights) {
+                if (kWeights && kMix) {
+                    // blobs of varying size: offsets and widths from the table, one copy per blob
+                    // into its fixed-stride slot; the widths reach the consumers through the
+                    // slot's word, ordered before them by this thread's arrival (release). A table
+                    // that does not describe this format inside the caller's buffer stops the CTA
+                    // with WQ_ERR_INVALID_ARG before any copy of that chunk.
+                    const uint32_t* te = p.mix_table + static_cast<size_t>(nt) * p.k_blocks + kb;
+                    uint32_t e[kMaxChunk + 1];
+                    for (int t = 0; t <= c; ++t) e[t] = __ldg(te + t);
+                    uint32_t bytes = 0;
+                    bool valid = true;
+                    for (int t = 0; t < c; ++t) {
+                        const unsigned long long lo = (e[t] >> 4) * 16ull, hi = (e[t + 1] >> 4) * 16ull;
+                        const unsigned long long want =
+                            static_cast<unsigned long long>(kMixBlock2) * (4 + __popc(e[t] & 0xFu)) + (p.blob_bytes - kCodeBytes);
+                        valid = valid && hi > lo && hi - lo == want && hi <= p.wp_bytes;
+                        bytes += static_cast<uint32_t>(want);
+                    }
+                    if (!valid) {  // no copy; the arrival lets the chunk's phase complete with the activations
+                        raise_error(ctl, WQ_ERR_INVALID_ARG);
+                        ok = false;
+                        mbar_arrive(fbar);
+                    } else {
+                        for (int t = 0; t < c; ++t) b.wbits[pos + t] = e[t] & 0xFu;
+                        mbar_arrive_expect_tx(fbar, bytes);
+                        for (int t = 0; t < c; ++t)
+                            bulk_g2s(wring + static_cast<size_t>(pos + t) * p.blob_bytes,
+                                     p.wp + static_cast<size_t>(e[t] >> 4) * 16, ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u,
+                                     fbar, policy);
+                    }
+                } else if (kWeights) {
                     mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(c * p.blob_bytes));
                     bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes,
                              wtile + static_cast<size_t>(kb) * p.blob_bytes, static_cast<uint32_t>(c * p.blob_bytes),
@@ -616,7 +647,13 @@ __device__ __forceinline__ uint8_t* align_ring(uint8_t* smem_dyn) {
 // (A prefetch only fills L2, the point of coherence: it cannot observe stale data.)
 constexpr int kPrefetchBlobs = 24;
 
+template <bool kMix = false>
 __device__ void prefetch_first_blobs(const GemmArgs& p, long long beg, long long end) {
+    if (kMix) {  // blobs of varying size: the CTA's table entries (16-byte aligned, inside the table)
+        const long long lo = (beg * 4) & ~15ll, hi = ((end + 1) * 4 + 15) & ~15ll;
+        if (hi > lo) prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(p.mix_table) + lo, static_cast<uint32_t>(hi - lo));
+        return;
+    }
     SegCursor seg(beg, end, p.k_blocks);
     int left = kPrefetchBlobs;
     while (left > 0 && seg.next()) {
@@ -1393,18 +1430,65 @@ __device__ __forceinline__ void rf_sp_mma_block(uint32_t x, uint32_t e, __half2 
     for (int nb = 0; nb < NB; ++nb) mma_sp_m16n8k32_f16_f32(d[nb], a, bf[nb], e);
 }
 
+// Mixed 2/4-bit weights, a 2-bit block: lane (g, q) holds in one word the 2-bit codes of rows
+// 8q .. 8q + 7 of columns g and g + 8 of its row tile, the fp16 pair (rows 8q + 2s, + 1) of
+// column g in fields (s, s + 8) and of column g + 8 in fields (s + 4, s + 12). Field pair P
+// (0..3) of a word y (the word, or the word shifted right by 8 for column g + 8): masking
+// (3 << 2P) in each 16-bit half and OR-ing 0x6400 gives 1024 + 4^P q exactly, and
+// u * 4^-P - (1024 / 4^P + 2) is q - 2 exactly (one fused multiply-add).
+template <int P, bool kScaled>
+__device__ __forceinline__ uint32_t pair2_f16(uint32_t y, __half2 sc) {
+    const uint32_t u = lop3_and_or(y, (0x3u << (2 * P)) * 0x10001u, 0x64006400u);
+    __half2 h;
+    if constexpr (P == 0) {
+        h = __hsub2(half2_bits(u), half2_bits(0x64026402u));  // - 1026
+    } else {
+        constexpr uint32_t kMul = P == 1 ? 0x34003400u : (P == 2 ? 0x2C002C00u : 0x24002400u);  // 1/4, 1/16, 1/64
+        constexpr uint32_t kAdd = P == 1 ? 0xDC08DC08u : (P == 2 ? 0xD420D420u : 0xCC80CC80u);  // -258, -66, -18
+        h = __hfma2(half2_bits(u), half2_bits(kMul), half2_bits(kAdd));
+    }
+    if constexpr (kScaled) h = __hmul2(h, sc);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// The two MMAs of one row tile and one 32-row 2-bit block: MMA t takes pairs 2t, 2t + 1 of both
+// columns, the same k order as the 4-bit path, so the B fragments are the same registers.
+template <bool kScaled, int NB>
+__device__ __forceinline__ void rf_mma_block_2b(uint32_t x, __half2 sc0, __half2 sc1, const uint4 (&act)[NB],
+                                                float (&d)[NB][4]) {
+    const uint32_t x8 = x >> 8;
+    {
+        const uint32_t afrag[4] = {pair2_f16<0, kScaled>(x, sc0), pair2_f16<0, kScaled>(x8, sc1),
+                                   pair2_f16<1, kScaled>(x, sc0), pair2_f16<1, kScaled>(x8, sc1)};
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_m16n8k16_f16_f32(d[nb], afrag, act[nb].x, act[nb].y);
+    }
+    {
+        const uint32_t afrag[4] = {pair2_f16<2, kScaled>(x, sc0), pair2_f16<2, kScaled>(x8, sc1),
+                                   pair2_f16<3, kScaled>(x, sc0), pair2_f16<3, kScaled>(x8, sc1)};
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) mma_m16n8k16_f16_f32(d[nb], afrag, act[nb].z, act[nb].w);
+    }
+}
+
+// Formats of the register-operand kernel's weights.
+enum RfFmt : int { kFmtDense = 0, kFmtSparse = 1, kFmtMixed = 2 };
+
 // Consumer warp of a register-operand tile (warps 0..15): residue r = warp / 4 takes the walk's
 // k-blocks i with i mod 4 = r; column group cg = warp mod 4 owns columns 32 cg .. 32 cg + 31
 // of every such k-block, all 128 rows. Lane (g, q) handles two MMA row tiles (columns
 // 32 cg + 16 tau + g and + 8, tau = 0, 1) in each of the four 32-row blocks.
 // red: 4 x TM x 128 floats of shared memory (residue, row, column).
-// SP: 2:4 sparse blobs. Lane (g, q) then reads, per 32-row block and row tile, one code word
-// and one metadata word, and the activation slot holds AR = max(TM, 8) rows in the 128-byte
-// swizzled layout of the copy engine (16-byte chunk c of row m at chunk c ^ (m mod 8)), so
-// that the eight rows of each 8 x 8 matrix of an ldmatrix fall in eight different banks.
-template <int MODE, int TM, int SCALE, bool SP>
+// FMT kFmtSparse: 2:4 sparse blobs. Lane (g, q) then reads, per 32-row block and row tile, one
+// code word and one metadata word, and the activation slot holds AR = max(TM, 8) rows in the
+// 128-byte swizzled layout of the copy engine (16-byte chunk c of row m at chunk c ^ (m mod 8)),
+// so that the eight rows of each 8 x 8 matrix of an ldmatrix fall in eight different banks.
+// FMT kFmtMixed: mixed 2/4-bit blobs; the slot's widths word says which 32-row blocks are 4-bit
+// (read as in a W4A16 blob) and which 2-bit (one word per row tile and lane).
+template <int MODE, int TM, int SCALE, int FMT>
 __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* wring, Barriers& b, float* red,
                         const Ctl& ctl, long long beg, long long end) {
+    constexpr bool SP = FMT == kFmtSparse, MIX = FMT == kFmtMixed;
     constexpr int NB = (TM + 7) / 8;  // MMAs of 8 activation rows per k-step
     constexpr int AR = (SP && TM < kSpMinActRows) ? kSpMinActRows : TM;  // activation rows per slot piece
     constexpr bool kScaled = SCALE == kRfScaleWeight;
@@ -1454,7 +1538,9 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             if (!ok) continue;  // an expired wait: the CTA winds down (nothing more is read or released)
             const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
             const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
-            const uint16_t* scs = reinterpret_cast<const uint16_t*>(blob + (SP ? kSpHeadBytes : kCodeBytes));
+            const uint32_t wb = MIX ? (b.wbits[s] & 0xFu) : 0xFu;  // mixed: bit v set = block v is 4-bit
+            const uint16_t* scs = reinterpret_cast<const uint16_t*>(
+                blob + (SP ? kSpHeadBytes : (MIX ? kMixBlock2 * (4 + __popc(wb)) : kCodeBytes)));
             const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;
             uint32_t w[4][2][2];  // [block hv][tau][j]: word q of column colb + 16 tau + 8 j
                                   // SP: [hv][tau][0] code word, [hv][tau][1] metadata word of row tile 2 cg + tau
@@ -1466,6 +1552,15 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                         const int tile16 = hv * 8 + 2 * cg + tau;
                         w[hv][tau][0] = words[tile16 * 32 + lane];
                         w[hv][tau][1] = words[kSpCodeBytes / 4 + tile16 * 16 + 2 * g + (q & 1)];
+                    } else if constexpr (MIX) {
+                        const uint32_t* blk = words + (kMixBlock2 / 4) * (hv + __popc(wb & ((1u << hv) - 1u)));
+                        if ((wb >> hv) & 1u) {
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) w[hv][tau][j] = blk[(colb + 16 * tau + 8 * j) * 4 + q];
+                        } else {
+                            w[hv][tau][0] = blk[(2 * cg + tau) * 32 + lane];
+                            w[hv][tau][1] = 0u;
+                        }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 2; ++j) w[hv][tau][j] = words[(hv * kTileN + colb + 16 * tau + 8 * j) * 4 + q];
@@ -1550,6 +1645,8 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
                     float (&dst)[NB][4] = (SCALE == kRfScalePair || SCALE == kRfScaleBlock) ? part[tau] : acc[tau];
                     if constexpr (SP)
                         rf_sp_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], sc[tau][0], sc[tau][1], bf, dst);
+                    else if (MIX && !((wb >> hv) & 1u))
+                        rf_mma_block_2b<kScaled, NB>(w[hv][tau][0], sc[tau][0], sc[tau][1], a16, dst);
                     else
                         rf_mma_block<kScaled, NB>(w[hv][tau][0], w[hv][tau][1], klo[tau][0], khi[tau][0], klo[tau][1],
                                                   khi[tau][1], sc[tau][0], sc[tau][1], a16, dst);
@@ -1618,7 +1715,7 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
     }
 }
 
-template <int MODE, int TM, bool SP = false>
+template <int MODE, int TM, int FMT = kFmtDense>
 __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constant__ ActMaps maps, const GemmArgs p) {
     extern __shared__ uint8_t smem_dyn[];
     __shared__ Barriers bars;
@@ -1632,7 +1729,7 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
     const long long end = unit_start(blockIdx.x + 1, p.units, p.grid);
     if (threadIdx.x == 0) griddep_launch_dependents();
-    if (warp == kWeightWarpR && lane == 0) prefetch_first_blobs(p, beg, end);
+    if (warp == kWeightWarpR && lane == 0) prefetch_first_blobs<FMT == kFmtMixed>(p, beg, end);
     if (warp == 0) {
         for (int k = lane; k < kChunkBars; k += 32) mbar_init(&bars.full[k], 2);
         for (int s = lane; s < p.slots; s += 32) {
@@ -1650,16 +1747,16 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
     if (warp < kRfWarps) {
         if constexpr (is_group(MODE)) {
             if (p.scale_in_dequant)
-                rf_role<MODE, TM, kRfScaleWeight, SP>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScaleWeight, FMT>(p, aring, wring, bars, red, ctl, beg, end);
             else if (p.group_rows < kTileK)
-                rf_role<MODE, TM, kRfScalePair, SP>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScalePair, FMT>(p, aring, wring, bars, red, ctl, beg, end);
             else
-                rf_role<MODE, TM, kRfScaleBlock, SP>(p, aring, wring, bars, red, ctl, beg, end);
+                rf_role<MODE, TM, kRfScaleBlock, FMT>(p, aring, wring, bars, red, ctl, beg, end);
         } else {
-            rf_role<MODE, TM, kRfScaleNone, SP>(p, aring, wring, bars, red, ctl, beg, end);
+            rf_role<MODE, TM, kRfScaleNone, FMT>(p, aring, wring, bars, red, ctl, beg, end);
         }
     } else if (warp == kWeightWarpR) {
-        if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
+        if (lane == 0) producer_role<MODE, true, FMT == kFmtMixed>(&maps, p, aring, wring, bars, ctl, beg, end);
     } else {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     }
@@ -1669,12 +1766,14 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
 // Bytes of the register-operand kernel's residue sums (after the ring in dynamic shared memory).
 static int rf_red_bytes(int tm) { return 4 * tm * kTileN * 4; }
 
-int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl, bool sparse) {
+int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* pl, int fmt) {
     pl->mode = mode;
     pl->k_blocks = K / kTileK;
     pl->n_tiles = n_tiles(N);
+    const bool sparse = fmt == kFmtSparse;
     pl->sparse = sparse;
-    if (sparse && (M > kRfMaxM || (mode != kModeGroup && mode != kModeChannel))) return -1;
+    pl->mixed = fmt == kFmtMixed;  // slots sized for the largest blob: every block 4-bit
+    if (fmt != kFmtDense && (M > kRfMaxM || (mode != kModeGroup && mode != kModeChannel))) return -1;
     pl->blob_bytes = sparse                   ? static_cast<int>(blob_bytes_sp24(slots))
                      : (mode == kModeGroup)   ? static_cast<int>(blob_bytes_w4a16(slots))
                      : (mode == kModeGroupZP) ? static_cast<int>(blob_bytes_w4a16_zp(slots))
@@ -1767,16 +1866,26 @@ cudaError_t configure_gemm_kernels(int max_dynamic_smem) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroupZP, 16>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeW4A8, 16>, max_dynamic_smem);
     }
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 4, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 1, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 2, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 4, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8, true>, max_dynamic_smem);
-    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16, true>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 4, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 1, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 2, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 4, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16, kFmtSparse>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 1, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 2, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 4, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 8, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 16, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 1, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 2, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 4, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 8, kFmtMixed>, max_dynamic_smem);
+    if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 16, kFmtMixed>, max_dynamic_smem);
     if constexpr (kRfMaxM > 16) {
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeGroup, 32>, max_dynamic_smem);
         if (e == cudaSuccess) e = allow_smem(wq_gemm_rf<kModeChannel, 32>, max_dynamic_smem);
@@ -1813,15 +1922,25 @@ static cudaError_t launch_mode(const ActMaps& maps, const GemmArgs& args, const 
     {
         if (plan.rf && plan.sparse) {
             if constexpr (MODE == kModeGroup || MODE == kModeChannel) {
-                if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1, true>, maps, args, plan, st);
-                if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2, true>, maps, args, plan, st);
-                if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4, true>, maps, args, plan, st);
-                if (plan.tile_m == 8) return launch_kernel(wq_gemm_rf<MODE, 8, true>, maps, args, plan, st);
-                if (plan.tile_m == 16) return launch_kernel(wq_gemm_rf<MODE, 16, true>, maps, args, plan, st);
+                if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1, kFmtSparse>, maps, args, plan, st);
+                if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2, kFmtSparse>, maps, args, plan, st);
+                if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4, kFmtSparse>, maps, args, plan, st);
+                if (plan.tile_m == 8) return launch_kernel(wq_gemm_rf<MODE, 8, kFmtSparse>, maps, args, plan, st);
+                if (plan.tile_m == 16) return launch_kernel(wq_gemm_rf<MODE, 16, kFmtSparse>, maps, args, plan, st);
             }
             return cudaErrorInvalidConfiguration;
         }
-        if (plan.sparse) return cudaErrorInvalidConfiguration;
+        if (plan.rf && plan.mixed) {
+            if constexpr (MODE == kModeGroup || MODE == kModeChannel) {
+                if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1, kFmtMixed>, maps, args, plan, st);
+                if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2, kFmtMixed>, maps, args, plan, st);
+                if (plan.tile_m == 4) return launch_kernel(wq_gemm_rf<MODE, 4, kFmtMixed>, maps, args, plan, st);
+                if (plan.tile_m == 8) return launch_kernel(wq_gemm_rf<MODE, 8, kFmtMixed>, maps, args, plan, st);
+                if (plan.tile_m == 16) return launch_kernel(wq_gemm_rf<MODE, 16, kFmtMixed>, maps, args, plan, st);
+            }
+            return cudaErrorInvalidConfiguration;
+        }
+        if (plan.sparse || plan.mixed) return cudaErrorInvalidConfiguration;
         if (plan.rf) {
             if (plan.tile_m == 1) return launch_kernel(wq_gemm_rf<MODE, 1>, maps, args, plan, st);
             if (plan.tile_m == 2) return launch_kernel(wq_gemm_rf<MODE, 2>, maps, args, plan, st);

@@ -31,6 +31,8 @@ struct GemmArgs {
     int small;                 // 1: per-k-block partials summed by the dequant warps (tile_m <= 32)
     int scale_in_dequant;      // 1: the dequant multiplies by the group scale (fp16 weights)
     int zp_offset;             // asymmetric groups: byte offset of the zero points within a blob
+    const uint32_t* mix_table; // mixed 2/4-bit: the blob table at the start of wp (null otherwise)
+    unsigned long long wp_bytes;  // mixed 2/4-bit: bytes of the caller's buffer (copies stay inside)
     long long units;           // tiles * k_blocks
     int grid;
     unsigned long long timeout_ns;
@@ -50,11 +52,12 @@ struct Plan {
     bool small;
     bool rf;    // M <= kRfMaxM: the register-operand kernel, unswizzled activation slots
     bool sparse;   // 2:4 sparse weights (register-operand kernel only; swizzled activation slots)
+    bool mixed;    // mixed 2/4-bit weights (register-operand kernel only; blobs of varying size)
     int act_rows;  // rows of one activation copy: tile_m, or at least kSpMinActRows when sparse
 };
 
-int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan,
-              bool sparse = false);
+// fmt: 0 dense, 1 2:4 sparse, 2 mixed 2/4-bit (the last two only for M <= kRfMaxM)
+int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_optin, Plan* plan, int fmt = 0);
 
 cudaError_t configure_gemm_kernels(int max_dynamic_smem);
 
@@ -69,6 +72,8 @@ int launch_unpack_w4a8(const void* Wp, int K, int N, int32_t* Q, cudaStream_t st
 int launch_prepack_sp24(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, int* bad,
                         cudaStream_t st);
 int launch_unpack_sp24(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, cudaStream_t st);
+int launch_prepack_mixed(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, int* bad, cudaStream_t st);
+int launch_unpack_mixed(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* widths, cudaStream_t st);
 int launch_quantize_act(const uint16_t* A, int M, int K, int bits, int8_t* Aq, float* sa, cudaStream_t st);
 int launch_permute_codes(const int32_t* Q, const int32_t* perm, int K, int N, int32_t* Qp, cudaStream_t st);
 int launch_permute_act(const uint16_t* A, const int32_t* perm, int M, int K, uint16_t* Ap, int* status,

@@ -31,6 +31,19 @@
 //   other rows. Code word 32*(b*8 + rt) + lane is exactly lane's A operand of the sparse warp
 //   MMA (m16n8k32, groups of 4 along k) for that row tile and block, and metadata word
 //   16*(b*8 + rt) + lane / 2 its metadata operand (lanes 4gc, 4gc + 1).
+// Prepacked mixed 2/4-bit W4A16 buffer (a bit width per aligned block of 32 rows x 128
+//   columns; a b-bit code q stands for q - 2^(b-1)):
+//   a table of NT*KT + 1 uint32 entries (padded to 16 bytes): entry nt*KT + kt =
+//     (byte offset of blob (nt, kt) / 16) << 4 | wbits (bit v set: 32-row block v is 4-bit),
+//     the last entry (end of the blobs / 16) << 4;
+//   for g == K, NT*128 fp16 column scales right after the table (padded to 16 bytes);
+//   then the blobs, nt-major: for v = 0..3 the block of rows 32v .. 32v + 31, either 2048
+//   bytes of 4-bit words laid out as block v of a W4A16 blob (word r*4 + i: rows 32v + 8i +
+//   j of column r, nibble kNibblePos[j]) or 1024 bytes of 2-bit words (word rt*32 + 4gc + t:
+//   rows 32v + 8t + r of columns 16rt + gc + 8j, 2-bit field r/2 + 4j + 8(r%2)), then the
+//   `slots` rows of fp16 scales. Word rt*32 + lane of a 2-bit block is exactly what lane
+//   (gc, t) of a warp multiplies for row tile rt: its fields (p, p + 8) are the fp16 pairs of
+//   rows 8t + 2s, 8t + 2s + 1 of column 16rt + gc + 8j for p = s + 4j.
 //
 // Nibble orders. Within a word the W4A16 order puts codes (2p, 2p+1) at nibble positions
 // (p, p+4) for p = 0..3, so that masking 0x000F000F (p = 0) or 0x00F000F0 (p = 1) of the
@@ -82,6 +95,10 @@ constexpr int kSpMetaBytes = 2048;           // then 2-bit positions of the kept
 constexpr int kSpHeadBytes = kSpCodeBytes + kSpMetaBytes;  // the scale rows start here
 constexpr int kSpMinActRows = 8;             // sparse: activation rows per slot (one 128-byte swizzle atom)
 
+constexpr int kMixBlockRows = 32;            // mixed 2/4-bit: rows per width block
+constexpr int kMixBlock2 = 1024;             // bytes of a 2-bit block (128 columns x 32 rows)
+constexpr int kMixBlock4 = 2048;             // bytes of a 4-bit block
+
 enum Mode : int { kModeGroup = 0, kModeChannel = 1, kModeW4A8 = 2, kModeGroupZP = 3 };
 
 // Scale rows per blob for W4A16; 0 means per-column scales (g == K); -1 unsupported.
@@ -104,6 +121,9 @@ inline size_t blob_bytes_w4a16_zp(int slots) { return blob_bytes_w4a16(slots) + 
 
 // 2:4 sparse W4A16: code and metadata words, then `slots` rows of 128 fp16 scales.
 inline size_t blob_bytes_sp24(int slots) { return kSpHeadBytes + 2u * kTileN * static_cast<size_t>(slots); }
+
+// Mixed 2/4-bit: bytes of the blob table (NT*KT + 1 uint32 entries, padded to 16 bytes).
+inline size_t mixed_table_bytes(long long nblob) { return (static_cast<size_t>(nblob + 1) * 4 + 15) / 16 * 16; }
 
 inline size_t channel_tail_bytes(int N) { return ((2u * n_tiles(N) * kTileN) + 15u) / 16u * 16u; }
 

@@ -338,4 +338,169 @@ int launch_unpack_sp24(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
+// ------------------------------------------------------------------ mixed 2/4-bit weights
+// The blob table at the start of the buffer is written by the host first (offsets are a
+// prefix sum over the widths); these kernels read it for each blob's offset and widths.
+__device__ __forceinline__ int mixed_block_offset(uint32_t wbits, int v) {
+    return kMixBlock2 * (v + __popc(wbits & ((1u << v) - 1u)));
+}
+
+// 2-bit field of row 8t + r of column 16rt + gc + 8j within the word of lane (gc, t).
+__device__ __forceinline__ int mixed_field(int r, int j) { return (r >> 1) + 4 * j + 8 * (r & 1); }
+
+// One thread per (blob, block v, r < 128). A 4-bit block: the four words of column r, as in a
+// W4A16 blob. A 2-bit block: words r and r + 128 of the block (word w = rt*32 + 4gc + t covers
+// columns 16rt + gc and + 8, rows 8t .. 8t + 7). A code above 3 in a 2-bit block sets *bad.
+// Padded columns hold the block's zero point (8 or 2): weight 0.
+__global__ void prepack_mixed_codes_kernel(const uint32_t* __restrict__ Q, int N, int KT, long long total,
+                                           uint8_t* __restrict__ wp, int* __restrict__ bad) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int v = static_cast<int>((idx / kTileN) % 4);
+    const long long blob = idx / (4 * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const uint32_t e = reinterpret_cast<const uint32_t*>(wp)[blob];
+    uint8_t* block = wp + static_cast<size_t>(e >> 4) * 16 + mixed_block_offset(e & 0xFu, v);
+    if ((e >> v) & 1u) {
+        const long long n = nt * kTileN + r;
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const long long row = static_cast<long long>(kt) * 16 + v * 4 + i;  // row of Q (8 codes)
+            w[i] = (n < N) ? permute_word<false>(__ldg(Q + row * N + n)) : 0x88888888u;
+        }
+        *reinterpret_cast<uint4*>(block + static_cast<size_t>(r) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        return;
+    }
+    bool over = false;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int wi = r + h * kTileN;
+        const int rt = wi >> 5, gc = (wi >> 2) & 7, t = wi & 3;
+        const long long row = static_cast<long long>(kt) * 16 + v * 4 + t;  // rows 32v + 8t .. + 7
+        uint32_t out = 0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const long long n = nt * kTileN + 16 * rt + gc + 8 * j;
+            const uint32_t src = (n < N) ? __ldg(Q + row * N + n) : 0x22222222u;
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) {
+                const uint32_t c = (src >> (4 * rr)) & 0xFu;
+                over = over || c > 3u;
+                out |= (c & 3u) << (2 * mixed_field(rr, j));
+            }
+        }
+        reinterpret_cast<uint32_t*>(block)[wi] = out;
+    }
+    if (over) *bad = 1;
+}
+
+// One thread per (blob, slot, r): the group scale of column r after the blob's code blocks.
+__global__ void prepack_mixed_scales_kernel(const uint16_t* __restrict__ s, int N, int KT, int g, int slots,
+                                            long long total, uint8_t* __restrict__ wp) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int u = static_cast<int>((idx / kTileN) % slots);
+    const long long blob = idx / (static_cast<long long>(slots) * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const long long n = nt * kTileN + r;
+    const uint32_t e = reinterpret_cast<const uint32_t*>(wp)[blob];
+    const long long grp = (static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g) / g;
+    uint16_t* sc = reinterpret_cast<uint16_t*>(wp + static_cast<size_t>(e >> 4) * 16 + mixed_block_offset(e & 0xFu, 4));
+    sc[u * kTileN + r] = (n < N) ? s[grp * N + n] : static_cast<uint16_t>(0);
+}
+
+// Inverse (a test aid): one thread per (blob, block v, r): the Q words of column r in block v and
+// (r == 0) the block's width.
+__global__ void unpack_mixed_codes_kernel(const uint8_t* __restrict__ wp, int N, int KT, int NT, long long total,
+                                          uint32_t* __restrict__ Q, uint8_t* __restrict__ widths) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int v = static_cast<int>((idx / kTileN) % 4);
+    const long long blob = idx / (4 * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const uint32_t e = reinterpret_cast<const uint32_t*>(wp)[blob];
+    const bool four = (e >> v) & 1u;
+    if (r == 0) widths[(static_cast<long long>(kt) * 4 + v) * NT + nt] = four ? 4 : 2;
+    const long long n = nt * kTileN + r;
+    if (n >= N) return;
+    const uint8_t* block = wp + static_cast<size_t>(e >> 4) * 16 + mixed_block_offset(e & 0xFu, v);
+    const int rt = r >> 4, j = (r >> 3) & 1, gc = r & 7;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t out;
+        if (four) {
+            out = unpermute_word<false>(reinterpret_cast<const uint32_t*>(block)[r * 4 + i]);
+        } else {
+            const uint32_t x = reinterpret_cast<const uint32_t*>(block)[rt * 32 + 4 * gc + i];
+            out = 0;
+#pragma unroll
+            for (int rr = 0; rr < 8; ++rr) out |= ((x >> (2 * mixed_field(rr, j))) & 3u) << (4 * rr);
+        }
+        Q[(static_cast<long long>(kt) * 16 + v * 4 + i) * N + n] = out;
+    }
+}
+
+__global__ void unpack_mixed_scales_kernel(const uint8_t* __restrict__ wp, int N, int KT, int g, int slots,
+                                           long long total, uint16_t* __restrict__ s) {
+    const long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    if (idx >= total) return;
+    const int r = static_cast<int>(idx % kTileN);
+    const int u = static_cast<int>((idx / kTileN) % slots);
+    const long long blob = idx / (static_cast<long long>(slots) * kTileN);
+    const int kt = static_cast<int>(blob % KT);
+    const long long nt = blob / KT;
+    const long long n = nt * kTileN + r;
+    const long long row0 = static_cast<long long>(kt) * kTileK + static_cast<long long>(u) * g;
+    if (n >= N || row0 % g != 0) return;
+    const uint32_t e = reinterpret_cast<const uint32_t*>(wp)[blob];
+    s[(row0 / g) * N + n] = reinterpret_cast<const uint16_t*>(
+        wp + static_cast<size_t>(e >> 4) * 16 + mixed_block_offset(e & 0xFu, 4))[u * kTileN + r];
+}
+
+int launch_prepack_mixed(const int32_t* Q, const uint16_t* s, int K, int N, int g, void* Wp, int* bad,
+                         cudaStream_t st) {
+    const int slots = scale_slots(K, g);
+    const int KT = K / kTileK, NT = n_tiles(N);
+    uint8_t* wp = static_cast<uint8_t*>(Wp);
+    const long long nblob = static_cast<long long>(NT) * KT;
+    const long long tc = nblob * 4 * kTileN;
+    prepack_mixed_codes_kernel<<<blocks_for(tc, 256), 256, 0, st>>>(reinterpret_cast<const uint32_t*>(Q), N, KT, tc,
+                                                                     wp, bad);
+    if (slots > 0) {
+        const long long ts = nblob * slots * kTileN;
+        prepack_mixed_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(s, N, KT, g, slots, ts, wp);
+    } else {
+        const int tail_elems = static_cast<int>(channel_tail_bytes(N) / 2);
+        channel_tail_kernel<<<blocks_for(tail_elems, 256), 256, 0, st>>>(
+            s, N, NT * kTileN, tail_elems, reinterpret_cast<uint16_t*>(wp + mixed_table_bytes(nblob)));
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+int launch_unpack_mixed(const void* Wp, int K, int N, int g, int32_t* Q, uint16_t* s, uint8_t* widths,
+                        cudaStream_t st) {
+    const int slots = scale_slots(K, g);
+    const int KT = K / kTileK, NT = n_tiles(N);
+    const uint8_t* wp = static_cast<const uint8_t*>(Wp);
+    const long long nblob = static_cast<long long>(NT) * KT;
+    const long long tc = nblob * 4 * kTileN;
+    unpack_mixed_codes_kernel<<<blocks_for(tc, 256), 256, 0, st>>>(wp, N, KT, NT, tc, reinterpret_cast<uint32_t*>(Q),
+                                                                    widths);
+    if (slots > 0) {
+        const long long ts = nblob * slots * kTileN;
+        unpack_mixed_scales_kernel<<<blocks_for(ts, 256), 256, 0, st>>>(wp, N, KT, g, slots, ts, s);
+    } else {
+        channel_untail_kernel<<<blocks_for(N, 256), 256, 0, st>>>(
+            reinterpret_cast<const uint16_t*>(wp + mixed_table_bytes(nblob)), N, s);
+    }
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 }  // namespace wq

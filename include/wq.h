@@ -184,6 +184,37 @@ WQ_API int wq_unpack_sparse24(const void* Wp, int K, int N, int g, int32_t* Q_ou
 WQ_API int wq_gemm_w4a16_sparse24(const uint16_t* A, const void* Wp, uint16_t* Y, int M, int N, int K, int g,
                  void* stream);
 
+/* ---------------------------------------------------------------- mixed 2/4-bit weights
+ * "Enabling Fast 2-bit LLM on GPUs: Memory Alignment and Asynchronous Dequantization",
+ * Abstract: most groups of weights at 2 bits, the few groups with a large range at 4 bits,
+ * placed with the GPU's memory alignment in mind. Here the width is chosen per aligned block of
+ * 32 rows and 128 columns: widths uint8 [K/32, ceil(N/128)] (device memory), each 2 or 4; a
+ * b-bit code q stands for q - 2^(b-1), W[k,n] = (q[k,n] - z) * s[k/g, n] with z = 2 or 8 (the
+ * block's midpoint). Q keeps the usual 4-bit packing (int32 [K/8, N]); codes of 2-bit blocks
+ * must be 0..3. g as for wq_gemm_w4a16, g == K included.
+ * wq_prepacked_bytes_mixed: the buffer's size for n4 blocks of 4 bits (0 when unsupported).
+ * wq_prepack_mixed: Q, s, widths -> Wp (wp_bytes: the size of the caller's buffer). The call
+ * reads the widths on the host (it synchronises `stream`, returns WQ_ERR_CAPTURING while the
+ * stream is being captured), writes a blob table (each blob's offset and widths) at the start
+ * of Wp, then the blobs of 2-bit (1024 bytes) and 4-bit (2048 bytes) blocks and their scales.
+ * WQ_ERR_INVALID_ARG: a width other than 2 or 4, wp_bytes too small, or a code above 3 in a
+ * 2-bit block (checked on the device; Wp's content is then unspecified).
+ * wq_unpack_mixed: the inverse (test aid): Q_out, s_out and widths_out.
+ * wq_gemm_w4a16_mixed: Y [M, N] = A . W with the rounding of wq_gemm_w4a16, 0 <= M <= 16
+ * (WQ_ERR_UNSUPPORTED_SHAPE above); wp_bytes: the size of the buffer Wp points to (at least
+ * wq_prepacked_bytes_mixed(K, N, g, 0), else WQ_ERR_INVALID_ARG). The kernel copies each blob
+ * at the offset the table gives only when the blob lies inside wp_bytes and has the size its
+ * widths imply; otherwise it copies nothing more, records WQ_ERR_INVALID_ARG in the device
+ * status word (wq_get_device_status) and Y is undefined; the call may then last up to the
+ * device-side wait limit. Workspace: wq_workspace_bytes(6, ...). */
+WQ_API size_t wq_prepacked_bytes_mixed(int K, int N, int g, long long n4);
+WQ_API int wq_prepack_mixed(const int32_t* Q, const uint16_t* s, const uint8_t* widths, int K, int N, int g,
+                 void* Wp, size_t wp_bytes, void* stream);
+WQ_API int wq_unpack_mixed(const void* Wp, int K, int N, int g, int32_t* Q_out, uint16_t* s_out, uint8_t* widths_out,
+                 void* stream);
+WQ_API int wq_gemm_w4a16_mixed(const uint16_t* A, const void* Wp, size_t wp_bytes, uint16_t* Y, int M, int N,
+                 int K, int g, void* stream);
+
 /* W4A8: acc[m,n] = sum_k A[m,k] * (q[k,n] - 8) exactly in int32 (A int8 [M,K]),
  * Y[m,n] = fp16_rn((float(acc) * sa[m]) * sw[n]) with sa fp32 [M] per token and sw fp32
  * [N] per column. acc_out (int32 [M,N]) may be NULL; when given it receives acc.
@@ -244,7 +275,8 @@ WQ_API int wq_gemm_w4a16_noalloc(const uint16_t* A, const void* Wp, uint16_t* Y,
 /* ---------------------------------------------------------------- workspace and status
  * Bytes of library workspace one call of the given kind and shape needs (kind 0 = W4A16,
  * 1 = W4A8, 2 = W4A8 on fp16 activations, wq_gemm_w4a8_fp16act, 3 = wq_gemm_w4a16_zp,
- * 4 = wq_gemm_w4a16_act_order, 5 = wq_gemm_w4a16_sparse24 (0 for M > 16)). */
+ * 4 = wq_gemm_w4a16_act_order, 5 = wq_gemm_w4a16_sparse24, 6 = wq_gemm_w4a16_mixed (0 for
+ * M > 16 for the last two)). */
 WQ_API size_t wq_workspace_bytes(int kind, int M, int N, int K);
 
 /* Make sure the workspace of (current device, stream) holds at least `bytes`. Call it
@@ -264,8 +296,8 @@ WQ_API int wq_workspace_reserve(size_t bytes, void* stream);
 WQ_API int wq_get_device_status(void* stream);
 
 /* ---------------------------------------------------------------- introspection and test hooks
- * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8, 5 = 2:4 sparse W4A16
- * (M <= 16). */
+ * The launch plan a call would use. kind 0 = W4A16, 1 = W4A8, 5 = 2:4 sparse W4A16, 6 = mixed
+ * 2/4-bit W4A16 (5 and 6: M <= 16). */
 typedef struct {
     int grid;         /* persistent CTAs launched (<= number of SMs) */
     int tile_m;       /* activation rows per tile: 1, 2, 4, 8 or 16 for the register-operand kernel

@@ -63,6 +63,16 @@ def test_sparse_prepacked_bytes_agree_with_oracle(wq, K, N, g):
     assert wq.wq_prepacked_bytes_sparse24(K, N, g) == oracle.prepacked_bytes_w4a16_sparse24(K, N, g)
 
 
+@pytest.mark.parametrize("K,N,g,frac4", [(128, 8, 128, 0.5), (256, 136, 128, 0.4), (384, 296, 32, 0.2),
+                                         (4096, 4096, 4096, 0.3), (1280, 520, 640, 1.0), (256, 200, 64, 0.0)])
+def test_mixed_prepacked_bytes_agree_with_oracle(wq, K, N, g, frac4):
+    import synth
+    w = synth.w4a16_mixed_inputs(K, N, g, 1, seed=K, frac4=frac4)["widths"]
+    assert wq.wq_prepacked_bytes_mixed(K, N, g, int((w == 4).sum())) == oracle.prepacked_bytes_mixed(K, N, g, w)
+    assert wq.wq_prepacked_bytes_mixed(K, N, g, -1) == 0
+    assert wq.wq_prepacked_bytes_mixed(K, N, g, w.size + 1) == 0
+
+
 @pytest.mark.parametrize("K,N,g", [(100, 128, 100), (128, 12, 128), (0, 128, 128), (256, 128, 48),
                                    (256, 128, 96), (384, 128, 256), (256, -8, 128)])
 def test_unsupported_shapes_have_no_size(wq, K, N, g):
@@ -110,6 +120,15 @@ def test_host_side_argument_checks(wq):
     assert L.wq_prepack_sparse24(good, None, 128, 128, 128, good, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_unpack_sparse24(good, 128, 128, 128, good, odd, None) == wq.WQ_ERR_MISALIGNED
     assert wq.wq_prepacked_bytes_sparse24(256, 128, 96) == 0
+    # mixed 2/4-bit: M <= 16, the caller's buffer size, the usual checks
+    least = wq.wq_prepacked_bytes_mixed(128, 128, 128, 0)
+    assert L.wq_gemm_w4a16_mixed(good, good, least, good, 17, 128, 128, 128, None) == wq.WQ_ERR_UNSUPPORTED_SHAPE
+    assert L.wq_gemm_w4a16_mixed(good, good, least - 16, good, 1, 128, 128, 128, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_gemm_w4a16_mixed(good, odd, least, good, 1, 128, 128, 128, None) == wq.WQ_ERR_MISALIGNED
+    assert L.wq_gemm_w4a16_mixed(None, good, least, None, 0, 128, 128, 128, None) == wq.WQ_OK
+    assert L.wq_prepack_mixed(good, good, None, 128, 128, 128, good, least, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_prepack_mixed(good, good, good, 256, 128, 96, good, least, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_unpack_mixed(good, 128, 128, 128, good, good, None, None) == wq.WQ_ERR_INVALID_ARG
     # an empty batch is a no-op that needs no activation or output pointer
     assert L.wq_gemm_w4a16(None, good, None, 0, 128, 128, 128, None) == wq.WQ_OK
     assert L.wq_gemm_w4a8(None, None, good, None, None, None, 0, 128, 128, None) == wq.WQ_OK

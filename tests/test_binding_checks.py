@@ -12,7 +12,7 @@ class _Recorder:
     """Stands in for the loaded library: records every entry point called, except the pure size
     queries, which it forwards to the real library."""
     PURE = {"wq_prepacked_bytes", "wq_prepacked_bytes_w4a8", "wq_prepacked_bytes_zp", "wq_prepacked_bytes_sparse24",
-            "wq_status_string"}
+            "wq_prepacked_bytes_mixed", "wq_status_string"}
 
     def __init__(self, real):
         self.real, self.calls = real, []
@@ -165,4 +165,25 @@ def test_sparse_calls_refuse_wrong_sizes(rec):
                                   Y=torch.zeros((M, N + 8), dtype=torch.float16))
     with pytest.raises(ValueError):
         wq.wq_unpack_sparse24(torch.zeros(16, dtype=torch.uint8), K, N, g)
+    assert rec.calls == []
+
+
+def test_mixed_calls_refuse_wrong_sizes(rec):
+    Q = torch.zeros((K // 8, N), dtype=torch.int32)
+    s = torch.zeros((K // g, N), dtype=torch.float16)
+    W = torch.full((K // 32, 2), 2, dtype=torch.uint8)
+    with pytest.raises(ValueError):  # widths must be [K/32, ceil(N/128)]
+        wq.wq_prepack_mixed(Q, s, W[:, :1], g)
+    with pytest.raises(TypeError):  # widths must be uint8
+        wq.wq_prepack_mixed(Q, s, W.int(), g)
+    with pytest.raises(ValueError):  # s must be [K/g, N]
+        wq.wq_prepack_mixed(Q, s[:1], W, g)
+    least = wq.wq_prepacked_bytes_mixed(K, N, g, 0)
+    with pytest.raises(ValueError):  # smaller than any mixed buffer of this shape
+        wq.wq_gemm_w4a16_mixed(torch.zeros((M, K), dtype=torch.float16), torch.zeros(least - 1, dtype=torch.uint8), N, g)
+    with pytest.raises(ValueError):
+        wq.wq_gemm_w4a16_mixed(torch.zeros((M, K), dtype=torch.float16), torch.zeros(least, dtype=torch.uint8), N, g,
+                               Y=torch.zeros((M + 1, N), dtype=torch.float16))
+    with pytest.raises(ValueError):
+        wq.wq_unpack_mixed(torch.zeros(16, dtype=torch.uint8), K, N, g)
     assert rec.calls == []

@@ -82,6 +82,20 @@ def test_sparse_plan_invariants(wq, K, N, g):
         assert e.value.status == wq.WQ_ERR_UNSUPPORTED_SHAPE
 
 
+@pytest.mark.parametrize("K,N", SHAPES)
+@pytest.mark.parametrize("g", [32, 128, None])
+def test_mixed_plan_is_the_dense_register_operand_plan(wq, K, N, g):
+    # mixed 2/4-bit (kind 6): the slots hold the largest blob (every block 4-bit), so the plan is
+    # the dense one's; M > 16 is refused
+    g = K if g is None else g
+    if K % g:
+        pytest.skip("group size must divide K")
+    for M in [m for m in MS if m <= 16]:
+        assert wq.wq_plan_for(6, M, N, K, g, SMS, SMEM) == wq.wq_plan_for(0, M, N, K, g, SMS, SMEM)
+    with pytest.raises(wq.WqError):
+        wq.wq_plan_for(6, 17, N, K, g, SMS, SMEM)
+
+
 def test_plan_uses_the_largest_ring_that_fits(wq):
     for M, kind in itertools.product([1, 16, 32, 64, 256], [0, 1]):
         p = wq.wq_plan_for(kind, M, 4096, 4096, 128 if kind == 0 else 4096, SMS, SMEM)
