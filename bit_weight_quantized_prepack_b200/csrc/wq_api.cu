@@ -737,7 +737,7 @@ int wq_prepack_mixed(const int32_t* Q, const uint16_t* s, const uint8_t* widths,
         return WQ_ERR_CUDA;
     }
     // the blob table: each blob's offset (a prefix sum over the widths) and its widths
-    std::vector<uint32_t> table(static_cast<size_t>(nblob) + 1);
+    std::vector<uint32_t> table(mixed_table_bytes(nblob) / 4, 0u);  // the padding written as zeros too
     size_t pos = mixed_table_bytes(nblob) + (slots ? 0 : channel_tail_bytes(N));
     for (int nt = 0; nt < NT; ++nt)
         for (int kt = 0; kt < KT; ++kt) {
