@@ -72,6 +72,7 @@ struct Barriers {
     uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
     uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
     uint32_t wbits[kMaxSlots];     // mixed 2/4-bit: the widths of the blob in each weight slot
+    uint64_t tbl_full;             // mixed 2/4-bit: the CTA's table entries landed in shared memory
 };
 
 struct Ctl {
@@ -486,9 +487,11 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
 }
 
 // Weight producer (kWeightWarp, one thread) or activation producer (kActWarp, one thread).
+// kMix (mixed 2/4-bit weights, weight producer): tbl is shared memory for the CTA's table
+// entries (units beg .. end; a unit's index is its blob's index), copied there once.
 template <int MODE, bool kWeights, bool kMix = false>
 __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* aring, uint8_t* wring, Barriers& b,
-                              const Ctl& ctl, long long beg, long long end) {
+                              const Ctl& ctl, long long beg, long long end, uint32_t* tbl = nullptr) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
     uint32_t ebits = 0, ch = 0, armed = 0;
     ChunkBar cb;
@@ -500,6 +503,14 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
     // reads or writes memory shared with it (the partials, flags and Y) comes after these
     // copies.
     griddep_wait();
+    long long tlo = 0;  // kMix: first table entry held in tbl (a multiple of 4 entries)
+    if (kWeights && kMix) {
+        tlo = beg & ~3ll;
+        const long long thi = (end + 1 + 3) & ~3ll;  // entries beg .. end, 16-byte aligned around them
+        mbar_arrive_expect_tx(&b.tbl_full, static_cast<uint32_t>((thi - tlo) * 4));
+        bulk_g2s(tbl, p.mix_table + tlo, static_cast<uint32_t>((thi - tlo) * 4), &b.tbl_full, policy);
+        ok = wait_bar(&b.tbl_full, 0, ctl);
+    }
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
@@ -520,9 +531,9 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                     // slot's word, ordered before them by this thread's arrival (release). A table
                     // that does not describe this format inside the caller's buffer stops the CTA
                     // with WQ_ERR_INVALID_ARG before any copy of that chunk.
-                    const uint32_t* te = p.mix_table + static_cast<size_t>(nt) * p.k_blocks + kb;
+                    const uint32_t* te = tbl + (static_cast<long long>(nt) * p.k_blocks + kb - tlo);
                     uint32_t e[kMaxChunk + 1];
-                    for (int t = 0; t <= c; ++t) e[t] = __ldg(te + t);
+                    for (int t = 0; t <= c; ++t) e[t] = te[t];
                     uint32_t bytes = 0;
                     bool valid = true;
                     for (int t = 0; t < c; ++t) {
@@ -1724,6 +1735,7 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
     uint8_t* aring = align_ring(smem_dyn);
     uint8_t* wring = aring + static_cast<size_t>(p.slots) * p.act_slot;
     float* red = reinterpret_cast<float*>(wring + static_cast<size_t>(p.slots) * p.blob_bytes);
+    uint32_t* tbl = reinterpret_cast<uint32_t*>(red + 4 * TM * kTileN);  // mixed: the CTA's table entries
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const long long beg = unit_start(blockIdx.x, p.units, p.grid);
@@ -1737,6 +1749,7 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
             mbar_init(&bars.empty_a[s], 4);
         }
         if (lane == 0) abort_flag = 0;
+        if (FMT == kFmtMixed && lane == 0) mbar_init(&bars.tbl_full, 1);
         fence_barrier_init();
     }
     if (warp == kActWarpR && lane == 0)
@@ -1756,7 +1769,7 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
             rf_role<MODE, TM, kRfScaleNone, FMT>(p, aring, wring, bars, red, ctl, beg, end);
         }
     } else if (warp == kWeightWarpR) {
-        if (lane == 0) producer_role<MODE, true, FMT == kFmtMixed>(&maps, p, aring, wring, bars, ctl, beg, end);
+        if (lane == 0) producer_role<MODE, true, FMT == kFmtMixed>(&maps, p, aring, wring, bars, ctl, beg, end, tbl);
     } else {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     }
@@ -1789,7 +1802,13 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
         // TM rows x 128 int8 or fp16, unswizzled; sparse: at least 8 rows, swizzled
         pl->act_rows = (sparse && tm < kSpMinActRows) ? kSpMinActRows : tm;
         pl->act_slot = (mode == kModeW4A8) ? tm * 128 : pl->act_rows * 256;
-        const int budget = smem_optin - 2048 - 1024 - rf_red_bytes(tm);
+        // mixed: room for the CTA's table entries (at most ceil(units / grid) + 1 of them, widened to
+        // 16-byte boundaries on both sides)
+        const long long units = static_cast<long long>(pl->n_tiles) * pl->k_blocks;
+        const long long per_cta = (units + num_sms - 1) / num_sms;
+        const int tbl = pl->mixed ? static_cast<int>(((per_cta + 1 + 6) * 4 + 15) / 16 * 16) : 0;
+        if (tbl > smem_optin) return -1;
+        const int budget = smem_optin - 2048 - 1024 - rf_red_bytes(tm) - tbl;
         int s = budget / (pl->act_slot + pl->blob_bytes);
         if (s > kMaxSlots) s = kMaxSlots;
         if (s < 2) return -1;
@@ -1797,7 +1816,7 @@ int make_plan(int mode, int M, int N, int K, int slots, int num_sms, int smem_op
         int c = s / 2;
         if (c > kMaxChunk) c = kMaxChunk;
         pl->chunk = c;
-        pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + rf_red_bytes(tm);
+        pl->smem_bytes = s * (pl->act_slot + pl->blob_bytes) + 1024 + rf_red_bytes(tm) + tbl;
         pl->units = static_cast<long long>(pl->n_tiles) * pl->k_blocks;
         pl->grid = static_cast<int>(pl->units < num_sms ? pl->units : num_sms);
         return 0;

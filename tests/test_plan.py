@@ -85,13 +85,22 @@ def test_sparse_plan_invariants(wq, K, N, g):
 @pytest.mark.parametrize("K,N", SHAPES)
 @pytest.mark.parametrize("g", [32, 128, None])
 def test_mixed_plan_is_the_dense_register_operand_plan(wq, K, N, g):
-    # mixed 2/4-bit (kind 6): the slots hold the largest blob (every block 4-bit), so the plan is
-    # the dense one's; M > 16 is refused
+    # mixed 2/4-bit (kind 6): the slots hold the largest blob (every block 4-bit) and shared memory
+    # also holds the CTA's table entries (at most ceil(units / grid) + 1, widened to 16-byte
+    # boundaries); otherwise the dense register-operand plan. M > 16 is refused
     g = K if g is None else g
     if K % g:
         pytest.skip("group size must divide K")
     for M in [m for m in MS if m <= 16]:
-        assert wq.wq_plan_for(6, M, N, K, g, SMS, SMEM) == wq.wq_plan_for(0, M, N, K, g, SMS, SMEM)
+        p = wq.wq_plan_for(6, M, N, K, g, SMS, SMEM)
+        d = wq.wq_plan_for(0, M, N, K, g, SMS, SMEM)
+        for key in ("grid", "tile_m", "m_tiles", "n_tiles", "k_blocks", "threads", "units"):
+            assert p[key] == d[key], key
+        tbl = ((-(-p["units"] // SMS) + 7) * 4 + 15) // 16 * 16
+        act = p["tile_m"] * 256
+        blob = 8192 + (256 * (128 // min(g, 128)) if g < K else 0)
+        assert p["smem_bytes"] == p["stages"] * (act + blob) + 1024 + _red(p) + tbl
+        assert p["smem_bytes"] + 2048 <= SMEM and p["stages"] <= d["stages"]
     with pytest.raises(wq.WqError):
         wq.wq_plan_for(6, 17, N, K, g, SMS, SMEM)
 
