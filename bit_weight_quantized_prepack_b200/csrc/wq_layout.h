@@ -33,7 +33,8 @@
 //   16*(b*8 + rt) + lane / 2 its metadata operand (lanes 4gc, 4gc + 1).
 // Prepacked mixed 2/4-bit W4A16 buffer (a bit width per aligned block of 32 rows x 128
 //   columns; a b-bit code q stands for q - 2^(b-1)):
-//   a table of NT*KT + 1 uint32 entries (padded to 16 bytes): entry nt*KT + kt =
+//   a table of NT*KT + 1 uint32 entries (padded to 128 bytes, so that every blob starts on a
+//   128-byte boundary): entry nt*KT + kt =
 //     (byte offset of blob (nt, kt) / 16) << 4 | wbits (bit v set: 32-row block v is 4-bit),
 //     the last entry (end of the blobs / 16) << 4;
 //   for g == K, NT*128 fp16 column scales right after the table (padded to 16 bytes);
@@ -122,8 +123,8 @@ inline size_t blob_bytes_w4a16_zp(int slots) { return blob_bytes_w4a16(slots) + 
 // 2:4 sparse W4A16: code and metadata words, then `slots` rows of 128 fp16 scales.
 inline size_t blob_bytes_sp24(int slots) { return kSpHeadBytes + 2u * kTileN * static_cast<size_t>(slots); }
 
-// Mixed 2/4-bit: bytes of the blob table (NT*KT + 1 uint32 entries, padded to 16 bytes).
-inline size_t mixed_table_bytes(long long nblob) { return (static_cast<size_t>(nblob + 1) * 4 + 15) / 16 * 16; }
+// Mixed 2/4-bit: bytes of the blob table (NT*KT + 1 uint32 entries, padded to 128 bytes).
+inline size_t mixed_table_bytes(long long nblob) { return (static_cast<size_t>(nblob + 1) * 4 + 127) / 128 * 128; }
 
 inline size_t channel_tail_bytes(int N) { return ((2u * n_tiles(N) * kTileN) + 15u) / 16u * 16u; }
 

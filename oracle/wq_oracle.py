@@ -716,7 +716,7 @@ def w4a16_mixed_absdot(A: np.ndarray, Q: np.ndarray, s: np.ndarray, g: int, widt
 
 
 # Prepacked mixed buffer (the library's own format):
-#   a table of NT*KT + 1 uint32 entries (padded to 16 bytes): entry nt*KT + kt = (byte offset of
+#   a table of NT*KT + 1 uint32 entries (padded to 128 bytes): entry nt*KT + kt = (byte offset of
 #     blob (nt, kt) / 16) << 4 | wbits, bit v of wbits set when 32-row block v of the blob is
 #     4-bit; the last entry = (end of the blobs / 16) << 4;
 #   for g == K the column scales (NT*128 fp16, padded to 16 bytes) right after the table;
@@ -731,7 +731,7 @@ def _mixed_field(r: int, j: int) -> int:
 
 
 def _mixed_table_bytes(nblob: int) -> int:
-    return ((nblob + 1) * 4 + 15) // 16 * 16
+    return ((nblob + 1) * 4 + 127) // 128 * 128
 
 
 def prepacked_bytes_mixed(K: int, N: int, g: int, widths: np.ndarray) -> int:

@@ -629,7 +629,7 @@ def pin_mixed_all_four_bit_is_w4a16(o):
     assert np.array_equal(o.w4a16_mixed(d["A"], d["Q"], d["s"], 64, W4), o.w4a16(d["A"], d["Q"], d["s"], 64))
     mixed = o.prepack_mixed(d["Q"], d["s"], 64, W4)
     dense = o.prepack_w4a16(d["Q"], d["s"], 64)
-    head = (4 * (2 * 2 + 1) + 15) // 16 * 16
+    head = (4 * (2 * 2 + 1) + 127) // 128 * 128
     assert np.array_equal(mixed[head:], dense)
 
 

@@ -383,7 +383,7 @@ def _mut_mixed_field_halves_swapped(mp):
 
 
 def _mut_mixed_table_padded_twice(mp):
-    mp.setattr(O, "_mixed_table_bytes", lambda nblob: ((nblob + 1) * 4 + 15) // 16 * 16 + 16)
+    mp.setattr(O, "_mixed_table_bytes", lambda nblob: ((nblob + 1) * 4 + 127) // 128 * 128 + 16)
 
 
 @pytest.mark.parametrize("mutate", [_mut_mixed_field_halves_swapped, _mut_mixed_table_padded_twice],
