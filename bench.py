@@ -298,6 +298,49 @@ def rows_sparse24(torch, wq, dev, stream, hbm_gbs):
     return out
 
 
+MIXED_FRAC4 = 0.15
+
+
+def mixed_algo_bytes(M, K, N, n4, g=G):
+    """Algorithmic bytes of one mixed 2/4-bit call: 2-bit and 4-bit code blocks (1024 or 2048
+    bytes per 32 x 128 block), the scales, A and Y (the blob table is bookkeeping, not counted)."""
+    blocks = (K // 32) * -(-N // 128)
+    return (blocks - n4) * 1024 + n4 * 2048 + 2 * (K // g) * N + 2 * M * K + 2 * M * N
+
+
+def rows_mixed(torch, wq, dev, stream, hbm_gbs):
+    """Mixed 2/4-bit W4A16 (the Llama-7B layers and the 70B gate/up layer, g = 128, 15 % of the
+    32 x 128 blocks at 4 bits, M in {1, 4, 16}): the same weight through the dense buffer and the
+    mixed one, each call back to back in a CUDA graph over rotated copies; per call:
+    microseconds, GB/s of the mixed call's own algorithmic bytes, its roofline fraction, and the
+    dense call's time over the mixed call's."""
+    out = {}
+    for K, N in SPARSE_LAYERS:
+        d = synth.w4a16_mixed_inputs(K, N, G, max(SPARSE_M), seed=37, frac4=MIXED_FRAC4)
+        Q, s = torch.from_numpy(d["Q"]).to(dev), torch.from_numpy(d["s"]).to(dev)
+        W = torch.from_numpy(d["widths"]).to(dev)
+        n4 = int((d["widths"] == 4).sum())
+        nb = wq.wq_prepacked_bytes_mixed(K, N, G, n4)
+        copies = int(min(12, max(2, -(-3 * 126_000_000 // nb))))
+        Wd = [wq.wq_prepack(Q, s, G) for _ in range(copies)]
+        Wm = [wq.wq_prepack_mixed(Q, s, W, G) for _ in range(copies)]
+        A = torch.from_numpy(d["A"]).to(dev)
+        for M in SPARSE_M:
+            Am = A[:M].contiguous()
+            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            wq.wq_workspace_reserve(wq.wq_workspace_bytes(0, M, N, K), stream=stream)
+            td = _graph_time(torch, stream, lambda r: wq.wq_gemm_w4a16(Am, Wd[r % copies], N, G, Y=Y, stream=stream),
+                             2 * copies)
+            tm = _graph_time(torch, stream,
+                             lambda r: wq.wq_gemm_w4a16_mixed(Am, Wm[r % copies], N, G, Y=Y, stream=stream), 2 * copies)
+            b = mixed_algo_bytes(M, K, N, n4)
+            out[f"{K}x{N}_M{M}"] = {"us": round(tm * 1e6, 2), "dense_us": round(td * 1e6, 2),
+                                   "gbs": round(b / tm / 1e9, 1), "roofline_frac": round(b / (hbm_gbs * 1e9) / tm, 3),
+                                   "speedup_vs_dense": round(td / tm, 3), "bits_per_weight": round(8 * nb / (K * N), 2)}
+        del Wd, Wm, Q, s, A
+    return out
+
+
 def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
     """The compute-bound W4A16 sweep (K = N = 8192) and the W4A8 layers, each timed alone."""
     out = {"compute_sweep": {}, "w4a8": {}}
@@ -366,6 +409,7 @@ def extra_breakdowns(torch, wq, dev, stream, hbm_gbs, tflops):
                     "note": "int8 peak = measured bf16 peak x the nominal 2x ratio"}
     out["layers_70b"] = rows_70b(torch, wq, dev, stream, hbm_gbs, tflops)
     out["sparse24"] = rows_sparse24(torch, wq, dev, stream, hbm_gbs)
+    out["mixed24"] = rows_mixed(torch, wq, dev, stream, hbm_gbs)
     return out
 
 

@@ -71,8 +71,7 @@ struct Barriers {
     uint64_t aempty[kASlotsS];     // MMAs done with a tensor-memory slot
     uint64_t dfull;                // accumulators of a segment complete (one commit per issuer)
     uint64_t drain[kMaxIssuers];   // all MMAs of an issuer complete
-    uint32_t wbits[kMaxSlots];     // mixed 2/4-bit: per weight slot, (bytes its blob starts before the
-                                   // slot) << 4 | the blob's widths
+    uint32_t wbits[kMaxSlots];     // mixed 2/4-bit: the widths of the blob in each weight slot
     uint64_t tbl_full;             // mixed 2/4-bit: the CTA's table entries landed in shared memory
 };
 
@@ -495,8 +494,6 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                               const Ctl& ctl, long long beg, long long end, uint32_t* tbl = nullptr) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
     uint32_t ebits = 0, ch = 0, armed = 0;
-    uint32_t waited = 0;                        // kMix: slots whose previous use was waited for early
-    uint64_t cur_starts = 0, prev_starts = 0;   // kMix: slots where a chunk started, this and the last pass
     ChunkBar cb;
     uint32_t first_pass_chunks = 0xffffffffu;  // chunks before the ring first wraps
     int pos = 0;
@@ -520,44 +517,20 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
         const uint8_t* wtile = p.wp + static_cast<size_t>(nt) * p.k_blocks * p.blob_bytes;
         for (int kb = seg.kb_lo; kb <= seg.kb_hi;) {
             const int c = chunk_len(p.chunk, kb, seg.kb_hi, pos, p.slots, ch == 0);
-            if constexpr (kWeights && kMix) {
-                // A chunk's blobs are copied packed from its first slot, so a blob of the previous
-                // ring pass may lie in slots before the one it releases. Before this chunk overwrites
-                // slots pos .. pos + c - 1, every previous-pass blob that may lie there is consumed:
-                // those released by these slots and by the rest of the previous-pass chunk that holds
-                // slot pos + c - 1 (slots waited for ahead of their own chunk are marked, and that
-                // chunk does not wait for the same phase again).
-                int e_end = pos + c;
-                if (ch >= first_pass_chunks) {
-                    const uint64_t after = prev_starts & ~((2ull << (pos + c - 1)) - 1ull);
-                    e_end = after ? __ffsll(static_cast<long long>(after)) - 1 : p.slots;
-                }
-                for (int x = pos; x < e_end; ++x) {
-                    if (ok && ch >= first_pass_chunks && !((waited >> x) & 1u))
-                        ok = wait_bar(&b.empty_w[x], ((ebits >> x) & 1u) ^ 1u, ctl);
-                    if (x >= pos + c)
-                        waited |= 1u << x;
-                    else
-                        waited &= ~(1u << x);
-                }
-                for (int t = 0; t < c; ++t) ebits ^= 1u << (pos + t);
-                cur_starts |= 1ull << pos;
-            } else {
-                for (int t = 0; t < c; ++t) {
-                    const int s = pos + t;
-                    if (ok && ch >= first_pass_chunks)  // a slot's first use needs no wait
-                        ok = wait_bar(kWeights ? &b.empty_w[s] : &b.empty_a[s], ((ebits >> s) & 1u) ^ 1u, ctl);
-                    ebits ^= 1u << s;
-                }
+            for (int t = 0; t < c; ++t) {
+                const int s = pos + t;
+                if (ok && ch >= first_pass_chunks)  // a slot's first use needs no wait
+                    ok = wait_bar(kWeights ? &b.empty_w[s] : &b.empty_a[s], ((ebits >> s) & 1u) ^ 1u, ctl);
+                ebits ^= 1u << s;
             }
             if (ok) {
                 uint64_t* fbar = &b.full[cb.bar];
                 if (kWeights && kMix) {
-                    // blobs of varying size: offsets and widths from the table, one copy per blob
-                    // into its fixed-stride slot; the widths reach the consumers through the
-                    // slot's word, ordered before them by this thread's arrival (release). A table
-                    // that does not describe this format inside the caller's buffer stops the CTA
-                    // with WQ_ERR_INVALID_ARG before any copy of that chunk.
+                    // blobs of varying size: offsets and widths from the CTA's table entries, one
+                    // copy per blob into its fixed-stride slot; the widths reach the consumers
+                    // through the slot's word, ordered before them by this thread's arrival
+                    // (release). A table that does not describe this format inside the caller's
+                    // buffer stops the CTA with WQ_ERR_INVALID_ARG before any copy of that chunk.
                     const uint32_t* te = tbl + (static_cast<long long>(nt) * p.k_blocks + kb - tlo);
                     uint32_t e[kMaxChunk + 1];
 #pragma unroll
@@ -580,24 +553,20 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
                             if (t < c) b.wbits[pos + t] = 0xFu;
                         mbar_arrive(fbar);
                     } else {
-                        // one copy of the chunk's consecutive blobs, packed from slot pos: blob t
-                        // starts back_t = t * stride - (its offset in the chunk) bytes before slot
-                        // pos + t, which the slot's word carries above the widths
-                        uint32_t e_c = e[1];  // e[c], selected without indexing the array at run time
-#pragma unroll
-                        for (int t = 2; t <= kMaxChunk; ++t)
-                            if (t == c) e_c = e[t];
-                        const uint32_t total = ((e_c >> 4) - (e[0] >> 4)) * 16u;
+                        uint32_t bytes = 0;
 #pragma unroll
                         for (int t = 0; t < kMaxChunk; ++t)
                             if (t < c) {
-                                const uint32_t back = static_cast<uint32_t>(t) * static_cast<uint32_t>(p.blob_bytes) -
-                                                      ((e[t] >> 4) - (e[0] >> 4)) * 16u;
-                                b.wbits[pos + t] = (back << 4) | (e[t] & 0xFu);
+                                b.wbits[pos + t] = e[t] & 0xFu;
+                                bytes += ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u;
                             }
-                        mbar_arrive_expect_tx(fbar, total);
-                        bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes, p.wp + static_cast<size_t>(e[0] >> 4) * 16,
-                                 total, fbar, policy);
+                        mbar_arrive_expect_tx(fbar, bytes);
+#pragma unroll
+                        for (int t = 0; t < kMaxChunk; ++t)
+                            if (t < c)
+                                bulk_g2s(wring + static_cast<size_t>(pos + t) * p.blob_bytes,
+                                         p.wp + static_cast<size_t>(e[t] >> 4) * 16, ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u,
+                                         fbar, policy);
                     }
                 } else if (kWeights) {
                     mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(c * p.blob_bytes));
@@ -618,8 +587,6 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
             if (pos == p.slots) {
                 pos = 0;
                 if (first_pass_chunks == 0xffffffffu) first_pass_chunks = ch;
-                prev_starts = cur_starts;
-                cur_starts = 0;
             }
         }
     }
@@ -1593,12 +1560,9 @@ __device__ void rf_role(const GemmArgs& p, const uint8_t* aring, const uint8_t* 
             if (!mine) continue;
             ok = __all_sync(0xffffffffu, ok && wait_bar(&b.full[fb], fpar, ctl));
             if (!ok) continue;  // an expired wait: the CTA winds down (nothing more is read or released)
-            // mixed: the slot's word = (bytes the packed blob starts before the slot) << 4 | widths
-            const uint32_t mixw = MIX ? b.wbits[s] : 0u;
-            const uint32_t back = MIX ? min(mixw >> 4, static_cast<uint32_t>(s) * static_cast<uint32_t>(p.blob_bytes)) : 0u;
-            const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes - back;
+            const uint8_t* blob = wring + static_cast<size_t>(s) * p.blob_bytes;
             const uint32_t* words = reinterpret_cast<const uint32_t*>(blob);
-            const uint32_t wb = MIX ? (mixw & 0xFu) : 0xFu;  // mixed: bit v set = block v is 4-bit
+            const uint32_t wb = MIX ? (b.wbits[s] & 0xFu) : 0xFu;  // mixed: bit v set = block v is 4-bit
             const uint16_t* scs = reinterpret_cast<const uint16_t*>(
                 blob + (SP ? kSpHeadBytes : (MIX ? kMixBlock2 * (4 + __popc(wb)) : kCodeBytes)));
             const uint8_t* act = aring + static_cast<size_t>(s) * p.act_slot;

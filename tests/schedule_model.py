@@ -937,58 +937,3 @@ def simulate_rf(units, grid, kbs, chunk, slots, rng=None, ctas_only=None):
     stuck = [(st["cta"], name, st["cur"][name]) for st in ctas for name in st["roles"] if name not in st["done"]]
     return problems + stuck
 
-
-# ------------------------------------------------------------------ packed copies (mixed widths)
-PACKED_EXTENDED_WAITS = True  # the kernel's rule; False plants the hazard the rule removes
-
-
-def check_packed_copies(units, grid, kbs, chunk, slots, stride, sizes_rng):
-    """The weight producer of the mixed 2/4-bit kernel copies a chunk's c blobs (each at most
-    ``stride`` bytes) packed from slot pos, so blob t may start before slot pos + t, the slot
-    whose empty barrier its consumers release. Before each chunk the producer waits, in the
-    kernel's order, for the previous use of every slot from pos to the end of the previous-pass
-    chunk that holds slot pos + c - 1 (slots waited for early are not waited for again by their
-    own chunk). Returns the problems: ("overwrite", cta, chunk, blob) when a chunk's bytes meet
-    a blob whose consumption the producer has not waited for."""
-    problems = []
-    for cta in range(grid):
-        beg, end = unit_start(cta, units, grid), unit_start(cta + 1, units, grid)
-        uses = [0] * slots            # writes of each slot so far (its release barrier's phase)
-        waited_use = [-1] * slots     # highest use of each slot whose consumption was waited for
-        waited = 0
-        cur_starts = prev_starts = 0
-        first_pass = None
-        live = []                     # (chunk, slot, use, byte lo, byte hi) of every blob written
-        for seg, pos, c, it0, ch in chunks(beg, end, kbs, chunk, slots):
-            if pos is None:
-                continue
-            e_end = pos + c
-            if first_pass is not None and PACKED_EXTENDED_WAITS:
-                after = prev_starts & ~((2 << (pos + c - 1)) - 1)
-                e_end = (after & -after).bit_length() - 1 if after else slots
-            for x in range(pos, e_end):
-                if first_pass is not None and not (waited >> x) & 1 and uses[x] > 0:
-                    waited_use[x] = max(waited_use[x], uses[x] - 1)
-                if x >= pos + c:
-                    waited |= 1 << x
-                else:
-                    waited &= ~(1 << x)
-            sizes = [int(sizes_rng.integers(1, stride // 16 + 1)) * 16 for _ in range(c)]
-            lo = pos * stride
-            hi = lo + sum(sizes)
-            for blob in live:
-                b_ch, b_slot, b_use, b_lo, b_hi = blob
-                if b_lo < hi and lo < b_hi and waited_use[b_slot] < b_use:
-                    problems.append(("overwrite", cta, ch, blob))
-            off = lo
-            for t in range(c):
-                live.append((ch, pos + t, uses[pos + t], off, off + sizes[t]))
-                assert off <= (pos + t) * stride and off + sizes[t] <= (pos + t + 1) * stride
-                off += sizes[t]
-                uses[pos + t] += 1
-            cur_starts |= 1 << pos
-            if pos + c == slots:
-                if first_pass is None:
-                    first_pass = ch + 1
-                prev_starts, cur_starts = cur_starts, 0
-    return problems

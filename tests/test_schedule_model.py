@@ -10,10 +10,8 @@ parity test and measured slower on B200: dequantised k-blocks in a ring of 4, 6 
 indexed by walk position, chunks fixed by walk position. Its tests keep the hazards that model
 found before that kernel ran (a slot's consecutive uses by different issuers, a partial barrier
 that the residue's next k-block completes first)."""
-import numpy as np
 import pytest
 
-import schedule_model as M
 from schedule_model import simulate
 
 SHAPES = [(4096, 4096), (4096, 12288), (4096, 22016), (11008, 4096), (8192, 10240), (8192, 8192),
@@ -437,28 +435,3 @@ def test_rf_model_catches_a_missing_second_barrier():
         sm.RED_SECOND_BARRIER = saved
     assert races
 
-
-# packed copies of the mixed 2/4-bit kernel: no chunk overwrites a blob not yet consumed
-@pytest.mark.parametrize("K,N,slots", [(4096, 4096, 26), (4096, 22016, 26), (11008, 4096, 17), (8192, 57344, 26),
-                                       (1024, 392, 5), (2048, 136, 7), (128, 8, 3)])
-def test_packed_copies_never_overwrite_unconsumed_blobs(K, N, slots):
-    kbs, nt = K // 128, -(-N // 128)
-    units = kbs * nt
-    grid = min(units, 148)
-    rng = np.random.default_rng(K + N + slots)
-    for chunk in (1, 2, 3, 4):
-        if chunk > max(1, slots // 2):
-            continue
-        assert M.check_packed_copies(units, grid, kbs, chunk, slots, 8448, rng) == []
-
-
-def test_packed_copies_model_catches_waits_only_on_the_chunks_own_slots(monkeypatch):
-    # without the waits that reach to the end of the previous pass's chunk, a packed chunk
-    # overwrites blobs still being read
-    monkeypatch.setattr(M, "PACKED_EXTENDED_WAITS", False)
-    rng = np.random.default_rng(1)
-    found = []
-    for K, N, slots in [(4096, 22016, 26), (8192, 57344, 26), (11008, 4096, 17)]:
-        kbs, nt = K // 128, -(-N // 128)
-        found += M.check_packed_copies(kbs * nt, min(kbs * nt, 148), kbs, 4, slots, 8448, rng)
-    assert found
