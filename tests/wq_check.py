@@ -1,6 +1,6 @@
 """Helpers of the GPU parity tests: move synthetic inputs to the device, compare with the oracle.
 
-The comparison is the benchmark spec's tolerance, elementwise over every compared output:
+The comparison is the layer's stated tolerance, elementwise over every compared output:
 ``|y - y_ref| <= 2^-10 |y_ref| + 1e-3 sum_k |a_k w_k|`` with ``y_ref`` the fp64 oracle.
 NaN or Inf in the CUDA output always fails.
 """
