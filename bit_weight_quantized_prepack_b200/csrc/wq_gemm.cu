@@ -487,11 +487,43 @@ __device__ void dequant_role(const GemmArgs& p, const uint8_t* wring, Barriers& 
 }
 
 // Weight producer (kWeightWarp, one thread) or activation producer (kActWarp, one thread).
-// kMix (mixed 2/4-bit weights, weight producer): tbl is shared memory for the CTA's table
-// entries (units beg .. end; a unit's index is its blob's index), copied there once.
+// Mixed 2/4-bit weights: the weight producer warp (all 32 lanes) copies the CTA's table entries
+// (units beg .. end, entries tlo .. thi - 1 around them; a unit's index is its blob's index) into
+// shared memory once, after the grid dependency, and checks every blob the CTA will copy: it lies
+// inside the caller's buffer and has the size its widths imply. A table that does not describe
+// the format stops the CTA with WQ_ERR_INVALID_ARG before any weight copy. Returns whether the
+// producer may go on (the same on every lane).
+__device__ bool mixed_table_window(const GemmArgs& p, Barriers& b, uint32_t* tbl, const Ctl& ctl, long long beg,
+                                   long long end, int lane, long long* tlo_out) {
+    griddep_wait();  // the table is caller memory a preceding kernel may still write
+    const long long tlo = beg & ~3ll;
+    const long long thi = (end + 1 + 3) & ~3ll;  // entries beg .. end, 16-byte aligned around them
+    *tlo_out = tlo;
+    if (lane == 0) {
+        mbar_arrive_expect_tx(&b.tbl_full, static_cast<uint32_t>((thi - tlo) * 4));
+        bulk_g2s(tbl, p.mix_table + tlo, static_cast<uint32_t>((thi - tlo) * 4), &b.tbl_full, l2_policy_evict_first());
+    }
+    const bool landed = __all_sync(0xffffffffu, wait_bar(&b.tbl_full, 0, ctl));
+    if (!landed) return false;
+    const unsigned long long scale_bytes = static_cast<unsigned long long>(p.blob_bytes - kCodeBytes);
+    bool valid = true;
+    for (long long u = beg + lane; u < end; u += 32) {
+        const uint32_t e0 = tbl[u - tlo], e1 = tbl[u + 1 - tlo];
+        const unsigned long long lo = (e0 >> 4) * 16ull, hi = (e1 >> 4) * 16ull;
+        const unsigned long long want = static_cast<unsigned long long>(kMixBlock2) * (4 + __popc(e0 & 0xFu)) + scale_bytes;
+        valid = valid && hi > lo && hi - lo == want && hi <= p.wp_bytes;
+    }
+    valid = __all_sync(0xffffffffu, valid);
+    if (!valid && lane == 0) raise_error(ctl, WQ_ERR_INVALID_ARG);
+    return valid;
+}
+
+// kMix (mixed 2/4-bit weights, weight producer): tbl holds the CTA's table entries from entry
+// tlo on, checked by mixed_table_window (tbl_ok).
 template <int MODE, bool kWeights, bool kMix = false>
 __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* aring, uint8_t* wring, Barriers& b,
-                              const Ctl& ctl, long long beg, long long end, uint32_t* tbl = nullptr) {
+                              const Ctl& ctl, long long beg, long long end, const uint32_t* tbl = nullptr,
+                              long long tlo_in = 0, bool tbl_ok = true) {
     const uint64_t policy = l2_policy_evict_first();  // every weight byte is read once
     uint32_t ebits = 0, ch = 0, armed = 0;
     ChunkBar cb;
@@ -503,14 +535,8 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
     // reads or writes memory shared with it (the partials, flags and Y) comes after these
     // copies.
     griddep_wait();
-    long long tlo = 0;  // kMix: first table entry held in tbl (a multiple of 4 entries)
-    if (kWeights && kMix) {
-        tlo = beg & ~3ll;
-        const long long thi = (end + 1 + 3) & ~3ll;  // entries beg .. end, 16-byte aligned around them
-        mbar_arrive_expect_tx(&b.tbl_full, static_cast<uint32_t>((thi - tlo) * 4));
-        bulk_g2s(tbl, p.mix_table + tlo, static_cast<uint32_t>((thi - tlo) * 4), &b.tbl_full, policy);
-        ok = wait_bar(&b.tbl_full, 0, ctl);
-    }
+    const long long tlo = tlo_in;  // kMix: first table entry held in tbl (a multiple of 4 entries)
+    if (kWeights && kMix) ok = tbl_ok;
     SegCursor seg(beg, end, p.k_blocks);
     while (seg.next()) {
         const int nt = seg.tile / p.m_tiles, mt = seg.tile % p.m_tiles;
@@ -526,48 +552,28 @@ __device__ void producer_role(const ActMaps* maps, const GemmArgs& p, uint8_t* a
             if (ok) {
                 uint64_t* fbar = &b.full[cb.bar];
                 if (kWeights && kMix) {
-                    // blobs of varying size: offsets and widths from the CTA's table entries, one
-                    // copy per blob into its fixed-stride slot; the widths reach the consumers
-                    // through the slot's word, ordered before them by this thread's arrival
-                    // (release). A table that does not describe this format inside the caller's
-                    // buffer stops the CTA with WQ_ERR_INVALID_ARG before any copy of that chunk.
+                    // blobs of varying size: offsets and widths from the CTA's table entries (checked
+                    // once, before the walk), one copy per blob into its fixed-stride slot; the
+                    // widths reach the consumers through the slot's word, ordered before them by
+                    // this thread's arrival (release)
                     const uint32_t* te = tbl + (static_cast<long long>(nt) * p.k_blocks + kb - tlo);
                     uint32_t e[kMaxChunk + 1];
 #pragma unroll
                     for (int t = 0; t <= kMaxChunk; ++t) e[t] = (t <= c) ? te[t] : 0u;
-                    bool valid = true;
+                    uint32_t bytes = 0;
 #pragma unroll
                     for (int t = 0; t < kMaxChunk; ++t)
                         if (t < c) {
-                            const unsigned long long lo = (e[t] >> 4) * 16ull, hi = (e[t + 1] >> 4) * 16ull;
-                            const unsigned long long want = static_cast<unsigned long long>(kMixBlock2) *
-                                                                (4 + __popc(e[t] & 0xFu)) +
-                                                            (p.blob_bytes - kCodeBytes);
-                            valid = valid && hi > lo && hi - lo == want && hi <= p.wp_bytes;
+                            b.wbits[pos + t] = e[t] & 0xFu;
+                            bytes += ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u;
                         }
-                    if (!valid) {  // no copy; the arrival lets the chunk's phase complete with the activations
-                        raise_error(ctl, WQ_ERR_INVALID_ARG);
-                        ok = false;
+                    mbar_arrive_expect_tx(fbar, bytes);
 #pragma unroll
-                        for (int t = 0; t < kMaxChunk; ++t)
-                            if (t < c) b.wbits[pos + t] = 0xFu;
-                        mbar_arrive(fbar);
-                    } else {
-                        uint32_t bytes = 0;
-#pragma unroll
-                        for (int t = 0; t < kMaxChunk; ++t)
-                            if (t < c) {
-                                b.wbits[pos + t] = e[t] & 0xFu;
-                                bytes += ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u;
-                            }
-                        mbar_arrive_expect_tx(fbar, bytes);
-#pragma unroll
-                        for (int t = 0; t < kMaxChunk; ++t)
-                            if (t < c)
-                                bulk_g2s(wring + static_cast<size_t>(pos + t) * p.blob_bytes,
-                                         p.wp + static_cast<size_t>(e[t] >> 4) * 16, ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u,
-                                         fbar, policy);
-                    }
+                    for (int t = 0; t < kMaxChunk; ++t)
+                        if (t < c)
+                            bulk_g2s(wring + static_cast<size_t>(pos + t) * p.blob_bytes,
+                                     p.wp + static_cast<size_t>(e[t] >> 4) * 16, ((e[t + 1] >> 4) - (e[t] >> 4)) * 16u,
+                                     fbar, policy);
                 } else if (kWeights) {
                     mbar_arrive_expect_tx(fbar, static_cast<uint32_t>(c * p.blob_bytes));
                     bulk_g2s(wring + static_cast<size_t>(pos) * p.blob_bytes,
@@ -1782,7 +1788,13 @@ __global__ void __launch_bounds__(kThreadsRf, 1) wq_gemm_rf(const __grid_constan
             rf_role<MODE, TM, kRfScaleNone, FMT>(p, aring, wring, bars, red, ctl, beg, end);
         }
     } else if (warp == kWeightWarpR) {
-        if (lane == 0) producer_role<MODE, true, FMT == kFmtMixed>(&maps, p, aring, wring, bars, ctl, beg, end, tbl);
+        if constexpr (FMT == kFmtMixed) {
+            long long tlo = 0;
+            const bool tbl_ok = mixed_table_window(p, bars, tbl, ctl, beg, end, lane, &tlo);
+            if (lane == 0) producer_role<MODE, true, true>(&maps, p, aring, wring, bars, ctl, beg, end, tbl, tlo, tbl_ok);
+        } else {
+            if (lane == 0) producer_role<MODE, true>(&maps, p, aring, wring, bars, ctl, beg, end);
+        }
     } else {
         if (lane == 0) producer_role<MODE, false>(&maps, p, aring, wring, bars, ctl, beg, end);
     }
