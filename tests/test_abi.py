@@ -30,7 +30,10 @@ def wq():
 def test_header_declares_the_entry_points():
     names = set(_declared_functions())
     for must in ("wq_prepack", "wq_gemm_w4a16", "wq_gemm_w4a8", "wq_prepacked_bytes", "wq_unpack",
-                 "wq_get_device_status", "wq_workspace_reserve"):
+                 "wq_get_device_status", "wq_workspace_reserve", "wq_prepack_zp", "wq_gemm_w4a16_zp",
+                 "wq_prepack_act_order", "wq_gemm_w4a16_act_order", "wq_quantize_act", "wq_gemm_w4a8_fp16act",
+                 "wq_prepack_sparse24", "wq_gemm_w4a16_sparse24", "wq_prepack_mixed", "wq_gemm_w4a16_mixed",
+                 "wq_gemm_w4a16_noalloc"):
         assert must in names
 
 
