@@ -199,7 +199,9 @@ WQ_API int wq_gemm_w4a16_sparse24(const uint16_t* A, const void* Wp, uint16_t* Y
  * of Wp, then the blobs of 2-bit (1024 bytes) and 4-bit (2048 bytes) blocks and their scales.
  * WQ_ERR_INVALID_ARG: a width other than 2 or 4, wp_bytes too small, or a code above 3 in a
  * 2-bit block (checked on the device; Wp's content is then unspecified).
- * wq_unpack_mixed: the inverse (test aid): Q_out, s_out and widths_out.
+ * wq_unpack_mixed: the inverse (test aid): Q_out, s_out and widths_out. It reads the blobs where
+ * the buffer's table points, unchecked: pass only a buffer written by wq_prepack_mixed (the
+ * layer itself, wq_gemm_w4a16_mixed, checks every blob against wp_bytes before reading it).
  * wq_gemm_w4a16_mixed: Y [M, N] = A . W with the rounding of wq_gemm_w4a16, 0 <= M <= 16
  * (WQ_ERR_UNSUPPORTED_SHAPE above); wp_bytes: the size of the buffer Wp points to (at least
  * wq_prepacked_bytes_mixed(K, N, g, 0), else WQ_ERR_INVALID_ARG). The kernel copies each blob
