@@ -511,7 +511,8 @@ def wq_prepack_mixed(Q: torch.Tensor, s: torch.Tensor, widths: torch.Tensor, g: 
 
 
 def wq_unpack_mixed(Wp: torch.Tensor, K: int, N: int, g: int, stream=None):
-    """Inverse of wq_prepack_mixed: (Q int32 [K/8, N], s fp16 [K/g, N], widths uint8 [K/32, ceil(N/128)])."""
+    """Inverse of wq_prepack_mixed: (Q int32 [K/8, N], s fp16 [K/g, N], widths uint8 [K/32, ceil(N/128)]).
+    A test aid: it reads the blobs where Wp's table points, so Wp must come from wq_prepack_mixed."""
     if g <= 0 or K <= 0 or K % g:
         raise WqError(WQ_ERR_INVALID_ARG, "wq_unpack_mixed")
     least = wq_prepacked_bytes_mixed(K, N, g, 0)
